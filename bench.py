@@ -1,0 +1,469 @@
+"""Benchmark of the gated delta-rule library on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--quick]
+
+One step = one gdn_chunk_fwd over the hybrid-LM prefill batch (B=8, T=4096, H=12, dk=dv=64,
+chunk 64, bf16 q/k/v, fp32 gates and state): the whole chunkwise path (gates, intra-chunk
+products, triangular inverse, state chain, outputs, final state) in the library's kernels.
+Inputs are synthetic (seeded, see workloads.py) and resident in HBM before timing; L2 is flushed
+(a 256 MB device write) between timed steps because the batch is smaller than L2.  Rank 0 prints
+one JSON line.  Extra objects report the decode workload (N=256, H=32, d=128, 1000 steps;
+state-updates/s, HBM fraction) and the long-context and varlen prefill workloads.
+
+With --gpus N (under torchrun) every rank runs its own batch (independent sequences need no
+exchange): weak scaling, time = max over ranks.  --impl reference times the fp64 CPU oracle on
+the host cores on a bounded sample of the same workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+METRIC = "gated-delta chunk-fwd tokens/s & % roofline; decode state-updates/s & HBM %"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+KERNEL_SOURCES = {
+    "chunk": "linear_attention_sequence_rule_b200/csrc/gdn_chunk_simt.cu",
+    "decode": "linear_attention_sequence_rule_b200/csrc/gdn_decode.cu",
+}
+
+
+# ---- algorithmic work (per token-head, chunk C = 64; a multiply-add counts 2 flops) -----------
+
+def algo_bytes(token_heads, n_states, dk, dv, elem, has_s0, has_sfinal):
+    b = token_heads * (elem * (2 * dk + 2 * dv) + 8)
+    b += n_states * 4 * dk * dv * (int(has_s0) + int(has_sfinal))
+    return b
+
+
+def algo_flops(token_heads, dk, dv, C=64):
+    return token_heads * ((3 * C - 1) * dk + 2 * C * dv + C * C / 3 + 6 * dk * dv)
+
+
+DECODE_BYTES_PER_STATE = lambda dk, dv, e: 8 * dk * dv + e * (2 * dk + 2 * dv) + 8
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def source_sha(rel):
+    with open(os.path.join(ROOT, rel), "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def ncu_traffic(kernel_key, workload):
+    """DRAM bytes per launch from the committed ncu summary, if taken on the current source."""
+    p = os.path.join(ROOT, "profiles", "ncu_traffic.txt")
+    if not os.path.exists(p):
+        return None
+    sha = source_sha(KERNEL_SOURCES[kernel_key])
+    for line in open(p):
+        f = dict(kv.split("=", 1) for kv in line.split() if "=" in kv)
+        if f.get("kernel") == kernel_key and f.get("workload") == workload and f.get("sha") == sha:
+            return float(f["dram_bytes_per_launch"])
+    return None
+
+
+# ---- clocks during the timed region (NVML reads only) -------------------------------------
+
+class ClockSampler:
+    REASONS = {
+        "gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4,
+        "hw_slowdown": 0x8, "sync_boost": 0x10, "sw_thermal_slowdown": 0x20,
+        "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80,
+    }
+
+    def __init__(self, index, period=0.005):
+        self.ok = False
+        self.samples, self.reasons = [], set()
+        self.period = period
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.max_mhz = None
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for name, bit in self.REASONS.items():
+                    if r & bit and name != "gpu_idle":
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self._stop = threading.Event()
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self._t.join()
+
+    def result(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                    "samples": 0}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ---- distributed plumbing ------------------------------------------------------------------
+
+def dist_setup(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---- our arm -------------------------------------------------------------------------------
+
+def to_dev(inp):
+    return {k: (v.cuda().contiguous() if torch.is_tensor(v) else v) for k, v in inp.items()}
+
+
+def time_chunk(gdn, d, steps, warmup, flush, stream):
+    """Per-step CUDA-event time (ms) of gdn.chunk_fwd, L2 flushed before every step."""
+    out = torch.empty_like(d["v"])
+    Sf = torch.empty((d["B"], d["H"], d["dk"], d["dv"]), dtype=torch.float32, device="cuda")
+    call = lambda: gdn.chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], S0=d["S0"],
+                                 cu_seqlens=d["cu_seqlens"], out=out, S_final=Sf, stream=stream)
+    with torch.cuda.stream(stream):
+        for _ in range(warmup):
+            flush.zero_()
+            call()
+        stream.synchronize()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(steps)]
+        for s, e in ev:
+            flush.zero_()
+            s.record(stream)
+            call()
+            e.record(stream)
+        stream.synchronize()
+    return [s.elapsed_time(e) for s, e in ev]
+
+
+def chunk_numbers(name, d, times_ms, peaks):
+    ms = statistics.mean(times_ms)
+    th = d["q"].shape[0] * (d["q"].shape[1] if d["cu_seqlens"] is None else 1) * d["H"]
+    tokens = th // d["H"]
+    elem = d["q"].element_size()
+    by = algo_bytes(th, d["B"] * d["H"], d["dk"], d["dv"], elem, d["S0"] is not None, True)
+    fl = algo_flops(th, d["dk"], d["dv"])
+    gbs = by / (ms * 1e-3) / 1e9
+    tfs = fl / (ms * 1e-3) / 1e12
+    return dict(workload=name, ms=ms, tokens=tokens, tokens_per_s=tokens / (ms * 1e-3),
+                algo_bytes=by, algo_flops=fl, gbs=gbs, hbm_frac=gbs / peaks["hbm_gbs"],
+                tflops=tfs, tensor_frac=tfs / peaks["bf16_tflops"])
+
+
+def time_decode(gdn, steps, warmup, stream, pool=32):
+    cfg = workloads.CONFIGS["decode"]
+    N, H, dk, dv = cfg["N"], cfg["H"], cfg["dk"], cfg["dv"]
+    S = workloads.make_decode_state(N, H, dk, dv, cfg["seed"]).cuda()
+    xs = [to_dev(workloads.make_decode_step_inputs(N, H, dk, dv, cfg["dtype"], seed=cfg["seed"],
+                                                   step=i, la_scale=cfg["la_scale"]))
+          for i in range(pool)]
+    out = torch.empty((N, H, dv), dtype=torch.bfloat16, device="cuda")
+    call = lambda x: gdn.decode_step(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], S,
+                                     out=out, stream=stream)
+    with torch.cuda.stream(stream):
+        for i in range(warmup):
+            call(xs[i % pool])
+        stream.synchronize()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(steps)]
+        for i, (s, e) in enumerate(ev):
+            s.record(stream)
+            call(xs[i % pool])
+            e.record(stream)
+        stream.synchronize()
+    t = [s.elapsed_time(e) for s, e in ev]
+    ms = statistics.mean(t)
+    by = N * H * DECODE_BYTES_PER_STATE(dk, dv, 2)
+    return dict(workload=f"decode N={N} H={H} dk=dv={dk} bf16, fp32 state", steps=steps,
+                input_pool=pool, ms_per_step=ms, state_updates_per_s=N * H / (ms * 1e-3),
+                tokens_per_s=N / (ms * 1e-3), algo_bytes_per_step=by,
+                gbs=by / (ms * 1e-3) / 1e9)
+
+
+def e2e_chunk(gdn, inp, steps, warmup, stream):
+    """Same workload through the public call with HOST buffers: H2D of the step's inputs from
+    pinned memory, the forward, D2H of out and S_final, all inside the timed region."""
+    host = {k: (v.pin_memory() if torch.is_tensor(v) else v) for k, v in inp.items()}
+    dev = {k: (torch.empty_like(v, device="cuda") if torch.is_tensor(v) else v)
+           for k, v in inp.items()}
+    out_h = torch.empty(inp["v"].shape, dtype=inp["v"].dtype).pin_memory()
+    sf_h = torch.empty((inp["B"], inp["H"], inp["dk"], inp["dv"]), dtype=torch.float32).pin_memory()
+    out_d = torch.empty_like(dev["v"])
+    sf_d = torch.empty(sf_h.shape, dtype=torch.float32, device="cuda")
+    keys = [k for k in ("q", "k", "v", "log_alpha", "beta", "S0", "cu_seqlens") if host.get(k) is not None]
+    h2d = sum(host[k].numel() * host[k].element_size() for k in keys)
+    d2h = out_h.numel() * out_h.element_size() + sf_h.numel() * 4
+
+    def step():
+        for k in keys:
+            dev[k].copy_(host[k], non_blocking=True)
+        gdn.chunk_fwd(dev["q"], dev["k"], dev["v"], dev["log_alpha"], dev["beta"], S0=dev.get("S0"),
+                      cu_seqlens=dev.get("cu_seqlens"), out=out_d, S_final=sf_d, stream=stream)
+        out_h.copy_(out_d, non_blocking=True)
+        sf_h.copy_(sf_d, non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        for _ in range(warmup):
+            step()
+        stream.synchronize()
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record(stream)
+        for _ in range(steps):
+            step()
+        e.record(stream)
+        stream.synchronize()
+    ms = s.elapsed_time(e) / steps
+    return ms, h2d, d2h
+
+
+def cpu_oracle_baseline(inp, budget_s=12.0):
+    """Time the fp64 oracle, as it stands, on the host cores over whole (sequence, head) chains of
+    the workload until about budget_s seconds of work; returns tokens/s and the sample."""
+    import oracle
+    H = inp["H"]
+    n_units = inp["B"] * H
+    threads = oracle.max_threads()
+    # first a small probe to size the sample
+    probe = list(range(min(n_units, max(threads, 1))))
+    t0 = time.perf_counter()
+    oracle.forward(inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["beta"], inp["S0"],
+                   cu_seqlens=inp["cu_seqlens"], units=probe)
+    t_probe = time.perf_counter() - t0
+    per_unit = t_probe / len(probe)
+    n = max(len(probe), min(n_units, int(budget_s / max(per_unit, 1e-9))))
+    units = list(range(n))
+    t0 = time.perf_counter()
+    oracle.forward(inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["beta"], inp["S0"],
+                   cu_seqlens=inp["cu_seqlens"], units=units)
+    dt = time.perf_counter() - t0
+    if inp["cu_seqlens"] is None:
+        th = n * inp["T"]
+    else:
+        cu = inp["cu_seqlens"]
+        th = sum(int(cu[u // H + 1] - cu[u // H]) for u in units)
+    return dict(value=(th / H) / dt, unit="tokens/s", cores=threads, kind="oracle",
+                sample=f"{n} of {n_units} (sequence, head) chains, each in full "
+                       f"({th} token-heads, {dt:.2f} s, fp64 sequential recurrence)")
+
+
+def run_ours(args, world, rank, local):
+    import linear_attention_sequence_rule_b200 as gdn
+    peaks, peak_kind = load_peaks()
+    stream = torch.cuda.Stream()
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device="cuda")
+    name = "hybrid_lm"
+    cfg = workloads.CONFIGS[name]
+    inp = workloads.config_inputs(name, seed=cfg["seed"] + rank)
+    d = to_dev(inp)
+
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        times = time_chunk(gdn, d, args.steps, args.warmup, flush, stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    ms_local = statistics.mean(times)
+    ms = max_over_ranks(ms_local, world)
+    main = chunk_numbers(name, d, times, peaks)
+    tokens_all = main["tokens"] * world
+    value = tokens_all / (ms * 1e-3)
+
+    e2e_ms, h2d, d2h = e2e_chunk(gdn, inp, max(3, args.steps // 10), 2, stream)
+    e2e_ms = max_over_ranks(e2e_ms, world)
+
+    extra = {}
+    decode = None
+    if not args.quick:
+        decode = time_decode(gdn, 1000, 10, stream)
+        decode["hbm_frac"] = decode["gbs"] / peaks["hbm_gbs"]
+        for w in ("long_context", "varlen"):
+            dw = to_dev(workloads.config_inputs(w))
+            tw = time_chunk(gdn, dw, max(3, args.steps // 20), 2, flush, stream)
+            nums = chunk_numbers(w, dw, tw, peaks)
+            extra[w] = {k: (round(v, 6) if isinstance(v, float) else v) for k, v in nums.items()}
+            del dw
+    cpu = None
+    if rank == 0 and world == 1:
+        cpu = cpu_oracle_baseline(inp)
+
+    if rank != 0:
+        return
+    traffic = ncu_traffic("chunk", name)
+    line = {
+        "metric": METRIC,
+        "value": value,
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded; q,k L2-normalised N(0,1), v N(0,1), beta=sigmoid(N(0,1)), "
+                "log_alpha=-0.1*softplus(N(0,1)), S0=0)",
+        "config": {"workload": "hybrid_lm prefill chunk forward: B=8 T=4096 H=12 dk=dv=64 "
+                               "chunk=64, bf16 q/k/v/out, fp32 gates and state",
+                   "global_batch": 8 * world, "seq_len": 4096, "heads": 12, "head_dim": 64,
+                   "parallelism": f"dp{world} (independent sequences per rank)",
+                   "l2": "flushed between timed steps (256 MB device write)"},
+        "roofline": {"bound": "hbm", "achieved": main["gbs"], "peak": peaks["hbm_gbs"],
+                     "unit": "GB/s", "frac": main["gbs"] / peaks["hbm_gbs"],
+                     "traffic": traffic, "peak_source": f"{peak_kind} hbm_gbs",
+                     "algo_bytes_per_launch": main["algo_bytes"]},
+        "tensor": {"achieved_tflops": main["tflops"], "peak_tflops": peaks["bf16_tflops"],
+                   "frac": main["tensor_frac"], "algo_flops_per_launch": main["algo_flops"]},
+        "e2e": {"value": tokens_all / (e2e_ms * 1e-3), "unit": "tokens/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "gpu_launches": args.steps,
+        "clocks": clk.result(),
+        "cpu_baseline": cpu,
+    }
+    if decode is not None:
+        line["decode"] = decode
+    if extra:
+        line["workloads"] = extra
+    print(json.dumps(line), flush=True)
+
+
+# ---- reference arm: the fp64 oracle on the host cores ----------------------------------------
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return
+    import oracle
+    name = "hybrid_lm"
+    inp = workloads.config_inputs(name)
+    H = inp["H"]
+    n_units = inp["B"] * H
+    threads = oracle.max_threads()
+    # each step: a bounded sample of whole chains, sized so the whole run takes a few minutes
+    per_step = max(threads, 8)
+    times = []
+    for i in range(args.warmup + args.steps):
+        units = [(i * per_step + j) % n_units for j in range(per_step)]
+        t0 = time.perf_counter()
+        oracle.forward(inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["beta"], inp["S0"],
+                       units=units)
+        dt = time.perf_counter() - t0
+        if i >= args.warmup:
+            times.append(dt)
+    s = statistics.mean(times)
+    value = (per_step * inp["T"]) / s
+    sample = (f"{per_step} of {n_units} (sequence, head) chains per step, each in full "
+              f"({per_step * inp['T']} token-heads), fp64 sequential recurrence")
+    line = {
+        "impl": "reference",
+        "metric": METRIC,
+        "value": value,
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": s * 1e3,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f64",
+        "data": "synthetic (seeded, same inputs as the GPU arm)",
+        "config": {"workload": "hybrid_lm prefill chunk forward: B=8 T=4096 H=12 dk=dv=64 "
+                               "chunk=64, bf16 q/k/v/out, fp32 gates and state",
+                   "global_batch": 8, "seq_len": 4096, "heads": 12, "head_dim": 64,
+                   "parallelism": "host cores (OpenMP over chains)"},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--quick", action="store_true", help="main workload only")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        rank = int(os.environ.get("RANK", "0"))
+        run_reference(args, world, rank)
+        return
+    world, rank, local = dist_setup(args.gpus)
+    try:
+        run_ours(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

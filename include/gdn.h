@@ -1,0 +1,134 @@
+/*
+ * gdn.h -- C-ABI of libgdn: the gated delta-rule recurrence on one NVIDIA B200 (sm_100a).
+ *
+ * The operation, per (sequence, head), with state S in R^{dk x dv}:
+ *
+ *     S_t = a_t (I - b_t k_t k_t^T) S_{t-1} + b_t k_t v_t^T,     o_t = S_t^T q_t
+ *
+ * with a_t = exp(log_alpha_t) in [0, 1] (data-dependent forget gate) and b_t = beta_t in [0, 2].
+ * Sources:
+ *   - Sykra README, "Architectural Highlights": Gated DeltaNet layers trained chunk-parallel
+ *     through the WY / unit-triangular transform (a triangular solve per chunk, the rest as
+ *     matrix products); a data-dependent forget gate a_t; generation as an O(d^2) update of a
+ *     fixed d x d state.  Also its "Computational Complexity" table (O(N d) training, O(d^2)
+ *     per decode step).
+ *   - DeltaPhase README, section 1 "Extended Householder Beta Range": beta in (0, 2), beta = 2 an
+ *     exact Householder reflection; "Fast Triangular Solve": an exact O(C^2) per-chunk solve.
+ *   - DeltaPhase README, section 2: the delta rule as read-out -> error -> rank-one update.
+ * Readings taken where the pages are silent: the read-out uses the post-update state; there is
+ * no 1/sqrt(dk) query scale; a_t and b_t are scalars per (token, head); the library does not
+ * normalise q or k.
+ *
+ * Conventions shared by every entry point
+ *   - Every tensor pointer is a DEVICE pointer owned by the caller.  The library allocates no
+ *     memory, keeps no state between calls and may be called from several host threads.
+ *   - Calls are asynchronous: they validate on the host, enqueue kernels on `stream` (a
+ *     cudaStream_t; NULL = the legacy default stream) and return.  Errors found on the host are
+ *     returned before anything is enqueued, so a failed call writes nothing.
+ *   - Element type of q, k, v and out: `dtype` (GDN_DTYPE_BF16 or GDN_DTYPE_F32).  Gates
+ *     (log_alpha, beta) and states (S0, S_final, S_inout) are always fp32.
+ *   - All tensors are contiguous row-major; every pointer must be 16-byte aligned.
+ *   - Return value: GDN_OK (0) or a negative GDN_ERR_* code; gdn_last_error() then gives a
+ *     one-line reason (per host thread).
+ */
+#ifndef GDN_H_
+#define GDN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define GDN_API __attribute__((visibility("default")))
+#else
+#define GDN_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum gdn_status {
+    GDN_OK = 0,
+    GDN_ERR_INVALID_ARGUMENT = -1, /* null required pointer, bad size, misaligned pointer      */
+    GDN_ERR_UNSUPPORTED = -2,      /* dk/dv not in {64,128}, chunk != 64, unknown dtype        */
+    GDN_ERR_WORKSPACE = -3,        /* workspace NULL or smaller than the query function says   */
+    GDN_ERR_CUDA = -4,             /* a CUDA launch or driver call failed (see gdn_last_error) */
+    GDN_ERR_TIMEOUT = -5           /* reserved: a bounded device-side wait ran out             */
+};
+
+enum gdn_dtype {
+    GDN_DTYPE_F32 = 0,
+    GDN_DTYPE_BF16 = 1
+};
+
+/*
+ * gdn_chunk_fwd -- prefill / training forward of the recurrence over whole sequences, computed
+ * chunk by chunk in the WY / UT-transform form (Sykra README, "Architectural Highlights";
+ * DeltaPhase README, section 1 "Fast Triangular Solve").  Per chunk of C = 64 tokens:
+ *     A = strictly_lower(diag(b) (Gam o K K^T)),  T = (I + A)^{-1},
+ *     W = T diag(b gam) K,  U~ = T diag(b) V,  U = U~ - W S,
+ *     O = diag(gam) Q S + lower_incl(Gam o Q K^T) U,  S <- gam_C S + (diag(lam) K)^T U,
+ * where gam, lam, Gam are the products of a_j from the chunk start / to the chunk end / between
+ * two tokens.  The result equals the sequential recurrence up to rounding.
+ *
+ * Layouts
+ *   dense  (cu_seqlens == NULL): q,k [B,T,H,dk]; v,out [B,T,H,dv]; log_alpha,beta [B,T,H]
+ *   varlen (cu_seqlens != NULL): B = number of sequences, T = total tokens; q,k [T,H,dk];
+ *          v,out [T,H,dv]; log_alpha,beta [T,H]; cu_seqlens: DEVICE int32 [B+1], cu[0] = 0,
+ *          cu[B] = T, non-decreasing (contents are not checked: malformed offsets are undefined
+ *          behaviour).  Sequence s owns tokens cu[s] .. cu[s+1]-1 and is chunked from its own
+ *          first token; a sequence of length 0 gets S_final = S0 and no outputs.
+ *   S0, S_final: [B,H,dk,dv] fp32.  S0 == NULL: zero initial state.  S_final == NULL: not
+ *          written.  S_final == S0 (same pointer) is allowed (in-place carry); no other
+ *          overlap between any output and any input is allowed.
+ * Arguments
+ *   B >= 1, T >= 0 (T == 0 only with cu_seqlens), H >= 1; dk, dv in {64, 128}; chunk == 64.
+ *   log_alpha <= 0 expected (-inf allowed: an exact reset); positive values are accepted but
+ *   may overflow.  beta in [0, 2].
+ *   workspace / workspace_bytes: device scratch of at least gdn_chunk_fwd_workspace_bytes(...)
+ *   bytes, 256-byte aligned (may be NULL when that function returns 0).  Its contents on entry
+ *   do not matter; calls that share a workspace must not overlap in time.
+ */
+GDN_API int gdn_chunk_fwd(const void *q, const void *k, const void *v, const float *log_alpha,
+                  const float *beta, const float *S0, void *out, float *S_final, int B, int T,
+                  int H, int dk, int dv, int chunk, const int32_t *cu_seqlens, int dtype,
+                  void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * gdn_chunk_fwd_workspace_bytes -- device scratch that gdn_chunk_fwd needs for these sizes
+ * (varlen: non-zero when cu_seqlens will be passed).  Returns 0 when no scratch is needed and
+ * (size_t)-1 for arguments gdn_chunk_fwd would reject.
+ */
+GDN_API size_t gdn_chunk_fwd_workspace_bytes(int B, int T, int H, int dk, int dv, int chunk, int varlen,
+                                     int dtype);
+
+/*
+ * gdn_decode_step -- one generation step: every (n, h) state takes exactly one token, in place
+ * (Sykra README, "Architectural Highlights" and "Computational Complexity": an O(d^2) update of
+ * a fixed d x d state per token).  With r = S^T k, s = S^T q (both from the state before the
+ * step):
+ *     u   = b (v - a r)
+ *     out = a s + (k . q) u
+ *     S  <- a S + k u^T
+ *   q,k [N,H,dk]; v,out [N,H,dv] in dtype; log_alpha,beta [N,H] fp32; S_inout [N,H,dk,dv] fp32,
+ *   read and overwritten.  N >= 1, H >= 1, dk and dv in {64, 128}.  No overlap between S_inout
+ *   and the other arguments.
+ */
+GDN_API int gdn_decode_step(const void *q, const void *k, const void *v, const float *log_alpha,
+                    const float *beta, float *S_inout, void *out, int N, int H, int dk, int dv,
+                    int dtype, void *stream);
+
+/* Static text for a status code. */
+GDN_API const char *gdn_status_string(int status);
+
+/* One-line reason for the last failed call on this host thread ("" when none). */
+GDN_API const char *gdn_last_error(void);
+
+/* Library version string. */
+GDN_API const char *gdn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDN_H_ */

@@ -1,0 +1,196 @@
+"""Python binding of libgdn, the B200 (sm_100a) gated delta-rule library.
+
+Argument marshalling only: every step of the computation runs in the library's CUDA kernels.
+PyTorch provides device memory and streams.  The binding has two layers:
+
+* ``gdn_chunk_fwd``, ``gdn_decode_step``, ``gdn_chunk_fwd_workspace_bytes``,
+  ``gdn_status_string``, ``gdn_last_error``, ``gdn_version`` -- the C-ABI entry points of
+  ``include/gdn.h`` with the same names and arguments (pointers as Python ints);
+* ``chunk_fwd`` and ``decode_step`` -- the same calls taking torch tensors; they check shapes,
+  devices and dtypes, allocate outputs with torch when none are given, and raise ``GdnError``
+  on a non-zero status.
+
+If ``libgdn.so`` has not been built, importing this package raises: there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+__all__ = [
+    "GdnError", "GDN_OK", "GDN_ERR_INVALID_ARGUMENT", "GDN_ERR_UNSUPPORTED", "GDN_ERR_WORKSPACE",
+    "GDN_ERR_CUDA", "GDN_ERR_TIMEOUT", "GDN_DTYPE_F32", "GDN_DTYPE_BF16", "LIB_PATH",
+    "gdn_chunk_fwd", "gdn_decode_step", "gdn_chunk_fwd_workspace_bytes", "gdn_status_string",
+    "gdn_last_error", "gdn_version", "chunk_fwd", "decode_step", "workspace_bytes",
+]
+
+GDN_OK = 0
+GDN_ERR_INVALID_ARGUMENT = -1
+GDN_ERR_UNSUPPORTED = -2
+GDN_ERR_WORKSPACE = -3
+GDN_ERR_CUDA = -4
+GDN_ERR_TIMEOUT = -5
+GDN_DTYPE_F32 = 0
+GDN_DTYPE_BF16 = 1
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libgdn.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is missing: build it with `python -m linear_attention_sequence_rule_b200.build`"
+        " (there is no fallback implementation)")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+_vp, _sz, _i = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int
+_lib.gdn_chunk_fwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i,
+                               _vp, _i, _vp, _sz, _vp]
+_lib.gdn_chunk_fwd.restype = _i
+_lib.gdn_chunk_fwd_workspace_bytes.argtypes = [_i, _i, _i, _i, _i, _i, _i, _i]
+_lib.gdn_chunk_fwd_workspace_bytes.restype = _sz
+_lib.gdn_decode_step.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp]
+_lib.gdn_decode_step.restype = _i
+_lib.gdn_status_string.argtypes = [_i]
+_lib.gdn_status_string.restype = ctypes.c_char_p
+_lib.gdn_last_error.argtypes = []
+_lib.gdn_last_error.restype = ctypes.c_char_p
+_lib.gdn_version.argtypes = []
+_lib.gdn_version.restype = ctypes.c_char_p
+
+
+class GdnError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"{gdn_status_string(status)}: {message}")
+        self.status = status
+
+
+# ---- C-ABI mirrors ---------------------------------------------------------------------------
+
+def gdn_chunk_fwd(q, k, v, log_alpha, beta, S0, out, S_final, B, T, H, dk, dv, chunk, cu_seqlens,
+                  dtype, workspace, workspace_bytes, stream) -> int:
+    return _lib.gdn_chunk_fwd(q, k, v, log_alpha, beta, S0, out, S_final, B, T, H, dk, dv, chunk,
+                              cu_seqlens, dtype, workspace, workspace_bytes, stream)
+
+
+def gdn_chunk_fwd_workspace_bytes(B, T, H, dk, dv, chunk, varlen, dtype) -> int:
+    return _lib.gdn_chunk_fwd_workspace_bytes(B, T, H, dk, dv, chunk, varlen, dtype)
+
+
+def gdn_decode_step(q, k, v, log_alpha, beta, S_inout, out, N, H, dk, dv, dtype, stream) -> int:
+    return _lib.gdn_decode_step(q, k, v, log_alpha, beta, S_inout, out, N, H, dk, dv, dtype, stream)
+
+
+def gdn_status_string(status: int) -> str:
+    return _lib.gdn_status_string(status).decode()
+
+
+def gdn_last_error() -> str:
+    return _lib.gdn_last_error().decode()
+
+
+def gdn_version() -> str:
+    return _lib.gdn_version().decode()
+
+
+# ---- torch-level calls ------------------------------------------------------------------------
+
+_DT = {torch.bfloat16: GDN_DTYPE_BF16, torch.float32: GDN_DTYPE_F32}
+
+
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+def _stream_ptr(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream
+
+
+def _need(t, name, dtype=None, shape=None, device=None):
+    if t is None:
+        raise ValueError(f"{name} is required")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+
+
+def workspace_bytes(B, T, H, dk, dv, varlen=False, dtype=torch.bfloat16, chunk=64) -> int:
+    n = gdn_chunk_fwd_workspace_bytes(B, T, H, dk, dv, chunk, int(bool(varlen)), _DT[dtype])
+    if n == ctypes.c_size_t(-1).value:
+        raise GdnError(GDN_ERR_INVALID_ARGUMENT, gdn_last_error())
+    return n
+
+
+def chunk_fwd(q, k, v, log_alpha, beta, S0=None, cu_seqlens=None, out=None, S_final=None,
+              output_final_state=True, workspace=None, chunk=64, stream=None):
+    """Chunkwise forward.  Dense q,k [B,T,H,dk], v [B,T,H,dv]; varlen (cu_seqlens int32 [B+1] on
+    the device) packs q,k [T,H,dk] ...  Returns (out, S_final or None)."""
+    dt = q.dtype
+    if dt not in _DT:
+        raise ValueError(f"unsupported dtype {dt}")
+    dev = q.device
+    if cu_seqlens is not None:
+        T, H, dk = q.shape
+        B = cu_seqlens.shape[0] - 1
+        lead = (T,)
+        _need(cu_seqlens, "cu_seqlens", torch.int32, (B + 1,), dev)
+    else:
+        B, T, H, dk = q.shape
+        lead = (B, T)
+    dv = v.shape[-1]
+    _need(q, "q", dt, (*lead, H, dk), dev)
+    _need(k, "k", dt, (*lead, H, dk), dev)
+    _need(v, "v", dt, (*lead, H, dv), dev)
+    _need(log_alpha, "log_alpha", torch.float32, (*lead, H), dev)
+    _need(beta, "beta", torch.float32, (*lead, H), dev)
+    if S0 is not None:
+        _need(S0, "S0", torch.float32, (B, H, dk, dv), dev)
+    if out is None:
+        out = torch.empty((*lead, H, dv), dtype=dt, device=dev)
+    _need(out, "out", dt, (*lead, H, dv), dev)
+    if S_final is None and output_final_state:
+        S_final = torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev)
+    if S_final is not None:
+        _need(S_final, "S_final", torch.float32, (B, H, dk, dv), dev)
+    need = workspace_bytes(B, T, H, dk, dv, cu_seqlens is not None, dt, chunk)
+    if need and workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    rc = gdn_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(S0), _ptr(out),
+                       _ptr(S_final), B, T, H, dk, dv, chunk, _ptr(cu_seqlens), _DT[dt],
+                       _ptr(workspace), wbytes, _stream_ptr(stream))
+    if rc != GDN_OK:
+        raise GdnError(rc, gdn_last_error())
+    return out, S_final
+
+
+def decode_step(q, k, v, log_alpha, beta, S, out=None, stream=None):
+    """One decode step, S [N,H,dk,dv] fp32 updated in place.  Returns out [N,H,dv]."""
+    dt = q.dtype
+    if dt not in _DT:
+        raise ValueError(f"unsupported dtype {dt}")
+    dev = q.device
+    N, H, dk = q.shape
+    dv = v.shape[-1]
+    _need(q, "q", dt, (N, H, dk), dev)
+    _need(k, "k", dt, (N, H, dk), dev)
+    _need(v, "v", dt, (N, H, dv), dev)
+    _need(log_alpha, "log_alpha", torch.float32, (N, H), dev)
+    _need(beta, "beta", torch.float32, (N, H), dev)
+    _need(S, "S", torch.float32, (N, H, dk, dv), dev)
+    if out is None:
+        out = torch.empty((N, H, dv), dtype=dt, device=dev)
+    _need(out, "out", dt, (N, H, dv), dev)
+    rc = gdn_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(S), _ptr(out),
+                         N, H, dk, dv, _DT[dt], _stream_ptr(stream))
+    if rc != GDN_OK:
+        raise GdnError(rc, gdn_last_error())
+    return out

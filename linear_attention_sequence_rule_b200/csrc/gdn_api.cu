@@ -1,0 +1,158 @@
+// gdn_api.cu -- the C-ABI of libgdn (declared in include/gdn.h): argument validation on the
+// host, choice of kernel, and launch on the caller's stream.  No device memory is allocated here
+// or anywhere else in the library.
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include "gdn_internal.h"
+#include "../../include/gdn.h"
+
+namespace gdn {
+
+static thread_local char g_last_error[512];
+
+void set_error(const char *fmt, ...)
+{
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
+    va_end(ap);
+}
+
+static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+static int fail(int code, const char *fmt, ...)
+{
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
+    va_end(ap);
+    return code;
+}
+
+static int cuda_fail(cudaError_t e, const char *where)
+{
+    return fail(GDN_ERR_CUDA, "%s: %s (%s)", where, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+static bool head_dim_ok(int d) { return d == 64 || d == 128; }
+
+// Shared shape/type checks of the chunk forward; returns GDN_OK or an error code.
+static int check_chunk_shape(int B, int T, int H, int dk, int dv, int chunk, int varlen, int dtype)
+{
+    if (dtype != GDN_DTYPE_BF16 && dtype != GDN_DTYPE_F32)
+        return fail(GDN_ERR_UNSUPPORTED, "gdn_chunk_fwd: unknown dtype %d", dtype);
+    if (!head_dim_ok(dk) || !head_dim_ok(dv))
+        return fail(GDN_ERR_UNSUPPORTED, "gdn_chunk_fwd: dk=%d dv=%d, supported: 64 or 128", dk, dv);
+    if (chunk != 64)
+        return fail(GDN_ERR_UNSUPPORTED, "gdn_chunk_fwd: chunk=%d, supported: 64", chunk);
+    if (B < 1 || H < 1)
+        return fail(GDN_ERR_INVALID_ARGUMENT, "gdn_chunk_fwd: B=%d H=%d must be >= 1", B, H);
+    if (T < 0 || (!varlen && T < 1))
+        return fail(GDN_ERR_INVALID_ARGUMENT, "gdn_chunk_fwd: T=%d (dense needs T >= 1)", T);
+    const long long tokens = varlen ? (long long)T : (long long)B * T;
+    if (tokens * H * (dk > dv ? dk : dv) >= (1LL << 40))
+        return fail(GDN_ERR_INVALID_ARGUMENT, "gdn_chunk_fwd: problem too large");
+    if ((long long)B * H > (1LL << 30))
+        return fail(GDN_ERR_INVALID_ARGUMENT, "gdn_chunk_fwd: B*H too large");
+    return GDN_OK;
+}
+
+static size_t chunk_workspace(int B, int T, int H, int dk, int dv, int varlen, int dtype)
+{
+    (void)B; (void)T; (void)H; (void)dk; (void)dv; (void)varlen; (void)dtype;
+    return 0;
+}
+
+}  // namespace gdn
+
+using namespace gdn;
+
+extern "C" {
+
+const char *gdn_version(void) { return "gdn-b200 0.1"; }
+
+const char *gdn_last_error(void) { return g_last_error; }
+
+const char *gdn_status_string(int status)
+{
+    switch (status) {
+    case GDN_OK: return "GDN_OK";
+    case GDN_ERR_INVALID_ARGUMENT: return "GDN_ERR_INVALID_ARGUMENT";
+    case GDN_ERR_UNSUPPORTED: return "GDN_ERR_UNSUPPORTED";
+    case GDN_ERR_WORKSPACE: return "GDN_ERR_WORKSPACE";
+    case GDN_ERR_CUDA: return "GDN_ERR_CUDA";
+    case GDN_ERR_TIMEOUT: return "GDN_ERR_TIMEOUT";
+    default: return "GDN_ERR_UNKNOWN";
+    }
+}
+
+size_t gdn_chunk_fwd_workspace_bytes(int B, int T, int H, int dk, int dv, int chunk, int varlen,
+                                     int dtype)
+{
+    if (check_chunk_shape(B, T, H, dk, dv, chunk, varlen, dtype) != GDN_OK) return (size_t)-1;
+    return chunk_workspace(B, T, H, dk, dv, varlen, dtype);
+}
+
+int gdn_chunk_fwd(const void *q, const void *k, const void *v, const float *log_alpha,
+                  const float *beta, const float *S0, void *out, float *S_final, int B, int T,
+                  int H, int dk, int dv, int chunk, const int32_t *cu_seqlens, int dtype,
+                  void *workspace, size_t workspace_bytes, void *stream)
+{
+    g_last_error[0] = 0;
+    const int varlen = cu_seqlens != nullptr;
+    int rc = check_chunk_shape(B, T, H, dk, dv, chunk, varlen, dtype);
+    if (rc != GDN_OK) return rc;
+    if (!q || !k || !v || !log_alpha || !beta || !out)
+        return fail(GDN_ERR_INVALID_ARGUMENT, "gdn_chunk_fwd: q, k, v, log_alpha, beta and out are required");
+    const void *ptrs[] = {q, k, v, log_alpha, beta, S0, out, S_final, cu_seqlens};
+    for (const void *p : ptrs)
+        if (p && !aligned16(p))
+            return fail(GDN_ERR_INVALID_ARGUMENT, "gdn_chunk_fwd: pointer %p is not 16-byte aligned", p);
+    if (S_final && S_final != S0 && S0) {
+        const size_t bytes = (size_t)B * H * dk * dv * sizeof(float);
+        const char *a0 = (const char *)S0, *b0 = (const char *)S_final;
+        if (a0 < b0 + bytes && b0 < a0 + bytes)
+            return fail(GDN_ERR_INVALID_ARGUMENT, "gdn_chunk_fwd: S0 and S_final overlap partially");
+    }
+    const size_t need = chunk_workspace(B, T, H, dk, dv, varlen, dtype);
+    if (need > 0) {
+        if (!workspace || workspace_bytes < need)
+            return fail(GDN_ERR_WORKSPACE, "gdn_chunk_fwd: workspace of %zu bytes needed, %zu given", need,
+                        workspace ? workspace_bytes : (size_t)0);
+        if (reinterpret_cast<uintptr_t>(workspace) & 255u)
+            return fail(GDN_ERR_INVALID_ARGUMENT, "gdn_chunk_fwd: workspace must be 256-byte aligned");
+    }
+    ChunkArgs a{q, k, v, log_alpha, beta, S0, out, S_final, cu_seqlens, B, T, H, dk, dv, dtype,
+                workspace, workspace_bytes};
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    cudaError_t e = launch_chunk_simt(a, st);
+    if (e != cudaSuccess) return cuda_fail(e, "gdn_chunk_fwd");
+    return GDN_OK;
+}
+
+int gdn_decode_step(const void *q, const void *k, const void *v, const float *log_alpha,
+                    const float *beta, float *S_inout, void *out, int N, int H, int dk, int dv,
+                    int dtype, void *stream)
+{
+    g_last_error[0] = 0;
+    if (dtype != GDN_DTYPE_BF16 && dtype != GDN_DTYPE_F32)
+        return fail(GDN_ERR_UNSUPPORTED, "gdn_decode_step: unknown dtype %d", dtype);
+    if (!head_dim_ok(dk) || !head_dim_ok(dv))
+        return fail(GDN_ERR_UNSUPPORTED, "gdn_decode_step: dk=%d dv=%d, supported: 64 or 128", dk, dv);
+    if (N < 1 || H < 1 || (long long)N * H > (1LL << 30))
+        return fail(GDN_ERR_INVALID_ARGUMENT, "gdn_decode_step: N=%d H=%d out of range", N, H);
+    if (!q || !k || !v || !log_alpha || !beta || !S_inout || !out)
+        return fail(GDN_ERR_INVALID_ARGUMENT, "gdn_decode_step: every pointer is required");
+    const void *ptrs[] = {q, k, v, log_alpha, beta, S_inout, out};
+    for (const void *p : ptrs)
+        if (!aligned16(p))
+            return fail(GDN_ERR_INVALID_ARGUMENT, "gdn_decode_step: pointer %p is not 16-byte aligned", p);
+    cudaError_t e = launch_decode(q, k, v, log_alpha, beta, S_inout, out, N, H, dk, dv, dtype,
+                                  static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "gdn_decode_step");
+    return GDN_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,151 @@
+// gdn_decode.cu -- one-token decode step of the gated delta rule, streamed at HBM speed.
+//
+// Source: Sykra README, "Architectural Highlights" (generation updates a fixed d x d state per
+// token) and "Computational Complexity" (O(d^2) per decode step).  With r = S^T k and s = S^T q
+// taken from the state before the step:
+//     u = b (v - a r),   out = a s + (k . q) u,   S <- a S + k u^T
+// which is S_t = a (I - b k k^T) S + b k v^T followed by out = S_t^T q, regrouped so that the
+// state is read once and written once.
+//
+// Design: one CTA of 256 threads per (n, h) state.  Thread t owns four adjacent value columns
+// (one float4) of every (256 / (dv/4))-th row: a warp covers whole 512-byte rows, so every load
+// and store is a coalesced 16-byte access.  The whole state is loaded into registers before any
+// arithmetic (dk*dv*4 bytes in flight per CTA), the two column sums S^T k and S^T q are reduced
+// across row groups through shared memory, and the updated state is written back with
+// streaming stores.  The state is touched by no other CTA, so there is no inter-CTA traffic.
+#include <cuda_bf16.h>
+
+#include "gdn_internal.h"
+#include "../../include/gdn.h"
+
+namespace gdn {
+namespace {
+
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+template <typename T> __device__ __forceinline__ T from_f32(float x);
+template <> __device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
+    return __float2bfloat16_rn(x);
+}
+
+constexpr int kThreads = 256;
+
+template <int DK, int DV, typename TIn>
+__global__ void __launch_bounds__(kThreads, 2)
+decode_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const TIn *__restrict__ v,
+              const float *__restrict__ log_alpha, const float *__restrict__ beta,
+              float *__restrict__ S, TIn *__restrict__ out)
+{
+    constexpr int TPR = DV / 4;          // threads per state row (one float4 each)
+    constexpr int RPP = kThreads / TPR;  // rows covered per pass
+    constexpr int R = DK / RPP;          // rows per thread
+    static_assert(R * RPP == DK, "row split");
+
+    __shared__ float4 red_r[RPP][TPR];
+    __shared__ float4 red_s[RPP][TPR];
+    __shared__ float red_kq[RPP];
+
+    const size_t u = blockIdx.x;  // state index n * H + h
+    const int tid = threadIdx.x;
+    const int c4 = tid % TPR;
+    const int rg = tid / TPR;  // row group: rows rg, rg + RPP, ...
+
+    float4 *Sp = reinterpret_cast<float4 *>(S + u * (size_t)(DK * DV));
+    float4 s[R];
+#pragma unroll
+    for (int p = 0; p < R; ++p) s[p] = __ldcs(&Sp[(rg + p * RPP) * TPR + c4]);
+
+    const TIn *kp = k + u * DK;
+    const TIn *qp = q + u * DK;
+    float kr[R], qr[R];
+#pragma unroll
+    for (int p = 0; p < R; ++p) {
+        kr[p] = to_f32(kp[rg + p * RPP]);
+        qr[p] = to_f32(qp[rg + p * RPP]);
+    }
+    const float a = expf(log_alpha[u]);
+    const float b = beta[u];
+    float vv[4];
+    {
+        const TIn *vp = v + u * DV + 4 * c4;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) vv[j] = to_f32(vp[j]);
+    }
+
+    // partial column sums over this thread's rows
+    float4 pr = make_float4(0.f, 0.f, 0.f, 0.f), ps = pr;
+    float pkq = 0.f;
+#pragma unroll
+    for (int p = 0; p < R; ++p) {
+        pr.x = fmaf(s[p].x, kr[p], pr.x); pr.y = fmaf(s[p].y, kr[p], pr.y);
+        pr.z = fmaf(s[p].z, kr[p], pr.z); pr.w = fmaf(s[p].w, kr[p], pr.w);
+        ps.x = fmaf(s[p].x, qr[p], ps.x); ps.y = fmaf(s[p].y, qr[p], ps.y);
+        ps.z = fmaf(s[p].z, qr[p], ps.z); ps.w = fmaf(s[p].w, qr[p], ps.w);
+        pkq = fmaf(kr[p], qr[p], pkq);
+    }
+    red_r[rg][c4] = pr;
+    red_s[rg][c4] = ps;
+    if (c4 == 0) red_kq[rg] = pkq;
+    __syncthreads();
+
+    float4 r = make_float4(0.f, 0.f, 0.f, 0.f), sq = r;
+    float kq = 0.f;
+#pragma unroll
+    for (int g = 0; g < RPP; ++g) {
+        const float4 x = red_r[g][c4], y = red_s[g][c4];
+        r.x += x.x; r.y += x.y; r.z += x.z; r.w += x.w;
+        sq.x += y.x; sq.y += y.y; sq.z += y.z; sq.w += y.w;
+        kq += red_kq[g];
+    }
+    // u = b (v - a r)
+    const float u0 = b * (vv[0] - a * r.x), u1 = b * (vv[1] - a * r.y);
+    const float u2 = b * (vv[2] - a * r.z), u3 = b * (vv[3] - a * r.w);
+
+#pragma unroll
+    for (int p = 0; p < R; ++p) {
+        float4 t;
+        t.x = fmaf(a, s[p].x, kr[p] * u0);
+        t.y = fmaf(a, s[p].y, kr[p] * u1);
+        t.z = fmaf(a, s[p].z, kr[p] * u2);
+        t.w = fmaf(a, s[p].w, kr[p] * u3);
+        __stcs(&Sp[(rg + p * RPP) * TPR + c4], t);
+    }
+    if (rg == 0) {
+        TIn *op = out + u * DV + 4 * c4;
+        op[0] = from_f32<TIn>(fmaf(a, sq.x, kq * u0));
+        op[1] = from_f32<TIn>(fmaf(a, sq.y, kq * u1));
+        op[2] = from_f32<TIn>(fmaf(a, sq.z, kq * u2));
+        op[3] = from_f32<TIn>(fmaf(a, sq.w, kq * u3));
+    }
+}
+
+template <typename TIn>
+cudaError_t launch_typed(const void *q, const void *k, const void *v, const float *la,
+                         const float *be, float *S, void *out, int NH, int dk, int dv,
+                         cudaStream_t st)
+{
+    const dim3 grid(NH), block(kThreads);
+    const TIn *Q = static_cast<const TIn *>(q), *K = static_cast<const TIn *>(k),
+              *V = static_cast<const TIn *>(v);
+    TIn *O = static_cast<TIn *>(out);
+    if (dk == 128 && dv == 128) decode_kernel<128, 128, TIn><<<grid, block, 0, st>>>(Q, K, V, la, be, S, O);
+    else if (dk == 128 && dv == 64) decode_kernel<128, 64, TIn><<<grid, block, 0, st>>>(Q, K, V, la, be, S, O);
+    else if (dk == 64 && dv == 128) decode_kernel<64, 128, TIn><<<grid, block, 0, st>>>(Q, K, V, la, be, S, O);
+    else decode_kernel<64, 64, TIn><<<grid, block, 0, st>>>(Q, K, V, la, be, S, O);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_decode(const void *q, const void *k, const void *v, const float *log_alpha,
+                          const float *beta, float *S, void *out, int N, int H, int dk, int dv,
+                          int dtype, cudaStream_t stream)
+{
+    const int NH = N * H;
+    if (dtype == GDN_DTYPE_BF16)
+        return launch_typed<__nv_bfloat16>(q, k, v, log_alpha, beta, S, out, NH, dk, dv, stream);
+    return launch_typed<float>(q, k, v, log_alpha, beta, S, out, NH, dk, dv, stream);
+}
+
+}  // namespace gdn

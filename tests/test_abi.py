@@ -1,0 +1,101 @@
+"""The C-ABI library loads and exports every symbol include/gdn.h declares; host-side validation
+rejects bad arguments before anything is launched (CPU only: no call here reaches a kernel)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import linear_attention_sequence_rule_b200 as gdn
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+FAKE = 1 << 20  # a 16-byte-aligned, never-dereferenced address: every call below fails first
+
+
+def declared_symbols():
+    names = set()
+    for hdr in os.listdir(os.path.join(ROOT, "include")):
+        if hdr.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", hdr)).read()
+            names |= set(re.findall(r"GDN_API[^;(]*?\b(gdn_\w+)\s*\(", text))
+    return names
+
+
+def test_library_exports_every_declared_symbol():
+    names = declared_symbols()
+    assert {"gdn_chunk_fwd", "gdn_decode_step", "gdn_chunk_fwd_workspace_bytes",
+            "gdn_status_string", "gdn_last_error", "gdn_version"} <= names
+    lib = ctypes.CDLL(gdn.LIB_PATH)
+    for n in sorted(names):
+        assert hasattr(lib, n), f"{n} declared in include/ but not exported by libgdn.so"
+
+
+def test_status_strings_and_version():
+    assert gdn.gdn_status_string(0) == "GDN_OK"
+    assert gdn.gdn_status_string(-2) == "GDN_ERR_UNSUPPORTED"
+    assert gdn.gdn_status_string(-99) == "GDN_ERR_UNKNOWN"
+    assert gdn.gdn_version().startswith("gdn-b200")
+
+
+def chunk(**kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, log_alpha=FAKE, beta=FAKE, S0=None, out=FAKE, S_final=None,
+             B=1, T=64, H=1, dk=64, dv=64, chunk=64, cu_seqlens=None, dtype=gdn.GDN_DTYPE_BF16,
+             workspace=None, workspace_bytes=0, stream=None)
+    a.update(kw)
+    return gdn.gdn_chunk_fwd(**a)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(dtype=7), gdn.GDN_ERR_UNSUPPORTED),
+    (dict(dk=96), gdn.GDN_ERR_UNSUPPORTED),
+    (dict(dv=256), gdn.GDN_ERR_UNSUPPORTED),
+    (dict(chunk=32), gdn.GDN_ERR_UNSUPPORTED),
+    (dict(B=0), gdn.GDN_ERR_INVALID_ARGUMENT),
+    (dict(H=0), gdn.GDN_ERR_INVALID_ARGUMENT),
+    (dict(T=0), gdn.GDN_ERR_INVALID_ARGUMENT),
+    (dict(T=-5, cu_seqlens=FAKE), gdn.GDN_ERR_INVALID_ARGUMENT),
+    (dict(q=None), gdn.GDN_ERR_INVALID_ARGUMENT),
+    (dict(out=None), gdn.GDN_ERR_INVALID_ARGUMENT),
+    (dict(beta=None), gdn.GDN_ERR_INVALID_ARGUMENT),
+    (dict(k=FAKE + 4), gdn.GDN_ERR_INVALID_ARGUMENT),
+    (dict(cu_seqlens=FAKE + 8), gdn.GDN_ERR_INVALID_ARGUMENT),
+    (dict(S0=FAKE, S_final=FAKE + 16), gdn.GDN_ERR_INVALID_ARGUMENT),
+])
+def test_chunk_fwd_rejects_bad_arguments(kw, code):
+    assert chunk(**kw) == code
+    assert gdn.gdn_last_error() != ""
+
+
+def test_workspace_query():
+    assert gdn.gdn_chunk_fwd_workspace_bytes(1, 64, 1, 64, 64, 64, 0, 1) >= 0
+    bad = ctypes.c_size_t(-1).value
+    assert gdn.gdn_chunk_fwd_workspace_bytes(1, 64, 1, 96, 64, 64, 0, 1) == bad
+    assert gdn.gdn_chunk_fwd_workspace_bytes(0, 64, 1, 64, 64, 64, 0, 1) == bad
+    assert gdn.gdn_chunk_fwd_workspace_bytes(1, 64, 1, 64, 64, 128, 0, 1) == bad
+
+
+def decode(**kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, log_alpha=FAKE, beta=FAKE, S_inout=FAKE, out=FAKE, N=1, H=1,
+             dk=128, dv=128, dtype=gdn.GDN_DTYPE_BF16, stream=None)
+    a.update(kw)
+    return gdn.gdn_decode_step(**a)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(dtype=3), gdn.GDN_ERR_UNSUPPORTED),
+    (dict(dk=32), gdn.GDN_ERR_UNSUPPORTED),
+    (dict(N=0), gdn.GDN_ERR_INVALID_ARGUMENT),
+    (dict(H=-1), gdn.GDN_ERR_INVALID_ARGUMENT),
+    (dict(S_inout=None), gdn.GDN_ERR_INVALID_ARGUMENT),
+    (dict(out=FAKE + 2), gdn.GDN_ERR_INVALID_ARGUMENT),
+])
+def test_decode_rejects_bad_arguments(kw, code):
+    assert decode(**kw) == code
+    assert gdn.gdn_last_error() != ""
+
+
+def test_torch_layer_checks_shapes_without_launching():
+    import torch
+    q = torch.zeros(1, 64, 1, 64)
+    with pytest.raises(ValueError):
+        gdn.chunk_fwd(q, q, q[..., :32], torch.zeros(1, 64, 1), torch.zeros(1, 64, 2))
