@@ -389,6 +389,22 @@ def run_ours(args, world, rank, local):
     print(json.dumps(line), flush=True)
 
 
+def run_only(args):
+    """One workload's timing loop, no e2e / CPU baseline; prints that workload's numbers."""
+    import linear_attention_sequence_rule_b200 as gdn
+    peaks, _ = load_peaks()
+    stream = torch.cuda.Stream()
+    if args.only == "decode":
+        r = time_decode(gdn, args.steps, args.warmup, stream)
+        r["hbm_frac"] = r["gbs"] / peaks["hbm_gbs"]
+    else:
+        flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device="cuda")
+        d = to_dev(workloads.config_inputs(args.only))
+        r = chunk_numbers(args.only, d, time_chunk(gdn, d, args.steps, args.warmup, flush, stream),
+                          peaks)
+    print(json.dumps({"only": args.only, **r}), flush=True)
+
+
 # ---- reference arm: the fp64 oracle on the host cores ----------------------------------------
 
 def run_reference(args, world, rank):
@@ -448,6 +464,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--quick", action="store_true", help="main workload only")
+    ap.add_argument("--only", choices=["hybrid_lm", "long_context", "varlen", "tiny", "decode"],
+                    help="time one workload's kernel loop only (for profiler runs)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -458,7 +476,10 @@ def main():
         return
     world, rank, local = dist_setup(args.gpus)
     try:
-        run_ours(args, world, rank, local)
+        if args.only:
+            run_only(args)
+        else:
+            run_ours(args, world, rank, local)
     finally:
         if world > 1:
             import torch.distributed as dist

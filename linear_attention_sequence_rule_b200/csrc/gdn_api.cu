@@ -127,7 +127,7 @@ int gdn_chunk_fwd(const void *q, const void *k, const void *v, const float *log_
     ChunkArgs a{q, k, v, log_alpha, beta, S0, out, S_final, cu_seqlens, B, T, H, dk, dv, dtype,
                 workspace, workspace_bytes};
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    cudaError_t e = launch_chunk_simt(a, st);
+    cudaError_t e = dtype == GDN_DTYPE_BF16 ? launch_chunk_tc(a, st) : launch_chunk_simt(a, st);
     if (e != cudaSuccess) return cuda_fail(e, "gdn_chunk_fwd");
     return GDN_OK;
 }

@@ -28,7 +28,14 @@ struct ChunkArgs {
     size_t workspace_bytes;
 };
 
-// Chunk forward on CUDA cores, fp32 arithmetic throughout (any supported dtype).
+// Chunk forward on CUDA cores, fp32 arithmetic throughout (fp32 inputs).
 cudaError_t launch_chunk_simt(const ChunkArgs &a, cudaStream_t stream);
+
+// Chunk forward on the tcgen05 tensor cores (bf16 inputs).
+cudaError_t launch_chunk_tc(const ChunkArgs &a, cudaStream_t stream);
+
+// Device error word of the tensor-core kernels (bounded waits that ran out); read and cleared
+// after synchronising the device.  Returns -1 when the read itself failed.
+int read_and_clear_tc_error();
 
 }  // namespace gdn
