@@ -118,6 +118,15 @@ GDN_API int gdn_decode_step(const void *q, const void *k, const void *v, const f
                     const float *beta, float *S_inout, void *out, int N, int H, int dk, int dv,
                     int dtype, void *stream);
 
+/*
+ * gdn_device_status -- synchronise `stream`, then report whether any kernel of this library
+ * recorded a device-side failure since the previous call (a bounded wait on an mbarrier that ran
+ * out, after which the kernel stopped issuing work and returned): GDN_ERR_TIMEOUT if so, GDN_OK
+ * if not, GDN_ERR_CUDA if the synchronisation itself failed.  The record is per device and is
+ * cleared by this call.
+ */
+GDN_API int gdn_device_status(void *stream);
+
 /* Static text for a status code. */
 GDN_API const char *gdn_status_string(int status);
 

@@ -23,7 +23,7 @@ __all__ = [
     "GdnError", "GDN_OK", "GDN_ERR_INVALID_ARGUMENT", "GDN_ERR_UNSUPPORTED", "GDN_ERR_WORKSPACE",
     "GDN_ERR_CUDA", "GDN_ERR_TIMEOUT", "GDN_DTYPE_F32", "GDN_DTYPE_BF16", "LIB_PATH",
     "gdn_chunk_fwd", "gdn_decode_step", "gdn_chunk_fwd_workspace_bytes", "gdn_status_string",
-    "gdn_last_error", "gdn_version", "chunk_fwd", "decode_step", "workspace_bytes",
+    "gdn_last_error", "gdn_version", "gdn_device_status", "device_status", "chunk_fwd", "decode_step", "workspace_bytes",
 ]
 
 GDN_OK = 0
@@ -39,7 +39,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libgdn.so")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
-        f"{LIB_PATH} is missing: build it with `python -m linear_attention_sequence_rule_b200.build`"
+        f"{LIB_PATH} is missing: build it with `python linear_attention_sequence_rule_b200/build.py`"
         " (there is no fallback implementation)")
 
 _lib = ctypes.CDLL(LIB_PATH)
@@ -52,6 +52,8 @@ _lib.gdn_chunk_fwd_workspace_bytes.argtypes = [_i, _i, _i, _i, _i, _i, _i, _i]
 _lib.gdn_chunk_fwd_workspace_bytes.restype = _sz
 _lib.gdn_decode_step.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp]
 _lib.gdn_decode_step.restype = _i
+_lib.gdn_device_status.argtypes = [_vp]
+_lib.gdn_device_status.restype = _i
 _lib.gdn_status_string.argtypes = [_i]
 _lib.gdn_status_string.restype = ctypes.c_char_p
 _lib.gdn_last_error.argtypes = []
@@ -80,6 +82,17 @@ def gdn_chunk_fwd_workspace_bytes(B, T, H, dk, dv, chunk, varlen, dtype) -> int:
 
 def gdn_decode_step(q, k, v, log_alpha, beta, S_inout, out, N, H, dk, dv, dtype, stream) -> int:
     return _lib.gdn_decode_step(q, k, v, log_alpha, beta, S_inout, out, N, H, dk, dv, dtype, stream)
+
+
+def gdn_device_status(stream) -> int:
+    return _lib.gdn_device_status(stream)
+
+
+def device_status(stream=None) -> None:
+    """Synchronise and raise GdnError if a kernel recorded a device-side timeout."""
+    rc = gdn_device_status(_stream_ptr(stream))
+    if rc != GDN_OK:
+        raise GdnError(rc, gdn_last_error())
 
 
 def gdn_status_string(status: int) -> str:

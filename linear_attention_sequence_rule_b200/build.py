@@ -1,6 +1,8 @@
 """Build libgdn.so (the C-ABI library) in-tree with nvcc for sm_100a.
 
-    python -m linear_attention_sequence_rule_b200.build [--force]
+    python linear_attention_sequence_rule_b200/build.py [--force] [--ptxas-v]
+
+(run as a script, not with -m, so the package -- which loads the library -- is not imported)
 
 The CUDA runtime is linked statically, so the library loads on a machine without a GPU (it only
 needs a driver when a kernel is launched); the driver API is reached through the runtime's
@@ -28,6 +30,11 @@ NVCC_FLAGS = [
 ]
 
 
+# per-file extra flags: the tensor-core kernel runs 288 threads (9 warps), for which 224 registers
+# per thread fit the register file; without the cap the compiler assumes 12 warps (168 registers).
+FILE_FLAGS = {"gdn_chunk_tc.cu": ["-maxrregcount=224"]}
+
+
 def sources():
     return sorted(glob.glob(os.path.join(CSRC, "*.cu")))
 
@@ -50,7 +57,8 @@ def build(force: bool = False, verbose: bool = False, extra_flags=()) -> str:
     objs = []
     for src in sources():
         obj = os.path.join(objdir, os.path.basename(src) + ".o")
-        cmd = [NVCC, *NVCC_FLAGS, *extra_flags, "-c", src, "-o", obj]
+        cmd = [NVCC, *NVCC_FLAGS, *FILE_FLAGS.get(os.path.basename(src), []), *extra_flags, "-c", src,
+               "-o", obj]
         if verbose:
             print(" ".join(cmd), flush=True)
         subprocess.run(cmd, check=True)

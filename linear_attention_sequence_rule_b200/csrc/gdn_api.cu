@@ -155,4 +155,15 @@ int gdn_decode_step(const void *q, const void *k, const void *v, const float *lo
     return GDN_OK;
 }
 
+int gdn_device_status(void *stream)
+{
+    g_last_error[0] = 0;
+    cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "gdn_device_status");
+    const int v = read_and_clear_tc_error();
+    if (v < 0) return fail(GDN_ERR_CUDA, "gdn_device_status: reading the device record failed");
+    if (v) return fail(GDN_ERR_TIMEOUT, "a device-side wait ran out (record 0x%x)", v);
+    return GDN_OK;
+}
+
 }  // extern "C"

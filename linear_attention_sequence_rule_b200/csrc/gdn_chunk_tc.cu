@@ -11,26 +11,26 @@
 //   O  = diag(gam) Q S + lower_incl(Gam o Q K^T) U
 //   S' = gam_C S + K^T diag(lam) U
 //
-// Data flow in one CTA per (sequence, head); 4 warps; thread j owns value column j.
-//   TMA  : K, Q (64 tokens x dk) and V (64 x dv) tiles, 128-byte swizzled, into shared memory.
-//   MMA 1: [K; Q] K^T                   -> TMEM (M=128, N=64)   Gram matrices of the chunk
-//   CUDA : A and P = lower_incl(Gam o Q K^T) with the decays; T = (I + A)^{-1} (fp32 blocked
-//          forward substitution in shared memory); T diag(b), T diag(b gam) in bf16
-//   MMA 2: V^T (T diag b)^T  -> U~^T      K^T (T diag(b gam))^T -> W^T
-//   MMA 3: U^T = U~^T - S^T W^T   (accumulated onto U~^T, A operand negated)
-//          S^T Q^T -> first output term
-//   MMA 4: U^T P^T -> second output term;   (U^T diag lam) K -> state increment
-//   CUDA : S^T <- gam_C S^T + increment (fp32 state kept in TMEM), bf16 copy for the next
-//          chunk's MMAs; outputs o[r][j] = gam_r (S^T Q^T)[j][r] + (U^T P^T)[j][r].
-// Everything after MMA 3 is transposed (value column = TMEM lane), so the chain MMAs have
-// M = dv and each thread handles one value column end to end.
+// One CTA per (sequence, head) runs three roles concurrently (288 threads):
+//   producer warp (warp 8): TMA loads of the K, Q tiles (NS-stage ring) and the V tile.
+//   intra warpgroup (warps 4-7): everything of chunk c+1 that does not depend on the state --
+//       gate sums (warp-shuffle segmented scan), Gram matrices [K;Q] K^T (tcgen05, M=128),
+//       A and P with the decays, T = (I+A)^{-1} (16x16 diagonal blocks by substitution on CUDA
+//       cores, the 16->32->64 merges with mma.sync TF32), T diag(b) and T diag(b gam) in bf16,
+//       U~^T and W^T (tcgen05), then gam-scaled Q and lam-scaled K in place.
+//   chain warpgroup (warps 0-3): the state-dependent part of chunk c, thread j = value column j:
+//       U^T   = U~^T - S^T W^T           (accumulated onto U~^T, A operand negated)
+//       O^T   = S^T (gam Q)^T + U^T P^T  (one accumulator, double-buffered across chunks)
+//       S'^T  = gam_C S^T + U^T (lam K)  (accumulated onto the pre-scaled fp32 state in TMEM)
+//   so the chain's critical path per chunk is two MMA round trips.
+// The output epilogue of chunk c overlaps the first chain MMA of chunk c+1.
 //
 // Gates: decays are exp of log_alpha sums taken from the last exact reset (log_alpha = -inf)
 // inside the chunk.  Padded rows of a partial chunk get b = 0 and log_alpha = 0, which makes
 // their (finite) K/Q/V contents contribute nothing.
 //
-// Every wait on an mbarrier is bounded (2 s); on timeout the kernel records an error word and
-// stops issuing work, then frees its TMEM and returns.
+// Every mbarrier wait is bounded (2 s).  On timeout the kernel records an error word, stops
+// issuing work and skips all later waits, so it always reaches the end, frees TMEM and returns.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_bf16.h>
@@ -49,142 +49,288 @@ namespace {
 using namespace sm100;
 
 constexpr int CH = 64;
-constexpr int kThreads = 128;
+constexpr int kThreads = 256;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
-constexpr int LDF = 65;  // padded fp32 row stride of the 64 x 64 scratch matrices
+constexpr int LDF = 68;  // fp32 row stride of the 64 x 64 solve matrices
+// Thread roles inside the intra warpgroup: its MMAs and V loads are issued by warp 7 and the gate
+// scan runs on warp 5, away from warp 4, which shares an SM sub-partition with the chain's
+// issuing thread (thread 0).
+constexpr int kIntraIssuer = 96;
+constexpr int kScanWarp = 1;
 
 template <int DK, int DV>
-struct TcLayout {
-    static constexpr int KQ = 0;                             // per 64-feature block: K (8 KB) | Q (8 KB)
-    static constexpr int V = KQ + (DK / 64) * 16384;         // per 64-column block: 8 KB
-    static constexpr int ST = V + (DV / 64) * 8192;          // S^T bf16, per 64-feature block DV x 128 B
-    static constexpr int WT = ST + (DK / 64) * DV * 128;     // W^T bf16, DK rows x 128 B
-    static constexpr int PM = WT + DK * 128;                 // P bf16, 64 x 128 B
-    static constexpr int TB = PM + 8192;                     // T diag(b)
-    static constexpr int TG = TB + 8192;                     // T diag(b gam)
-    static constexpr int UT = TG + 8192;                     // U^T bf16, DV x 128 B
-    static constexpr int UL = UT + DV * 128;                 // (U^T diag lam) bf16
-    static constexpr int AF = UL + DV * 128;                 // A fp32 [64][65]
-    static constexpr int TF = AF + CH * LDF * 4;             // T fp32 [64][65]
-    static constexpr int XF = TF + CH * LDF * 4;             // merge scratch fp32 [64][65]
-    static constexpr int GT = XF + CH * LDF * 4;             // gate vectors (8 x 64 x 4 B)
-    static constexpr int BAR = GT + 8 * CH * 4;              // mbarriers + TMEM slot
-    static constexpr int TOTAL = BAR + 64;
+struct TcCfg {
+    static constexpr int NS = (DK == 128 || DV == 128) ? 2 : 3;  // K/Q stages
+    // shared memory byte offsets (swizzled tiles first, all 1024-aligned)
+    static constexpr int KQ = 0;                                 // per stage: per 64-feature block K (8K) | Q (8K)
+    static constexpr int KQ_STAGE = (DK / 64) * 16384;
+    static constexpr int V = KQ + NS * KQ_STAGE;                 // per 64-column block 8 KB
+    static constexpr int WT = V + (DV / 64) * 8192;              // W^T bf16, DK rows x 128 B
+    static constexpr int PM = WT + DK * 128;                     // per stage: P bf16, 64 x 128 B
+    static constexpr int TB = PM + NS * 8192;                    // T diag(b)
+    static constexpr int TG = TB + 8192;                         // T diag(b gam)
+    static constexpr int ST = TG + 8192;                         // S^T bf16, per 64-feature block DV x 128 B
+    static constexpr int UT = ST + (DK / 64) * DV * 128;         // U^T bf16, DV x 128 B
+    static constexpr int AF = UT + DV * 128;                     // A fp32 [64][LDF]
+    static constexpr int TF = AF + CH * LDF * 4;                 // T fp32 [64][LDF]
+    static constexpr int XS = TF + CH * LDF * 4;                 // per-warp merge scratch, 4 x 256 fp32
+    static constexpr int GT = XS + 4 * 256 * 4;                  // per stage: gate vectors
+    static constexpr int GT_STAGE = 7 * CH * 4;                  //   graw, G2, gam, lam, bet, last, (gC)
+    static constexpr int BAR = GT + NS * GT_STAGE;
+    static constexpr int NBAR = 5 * NS + 8;
+    static constexpr int MISC = BAR + NBAR * 8;                  // TMEM slot, abort flag
+    static constexpr int TOTAL = MISC + 16;
+    // TMEM columns
+    static constexpr uint32_t T_O = 0;                            // DV: output rows (M = 64 tokens)
+    static constexpr uint32_t T_S = DV;                           // DK: fp32 state (transposed)
+    static constexpr uint32_t T_G = DV + DK;                      // 64: Gram, then W^T (intra)
+    static constexpr uint32_t T_W = T_G;
+    static constexpr uint32_t T_U = T_G + 64;                     // NS x 64: U~^T / U^T
+    static_assert(T_U + NS * 64 <= 512, "TMEM budget");
+    static_assert(TOTAL + 1024 <= 232448, "shared memory budget");
 };
 
-__device__ __forceinline__ void record_error(int code, int *abort_flag)
+// barrier indices
+template <int NS> struct Bars {
+    static constexpr int kq_full = 0;            // [NS]
+    static constexpr int v_full = NS;
+    static constexpr int v_empty = NS + 1;
+    static constexpr int cdone = NS + 2;         // [NS]
+    static constexpr int ready = 2 * NS + 2;     // [NS]
+    static constexpr int gready = 3 * NS + 2;    // [NS]
+    static constexpr int wt_free = 4 * NS + 2;
+    static constexpr int gram = 4 * NS + 3;
+    static constexpr int uw = 4 * NS + 4;
+    static constexpr int u = 4 * NS + 5;
+    static constexpr int s = 4 * NS + 6;
+    static constexpr int o = 4 * NS + 7;
+    static constexpr int gfull = 4 * NS + 8;     // [NS], 32 arrivals (cp.async of chain warp 0)
+};
+
+struct Ctl {
+    uint64_t *bar;
+    int *abort;
+    __device__ void wait(int i, uint32_t parity) const
+    {
+        if (*(volatile int *)abort) return;
+        if (!mbar_wait_bounded(&bar[i], parity, kWaitLimitNs)) {
+            atomicOr(&g_tc_device_error, 1);
+            *(volatile int *)abort = 1;
+        }
+    }
+    __device__ bool aborted() const { return *(volatile int *)abort != 0; }
+    __device__ void arrive(int i) const
+    {
+        asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&bar[i])) : "memory");
+    }
+};
+
+__device__ __forceinline__ void named_bar(int id, int n) { asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory"); }
+
+__device__ __forceinline__ uint32_t f2tf32(float x)
 {
-    atomicOr(&g_tc_device_error, code);
-    *abort_flag = 1;
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return r;
 }
 
-// T = (I + A)^{-1} for strictly lower triangular A (64 x 64 fp32, row stride LDF), by blocked
-// forward substitution: the four 16 x 16 diagonal blocks by substitution, then the 16 -> 32
-// and 32 -> 64 merges T_ba = -T_bb A_ba T_aa.  Only the lower triangle of Tm is written.
-// Called by all 128 threads; contains __syncthreads.
-__device__ void solve_unit_lower(const float *A, float *Tm, float *X, int tid)
+__device__ __forceinline__ void mma_tf32(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1)
 {
-    if (tid < 64) {
-        const int o = (tid >> 4) * 16, c = tid & 15;
-        float x[16];
-#pragma unroll
-        for (int r = 0; r < 16; ++r) {
-            float v = 0.f;
-#pragma unroll
-            for (int i = 0; i < r; ++i)
-                if (i >= c) v = fmaf(A[(o + r) * LDF + o + i], x[i], v);
-            x[r] = (r < c) ? 0.f : (r == c ? 1.f : -v);
-        }
-#pragma unroll
-        for (int r = 0; r < 16; ++r)
-            if (r >= c) Tm[(o + r) * LDF + o + c] = x[r];
-    }
-    __syncthreads();
-    // 16 -> 32: pairs (blocks 0,1) and (2,3).  X = A_ba T_aa, then T_ba = -T_bb X.
+    asm volatile(
+        "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Final value v of T[r][c]: keep it in fp32 for later merges and write the bf16 entries of
+// T diag(b) and T diag(b gam) (128B-swizzled rows, the B operands of the WY products).
+struct TOut {
+    float *Tm;
+    unsigned char *TB, *TG;
+    const float *bet, *gam;
+    __device__ __forceinline__ void put(int r, int c, float v) const
     {
-        const int p = tid >> 6, rem = tid & 63, r = rem >> 2, c0 = (rem & 3) * 4;
-        const int oa = 32 * p, ob = oa + 16;
-        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+        Tm[r * LDF + c] = v;
+        const float b = v * bet[c];
+        *reinterpret_cast<__nv_bfloat16 *>(TB + sw128_off(r, c)) = __float2bfloat16_rn(b);
+        *reinterpret_cast<__nv_bfloat16 *>(TG + sw128_off(r, c)) = __float2bfloat16_rn(b * gam[c]);
+    }
+    __device__ __forceinline__ void put2(int r, int c, float v0, float v1) const  // c even
+    {
+        *reinterpret_cast<float2 *>(&Tm[r * LDF + c]) = make_float2(v0, v1);
+        const float b0 = v0 * bet[c], b1 = v1 * bet[c + 1];
+        *reinterpret_cast<uint32_t *>(TB + sw128_off(r, c)) = pack_bf16x2(b0, b1);
+        *reinterpret_cast<uint32_t *>(TG + sw128_off(r, c)) = pack_bf16x2(b0 * gam[c], b1 * gam[c + 1]);
+    }
+};
+
+// T = (I + A)^{-1} for strictly lower triangular A (64 x 64 fp32, row stride LDF; only entries
+// below the diagonal are read), executed by the 128 threads of the intra warpgroup (t = 0..127).
+// Warp w inverts the 16 x 16 diagonal block w by recursive doubling (2 -> 4 -> 8 -> 16,
+// warp-synchronous, CUDA cores); the 16 -> 32 and 32 -> 64 merges T_ba = -T_bb (A_ba T_aa) run on
+// mma.sync TF32 (T is rounded to bf16 afterwards, so TF32 products stay below that rounding).
+// Every entry of the lower triangle is written exactly once, through `out`; entries above the
+// diagonal are never written (the caller keeps them zero in the bf16 copies).
+__device__ void solve_unit_lower(const float *A, const TOut &out, float *XS, int t, int bar_id)
+{
+    float *Tm = out.Tm;
+    const int w = t >> 5, lane = t & 31, g = lane >> 2, tq = lane & 3;
+    float *xs = XS + w * 256;
+    {
+        const int o = 16 * w;
+        if (lane < 16) out.put(o + lane, o + lane, 1.f);
+        __syncwarp();
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            const float a = A[(ob + r) * LDF + oa + i];
+        for (int s = 1; s <= 8; s <<= 1) {
+            const int nout = 8 * s;  // (16 / 2s) pairs x s^2 outputs
 #pragma unroll
-            for (int q = 0; q < 4; ++q)
-                if (i >= c0 + q) acc[q] = fmaf(a, Tm[(oa + i) * LDF + oa + c0 + q], acc[q]);
+            for (int q0 = 0; q0 < nout; q0 += 32) {
+                const int q = q0 + lane;
+                if (q < nout) {
+                    const int p = q / (s * s), rem = q % (s * s), i = rem / s, jj = rem % s;
+                    const int a0 = o + 2 * p * s, b0 = a0 + s;
+                    float acc = 0.f;
+#pragma unroll
+                    for (int k = 0; k < s; ++k)
+                        if (k >= jj) acc = fmaf(A[(b0 + i) * LDF + a0 + k], Tm[(a0 + k) * LDF + a0 + jj], acc);
+                    xs[i * 16 + p * s + jj] = acc;
+                }
+            }
+            __syncwarp();
+#pragma unroll
+            for (int q0 = 0; q0 < nout; q0 += 32) {
+                const int q = q0 + lane;
+                if (q < nout) {
+                    const int p = q / (s * s), rem = q % (s * s), i = rem / s, jj = rem % s;
+                    const int a0 = o + 2 * p * s, b0 = a0 + s;
+                    float acc = xs[i * 16 + p * s + jj];  // diagonal term (T_bb[i][i] = 1)
+#pragma unroll
+                    for (int k = 0; k < s; ++k)
+                        if (k < i) acc = fmaf(Tm[(b0 + i) * LDF + b0 + k], xs[k * 16 + p * s + jj], acc);
+                    out.put(b0 + i, a0 + jj, -acc);
+                }
+            }
+            __syncwarp();
         }
+    }
+    named_bar(bar_id, 128);
+    // ---- 16 -> 32: pair p = w/2 (blocks 2p, 2p+1), output column tile nt = w%2 ----
+    {
+        const int p = w >> 1, nt = w & 1, oa = 32 * p, ob = oa + 16, n = oa + 8 * nt + g;
+        float d[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int q = 0; q < 4; ++q) X[(ob + r) * LDF + oa + c0 + q] = acc[q];
-        __syncthreads();
-        float t[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int kk = 0; kk < 2; ++kk) {
+            if (kk < nt) continue;
+            const int k0 = oa + 8 * kk + tq, k1 = k0 + 4;
+            mma_tf32(d, f2tf32(A[(ob + g) * LDF + k0]), f2tf32(A[(ob + g + 8) * LDF + k0]),
+                     f2tf32(A[(ob + g) * LDF + k1]), f2tf32(A[(ob + g + 8) * LDF + k1]),
+                     f2tf32(k0 >= n ? Tm[k0 * LDF + n] : 0.f), f2tf32(k1 >= n ? Tm[k1 * LDF + n] : 0.f));
+        }
+        xs[g * 8 + 2 * tq] = d[0];
+        xs[g * 8 + 2 * tq + 1] = d[1];
+        xs[(g + 8) * 8 + 2 * tq] = d[2];
+        xs[(g + 8) * 8 + 2 * tq + 1] = d[3];
+        __syncwarp();
+        float e[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            if (i <= r) {
-                const float b = Tm[(ob + r) * LDF + ob + i];
+        for (int kk = 0; kk < 2; ++kk) {
+            const int k0 = 8 * kk + tq, k1 = k0 + 4;
+            mma_tf32(e, f2tf32(k0 <= g ? Tm[(ob + g) * LDF + ob + k0] : 0.f),
+                     f2tf32(k0 <= g + 8 ? Tm[(ob + g + 8) * LDF + ob + k0] : 0.f),
+                     f2tf32(k1 <= g ? Tm[(ob + g) * LDF + ob + k1] : 0.f),
+                     f2tf32(k1 <= g + 8 ? Tm[(ob + g + 8) * LDF + ob + k1] : 0.f),
+                     f2tf32(xs[k0 * 8 + g]), f2tf32(xs[k1 * 8 + g]));
+        }
+        const int c0 = oa + 8 * nt + 2 * tq;
+        out.put2(ob + g, c0, -e[0], -e[1]);
+        out.put2(ob + g + 8, c0, -e[2], -e[3]);
+    }
+    named_bar(bar_id, 128);
+    // ---- 32 -> 64: a = [0,32), b = [32,64); warp w takes output column tile wt = 3 - w (columns
+    //      8wt..8wt+7; tile 3 has the fewest products and goes to warp 0) ----
+    {
+        const int wt = 3 - w;
+        const int n = 8 * wt + g;
+        float d[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
-                for (int q = 0; q < 4; ++q) t[q] = fmaf(b, X[(ob + i) * LDF + oa + c0 + q], t[q]);
+        for (int kk = 0; kk < 4; ++kk) {
+            if (kk < wt) continue;
+            const int k0 = 8 * kk + tq, k1 = k0 + 4;
+            const uint32_t b0 = f2tf32(k0 >= n ? Tm[k0 * LDF + n] : 0.f);
+            const uint32_t b1 = f2tf32(k1 >= n ? Tm[k1 * LDF + n] : 0.f);
+#pragma unroll
+            for (int mt = 0; mt < 2; ++mt) {
+                const int r = 32 + 16 * mt + g;
+                mma_tf32(d[mt], f2tf32(A[r * LDF + k0]), f2tf32(A[(r + 8) * LDF + k0]),
+                         f2tf32(A[r * LDF + k1]), f2tf32(A[(r + 8) * LDF + k1]), b0, b1);
             }
         }
 #pragma unroll
-        for (int q = 0; q < 4; ++q) Tm[(ob + r) * LDF + oa + c0 + q] = -t[q];
-    }
-    __syncthreads();
-    // 32 -> 64: X = A_ba T_aa with a = [0,32), b = [32,64); then T_ba = -T_bb X.
-    {
-        const int r = tid >> 2, c0 = (tid & 3) * 8;
-        float acc[8];
-#pragma unroll
-        for (int q = 0; q < 8; ++q) acc[q] = 0.f;
-#pragma unroll 8
-        for (int i = 0; i < 32; ++i) {
-            const float a = A[(32 + r) * LDF + i];
-#pragma unroll
-            for (int q = 0; q < 8; ++q)
-                if (i >= c0 + q) acc[q] = fmaf(a, Tm[i * LDF + c0 + q], acc[q]);
+        for (int mt = 0; mt < 2; ++mt) {
+            xs[(16 * mt + g) * 8 + 2 * tq] = d[mt][0];
+            xs[(16 * mt + g) * 8 + 2 * tq + 1] = d[mt][1];
+            xs[(16 * mt + g + 8) * 8 + 2 * tq] = d[mt][2];
+            xs[(16 * mt + g + 8) * 8 + 2 * tq + 1] = d[mt][3];
         }
+        __syncwarp();
 #pragma unroll
-        for (int q = 0; q < 8; ++q) X[(32 + r) * LDF + c0 + q] = acc[q];
-        __syncthreads();
-        float t[8];
+        for (int mt = 0; mt < 2; ++mt) {
+            float e[4] = {0.f, 0.f, 0.f, 0.f};
+            const int rl = 16 * mt + g, rh = rl + 8;
 #pragma unroll
-        for (int q = 0; q < 8; ++q) t[q] = 0.f;
-#pragma unroll 8
-        for (int i = 0; i < 32; ++i) {
-            if (i <= r) {
-                const float b = Tm[(32 + r) * LDF + 32 + i];
-#pragma unroll
-                for (int q = 0; q < 8; ++q) t[q] = fmaf(b, X[(32 + i) * LDF + c0 + q], t[q]);
+            for (int kk = 0; kk < 4; ++kk) {
+                if (kk > 2 * mt + 1) continue;
+                const int k0 = 8 * kk + tq, k1 = k0 + 4;
+                mma_tf32(e, f2tf32(k0 <= rl ? Tm[(32 + rl) * LDF + 32 + k0] : 0.f),
+                         f2tf32(k0 <= rh ? Tm[(32 + rh) * LDF + 32 + k0] : 0.f),
+                         f2tf32(k1 <= rl ? Tm[(32 + rl) * LDF + 32 + k1] : 0.f),
+                         f2tf32(k1 <= rh ? Tm[(32 + rh) * LDF + 32 + k1] : 0.f),
+                         f2tf32(xs[k0 * 8 + g]), f2tf32(xs[k1 * 8 + g]));
             }
+            const int c0 = 8 * wt + 2 * tq;
+            out.put2(32 + rl, c0, -e[0], -e[1]);
+            out.put2(32 + rh, c0, -e[2], -e[3]);
         }
-#pragma unroll
-        for (int q = 0; q < 8; ++q) Tm[(32 + r) * LDF + c0 + q] = -t[q];
     }
-    __syncthreads();
+}
+
+// Scale row r (64 bf16 = 128 swizzled bytes, 8 chunks of 16 B) of a tile by s, chunks [c0, c1).
+__device__ __forceinline__ void scale_row_bf16(unsigned char *tile, int row, float s, int c0, int c1)
+{
+#pragma unroll
+    for (int c = c0; c < c1; ++c) {
+        uint4 *p = reinterpret_cast<uint4 *>(tile + row * 128 + c * 16);
+        uint4 w = *p;
+        uint32_t *u = reinterpret_cast<uint32_t *>(&w);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            __nv_bfloat162 h = *reinterpret_cast<__nv_bfloat162 *>(&u[e]);
+            float2 f = __bfloat1622float2(h);
+            u[e] = pack_bf16x2(f.x * s, f.y * s);
+        }
+        *p = w;
+    }
 }
 
 template <int DK, int DV>
-__global__ void __launch_bounds__(kThreads, 1)
-chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+__global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                 const __grid_constant__ CUtensorMap tmV, const float *__restrict__ log_alpha,
                 const float *__restrict__ beta, const float *__restrict__ S0,
                 __nv_bfloat16 *__restrict__ out, float *__restrict__ S_final,
                 const int32_t *__restrict__ cu_seqlens, int T, int H)
 {
-    using L = TcLayout<DK, DV>;
+    using L = TcCfg<DK, DV>;
+    constexpr int NS = L::NS;
+    using B = Bars<NS>;
     extern __shared__ unsigned char smem_raw[];
     unsigned char *sm = reinterpret_cast<unsigned char *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-    float *Af = reinterpret_cast<float *>(sm + L::AF);
-    float *Tf = reinterpret_cast<float *>(sm + L::TF);
-    float *Xf = reinterpret_cast<float *>(sm + L::XF);
-    float *graw = reinterpret_cast<float *>(sm + L::GT);
-    float *Gs = graw + CH;
-    float *gam = graw + 2 * CH;
-    float *lam = graw + 3 * CH;
-    float *bet = graw + 4 * CH;
-    int *last = reinterpret_cast<int *>(graw + 5 * CH);
-    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + L::BAR);  // [0] TMA, [1] MMA
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + L::BAR + 16);
-    int *abort_flag = reinterpret_cast<int *>(sm + L::BAR + 20);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + L::BAR);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + L::MISC);
+    int *abort_flag = reinterpret_cast<int *>(sm + L::MISC + 4);
+    const Ctl ctl{bars, abort_flag};
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int h = blockIdx.y, s = blockIdx.z;
@@ -196,16 +342,13 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         tok0 = (long)s * T;
         len = T;
     }
+    const int nchunks = (int)((len + CH - 1) / CH);
     const size_t sbase = ((size_t)s * H + h) * (size_t)DK * DV;
 
     if (tid == 0) {
-        mbar_init(&bars[0], 1);
-        mbar_init(&bars[1], 1);
+        for (int i = 0; i < L::NBAR; ++i) mbar_init(&bars[i], i >= B::gfull ? 32 : 1);
         fence_mbar_init();
         *abort_flag = 0;
-        prefetch_tmap(&tmQ);
-        prefetch_tmap(&tmK);
-        prefetch_tmap(&tmV);
     }
     if (warp == 0) {
         tmem_alloc(tmem_slot, 512);
@@ -215,291 +358,396 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);  // this warp's TMEM lanes
-    constexpr uint32_t C_G = 0, C_O1 = 0, C_W = 64, C_O2 = 64, C_U = 128, C_DS = 192,
-                       C_S = 192 + DK;
-    // Rows owned in accumulators with M = DV (value columns) and M = DK (key features).
-    // M = 128: row = thread; M = 64: rows 16w..16w+15 sit in lanes 0..15 of warp w.
-    const int jrow = (DV == 128) ? tid : (lane < 16 ? warp * 16 + lane : -1);
-    const int crow = (DK == 128) ? tid : (lane < 16 ? warp * 16 + lane : -1);
 
-    // ---- initial state: thread jrow holds column jrow of S as a row of S^T ----
-#pragma unroll 1
-    for (int cb = 0; cb < DK / 32; ++cb) {
-        float x[32];
+    auto gates = [&](int stage) { return reinterpret_cast<float *>(sm + L::GT + stage * L::GT_STAGE); };
+    // Loads of chunk c into K/Q stage c % NS: gates by cp.async from the 32 lanes of warp 0
+    // (rows past the sequence end are zero-filled), K and Q tiles by TMA from thread 0.
+    auto load_kq = [&](int c) {
+        const int st = c % NS;
+        const long tk = tok0 + (long)c * CH;
+        const int n = (int)min((long)CH, len - (long)c * CH);
+        float *gv = gates(st);
 #pragma unroll
-        for (int i = 0; i < 32; ++i)
-            x[i] = (jrow >= 0 && S0) ? S0[sbase + (size_t)(cb * 32 + i) * DV + jrow] : 0.f;
-        tmem_st32(tl + C_S + cb * 32, x);
-        if (jrow >= 0) {
-            unsigned char *st = sm + L::ST + (cb >> 1) * (DV * 128);
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                const int chunk = (cb & 1) * 4 + c;
-                uint4 w;
-                w.x = pack_bf16x2(x[8 * c + 0], x[8 * c + 1]);
-                w.y = pack_bf16x2(x[8 * c + 2], x[8 * c + 3]);
-                w.z = pack_bf16x2(x[8 * c + 4], x[8 * c + 5]);
-                w.w = pack_bf16x2(x[8 * c + 6], x[8 * c + 7]);
-                *reinterpret_cast<uint4 *>(st + jrow * 128 + (((chunk ^ (jrow & 7)) & 7) << 4)) = w;
-            }
+        for (int k2 = 0; k2 < 2; ++k2) {
+            const int r = lane + 32 * k2;
+            const size_t off = (size_t)(tk + min(r, n - 1)) * H + h;
+            cp_async_4(&gv[r], log_alpha + off, r < n ? 4u : 0u);
+            cp_async_4(&gv[4 * CH + r], beta + off, r < n ? 4u : 0u);
         }
-    }
-    tmem_wait_st();
-    fence_proxy_async_smem();
-    tc_fence_before();
-    __syncthreads();
-
-    uint32_t ph_tma = 0, ph_mma = 0;
-    auto wait_mma = [&]() {
-        if (!*abort_flag && !mbar_wait_bounded(&bars[1], ph_mma, kWaitLimitNs)) record_error(1, abort_flag);
-        ph_mma ^= 1;
-        tc_fence_after();
-    };
-
-#pragma unroll 1
-    for (long c0 = 0; c0 < len; c0 += CH) {
-        if (*abort_flag) break;
-        const int n = (int)min((long)CH, len - c0);
-        const long tk = tok0 + c0;
-        if (tid == 0) {
-            mbar_arrive_expect_tx(&bars[0], (2 * (DK / 64) + DV / 64) * 8192);
-#pragma unroll
+        cp_async_mbar_arrive(&bars[B::gfull + st]);
+        if (lane == 0 && !ctl.aborted()) {
+            mbar_arrive_expect_tx(&bars[B::kq_full + st], 2 * (DK / 64) * 8192);
+            unsigned char *kq = sm + L::KQ + st * L::KQ_STAGE;
             for (int kb = 0; kb < DK / 64; ++kb) {
-                tma_load_3d(sm + L::KQ + kb * 16384, &tmK, &bars[0], kb * 64, h, (int)tk);
-                tma_load_3d(sm + L::KQ + kb * 16384 + 8192, &tmQ, &bars[0], kb * 64, h, (int)tk);
+                tma_load_3d(kq + kb * 16384, &tmK, &bars[B::kq_full + st], kb * 64, h, (int)tk);
+                tma_load_3d(kq + kb * 16384 + 8192, &tmQ, &bars[B::kq_full + st], kb * 64, h, (int)tk);
             }
+        }
+    };
+    auto load_v = [&](int c) {
+        if (ctl.aborted()) return;
+        const int tk = (int)(tok0 + (long)c * CH);
+        mbar_arrive_expect_tx(&bars[B::v_full], (DV / 64) * 8192);
+        for (int vb = 0; vb < DV / 64; ++vb)
+            tma_load_3d(sm + L::V + vb * 8192, &tmV, &bars[B::v_full], vb * 64, h, tk);
+    };
+    if (warp == 0) {
+        if (lane == 0) {
+            prefetch_tmap(&tmQ);
+            prefetch_tmap(&tmK);
+            prefetch_tmap(&tmV);
+        }
+        for (int c = 0; c < min(nchunks, NS); ++c) load_kq(c);
+    }
+    if (tid == 128 + kIntraIssuer && nchunks > 0) load_v(0);
+
+    if (warp >= 4) {
+        // ======================= intra warpgroup =======================
+        const int t = tid - 128, wi = t >> 5;
+        const uint32_t tl = tmem + ((uint32_t)(wi * 32) << 16);
+        const int crow = (DK == 128) ? t : (lane < 16 ? wi * 16 + lane : -1);  // row of W^T
+        float *AF = reinterpret_cast<float *>(sm + L::AF);
+        float *TFm = reinterpret_cast<float *>(sm + L::TF);
+        float *XSm = reinterpret_cast<float *>(sm + L::XS);
+        for (int i = t; i < 2 * 8192 / 16; i += 128)
+            reinterpret_cast<uint4 *>(sm + L::TB)[i] = make_uint4(0u, 0u, 0u, 0u);
+        for (int c = 0; c < nchunks; ++c) {
+            const int st = c % NS;
+            const long tk = tok0 + (long)c * CH;
+            const int n = (int)min((long)CH, len - (long)c * CH);
+            float *gv = gates(st);
+            float *graw = gv, *Gs = gv + CH, *gam = gv + 2 * CH, *lam = gv + 3 * CH, *bet = gv + 4 * CH;
+            int *last = reinterpret_cast<int *>(gv + 5 * CH);
+            float *gC = gv + 6 * CH;
+            unsigned char *Kt = sm + L::KQ + st * L::KQ_STAGE;  // K at +0, Q at +8192 per block
+            if (c >= NS) ctl.wait(B::cdone + st, ((c / NS) - 1) & 1);
+            // ---- gates: segmented scan of log_alpha (restarts at exact resets) ----
+            if (wi == kScanWarp) {
+                ctl.wait(B::gfull + st, (c / NS) & 1);
+                const int r0 = 2 * lane, r1 = r0 + 1;
+                const float g0 = graw[r0], g1 = graw[r1];
+                const bool f0 = (g0 == -INFINITY), f1 = (g1 == -INFINITY);
+                const float v0 = f0 ? 0.f : g0, v1 = f1 ? 0.f : g1;
+                // inclusive pair value and reset flag, then a segmented warp scan over lanes
+                float a = f1 ? v1 : v0 + v1;
+                int fa = (f0 || f1) ? 1 : 0;
+                int li = f1 ? r1 : (f0 ? r0 : -1);
 #pragma unroll
-            for (int vb = 0; vb < DV / 64; ++vb)
-                tma_load_3d(sm + L::V + vb * 8192, &tmV, &bars[0], vb * 64, h, (int)tk);
-        }
-        // ---- gates: sums of log_alpha from the last reset (or the chunk start) ----
-        if (tid < CH) {
-            const bool ok = tid < n;
-            graw[tid] = ok ? log_alpha[(size_t)(tk + tid) * H + h] : 0.f;
-            bet[tid] = ok ? beta[(size_t)(tk + tid) * H + h] : 0.f;
-        }
-        __syncthreads();
-        if (tid < CH) {
-            float acc = 0.f;
-            int lst = -1;
-            for (int j = 0; j <= tid; ++j) {
-                const float g = graw[j];
-                if (g == -INFINITY) {
-                    lst = j;
-                    acc = 0.f;
-                } else {
-                    acc += g;
+                for (int off = 1; off < 32; off <<= 1) {
+                    const float ab = __shfl_up_sync(0xffffffffu, a, off);
+                    const int fb = __shfl_up_sync(0xffffffffu, fa, off);
+                    const int lb = __shfl_up_sync(0xffffffffu, li, off);
+                    if (lane >= off) {
+                        a = fa ? a : ab + a;
+                        fa |= fb;
+                        li = max(li, lb);
+                    }
+                }
+                float ex = __shfl_up_sync(0xffffffffu, a, 1);
+                int lex = __shfl_up_sync(0xffffffffu, li, 1);
+                if (lane == 0) { ex = 0.f; lex = -1; }
+                // sums in the log2 domain, so every decay below is a single exp2
+                constexpr float kLog2e = 1.4426950408889634f;
+                const float G0 = f0 ? 0.f : ex + v0;
+                const float G1 = f1 ? 0.f : G0 + v1;
+                const float H0 = G0 * kLog2e, H1 = G1 * kLog2e;
+                const int L0 = f0 ? r0 : lex;
+                const int L1 = f1 ? r1 : L0;
+                Gs[r0] = H0; Gs[r1] = H1;
+                last[r0] = L0; last[r1] = L1;
+                __syncwarp();
+                const int l63 = last[CH - 1];
+                const float G63 = Gs[CH - 1];
+                gam[r0] = L0 >= 0 ? 0.f : exp2f(H0);
+                gam[r1] = L1 >= 0 ? 0.f : exp2f(H1);
+                lam[r0] = l63 > r0 ? 0.f : exp2f(G63 - H0);
+                lam[r1] = l63 > r1 ? 0.f : exp2f(G63 - H1);
+                __syncwarp();
+                if (lane == 0) {
+                    gC[0] = gam[CH - 1];
+                    ctl.arrive(B::gready + st);
                 }
             }
-            Gs[tid] = acc;
-            last[tid] = lst;
-        }
-        __syncthreads();
-        if (tid < CH) {
-            gam[tid] = last[tid] >= 0 ? 0.f : expf(Gs[tid]);
-            lam[tid] = last[CH - 1] > tid ? 0.f : expf(Gs[CH - 1] - Gs[tid]);
-        }
-        if (!*abort_flag && !mbar_wait_bounded(&bars[0], ph_tma, kWaitLimitNs)) record_error(2, abort_flag);
-        ph_tma ^= 1;
-        __syncthreads();
-
-        // ---- MMA 1: Gram matrices [K; Q] K^T ----
-        if (tid == 0 && !*abort_flag) {
+            named_bar(2, 128);
+            // ---- Gram matrices [K; Q] K^T ----
+            ctl.wait(B::kq_full + st, (c / NS) & 1);
+            if (t == kIntraIssuer && !ctl.aborted()) {
+                tc_fence_after();
+                constexpr uint32_t id = idesc_bf16(128, 64, 0, 0);
+#pragma unroll
+                for (int kk = 0; kk < DK / 16; ++kk) {
+                    const uint32_t a = smem_u32(Kt + (kk >> 2) * 16384 + (kk & 3) * 32);
+                    mma_bf16(tmem + L::T_G, sdesc_sw128(a, 16, 1024), sdesc_sw128(a, 16, 1024), id, kk > 0);
+                }
+                mma_commit(&bars[B::gram]);
+            }
+            // ---- decays Gam[r][i] (lower triangle; zero across a reset) into the T scratch ----
+            {
+                const int r = t & 63, c0 = (t >> 6) * 32;
+                const float Gr = Gs[r];
+                const int lr = last[r];
+                float *gm = TFm + r * LDF + c0;
+#pragma unroll
+                for (int j4 = 0; j4 < 32; j4 += 4) {
+                    const float4 g4 = *reinterpret_cast<const float4 *>(&Gs[c0 + j4]);
+                    const float gi[4] = {g4.x, g4.y, g4.z, g4.w};
+                    float v[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int i = c0 + j4 + e;
+                        const float ex = ex2_approx(Gr - gi[e]);
+                        v[e] = (i <= r && lr <= i) ? ex : 0.f;
+                    }
+                    *reinterpret_cast<float4 *>(gm + j4) = make_float4(v[0], v[1], v[2], v[3]);
+                }
+            }
+            ctl.wait(B::gram, c & 1);
             tc_fence_after();
-            constexpr uint32_t id = idesc_bf16(128, 64, 0, 0);
+            named_bar(2, 128);
+            {
+                // A = diag(b) (Gam o K K^T) (fp32; its diagonal and upper part are never read) and
+                // P = Gam o Q K^T (bf16)
+                float x[64];
+                tmem_ld32(tl + L::T_G, *reinterpret_cast<float(*)[32]>(&x[0]));
+                tmem_ld32(tl + L::T_G + 32, *reinterpret_cast<float(*)[32]>(&x[32]));
+                tmem_wait_ld();
+                const int r = t & 63;
+                const bool isq = t >= 64;
+                const float sc = isq ? 1.f : bet[r];
 #pragma unroll
-            for (int kk = 0; kk < DK / 16; ++kk) {
-                const uint32_t a = smem_u32(sm + L::KQ + (kk >> 2) * 16384 + (kk & 3) * 32);
-                mma_bf16(tmem + C_G, sdesc_sw128(a, 16, 1024), sdesc_sw128(a, 16, 1024), id, kk > 0);
-            }
-            mma_commit(&bars[1]);
-        }
-        wait_mma();
-        {
-            float x[64];
-            tmem_ld32(tl + C_G, *reinterpret_cast<float(*)[32]>(&x[0]));
-            tmem_ld32(tl + C_G + 32, *reinterpret_cast<float(*)[32]>(&x[32]));
-            tmem_wait_ld();
-            const int r = tid & 63;
-            const bool isq = tid >= 64;
-            const float Gr = Gs[r], br = bet[r];
-            const int lr = last[r];
+                for (int i4 = 0; i4 < CH; i4 += 4) {
+                    const float4 gm = *reinterpret_cast<const float4 *>(&TFm[r * LDF + i4]);
+                    x[i4] *= gm.x * sc;
+                    x[i4 + 1] *= gm.y * sc;
+                    x[i4 + 2] *= gm.z * sc;
+                    x[i4 + 3] *= gm.w * sc;
+                }
+                if (isq) {
+                    st_row_bf16_sw128(sm + L::PM + st * 8192, r, x);
+                } else {
 #pragma unroll
-            for (int i = 0; i < CH; ++i) {
-                const float gm = (i <= r && lr <= i) ? expf(Gr - Gs[i]) : 0.f;
-                x[i] = isq ? gm * x[i] : (i < r ? br * gm * x[i] : 0.f);
+                    for (int i = 0; i < CH; i += 4)
+                        *reinterpret_cast<float4 *>(&AF[r * LDF + i]) = make_float4(x[i], x[i + 1], x[i + 2], x[i + 3]);
+                }
+                // gam-scaled Q in place (Q is no longer read by the Gram MMA)
+                const float gr = gam[r];
+                if (DK == 128) {
+                    scale_row_bf16(Kt + (t >> 6) * 16384 + 8192, r, gr, 0, 8);
+                } else {
+                    scale_row_bf16(Kt + 8192, r, gr, (t >> 6) * 4, (t >> 6) * 4 + 4);
+                }
             }
-            if (isq) {
-                st_row_bf16_sw128(sm + L::PM, r, x);
-            } else {
+            tc_fence_before();
+            named_bar(2, 128);
+            // ---- T = (I + A)^{-1}, written with the bf16 rows of T diag(b), T diag(b gam) ----
+            solve_unit_lower(AF, TOut{TFm, sm + L::TB, sm + L::TG, bet, gam}, XSm, t, 2);
+            fence_proxy_async_smem();
+            named_bar(2, 128);
+            // ---- U~^T = V^T (T diag b)^T ;  W^T = K^T (T diag(b gam))^T ----
+            ctl.wait(B::v_full, c & 1);
+            if (t == kIntraIssuer && !ctl.aborted()) {
+                tc_fence_after();
+                constexpr uint32_t idU = idesc_bf16(DV, 64, 1, 0);
+                constexpr uint32_t idW = idesc_bf16(DK, 64, 1, 0);
 #pragma unroll
-                for (int i = 0; i < CH; ++i) Af[r * LDF + i] = x[i];
-            }
-        }
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncthreads();
-
-        // ---- T = (I + A)^{-1}; rows of T diag(b) and T diag(b gam) in bf16 ----
-        solve_unit_lower(Af, Tf, Xf, tid);
-        if (tid < CH) {
-            const int r = tid;
-            float a[64], b[64];
+                for (int kk = 0; kk < 4; ++kk)
+                    mma_bf16(tmem + L::T_U + st * 64, sdesc_sw128(smem_u32(sm + L::V + kk * 2048), 8192, 1024),
+                             sdesc_sw128(smem_u32(sm + L::TB + kk * 32), 16, 1024), idU, kk > 0);
 #pragma unroll
-            for (int i = 0; i < CH; ++i) {
-                const float t = (i <= r) ? Tf[r * LDF + i] : 0.f;
-                a[i] = t * bet[i];
-                b[i] = a[i] * gam[i];
+                for (int kk = 0; kk < 4; ++kk)
+                    mma_bf16(tmem + L::T_W, sdesc_sw128(smem_u32(Kt + kk * 2048), 16384, 1024),
+                             sdesc_sw128(smem_u32(sm + L::TG + kk * 32), 16, 1024), idW, kk > 0);
+                mma_commit(&bars[B::uw]);
             }
-            st_row_bf16_sw128(sm + L::TB, r, a);
-            st_row_bf16_sw128(sm + L::TG, r, b);
-        }
-        fence_proxy_async_smem();
-        __syncthreads();
-
-        // ---- MMA 2: U~^T = V^T (T diag b)^T ;  W^T = K^T (T diag(b gam))^T ----
-        if (tid == 0 && !*abort_flag) {
+            ctl.wait(B::uw, c & 1);
             tc_fence_after();
-            constexpr uint32_t idU = idesc_bf16(DV, 64, 1, 0);
-            constexpr uint32_t idW = idesc_bf16(DK, 64, 1, 0);
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-                mma_bf16(tmem + C_U, sdesc_sw128(smem_u32(sm + L::V + kk * 2048), 8192, 1024),
-                         sdesc_sw128(smem_u32(sm + L::TB + kk * 32), 16, 1024), idU, kk > 0);
+            if (t == kIntraIssuer && c + 1 < nchunks) load_v(c + 1);
+            {
+                // lam-scaled K in place (K is no longer read by the intra MMAs)
+                const int r = t & 63;
+                if (DK == 128) {
+                    scale_row_bf16(Kt + (t >> 6) * 16384, r, lam[r], 0, 8);
+                } else {
+                    scale_row_bf16(Kt, r, lam[r], (t >> 6) * 4, (t >> 6) * 4 + 4);
+                }
+                float x[64];
+                tmem_ld32(tl + L::T_W, *reinterpret_cast<float(*)[32]>(&x[0]));
+                tmem_ld32(tl + L::T_W + 32, *reinterpret_cast<float(*)[32]>(&x[32]));
+                tmem_wait_ld();
+                if (c >= 1) ctl.wait(B::wt_free, (c - 1) & 1);
+                if (crow >= 0) st_row_bf16_sw128(sm + L::WT, crow, x);
             }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            named_bar(2, 128);
+            if (t == 0) ctl.arrive(B::ready + st);
+        }
+    } else {
+        // ======================= chain warpgroup =======================
+        const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);
+        const int j = (DV == 128) ? tid : (lane < 16 ? warp * 16 + lane : -1);  // value column
+        auto store_state_bf16 = [&](int cb, const float (&x)[32]) {
+            if (j < 0) return;
+            unsigned char *stt = sm + L::ST + (cb >> 1) * (DV * 128);
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-                mma_bf16(tmem + C_W, sdesc_sw128(smem_u32(sm + L::KQ + kk * 2048), 16384, 1024),
-                         sdesc_sw128(smem_u32(sm + L::TG + kk * 32), 16, 1024), idW, kk > 0);
+            for (int cc = 0; cc < 4; ++cc) {
+                const int chunk = (cb & 1) * 4 + cc;
+                uint4 w;
+                w.x = pack_bf16x2(x[8 * cc + 0], x[8 * cc + 1]);
+                w.y = pack_bf16x2(x[8 * cc + 2], x[8 * cc + 3]);
+                w.z = pack_bf16x2(x[8 * cc + 4], x[8 * cc + 5]);
+                w.w = pack_bf16x2(x[8 * cc + 6], x[8 * cc + 7]);
+                *reinterpret_cast<uint4 *>(stt + j * 128 + (((chunk ^ (j & 7)) & 7) << 4)) = w;
             }
-            mma_commit(&bars[1]);
-        }
-        wait_mma();
-        {
-            float x[64];
-            tmem_ld32(tl + C_W, *reinterpret_cast<float(*)[32]>(&x[0]));
-            tmem_ld32(tl + C_W + 32, *reinterpret_cast<float(*)[32]>(&x[32]));
-            tmem_wait_ld();
-            if (crow >= 0) st_row_bf16_sw128(sm + L::WT, crow, x);
-        }
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncthreads();
-
-        // ---- MMA 3: U^T = U~^T - S^T W^T ;  O1 = S^T Q^T ----
-        if (tid == 0 && !*abort_flag) {
+        };
+        // Output rows: O (M = 64 tokens, N = DV) sits in lanes 0..15 of each warp, row 16w + lane.
+        auto out_epilogue = [&](int c) {
+            const long tk = tok0 + (long)c * CH;
+            const int n = (int)min((long)CH, len - (long)c * CH);
+            ctl.wait(B::o, c & 1);
             tc_fence_after();
-            constexpr uint32_t idN = idesc_bf16(DV, 64, 0, 1, 1);
-            constexpr uint32_t idQ = idesc_bf16(DV, 64, 0, 0);
+            const int r = 16 * warp + (lane & 15);
+            __nv_bfloat16 *op = out + ((size_t)(tk + r) * H + h) * DV;
+#pragma unroll 1
+            for (int cb = 0; cb < DV / 32; ++cb) {
+                float o[32];
+                tmem_ld32(tl + L::T_O + cb * 32, o);
+                tmem_wait_ld();
+                if (lane < 16 && r < n) {
+                    uint4 *dst = reinterpret_cast<uint4 *>(op + cb * 32);
 #pragma unroll
-            for (int kk = 0; kk < DK / 16; ++kk) {
-                const uint64_t a = sdesc_sw128(smem_u32(sm + L::ST + (kk >> 2) * (DV * 128) + (kk & 3) * 32), 16, 1024);
-                mma_bf16(tmem + C_U, a, sdesc_sw128(smem_u32(sm + L::WT + kk * 2048), 16, 1024), idN, 1);
+                    for (int q = 0; q < 4; ++q) {
+                        uint4 w;
+                        w.x = pack_bf16x2(o[8 * q + 0], o[8 * q + 1]);
+                        w.y = pack_bf16x2(o[8 * q + 2], o[8 * q + 3]);
+                        w.z = pack_bf16x2(o[8 * q + 4], o[8 * q + 5]);
+                        w.w = pack_bf16x2(o[8 * q + 6], o[8 * q + 7]);
+                        dst[q] = w;
+                    }
+                }
             }
-#pragma unroll
-            for (int kk = 0; kk < DK / 16; ++kk) {
-                const uint64_t a = sdesc_sw128(smem_u32(sm + L::ST + (kk >> 2) * (DV * 128) + (kk & 3) * 32), 16, 1024);
-                const uint32_t b = smem_u32(sm + L::KQ + (kk >> 2) * 16384 + 8192 + (kk & 3) * 32);
-                mma_bf16(tmem + C_O1, a, sdesc_sw128(b, 16, 1024), idQ, kk > 0);
-            }
-            mma_commit(&bars[1]);
-        }
-        wait_mma();
-        {
-            float x[64];
-            tmem_ld32(tl + C_U, *reinterpret_cast<float(*)[32]>(&x[0]));
-            tmem_ld32(tl + C_U + 32, *reinterpret_cast<float(*)[32]>(&x[32]));
-            tmem_wait_ld();
-            if (jrow >= 0) {
-                st_row_bf16_sw128(sm + L::UT, jrow, x);
-#pragma unroll
-                for (int r = 0; r < CH; ++r) x[r] *= lam[r];
-                st_row_bf16_sw128(sm + L::UL, jrow, x);
-            }
-        }
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncthreads();
-
-        // ---- MMA 4: O2 = U^T P^T ;  dS^T = (U^T diag lam) K ----
-        if (tid == 0 && !*abort_flag) {
-            tc_fence_after();
-            constexpr uint32_t idP = idesc_bf16(DV, 64, 0, 0);
-            constexpr uint32_t idS = idesc_bf16(DV, DK, 0, 1);
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-                mma_bf16(tmem + C_O2, sdesc_sw128(smem_u32(sm + L::UT + kk * 32), 16, 1024),
-                         sdesc_sw128(smem_u32(sm + L::PM + kk * 32), 16, 1024), idP, kk > 0);
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-                mma_bf16(tmem + C_DS, sdesc_sw128(smem_u32(sm + L::UL + kk * 32), 16, 1024),
-                         sdesc_sw128(smem_u32(sm + L::KQ + kk * 2048), 16384, 1024), idS, kk > 0);
-            mma_commit(&bars[1]);
-        }
-        wait_mma();
-        // ---- state: S^T <- gam_C S^T + dS^T (fp32 in TMEM), bf16 copy for the next chunk ----
-        {
-            const float gC = gam[CH - 1];
+            tc_fence_before();
+            named_bar(1, 128);
+            if (tid == 0) ctl.arrive(B::cdone + (c % NS));
+        };
+        if (nchunks > 0) {
+            // initial state: S^T row j (fp32, pre-scaled by gam_C of chunk 0) and its bf16 copy
+            ctl.wait(B::gready + 0, 0);
+            const float g0 = gates(0)[6 * CH];
 #pragma unroll 1
             for (int cb = 0; cb < DK / 32; ++cb) {
-                float x[32], d[32];
-                tmem_ld32(tl + C_S + cb * 32, x);
-                tmem_ld32(tl + C_DS + cb * 32, d);
-                tmem_wait_ld();
+                float x[32];
 #pragma unroll
-                for (int i = 0; i < 32; ++i) x[i] = fmaf(gC, x[i], d[i]);
-                tmem_st32(tl + C_S + cb * 32, x);
-                if (jrow >= 0) {
-                    unsigned char *st = sm + L::ST + (cb >> 1) * (DV * 128);
+                for (int i = 0; i < 32; ++i)
+                    x[i] = (j >= 0 && S0) ? S0[sbase + (size_t)(cb * 32 + i) * DV + j] : 0.f;
+                store_state_bf16(cb, x);
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        const int chunk = (cb & 1) * 4 + c;
-                        uint4 w;
-                        w.x = pack_bf16x2(x[8 * c + 0], x[8 * c + 1]);
-                        w.y = pack_bf16x2(x[8 * c + 2], x[8 * c + 3]);
-                        w.z = pack_bf16x2(x[8 * c + 4], x[8 * c + 5]);
-                        w.w = pack_bf16x2(x[8 * c + 6], x[8 * c + 7]);
-                        *reinterpret_cast<uint4 *>(st + jrow * 128 + (((chunk ^ (jrow & 7)) & 7) << 4)) = w;
-                    }
-                }
+                for (int i = 0; i < 32; ++i) x[i] *= g0;
+                tmem_st32(tl + L::T_S + cb * 32, x);
             }
             tmem_wait_st();
+            fence_proxy_async_smem();
+            tc_fence_before();
+            named_bar(1, 128);
         }
-        // ---- outputs: o[r][j] = gam_r O1[j][r] + O2[j][r] ----
-        {
-            float o1[32], o2[32];
-#pragma unroll 1
-            for (int hb = 0; hb < 2; ++hb) {
-                tmem_ld32(tl + C_O1 + hb * 32, o1);
-                tmem_ld32(tl + C_O2 + hb * 32, o2);
-                tmem_wait_ld();
-                if (jrow >= 0) {
+        for (int c = 0; c < nchunks; ++c) {
+            const int st = c % NS;
+            const uint32_t tO = tmem + L::T_O;
+            unsigned char *Kt = sm + L::KQ + st * L::KQ_STAGE;
+            ctl.wait(B::ready + st, (c / NS) & 1);
+            if (tid == 0 && !ctl.aborted()) {
+                tc_fence_after();
+                constexpr uint32_t idN = idesc_bf16(DV, 64, 0, 1, 1);
+                constexpr uint32_t idQ = idesc_bf16(64, DV, 0, 0);
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        const int r = hb * 32 + i;
-                        if (r < n)
-                            out[((size_t)(tk + r) * H + h) * DV + jrow] =
-                                __float2bfloat16_rn(fmaf(gam[r], o1[i], o2[i]));
-                    }
+                for (int kk = 0; kk < DK / 16; ++kk) {
+                    const uint64_t a = sdesc_sw128(smem_u32(sm + L::ST + (kk >> 2) * (DV * 128) + (kk & 3) * 32), 16, 1024);
+                    mma_bf16(tmem + L::T_U + st * 64, a, sdesc_sw128(smem_u32(sm + L::WT + kk * 2048), 16, 1024), idN, 1);
+                }
+                mma_commit(&bars[B::u]);
+#pragma unroll
+                for (int kk = 0; kk < DK / 16; ++kk) {
+                    // O = (gam Q) S: A = gam-scaled Q tile (K-major), B = S^T rows (K-major)
+                    const uint32_t a = smem_u32(Kt + (kk >> 2) * 16384 + 8192 + (kk & 3) * 32);
+                    const uint64_t b = sdesc_sw128(smem_u32(sm + L::ST + (kk >> 2) * (DV * 128) + (kk & 3) * 32), 16, 1024);
+                    mma_bf16(tO, sdesc_sw128(a, 16, 1024), b, idQ, kk > 0);
                 }
             }
-        }
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncthreads();
-    }
-
-    // ---- final state ----
-    if (S_final) {
-#pragma unroll 1
-        for (int cb = 0; cb < DK / 32; ++cb) {
-            float x[32];
-            tmem_ld32(tl + C_S + cb * 32, x);
-            tmem_wait_ld();
-            if (jrow >= 0) {
+            ctl.wait(B::u, c & 1);
+            tc_fence_after();
+            if (tid == 0) ctl.arrive(B::wt_free);
+            {
+                float x[64];
+                tmem_ld32(tl + L::T_U + st * 64, *reinterpret_cast<float(*)[32]>(&x[0]));
+                tmem_ld32(tl + L::T_U + st * 64 + 32, *reinterpret_cast<float(*)[32]>(&x[32]));
+                tmem_wait_ld();
+                if (j >= 0) st_row_bf16_sw128(sm + L::UT, j, x);
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            named_bar(1, 128);
+            if (tid == 0 && !ctl.aborted()) {
+                tc_fence_after();
+                constexpr uint32_t idS = idesc_bf16(DV, DK, 0, 1);
+                constexpr uint32_t idP = idesc_bf16(64, DV, 0, 0);
 #pragma unroll
-                for (int i = 0; i < 32; ++i) S_final[sbase + (size_t)(cb * 32 + i) * DV + jrow] = x[i];
+                for (int kk = 0; kk < 4; ++kk)
+                    mma_bf16(tmem + L::T_S, sdesc_sw128(smem_u32(sm + L::UT + kk * 32), 16, 1024),
+                             sdesc_sw128(smem_u32(Kt + kk * 2048), 16384, 1024), idS, 1);
+                mma_commit(&bars[B::s]);
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)  // O += P U: A = P rows (K-major), B = U^T rows (K-major)
+                    mma_bf16(tO, sdesc_sw128(smem_u32(sm + L::PM + st * 8192 + kk * 32), 16, 1024),
+                             sdesc_sw128(smem_u32(sm + L::UT + kk * 32), 16, 1024), idP, 1);
+                mma_commit(&bars[B::o]);
+            }
+            ctl.wait(B::s, c & 1);
+            tc_fence_after();
+            if (warp == 0 && c + NS < nchunks) load_kq(c + NS);
+            {
+                // S_{c+1} = gam_C(c) S_c + increment is in TMEM; keep a bf16 copy and pre-scale the
+                // fp32 state by gam_C of the next chunk
+                const bool more = c + 1 < nchunks;
+                float gn = 1.f;
+                if (more) {
+                    ctl.wait(B::gready + (c + 1) % NS, ((c + 1) / NS) & 1);
+                    gn = gates((c + 1) % NS)[6 * CH];
+                }
+#pragma unroll 1
+                for (int cb = 0; cb < DK / 32; ++cb) {
+                    float x[32];
+                    tmem_ld32(tl + L::T_S + cb * 32, x);
+                    tmem_wait_ld();
+                    store_state_bf16(cb, x);
+                    if (more) {
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) x[i] *= gn;
+                        tmem_st32(tl + L::T_S + cb * 32, x);
+                    }
+                }
+                tmem_wait_st();
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            named_bar(1, 128);
+            out_epilogue(c);
+        }
+        // final state
+        if (S_final) {
+            if (nchunks > 0) {
+#pragma unroll 1
+                for (int cb = 0; cb < DK / 32; ++cb) {
+                    float x[32];
+                    tmem_ld32(tl + L::T_S + cb * 32, x);
+                    tmem_wait_ld();
+                    if (j >= 0) {
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) S_final[sbase + (size_t)(cb * 32 + i) * DV + j] = x[i];
+                    }
+                }
+            } else if (j >= 0) {
+                for (int c2 = 0; c2 < DK; ++c2)
+                    S_final[sbase + (size_t)c2 * DV + j] = S0 ? S0[sbase + (size_t)c2 * DV + j] : 0.f;
             }
         }
     }
@@ -544,17 +792,17 @@ bool make_map(CUtensorMap *m, const void *base, long tokens, int H, int d)
 template <int DK, int DV>
 cudaError_t launch_tc(const ChunkArgs &a, cudaStream_t st)
 {
-    using L = TcLayout<DK, DV>;
+    using L = TcCfg<DK, DV>;
     const long tokens = a.cu_seqlens ? (long)a.T : (long)a.B * a.T;
     CUtensorMap mq, mk, mv;
-    if (tokens <= 0) return cudaSuccess;
-    if (!make_map(&mq, a.q, tokens, a.H, DK) || !make_map(&mk, a.k, tokens, a.H, DK) ||
-        !make_map(&mv, a.v, tokens, a.H, DV)) {
+    // a zero-token varlen call still launches so that S_final = S0 is written
+    const long map_tokens = tokens > 0 ? tokens : 1;
+    if (!make_map(&mq, a.q, map_tokens, a.H, DK) || !make_map(&mk, a.k, map_tokens, a.H, DK) ||
+        !make_map(&mv, a.v, map_tokens, a.H, DV)) {
         set_error("cuTensorMapEncodeTiled failed");
         return cudaErrorInvalidValue;
     }
-    // at least 116 KB so that two CTAs (each holding 512 TMEM columns) never share an SM
-    const int smem = (L::TOTAL + 1024) > 118784 ? (L::TOTAL + 1024) : 118784;
+    const int smem = L::TOTAL + 1024;
     auto kern = chunk_tc_kernel<DK, DV>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;

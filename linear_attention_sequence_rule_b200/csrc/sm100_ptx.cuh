@@ -83,6 +83,22 @@ __device__ __forceinline__ void prefetch_tmap(const CUtensorMap *map)
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
 
+// ---- cp.async (4-byte elements, zero-filled when src_bytes == 0) with mbarrier completion -----
+
+__device__ __forceinline__ void cp_async_4(void *smem_dst, const void *gsrc, uint32_t src_bytes)
+{
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(smem_u32(smem_dst)), "l"(gsrc),
+                 "r"(src_bytes)
+                 : "memory");
+}
+
+// The mbarrier receives one arrival from this thread once all its earlier cp.async copies have
+// landed (the arrival is pre-counted in the barrier's expected count).
+__device__ __forceinline__ void cp_async_mbar_arrive(uint64_t *bar)
+{
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
 // ---- proxy / tcgen05 fences ------------------------------------------------------------------
 
 // Make this thread's generic-proxy shared-memory writes visible to the async proxy (MMA, TMA).
@@ -199,6 +215,14 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32])
 
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// 2^x by the special-function unit (ex2.approx, flush-to-zero): relative error below 2^-22.
+__device__ __forceinline__ float ex2_approx(float x)
+{
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
 
 // ---- bf16 packing ----------------------------------------------------------------------------
 

@@ -22,7 +22,7 @@ def run_gpu_chunk(inp, S_final=True, **kw):
     d = to_dev(inp)
     out, Sf = gdn.chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], S0=d["S0"],
                             cu_seqlens=d["cu_seqlens"], output_final_state=S_final, **kw)
-    torch.cuda.synchronize()
+    gdn.device_status()  # synchronises; raises if a device-side wait ran out
     return out, Sf
 
 
