@@ -161,13 +161,26 @@ def barrier(world):
         dist.barrier()
 
 
-def max_over_ranks(x, world):
+def max_over_ranks(x, world, device=None):
+    """Max of a per-rank number over all ranks (the job's time is its slowest rank's)."""
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    if device is None:
+        device = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def rank_seed(base_seed, rank):
+    """Every rank runs its own independent batch (weak scaling), drawn with its own seed."""
+    return int(base_seed) + 7919 * int(rank)
+
+
+def aggregate_tokens_per_s(tokens_per_rank, world, ms_max):
+    """Whole-job throughput: all ranks' tokens over the slowest rank's time."""
+    return tokens_per_rank * world / (ms_max * 1e-3)
 
 
 # ---- our arm -------------------------------------------------------------------------------
@@ -315,7 +328,7 @@ def run_ours(args, world, rank, local):
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device="cuda")
     name = "hybrid_lm"
     cfg = workloads.CONFIGS[name]
-    inp = workloads.config_inputs(name, seed=cfg["seed"] + rank)
+    inp = workloads.config_inputs(name, seed=rank_seed(cfg["seed"], rank))
     d = to_dev(inp)
 
     barrier(world)
@@ -328,7 +341,7 @@ def run_ours(args, world, rank, local):
     ms = max_over_ranks(ms_local, world)
     main = chunk_numbers(name, d, times, peaks)
     tokens_all = main["tokens"] * world
-    value = tokens_all / (ms * 1e-3)
+    value = aggregate_tokens_per_s(main["tokens"], world, ms)
 
     e2e_ms, h2d, d2h = e2e_chunk(gdn, inp, max(3, args.steps // 10), 2, stream)
     e2e_ms = max_over_ranks(e2e_ms, world)

@@ -15,8 +15,8 @@
 //   producer warp (warp 8): TMA loads of the K, Q tiles (NS-stage ring) and the V tile.
 //   intra warpgroup (warps 4-7): everything of chunk c+1 that does not depend on the state --
 //       gate sums (warp-shuffle segmented scan), Gram matrices [K;Q] K^T (tcgen05, M=128),
-//       A and P with the decays, T = (I+A)^{-1} (16x16 diagonal blocks by substitution on CUDA
-//       cores, the 16->32->64 merges with mma.sync TF32), T diag(b) and T diag(b gam) in bf16,
+//       A and P with the decays, T = (I+A)^{-1} (16x16 diagonal blocks by recursive doubling on
+//       CUDA cores, the 16->32->64 merges with mma.sync TF32), T diag(b) and T diag(b gam) in bf16,
 //       U~^T and W^T (tcgen05), then gam-scaled Q and lam-scaled K in place.
 //   chain warpgroup (warps 0-3): the state-dependent part of chunk c, thread j = value column j:
 //       U^T   = U~^T - S^T W^T           (accumulated onto U~^T, A operand negated)
@@ -169,8 +169,8 @@ struct TOut {
 // T = (I + A)^{-1} for strictly lower triangular A (64 x 64 fp32, row stride LDF; only entries
 // below the diagonal are read), executed by the 128 threads of the intra warpgroup (t = 0..127).
 // Warp w inverts the 16 x 16 diagonal block w by recursive doubling (2 -> 4 -> 8 -> 16,
-// warp-synchronous, CUDA cores); the 16 -> 32 and 32 -> 64 merges T_ba = -T_bb (A_ba T_aa) run on
-// mma.sync TF32 (T is rounded to bf16 afterwards, so TF32 products stay below that rounding).
+// warp-synchronous, CUDA cores); the 16 -> 32 and 32 -> 64 merges T_ba = -T_bb (A_ba T_aa) run
+// on mma.sync TF32 (T is rounded to bf16 afterwards, so TF32 products stay below that rounding).
 // Every entry of the lower triangle is written exactly once, through `out`; entries above the
 // diagonal are never written (the caller keeps them zero in the bf16 copies).
 __device__ void solve_unit_lower(const float *A, const TOut &out, float *XS, int t, int bar_id)
@@ -296,20 +296,19 @@ __device__ void solve_unit_lower(const float *A, const TOut &out, float *XS, int
     }
 }
 
-// Scale row r (64 bf16 = 128 swizzled bytes, 8 chunks of 16 B) of a tile by s, chunks [c0, c1).
+// Scale row r (64 bf16 = 128 swizzled bytes, 8 chunks of 16 B) of a tile by s: the caller owns
+// chunks [c0, c1) counted from position row % 8, so that the threads of a warp (consecutive rows)
+// touch 8 different bank groups at every step.  Packed bf16x2 multiplies (s rounded to bf16).
 __device__ __forceinline__ void scale_row_bf16(unsigned char *tile, int row, float s, int c0, int c1)
 {
+    const __nv_bfloat162 s2 = __float2bfloat162_rn(s);
 #pragma unroll
     for (int c = c0; c < c1; ++c) {
-        uint4 *p = reinterpret_cast<uint4 *>(tile + row * 128 + c * 16);
+        uint4 *p = reinterpret_cast<uint4 *>(tile + row * 128 + (((c + row) & 7) << 4));
         uint4 w = *p;
-        uint32_t *u = reinterpret_cast<uint32_t *>(&w);
+        __nv_bfloat162 *h = reinterpret_cast<__nv_bfloat162 *>(&w);
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            __nv_bfloat162 h = *reinterpret_cast<__nv_bfloat162 *>(&u[e]);
-            float2 f = __bfloat1622float2(h);
-            u[e] = pack_bf16x2(f.x * s, f.y * s);
-        }
+        for (int e = 0; e < 4; ++e) h[e] = __hmul2(h[e], s2);
         *p = w;
     }
 }
@@ -775,6 +774,8 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn()
 }
 
 // 3-D view [tokens][H][d] of a bf16 tensor; box = 64 features x 1 head x 64 tokens, 128B swizzle.
+// A box row is 128 bytes of one head; L2 promotion is kept at 128 bytes so that a fetch does not
+// pull in the neighbouring head's row.
 bool make_map(CUtensorMap *m, const void *base, long tokens, int H, int d)
 {
     auto enc = get_encode_fn();
@@ -785,7 +786,7 @@ bool make_map(CUtensorMap *m, const void *base, long tokens, int H, int d)
     cuuint32_t es[3] = {1, 1, 1};
     CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, es,
                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
 
