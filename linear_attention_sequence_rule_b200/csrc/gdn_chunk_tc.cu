@@ -15,8 +15,8 @@
 //   producer warp (warp 8): TMA loads of the K, Q tiles (NS-stage ring) and the V tile.
 //   intra warpgroup (warps 4-7): everything of chunk c+1 that does not depend on the state --
 //       gate sums (warp-shuffle segmented scan), Gram matrices [K;Q] K^T (tcgen05, M=128),
-//       A and P with the decays, T = (I+A)^{-1} (16x16 diagonal blocks by recursive doubling on
-//       CUDA cores, the 16->32->64 merges with mma.sync TF32), T diag(b) and T diag(b gam) in bf16,
+//       A and P with the decays, T = (I+A)^{-1} (8x8 diagonal blocks by substitution on CUDA
+//       cores, the 8->16->32->64 merges on CUDA cores / mma.sync TF32), T diag(b) and T diag(b gam) in bf16,
 //       U~^T and W^T (tcgen05), then gam-scaled Q and lam-scaled K in place.
 //   chain warpgroup (warps 0-3): the state-dependent part of chunk c, thread j = value column j:
 //       U^T   = U~^T - S^T W^T           (accumulated onto U~^T, A operand negated)
@@ -127,13 +127,6 @@ struct Ctl {
 
 __device__ __forceinline__ void named_bar(int id, int n) { asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory"); }
 
-__device__ __forceinline__ uint32_t f2tf32(float x)
-{
-    uint32_t r;
-    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
-    return r;
-}
-
 __device__ __forceinline__ void mma_tf32(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                          uint32_t b0, uint32_t b1)
 {
@@ -144,8 +137,8 @@ __device__ __forceinline__ void mma_tf32(float (&d)[4], uint32_t a0, uint32_t a1
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-// Final value v of T[r][c]: keep it in fp32 for later merges and write the bf16 entries of
-// T diag(b) and T diag(b gam) (128B-swizzled rows, the B operands of the WY products).
+// Final value v of T[r][c]: written as the bf16 entries of T diag(b) and T diag(b gam)
+// (128B-swizzled rows, the B operands of the WY products) and, where later merges read it, in fp32.
 struct TOut {
     float *Tm;
     unsigned char *TB, *TG;
@@ -157,22 +150,28 @@ struct TOut {
         *reinterpret_cast<__nv_bfloat16 *>(TB + sw128_off(r, c)) = __float2bfloat16_rn(b);
         *reinterpret_cast<__nv_bfloat16 *>(TG + sw128_off(r, c)) = __float2bfloat16_rn(b * gam[c]);
     }
-    __device__ __forceinline__ void put2(int r, int c, float v0, float v1) const  // c even
+    // c even; (b0, b1, g0, g1) = bet/gam of columns c, c+1; keep: also store the fp32 values
+    __device__ __forceinline__ void put2(int r, int c, float v0, float v1, float b0, float b1, float g0, float g1,
+                                         bool keep) const
     {
-        *reinterpret_cast<float2 *>(&Tm[r * LDF + c]) = make_float2(v0, v1);
-        const float b0 = v0 * bet[c], b1 = v1 * bet[c + 1];
-        *reinterpret_cast<uint32_t *>(TB + sw128_off(r, c)) = pack_bf16x2(b0, b1);
-        *reinterpret_cast<uint32_t *>(TG + sw128_off(r, c)) = pack_bf16x2(b0 * gam[c], b1 * gam[c + 1]);
+        if (keep) *reinterpret_cast<float2 *>(&Tm[r * LDF + c]) = make_float2(v0, v1);
+        const float x0 = v0 * b0, x1 = v1 * b1;
+        *reinterpret_cast<uint32_t *>(TB + sw128_off(r, c)) = pack_bf16x2(x0, x1);
+        *reinterpret_cast<uint32_t *>(TG + sw128_off(r, c)) = pack_bf16x2(x0 * g0, x1 * g1);
     }
 };
 
+// fp32 bits used as a TF32 operand: the tensor core ignores the low 13 mantissa bits.
+__device__ __forceinline__ uint32_t tf(float x) { return __float_as_uint(x); }
+
 // T = (I + A)^{-1} for strictly lower triangular A (64 x 64 fp32, row stride LDF; only entries
 // below the diagonal are read), executed by the 128 threads of the intra warpgroup (t = 0..127).
-// Warp w inverts the 16 x 16 diagonal block w by recursive doubling (2 -> 4 -> 8 -> 16,
-// warp-synchronous, CUDA cores); the 16 -> 32 and 32 -> 64 merges T_ba = -T_bb (A_ba T_aa) run
-// on mma.sync TF32 (T is rounded to bf16 afterwards, so TF32 products stay below that rounding).
-// Every entry of the lower triangle is written exactly once, through `out`; entries above the
-// diagonal are never written (the caller keeps them zero in the bf16 copies).
+// Warp w owns the 16 x 16 diagonal block w: its two 8 x 8 diagonal sub-blocks are inverted by
+// column-parallel forward substitution (lane = column, running sums, 7 dependent steps), then one
+// doubling step T_ba = -T_bb (A_ba T_aa) joins them.  The 16 -> 32 and 32 -> 64 merges run the
+// same step on mma.sync TF32 (T is rounded to bf16 afterwards, so TF32 products stay below that
+// rounding).  Every entry of the lower triangle is written exactly once, through `out`; entries
+// above the diagonal are never written (the caller keeps them zero in the bf16 copies).
 __device__ void solve_unit_lower(const float *A, const TOut &out, float *XS, int t, int bar_id)
 {
     float *Tm = out.Tm;
@@ -180,39 +179,40 @@ __device__ void solve_unit_lower(const float *A, const TOut &out, float *XS, int
     float *xs = XS + w * 256;
     {
         const int o = 16 * w;
-        if (lane < 16) out.put(o + lane, o + lane, 1.f);
+        if (lane < 16) {
+            const int sb = o + 8 * (lane >> 3), c = lane & 7;
+            float p[8], x[8];
+#pragma unroll
+            for (int r = 0; r < 8; ++r) p[r] = 0.f;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                x[i] = (i < c) ? 0.f : (i == c ? 1.f : -p[i]);
+#pragma unroll
+                for (int r = i + 1; r < 8; ++r) p[r] = fmaf(A[(sb + r) * LDF + sb + i], x[i], p[r]);
+            }
+#pragma unroll
+            for (int r = 0; r < 8; ++r)
+                if (r >= c) out.put(sb + r, sb + c, x[r]);
+        }
         __syncwarp();
 #pragma unroll
-        for (int s = 1; s <= 8; s <<= 1) {
-            const int nout = 8 * s;  // (16 / 2s) pairs x s^2 outputs
+        for (int q0 = 0; q0 < 64; q0 += 32) {
+            const int q = q0 + lane, i = q >> 3, j = q & 7;
+            float acc = 0.f;
 #pragma unroll
-            for (int q0 = 0; q0 < nout; q0 += 32) {
-                const int q = q0 + lane;
-                if (q < nout) {
-                    const int p = q / (s * s), rem = q % (s * s), i = rem / s, jj = rem % s;
-                    const int a0 = o + 2 * p * s, b0 = a0 + s;
-                    float acc = 0.f;
+            for (int k = 0; k < 8; ++k)
+                if (k >= j) acc = fmaf(A[(o + 8 + i) * LDF + o + k], Tm[(o + k) * LDF + o + j], acc);
+            xs[i * 8 + j] = acc;
+        }
+        __syncwarp();
 #pragma unroll
-                    for (int k = 0; k < s; ++k)
-                        if (k >= jj) acc = fmaf(A[(b0 + i) * LDF + a0 + k], Tm[(a0 + k) * LDF + a0 + jj], acc);
-                    xs[i * 16 + p * s + jj] = acc;
-                }
-            }
-            __syncwarp();
+        for (int q0 = 0; q0 < 64; q0 += 32) {
+            const int q = q0 + lane, i = q >> 3, j = q & 7;
+            float acc = xs[i * 8 + j];
 #pragma unroll
-            for (int q0 = 0; q0 < nout; q0 += 32) {
-                const int q = q0 + lane;
-                if (q < nout) {
-                    const int p = q / (s * s), rem = q % (s * s), i = rem / s, jj = rem % s;
-                    const int a0 = o + 2 * p * s, b0 = a0 + s;
-                    float acc = xs[i * 16 + p * s + jj];  // diagonal term (T_bb[i][i] = 1)
-#pragma unroll
-                    for (int k = 0; k < s; ++k)
-                        if (k < i) acc = fmaf(Tm[(b0 + i) * LDF + b0 + k], xs[k * 16 + p * s + jj], acc);
-                    out.put(b0 + i, a0 + jj, -acc);
-                }
-            }
-            __syncwarp();
+            for (int k = 0; k < 8; ++k)
+                if (k < i) acc = fmaf(Tm[(o + 8 + i) * LDF + o + 8 + k], xs[k * 8 + j], acc);
+            out.put(o + 8 + i, o + j, -acc);
         }
     }
     named_bar(bar_id, 128);
@@ -224,9 +224,9 @@ __device__ void solve_unit_lower(const float *A, const TOut &out, float *XS, int
         for (int kk = 0; kk < 2; ++kk) {
             if (kk < nt) continue;
             const int k0 = oa + 8 * kk + tq, k1 = k0 + 4;
-            mma_tf32(d, f2tf32(A[(ob + g) * LDF + k0]), f2tf32(A[(ob + g + 8) * LDF + k0]),
-                     f2tf32(A[(ob + g) * LDF + k1]), f2tf32(A[(ob + g + 8) * LDF + k1]),
-                     f2tf32(k0 >= n ? Tm[k0 * LDF + n] : 0.f), f2tf32(k1 >= n ? Tm[k1 * LDF + n] : 0.f));
+            mma_tf32(d, tf(A[(ob + g) * LDF + k0]), tf(A[(ob + g + 8) * LDF + k0]),
+                     tf(A[(ob + g) * LDF + k1]), tf(A[(ob + g + 8) * LDF + k1]),
+                     tf(k0 >= n ? Tm[k0 * LDF + n] : 0.f), tf(k1 >= n ? Tm[k1 * LDF + n] : 0.f));
         }
         xs[g * 8 + 2 * tq] = d[0];
         xs[g * 8 + 2 * tq + 1] = d[1];
@@ -237,19 +237,19 @@ __device__ void solve_unit_lower(const float *A, const TOut &out, float *XS, int
 #pragma unroll
         for (int kk = 0; kk < 2; ++kk) {
             const int k0 = 8 * kk + tq, k1 = k0 + 4;
-            mma_tf32(e, f2tf32(k0 <= g ? Tm[(ob + g) * LDF + ob + k0] : 0.f),
-                     f2tf32(k0 <= g + 8 ? Tm[(ob + g + 8) * LDF + ob + k0] : 0.f),
-                     f2tf32(k1 <= g ? Tm[(ob + g) * LDF + ob + k1] : 0.f),
-                     f2tf32(k1 <= g + 8 ? Tm[(ob + g + 8) * LDF + ob + k1] : 0.f),
-                     f2tf32(xs[k0 * 8 + g]), f2tf32(xs[k1 * 8 + g]));
+            mma_tf32(e, tf(k0 <= g ? Tm[(ob + g) * LDF + ob + k0] : 0.f),
+                     tf(k0 <= g + 8 ? Tm[(ob + g + 8) * LDF + ob + k0] : 0.f),
+                     tf(k1 <= g ? Tm[(ob + g) * LDF + ob + k1] : 0.f),
+                     tf(k1 <= g + 8 ? Tm[(ob + g + 8) * LDF + ob + k1] : 0.f),
+                     tf(xs[k0 * 8 + g]), tf(xs[k1 * 8 + g]));
         }
         const int c0 = oa + 8 * nt + 2 * tq;
-        out.put2(ob + g, c0, -e[0], -e[1]);
-        out.put2(ob + g + 8, c0, -e[2], -e[3]);
+        const float b0 = out.bet[c0], b1 = out.bet[c0 + 1], g0 = out.gam[c0], g1 = out.gam[c0 + 1];
+        out.put2(ob + g, c0, -e[0], -e[1], b0, b1, g0, g1, true);
+        out.put2(ob + g + 8, c0, -e[2], -e[3], b0, b1, g0, g1, true);
     }
     named_bar(bar_id, 128);
-    // ---- 32 -> 64: a = [0,32), b = [32,64); warp w takes output column tile wt = 3 - w (columns
-    //      8wt..8wt+7; tile 3 has the fewest products and goes to warp 0) ----
+    // ---- 32 -> 64: warp w takes output column tile wt = 3 - w ----
     {
         const int wt = 3 - w;
         const int n = 8 * wt + g;
@@ -258,13 +258,13 @@ __device__ void solve_unit_lower(const float *A, const TOut &out, float *XS, int
         for (int kk = 0; kk < 4; ++kk) {
             if (kk < wt) continue;
             const int k0 = 8 * kk + tq, k1 = k0 + 4;
-            const uint32_t b0 = f2tf32(k0 >= n ? Tm[k0 * LDF + n] : 0.f);
-            const uint32_t b1 = f2tf32(k1 >= n ? Tm[k1 * LDF + n] : 0.f);
+            const uint32_t b0 = tf(k0 >= n ? Tm[k0 * LDF + n] : 0.f);
+            const uint32_t b1 = tf(k1 >= n ? Tm[k1 * LDF + n] : 0.f);
 #pragma unroll
             for (int mt = 0; mt < 2; ++mt) {
                 const int r = 32 + 16 * mt + g;
-                mma_tf32(d[mt], f2tf32(A[r * LDF + k0]), f2tf32(A[(r + 8) * LDF + k0]),
-                         f2tf32(A[r * LDF + k1]), f2tf32(A[(r + 8) * LDF + k1]), b0, b1);
+                mma_tf32(d[mt], tf(A[r * LDF + k0]), tf(A[(r + 8) * LDF + k0]), tf(A[r * LDF + k1]),
+                         tf(A[(r + 8) * LDF + k1]), b0, b1);
             }
         }
 #pragma unroll
@@ -275,6 +275,8 @@ __device__ void solve_unit_lower(const float *A, const TOut &out, float *XS, int
             xs[(16 * mt + g + 8) * 8 + 2 * tq + 1] = d[mt][3];
         }
         __syncwarp();
+        const int c0 = 8 * wt + 2 * tq;
+        const float bb0 = out.bet[c0], bb1 = out.bet[c0 + 1], gg0 = out.gam[c0], gg1 = out.gam[c0 + 1];
 #pragma unroll
         for (int mt = 0; mt < 2; ++mt) {
             float e[4] = {0.f, 0.f, 0.f, 0.f};
@@ -283,15 +285,14 @@ __device__ void solve_unit_lower(const float *A, const TOut &out, float *XS, int
             for (int kk = 0; kk < 4; ++kk) {
                 if (kk > 2 * mt + 1) continue;
                 const int k0 = 8 * kk + tq, k1 = k0 + 4;
-                mma_tf32(e, f2tf32(k0 <= rl ? Tm[(32 + rl) * LDF + 32 + k0] : 0.f),
-                         f2tf32(k0 <= rh ? Tm[(32 + rh) * LDF + 32 + k0] : 0.f),
-                         f2tf32(k1 <= rl ? Tm[(32 + rl) * LDF + 32 + k1] : 0.f),
-                         f2tf32(k1 <= rh ? Tm[(32 + rh) * LDF + 32 + k1] : 0.f),
-                         f2tf32(xs[k0 * 8 + g]), f2tf32(xs[k1 * 8 + g]));
+                mma_tf32(e, tf(k0 <= rl ? Tm[(32 + rl) * LDF + 32 + k0] : 0.f),
+                         tf(k0 <= rh ? Tm[(32 + rh) * LDF + 32 + k0] : 0.f),
+                         tf(k1 <= rl ? Tm[(32 + rl) * LDF + 32 + k1] : 0.f),
+                         tf(k1 <= rh ? Tm[(32 + rh) * LDF + 32 + k1] : 0.f),
+                         tf(xs[k0 * 8 + g]), tf(xs[k1 * 8 + g]));
             }
-            const int c0 = 8 * wt + 2 * tq;
-            out.put2(32 + rl, c0, -e[0], -e[1]);
-            out.put2(32 + rh, c0, -e[2], -e[3]);
+            out.put2(32 + rl, c0, -e[0], -e[1], bb0, bb1, gg0, gg1, false);
+            out.put2(32 + rh, c0, -e[2], -e[3], bb0, bb1, gg0, gg1, false);
         }
     }
 }
