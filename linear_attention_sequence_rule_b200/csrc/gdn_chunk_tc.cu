@@ -11,19 +11,21 @@
 //   O  = diag(gam) Q S + lower_incl(Gam o Q K^T) U
 //   S' = gam_C S + K^T diag(lam) U
 //
-// One CTA per (sequence, head) runs three roles concurrently (288 threads):
-//   producer warp (warp 8): TMA loads of the K, Q tiles (NS-stage ring) and the V tile.
-//   intra warpgroup (warps 4-7): everything of chunk c+1 that does not depend on the state --
-//       gate sums (warp-shuffle segmented scan), Gram matrices [K;Q] K^T (tcgen05, M=128),
-//       A and P with the decays, T = (I+A)^{-1} (8x8 diagonal blocks by substitution on CUDA
-//       cores, the 8->16->32->64 merges on CUDA cores / mma.sync TF32), T diag(b) and T diag(b gam) in bf16,
-//       U~^T and W^T (tcgen05), then gam-scaled Q and lam-scaled K in place.
-//   chain warpgroup (warps 0-3): the state-dependent part of chunk c, thread j = value column j:
+// One CTA of 256 threads per (sequence, head); two warpgroups work concurrently:
+//   intra warpgroup (warps 4-7), one chunk ahead of the state: gate sums (warp-shuffle segmented
+//       scan), Gram matrices [K;Q] K^T (tcgen05, M=128), decays, A = diag(b)(Gam o K K^T) and
+//       P = Gam o Q K^T, then T = (I+A)^{-1} (8x8 diagonal blocks by substitution on CUDA cores,
+//       8->16->32->64 merges on CUDA cores / mma.sync TF32), written as T diag(b) and
+//       T diag(b gam) in bf16.
+//   chain warpgroup (warps 0-3), thread j = value column j, for chunk c:
 //       U^T   = U~^T - S^T W^T           (accumulated onto U~^T, A operand negated)
-//       O^T   = S^T (gam Q)^T + U^T P^T  (one accumulator, double-buffered across chunks)
+//       O     = (gam Q) S + P U          (M = 64 token rows, 16-byte row stores)
 //       S'^T  = gam_C S^T + U^T (lam K)  (accumulated onto the pre-scaled fp32 state in TMEM)
-//   so the chain's critical path per chunk is two MMA round trips.
-// The output epilogue of chunk c overlaps the first chain MMA of chunk c+1.
+//     and, in the shadow of those MMAs, the WY part of chunk c+1: U~^T = V^T (T diag b)^T and
+//     W^T = K^T (T diag(b gam))^T (tcgen05), W^T to shared memory, gam Q and lam K in place.
+//   Loads: K/Q through a TMA stage ring (reissued as soon as a stage's last MMA completes), V
+//   single-buffered, gates by cp.async onto an mbarrier.
+// The state chain's critical path per chunk is two MMA round trips plus their epilogues.
 //
 // Gates: decays are exp of log_alpha sums taken from the last exact reset (log_alpha = -inf)
 // inside the chunk.  Padded rows of a partial chunk get b = 0 and log_alpha = 0, which makes
@@ -52,9 +54,9 @@ constexpr int CH = 64;
 constexpr int kThreads = 256;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 constexpr int LDF = 68;  // fp32 row stride of the 64 x 64 solve matrices
-// Thread roles inside the intra warpgroup: its MMAs and V loads are issued by warp 7 and the gate
-// scan runs on warp 5, away from warp 4, which shares an SM sub-partition with the chain's
-// issuing thread (thread 0).
+// Thread roles inside the intra warpgroup: its Gram MMA is issued by warp 7 and the gate scan runs
+// on warp 5, away from warp 4, which shares an SM sub-partition with the chain's issuing thread
+// (thread 0).
 constexpr int kIntraIssuer = 96;
 constexpr int kScanWarp = 1;
 
@@ -83,9 +85,9 @@ struct TcCfg {
     // TMEM columns
     static constexpr uint32_t T_O = 0;                            // DV: output rows (M = 64 tokens)
     static constexpr uint32_t T_S = DV;                           // DK: fp32 state (transposed)
-    static constexpr uint32_t T_G = DV + DK;                      // 64: Gram, then W^T (intra)
-    static constexpr uint32_t T_W = T_G;
-    static constexpr uint32_t T_U = T_G + 64;                     // NS x 64: U~^T / U^T
+    static constexpr uint32_t T_G = DV + DK;                      // 64: Gram matrices (intra)
+    static constexpr uint32_t T_W = T_G + 64;                     // 64: W^T (chain)
+    static constexpr uint32_t T_U = T_W + 64;                     // NS x 64: U~^T / U^T
     static_assert(T_U + NS * 64 <= 512, "TMEM budget");
     static_assert(TOTAL + 1024 <= 232448, "shared memory budget");
 };
@@ -96,9 +98,9 @@ template <int NS> struct Bars {
     static constexpr int v_full = NS;
     static constexpr int v_empty = NS + 1;
     static constexpr int cdone = NS + 2;         // [NS]
-    static constexpr int ready = 2 * NS + 2;     // [NS]
+    static constexpr int tready = 2 * NS + 2;    // [NS] intra -> chain: P, T diag(b), T diag(b gam) ready
     static constexpr int gready = 3 * NS + 2;    // [NS]
-    static constexpr int wt_free = 4 * NS + 2;
+    static constexpr int tfree = 4 * NS + 2;     // chain -> intra: the WY MMAs have read T diag(b..)
     static constexpr int gram = 4 * NS + 3;
     static constexpr int uw = 4 * NS + 4;
     static constexpr int u = 4 * NS + 5;
@@ -324,6 +326,10 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
     using L = TcCfg<DK, DV>;
     constexpr int NS = L::NS;
     using B = Bars<NS>;
+    // dk = 64: the chain warpgroup does the WY part of the next chunk in the shadow of its MMAs.
+    // dk = 128: the chain's own epilogues are twice as large, so the intra warpgroup does it.
+    constexpr bool kChainWY = DK == 64;
+    constexpr bool kIntraScalesQ = !kChainWY;
     extern __shared__ unsigned char smem_raw[];
     unsigned char *sm = reinterpret_cast<unsigned char *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -399,13 +405,61 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
         }
         for (int c = 0; c < min(nchunks, NS); ++c) load_kq(c);
     }
-    if (tid == 128 + kIntraIssuer && nchunks > 0) load_v(0);
+    if (tid == 0 && nchunks > 0) load_v(0);
+        // WY MMAs of chunk c2 (thread 0): U~^T = V^T (T diag b)^T into its U slot, W^T = K^T (T diag(b gam))^T.
+    auto issue_wy = [&](int c2) {
+        ctl.wait(B::v_full, c2 & 1);
+        if (ctl.aborted()) return;
+        tc_fence_after();
+        unsigned char *K2 = sm + L::KQ + (c2 % NS) * L::KQ_STAGE;
+        constexpr uint32_t idU = idesc_bf16(DV, 64, 1, 0);
+        constexpr uint32_t idW = idesc_bf16(DK, 64, 1, 0);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+            mma_bf16(tmem + L::T_U + (c2 % NS) * 64, sdesc_sw128(smem_u32(sm + L::V + kk * 2048), 8192, 1024),
+                     sdesc_sw128(smem_u32(sm + L::TB + kk * 32), 16, 1024), idU, kk > 0);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+            mma_bf16(tmem + L::T_W, sdesc_sw128(smem_u32(K2 + kk * 2048), 16384, 1024),
+                     sdesc_sw128(smem_u32(sm + L::TG + kk * 32), 16, 1024), idW, kk > 0);
+        mma_commit(&bars[B::uw]);
+    };
+    // After the WY MMAs of chunk c2, run by a whole warpgroup (u = thread index 0..127 in it,
+    // tlw = its warp's TMEM lane base): the next V load, W^T to shared memory (bf16), the
+    // lam-scaled K tile in place and, unless the intra side did it, the gam-scaled Q tile (the
+    // MMAs that read them unscaled are done).
+    auto finish_wy = [&](int c2, int u, uint32_t tlw) {
+        const int crow = (DK == 128) ? u : ((u & 31) < 16 ? (u >> 5) * 16 + (u & 31) : -1);  // row of W^T
+        ctl.wait(B::uw, c2 & 1);
+        tc_fence_after();
+        if (u == 0) {
+            if (c2 + 1 < nchunks) load_v(c2 + 1);
+            ctl.arrive(B::tfree);
+        }
+        float x[64];
+        tmem_ld32(tlw + L::T_W, *reinterpret_cast<float(*)[32]>(&x[0]));
+        tmem_ld32(tlw + L::T_W + 32, *reinterpret_cast<float(*)[32]>(&x[32]));
+        tmem_wait_ld();
+        if (crow >= 0) st_row_bf16_sw128(sm + L::WT, crow, x);
+        const float *gv = gates(c2 % NS);
+        unsigned char *K2 = sm + L::KQ + (c2 % NS) * L::KQ_STAGE;
+        const int r = u & 63;
+        const float gr = gv[2 * CH + r], lr = gv[3 * CH + r];
+        if (DK == 128) {
+            scale_row_bf16(K2 + (u >> 6) * 16384, r, lr, 0, 8);
+        } else {
+            scale_row_bf16(K2 + 8192, r, gr, (u >> 6) * 4, (u >> 6) * 4 + 4);
+            scale_row_bf16(K2, r, lr, (u >> 6) * 4, (u >> 6) * 4 + 4);
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+    };
+
 
     if (warp >= 4) {
         // ======================= intra warpgroup =======================
         const int t = tid - 128, wi = t >> 5;
         const uint32_t tl = tmem + ((uint32_t)(wi * 32) << 16);
-        const int crow = (DK == 128) ? t : (lane < 16 ? wi * 16 + lane : -1);  // row of W^T
         float *AF = reinterpret_cast<float *>(sm + L::AF);
         float *TFm = reinterpret_cast<float *>(sm + L::TF);
         float *XSm = reinterpret_cast<float *>(sm + L::XS);
@@ -529,58 +583,24 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
                     for (int i = 0; i < CH; i += 4)
                         *reinterpret_cast<float4 *>(&AF[r * LDF + i]) = make_float4(x[i], x[i + 1], x[i + 2], x[i + 3]);
                 }
-                // gam-scaled Q in place (Q is no longer read by the Gram MMA)
-                const float gr = gam[r];
-                if (DK == 128) {
-                    scale_row_bf16(Kt + (t >> 6) * 16384 + 8192, r, gr, 0, 8);
-                } else {
-                    scale_row_bf16(Kt + 8192, r, gr, (t >> 6) * 4, (t >> 6) * 4 + 4);
-                }
+                // with dk = 128 the intra side takes the gam-scaling of Q (no MMA reads Q unscaled
+                // after the Gram MMA); with dk = 64 the chain side does it
+                if (kIntraScalesQ) scale_row_bf16(Kt + (t >> 6) * 16384 + 8192, r, gam[r], 0, 8);
             }
             tc_fence_before();
+            // the WY MMAs of the previous chunk must have read T diag(b), T diag(b gam)
+            if (c >= 1) ctl.wait(B::tfree, (c - 1) & 1);
             named_bar(2, 128);
             // ---- T = (I + A)^{-1}, written with the bf16 rows of T diag(b), T diag(b gam) ----
             solve_unit_lower(AF, TOut{TFm, sm + L::TB, sm + L::TG, bet, gam}, XSm, t, 2);
             fence_proxy_async_smem();
             named_bar(2, 128);
-            // ---- U~^T = V^T (T diag b)^T ;  W^T = K^T (T diag(b gam))^T ----
-            ctl.wait(B::v_full, c & 1);
-            if (t == kIntraIssuer && !ctl.aborted()) {
-                tc_fence_after();
-                constexpr uint32_t idU = idesc_bf16(DV, 64, 1, 0);
-                constexpr uint32_t idW = idesc_bf16(DK, 64, 1, 0);
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    mma_bf16(tmem + L::T_U + st * 64, sdesc_sw128(smem_u32(sm + L::V + kk * 2048), 8192, 1024),
-                             sdesc_sw128(smem_u32(sm + L::TB + kk * 32), 16, 1024), idU, kk > 0);
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    mma_bf16(tmem + L::T_W, sdesc_sw128(smem_u32(Kt + kk * 2048), 16384, 1024),
-                             sdesc_sw128(smem_u32(sm + L::TG + kk * 32), 16, 1024), idW, kk > 0);
-                mma_commit(&bars[B::uw]);
+            if (!kChainWY) {
+                if (t == kIntraIssuer) issue_wy(c);
+                finish_wy(c, t, tl);
+                named_bar(2, 128);
             }
-            ctl.wait(B::uw, c & 1);
-            tc_fence_after();
-            if (t == kIntraIssuer && c + 1 < nchunks) load_v(c + 1);
-            {
-                // lam-scaled K in place (K is no longer read by the intra MMAs)
-                const int r = t & 63;
-                if (DK == 128) {
-                    scale_row_bf16(Kt + (t >> 6) * 16384, r, lam[r], 0, 8);
-                } else {
-                    scale_row_bf16(Kt, r, lam[r], (t >> 6) * 4, (t >> 6) * 4 + 4);
-                }
-                float x[64];
-                tmem_ld32(tl + L::T_W, *reinterpret_cast<float(*)[32]>(&x[0]));
-                tmem_ld32(tl + L::T_W + 32, *reinterpret_cast<float(*)[32]>(&x[32]));
-                tmem_wait_ld();
-                if (c >= 1) ctl.wait(B::wt_free, (c - 1) & 1);
-                if (crow >= 0) st_row_bf16_sw128(sm + L::WT, crow, x);
-            }
-            fence_proxy_async_smem();
-            tc_fence_before();
-            named_bar(2, 128);
-            if (t == 0) ctl.arrive(B::ready + st);
+            if (t == 0) ctl.arrive(B::tready + st);
         }
     } else {
         // ======================= chain warpgroup =======================
@@ -646,6 +666,13 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
                 tmem_st32(tl + L::T_S + cb * 32, x);
             }
             tmem_wait_st();
+            if (kChainWY) {
+                if (tid == 0) {
+                    ctl.wait(B::tready + 0, 0);
+                    issue_wy(0);
+                }
+                finish_wy(0, tid, tl);
+            }
             fence_proxy_async_smem();
             tc_fence_before();
             named_bar(1, 128);
@@ -654,7 +681,10 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
             const int st = c % NS;
             const uint32_t tO = tmem + L::T_O;
             unsigned char *Kt = sm + L::KQ + st * L::KQ_STAGE;
-            ctl.wait(B::ready + st, (c / NS) & 1);
+            const bool has_next = c + 1 < nchunks;
+            const bool wy_chain = kChainWY && has_next;  // this warpgroup does the WY part of c+1
+            bool wy_next = false;  // thread 0: WY MMAs of chunk c+1 already issued
+            if (!kChainWY) ctl.wait(B::tready + st, (c / NS) & 1);
             if (tid == 0 && !ctl.aborted()) {
                 tc_fence_after();
                 constexpr uint32_t idN = idesc_bf16(DV, 64, 0, 1, 1);
@@ -675,7 +705,6 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
             }
             ctl.wait(B::u, c & 1);
             tc_fence_after();
-            if (tid == 0) ctl.arrive(B::wt_free);
             {
                 float x[64];
                 tmem_ld32(tl + L::T_U + st * 64, *reinterpret_cast<float(*)[32]>(&x[0]));
@@ -695,6 +724,12 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
                     mma_bf16(tmem + L::T_S, sdesc_sw128(smem_u32(sm + L::UT + kk * 32), 16, 1024),
                              sdesc_sw128(smem_u32(Kt + kk * 2048), 16384, 1024), idS, 1);
                 mma_commit(&bars[B::s]);
+                // The tensor pipe runs a CTA's MMAs in issue order: the WY MMAs of chunk c+1 go
+                // behind the state increment, and only if the intra side is already done with it.
+                if (wy_chain && mbar_test_wait(&bars[B::tready + (c + 1) % NS], ((c + 1) / NS) & 1)) {
+                    issue_wy(c + 1);
+                    wy_next = true;
+                }
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)  // O += P U: A = P rows (K-major), B = U^T rows (K-major)
                     mma_bf16(tO, sdesc_sw128(smem_u32(sm + L::PM + st * 8192 + kk * 32), 16, 1024),
@@ -729,6 +764,13 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
             }
             fence_proxy_async_smem();
             tc_fence_before();
+            if (wy_chain) {
+                if (tid == 0 && !wy_next) {
+                    ctl.wait(B::tready + (c + 1) % NS, ((c + 1) / NS) & 1);
+                    issue_wy(c + 1);
+                }
+                finish_wy(c + 1, tid, tl);
+            }
             named_bar(1, 128);
             out_epilogue(c);
         }
