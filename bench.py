@@ -36,7 +36,7 @@ import workloads  # noqa: E402
 METRIC = "gated-delta chunk-fwd tokens/s & % roofline; decode state-updates/s & HBM %"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 KERNEL_SOURCES = {
-    "chunk": "linear_attention_sequence_rule_b200/csrc/gdn_chunk_simt.cu",
+    "chunk": "linear_attention_sequence_rule_b200/csrc/gdn_chunk_tc.cu",
     "decode": "linear_attention_sequence_rule_b200/csrc/gdn_decode.cu",
 }
 
@@ -189,12 +189,27 @@ def to_dev(inp):
     return {k: (v.cuda().contiguous() if torch.is_tensor(v) else v) for k, v in inp.items()}
 
 
+def chunk_workspace(gdn, d):
+    """The workspace a chunk call needs (the segment scan of long dense sequences), or None."""
+    n = gdn.workspace_bytes(d["B"], d["T"], d["H"], d["dk"], d["dv"], d["cu_seqlens"] is not None,
+                            d["q"].dtype)
+    return torch.empty(n, dtype=torch.uint8, device="cuda") if n else None
+
+
+def chunk_launches(gdn, d):
+    """Kernels one chunk call launches: one chunk kernel, or with the segment scan a segment table,
+    two local passes, the combine and the output pass."""
+    return 5 if chunk_workspace(gdn, d) is not None else 1
+
+
 def time_chunk(gdn, d, steps, warmup, flush, stream):
     """Per-step CUDA-event time (ms) of gdn.chunk_fwd, L2 flushed before every step."""
     out = torch.empty_like(d["v"])
     Sf = torch.empty((d["B"], d["H"], d["dk"], d["dv"]), dtype=torch.float32, device="cuda")
+    ws = chunk_workspace(gdn, d)
     call = lambda: gdn.chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], S0=d["S0"],
-                                 cu_seqlens=d["cu_seqlens"], out=out, S_final=Sf, stream=stream)
+                                 cu_seqlens=d["cu_seqlens"], out=out, S_final=Sf, workspace=ws,
+                                 stream=stream)
     with torch.cuda.stream(stream):
         for _ in range(warmup):
             flush.zero_()
@@ -211,6 +226,11 @@ def time_chunk(gdn, d, steps, warmup, flush, stream):
     return [s.elapsed_time(e) for s, e in ev]
 
 
+def gdn_mod():
+    import linear_attention_sequence_rule_b200 as gdn
+    return gdn
+
+
 def chunk_numbers(name, d, times_ms, peaks):
     ms = statistics.mean(times_ms)
     th = d["q"].shape[0] * (d["q"].shape[1] if d["cu_seqlens"] is None else 1) * d["H"]
@@ -221,6 +241,7 @@ def chunk_numbers(name, d, times_ms, peaks):
     gbs = by / (ms * 1e-3) / 1e9
     tfs = fl / (ms * 1e-3) / 1e12
     return dict(workload=name, ms=ms, tokens=tokens, tokens_per_s=tokens / (ms * 1e-3),
+                launches_per_call=chunk_launches(gdn_mod(), d),
                 algo_bytes=by, algo_flops=fl, gbs=gbs, hbm_frac=gbs / peaks["hbm_gbs"],
                 tflops=tfs, tensor_frac=tfs / peaks["bf16_tflops"])
 
@@ -391,7 +412,7 @@ def run_ours(args, world, rank, local):
                    "frac": main["tensor_frac"], "algo_flops_per_launch": main["algo_flops"]},
         "e2e": {"value": tokens_all / (e2e_ms * 1e-3), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
-        "gpu_launches": args.steps,
+        "gpu_launches": args.steps * main["launches_per_call"],
         "clocks": clk.result(),
         "cpu_baseline": cpu,
     }

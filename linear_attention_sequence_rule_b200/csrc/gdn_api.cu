@@ -61,8 +61,8 @@ static int check_chunk_shape(int B, int T, int H, int dk, int dv, int chunk, int
 
 static size_t chunk_workspace(int B, int T, int H, int dk, int dv, int varlen, int dtype)
 {
-    (void)B; (void)T; (void)H; (void)dk; (void)dv; (void)varlen; (void)dtype;
-    return 0;
+    if (dtype != GDN_DTYPE_BF16) return 0;
+    return chunk_tc_workspace_bytes(B, T, H, dk, dv, varlen, dtype);
 }
 
 }  // namespace gdn

@@ -58,6 +58,10 @@ constexpr int LDF = 68;  // fp32 row stride of the 64 x 64 solve matrices
 // on warp 5, away from warp 4, which shares an SM sub-partition with the chain's issuing thread
 // (thread 0).
 constexpr int kIntraIssuer = 96;
+// Kernel flags (used by the segment scan): V is taken as zero (nothing of V is loaded), and the
+// initial state is the identity (dv must equal dk).  With out == nullptr no output is formed.
+constexpr int kFlagVZero = 1;
+constexpr int kFlagS0Identity = 2;
 constexpr int kScanWarp = 1;
 
 template <int DK, int DV>
@@ -321,7 +325,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
                 const __grid_constant__ CUtensorMap tmV, const float *__restrict__ log_alpha,
                 const float *__restrict__ beta, const float *__restrict__ S0,
                 __nv_bfloat16 *__restrict__ out, float *__restrict__ S_final,
-                const int32_t *__restrict__ cu_seqlens, int T, int H)
+                const int32_t *__restrict__ cu_seqlens, int T, int H, int flags)
 {
     using L = TcCfg<DK, DV>;
     constexpr int NS = L::NS;
@@ -390,8 +394,10 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
             }
         }
     };
+    const bool v_zero = (flags & kFlagVZero) != 0;
+    const bool want_out = out != nullptr;
     auto load_v = [&](int c) {
-        if (ctl.aborted()) return;
+        if (ctl.aborted() || v_zero) return;
         const int tk = (int)(tok0 + (long)c * CH);
         mbar_arrive_expect_tx(&bars[B::v_full], (DV / 64) * 8192);
         for (int vb = 0; vb < DV / 64; ++vb)
@@ -408,16 +414,18 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
     if (tid == 0 && nchunks > 0) load_v(0);
         // WY MMAs of chunk c2 (thread 0): U~^T = V^T (T diag b)^T into its U slot, W^T = K^T (T diag(b gam))^T.
     auto issue_wy = [&](int c2) {
-        ctl.wait(B::v_full, c2 & 1);
+        if (!v_zero) ctl.wait(B::v_full, c2 & 1);
         if (ctl.aborted()) return;
         tc_fence_after();
         unsigned char *K2 = sm + L::KQ + (c2 % NS) * L::KQ_STAGE;
         constexpr uint32_t idU = idesc_bf16(DV, 64, 1, 0);
         constexpr uint32_t idW = idesc_bf16(DK, 64, 1, 0);
+        if (!v_zero) {
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-            mma_bf16(tmem + L::T_U + (c2 % NS) * 64, sdesc_sw128(smem_u32(sm + L::V + kk * 2048), 8192, 1024),
-                     sdesc_sw128(smem_u32(sm + L::TB + kk * 32), 16, 1024), idU, kk > 0);
+            for (int kk = 0; kk < 4; ++kk)
+                mma_bf16(tmem + L::T_U + (c2 % NS) * 64, sdesc_sw128(smem_u32(sm + L::V + kk * 2048), 8192, 1024),
+                         sdesc_sw128(smem_u32(sm + L::TB + kk * 32), 16, 1024), idU, kk > 0);
+        }
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
             mma_bf16(tmem + L::T_W, sdesc_sw128(smem_u32(K2 + kk * 2048), 16384, 1024),
@@ -624,6 +632,11 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
         auto out_epilogue = [&](int c) {
             const long tk = tok0 + (long)c * CH;
             const int n = (int)min((long)CH, len - (long)c * CH);
+            if (!want_out) {
+                named_bar(1, 128);
+                if (tid == 0) ctl.arrive(B::cdone + (c % NS));
+                return;
+            }
             ctl.wait(B::o, c & 1);
             tc_fence_after();
             const int r = 16 * warp + (lane & 15);
@@ -659,7 +672,8 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
                 float x[32];
 #pragma unroll
                 for (int i = 0; i < 32; ++i)
-                    x[i] = (j >= 0 && S0) ? S0[sbase + (size_t)(cb * 32 + i) * DV + j] : 0.f;
+                    x[i] = (flags & kFlagS0Identity) ? ((cb * 32 + i == j) ? 1.f : 0.f)
+                                                     : ((j >= 0 && S0) ? S0[sbase + (size_t)(cb * 32 + i) * DV + j] : 0.f);
                 store_state_bf16(cb, x);
 #pragma unroll
                 for (int i = 0; i < 32; ++i) x[i] *= g0;
@@ -692,11 +706,13 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
 #pragma unroll
                 for (int kk = 0; kk < DK / 16; ++kk) {
                     const uint64_t a = sdesc_sw128(smem_u32(sm + L::ST + (kk >> 2) * (DV * 128) + (kk & 3) * 32), 16, 1024);
-                    mma_bf16(tmem + L::T_U + st * 64, a, sdesc_sw128(smem_u32(sm + L::WT + kk * 2048), 16, 1024), idN, 1);
+                    mma_bf16(tmem + L::T_U + st * 64, a, sdesc_sw128(smem_u32(sm + L::WT + kk * 2048), 16, 1024), idN,
+                             v_zero ? (kk > 0) : 1);
                 }
                 mma_commit(&bars[B::u]);
 #pragma unroll
                 for (int kk = 0; kk < DK / 16; ++kk) {
+                    if (!want_out) break;
                     // O = (gam Q) S: A = gam-scaled Q tile (K-major), B = S^T rows (K-major)
                     const uint32_t a = smem_u32(Kt + (kk >> 2) * 16384 + 8192 + (kk & 3) * 32);
                     const uint64_t b = sdesc_sw128(smem_u32(sm + L::ST + (kk >> 2) * (DV * 128) + (kk & 3) * 32), 16, 1024);
@@ -730,11 +746,13 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
                     issue_wy(c + 1);
                     wy_next = true;
                 }
+                if (want_out) {
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk)  // O += P U: A = P rows (K-major), B = U^T rows (K-major)
-                    mma_bf16(tO, sdesc_sw128(smem_u32(sm + L::PM + st * 8192 + kk * 32), 16, 1024),
-                             sdesc_sw128(smem_u32(sm + L::UT + kk * 32), 16, 1024), idP, 1);
-                mma_commit(&bars[B::o]);
+                    for (int kk = 0; kk < 4; ++kk)  // O += P U: A = P rows (K-major), B = U^T rows (K-major)
+                        mma_bf16(tO, sdesc_sw128(smem_u32(sm + L::PM + st * 8192 + kk * 32), 16, 1024),
+                                 sdesc_sw128(smem_u32(sm + L::UT + kk * 32), 16, 1024), idP, 1);
+                    mma_commit(&bars[B::o]);
+                }
             }
             ctl.wait(B::s, c & 1);
             tc_fence_after();
@@ -789,7 +807,8 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
                 }
             } else if (j >= 0) {
                 for (int c2 = 0; c2 < DK; ++c2)
-                    S_final[sbase + (size_t)c2 * DV + j] = S0 ? S0[sbase + (size_t)c2 * DV + j] : 0.f;
+                    S_final[sbase + (size_t)c2 * DV + j] =
+                        (flags & kFlagS0Identity) ? (c2 == j ? 1.f : 0.f) : (S0 ? S0[sbase + (size_t)c2 * DV + j] : 0.f);
             }
         }
     }
@@ -833,16 +852,31 @@ bool make_map(CUtensorMap *m, const void *base, long tokens, int H, int d)
     return r == CUDA_SUCCESS;
 }
 
+// One launch of the chunk kernel over `nseq` sequences given either densely (cu == nullptr:
+// sequence s owns tokens s*T .. s*T+T-1) or by offsets cu[0..nseq].
+struct TcLaunch {
+    const void *q, *k, *v;
+    const float *log_alpha, *beta, *S0;
+    void *out;
+    float *S_final;
+    const int32_t *cu;
+    int nseq, T, H;
+    long tokens;  // rows of the q/k/v tensors
+    int flags;
+};
+
 template <int DK, int DV>
-cudaError_t launch_tc(const ChunkArgs &a, cudaStream_t st)
+cudaError_t launch_tc(const TcLaunch &a, cudaStream_t st)
 {
     using L = TcCfg<DK, DV>;
-    const long tokens = a.cu_seqlens ? (long)a.T : (long)a.B * a.T;
     CUtensorMap mq, mk, mv;
     // a zero-token varlen call still launches so that S_final = S0 is written
-    const long map_tokens = tokens > 0 ? tokens : 1;
+    const long map_tokens = a.tokens > 0 ? a.tokens : 1;
+    // with V taken as zero nothing is loaded through the V map; any valid map will do
+    const void *vsrc = (a.flags & kFlagVZero) ? a.k : a.v;
+    const int vdim = (a.flags & kFlagVZero) ? DK : DV;
     if (!make_map(&mq, a.q, map_tokens, a.H, DK) || !make_map(&mk, a.k, map_tokens, a.H, DK) ||
-        !make_map(&mv, a.v, map_tokens, a.H, DV)) {
+        !make_map(&mv, vsrc, map_tokens, a.H, vdim)) {
         set_error("cuTensorMapEncodeTiled failed");
         return cudaErrorInvalidValue;
     }
@@ -850,21 +884,200 @@ cudaError_t launch_tc(const ChunkArgs &a, cudaStream_t st)
     auto kern = chunk_tc_kernel<DK, DV>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    const dim3 grid(1, a.H, a.B);
+    const dim3 grid(1, a.H, a.nseq);
     kern<<<grid, kThreads, smem, st>>>(mq, mk, mv, a.log_alpha, a.beta, a.S0,
-                                       static_cast<__nv_bfloat16 *>(a.out), a.S_final, a.cu_seqlens,
-                                       a.T, a.H);
+                                       static_cast<__nv_bfloat16 *>(a.out), a.S_final, a.cu, a.T, a.H,
+                                       a.flags);
     return cudaGetLastError();
+}
+
+// ---- segment scan for long sequences with few (sequence, head) chains ------------------------
+//
+// The state map over a stretch of tokens is affine, S_end = M S_in + S_loc, with M the
+// transition of the stretch (the recurrence started from S = I with V = 0) and S_loc the state
+// it reaches from S = 0.  A sequence is cut into G segments of L chunks:
+//   pass A: per segment, S_loc (value chains from zero) and M (transition chains from the
+//           identity with V = 0), both by the chunk kernel with outputs off, all segments at once;
+//   pass B: per (sequence, head), the scan S_in,g+1 = M_g S_in,g + S_loc,g in fp32, ending with
+//           S_final = M_{G-1} S_in,G-1 + S_loc,G-1;
+//   pass C: the chunk kernel over every segment from its S_in, writing the outputs.
+
+struct SegPlan {
+    int G = 1, L = 0;  // segments per sequence, chunks per segment
+};
+
+SegPlan plan_segments(int B, int T, int H, int varlen, int dtype)
+{
+    SegPlan p;
+    if (varlen || dtype != GDN_DTYPE_BF16) return p;
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+        cudaGetLastError();
+        return p;
+    }
+    const long nchunks = ((long)T + CH - 1) / CH;
+    const long chains = (long)B * H;
+    long G = sms / chains;     // pass C then fills the SMs
+    G = min(G, nchunks / 16);  // at least 16 chunks per segment
+    if (G < 2) return p;
+    const long L = (nchunks + G - 1) / G;
+    p.L = (int)L;
+    p.G = (int)((nchunks + L - 1) / L);
+    return p;
+}
+
+struct SegWork {
+    int32_t *cu;
+    float *Sloc, *M, *Sin;
+    size_t bytes;
+};
+
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+SegWork seg_layout(void *base, int B, int H, int dk, int dv, const SegPlan &p)
+{
+    SegWork w{};
+    const size_t nseg = (size_t)B * p.G;
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        const size_t o = off;
+        off += align256(bytes);
+        return o;
+    };
+    const size_t o_cu = take((nseg + 1) * sizeof(int32_t));
+    const size_t o_sloc = take(nseg * H * (size_t)dk * dv * sizeof(float));
+    const size_t o_m = take(nseg * H * (size_t)dk * dk * sizeof(float));
+    const size_t o_sin = take(nseg * H * (size_t)dk * dv * sizeof(float));
+    w.bytes = off;
+    char *b = static_cast<char *>(base);
+    if (b) {
+        w.cu = reinterpret_cast<int32_t *>(b + o_cu);
+        w.Sloc = reinterpret_cast<float *>(b + o_sloc);
+        w.M = reinterpret_cast<float *>(b + o_m);
+        w.Sin = reinterpret_cast<float *>(b + o_sin);
+    }
+    return w;
+}
+
+// cu[b*G + g] = first token of segment g of sequence b; cu[B*G] = B*T.
+__global__ void seg_table_kernel(int32_t *cu, int B, int T, int G, int L)
+{
+    const int n = B * G;
+    for (int s = blockIdx.x * blockDim.x + threadIdx.x; s <= n; s += gridDim.x * blockDim.x) {
+        if (s == n) {
+            cu[s] = B * T;
+        } else {
+            const int b = s / G, g = s % G;
+            const long start = min((long)g * L * CH, (long)T);
+            cu[s] = (int32_t)((long)b * T + start);
+        }
+    }
+}
+
+// Pass B: one CTA of 256 threads per (32 value columns, head, sequence).  S (dk x 32, fp32) is
+// kept in shared memory; S_in of every segment is written out, then S <- M_g S + S_loc,g.
+__global__ void __launch_bounds__(256) seg_combine_kernel(const float *__restrict__ M, const float *__restrict__ Sloc,
+                                                          const float *__restrict__ S0, float *__restrict__ Sin,
+                                                          float *__restrict__ S_final, int G, int H, int dk, int dv)
+{
+    extern __shared__ float sh[];  // two dk x 32 buffers
+    const int cb = blockIdx.x, h = blockIdx.y, b = blockIdx.z, t = threadIdx.x;
+    const int c0 = cb * 32;
+    float *cur = sh, *nxt = sh + dk * 32;
+    const size_t st0 = ((size_t)b * H + h) * dk * dv;
+    for (int i = t; i < dk * 32; i += 256) {
+        const int r = i / 32, c = i % 32;
+        cur[i] = S0 ? S0[st0 + (size_t)r * dv + c0 + c] : 0.f;
+    }
+    __syncthreads();
+    const int per = dk * 32 / 256;  // outputs per thread, all in one row: 8 (dk = 64) or 16 (dk = 128)
+    const int first = t * per, r = first / 32, cc = first % 32;
+    for (int g = 0; g < G; ++g) {
+        const size_t seg = (size_t)b * G + g;
+        const size_t sv = (seg * H + h) * (size_t)dk * dv;
+        const size_t smi = (seg * H + h) * (size_t)dk * dk;
+        for (int i = t; i < dk * 32; i += 256) {
+            const int rr = i / 32, c = i % 32;
+            Sin[sv + (size_t)rr * dv + c0 + c] = cur[i];
+        }
+        float acc[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) acc[e] = 0.f;
+        const float *mrow = M + smi + (size_t)r * dk;
+        for (int k = 0; k < dk; ++k) {
+            const float m = mrow[k];
+#pragma unroll
+            for (int e = 0; e < 16; ++e)
+                if (e < per) acc[e] = fmaf(m, cur[k * 32 + cc + e], acc[e]);
+        }
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+            if (e < per) nxt[r * 32 + cc + e] = acc[e] + Sloc[sv + (size_t)r * dv + c0 + cc + e];
+        __syncthreads();
+        float *tmp = cur;
+        cur = nxt;
+        nxt = tmp;
+    }
+    if (S_final) {
+        for (int i = t; i < dk * 32; i += 256) {
+            const int rr = i / 32, c = i % 32;
+            S_final[st0 + (size_t)rr * dv + c0 + c] = cur[i];
+        }
+    }
+}
+
+template <int DK, int DV>
+cudaError_t run_chunk(const ChunkArgs &a, cudaStream_t st)
+{
+    const long tokens = a.cu_seqlens ? (long)a.T : (long)a.B * a.T;
+    const SegPlan p = plan_segments(a.B, a.T, a.H, a.cu_seqlens != nullptr, a.dtype);
+    if (p.G <= 1) {
+        return launch_tc<DK, DV>(TcLaunch{a.q, a.k, a.v, a.log_alpha, a.beta, a.S0, a.out, a.S_final,
+                                          a.cu_seqlens, a.B, a.T, a.H, tokens, 0},
+                                 st);
+    }
+    const SegWork w = seg_layout(a.workspace, a.B, a.H, DK, DV, p);
+    const int nseg = a.B * p.G;
+    seg_table_kernel<<<(nseg + 256) / 256, 256, 0, st>>>(w.cu, a.B, a.T, p.G, p.L);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    // pass A: local states from zero, and transitions from the identity with V = 0
+    e = launch_tc<DK, DV>(TcLaunch{a.q, a.k, a.v, a.log_alpha, a.beta, nullptr, nullptr, w.Sloc, w.cu, nseg,
+                                   a.T, a.H, tokens, 0},
+                          st);
+    if (e != cudaSuccess) return e;
+    e = launch_tc<DK, DK>(TcLaunch{a.q, a.k, nullptr, a.log_alpha, a.beta, nullptr, nullptr, w.M, w.cu, nseg,
+                                   a.T, a.H, tokens, kFlagVZero | kFlagS0Identity},
+                          st);
+    if (e != cudaSuccess) return e;
+    // pass B: segment scan of the states
+    const size_t shm = 2 * (size_t)DK * 32 * sizeof(float);
+    seg_combine_kernel<<<dim3(DV / 32, a.H, a.B), 256, shm, st>>>(w.M, w.Sloc, a.S0, w.Sin, a.S_final, p.G,
+                                                                  a.H, DK, DV);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    // pass C: outputs of every segment from its entry state
+    return launch_tc<DK, DV>(TcLaunch{a.q, a.k, a.v, a.log_alpha, a.beta, w.Sin, a.out, nullptr, w.cu, nseg,
+                                      a.T, a.H, tokens, 0},
+                             st);
 }
 
 }  // namespace
 
+size_t chunk_tc_workspace_bytes(int B, int T, int H, int dk, int dv, int varlen, int dtype)
+{
+    const SegPlan p = plan_segments(B, T, H, varlen, dtype);
+    if (p.G <= 1) return 0;
+    return seg_layout(nullptr, B, H, dk, dv, p).bytes;
+}
+
 cudaError_t launch_chunk_tc(const ChunkArgs &a, cudaStream_t stream)
 {
-    if (a.dk == 128 && a.dv == 128) return launch_tc<128, 128>(a, stream);
-    if (a.dk == 128 && a.dv == 64) return launch_tc<128, 64>(a, stream);
-    if (a.dk == 64 && a.dv == 128) return launch_tc<64, 128>(a, stream);
-    return launch_tc<64, 64>(a, stream);
+    if (a.dk == 128 && a.dv == 128) return run_chunk<128, 128>(a, stream);
+    if (a.dk == 128 && a.dv == 64) return run_chunk<128, 64>(a, stream);
+    if (a.dk == 64 && a.dv == 128) return run_chunk<64, 128>(a, stream);
+    return run_chunk<64, 64>(a, stream);
 }
 
 int read_and_clear_tc_error()

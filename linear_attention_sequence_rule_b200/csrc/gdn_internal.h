@@ -31,8 +31,11 @@ struct ChunkArgs {
 // Chunk forward on CUDA cores, fp32 arithmetic throughout (fp32 inputs).
 cudaError_t launch_chunk_simt(const ChunkArgs &a, cudaStream_t stream);
 
-// Chunk forward on the tcgen05 tensor cores (bf16 inputs).
+// Chunk forward on the tcgen05 tensor cores (bf16 inputs).  Dense inputs with few (sequence,
+// head) chains for the SM count run as a segment scan, which needs a workspace of
+// chunk_tc_workspace_bytes(...) bytes (0 when not).
 cudaError_t launch_chunk_tc(const ChunkArgs &a, cudaStream_t stream);
+size_t chunk_tc_workspace_bytes(int B, int T, int H, int dk, int dv, int varlen, int dtype);
 
 // Device error word of the tensor-core kernels (bounded waits that ran out); read and cleared
 // after synchronising the device.  Returns -1 when the read itself failed.
