@@ -98,6 +98,13 @@ GDN_API int gdn_chunk_fwd(const void *q, const void *k, const void *v, const flo
  * gdn_chunk_fwd_workspace_bytes -- device scratch that gdn_chunk_fwd needs for these sizes
  * (varlen: non-zero when cu_seqlens will be passed).  Returns 0 when no scratch is needed and
  * (size_t)-1 for arguments gdn_chunk_fwd would reject.
+ *   Scratch is needed only by the segment scan: dense bf16 calls whose B*H (sequence, head)
+ *   chains number at most half the SMs of the CURRENT device and whose sequences span at least
+ *   32 chunks are cut into segments, each segment's state map S -> M S + S_loc is computed in
+ *   parallel, the maps are scanned per chain, and the outputs are recomputed per segment.  The
+ *   scratch then holds, per segment and head, S_loc and the entry state (dk x dv fp32 each), M
+ *   (dk x dk fp32) and a segment offset table; it is at most about 3 * (SM count) * dk * dv * 4
+ *   bytes.  Query with the device current that the call will run on.
  */
 GDN_API size_t gdn_chunk_fwd_workspace_bytes(int B, int T, int H, int dk, int dv, int chunk, int varlen,
                                      int dtype);
