@@ -21,7 +21,8 @@
  *
  * Conventions shared by every entry point
  *   - Every tensor pointer is a DEVICE pointer owned by the caller.  The library allocates no
- *     memory, keeps no state between calls and may be called from several host threads.
+ *     memory, keeps no state between calls and may be called from several host threads (the
+ *     one exception, gdn_chunk_fwd_noalloc, owns a fixed scratch array per device).
  *   - Calls are asynchronous: they validate on the host, enqueue kernels on `stream` (a
  *     cudaStream_t; NULL = the legacy default stream) and return.  Errors found on the host are
  *     returned before anything is enqueued, so a failed call writes nothing.
@@ -108,6 +109,26 @@ GDN_API int gdn_chunk_fwd(const void *q, const void *k, const void *v, const flo
  */
 GDN_API size_t gdn_chunk_fwd_workspace_bytes(int B, int T, int H, int dk, int dv, int chunk, int varlen,
                                      int dtype);
+
+/*
+ * gdn_chunk_fwd_noalloc -- gdn_chunk_fwd without a workspace argument: the scratch of the segment
+ * scan (see gdn_chunk_fwd_workspace_bytes) comes from a fixed 32 MiB array of device memory that
+ * the library owns, one per device.  The pages that define the operation have no counterpart of
+ * this entry point; it exists for callers that cannot provide device scratch (a serving runtime
+ * that has reserved its device memory up front and admits no call-time allocation, or a C host
+ * program without a device allocator).  Arguments, layouts and results are those of
+ * gdn_chunk_fwd.
+ *   - The first call on each device looks up the array's address there (and loads the module);
+ *     make that first call before any stream capture on that device.
+ *   - Calls on the same device must not overlap in time (two streams, two host threads): they
+ *     share the one array.  Nothing in it needs to start at zero.
+ *   - Sizes whose scratch would exceed 32 MiB return GDN_ERR_WORKSPACE (about 3 * SMs * dk * dv
+ *     * 4 bytes are needed at most: 29.1 MB for dk = dv = 128 on 148 SMs).
+ */
+GDN_API int gdn_chunk_fwd_noalloc(const void *q, const void *k, const void *v, const float *log_alpha,
+                                  const float *beta, const float *S0, void *out, float *S_final, int B,
+                                  int T, int H, int dk, int dv, int chunk, const int32_t *cu_seqlens,
+                                  int dtype, void *stream);
 
 /*
  * gdn_decode_step -- one generation step: every (n, h) state takes exactly one token, in place

@@ -3,7 +3,7 @@
 Argument marshalling only: every step of the computation runs in the library's CUDA kernels.
 PyTorch provides device memory and streams.  The binding has two layers:
 
-* ``gdn_chunk_fwd``, ``gdn_decode_step``, ``gdn_chunk_fwd_workspace_bytes``,
+* ``gdn_chunk_fwd``, ``gdn_chunk_fwd_noalloc``, ``gdn_decode_step``, ``gdn_chunk_fwd_workspace_bytes``,
   ``gdn_status_string``, ``gdn_last_error``, ``gdn_version`` -- the C-ABI entry points of
   ``include/gdn.h`` with the same names and arguments (pointers as Python ints);
 * ``chunk_fwd`` and ``decode_step`` -- the same calls taking torch tensors; they check shapes,
@@ -22,7 +22,7 @@ import torch
 __all__ = [
     "GdnError", "GDN_OK", "GDN_ERR_INVALID_ARGUMENT", "GDN_ERR_UNSUPPORTED", "GDN_ERR_WORKSPACE",
     "GDN_ERR_CUDA", "GDN_ERR_TIMEOUT", "GDN_DTYPE_F32", "GDN_DTYPE_BF16", "LIB_PATH",
-    "gdn_chunk_fwd", "gdn_decode_step", "gdn_chunk_fwd_workspace_bytes", "gdn_status_string",
+    "gdn_chunk_fwd", "gdn_chunk_fwd_noalloc", "gdn_decode_step", "gdn_chunk_fwd_workspace_bytes", "gdn_status_string",
     "gdn_last_error", "gdn_version", "gdn_device_status", "device_status", "chunk_fwd", "decode_step", "workspace_bytes",
 ]
 
@@ -48,6 +48,9 @@ _vp, _sz, _i = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int
 _lib.gdn_chunk_fwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i,
                                _vp, _i, _vp, _sz, _vp]
 _lib.gdn_chunk_fwd.restype = _i
+_lib.gdn_chunk_fwd_noalloc.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i,
+                                       _i, _vp, _i, _vp]
+_lib.gdn_chunk_fwd_noalloc.restype = _i
 _lib.gdn_chunk_fwd_workspace_bytes.argtypes = [_i, _i, _i, _i, _i, _i, _i, _i]
 _lib.gdn_chunk_fwd_workspace_bytes.restype = _sz
 _lib.gdn_decode_step.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp]
@@ -74,6 +77,12 @@ def gdn_chunk_fwd(q, k, v, log_alpha, beta, S0, out, S_final, B, T, H, dk, dv, c
                   dtype, workspace, workspace_bytes, stream) -> int:
     return _lib.gdn_chunk_fwd(q, k, v, log_alpha, beta, S0, out, S_final, B, T, H, dk, dv, chunk,
                               cu_seqlens, dtype, workspace, workspace_bytes, stream)
+
+
+def gdn_chunk_fwd_noalloc(q, k, v, log_alpha, beta, S0, out, S_final, B, T, H, dk, dv, chunk,
+                          cu_seqlens, dtype, stream) -> int:
+    return _lib.gdn_chunk_fwd_noalloc(q, k, v, log_alpha, beta, S0, out, S_final, B, T, H, dk, dv,
+                                      chunk, cu_seqlens, dtype, stream)
 
 
 def gdn_chunk_fwd_workspace_bytes(B, T, H, dk, dv, chunk, varlen, dtype) -> int:

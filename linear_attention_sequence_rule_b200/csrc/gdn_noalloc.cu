@@ -1,0 +1,86 @@
+// gdn_noalloc.cu -- gdn_chunk_fwd_noalloc: the chunk forward with the scratch of its segment scan
+// taken from a fixed array of device memory that belongs to this library, so that the caller
+// passes no workspace and nothing is allocated at call time.
+//
+// Who needs it: callers that cannot hand over device scratch of their own.  A serving runtime
+// that reserves nearly all device memory up front for its recurrent-state cache has no room
+// left for a call-time cudaMalloc (it fails, or forces a device-wide synchronisation in the
+// middle of a step), and a host program in plain C that drives this library has no device
+// allocator to carve a workspace from.  Everything else goes through gdn_chunk_fwd unchanged.
+//
+// Limits: the scratch is one array per device, so calls on the same device must not overlap in
+// time (on two streams, or from two host threads): they would share it and corrupt each other's
+// results.  Calls whose scratch would exceed kScratchBytes are rejected with GDN_ERR_WORKSPACE.
+// Nothing in the scratch has to start at zero: the segment scan writes every byte it reads
+// (offset table, local states, transitions, entry states) earlier in the same call.
+#include <mutex>
+
+#include "gdn_internal.h"
+#include "../../include/gdn.h"
+
+namespace {
+
+// 32 MiB.  The segment scan keeps per (segment, head) a local state and an entry state
+// (dk x dv fp32) and a transition (dk x dk fp32), with segments x heads bounded by the SM count,
+// plus a small offset table: 3 * 148 * 128 * 128 * 4 B = 29.1 MB for dk = dv = 128 on a 148-SM
+// device, the largest case there.
+constexpr size_t kScratchBytes = size_t(32) << 20;
+constexpr int kMaxDevices = 64;
+
+std::mutex g_mu;
+void *g_scratch_ptr[kMaxDevices];
+
+}  // namespace
+
+static __device__ __align__(256) unsigned char g_scratch[kScratchBytes];
+
+// Device address of g_scratch on the current device, looked up once per device with that device
+// current.  The first call on a device loads this module there, so make it before any stream
+// capture on that device.
+static int scratch_on_current_device(void **ptr)
+{
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) {
+        gdn::set_error("gdn_chunk_fwd_noalloc: cudaGetDevice: %s", cudaGetErrorString(e));
+        return GDN_ERR_CUDA;
+    }
+    if (dev < 0 || dev >= kMaxDevices) {
+        gdn::set_error("gdn_chunk_fwd_noalloc: device %d beyond the %d supported", dev, kMaxDevices);
+        return GDN_ERR_UNSUPPORTED;
+    }
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (!g_scratch_ptr[dev]) {
+        void *p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_scratch);
+        if (e != cudaSuccess || p == nullptr) {
+            gdn::set_error("gdn_chunk_fwd_noalloc: cudaGetSymbolAddress: %s", cudaGetErrorString(e));
+            return GDN_ERR_CUDA;
+        }
+        g_scratch_ptr[dev] = p;
+    }
+    *ptr = g_scratch_ptr[dev];
+    return GDN_OK;
+}
+
+int gdn_chunk_fwd_noalloc(const void *q, const void *k, const void *v, const float *log_alpha,
+                          const float *beta, const float *S0, void *out, float *S_final, int B, int T,
+                          int H, int dk, int dv, int chunk, const int32_t *cu_seqlens, int dtype,
+                          void *stream)
+{
+    const size_t need = gdn_chunk_fwd_workspace_bytes(B, T, H, dk, dv, chunk, cu_seqlens != nullptr, dtype);
+    if (need == (size_t)-1)  // rejected sizes: gdn_chunk_fwd reports why, before touching the device
+        return gdn_chunk_fwd(q, k, v, log_alpha, beta, S0, out, S_final, B, T, H, dk, dv, chunk, cu_seqlens,
+                             dtype, nullptr, 0, stream);
+    void *scratch = nullptr;
+    const int rc = scratch_on_current_device(&scratch);
+    if (rc != GDN_OK) return rc;
+    if (need > kScratchBytes) {
+        gdn::set_error("gdn_chunk_fwd_noalloc: these sizes need %zu bytes of scratch; the static scratch "
+                       "holds %zu (use gdn_chunk_fwd with a workspace)",
+                       need, kScratchBytes);
+        return GDN_ERR_WORKSPACE;
+    }
+    return gdn_chunk_fwd(q, k, v, log_alpha, beta, S0, out, S_final, B, T, H, dk, dv, chunk, cu_seqlens, dtype,
+                         scratch, kScratchBytes, stream);
+}
