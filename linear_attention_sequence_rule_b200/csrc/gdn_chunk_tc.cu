@@ -51,67 +51,73 @@ namespace {
 using namespace sm100;
 
 constexpr int CH = 64;
-constexpr int kThreads = 256;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 constexpr int LDF = 68;  // fp32 row stride of the 64 x 64 solve matrices
-// Thread roles inside the intra warpgroup: its Gram MMA is issued by warp 7 and the gate scan runs
-// on warp 5, away from warp 4, which shares an SM sub-partition with the chain's issuing thread
-// (thread 0).
-constexpr int kIntraIssuer = 96;
 // Kernel flags (used by the segment scan): V is taken as zero (nothing of V is loaded), and the
 // initial state is the identity (dv must equal dk).  With out == nullptr no output is formed.
 constexpr int kFlagVZero = 1;
 constexpr int kFlagS0Identity = 2;
-constexpr int kScanWarp = 1;
 
 template <int DK, int DV>
 struct TcCfg {
+    // Intra warpgroups: two (alternate chunks) where shared memory and TMEM hold two sets of
+    // solve buffers, which is dk = dv = 64; otherwise one.
+    static constexpr int NI = (DK == 64 && DV == 64) ? 2 : 1;
+    static constexpr int THREADS = 128 * (1 + NI);
     static constexpr int NS = (DK == 128 || DV == 128) ? 2 : 3;  // K/Q stages
+    // W^T (DK x 64 bf16) is written over T diag(b gam) once the WY MMAs have read it (dk = 64)
+    static constexpr bool WT_IN_TG = DK == 64;
     // shared memory byte offsets (swizzled tiles first, all 1024-aligned)
     static constexpr int KQ = 0;                                 // per stage: per 64-feature block K (8K) | Q (8K)
     static constexpr int KQ_STAGE = (DK / 64) * 16384;
     static constexpr int V = KQ + NS * KQ_STAGE;                 // per 64-column block 8 KB
-    static constexpr int WT = V + (DV / 64) * 8192;              // W^T bf16, DK rows x 128 B
-    static constexpr int PM = WT + DK * 128;                     // per stage: P bf16, 64 x 128 B
-    static constexpr int TB = PM + NS * 8192;                    // T diag(b)
-    static constexpr int TG = TB + 8192;                         // T diag(b gam)
-    static constexpr int ST = TG + 8192;                         // S^T bf16, per 64-feature block DV x 128 B
+    static constexpr int PM = V + (DV / 64) * 8192;              // per stage: P bf16, 64 x 128 B
+    static constexpr int ST = PM + NS * 8192;                    // S^T bf16, per 64-feature block DV x 128 B
     static constexpr int UT = ST + (DK / 64) * DV * 128;         // U^T bf16, DV x 128 B
-    static constexpr int AF = UT + DV * 128;                     // A fp32 [64][LDF]
-    static constexpr int TF = AF + CH * LDF * 4;                 // T fp32 [64][LDF]
-    static constexpr int XS = TF + CH * LDF * 4;                 // per-warp merge scratch, 4 x 256 fp32
-    static constexpr int GT = XS + 4 * 256 * 4;                  // per stage: gate vectors
+    static constexpr int WG0 = UT + DV * 128;                    // per intra warpgroup:
+    static constexpr int W_TB = 0;                               //   T diag(b)      bf16 64 x 128 B
+    static constexpr int W_TG = 8192;                            //   T diag(b gam)  bf16 64 x 128 B
+    static constexpr int W_WT = WT_IN_TG ? W_TG : 16384;         //   W^T bf16, DK rows x 128 B
+    static constexpr int W_AF = WT_IN_TG ? 16384 : 16384 + DK * 128;  // A fp32 [64][LDF]
+    static constexpr int W_TF = W_AF + CH * LDF * 4;             //   decays, then T fp32 [64][LDF]
+    static constexpr int W_XS = W_TF + CH * LDF * 4;             //   merge scratch, 4 x 256 fp32
+    static constexpr int WG_BYTES = (W_XS + 4 * 256 * 4 + 1023) & ~1023;
+    static constexpr int GT = WG0 + NI * WG_BYTES;               // per stage: gate vectors
     static constexpr int GT_STAGE = 7 * CH * 4;                  //   graw, G2, gam, lam, bet, last, (gC)
     static constexpr int BAR = GT + NS * GT_STAGE;
-    static constexpr int NBAR = 5 * NS + 8;
+    static constexpr int NBAR = 5 * NS + 4 + 3 * NI;
     static constexpr int MISC = BAR + NBAR * 8;                  // TMEM slot, abort flag
     static constexpr int TOTAL = MISC + 16;
     // TMEM columns
     static constexpr uint32_t T_O = 0;                            // DV: output rows (M = 64 tokens)
     static constexpr uint32_t T_S = DV;                           // DK: fp32 state (transposed)
-    static constexpr uint32_t T_G = DV + DK;                      // 64: Gram matrices (intra)
-    static constexpr uint32_t T_W = T_G + 64;                     // 64: W^T (chain)
-    static constexpr uint32_t T_U = T_W + 64;                     // NS x 64: U~^T / U^T
+    static constexpr uint32_t T_G = DV + DK;                      // NI x 64: Gram, then W^T (intra)
+    static constexpr uint32_t T_U = T_G + NI * 64;                // NS x 64: U~^T, then U^T
     static_assert(T_U + NS * 64 <= 512, "TMEM budget");
     static_assert(TOTAL + 1024 <= 232448, "shared memory budget");
 };
 
 // barrier indices
-template <int NS> struct Bars {
-    static constexpr int kq_full = 0;            // [NS]
-    static constexpr int v_full = NS;
-    static constexpr int v_empty = NS + 1;
-    static constexpr int cdone = NS + 2;         // [NS]
-    static constexpr int tready = 2 * NS + 2;    // [NS] intra -> chain: P, T diag(b), T diag(b gam) ready
-    static constexpr int gready = 3 * NS + 2;    // [NS]
-    static constexpr int tfree = 4 * NS + 2;     // chain -> intra: the WY MMAs have read T diag(b..)
-    static constexpr int gram = 4 * NS + 3;
-    static constexpr int uw = 4 * NS + 4;
-    static constexpr int u = 4 * NS + 5;
-    static constexpr int s = 4 * NS + 6;
-    static constexpr int o = 4 * NS + 7;
-    static constexpr int gfull = 4 * NS + 8;     // [NS], 32 arrivals (cp.async of chain warp 0)
+template <int NS, int NI> struct Bars {
+    static constexpr int kq_full = 0;            // [NS] K/Q tiles of a stage landed (TMA)
+    static constexpr int gfull = NS;             // [NS] gates landed, 32 arrivals (cp.async of chain warp 0)
+    static constexpr int gready = 2 * NS;        // [NS] gate vectors (gam, lam, gam_C) computed
+    static constexpr int tready = 3 * NS;        // [NS] intra -> chain: P, U~^T, W^T, gam Q, lam K ready
+    static constexpr int cdone = 4 * NS;         // [NS] chain -> intra: the output MMA has read the stage's P
+    static constexpr int v_full = 5 * NS;
+    static constexpr int u = 5 * NS + 1;
+    static constexpr int s = 5 * NS + 2;
+    static constexpr int o = 5 * NS + 3;
+    static constexpr int gram = 5 * NS + 4;      // [NI] Gram MMA done
+    static constexpr int uw = 5 * NS + 4 + NI;   // [NI] WY MMAs done
+    static constexpr int tfree = 5 * NS + 4 + 2 * NI;  // [NI] chain -> intra: the U MMA has read W^T
 };
+
+// Thread roles inside an intra warpgroup (t = 0..127): the gate scan runs on warp scan_warp(wg)
+// and the MMAs are issued by thread kIssuer, away from SM sub-partition 0, which holds the
+// chain's issuing thread (thread 0).
+__device__ __forceinline__ int scan_warp(int wg) { return wg == 0 ? 1 : 2; }
+constexpr int kIssuer = 96;
 
 struct Ctl {
     uint64_t *bar;
@@ -149,12 +155,13 @@ struct TOut {
     float *Tm;
     unsigned char *TB, *TG;
     const float *bet, *gam;
-    __device__ __forceinline__ void put(int r, int c, float v) const
+    // (bc, gc) = bet/gam of column c, loaded once by the caller
+    __device__ __forceinline__ void put(int r, int c, float v, float bc, float gc) const
     {
         Tm[r * LDF + c] = v;
-        const float b = v * bet[c];
+        const float b = v * bc;
         *reinterpret_cast<__nv_bfloat16 *>(TB + sw128_off(r, c)) = __float2bfloat16_rn(b);
-        *reinterpret_cast<__nv_bfloat16 *>(TG + sw128_off(r, c)) = __float2bfloat16_rn(b * gam[c]);
+        *reinterpret_cast<__nv_bfloat16 *>(TG + sw128_off(r, c)) = __float2bfloat16_rn(b * gc);
     }
     // c even; (b0, b1, g0, g1) = bet/gam of columns c, c+1; keep: also store the fp32 values
     __device__ __forceinline__ void put2(int r, int c, float v0, float v1, float b0, float b1, float g0, float g1,
@@ -178,7 +185,7 @@ __device__ __forceinline__ uint32_t tf(float x) { return __float_as_uint(x); }
 // same step on mma.sync TF32 (T is rounded to bf16 afterwards, so TF32 products stay below that
 // rounding).  Every entry of the lower triangle is written exactly once, through `out`; entries
 // above the diagonal are never written (the caller keeps them zero in the bf16 copies).
-__device__ void solve_unit_lower(const float *A, const TOut &out, float *XS, int t, int bar_id)
+__device__ void solve_unit_lower(const float *__restrict__ A, const TOut &out, float *__restrict__ XS, int t, int bar_id)
 {
     float *Tm = out.Tm;
     const int w = t >> 5, lane = t & 31, g = lane >> 2, tq = lane & 3;
@@ -187,6 +194,7 @@ __device__ void solve_unit_lower(const float *A, const TOut &out, float *XS, int
         const int o = 16 * w;
         if (lane < 16) {
             const int sb = o + 8 * (lane >> 3), c = lane & 7;
+            const float bc = out.bet[sb + c], gc = out.gam[sb + c];
             float p[8], x[8];
 #pragma unroll
             for (int r = 0; r < 8; ++r) p[r] = 0.f;
@@ -198,7 +206,7 @@ __device__ void solve_unit_lower(const float *A, const TOut &out, float *XS, int
             }
 #pragma unroll
             for (int r = 0; r < 8; ++r)
-                if (r >= c) out.put(sb + r, sb + c, x[r]);
+                if (r >= c) out.put(sb + r, sb + c, x[r], bc, gc);
         }
         __syncwarp();
 #pragma unroll
@@ -211,6 +219,7 @@ __device__ void solve_unit_lower(const float *A, const TOut &out, float *XS, int
             xs[i * 8 + j] = acc;
         }
         __syncwarp();
+        const float bj = out.bet[o + (lane & 7)], gj = out.gam[o + (lane & 7)];
 #pragma unroll
         for (int q0 = 0; q0 < 64; q0 += 32) {
             const int q = q0 + lane, i = q >> 3, j = q & 7;
@@ -218,7 +227,7 @@ __device__ void solve_unit_lower(const float *A, const TOut &out, float *XS, int
 #pragma unroll
             for (int k = 0; k < 8; ++k)
                 if (k < i) acc = fmaf(Tm[(o + 8 + i) * LDF + o + 8 + k], xs[k * 8 + j], acc);
-            out.put(o + 8 + i, o + j, -acc);
+            out.put(o + 8 + i, o + j, -acc, bj, gj);
         }
     }
     named_bar(bar_id, 128);
@@ -321,22 +330,21 @@ __device__ __forceinline__ void scale_row_bf16(unsigned char *tile, int row, flo
 }
 
 template <int DK, int DV>
-__global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                const __grid_constant__ CUtensorMap tmV, const float *__restrict__ log_alpha,
-                const float *__restrict__ beta, const float *__restrict__ S0,
-                __nv_bfloat16 *__restrict__ out, float *__restrict__ S_final,
-                const int32_t *__restrict__ cu_seqlens, int T, int H, int flags)
+__global__ void __launch_bounds__(TcCfg<DK, DV>::THREADS, 1)
+    chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                    const __grid_constant__ CUtensorMap tmV, const float *__restrict__ log_alpha,
+                    const float *__restrict__ beta, const float *__restrict__ S0,
+                    __nv_bfloat16 *__restrict__ out, float *__restrict__ S_final,
+                    const int32_t *__restrict__ cu_seqlens, int T, int H, int flags)
 {
     using L = TcCfg<DK, DV>;
     constexpr int NS = L::NS;
-    using B = Bars<NS>;
-    // dk = 64: the chain warpgroup does the WY part of the next chunk in the shadow of its MMAs.
-    // dk = 128: the chain's own epilogues are twice as large, so the intra warpgroup does it.
-    constexpr bool kChainWY = DK == 64;
-    constexpr bool kIntraScalesQ = !kChainWY;
+    constexpr int NI = L::NI;
+    using B = Bars<NS, NI>;
     extern __shared__ unsigned char smem_raw[];
-    unsigned char *sm = reinterpret_cast<unsigned char *>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    // 1024-aligned base by pointer arithmetic on the shared array, so that the compiler keeps
+    // every access below in the shared address space
+    unsigned char *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + L::BAR);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + L::MISC);
     int *abort_flag = reinterpret_cast<int *>(sm + L::MISC + 4);
@@ -356,7 +364,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
     const size_t sbase = ((size_t)s * H + h) * (size_t)DK * DV;
 
     if (tid == 0) {
-        for (int i = 0; i < L::NBAR; ++i) mbar_init(&bars[i], i >= B::gfull ? 32 : 1);
+        for (int i = 0; i < L::NBAR; ++i) mbar_init(&bars[i], (i >= B::gfull && i < B::gfull + NS) ? 32 : 1);
         fence_mbar_init();
         *abort_flag = 0;
     }
@@ -386,7 +394,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
         }
         cp_async_mbar_arrive(&bars[B::gfull + st]);
         if (lane == 0 && !ctl.aborted()) {
-            mbar_arrive_expect_tx(&bars[B::kq_full + st], 2 * (DK / 64) * 8192);
+            mbar_arrive_expect_tx(&bars[B::kq_full + st], (DK / 64) * 16384);
             unsigned char *kq = sm + L::KQ + st * L::KQ_STAGE;
             for (int kb = 0; kb < DK / 64; ++kb) {
                 tma_load_3d(kq + kb * 16384, &tmK, &bars[B::kq_full + st], kb * 64, h, (int)tk);
@@ -396,6 +404,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
     };
     const bool v_zero = (flags & kFlagVZero) != 0;
     const bool want_out = out != nullptr;
+    // V tile of chunk c (single buffer: issued once the previous chunk's U~ MMA has read it)
     auto load_v = [&](int c) {
         if (ctl.aborted() || v_zero) return;
         const int tk = (int)(tok0 + (long)c * CH);
@@ -412,79 +421,32 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
         for (int c = 0; c < min(nchunks, NS); ++c) load_kq(c);
     }
     if (tid == 0 && nchunks > 0) load_v(0);
-        // WY MMAs of chunk c2 (thread 0): U~^T = V^T (T diag b)^T into its U slot, W^T = K^T (T diag(b gam))^T.
-    auto issue_wy = [&](int c2) {
-        if (!v_zero) ctl.wait(B::v_full, c2 & 1);
-        if (ctl.aborted()) return;
-        tc_fence_after();
-        unsigned char *K2 = sm + L::KQ + (c2 % NS) * L::KQ_STAGE;
-        constexpr uint32_t idU = idesc_bf16(DV, 64, 1, 0);
-        constexpr uint32_t idW = idesc_bf16(DK, 64, 1, 0);
-        if (!v_zero) {
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-                mma_bf16(tmem + L::T_U + (c2 % NS) * 64, sdesc_sw128(smem_u32(sm + L::V + kk * 2048), 8192, 1024),
-                         sdesc_sw128(smem_u32(sm + L::TB + kk * 32), 16, 1024), idU, kk > 0);
-        }
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-            mma_bf16(tmem + L::T_W, sdesc_sw128(smem_u32(K2 + kk * 2048), 16384, 1024),
-                     sdesc_sw128(smem_u32(sm + L::TG + kk * 32), 16, 1024), idW, kk > 0);
-        mma_commit(&bars[B::uw]);
-    };
-    // After the WY MMAs of chunk c2, run by a whole warpgroup (u = thread index 0..127 in it,
-    // tlw = its warp's TMEM lane base): the next V load, W^T to shared memory (bf16), the
-    // lam-scaled K tile in place and, unless the intra side did it, the gam-scaled Q tile (the
-    // MMAs that read them unscaled are done).
-    auto finish_wy = [&](int c2, int u, uint32_t tlw) {
-        const int crow = (DK == 128) ? u : ((u & 31) < 16 ? (u >> 5) * 16 + (u & 31) : -1);  // row of W^T
-        ctl.wait(B::uw, c2 & 1);
-        tc_fence_after();
-        if (u == 0) {
-            if (c2 + 1 < nchunks) load_v(c2 + 1);
-            ctl.arrive(B::tfree);
-        }
-        float x[64];
-        tmem_ld32(tlw + L::T_W, *reinterpret_cast<float(*)[32]>(&x[0]));
-        tmem_ld32(tlw + L::T_W + 32, *reinterpret_cast<float(*)[32]>(&x[32]));
-        tmem_wait_ld();
-        if (crow >= 0) st_row_bf16_sw128(sm + L::WT, crow, x);
-        const float *gv = gates(c2 % NS);
-        unsigned char *K2 = sm + L::KQ + (c2 % NS) * L::KQ_STAGE;
-        const int r = u & 63;
-        const float gr = gv[2 * CH + r], lr = gv[3 * CH + r];
-        if (DK == 128) {
-            scale_row_bf16(K2 + (u >> 6) * 16384, r, lr, 0, 8);
-        } else {
-            scale_row_bf16(K2 + 8192, r, gr, (u >> 6) * 4, (u >> 6) * 4 + 4);
-            scale_row_bf16(K2, r, lr, (u >> 6) * 4, (u >> 6) * 4 + 4);
-        }
-        fence_proxy_async_smem();
-        tc_fence_before();
-    };
-
 
     if (warp >= 4) {
-        // ======================= intra warpgroup =======================
-        const int t = tid - 128, wi = t >> 5;
+        // ======================= intra warpgroup(s): chunks wg, wg + NI, ... =======================
+        const int wg = (warp - 4) >> 2;
+        const int t = tid - 128 * (1 + wg), wi = t >> 5;
+        const int bar_id = 2 + wg;
         const uint32_t tl = tmem + ((uint32_t)(wi * 32) << 16);
-        float *AF = reinterpret_cast<float *>(sm + L::AF);
-        float *TFm = reinterpret_cast<float *>(sm + L::TF);
-        float *XSm = reinterpret_cast<float *>(sm + L::XS);
+        const uint32_t tG = L::T_G + wg * 64;  // Gram accumulator, then W^T
+        unsigned char *wsm = sm + L::WG0 + wg * L::WG_BYTES;
+        unsigned char *TBs = wsm + L::W_TB, *TGs = wsm + L::W_TG, *WTs = wsm + L::W_WT;
+        float *AF = reinterpret_cast<float *>(wsm + L::W_AF);
+        float *TFm = reinterpret_cast<float *>(wsm + L::W_TF);
+        float *XSm = reinterpret_cast<float *>(wsm + L::W_XS);
+        // entries above the diagonal of T diag(b..) stay zero (the solve writes the lower part)
         for (int i = t; i < 2 * 8192 / 16; i += 128)
-            reinterpret_cast<uint4 *>(sm + L::TB)[i] = make_uint4(0u, 0u, 0u, 0u);
-        for (int c = 0; c < nchunks; ++c) {
+            reinterpret_cast<uint4 *>(TBs)[i] = make_uint4(0u, 0u, 0u, 0u);
+        for (int c = wg; c < nchunks; c += NI) {
             const int st = c % NS;
-            const long tk = tok0 + (long)c * CH;
-            const int n = (int)min((long)CH, len - (long)c * CH);
+            const int kc = c / NI;  // this warpgroup's chunk count
             float *gv = gates(st);
             float *graw = gv, *Gs = gv + CH, *gam = gv + 2 * CH, *lam = gv + 3 * CH, *bet = gv + 4 * CH;
             int *last = reinterpret_cast<int *>(gv + 5 * CH);
             float *gC = gv + 6 * CH;
             unsigned char *Kt = sm + L::KQ + st * L::KQ_STAGE;  // K at +0, Q at +8192 per block
-            if (c >= NS) ctl.wait(B::cdone + st, ((c / NS) - 1) & 1);
             // ---- gates: segmented scan of log_alpha (restarts at exact resets) ----
-            if (wi == kScanWarp) {
+            if (wi == scan_warp(wg)) {
                 ctl.wait(B::gfull + st, (c / NS) & 1);
                 const int r0 = 2 * lane, r1 = r0 + 1;
                 const float g0 = graw[r0], g1 = graw[r1];
@@ -530,18 +492,18 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
                     ctl.arrive(B::gready + st);
                 }
             }
-            named_bar(2, 128);
+            named_bar(bar_id, 128);
             // ---- Gram matrices [K; Q] K^T ----
             ctl.wait(B::kq_full + st, (c / NS) & 1);
-            if (t == kIntraIssuer && !ctl.aborted()) {
+            if (t == kIssuer && !ctl.aborted()) {
                 tc_fence_after();
                 constexpr uint32_t id = idesc_bf16(128, 64, 0, 0);
 #pragma unroll
                 for (int kk = 0; kk < DK / 16; ++kk) {
                     const uint32_t a = smem_u32(Kt + (kk >> 2) * 16384 + (kk & 3) * 32);
-                    mma_bf16(tmem + L::T_G, sdesc_sw128(a, 16, 1024), sdesc_sw128(a, 16, 1024), id, kk > 0);
+                    mma_bf16(tmem + tG, sdesc_sw128(a, 16, 1024), sdesc_sw128(a, 16, 1024), id, kk > 0);
                 }
-                mma_commit(&bars[B::gram]);
+                mma_commit(&bars[B::gram + wg]);
             }
             // ---- decays Gam[r][i] (lower triangle; zero across a reset) into the T scratch ----
             {
@@ -563,15 +525,17 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
                     *reinterpret_cast<float4 *>(gm + j4) = make_float4(v[0], v[1], v[2], v[3]);
                 }
             }
-            ctl.wait(B::gram, c & 1);
+            ctl.wait(B::gram + wg, kc & 1);
+            // the stage's P tile is free once the output MMA of chunk c - NS has read it
+            if (c >= NS) ctl.wait(B::cdone + st, ((c / NS) - 1) & 1);
             tc_fence_after();
-            named_bar(2, 128);
+            named_bar(bar_id, 128);
             {
-                // A = diag(b) (Gam o K K^T) (fp32; its diagonal and upper part are never read) and
-                // P = Gam o Q K^T (bf16)
+                // A = diag(b) (Gam o K K^T) (fp32; its diagonal and upper part are never read),
+                // P = Gam o Q K^T (bf16), and gam Q in place (no MMA reads Q unscaled any more)
                 float x[64];
-                tmem_ld32(tl + L::T_G, *reinterpret_cast<float(*)[32]>(&x[0]));
-                tmem_ld32(tl + L::T_G + 32, *reinterpret_cast<float(*)[32]>(&x[32]));
+                tmem_ld32(tl + tG, *reinterpret_cast<float(*)[32]>(&x[0]));
+                tmem_ld32(tl + tG + 32, *reinterpret_cast<float(*)[32]>(&x[32]));
                 tmem_wait_ld();
                 const int r = t & 63;
                 const bool isq = t >= 64;
@@ -591,23 +555,71 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
                     for (int i = 0; i < CH; i += 4)
                         *reinterpret_cast<float4 *>(&AF[r * LDF + i]) = make_float4(x[i], x[i + 1], x[i + 2], x[i + 3]);
                 }
-                // with dk = 128 the intra side takes the gam-scaling of Q (no MMA reads Q unscaled
-                // after the Gram MMA); with dk = 64 the chain side does it
-                if (kIntraScalesQ) scale_row_bf16(Kt + (t >> 6) * 16384 + 8192, r, gam[r], 0, 8);
+                if (DK == 128)
+                    scale_row_bf16(Kt + (t >> 6) * 16384 + 8192, r, gam[r], 0, 8);
+                else
+                    scale_row_bf16(Kt + 8192, r, gam[r], (t >> 6) * 4, (t >> 6) * 4 + 4);
             }
             tc_fence_before();
-            // the WY MMAs of the previous chunk must have read T diag(b), T diag(b gam)
-            if (c >= 1) ctl.wait(B::tfree, (c - 1) & 1);
-            named_bar(2, 128);
-            // ---- T = (I + A)^{-1}, written with the bf16 rows of T diag(b), T diag(b gam) ----
-            solve_unit_lower(AF, TOut{TFm, sm + L::TB, sm + L::TG, bet, gam}, XSm, t, 2);
-            fence_proxy_async_smem();
-            named_bar(2, 128);
-            if (!kChainWY) {
-                if (t == kIntraIssuer) issue_wy(c);
-                finish_wy(c, t, tl);
-                named_bar(2, 128);
+            // this warpgroup's previous chunk: its W^T and T diag(b..) tiles must have been read
+            if (kc >= 1) ctl.wait(B::tfree + wg, (kc - 1) & 1);
+            if (L::WT_IN_TG) {
+                // W^T of the previous chunk sits in the T diag(b gam) tile: clear every 16-byte
+                // chunk from the diagonal block rightwards (the solve then writes the lower part)
+                for (int i = t; i < 64 * 8; i += 128) {
+                    const int r = i >> 3, cb = i & 7;
+                    if (cb >= (r >> 3))
+                        *reinterpret_cast<uint4 *>(TGs + r * 128 + ((cb ^ (r & 7)) << 4)) = make_uint4(0u, 0u, 0u, 0u);
+                }
             }
+            named_bar(bar_id, 128);
+            // ---- T = (I + A)^{-1}, written with the bf16 rows of T diag(b), T diag(b gam) ----
+            solve_unit_lower(AF, TOut{TFm, TBs, TGs, bet, gam}, XSm, t, bar_id);
+            fence_proxy_async_smem();
+            tc_fence_before();
+            named_bar(bar_id, 128);
+            // ---- WY products: U~^T = V^T (T diag b)^T into the stage's U slot and
+            //      W^T = K^T (T diag(b gam))^T over the Gram accumulator ----
+            if (t == kIssuer) {
+                if (!v_zero) ctl.wait(B::v_full, c & 1);
+                if (!ctl.aborted()) {
+                    tc_fence_after();
+                    constexpr uint32_t idU = idesc_bf16(DV, 64, 1, 0);
+                    constexpr uint32_t idW = idesc_bf16(DK, 64, 1, 0);
+                    if (!v_zero) {
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk)
+                            mma_bf16(tmem + L::T_U + st * 64, sdesc_sw128(smem_u32(sm + L::V + kk * 2048), 8192, 1024),
+                                     sdesc_sw128(smem_u32(TBs + kk * 32), 16, 1024), idU, kk > 0);
+                    }
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_bf16(tmem + tG, sdesc_sw128(smem_u32(Kt + kk * 2048), 16384, 1024),
+                                 sdesc_sw128(smem_u32(TGs + kk * 32), 16, 1024), idW, kk > 0);
+                    mma_commit(&bars[B::uw + wg]);
+                }
+            }
+            ctl.wait(B::uw + wg, kc & 1);
+            tc_fence_after();
+            if (t == kIssuer && c + 1 < nchunks) load_v(c + 1);  // the U~ MMA has read V
+            {
+                // W^T rows (one per feature) to shared memory in bf16, then lam K in place (the
+                // W MMA has read K unscaled)
+                const int crow = (DK == 128) ? t : ((t & 31) < 16 ? (t >> 5) * 16 + (t & 31) : -1);
+                float x[64];
+                tmem_ld32(tl + tG, *reinterpret_cast<float(*)[32]>(&x[0]));
+                tmem_ld32(tl + tG + 32, *reinterpret_cast<float(*)[32]>(&x[32]));
+                tmem_wait_ld();
+                if (crow >= 0) st_row_bf16_sw128(WTs, crow, x);
+                const int r = t & 63;
+                if (DK == 128)
+                    scale_row_bf16(Kt + (t >> 6) * 16384, r, lam[r], 0, 8);
+                else
+                    scale_row_bf16(Kt, r, lam[r], (t >> 6) * 4, (t >> 6) * 4 + 4);
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            named_bar(bar_id, 128);
             if (t == 0) ctl.arrive(B::tready + st);
         }
     } else {
@@ -628,40 +640,41 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
                 *reinterpret_cast<uint4 *>(stt + j * 128 + (((chunk ^ (j & 7)) & 7) << 4)) = w;
             }
         };
-        // Output rows: O (M = 64 tokens, N = DV) sits in lanes 0..15 of each warp, row 16w + lane.
+        // Output rows of chunk c: O (M = 64 tokens, N = DV) sits in lanes 0..15 of each warp,
+        // row 16w + lane.  The chunk's P tile is released to the intra side as soon as the
+        // output MMA has completed.
         auto out_epilogue = [&](int c) {
             const long tk = tok0 + (long)c * CH;
             const int n = (int)min((long)CH, len - (long)c * CH);
-            if (!want_out) {
-                named_bar(1, 128);
+            if (want_out) {
+                ctl.wait(B::o, c & 1);
+                tc_fence_after();
                 if (tid == 0) ctl.arrive(B::cdone + (c % NS));
-                return;
-            }
-            ctl.wait(B::o, c & 1);
-            tc_fence_after();
-            const int r = 16 * warp + (lane & 15);
-            __nv_bfloat16 *op = out + ((size_t)(tk + r) * H + h) * DV;
+                const int r = 16 * warp + (lane & 15);
+                __nv_bfloat16 *op = out + ((size_t)(tk + r) * H + h) * DV;
 #pragma unroll 1
-            for (int cb = 0; cb < DV / 32; ++cb) {
-                float o[32];
-                tmem_ld32(tl + L::T_O + cb * 32, o);
-                tmem_wait_ld();
-                if (lane < 16 && r < n) {
-                    uint4 *dst = reinterpret_cast<uint4 *>(op + cb * 32);
+                for (int cb = 0; cb < DV / 32; ++cb) {
+                    float o[32];
+                    tmem_ld32(tl + L::T_O + cb * 32, o);
+                    tmem_wait_ld();
+                    if (lane < 16 && r < n) {
+                        uint4 *dst = reinterpret_cast<uint4 *>(op + cb * 32);
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        uint4 w;
-                        w.x = pack_bf16x2(o[8 * q + 0], o[8 * q + 1]);
-                        w.y = pack_bf16x2(o[8 * q + 2], o[8 * q + 3]);
-                        w.z = pack_bf16x2(o[8 * q + 4], o[8 * q + 5]);
-                        w.w = pack_bf16x2(o[8 * q + 6], o[8 * q + 7]);
-                        dst[q] = w;
+                        for (int q = 0; q < 4; ++q) {
+                            uint4 w;
+                            w.x = pack_bf16x2(o[8 * q + 0], o[8 * q + 1]);
+                            w.y = pack_bf16x2(o[8 * q + 2], o[8 * q + 3]);
+                            w.z = pack_bf16x2(o[8 * q + 4], o[8 * q + 5]);
+                            w.w = pack_bf16x2(o[8 * q + 6], o[8 * q + 7]);
+                            dst[q] = w;
+                        }
                     }
                 }
+                tc_fence_before();
+            } else if (tid == 0) {
+                ctl.arrive(B::cdone + (c % NS));
             }
-            tc_fence_before();
             named_bar(1, 128);
-            if (tid == 0) ctl.arrive(B::cdone + (c % NS));
         };
         if (nchunks > 0) {
             // initial state: S^T row j (fp32, pre-scaled by gam_C of chunk 0) and its bf16 copy
@@ -680,13 +693,6 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
                 tmem_st32(tl + L::T_S + cb * 32, x);
             }
             tmem_wait_st();
-            if (kChainWY) {
-                if (tid == 0) {
-                    ctl.wait(B::tready + 0, 0);
-                    issue_wy(0);
-                }
-                finish_wy(0, tid, tl);
-            }
             fence_proxy_async_smem();
             tc_fence_before();
             named_bar(1, 128);
@@ -695,25 +701,28 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
             const int st = c % NS;
             const uint32_t tO = tmem + L::T_O;
             unsigned char *Kt = sm + L::KQ + st * L::KQ_STAGE;
-            const bool has_next = c + 1 < nchunks;
-            const bool wy_chain = kChainWY && has_next;  // this warpgroup does the WY part of c+1
-            bool wy_next = false;  // thread 0: WY MMAs of chunk c+1 already issued
-            if (!kChainWY) ctl.wait(B::tready + st, (c / NS) & 1);
+            const unsigned char *WTc = sm + L::WG0 + (c % NI) * L::WG_BYTES + L::W_WT;
+            ctl.wait(B::tready + st, (c / NS) & 1);
             if (tid == 0 && !ctl.aborted()) {
+                // U^T = U~^T - S^T W^T, accumulated onto U~^T (A operand negated)
                 tc_fence_after();
                 constexpr uint32_t idN = idesc_bf16(DV, 64, 0, 1, 1);
-                constexpr uint32_t idQ = idesc_bf16(64, DV, 0, 0);
 #pragma unroll
                 for (int kk = 0; kk < DK / 16; ++kk) {
                     const uint64_t a = sdesc_sw128(smem_u32(sm + L::ST + (kk >> 2) * (DV * 128) + (kk & 3) * 32), 16, 1024);
-                    mma_bf16(tmem + L::T_U + st * 64, a, sdesc_sw128(smem_u32(sm + L::WT + kk * 2048), 16, 1024), idN,
+                    mma_bf16(tmem + L::T_U + st * 64, a, sdesc_sw128(smem_u32(WTc + kk * 2048), 16, 1024), idN,
                              v_zero ? (kk > 0) : 1);
                 }
                 mma_commit(&bars[B::u]);
+            }
+            // the previous chunk's outputs leave while the U MMA runs; then O = (gam Q) S
+            if (c >= 1) out_epilogue(c - 1);
+            if (tid == 0 && want_out && !ctl.aborted()) {
+                tc_fence_after();
+                constexpr uint32_t idQ = idesc_bf16(64, DV, 0, 0);
 #pragma unroll
                 for (int kk = 0; kk < DK / 16; ++kk) {
-                    if (!want_out) break;
-                    // O = (gam Q) S: A = gam-scaled Q tile (K-major), B = S^T rows (K-major)
+                    // A = gam-scaled Q tile (K-major), B = S^T rows (K-major)
                     const uint32_t a = smem_u32(Kt + (kk >> 2) * 16384 + 8192 + (kk & 3) * 32);
                     const uint64_t b = sdesc_sw128(smem_u32(sm + L::ST + (kk >> 2) * (DV * 128) + (kk & 3) * 32), 16, 1024);
                     mma_bf16(tO, sdesc_sw128(a, 16, 1024), b, idQ, kk > 0);
@@ -721,6 +730,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
             }
             ctl.wait(B::u, c & 1);
             tc_fence_after();
+            if (tid == 0) ctl.arrive(B::tfree + (c % NI));  // W^T of this chunk has been read
             {
                 float x[64];
                 tmem_ld32(tl + L::T_U + st * 64, *reinterpret_cast<float(*)[32]>(&x[0]));
@@ -736,16 +746,10 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
                 constexpr uint32_t idS = idesc_bf16(DV, DK, 0, 1);
                 constexpr uint32_t idP = idesc_bf16(64, DV, 0, 0);
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
+                for (int kk = 0; kk < 4; ++kk)  // S^T += U^T (lam K)
                     mma_bf16(tmem + L::T_S, sdesc_sw128(smem_u32(sm + L::UT + kk * 32), 16, 1024),
                              sdesc_sw128(smem_u32(Kt + kk * 2048), 16384, 1024), idS, 1);
                 mma_commit(&bars[B::s]);
-                // The tensor pipe runs a CTA's MMAs in issue order: the WY MMAs of chunk c+1 go
-                // behind the state increment, and only if the intra side is already done with it.
-                if (wy_chain && mbar_test_wait(&bars[B::tready + (c + 1) % NS], ((c + 1) / NS) & 1)) {
-                    issue_wy(c + 1);
-                    wy_next = true;
-                }
                 if (want_out) {
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)  // O += P U: A = P rows (K-major), B = U^T rows (K-major)
@@ -782,16 +786,9 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(const __grid_cons
             }
             fence_proxy_async_smem();
             tc_fence_before();
-            if (wy_chain) {
-                if (tid == 0 && !wy_next) {
-                    ctl.wait(B::tready + (c + 1) % NS, ((c + 1) / NS) & 1);
-                    issue_wy(c + 1);
-                }
-                finish_wy(c + 1, tid, tl);
-            }
             named_bar(1, 128);
-            out_epilogue(c);
         }
+        if (nchunks > 0) out_epilogue(nchunks - 1);
         // final state
         if (S_final) {
             if (nchunks > 0) {
@@ -885,7 +882,7 @@ cudaError_t launch_tc(const TcLaunch &a, cudaStream_t st)
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     const dim3 grid(1, a.H, a.nseq);
-    kern<<<grid, kThreads, smem, st>>>(mq, mk, mv, a.log_alpha, a.beta, a.S0,
+    kern<<<grid, L::THREADS, smem, st>>>(mq, mk, mv, a.log_alpha, a.beta, a.S0,
                                        static_cast<__nv_bfloat16 *>(a.out), a.S_final, a.cu, a.T, a.H,
                                        a.flags);
     return cudaGetLastError();
