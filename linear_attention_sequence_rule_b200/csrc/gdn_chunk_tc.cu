@@ -65,15 +65,20 @@ struct TcCfg {
     static constexpr int NI = (DK == 64 && DV == 64) ? 2 : 1;
     static constexpr int THREADS = 128 * (1 + NI);
     static constexpr int NS = (DK == 128 || DV == 128) ? 2 : 3;  // K/Q stages
+    // buffers of V, of the bf16 S^T copy and of O: two with two intra warpgroups (the V load of a
+    // chunk then starts two chunks ahead, and the output epilogue overlaps the next state MMA)
+    static constexpr int NB = NI;
     // W^T (DK x 64 bf16) is written over T diag(b gam) once the WY MMAs have read it (dk = 64)
     static constexpr bool WT_IN_TG = DK == 64;
     // shared memory byte offsets (swizzled tiles first, all 1024-aligned)
     static constexpr int KQ = 0;                                 // per stage: per 64-feature block K (8K) | Q (8K)
     static constexpr int KQ_STAGE = (DK / 64) * 16384;
-    static constexpr int V = KQ + NS * KQ_STAGE;                 // per 64-column block 8 KB
-    static constexpr int PM = V + (DV / 64) * 8192;              // per stage: P bf16, 64 x 128 B
-    static constexpr int ST = PM + NS * 8192;                    // S^T bf16, per 64-feature block DV x 128 B
-    static constexpr int UT = ST + (DK / 64) * DV * 128;         // U^T bf16, DV x 128 B
+    static constexpr int V = KQ + NS * KQ_STAGE;                 // per buffer: per 64-column block 8 KB
+    static constexpr int V_BUF = (DV / 64) * 8192;
+    static constexpr int PM = V + NB * V_BUF;                    // per stage: P bf16, 64 x 128 B
+    static constexpr int ST = PM + NS * 8192;                    // per buffer: S^T bf16, per 64-feature block DV x 128 B
+    static constexpr int ST_BUF = (DK / 64) * DV * 128;
+    static constexpr int UT = ST + NB * ST_BUF;                  // U^T bf16, DV x 128 B
     static constexpr int WG0 = UT + DV * 128;                    // per intra warpgroup:
     static constexpr int W_TB = 0;                               //   T diag(b)      bf16 64 x 128 B
     static constexpr int W_TG = 8192;                            //   T diag(b gam)  bf16 64 x 128 B
@@ -85,32 +90,32 @@ struct TcCfg {
     static constexpr int GT = WG0 + NI * WG_BYTES;               // per stage: gate vectors
     static constexpr int GT_STAGE = 7 * CH * 4;                  //   graw, G2, gam, lam, bet, last, (gC)
     static constexpr int BAR = GT + NS * GT_STAGE;
-    static constexpr int NBAR = 5 * NS + 4 + 3 * NI;
+    static constexpr int NBAR = 5 * NS + 2 * NB + 2 + 3 * NI;
     static constexpr int MISC = BAR + NBAR * 8;                  // TMEM slot, abort flag
     static constexpr int TOTAL = MISC + 16;
     // TMEM columns
-    static constexpr uint32_t T_O = 0;                            // DV: output rows (M = 64 tokens)
-    static constexpr uint32_t T_S = DV;                           // DK: fp32 state (transposed)
-    static constexpr uint32_t T_G = DV + DK;                      // NI x 64: Gram, then W^T (intra)
+    static constexpr uint32_t T_O = 0;                            // NB x DV: output rows (M = 64 tokens)
+    static constexpr uint32_t T_S = NB * DV;                      // DK: fp32 state (transposed)
+    static constexpr uint32_t T_G = T_S + DK;                     // NI x 64: Gram, then W^T (intra)
     static constexpr uint32_t T_U = T_G + NI * 64;                // NS x 64: U~^T, then U^T
     static_assert(T_U + NS * 64 <= 512, "TMEM budget");
     static_assert(TOTAL + 1024 <= 232448, "shared memory budget");
 };
 
 // barrier indices
-template <int NS, int NI> struct Bars {
+template <int NS, int NI, int NB> struct Bars {
     static constexpr int kq_full = 0;            // [NS] K/Q tiles of a stage landed (TMA)
     static constexpr int gfull = NS;             // [NS] gates landed, 32 arrivals (cp.async of chain warp 0)
     static constexpr int gready = 2 * NS;        // [NS] gate vectors (gam, lam, gam_C) computed
     static constexpr int tready = 3 * NS;        // [NS] intra -> chain: P, U~^T, W^T, gam Q, lam K ready
     static constexpr int cdone = 4 * NS;         // [NS] chain -> intra: the output MMA has read the stage's P
-    static constexpr int v_full = 5 * NS;
-    static constexpr int u = 5 * NS + 1;
-    static constexpr int s = 5 * NS + 2;
-    static constexpr int o = 5 * NS + 3;
-    static constexpr int gram = 5 * NS + 4;      // [NI] Gram MMA done
-    static constexpr int uw = 5 * NS + 4 + NI;   // [NI] WY MMAs done
-    static constexpr int tfree = 5 * NS + 4 + 2 * NI;  // [NI] chain -> intra: the U MMA has read W^T
+    static constexpr int v_full = 5 * NS;        // [NB] V tile landed
+    static constexpr int u = 5 * NS + NB;
+    static constexpr int s = 5 * NS + NB + 1;
+    static constexpr int o = 5 * NS + NB + 2;    // [NB] output MMAs of a chunk done
+    static constexpr int gram = 5 * NS + 2 * NB + 2;   // [NI] Gram MMA done
+    static constexpr int uw = gram + NI;               // [NI] WY MMAs done
+    static constexpr int tfree = uw + NI;              // [NI] chain -> intra: the U MMA has read W^T
 };
 
 // Thread roles inside an intra warpgroup (t = 0..127): the gate scan runs on warp scan_warp(wg)
@@ -340,7 +345,8 @@ __global__ void __launch_bounds__(TcCfg<DK, DV>::THREADS, 1)
     using L = TcCfg<DK, DV>;
     constexpr int NS = L::NS;
     constexpr int NI = L::NI;
-    using B = Bars<NS, NI>;
+    constexpr int NB = L::NB;
+    using B = Bars<NS, NI, NB>;
     extern __shared__ unsigned char smem_raw[];
     // 1024-aligned base by pointer arithmetic on the shared array, so that the compiler keeps
     // every access below in the shared address space
@@ -404,13 +410,14 @@ __global__ void __launch_bounds__(TcCfg<DK, DV>::THREADS, 1)
     };
     const bool v_zero = (flags & kFlagVZero) != 0;
     const bool want_out = out != nullptr;
-    // V tile of chunk c (single buffer: issued once the previous chunk's U~ MMA has read it)
+    // V tile of chunk c into buffer c % NB (issued once the U~ MMA of chunk c - NB has read it)
     auto load_v = [&](int c) {
         if (ctl.aborted() || v_zero) return;
         const int tk = (int)(tok0 + (long)c * CH);
-        mbar_arrive_expect_tx(&bars[B::v_full], (DV / 64) * 8192);
+        uint64_t *vb_bar = &bars[B::v_full + c % NB];
+        mbar_arrive_expect_tx(vb_bar, L::V_BUF);
         for (int vb = 0; vb < DV / 64; ++vb)
-            tma_load_3d(sm + L::V + vb * 8192, &tmV, &bars[B::v_full], vb * 64, h, tk);
+            tma_load_3d(sm + L::V + (c % NB) * L::V_BUF + vb * 8192, &tmV, vb_bar, vb * 64, h, tk);
     };
     if (warp == 0) {
         if (lane == 0) {
@@ -420,7 +427,8 @@ __global__ void __launch_bounds__(TcCfg<DK, DV>::THREADS, 1)
         }
         for (int c = 0; c < min(nchunks, NS); ++c) load_kq(c);
     }
-    if (tid == 0 && nchunks > 0) load_v(0);
+    if (tid == 0)
+        for (int c = 0; c < min(nchunks, NB); ++c) load_v(c);
 
     if (warp >= 4) {
         // ======================= intra warpgroup(s): chunks wg, wg + NI, ... =======================
@@ -581,7 +589,7 @@ __global__ void __launch_bounds__(TcCfg<DK, DV>::THREADS, 1)
             // ---- WY products: U~^T = V^T (T diag b)^T into the stage's U slot and
             //      W^T = K^T (T diag(b gam))^T over the Gram accumulator ----
             if (t == kIssuer) {
-                if (!v_zero) ctl.wait(B::v_full, c & 1);
+                if (!v_zero) ctl.wait(B::v_full + c % NB, (c / NB) & 1);
                 if (!ctl.aborted()) {
                     tc_fence_after();
                     constexpr uint32_t idU = idesc_bf16(DV, 64, 1, 0);
@@ -589,7 +597,8 @@ __global__ void __launch_bounds__(TcCfg<DK, DV>::THREADS, 1)
                     if (!v_zero) {
 #pragma unroll
                         for (int kk = 0; kk < 4; ++kk)
-                            mma_bf16(tmem + L::T_U + st * 64, sdesc_sw128(smem_u32(sm + L::V + kk * 2048), 8192, 1024),
+                            mma_bf16(tmem + L::T_U + st * 64,
+                                     sdesc_sw128(smem_u32(sm + L::V + (c % NB) * L::V_BUF + kk * 2048), 8192, 1024),
                                      sdesc_sw128(smem_u32(TBs + kk * 32), 16, 1024), idU, kk > 0);
                     }
 #pragma unroll
@@ -601,7 +610,7 @@ __global__ void __launch_bounds__(TcCfg<DK, DV>::THREADS, 1)
             }
             ctl.wait(B::uw + wg, kc & 1);
             tc_fence_after();
-            if (t == kIssuer && c + 1 < nchunks) load_v(c + 1);  // the U~ MMA has read V
+            if (t == kIssuer && c + NB < nchunks) load_v(c + NB);  // the U~ MMA has read V
             {
                 // W^T rows (one per feature) to shared memory in bf16, then lam K in place (the
                 // W MMA has read K unscaled)
@@ -626,9 +635,10 @@ __global__ void __launch_bounds__(TcCfg<DK, DV>::THREADS, 1)
         // ======================= chain warpgroup =======================
         const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);
         const int j = (DV == 128) ? tid : (lane < 16 ? warp * 16 + lane : -1);  // value column
-        auto store_state_bf16 = [&](int cb, const float (&x)[32]) {
+        // bf16 copy of S^T row j, features 32cb .. 32cb+31, into S^T buffer b
+        auto store_state_bf16 = [&](int b, int cb, const float (&x)[32]) {
             if (j < 0) return;
-            unsigned char *stt = sm + L::ST + (cb >> 1) * (DV * 128);
+            unsigned char *stt = sm + L::ST + b * L::ST_BUF + (cb >> 1) * (DV * 128);
 #pragma unroll
             for (int cc = 0; cc < 4; ++cc) {
                 const int chunk = (cb & 1) * 4 + cc;
@@ -647,7 +657,7 @@ __global__ void __launch_bounds__(TcCfg<DK, DV>::THREADS, 1)
             const long tk = tok0 + (long)c * CH;
             const int n = (int)min((long)CH, len - (long)c * CH);
             if (want_out) {
-                ctl.wait(B::o, c & 1);
+                ctl.wait(B::o + c % NB, (c / NB) & 1);
                 tc_fence_after();
                 if (tid == 0) ctl.arrive(B::cdone + (c % NS));
                 const int r = 16 * warp + (lane & 15);
@@ -655,7 +665,7 @@ __global__ void __launch_bounds__(TcCfg<DK, DV>::THREADS, 1)
 #pragma unroll 1
                 for (int cb = 0; cb < DV / 32; ++cb) {
                     float o[32];
-                    tmem_ld32(tl + L::T_O + cb * 32, o);
+                    tmem_ld32(tl + L::T_O + (c % NB) * DV + cb * 32, o);
                     tmem_wait_ld();
                     if (lane < 16 && r < n) {
                         uint4 *dst = reinterpret_cast<uint4 *>(op + cb * 32);
@@ -687,7 +697,7 @@ __global__ void __launch_bounds__(TcCfg<DK, DV>::THREADS, 1)
                 for (int i = 0; i < 32; ++i)
                     x[i] = (flags & kFlagS0Identity) ? ((cb * 32 + i == j) ? 1.f : 0.f)
                                                      : ((j >= 0 && S0) ? S0[sbase + (size_t)(cb * 32 + i) * DV + j] : 0.f);
-                store_state_bf16(cb, x);
+                store_state_bf16(0, cb, x);
 #pragma unroll
                 for (int i = 0; i < 32; ++i) x[i] *= g0;
                 tmem_st32(tl + L::T_S + cb * 32, x);
@@ -699,9 +709,20 @@ __global__ void __launch_bounds__(TcCfg<DK, DV>::THREADS, 1)
         }
         for (int c = 0; c < nchunks; ++c) {
             const int st = c % NS;
-            const uint32_t tO = tmem + L::T_O;
+            const uint32_t tO = tmem + L::T_O + (c % NB) * DV;
+            const uint32_t stc = smem_u32(sm + L::ST + (c % NB) * L::ST_BUF);  // S_c^T, bf16
             unsigned char *Kt = sm + L::KQ + st * L::KQ_STAGE;
             const unsigned char *WTc = sm + L::WG0 + (c % NI) * L::WG_BYTES + L::W_WT;
+            // O = (gam Q) S: A = gam-scaled Q tile (K-major), B = S^T rows (K-major)
+            auto issue_o1 = [&]() {
+                constexpr uint32_t idQ = idesc_bf16(64, DV, 0, 0);
+#pragma unroll
+                for (int kk = 0; kk < DK / 16; ++kk) {
+                    const uint32_t a = smem_u32(Kt + (kk >> 2) * 16384 + 8192 + (kk & 3) * 32);
+                    mma_bf16(tO, sdesc_sw128(a, 16, 1024), sdesc_sw128(stc + (kk >> 2) * (DV * 128) + (kk & 3) * 32, 16, 1024),
+                             idQ, kk > 0);
+                }
+            };
             ctl.wait(B::tready + st, (c / NS) & 1);
             if (tid == 0 && !ctl.aborted()) {
                 // U^T = U~^T - S^T W^T, accumulated onto U~^T (A operand negated)
@@ -709,24 +730,19 @@ __global__ void __launch_bounds__(TcCfg<DK, DV>::THREADS, 1)
                 constexpr uint32_t idN = idesc_bf16(DV, 64, 0, 1, 1);
 #pragma unroll
                 for (int kk = 0; kk < DK / 16; ++kk) {
-                    const uint64_t a = sdesc_sw128(smem_u32(sm + L::ST + (kk >> 2) * (DV * 128) + (kk & 3) * 32), 16, 1024);
+                    const uint64_t a = sdesc_sw128(stc + (kk >> 2) * (DV * 128) + (kk & 3) * 32, 16, 1024);
                     mma_bf16(tmem + L::T_U + st * 64, a, sdesc_sw128(smem_u32(WTc + kk * 2048), 16, 1024), idN,
                              v_zero ? (kk > 0) : 1);
                 }
                 mma_commit(&bars[B::u]);
             }
-            // the previous chunk's outputs leave while the U MMA runs; then O = (gam Q) S
-            if (c >= 1) out_epilogue(c - 1);
+            // O1 goes before the state MMA's commit, so that its completion also covers O1's reads
+            // of the Q tile (reloaded right after) and of the S_c copy.  One O buffer: the previous
+            // chunk's outputs leave first, while the U MMA runs.
+            if (NB == 1 && c >= 1) out_epilogue(c - 1);
             if (tid == 0 && want_out && !ctl.aborted()) {
                 tc_fence_after();
-                constexpr uint32_t idQ = idesc_bf16(64, DV, 0, 0);
-#pragma unroll
-                for (int kk = 0; kk < DK / 16; ++kk) {
-                    // A = gam-scaled Q tile (K-major), B = S^T rows (K-major)
-                    const uint32_t a = smem_u32(Kt + (kk >> 2) * 16384 + 8192 + (kk & 3) * 32);
-                    const uint64_t b = sdesc_sw128(smem_u32(sm + L::ST + (kk >> 2) * (DV * 128) + (kk & 3) * 32), 16, 1024);
-                    mma_bf16(tO, sdesc_sw128(a, 16, 1024), b, idQ, kk > 0);
-                }
+                issue_o1();
             }
             ctl.wait(B::u, c & 1);
             tc_fence_after();
@@ -755,15 +771,17 @@ __global__ void __launch_bounds__(TcCfg<DK, DV>::THREADS, 1)
                     for (int kk = 0; kk < 4; ++kk)  // O += P U: A = P rows (K-major), B = U^T rows (K-major)
                         mma_bf16(tO, sdesc_sw128(smem_u32(sm + L::PM + st * 8192 + kk * 32), 16, 1024),
                                  sdesc_sw128(smem_u32(sm + L::UT + kk * 32), 16, 1024), idP, 1);
-                    mma_commit(&bars[B::o]);
+                    mma_commit(&bars[B::o + c % NB]);
                 }
             }
+            // two O buffers: the previous chunk's outputs leave while the state MMA runs
+            if (NB == 2 && c >= 1) out_epilogue(c - 1);
             ctl.wait(B::s, c & 1);
             tc_fence_after();
             if (warp == 0 && c + NS < nchunks) load_kq(c + NS);
             {
-                // S_{c+1} = gam_C(c) S_c + increment is in TMEM; keep a bf16 copy and pre-scale the
-                // fp32 state by gam_C of the next chunk
+                // S_{c+1} = gam_C(c) S_c + increment is in TMEM; keep a bf16 copy (buffer (c+1) % NB)
+                // and pre-scale the fp32 state by gam_C of the next chunk
                 const bool more = c + 1 < nchunks;
                 float gn = 1.f;
                 if (more) {
@@ -775,7 +793,7 @@ __global__ void __launch_bounds__(TcCfg<DK, DV>::THREADS, 1)
                     float x[32];
                     tmem_ld32(tl + L::T_S + cb * 32, x);
                     tmem_wait_ld();
-                    store_state_bf16(cb, x);
+                    store_state_bf16((c + 1) % NB, cb, x);
                     if (more) {
 #pragma unroll
                         for (int i = 0; i < 32; ++i) x[i] *= gn;
