@@ -453,6 +453,19 @@ __global__ void __launch_bounds__(TcCfg<DK, DV>::THREADS, 1)
             int *last = reinterpret_cast<int *>(gv + 5 * CH);
             float *gC = gv + 6 * CH;
             unsigned char *Kt = sm + L::KQ + st * L::KQ_STAGE;  // K at +0, Q at +8192 per block
+            // ---- Gram matrices [K; Q] K^T (issued first: they need no gates, so the scan below
+            //      runs while they are in flight) ----
+            ctl.wait(B::kq_full + st, (c / NS) & 1);
+            if (t == kIssuer && !ctl.aborted()) {
+                tc_fence_after();
+                constexpr uint32_t id = idesc_bf16(128, 64, 0, 0);
+#pragma unroll
+                for (int kk = 0; kk < DK / 16; ++kk) {
+                    const uint32_t a = smem_u32(Kt + (kk >> 2) * 16384 + (kk & 3) * 32);
+                    mma_bf16(tmem + tG, sdesc_sw128(a, 16, 1024), sdesc_sw128(a, 16, 1024), id, kk > 0);
+                }
+                mma_commit(&bars[B::gram + wg]);
+            }
             // ---- gates: segmented scan of log_alpha (restarts at exact resets) ----
             if (wi == scan_warp(wg)) {
                 ctl.wait(B::gfull + st, (c / NS) & 1);
@@ -501,18 +514,6 @@ __global__ void __launch_bounds__(TcCfg<DK, DV>::THREADS, 1)
                 }
             }
             named_bar(bar_id, 128);
-            // ---- Gram matrices [K; Q] K^T ----
-            ctl.wait(B::kq_full + st, (c / NS) & 1);
-            if (t == kIssuer && !ctl.aborted()) {
-                tc_fence_after();
-                constexpr uint32_t id = idesc_bf16(128, 64, 0, 0);
-#pragma unroll
-                for (int kk = 0; kk < DK / 16; ++kk) {
-                    const uint32_t a = smem_u32(Kt + (kk >> 2) * 16384 + (kk & 3) * 32);
-                    mma_bf16(tmem + tG, sdesc_sw128(a, 16, 1024), sdesc_sw128(a, 16, 1024), id, kk > 0);
-                }
-                mma_commit(&bars[B::gram + wg]);
-            }
             // ---- decays Gam[r][i] (lower triangle; zero across a reset) into the T scratch ----
             {
                 const int r = t & 63, c0 = (t >> 6) * 32;
@@ -614,12 +615,19 @@ __global__ void __launch_bounds__(TcCfg<DK, DV>::THREADS, 1)
             {
                 // W^T rows (one per feature) to shared memory in bf16, then lam K in place (the
                 // W MMA has read K unscaled)
-                const int crow = (DK == 128) ? t : ((t & 31) < 16 ? (t >> 5) * 16 + (t & 31) : -1);
-                float x[64];
-                tmem_ld32(tl + tG, *reinterpret_cast<float(*)[32]>(&x[0]));
-                tmem_ld32(tl + tG + 32, *reinterpret_cast<float(*)[32]>(&x[32]));
-                tmem_wait_ld();
-                if (crow >= 0) st_row_bf16_sw128(WTs, crow, x);
+                if (DK == 128) {
+                    float x[64];
+                    tmem_ld32(tl + tG, *reinterpret_cast<float(*)[32]>(&x[0]));
+                    tmem_ld32(tl + tG + 32, *reinterpret_cast<float(*)[32]>(&x[32]));
+                    tmem_wait_ld();
+                    st_row_bf16_sw128(WTs, t, x);
+                } else {
+                    // M = 64 layout: threads lane and lane + 16 take the two halves of a row
+                    float x[32];
+                    tmem_ld16x2_32<32>(tl + tG, x);
+                    tmem_wait_ld();
+                    st_half_row_bf16_sw128(WTs, wi * 16 + (t & 15), (t >> 4) & 1, x);
+                }
                 const int r = t & 63;
                 if (DK == 128)
                     scale_row_bf16(Kt + (t >> 6) * 16384, r, lam[r], 0, 8);
@@ -634,10 +642,25 @@ __global__ void __launch_bounds__(TcCfg<DK, DV>::THREADS, 1)
     } else {
         // ======================= chain warpgroup =======================
         const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);
-        const int j = (DV == 128) ? tid : (lane < 16 ? warp * 16 + lane : -1);  // value column
+        // dv = 64 puts S^T and U^T in the M = 64 accumulator layout (rows at lanes r % 16 of each
+        // warp quadrant); every row is then split between threads `lane` and `lane + 16`, which
+        // take the first and the second half of its columns (16x32bx2 TMEM accesses)
+        constexpr bool kHalf = DV == 64;
+        const int j = kHalf ? warp * 16 + (lane & 15) : tid;  // value column = S^T row
+        const int hh = kHalf ? (lane >> 4) : 0;               // column half of that row
+        // 32-feature blocks cb of S^T row j held by this thread, as the k-th of its loads
+        constexpr int kSB = kHalf ? DK / 64 : DK / 32;
+        auto s_block = [&](int k) { return kHalf ? k + hh * (DK / 64) : k; };
+        auto ld_state = [&](int k, float (&x)[32]) {
+            if (kHalf) tmem_ld16x2_32<DK / 2>(tl + L::T_S + 32 * k, x);
+            else tmem_ld32(tl + L::T_S + 32 * k, x);
+        };
+        auto st_state = [&](int k, const float (&x)[32]) {
+            if (kHalf) tmem_st16x2_32<DK / 2>(tl + L::T_S + 32 * k, x);
+            else tmem_st32(tl + L::T_S + 32 * k, x);
+        };
         // bf16 copy of S^T row j, features 32cb .. 32cb+31, into S^T buffer b
         auto store_state_bf16 = [&](int b, int cb, const float (&x)[32]) {
-            if (j < 0) return;
             unsigned char *stt = sm + L::ST + b * L::ST_BUF + (cb >> 1) * (DV * 128);
 #pragma unroll
             for (int cc = 0; cc < 4; ++cc) {
@@ -650,9 +673,9 @@ __global__ void __launch_bounds__(TcCfg<DK, DV>::THREADS, 1)
                 *reinterpret_cast<uint4 *>(stt + j * 128 + (((chunk ^ (j & 7)) & 7) << 4)) = w;
             }
         };
-        // Output rows of chunk c: O (M = 64 tokens, N = DV) sits in lanes 0..15 of each warp,
-        // row 16w + lane.  The chunk's P tile is released to the intra side as soon as the
-        // output MMA has completed.
+        // Output rows of chunk c: O (M = 64 tokens, N = DV) sits in lanes 0..15 of each warp
+        // quadrant, row 16w + lane % 16; threads lane and lane + 16 store the two halves of a row.
+        // The chunk's P tile is released to the intra side as soon as the output MMA has completed.
         auto out_epilogue = [&](int c) {
             const long tk = tok0 + (long)c * CH;
             const int n = (int)min((long)CH, len - (long)c * CH);
@@ -661,13 +684,13 @@ __global__ void __launch_bounds__(TcCfg<DK, DV>::THREADS, 1)
                 tc_fence_after();
                 if (tid == 0) ctl.arrive(B::cdone + (c % NS));
                 const int r = 16 * warp + (lane & 15);
-                __nv_bfloat16 *op = out + ((size_t)(tk + r) * H + h) * DV;
+                __nv_bfloat16 *op = out + ((size_t)(tk + r) * H + h) * DV + (lane >> 4) * (DV / 2);
 #pragma unroll 1
-                for (int cb = 0; cb < DV / 32; ++cb) {
+                for (int cb = 0; cb < DV / 64; ++cb) {
                     float o[32];
-                    tmem_ld32(tl + L::T_O + (c % NB) * DV + cb * 32, o);
+                    tmem_ld16x2_32<DV / 2>(tl + L::T_O + (c % NB) * DV + cb * 32, o);
                     tmem_wait_ld();
-                    if (lane < 16 && r < n) {
+                    if (r < n) {
                         uint4 *dst = reinterpret_cast<uint4 *>(op + cb * 32);
 #pragma unroll
                         for (int q = 0; q < 4; ++q) {
@@ -691,16 +714,17 @@ __global__ void __launch_bounds__(TcCfg<DK, DV>::THREADS, 1)
             ctl.wait(B::gready + 0, 0);
             const float g0 = gates(0)[6 * CH];
 #pragma unroll 1
-            for (int cb = 0; cb < DK / 32; ++cb) {
+            for (int k = 0; k < kSB; ++k) {
+                const int cb = s_block(k);
                 float x[32];
 #pragma unroll
                 for (int i = 0; i < 32; ++i)
                     x[i] = (flags & kFlagS0Identity) ? ((cb * 32 + i == j) ? 1.f : 0.f)
-                                                     : ((j >= 0 && S0) ? S0[sbase + (size_t)(cb * 32 + i) * DV + j] : 0.f);
+                                                     : (S0 ? S0[sbase + (size_t)(cb * 32 + i) * DV + j] : 0.f);
                 store_state_bf16(0, cb, x);
 #pragma unroll
                 for (int i = 0; i < 32; ++i) x[i] *= g0;
-                tmem_st32(tl + L::T_S + cb * 32, x);
+                st_state(k, x);
             }
             tmem_wait_st();
             fence_proxy_async_smem();
@@ -747,12 +771,17 @@ __global__ void __launch_bounds__(TcCfg<DK, DV>::THREADS, 1)
             ctl.wait(B::u, c & 1);
             tc_fence_after();
             if (tid == 0) ctl.arrive(B::tfree + (c % NI));  // W^T of this chunk has been read
-            {
+            if (kHalf) {
+                float x[32];
+                tmem_ld16x2_32<32>(tl + L::T_U + st * 64, x);
+                tmem_wait_ld();
+                st_half_row_bf16_sw128(sm + L::UT, j, hh, x);
+            } else {
                 float x[64];
                 tmem_ld32(tl + L::T_U + st * 64, *reinterpret_cast<float(*)[32]>(&x[0]));
                 tmem_ld32(tl + L::T_U + st * 64 + 32, *reinterpret_cast<float(*)[32]>(&x[32]));
                 tmem_wait_ld();
-                if (j >= 0) st_row_bf16_sw128(sm + L::UT, j, x);
+                st_row_bf16_sw128(sm + L::UT, j, x);
             }
             fence_proxy_async_smem();
             tc_fence_before();
@@ -789,15 +818,15 @@ __global__ void __launch_bounds__(TcCfg<DK, DV>::THREADS, 1)
                     gn = gates((c + 1) % NS)[6 * CH];
                 }
 #pragma unroll 1
-                for (int cb = 0; cb < DK / 32; ++cb) {
+                for (int k = 0; k < kSB; ++k) {
                     float x[32];
-                    tmem_ld32(tl + L::T_S + cb * 32, x);
+                    ld_state(k, x);
                     tmem_wait_ld();
-                    store_state_bf16((c + 1) % NB, cb, x);
+                    store_state_bf16((c + 1) % NB, s_block(k), x);
                     if (more) {
 #pragma unroll
                         for (int i = 0; i < 32; ++i) x[i] *= gn;
-                        tmem_st32(tl + L::T_S + cb * 32, x);
+                        st_state(k, x);
                     }
                 }
                 tmem_wait_st();
@@ -811,16 +840,15 @@ __global__ void __launch_bounds__(TcCfg<DK, DV>::THREADS, 1)
         if (S_final) {
             if (nchunks > 0) {
 #pragma unroll 1
-                for (int cb = 0; cb < DK / 32; ++cb) {
+                for (int k = 0; k < kSB; ++k) {
+                    const int cb = s_block(k);
                     float x[32];
-                    tmem_ld32(tl + L::T_S + cb * 32, x);
+                    ld_state(k, x);
                     tmem_wait_ld();
-                    if (j >= 0) {
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) S_final[sbase + (size_t)(cb * 32 + i) * DV + j] = x[i];
-                    }
+                    for (int i = 0; i < 32; ++i) S_final[sbase + (size_t)(cb * 32 + i) * DV + j] = x[i];
                 }
-            } else if (j >= 0) {
+            } else if (hh == 0) {
                 for (int c2 = 0; c2 < DK; ++c2)
                     S_final[sbase + (size_t)c2 * DV + j] =
                         (flags & kFlagS0Identity) ? (c2 == j ? 1.f : 0.f) : (S0 ? S0[sbase + (size_t)c2 * DV + j] : 0.f);

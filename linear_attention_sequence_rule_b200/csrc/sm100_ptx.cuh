@@ -227,6 +227,48 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32])
         : "memory");
 }
 
+// Shape 16x32bx2, 32 columns per thread: threads 0-15 of the warp read (write) lanes 0-15 of the
+// warp's quadrant at columns taddr.col + 0..31, threads 16-31 the same lanes at columns
+// taddr.col + OFF + 0..31.  For an M = 64 accumulator (rows at lanes r % 16 + 32 (r / 16)) this
+// splits each row between two threads, so a whole warp works on its 16 rows.
+template <int OFF>
+__device__ __forceinline__ void tmem_ld16x2_32(uint32_t taddr, float (&v)[32])
+{
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.16x32bx2.x32.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32], %33;"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+          "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+          "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+          "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr), "n"(OFF));
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+template <int OFF>
+__device__ __forceinline__ void tmem_st16x2_32(uint32_t taddr, const float (&v)[32])
+{
+    asm volatile(
+        "tcgen05.st.sync.aligned.16x32bx2.x32.b32 [%0], %33, "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+        "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
+        "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
+        "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])), "r"(__float_as_uint(v[8])),
+        "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
+        "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
+        "r"(__float_as_uint(v[15])), "r"(__float_as_uint(v[16])), "r"(__float_as_uint(v[17])),
+        "r"(__float_as_uint(v[18])), "r"(__float_as_uint(v[19])), "r"(__float_as_uint(v[20])),
+        "r"(__float_as_uint(v[21])), "r"(__float_as_uint(v[22])), "r"(__float_as_uint(v[23])),
+        "r"(__float_as_uint(v[24])), "r"(__float_as_uint(v[25])), "r"(__float_as_uint(v[26])),
+        "r"(__float_as_uint(v[27])), "r"(__float_as_uint(v[28])), "r"(__float_as_uint(v[29])),
+        "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31])), "n"(OFF)
+        : "memory");
+}
+
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
@@ -265,6 +307,20 @@ __device__ __forceinline__ void st_row_bf16_sw128(unsigned char *tile, int row, 
         w.z = pack_bf16x2(x[8 * c + 4], x[8 * c + 5]);
         w.w = pack_bf16x2(x[8 * c + 6], x[8 * c + 7]);
         *reinterpret_cast<uint4 *>(tile + row * 128 + (((c ^ (row & 7)) & 7) << 4)) = w;
+    }
+}
+
+// Write 32 fp32 values as half h (16-byte chunks 4h .. 4h+3) of a swizzled 128-byte bf16 row.
+__device__ __forceinline__ void st_half_row_bf16_sw128(unsigned char *tile, int row, int h, const float *x)
+{
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        uint4 w;
+        w.x = pack_bf16x2(x[8 * c + 0], x[8 * c + 1]);
+        w.y = pack_bf16x2(x[8 * c + 2], x[8 * c + 3]);
+        w.z = pack_bf16x2(x[8 * c + 4], x[8 * c + 5]);
+        w.w = pack_bf16x2(x[8 * c + 6], x[8 * c + 7]);
+        *reinterpret_cast<uint4 *>(tile + row * 128 + ((((4 * h + c) ^ (row & 7)) & 7) << 4)) = w;
     }
 }
 
