@@ -60,16 +60,13 @@ constexpr int kFlagS0Identity = 2;
 
 template <int DK, int DV>
 struct TcCfg {
-    // Intra warpgroups: two (alternate chunks) where shared memory and TMEM hold two sets of
-    // solve buffers, which is dk = dv = 64; otherwise one.
-    static constexpr int NI = (DK == 64 && DV == 64) ? 2 : 1;
+    // Two intra warpgroups take alternate chunks.
+    static constexpr int NI = 2;
     static constexpr int THREADS = 128 * (1 + NI);
     static constexpr int NS = (DK == 128 || DV == 128) ? 2 : 3;  // K/Q stages
-    // buffers of V, of the bf16 S^T copy and of O: two with two intra warpgroups (the V load of a
-    // chunk then starts two chunks ahead, and the output epilogue overlaps the next state MMA)
-    static constexpr int NB = NI;
-    // W^T (DK x 64 bf16) is written over T diag(b gam) once the WY MMAs have read it (dk = 64)
-    static constexpr bool WT_IN_TG = DK == 64;
+    // buffers of V, of the bf16 S^T copy and of O: two where TMEM holds two O buffers (the V load
+    // of a chunk then starts two chunks ahead, and the output epilogue overlaps the next state MMA)
+    static constexpr int NB = (2 * DV + DK + NI * 64 + NS * 64 <= 512) ? 2 : 1;
     // shared memory byte offsets (swizzled tiles first, all 1024-aligned)
     static constexpr int KQ = 0;                                 // per stage: per 64-feature block K (8K) | Q (8K)
     static constexpr int KQ_STAGE = (DK / 64) * 16384;
@@ -82,10 +79,11 @@ struct TcCfg {
     static constexpr int WG0 = UT + DV * 128;                    // per intra warpgroup:
     static constexpr int W_TB = 0;                               //   T diag(b)      bf16 64 x 128 B
     static constexpr int W_TG = 8192;                            //   T diag(b gam)  bf16 64 x 128 B
-    static constexpr int W_WT = WT_IN_TG ? W_TG : 16384;         //   W^T bf16, DK rows x 128 B
-    static constexpr int W_AF = WT_IN_TG ? 16384 : 16384 + DK * 128;  // A fp32 [64][LDF]
-    static constexpr int W_TF = W_AF + CH * LDF * 4;             //   decays, then T fp32 [64][LDF]
-    static constexpr int W_XS = W_TF + CH * LDF * 4;             //   merge scratch, 4 x 256 fp32
+    // W^T (DK rows x 128 B bf16) is written over T diag(b gam) (dk = 64) or over both T tiles
+    // (dk = 128) once the WY MMAs have read them
+    static constexpr int W_WT = DK == 64 ? W_TG : W_TB;
+    static constexpr int W_AT = 16384;                           //   decays, then A, then T: fp32 [64][LDF]
+    static constexpr int W_XS = W_AT + CH * LDF * 4;             //   merge scratch, 4 x 256 fp32
     static constexpr int WG_BYTES = (W_XS + 4 * 256 * 4 + 1023) & ~1023;
     static constexpr int GT = WG0 + NI * WG_BYTES;               // per stage: gate vectors
     static constexpr int GT_STAGE = 7 * CH * 4;                  //   graw, G2, gam, lam, bet, last, (gC)
@@ -184,13 +182,16 @@ __device__ __forceinline__ uint32_t tf(float x) { return __float_as_uint(x); }
 
 // T = (I + A)^{-1} for strictly lower triangular A (64 x 64 fp32, row stride LDF; only entries
 // below the diagonal are read), executed by the 128 threads of the intra warpgroup (t = 0..127).
+// T is written over A in place (out.Tm == A): every block of A is read before T's block at the
+// same place is written (registers, __syncwarp, or the barrier inside the 16 -> 32 step), and the
+// last step's lower-left block goes to the bf16 tiles only.
 // Warp w owns the 16 x 16 diagonal block w: its two 8 x 8 diagonal sub-blocks are inverted by
 // column-parallel forward substitution (lane = column, running sums, 7 dependent steps), then one
 // doubling step T_ba = -T_bb (A_ba T_aa) joins them.  The 16 -> 32 and 32 -> 64 merges run the
 // same step on mma.sync TF32 (T is rounded to bf16 afterwards, so TF32 products stay below that
 // rounding).  Every entry of the lower triangle is written exactly once, through `out`; entries
 // above the diagonal are never written (the caller keeps them zero in the bf16 copies).
-__device__ void solve_unit_lower(const float *__restrict__ A, const TOut &out, float *__restrict__ XS, int t, int bar_id)
+__device__ void solve_unit_lower(const float *A, const TOut &out, float *__restrict__ XS, int t, int bar_id)
 {
     float *Tm = out.Tm;
     const int w = t >> 5, lane = t & 31, g = lane >> 2, tq = lane & 3;
@@ -200,6 +201,11 @@ __device__ void solve_unit_lower(const float *__restrict__ A, const TOut &out, f
         if (lane < 16) {
             const int sb = o + 8 * (lane >> 3), c = lane & 7;
             const float bc = out.bet[sb + c], gc = out.gam[sb + c];
+            float a[8][8];  // the block's strictly lower part, read before any lane writes T there
+#pragma unroll
+            for (int r = 1; r < 8; ++r)
+#pragma unroll
+                for (int i = 0; i < r; ++i) a[r][i] = A[(sb + r) * LDF + sb + i];
             float p[8], x[8];
 #pragma unroll
             for (int r = 0; r < 8; ++r) p[r] = 0.f;
@@ -207,8 +213,9 @@ __device__ void solve_unit_lower(const float *__restrict__ A, const TOut &out, f
             for (int i = 0; i < 8; ++i) {
                 x[i] = (i < c) ? 0.f : (i == c ? 1.f : -p[i]);
 #pragma unroll
-                for (int r = i + 1; r < 8; ++r) p[r] = fmaf(A[(sb + r) * LDF + sb + i], x[i], p[r]);
+                for (int r = i + 1; r < 8; ++r) p[r] = fmaf(a[r][i], x[i], p[r]);
             }
+            __syncwarp(0xffffu);
 #pragma unroll
             for (int r = 0; r < 8; ++r)
                 if (r >= c) out.put(sb + r, sb + c, x[r], bc, gc);
@@ -252,7 +259,8 @@ __device__ void solve_unit_lower(const float *__restrict__ A, const TOut &out, f
         xs[g * 8 + 2 * tq + 1] = d[1];
         xs[(g + 8) * 8 + 2 * tq] = d[2];
         xs[(g + 8) * 8 + 2 * tq + 1] = d[3];
-        __syncwarp();
+        // both warps of the pair have read A's block before T's block replaces it
+        named_bar(bar_id, 128);
         float e[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int kk = 0; kk < 2; ++kk) {
@@ -439,8 +447,7 @@ __global__ void __launch_bounds__(TcCfg<DK, DV>::THREADS, 1)
         const uint32_t tG = L::T_G + wg * 64;  // Gram accumulator, then W^T
         unsigned char *wsm = sm + L::WG0 + wg * L::WG_BYTES;
         unsigned char *TBs = wsm + L::W_TB, *TGs = wsm + L::W_TG, *WTs = wsm + L::W_WT;
-        float *AF = reinterpret_cast<float *>(wsm + L::W_AF);
-        float *TFm = reinterpret_cast<float *>(wsm + L::W_TF);
+        float *AT = reinterpret_cast<float *>(wsm + L::W_AT);  // decays, then A, then T (in place)
         float *XSm = reinterpret_cast<float *>(wsm + L::W_XS);
         // entries above the diagonal of T diag(b..) stay zero (the solve writes the lower part)
         for (int i = t; i < 2 * 8192 / 16; i += 128)
@@ -514,12 +521,12 @@ __global__ void __launch_bounds__(TcCfg<DK, DV>::THREADS, 1)
                 }
             }
             named_bar(bar_id, 128);
-            // ---- decays Gam[r][i] (lower triangle; zero across a reset) into the T scratch ----
+            // ---- decays Gam[r][i] (lower triangle; zero across a reset) into the A/T buffer ----
             {
                 const int r = t & 63, c0 = (t >> 6) * 32;
                 const float Gr = Gs[r];
                 const int lr = last[r];
-                float *gm = TFm + r * LDF + c0;
+                float *gm = AT + r * LDF + c0;
 #pragma unroll
                 for (int j4 = 0; j4 < 32; j4 += 4) {
                     const float4 g4 = *reinterpret_cast<const float4 *>(&Gs[c0 + j4]);
@@ -551,18 +558,20 @@ __global__ void __launch_bounds__(TcCfg<DK, DV>::THREADS, 1)
                 const float sc = isq ? 1.f : bet[r];
 #pragma unroll
                 for (int i4 = 0; i4 < CH; i4 += 4) {
-                    const float4 gm = *reinterpret_cast<const float4 *>(&TFm[r * LDF + i4]);
+                    const float4 gm = *reinterpret_cast<const float4 *>(&AT[r * LDF + i4]);
                     x[i4] *= gm.x * sc;
                     x[i4 + 1] *= gm.y * sc;
                     x[i4 + 2] *= gm.z * sc;
                     x[i4 + 3] *= gm.w * sc;
                 }
+                // both threads of row r have read its decays before A overwrites them
+                named_bar(bar_id, 128);
                 if (isq) {
                     st_row_bf16_sw128(sm + L::PM + st * 8192, r, x);
                 } else {
 #pragma unroll
                     for (int i = 0; i < CH; i += 4)
-                        *reinterpret_cast<float4 *>(&AF[r * LDF + i]) = make_float4(x[i], x[i + 1], x[i + 2], x[i + 3]);
+                        *reinterpret_cast<float4 *>(&AT[r * LDF + i]) = make_float4(x[i], x[i + 1], x[i + 2], x[i + 3]);
                 }
                 if (DK == 128)
                     scale_row_bf16(Kt + (t >> 6) * 16384 + 8192, r, gam[r], 0, 8);
@@ -572,18 +581,21 @@ __global__ void __launch_bounds__(TcCfg<DK, DV>::THREADS, 1)
             tc_fence_before();
             // this warpgroup's previous chunk: its W^T and T diag(b..) tiles must have been read
             if (kc >= 1) ctl.wait(B::tfree + wg, (kc - 1) & 1);
-            if (L::WT_IN_TG) {
-                // W^T of the previous chunk sits in the T diag(b gam) tile: clear every 16-byte
-                // chunk from the diagonal block rightwards (the solve then writes the lower part)
-                for (int i = t; i < 64 * 8; i += 128) {
-                    const int r = i >> 3, cb = i & 7;
+            if (kc >= 1) {
+                // W^T of the previous chunk sits in T diag(b gam) (dk = 64) or in both T tiles
+                // (dk = 128): clear every 16-byte chunk from the diagonal block rightwards (the
+                // solve then writes the lower part)
+                constexpr int kTiles = DK / 64;
+                for (int i = t; i < kTiles * 64 * 8; i += 128) {
+                    const int r = (i >> 3) & 63, cb = i & 7;
+                    unsigned char *tile = (kTiles == 2 && i >= 64 * 8) ? TGs : (kTiles == 2 ? TBs : TGs);
                     if (cb >= (r >> 3))
-                        *reinterpret_cast<uint4 *>(TGs + r * 128 + ((cb ^ (r & 7)) << 4)) = make_uint4(0u, 0u, 0u, 0u);
+                        *reinterpret_cast<uint4 *>(tile + r * 128 + ((cb ^ (r & 7)) << 4)) = make_uint4(0u, 0u, 0u, 0u);
                 }
             }
             named_bar(bar_id, 128);
             // ---- T = (I + A)^{-1}, written with the bf16 rows of T diag(b), T diag(b gam) ----
-            solve_unit_lower(AF, TOut{TFm, TBs, TGs, bet, gam}, XSm, t, bar_id);
+            solve_unit_lower(AT, TOut{AT, TBs, TGs, bet, gam}, XSm, t, bar_id);
             fence_proxy_async_smem();
             tc_fence_before();
             named_bar(bar_id, 128);
