@@ -355,6 +355,9 @@ __global__ void __launch_bounds__(TcCfg<DK, DV>::THREADS, 1)
     constexpr int NI = L::NI;
     constexpr int NB = L::NB;
     using B = Bars<NS, NI, NB>;
+    // gam Q and lam K are formed in place by the chain (dk = 128, whose chain has slack while the
+    // U MMA runs) or by the intra side (dk = 64, where the chain is the busier side)
+    constexpr bool kChainScales = DK == 128;
     extern __shared__ unsigned char smem_raw[];
     // 1024-aligned base by pointer arithmetic on the shared array, so that the compiler keeps
     // every access below in the shared address space
@@ -548,7 +551,8 @@ __global__ void __launch_bounds__(TcCfg<DK, DV>::THREADS, 1)
             named_bar(bar_id, 128);
             {
                 // A = diag(b) (Gam o K K^T) (fp32; its diagonal and upper part are never read),
-                // P = Gam o Q K^T (bf16), and gam Q in place (no MMA reads Q unscaled any more)
+                // P = Gam o Q K^T (bf16) and, unless the chain does it, gam Q in place (no MMA
+                // reads Q unscaled any more)
                 float x[64];
                 tmem_ld32(tl + tG, *reinterpret_cast<float(*)[32]>(&x[0]));
                 tmem_ld32(tl + tG + 32, *reinterpret_cast<float(*)[32]>(&x[32]));
@@ -573,10 +577,7 @@ __global__ void __launch_bounds__(TcCfg<DK, DV>::THREADS, 1)
                     for (int i = 0; i < CH; i += 4)
                         *reinterpret_cast<float4 *>(&AT[r * LDF + i]) = make_float4(x[i], x[i + 1], x[i + 2], x[i + 3]);
                 }
-                if (DK == 128)
-                    scale_row_bf16(Kt + (t >> 6) * 16384 + 8192, r, gam[r], 0, 8);
-                else
-                    scale_row_bf16(Kt + 8192, r, gam[r], (t >> 6) * 4, (t >> 6) * 4 + 4);
+                if (!kChainScales) scale_row_bf16(Kt + 8192, r, gam[r], (t >> 6) * 4, (t >> 6) * 4 + 4);
             }
             tc_fence_before();
             // this warpgroup's previous chunk: its W^T and T diag(b..) tiles must have been read
@@ -625,8 +626,8 @@ __global__ void __launch_bounds__(TcCfg<DK, DV>::THREADS, 1)
             tc_fence_after();
             if (t == kIssuer && c + NB < nchunks) load_v(c + NB);  // the U~ MMA has read V
             {
-                // W^T rows (one per feature) to shared memory in bf16, then lam K in place (the
-                // W MMA has read K unscaled)
+                // W^T rows (one per feature) to shared memory in bf16, then (unless the chain does
+                // it) lam K in place: the W MMA has read K unscaled
                 if (DK == 128) {
                     float x[64];
                     tmem_ld32(tl + tG, *reinterpret_cast<float(*)[32]>(&x[0]));
@@ -640,11 +641,7 @@ __global__ void __launch_bounds__(TcCfg<DK, DV>::THREADS, 1)
                     tmem_wait_ld();
                     st_half_row_bf16_sw128(WTs, wi * 16 + (t & 15), (t >> 4) & 1, x);
                 }
-                const int r = t & 63;
-                if (DK == 128)
-                    scale_row_bf16(Kt + (t >> 6) * 16384, r, lam[r], 0, 8);
-                else
-                    scale_row_bf16(Kt, r, lam[r], (t >> 6) * 4, (t >> 6) * 4 + 4);
+                if (!kChainScales) scale_row_bf16(Kt, t & 63, lam[t & 63], (t >> 6) * 4, (t >> 6) * 4 + 4);
             }
             fence_proxy_async_smem();
             tc_fence_before();
@@ -772,10 +769,20 @@ __global__ void __launch_bounds__(TcCfg<DK, DV>::THREADS, 1)
                 }
                 mma_commit(&bars[B::u]);
             }
+            if (kChainScales) {
+                // while the U MMA runs: gam Q and lam K in place for O1 and the state MMA (every
+                // MMA that reads them unscaled, Gram and W, completed before the chunk was ready)
+                const float *gv = gates(st);
+                const int r = tid & 63;
+                scale_row_bf16(Kt + (tid >> 6) * 16384 + 8192, r, gv[2 * CH + r], 0, 8);
+                scale_row_bf16(Kt + (tid >> 6) * 16384, r, gv[3 * CH + r], 0, 8);
+                fence_proxy_async_smem();
+            }
             // O1 goes before the state MMA's commit, so that its completion also covers O1's reads
             // of the Q tile (reloaded right after) and of the S_c copy.  One O buffer: the previous
             // chunk's outputs leave first, while the U MMA runs.
             if (NB == 1 && c >= 1) out_epilogue(c - 1);
+            if (kChainScales) named_bar(1, 128);  // the scaled tiles are complete
             if (tid == 0 && want_out && !ctl.aborted()) {
                 tc_fence_after();
                 issue_o1();
@@ -801,13 +808,13 @@ __global__ void __launch_bounds__(TcCfg<DK, DV>::THREADS, 1)
             if (tid == 0 && !ctl.aborted()) {
                 tc_fence_after();
                 constexpr uint32_t idS = idesc_bf16(DV, DK, 0, 1);
-                constexpr uint32_t idP = idesc_bf16(64, DV, 0, 0);
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)  // S^T += U^T (lam K)
                     mma_bf16(tmem + L::T_S, sdesc_sw128(smem_u32(sm + L::UT + kk * 32), 16, 1024),
                              sdesc_sw128(smem_u32(Kt + kk * 2048), 16384, 1024), idS, 1);
                 mma_commit(&bars[B::s]);
                 if (want_out) {
+                    constexpr uint32_t idP = idesc_bf16(64, DV, 0, 0);
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)  // O += P U: A = P rows (K-major), B = U^T rows (K-major)
                         mma_bf16(tO, sdesc_sw128(smem_u32(sm + L::PM + st * 8192 + kk * 32), 16, 1024),
