@@ -84,6 +84,52 @@ def make_chunk_inputs(B=None, T=None, H=2, dk=64, dv=64, dtype="bf16", seed=0, b
                 dtype=dtype, lengths=lengths)
 
 
+def make_raw_chunk_inputs(B=None, T=None, H=2, dk=64, dv=64, dtype="bf16", seed=0, beta_scale=1.0,
+                          la_std=1.0, la_scale=1.0, s0_std=0.0, lengths=None, n_seqs=None,
+                          len_lo=None, len_hi=None, **_ignored):
+    """Raw-projection inputs for the fused-prologue chunk forward: the same draws, in the same
+    order and shapes, as ``make_chunk_inputs`` before any normalisation or gate activation.
+
+    q_raw, k_raw ~ N(0, 1) cast to dtype (not normalised); v ~ N(0, 1) in dtype; b_raw ~ N(0, 1)
+    and a_raw ~ N(0, la_std) in fp32; a_scale = la_scale and b_scale = beta_scale are the scales
+    of the prologue's gate forms.
+    """
+    g = torch.Generator().manual_seed(int(seed))
+    dt = DTYPES[dtype]
+    if n_seqs is not None and lengths is None:
+        lengths = torch.randint(int(len_lo), int(len_hi) + 1, (int(n_seqs),), generator=g).tolist()
+    if lengths is not None:
+        lengths = [int(x) for x in lengths]
+        cu = torch.zeros(len(lengths) + 1, dtype=torch.int32)
+        cu[1:] = torch.cumsum(torch.tensor(lengths, dtype=torch.int64), 0).to(torch.int32)
+        lead = (int(cu[-1]),)
+        nseq = len(lengths)
+    else:
+        cu = None
+        lead = (int(B), int(T))
+        nseq = int(B)
+    q_raw = torch.randn(*lead, H, dk, generator=g).to(dt)
+    k_raw = torch.randn(*lead, H, dk, generator=g).to(dt)
+    v = torch.randn(*lead, H, dv, generator=g).to(dt)
+    b_raw = torch.randn(*lead, H, generator=g).float()
+    a_raw = (la_std * torch.randn(*lead, H, generator=g)).float()
+    S0 = None
+    if s0_std:
+        S0 = (s0_std * torch.randn(nseq, H, dk, dv, generator=g)).float()
+    return dict(q_raw=q_raw, k_raw=k_raw, v=v, a_raw=a_raw, b_raw=b_raw, S0=S0, cu_seqlens=cu,
+                a_scale=float(la_scale), b_scale=float(beta_scale), B=nseq,
+                T=(lead[0] if cu is not None else int(T)), H=H, dk=dk, dv=dv, dtype=dtype,
+                lengths=lengths)
+
+
+def config_raw_inputs(name: str, **overrides):
+    """Raw-projection inputs of a named chunk workload (see ``make_raw_chunk_inputs``)."""
+    cfg = dict(CONFIGS[name])
+    cfg.update(overrides)
+    assert cfg["kind"] == "chunk"
+    return make_raw_chunk_inputs(**cfg)
+
+
 def config_inputs(name: str, **overrides):
     """Inputs of a named chunk workload (``tiny``, ``hybrid_lm``, ``long_context``, ``varlen``)."""
     cfg = dict(CONFIGS[name])
