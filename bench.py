@@ -231,6 +231,47 @@ def gdn_mod():
     return gdn
 
 
+def time_prologue(gdn, d, steps, warmup, flush, stream, fused):
+    """Per-step CUDA-event time (ms) from raw projections to outputs: the fused entry, or PyTorch
+    normalisation and activations (separate kernels, one more HBM pass over q, k and the gates)
+    followed by the plain entry."""
+    out = torch.empty_like(d["v"])
+    Sf = torch.empty((d["B"], d["H"], d["dk"], d["dv"]), dtype=torch.float32, device="cuda")
+    ws = chunk_workspace(gdn, d | {"q": d["q_raw"]})
+
+    def unfused_prologue():
+        qf, kf = d["q_raw"].float(), d["k_raw"].float()
+        q = (qf * torch.rsqrt((qf * qf).sum(-1, keepdim=True) + 1e-6)).to(d["q_raw"].dtype)
+        k = (kf * torch.rsqrt((kf * kf).sum(-1, keepdim=True) + 1e-6)).to(d["k_raw"].dtype)
+        la = -d["a_scale"] * torch.nn.functional.softplus(d["a_raw"])
+        be = d["b_scale"] * torch.sigmoid(d["b_raw"])
+        return q, k, la, be
+
+    def call():
+        if fused:
+            gdn.chunk_fwd_fused(d["q_raw"], d["k_raw"], d["v"], d["a_raw"], d["b_raw"], d["a_scale"],
+                                d["b_scale"], S0=d["S0"], cu_seqlens=d["cu_seqlens"], out=out, S_final=Sf,
+                                workspace=ws, stream=stream)
+        else:
+            q, k, la, be = unfused_prologue()
+            gdn.chunk_fwd(q, k, d["v"], la, be, S0=d["S0"], cu_seqlens=d["cu_seqlens"], out=out,
+                          S_final=Sf, workspace=ws, stream=stream)
+    with torch.cuda.stream(stream):
+        for _ in range(warmup):
+            flush.zero_()
+            call()
+        stream.synchronize()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(steps)]
+        for s0, e in ev:
+            flush.zero_()
+            s0.record(stream)
+            call()
+            e.record(stream)
+        stream.synchronize()
+    return [a.elapsed_time(b) for a, b in ev]
+
+
 def chunk_numbers(name, d, times_ms, peaks):
     ms = statistics.mean(times_ms)
     th = d["q"].shape[0] * (d["q"].shape[1] if d["cu_seqlens"] is None else 1) * d["H"]
@@ -378,6 +419,15 @@ def run_ours(args, world, rank, local):
             nums = chunk_numbers(w, dw, tw, peaks)
             extra[w] = {k: (round(v, 6) if isinstance(v, float) else v) for k, v in nums.items()}
             del dw
+        # the same hybrid-LM step from raw projections: fused prologue vs PyTorch prologue + call
+        dr = to_dev(workloads.config_raw_inputs(name, seed=rank_seed(cfg["seed"], rank)))
+        for key, fused in (("hybrid_lm_fused_prologue", True), ("hybrid_lm_pytorch_prologue", False)):
+            tw = time_prologue(gdn, dr, max(3, args.steps // 2), 3, flush, stream, fused)
+            ms_w = statistics.mean(tw)
+            extra[key] = {"workload": f"hybrid_lm from raw projections ({'fused entry' if fused else 'PyTorch normalisation and activations, then the plain entry'})",
+                          "ms": round(ms_w, 6), "tokens_per_s": round(main["tokens"] / (ms_w * 1e-3), 1),
+                          "launches_per_call": 1 if fused else None}
+        del dr
     cpu = None
     if rank == 0 and world == 1:
         cpu = cpu_oracle_baseline(inp)
@@ -431,6 +481,12 @@ def run_only(args):
     if args.only == "decode":
         r = time_decode(gdn, args.steps, args.warmup, stream)
         r["hbm_frac"] = r["gbs"] / peaks["hbm_gbs"]
+    elif args.only in ("hybrid_lm_fused", "hybrid_lm_unfused"):
+        flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device="cuda")
+        d = to_dev(workloads.config_raw_inputs("hybrid_lm"))
+        tw = time_prologue(gdn, d, args.steps, args.warmup, flush, stream, args.only.endswith("_fused"))
+        ms = statistics.mean(tw)
+        r = {"workload": args.only, "ms": ms, "tokens_per_s": 8 * 4096 / (ms * 1e-3)}
     else:
         flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device="cuda")
         d = to_dev(workloads.config_inputs(args.only))
@@ -498,7 +554,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--quick", action="store_true", help="main workload only")
-    ap.add_argument("--only", choices=["hybrid_lm", "long_context", "varlen", "tiny", "decode"],
+    ap.add_argument("--only", choices=["hybrid_lm", "long_context", "varlen", "tiny", "decode", "hybrid_lm_fused",
+                                             "hybrid_lm_unfused"],
                     help="time one workload's kernel loop only (for profiler runs)")
     args = ap.parse_args()
     if args.warmup < 3:

@@ -96,6 +96,28 @@ GDN_API int gdn_chunk_fwd(const void *q, const void *k, const void *v, const flo
                   void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * gdn_chunk_fwd_fused -- gdn_chunk_fwd with its input prologue fused into the kernel: q_raw and
+ * k_raw are the unnormalised projections, and a_raw, b_raw the raw gate projections, so the
+ * separate passes that would normalise and activate them (one read and one write of q, k and
+ * the gates in HBM) are not needed.  Per (token, head), in fp32 inside the kernel:
+ *     q = q_raw / sqrt(|q_raw|^2 + 1e-6),   k likewise   (rounded to bf16 for the MMAs)
+ *     log_alpha = -a_scale * softplus(a_raw)   (a_raw = +inf: an exact reset)
+ *     beta      =  b_scale * sigmoid(b_raw)    (DeltaPhase README, section 1 "Extended
+ *                                               Householder Beta Range": beta = 2 sigmoid(W_beta x))
+ * after which the operation is exactly gdn_chunk_fwd's (Sykra README, "Architectural
+ * Highlights": data-dependent forget gate alpha_t in (0, 1]).  Layouts, S0 / S_final, varlen,
+ * workspace (query gdn_chunk_fwd_workspace_bytes with the same sizes) and asynchrony as for
+ * gdn_chunk_fwd; a_raw, b_raw [tokens, H] fp32.  dtype must be GDN_DTYPE_BF16 (else
+ * GDN_ERR_UNSUPPORTED); a_scale must be finite and >= 0 and b_scale in [0, 2] (else
+ * GDN_ERR_INVALID_ARGUMENT).
+ */
+GDN_API int gdn_chunk_fwd_fused(const void *q_raw, const void *k_raw, const void *v, const float *a_raw,
+                                const float *b_raw, const float *S0, void *out, float *S_final, int B,
+                                int T, int H, int dk, int dv, int chunk, const int32_t *cu_seqlens,
+                                int dtype, float a_scale, float b_scale, void *workspace,
+                                size_t workspace_bytes, void *stream);
+
+/*
  * gdn_chunk_fwd_workspace_bytes -- device scratch that gdn_chunk_fwd needs for these sizes
  * (varlen: non-zero when cu_seqlens will be passed).  Returns 0 when no scratch is needed and
  * (size_t)-1 for arguments gdn_chunk_fwd would reject.

@@ -6,7 +6,7 @@ PyTorch provides device memory and streams.  The binding has two layers:
 * ``gdn_chunk_fwd``, ``gdn_chunk_fwd_noalloc``, ``gdn_decode_step``, ``gdn_chunk_fwd_workspace_bytes``,
   ``gdn_status_string``, ``gdn_last_error``, ``gdn_version`` -- the C-ABI entry points of
   ``include/gdn.h`` with the same names and arguments (pointers as Python ints);
-* ``chunk_fwd`` and ``decode_step`` -- the same calls taking torch tensors; they check shapes,
+* ``chunk_fwd``, ``chunk_fwd_fused`` and ``decode_step`` -- the same calls taking torch tensors; they check shapes,
   devices and dtypes, allocate outputs with torch when none are given, and raise ``GdnError``
   on a non-zero status.
 
@@ -22,8 +22,9 @@ import torch
 __all__ = [
     "GdnError", "GDN_OK", "GDN_ERR_INVALID_ARGUMENT", "GDN_ERR_UNSUPPORTED", "GDN_ERR_WORKSPACE",
     "GDN_ERR_CUDA", "GDN_ERR_TIMEOUT", "GDN_DTYPE_F32", "GDN_DTYPE_BF16", "LIB_PATH",
-    "gdn_chunk_fwd", "gdn_chunk_fwd_noalloc", "gdn_decode_step", "gdn_chunk_fwd_workspace_bytes", "gdn_status_string",
-    "gdn_last_error", "gdn_version", "gdn_device_status", "device_status", "chunk_fwd", "decode_step", "workspace_bytes",
+    "gdn_chunk_fwd", "gdn_chunk_fwd_noalloc", "gdn_chunk_fwd_fused", "gdn_decode_step", "gdn_chunk_fwd_workspace_bytes", "gdn_status_string",
+    "gdn_last_error", "gdn_version", "gdn_device_status", "device_status", "chunk_fwd", "chunk_fwd_fused",
+    "decode_step", "workspace_bytes",
 ]
 
 GDN_OK = 0
@@ -48,6 +49,9 @@ _vp, _sz, _i = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int
 _lib.gdn_chunk_fwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i,
                                _vp, _i, _vp, _sz, _vp]
 _lib.gdn_chunk_fwd.restype = _i
+_lib.gdn_chunk_fwd_fused.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i,
+                                     _vp, _i, ctypes.c_float, ctypes.c_float, _vp, _sz, _vp]
+_lib.gdn_chunk_fwd_fused.restype = _i
 _lib.gdn_chunk_fwd_noalloc.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i,
                                        _i, _vp, _i, _vp]
 _lib.gdn_chunk_fwd_noalloc.restype = _i
@@ -77,6 +81,13 @@ def gdn_chunk_fwd(q, k, v, log_alpha, beta, S0, out, S_final, B, T, H, dk, dv, c
                   dtype, workspace, workspace_bytes, stream) -> int:
     return _lib.gdn_chunk_fwd(q, k, v, log_alpha, beta, S0, out, S_final, B, T, H, dk, dv, chunk,
                               cu_seqlens, dtype, workspace, workspace_bytes, stream)
+
+
+def gdn_chunk_fwd_fused(q_raw, k_raw, v, a_raw, b_raw, S0, out, S_final, B, T, H, dk, dv, chunk,
+                        cu_seqlens, dtype, a_scale, b_scale, workspace, workspace_bytes, stream) -> int:
+    return _lib.gdn_chunk_fwd_fused(q_raw, k_raw, v, a_raw, b_raw, S0, out, S_final, B, T, H, dk, dv,
+                                    chunk, cu_seqlens, dtype, a_scale, b_scale, workspace,
+                                    workspace_bytes, stream)
 
 
 def gdn_chunk_fwd_noalloc(q, k, v, log_alpha, beta, S0, out, S_final, B, T, H, dk, dv, chunk,
@@ -151,10 +162,9 @@ def workspace_bytes(B, T, H, dk, dv, varlen=False, dtype=torch.bfloat16, chunk=6
     return n
 
 
-def chunk_fwd(q, k, v, log_alpha, beta, S0=None, cu_seqlens=None, out=None, S_final=None,
-              output_final_state=True, workspace=None, chunk=64, stream=None):
-    """Chunkwise forward.  Dense q,k [B,T,H,dk], v [B,T,H,dv]; varlen (cu_seqlens int32 [B+1] on
-    the device) packs q,k [T,H,dk] ...  Returns (out, S_final or None)."""
+def _chunk_prepare(q, k, v, ga, gb, S0, cu_seqlens, out, S_final, output_final_state, workspace,
+                   chunk, names):
+    """Shape/device/dtype checks and output/workspace allocation shared by the chunk entries."""
     dt = q.dtype
     if dt not in _DT:
         raise ValueError(f"unsupported dtype {dt}")
@@ -168,11 +178,11 @@ def chunk_fwd(q, k, v, log_alpha, beta, S0=None, cu_seqlens=None, out=None, S_fi
         B, T, H, dk = q.shape
         lead = (B, T)
     dv = v.shape[-1]
-    _need(q, "q", dt, (*lead, H, dk), dev)
-    _need(k, "k", dt, (*lead, H, dk), dev)
+    _need(q, names[0], dt, (*lead, H, dk), dev)
+    _need(k, names[1], dt, (*lead, H, dk), dev)
     _need(v, "v", dt, (*lead, H, dv), dev)
-    _need(log_alpha, "log_alpha", torch.float32, (*lead, H), dev)
-    _need(beta, "beta", torch.float32, (*lead, H), dev)
+    _need(ga, names[2], torch.float32, (*lead, H), dev)
+    _need(gb, names[3], torch.float32, (*lead, H), dev)
     if S0 is not None:
         _need(S0, "S0", torch.float32, (B, H, dk, dv), dev)
     if out is None:
@@ -186,12 +196,40 @@ def chunk_fwd(q, k, v, log_alpha, beta, S0=None, cu_seqlens=None, out=None, S_fi
     if need and workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=dev)
     wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    rc = gdn_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(S0), _ptr(out),
-                       _ptr(S_final), B, T, H, dk, dv, chunk, _ptr(cu_seqlens), _DT[dt],
-                       _ptr(workspace), wbytes, _stream_ptr(stream))
+    return dict(B=B, T=T, H=H, dk=dk, dv=dv, dt=dt, out=out, S_final=S_final, workspace=workspace,
+                wbytes=wbytes)
+
+
+def chunk_fwd(q, k, v, log_alpha, beta, S0=None, cu_seqlens=None, out=None, S_final=None,
+              output_final_state=True, workspace=None, chunk=64, stream=None):
+    """Chunkwise forward.  Dense q,k [B,T,H,dk], v [B,T,H,dv]; varlen (cu_seqlens int32 [B+1] on
+    the device) packs q,k [T,H,dk] ...  Returns (out, S_final or None)."""
+    p = _chunk_prepare(q, k, v, log_alpha, beta, S0, cu_seqlens, out, S_final, output_final_state,
+                       workspace, chunk, ("q", "k", "log_alpha", "beta"))
+    rc = gdn_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(S0), _ptr(p["out"]),
+                       _ptr(p["S_final"]), p["B"], p["T"], p["H"], p["dk"], p["dv"], chunk,
+                       _ptr(cu_seqlens), _DT[p["dt"]], _ptr(p["workspace"]), p["wbytes"],
+                       _stream_ptr(stream))
     if rc != GDN_OK:
         raise GdnError(rc, gdn_last_error())
-    return out, S_final
+    return p["out"], p["S_final"]
+
+
+def chunk_fwd_fused(q_raw, k_raw, v, a_raw, b_raw, a_scale, b_scale, S0=None, cu_seqlens=None,
+                    out=None, S_final=None, output_final_state=True, workspace=None, chunk=64,
+                    stream=None):
+    """Chunkwise forward with the input prologue in the kernel (bf16): q_raw, k_raw are
+    normalised per row, log_alpha = -a_scale softplus(a_raw), beta = b_scale sigmoid(b_raw).
+    Layouts as ``chunk_fwd``.  Returns (out, S_final or None)."""
+    p = _chunk_prepare(q_raw, k_raw, v, a_raw, b_raw, S0, cu_seqlens, out, S_final,
+                       output_final_state, workspace, chunk, ("q_raw", "k_raw", "a_raw", "b_raw"))
+    rc = gdn_chunk_fwd_fused(_ptr(q_raw), _ptr(k_raw), _ptr(v), _ptr(a_raw), _ptr(b_raw), _ptr(S0),
+                             _ptr(p["out"]), _ptr(p["S_final"]), p["B"], p["T"], p["H"], p["dk"],
+                             p["dv"], chunk, _ptr(cu_seqlens), _DT[p["dt"]], float(a_scale),
+                             float(b_scale), _ptr(p["workspace"]), p["wbytes"], _stream_ptr(stream))
+    if rc != GDN_OK:
+        raise GdnError(rc, gdn_last_error())
+    return p["out"], p["S_final"]
 
 
 def decode_step(q, k, v, log_alpha, beta, S, out=None, stream=None):

@@ -95,41 +95,76 @@ size_t gdn_chunk_fwd_workspace_bytes(int B, int T, int H, int dk, int dv, int ch
     return chunk_workspace(B, T, H, dk, dv, varlen, dtype);
 }
 
+namespace gdn {
+
+// Validation and launch shared by the plain and the fused-prologue chunk forward.
+static int chunk_fwd_common(const char *fn, const void *q, const void *k, const void *v,
+                            const float *log_alpha, const float *beta, const float *S0, void *out,
+                            float *S_final, int B, int T, int H, int dk, int dv, int chunk,
+                            const int32_t *cu_seqlens, int dtype, int prologue, float a_scale,
+                            float b_scale, void *workspace, size_t workspace_bytes, void *stream)
+{
+    const int varlen = cu_seqlens != nullptr;
+    int rc = check_chunk_shape(B, T, H, dk, dv, chunk, varlen, dtype);
+    if (rc != GDN_OK) return rc;
+    if (!q || !k || !v || !log_alpha || !beta || !out)
+        return fail(GDN_ERR_INVALID_ARGUMENT, "%s: q, k, v, the two gate arrays and out are required", fn);
+    const void *ptrs[] = {q, k, v, log_alpha, beta, S0, out, S_final, cu_seqlens};
+    for (const void *p : ptrs)
+        if (p && !aligned16(p))
+            return fail(GDN_ERR_INVALID_ARGUMENT, "%s: pointer %p is not 16-byte aligned", fn, p);
+    if (S_final && S_final != S0 && S0) {
+        const size_t bytes = (size_t)B * H * dk * dv * sizeof(float);
+        const char *a0 = (const char *)S0, *b0 = (const char *)S_final;
+        if (a0 < b0 + bytes && b0 < a0 + bytes)
+            return fail(GDN_ERR_INVALID_ARGUMENT, "%s: S0 and S_final overlap partially", fn);
+    }
+    const size_t need = chunk_workspace(B, T, H, dk, dv, varlen, dtype);
+    if (need > 0) {
+        if (!workspace || workspace_bytes < need)
+            return fail(GDN_ERR_WORKSPACE, "%s: workspace of %zu bytes needed, %zu given", fn, need,
+                        workspace ? workspace_bytes : (size_t)0);
+        if (reinterpret_cast<uintptr_t>(workspace) & 255u)
+            return fail(GDN_ERR_INVALID_ARGUMENT, "%s: workspace must be 256-byte aligned", fn);
+    }
+    ChunkArgs a{q, k, v, log_alpha, beta, S0, out, S_final, cu_seqlens, B, T, H, dk, dv, dtype,
+                workspace, workspace_bytes, prologue, a_scale, b_scale};
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    cudaError_t e = dtype == GDN_DTYPE_BF16 ? launch_chunk_tc(a, st) : launch_chunk_simt(a, st);
+    if (e != cudaSuccess) return cuda_fail(e, fn);
+    return GDN_OK;
+}
+
+}  // namespace gdn
+
 int gdn_chunk_fwd(const void *q, const void *k, const void *v, const float *log_alpha,
                   const float *beta, const float *S0, void *out, float *S_final, int B, int T,
                   int H, int dk, int dv, int chunk, const int32_t *cu_seqlens, int dtype,
                   void *workspace, size_t workspace_bytes, void *stream)
 {
     g_last_error[0] = 0;
-    const int varlen = cu_seqlens != nullptr;
-    int rc = check_chunk_shape(B, T, H, dk, dv, chunk, varlen, dtype);
-    if (rc != GDN_OK) return rc;
-    if (!q || !k || !v || !log_alpha || !beta || !out)
-        return fail(GDN_ERR_INVALID_ARGUMENT, "gdn_chunk_fwd: q, k, v, log_alpha, beta and out are required");
-    const void *ptrs[] = {q, k, v, log_alpha, beta, S0, out, S_final, cu_seqlens};
-    for (const void *p : ptrs)
-        if (p && !aligned16(p))
-            return fail(GDN_ERR_INVALID_ARGUMENT, "gdn_chunk_fwd: pointer %p is not 16-byte aligned", p);
-    if (S_final && S_final != S0 && S0) {
-        const size_t bytes = (size_t)B * H * dk * dv * sizeof(float);
-        const char *a0 = (const char *)S0, *b0 = (const char *)S_final;
-        if (a0 < b0 + bytes && b0 < a0 + bytes)
-            return fail(GDN_ERR_INVALID_ARGUMENT, "gdn_chunk_fwd: S0 and S_final overlap partially");
-    }
-    const size_t need = chunk_workspace(B, T, H, dk, dv, varlen, dtype);
-    if (need > 0) {
-        if (!workspace || workspace_bytes < need)
-            return fail(GDN_ERR_WORKSPACE, "gdn_chunk_fwd: workspace of %zu bytes needed, %zu given", need,
-                        workspace ? workspace_bytes : (size_t)0);
-        if (reinterpret_cast<uintptr_t>(workspace) & 255u)
-            return fail(GDN_ERR_INVALID_ARGUMENT, "gdn_chunk_fwd: workspace must be 256-byte aligned");
-    }
-    ChunkArgs a{q, k, v, log_alpha, beta, S0, out, S_final, cu_seqlens, B, T, H, dk, dv, dtype,
-                workspace, workspace_bytes};
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
-    cudaError_t e = dtype == GDN_DTYPE_BF16 ? launch_chunk_tc(a, st) : launch_chunk_simt(a, st);
-    if (e != cudaSuccess) return cuda_fail(e, "gdn_chunk_fwd");
-    return GDN_OK;
+    return chunk_fwd_common("gdn_chunk_fwd", q, k, v, log_alpha, beta, S0, out, S_final, B, T, H, dk, dv,
+                            chunk, cu_seqlens, dtype, 0, 0.f, 0.f, workspace, workspace_bytes, stream);
+}
+
+int gdn_chunk_fwd_fused(const void *q_raw, const void *k_raw, const void *v, const float *a_raw,
+                        const float *b_raw, const float *S0, void *out, float *S_final, int B, int T,
+                        int H, int dk, int dv, int chunk, const int32_t *cu_seqlens, int dtype,
+                        float a_scale, float b_scale, void *workspace, size_t workspace_bytes,
+                        void *stream)
+{
+    g_last_error[0] = 0;
+    if (dtype != GDN_DTYPE_BF16)
+        return fail(GDN_ERR_UNSUPPORTED, "gdn_chunk_fwd_fused: dtype %d, supported: bf16", dtype);
+    if (!(a_scale >= 0.f) || !(a_scale < INFINITY))
+        return fail(GDN_ERR_INVALID_ARGUMENT, "gdn_chunk_fwd_fused: a_scale %g, must be finite and >= 0",
+                    (double)a_scale);
+    if (!(b_scale >= 0.f && b_scale <= 2.f))
+        return fail(GDN_ERR_INVALID_ARGUMENT, "gdn_chunk_fwd_fused: b_scale %g, must lie in [0, 2]",
+                    (double)b_scale);
+    return chunk_fwd_common("gdn_chunk_fwd_fused", q_raw, k_raw, v, a_raw, b_raw, S0, out, S_final, B, T, H,
+                            dk, dv, chunk, cu_seqlens, dtype, 1, a_scale, b_scale, workspace,
+                            workspace_bytes, stream);
 }
 
 int gdn_decode_step(const void *q, const void *k, const void *v, const float *log_alpha,

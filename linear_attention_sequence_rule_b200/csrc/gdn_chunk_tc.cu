@@ -57,6 +57,11 @@ constexpr int LDF = 68;  // fp32 row stride of the 64 x 64 solve matrices
 // initial state is the identity (dv must equal dk).  With out == nullptr no output is formed.
 constexpr int kFlagVZero = 1;
 constexpr int kFlagS0Identity = 2;
+// Fused prologue: q and k arrive unnormalised and the gate arrays hold raw projections a, b;
+// rows are divided by sqrt(|x|^2 + kNormEps) and log alpha = -a_scale softplus(a),
+// beta = b_scale sigmoid(b) (DeltaPhase README, section 1: beta = 2 sigmoid(W_beta x)).
+constexpr int kFlagPrologue = 4;
+constexpr float kNormEps = 1e-6f;
 
 template <int DK, int DV>
 struct TcCfg {
@@ -325,6 +330,54 @@ __device__ void solve_unit_lower(const float *A, const TOut &out, float *__restr
     }
 }
 
+// Gate forms of the fused prologue (valid = the row lies inside the sequence; padded rows keep the
+// exact zeros of log alpha and beta that make them contribute nothing).
+__device__ __forceinline__ float prologue_log_alpha(float a, bool valid, float a_scale)
+{
+    if (!valid) return 0.f;
+    if (a == INFINITY) return -INFINITY;  // an exact reset
+    const float sp = a > 0.f ? a + log1pf(expf(-a)) : log1pf(expf(a));
+    return -a_scale * sp;
+}
+__device__ __forceinline__ float prologue_beta(float b, bool valid, float b_scale)
+{
+    return valid ? b_scale / (1.f + expf(-b)) : 0.f;
+}
+
+// Divide bf16 row `row` of a swizzled tile (NBLK blocks of 64 features at a 16 KB stride) by
+// sqrt(sum of squares + kNormEps), in fp32, rounding back to bf16.
+template <int NBLK>
+__device__ __forceinline__ void normalize_row_bf16(unsigned char *tile, int row)
+{
+    uint4 w[NBLK * 8];
+    float ss = 0.f;
+#pragma unroll
+    for (int b = 0; b < NBLK; ++b)
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            w[b * 8 + c] = *reinterpret_cast<const uint4 *>(tile + b * 16384 + row * 128 + ((c ^ (row & 7)) << 4));
+            const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&w[b * 8 + c]);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float2 f = __bfloat1622float2(h[e]);
+                ss = fmaf(f.x, f.x, fmaf(f.y, f.y, ss));
+            }
+        }
+    const float sc = rsqrtf(ss + kNormEps);
+#pragma unroll
+    for (int b = 0; b < NBLK; ++b)
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            __nv_bfloat162 *h = reinterpret_cast<__nv_bfloat162 *>(&w[b * 8 + c]);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float2 f = __bfloat1622float2(h[e]);
+                h[e] = __floats2bfloat162_rn(f.x * sc, f.y * sc);
+            }
+            *reinterpret_cast<uint4 *>(tile + b * 16384 + row * 128 + ((c ^ (row & 7)) << 4)) = w[b * 8 + c];
+        }
+}
+
 // Scale row r (64 bf16 = 128 swizzled bytes, 8 chunks of 16 B) of a tile by s: the caller owns
 // chunks [c0, c1) counted from position row % 8, so that the threads of a warp (consecutive rows)
 // touch 8 different bank groups at every step.  Packed bf16x2 multiplies (s rounded to bf16).
@@ -342,13 +395,16 @@ __device__ __forceinline__ void scale_row_bf16(unsigned char *tile, int row, flo
     }
 }
 
-template <int DK, int DV>
+// PRO: fused prologue (kFlagPrologue), a separate instantiation so that the plain path carries
+// none of its code.
+template <int DK, int DV, bool PRO>
 __global__ void __launch_bounds__(TcCfg<DK, DV>::THREADS, 1)
     chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const float *__restrict__ log_alpha,
                     const float *__restrict__ beta, const float *__restrict__ S0,
                     __nv_bfloat16 *__restrict__ out, float *__restrict__ S_final,
-                    const int32_t *__restrict__ cu_seqlens, int T, int H, int flags)
+                    const int32_t *__restrict__ cu_seqlens, int T, int H, int flags, float a_scale,
+                    float b_scale)
 {
     using L = TcCfg<DK, DV>;
     constexpr int NS = L::NS;
@@ -466,6 +522,12 @@ __global__ void __launch_bounds__(TcCfg<DK, DV>::THREADS, 1)
             // ---- Gram matrices [K; Q] K^T (issued first: they need no gates, so the scan below
             //      runs while they are in flight) ----
             ctl.wait(B::kq_full + st, (c / NS) & 1);
+            if (PRO) {
+                // fused prologue: unit rows of K (threads 0-63) and Q (threads 64-127)
+                normalize_row_bf16<DK / 64>(Kt + (t >= 64 ? 8192 : 0), t & 63);
+                fence_proxy_async_smem();
+                named_bar(bar_id, 128);
+            }
             if (t == kIssuer && !ctl.aborted()) {
                 tc_fence_after();
                 constexpr uint32_t id = idesc_bf16(128, 64, 0, 0);
@@ -480,7 +542,14 @@ __global__ void __launch_bounds__(TcCfg<DK, DV>::THREADS, 1)
             if (wi == scan_warp(wg)) {
                 ctl.wait(B::gfull + st, (c / NS) & 1);
                 const int r0 = 2 * lane, r1 = r0 + 1;
-                const float g0 = graw[r0], g1 = graw[r1];
+                float g0 = graw[r0], g1 = graw[r1];
+                if (PRO) {
+                    const int n = (int)min((long)CH, len - (long)c * CH);
+                    g0 = prologue_log_alpha(g0, r0 < n, a_scale);
+                    g1 = prologue_log_alpha(g1, r1 < n, a_scale);
+                    bet[r0] = prologue_beta(bet[r0], r0 < n, b_scale);
+                    bet[r1] = prologue_beta(bet[r1], r1 < n, b_scale);
+                }
                 const bool f0 = (g0 == -INFINITY), f1 = (g1 == -INFINITY);
                 const float v0 = f0 ? 0.f : g0, v1 = f1 ? 0.f : g1;
                 // inclusive pair value and reset flag, then a segmented warp scan over lanes
@@ -925,6 +994,7 @@ struct TcLaunch {
     int nseq, T, H;
     long tokens;  // rows of the q/k/v tensors
     int flags;
+    float a_scale, b_scale;  // fused prologue (kFlagPrologue)
 };
 
 template <int DK, int DV>
@@ -943,13 +1013,13 @@ cudaError_t launch_tc(const TcLaunch &a, cudaStream_t st)
         return cudaErrorInvalidValue;
     }
     const int smem = L::TOTAL + 1024;
-    auto kern = chunk_tc_kernel<DK, DV>;
+    auto kern = (a.flags & kFlagPrologue) ? chunk_tc_kernel<DK, DV, true> : chunk_tc_kernel<DK, DV, false>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     const dim3 grid(1, a.H, a.nseq);
     kern<<<grid, L::THREADS, smem, st>>>(mq, mk, mv, a.log_alpha, a.beta, a.S0,
                                        static_cast<__nv_bfloat16 *>(a.out), a.S_final, a.cu, a.T, a.H,
-                                       a.flags);
+                                       a.flags, a.a_scale, a.b_scale);
     return cudaGetLastError();
 }
 
@@ -1094,9 +1164,11 @@ cudaError_t run_chunk(const ChunkArgs &a, cudaStream_t st)
 {
     const long tokens = a.cu_seqlens ? (long)a.T : (long)a.B * a.T;
     const SegPlan p = plan_segments(a.B, a.T, a.H, a.cu_seqlens != nullptr, a.dtype);
+    const int pf = a.prologue ? kFlagPrologue : 0;
+    const float as = a.a_scale, bs = a.b_scale;
     if (p.G <= 1) {
         return launch_tc<DK, DV>(TcLaunch{a.q, a.k, a.v, a.log_alpha, a.beta, a.S0, a.out, a.S_final,
-                                          a.cu_seqlens, a.B, a.T, a.H, tokens, 0},
+                                          a.cu_seqlens, a.B, a.T, a.H, tokens, pf, as, bs},
                                  st);
     }
     const SegWork w = seg_layout(a.workspace, a.B, a.H, DK, DV, p);
@@ -1106,11 +1178,11 @@ cudaError_t run_chunk(const ChunkArgs &a, cudaStream_t st)
     if (e != cudaSuccess) return e;
     // pass A: local states from zero, and transitions from the identity with V = 0
     e = launch_tc<DK, DV>(TcLaunch{a.q, a.k, a.v, a.log_alpha, a.beta, nullptr, nullptr, w.Sloc, w.cu, nseg,
-                                   a.T, a.H, tokens, 0},
+                                   a.T, a.H, tokens, pf, as, bs},
                           st);
     if (e != cudaSuccess) return e;
     e = launch_tc<DK, DK>(TcLaunch{a.q, a.k, nullptr, a.log_alpha, a.beta, nullptr, nullptr, w.M, w.cu, nseg,
-                                   a.T, a.H, tokens, kFlagVZero | kFlagS0Identity},
+                                   a.T, a.H, tokens, kFlagVZero | kFlagS0Identity | pf, as, bs},
                           st);
     if (e != cudaSuccess) return e;
     // pass B: segment scan of the states
@@ -1121,7 +1193,7 @@ cudaError_t run_chunk(const ChunkArgs &a, cudaStream_t st)
     if (e != cudaSuccess) return e;
     // pass C: outputs of every segment from its entry state
     return launch_tc<DK, DV>(TcLaunch{a.q, a.k, a.v, a.log_alpha, a.beta, w.Sin, a.out, nullptr, w.cu, nseg,
-                                      a.T, a.H, tokens, 0},
+                                      a.T, a.H, tokens, pf, as, bs},
                              st);
 }
 

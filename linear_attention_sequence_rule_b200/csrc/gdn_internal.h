@@ -26,6 +26,9 @@ struct ChunkArgs {
     int B, T, H, dk, dv, dtype;
     void *workspace;
     size_t workspace_bytes;
+    // fused prologue (bf16 only): q, k unnormalised, log_alpha / beta hold the raw projections a, b
+    int prologue = 0;
+    float a_scale = 0.f, b_scale = 0.f;
 };
 
 // Chunk forward on CUDA cores, fp32 arithmetic throughout (fp32 inputs).

@@ -66,6 +66,30 @@ def test_chunk_fwd_rejects_bad_arguments(kw, code):
     assert gdn.gdn_last_error() != ""
 
 
+def fused(**kw):
+    a = dict(q_raw=FAKE, k_raw=FAKE, v=FAKE, a_raw=FAKE, b_raw=FAKE, S0=None, out=FAKE, S_final=None,
+             B=1, T=64, H=1, dk=64, dv=64, chunk=64, cu_seqlens=None, dtype=gdn.GDN_DTYPE_BF16,
+             a_scale=1.0, b_scale=1.0, workspace=None, workspace_bytes=0, stream=None)
+    a.update(kw)
+    return gdn.gdn_chunk_fwd_fused(**a)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(dtype=gdn.GDN_DTYPE_F32), gdn.GDN_ERR_UNSUPPORTED),
+    (dict(dk=96), gdn.GDN_ERR_UNSUPPORTED),
+    (dict(a_scale=-1.0), gdn.GDN_ERR_INVALID_ARGUMENT),
+    (dict(a_scale=float("inf")), gdn.GDN_ERR_INVALID_ARGUMENT),
+    (dict(a_scale=float("nan")), gdn.GDN_ERR_INVALID_ARGUMENT),
+    (dict(b_scale=2.5), gdn.GDN_ERR_INVALID_ARGUMENT),
+    (dict(b_scale=-0.1), gdn.GDN_ERR_INVALID_ARGUMENT),
+    (dict(b_raw=None), gdn.GDN_ERR_INVALID_ARGUMENT),
+    (dict(k_raw=FAKE + 4), gdn.GDN_ERR_INVALID_ARGUMENT),
+])
+def test_fused_chunk_fwd_rejects_bad_arguments(kw, code):
+    assert fused(**kw) == code
+    assert "gdn_chunk_fwd" in gdn.gdn_last_error()
+
+
 def test_workspace_query():
     assert gdn.gdn_chunk_fwd_workspace_bytes(1, 64, 1, 64, 64, 64, 0, 1) >= 0
     bad = ctypes.c_size_t(-1).value
