@@ -428,6 +428,33 @@ def run_ours(args, world, rank, local):
                           "ms": round(ms_w, 6), "tokens_per_s": round(main["tokens"] / (ms_w * 1e-3), 1),
                           "launches_per_call": 1 if fused else None}
         del dr
+        # grouped value heads: the hybrid-LM shape with 6 q/k heads for its 12 value heads
+        dg = to_dev(workloads.make_gva_chunk_inputs(B=8, T=4096, Hk=6, Hv=12, dk=64, dv=64, dtype="bf16",
+                                                    seed=rank_seed(cfg["seed"], rank), la_scale=0.1))
+        outg = torch.empty_like(dg["v"])
+        Sg = torch.empty((8, 12, 64, 64), dtype=torch.float32, device="cuda")
+
+        def call_gva():
+            gdn.chunk_fwd_gva(dg["q"], dg["k"], dg["v"], dg["log_alpha"], dg["beta"], out=outg, S_final=Sg,
+                              stream=stream)
+        with torch.cuda.stream(stream):
+            for _ in range(3):
+                flush.zero_()
+                call_gva()
+            stream.synchronize()
+            evg = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                   for _ in range(max(3, args.steps // 2))]
+            for a0, b0 in evg:
+                flush.zero_()
+                a0.record(stream)
+                call_gva()
+                b0.record(stream)
+            stream.synchronize()
+        ms_g = statistics.mean(a0.elapsed_time(b0) for a0, b0 in evg)
+        extra["hybrid_lm_gva"] = {"workload": "hybrid_lm shape, grouped value heads: Hk=6 q/k heads, Hv=12 value heads",
+                                  "ms": round(ms_g, 6), "tokens_per_s": round(8 * 4096 / (ms_g * 1e-3), 1),
+                                  "launches_per_call": 1}
+        del dg, outg, Sg
     cpu = None
     if rank == 0 and world == 1:
         cpu = cpu_oracle_baseline(inp)

@@ -118,6 +118,21 @@ GDN_API int gdn_chunk_fwd_fused(const void *q_raw, const void *k_raw, const void
                                 size_t workspace_bytes, void *stream);
 
 /*
+ * gdn_chunk_fwd_gva -- gdn_chunk_fwd with grouped value heads: Hv value heads share Hk q/k heads
+ * (Hv a multiple of Hk), value head h reading q/k head h / (Hv / Hk), as grouped-query attention
+ * shares key/value heads among query heads (Sykra README, "Architectural Highlights": GQA).
+ * Gates, values, outputs and states are per value head:
+ *   q,k [B,T,Hk,dk] (varlen [T,Hk,dk]); v,out [B,T,Hv,dv]; log_alpha,beta [B,T,Hv];
+ *   S0, S_final [B,Hv,dk,dv].
+ * Everything else (dtypes, varlen, workspace, in-place carry, errors) as gdn_chunk_fwd; query the
+ * workspace with H = Hv.  Hk = Hv is gdn_chunk_fwd.
+ */
+GDN_API int gdn_chunk_fwd_gva(const void *q, const void *k, const void *v, const float *log_alpha,
+                              const float *beta, const float *S0, void *out, float *S_final, int B, int T,
+                              int Hk, int Hv, int dk, int dv, int chunk, const int32_t *cu_seqlens,
+                              int dtype, void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * gdn_chunk_fwd_workspace_bytes -- device scratch that gdn_chunk_fwd needs for these sizes
  * (varlen: non-zero when cu_seqlens will be passed).  Returns 0 when no scratch is needed and
  * (size_t)-1 for arguments gdn_chunk_fwd would reject.
@@ -167,6 +182,15 @@ GDN_API int gdn_chunk_fwd_noalloc(const void *q, const void *k, const void *v, c
 GDN_API int gdn_decode_step(const void *q, const void *k, const void *v, const float *log_alpha,
                     const float *beta, float *S_inout, void *out, int N, int H, int dk, int dv,
                     int dtype, void *stream);
+
+/*
+ * gdn_decode_step_gva -- gdn_decode_step with grouped value heads (see gdn_chunk_fwd_gva):
+ * q,k [N,Hk,dk]; v,out [N,Hv,dv]; log_alpha,beta [N,Hv]; S_inout [N,Hv,dk,dv]; state (n, h)
+ * reads q/k head h / (Hv / Hk) of sequence n.
+ */
+GDN_API int gdn_decode_step_gva(const void *q, const void *k, const void *v, const float *log_alpha,
+                                const float *beta, float *S_inout, void *out, int N, int Hk, int Hv,
+                                int dk, int dv, int dtype, void *stream);
 
 /*
  * gdn_device_status -- synchronise `stream`, then report whether any kernel of this library

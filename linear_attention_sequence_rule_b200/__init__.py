@@ -6,7 +6,8 @@ PyTorch provides device memory and streams.  The binding has two layers:
 * ``gdn_chunk_fwd``, ``gdn_chunk_fwd_noalloc``, ``gdn_decode_step``, ``gdn_chunk_fwd_workspace_bytes``,
   ``gdn_status_string``, ``gdn_last_error``, ``gdn_version`` -- the C-ABI entry points of
   ``include/gdn.h`` with the same names and arguments (pointers as Python ints);
-* ``chunk_fwd``, ``chunk_fwd_fused`` and ``decode_step`` -- the same calls taking torch tensors; they check shapes,
+* ``chunk_fwd``, ``chunk_fwd_fused``, ``chunk_fwd_gva``, ``decode_step`` and ``decode_step_gva`` --
+  the same calls taking torch tensors; they check shapes,
   devices and dtypes, allocate outputs with torch when none are given, and raise ``GdnError``
   on a non-zero status.
 
@@ -22,9 +23,10 @@ import torch
 __all__ = [
     "GdnError", "GDN_OK", "GDN_ERR_INVALID_ARGUMENT", "GDN_ERR_UNSUPPORTED", "GDN_ERR_WORKSPACE",
     "GDN_ERR_CUDA", "GDN_ERR_TIMEOUT", "GDN_DTYPE_F32", "GDN_DTYPE_BF16", "LIB_PATH",
-    "gdn_chunk_fwd", "gdn_chunk_fwd_noalloc", "gdn_chunk_fwd_fused", "gdn_decode_step", "gdn_chunk_fwd_workspace_bytes", "gdn_status_string",
+    "gdn_chunk_fwd", "gdn_chunk_fwd_noalloc", "gdn_chunk_fwd_fused", "gdn_chunk_fwd_gva",
+    "gdn_decode_step", "gdn_decode_step_gva", "gdn_chunk_fwd_workspace_bytes", "gdn_status_string",
     "gdn_last_error", "gdn_version", "gdn_device_status", "device_status", "chunk_fwd", "chunk_fwd_fused",
-    "decode_step", "workspace_bytes",
+    "chunk_fwd_gva", "decode_step", "decode_step_gva", "workspace_bytes",
 ]
 
 GDN_OK = 0
@@ -52,6 +54,11 @@ _lib.gdn_chunk_fwd.restype = _i
 _lib.gdn_chunk_fwd_fused.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i,
                                      _vp, _i, ctypes.c_float, ctypes.c_float, _vp, _sz, _vp]
 _lib.gdn_chunk_fwd_fused.restype = _i
+_lib.gdn_chunk_fwd_gva.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i,
+                                   _vp, _i, _vp, _sz, _vp]
+_lib.gdn_chunk_fwd_gva.restype = _i
+_lib.gdn_decode_step_gva.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp]
+_lib.gdn_decode_step_gva.restype = _i
 _lib.gdn_chunk_fwd_noalloc.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i,
                                        _i, _vp, _i, _vp]
 _lib.gdn_chunk_fwd_noalloc.restype = _i
@@ -88,6 +95,18 @@ def gdn_chunk_fwd_fused(q_raw, k_raw, v, a_raw, b_raw, S0, out, S_final, B, T, H
     return _lib.gdn_chunk_fwd_fused(q_raw, k_raw, v, a_raw, b_raw, S0, out, S_final, B, T, H, dk, dv,
                                     chunk, cu_seqlens, dtype, a_scale, b_scale, workspace,
                                     workspace_bytes, stream)
+
+
+def gdn_chunk_fwd_gva(q, k, v, log_alpha, beta, S0, out, S_final, B, T, Hk, Hv, dk, dv, chunk,
+                      cu_seqlens, dtype, workspace, workspace_bytes, stream) -> int:
+    return _lib.gdn_chunk_fwd_gva(q, k, v, log_alpha, beta, S0, out, S_final, B, T, Hk, Hv, dk, dv, chunk,
+                                  cu_seqlens, dtype, workspace, workspace_bytes, stream)
+
+
+def gdn_decode_step_gva(q, k, v, log_alpha, beta, S_inout, out, N, Hk, Hv, dk, dv, dtype,
+                        stream) -> int:
+    return _lib.gdn_decode_step_gva(q, k, v, log_alpha, beta, S_inout, out, N, Hk, Hv, dk, dv, dtype,
+                                    stream)
 
 
 def gdn_chunk_fwd_noalloc(q, k, v, log_alpha, beta, S0, out, S_final, B, T, H, dk, dv, chunk,
@@ -163,23 +182,24 @@ def workspace_bytes(B, T, H, dk, dv, varlen=False, dtype=torch.bfloat16, chunk=6
 
 
 def _chunk_prepare(q, k, v, ga, gb, S0, cu_seqlens, out, S_final, output_final_state, workspace,
-                   chunk, names):
+                   chunk, names, grouped=False):
     """Shape/device/dtype checks and output/workspace allocation shared by the chunk entries."""
     dt = q.dtype
     if dt not in _DT:
         raise ValueError(f"unsupported dtype {dt}")
     dev = q.device
     if cu_seqlens is not None:
-        T, H, dk = q.shape
+        T, Hk, dk = q.shape
         B = cu_seqlens.shape[0] - 1
         lead = (T,)
         _need(cu_seqlens, "cu_seqlens", torch.int32, (B + 1,), dev)
     else:
-        B, T, H, dk = q.shape
+        B, T, Hk, dk = q.shape
         lead = (B, T)
     dv = v.shape[-1]
-    _need(q, names[0], dt, (*lead, H, dk), dev)
-    _need(k, names[1], dt, (*lead, H, dk), dev)
+    H = v.shape[-2] if grouped else Hk  # value heads
+    _need(q, names[0], dt, (*lead, Hk, dk), dev)
+    _need(k, names[1], dt, (*lead, Hk, dk), dev)
     _need(v, "v", dt, (*lead, H, dv), dev)
     _need(ga, names[2], torch.float32, (*lead, H), dev)
     _need(gb, names[3], torch.float32, (*lead, H), dev)
@@ -196,8 +216,8 @@ def _chunk_prepare(q, k, v, ga, gb, S0, cu_seqlens, out, S_final, output_final_s
     if need and workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=dev)
     wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    return dict(B=B, T=T, H=H, dk=dk, dv=dv, dt=dt, out=out, S_final=S_final, workspace=workspace,
-                wbytes=wbytes)
+    return dict(B=B, T=T, H=H, Hk=Hk, dk=dk, dv=dv, dt=dt, out=out, S_final=S_final,
+                workspace=workspace, wbytes=wbytes)
 
 
 def chunk_fwd(q, k, v, log_alpha, beta, S0=None, cu_seqlens=None, out=None, S_final=None,
@@ -230,6 +250,47 @@ def chunk_fwd_fused(q_raw, k_raw, v, a_raw, b_raw, a_scale, b_scale, S0=None, cu
     if rc != GDN_OK:
         raise GdnError(rc, gdn_last_error())
     return p["out"], p["S_final"]
+
+
+def chunk_fwd_gva(q, k, v, log_alpha, beta, S0=None, cu_seqlens=None, out=None, S_final=None,
+                  output_final_state=True, workspace=None, chunk=64, stream=None):
+    """Chunkwise forward with grouped value heads: q,k [B,T,Hk,dk], v [B,T,Hv,dv], gates
+    [B,T,Hv], states [B,Hv,dk,dv]; value head h reads q/k head h // (Hv // Hk).  Returns
+    (out [B,T,Hv,dv], S_final or None)."""
+    p = _chunk_prepare(q, k, v, log_alpha, beta, S0, cu_seqlens, out, S_final, output_final_state,
+                       workspace, chunk, ("q", "k", "log_alpha", "beta"), grouped=True)
+    rc = gdn_chunk_fwd_gva(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(S0),
+                           _ptr(p["out"]), _ptr(p["S_final"]), p["B"], p["T"], p["Hk"], p["H"], p["dk"],
+                           p["dv"], chunk, _ptr(cu_seqlens), _DT[p["dt"]], _ptr(p["workspace"]),
+                           p["wbytes"], _stream_ptr(stream))
+    if rc != GDN_OK:
+        raise GdnError(rc, gdn_last_error())
+    return p["out"], p["S_final"]
+
+
+def decode_step_gva(q, k, v, log_alpha, beta, S, out=None, stream=None):
+    """One decode step with grouped value heads: q,k [N,Hk,dk], v [N,Hv,dv], gates [N,Hv],
+    S [N,Hv,dk,dv] fp32 updated in place.  Returns out [N,Hv,dv]."""
+    dt = q.dtype
+    if dt not in _DT:
+        raise ValueError(f"unsupported dtype {dt}")
+    dev = q.device
+    N, Hk, dk = q.shape
+    Hv, dv = v.shape[-2], v.shape[-1]
+    _need(q, "q", dt, (N, Hk, dk), dev)
+    _need(k, "k", dt, (N, Hk, dk), dev)
+    _need(v, "v", dt, (N, Hv, dv), dev)
+    _need(log_alpha, "log_alpha", torch.float32, (N, Hv), dev)
+    _need(beta, "beta", torch.float32, (N, Hv), dev)
+    _need(S, "S", torch.float32, (N, Hv, dk, dv), dev)
+    if out is None:
+        out = torch.empty((N, Hv, dv), dtype=dt, device=dev)
+    _need(out, "out", dt, (N, Hv, dv), dev)
+    rc = gdn_decode_step_gva(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(S), _ptr(out),
+                             N, Hk, Hv, dk, dv, _DT[dt], _stream_ptr(stream))
+    if rc != GDN_OK:
+        raise GdnError(rc, gdn_last_error())
+    return out
 
 
 def decode_step(q, k, v, log_alpha, beta, S, out=None, stream=None):

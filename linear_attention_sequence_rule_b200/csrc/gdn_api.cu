@@ -102,7 +102,8 @@ static int chunk_fwd_common(const char *fn, const void *q, const void *k, const 
                             const float *log_alpha, const float *beta, const float *S0, void *out,
                             float *S_final, int B, int T, int H, int dk, int dv, int chunk,
                             const int32_t *cu_seqlens, int dtype, int prologue, float a_scale,
-                            float b_scale, void *workspace, size_t workspace_bytes, void *stream)
+                            float b_scale, void *workspace, size_t workspace_bytes, void *stream,
+                            int G = 1)
 {
     const int varlen = cu_seqlens != nullptr;
     int rc = check_chunk_shape(B, T, H, dk, dv, chunk, varlen, dtype);
@@ -128,7 +129,7 @@ static int chunk_fwd_common(const char *fn, const void *q, const void *k, const 
             return fail(GDN_ERR_INVALID_ARGUMENT, "%s: workspace must be 256-byte aligned", fn);
     }
     ChunkArgs a{q, k, v, log_alpha, beta, S0, out, S_final, cu_seqlens, B, T, H, dk, dv, dtype,
-                workspace, workspace_bytes, prologue, a_scale, b_scale};
+                workspace, workspace_bytes, prologue, a_scale, b_scale, G};
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     cudaError_t e = dtype == GDN_DTYPE_BF16 ? launch_chunk_tc(a, st) : launch_chunk_simt(a, st);
     if (e != cudaSuccess) return cuda_fail(e, fn);
@@ -167,27 +168,72 @@ int gdn_chunk_fwd_fused(const void *q_raw, const void *k_raw, const void *v, con
                             workspace_bytes, stream);
 }
 
+namespace gdn {
+
+static int decode_common(const char *fn, const void *q, const void *k, const void *v, const float *log_alpha,
+                         const float *beta, float *S_inout, void *out, int N, int H, int G, int dk, int dv,
+                         int dtype, void *stream)
+{
+    if (dtype != GDN_DTYPE_BF16 && dtype != GDN_DTYPE_F32)
+        return fail(GDN_ERR_UNSUPPORTED, "%s: unknown dtype %d", fn, dtype);
+    if (!head_dim_ok(dk) || !head_dim_ok(dv))
+        return fail(GDN_ERR_UNSUPPORTED, "%s: dk=%d dv=%d, supported: 64 or 128", fn, dk, dv);
+    if (N < 1 || H < 1 || (long long)N * H > (1LL << 30))
+        return fail(GDN_ERR_INVALID_ARGUMENT, "%s: N=%d H=%d out of range", fn, N, H);
+    if (!q || !k || !v || !log_alpha || !beta || !S_inout || !out)
+        return fail(GDN_ERR_INVALID_ARGUMENT, "%s: every pointer is required", fn);
+    const void *ptrs[] = {q, k, v, log_alpha, beta, S_inout, out};
+    for (const void *p : ptrs)
+        if (!aligned16(p))
+            return fail(GDN_ERR_INVALID_ARGUMENT, "%s: pointer %p is not 16-byte aligned", fn, p);
+    cudaError_t e = launch_decode(q, k, v, log_alpha, beta, S_inout, out, N, H, dk, dv, dtype,
+                                  static_cast<cudaStream_t>(stream), G);
+    if (e != cudaSuccess) return cuda_fail(e, fn);
+    return GDN_OK;
+}
+
+// Head counts of the grouped-value-head entries: Hv value heads share Hk q/k heads.
+static int check_groups(const char *fn, int Hk, int Hv)
+{
+    if (Hk < 1 || Hv < 1 || Hv % Hk != 0)
+        return fail(GDN_ERR_INVALID_ARGUMENT, "%s: Hk=%d Hv=%d, need Hk >= 1 and Hv a multiple of Hk", fn, Hk,
+                    Hv);
+    return GDN_OK;
+}
+
+}  // namespace gdn
+
 int gdn_decode_step(const void *q, const void *k, const void *v, const float *log_alpha,
                     const float *beta, float *S_inout, void *out, int N, int H, int dk, int dv,
                     int dtype, void *stream)
 {
     g_last_error[0] = 0;
-    if (dtype != GDN_DTYPE_BF16 && dtype != GDN_DTYPE_F32)
-        return fail(GDN_ERR_UNSUPPORTED, "gdn_decode_step: unknown dtype %d", dtype);
-    if (!head_dim_ok(dk) || !head_dim_ok(dv))
-        return fail(GDN_ERR_UNSUPPORTED, "gdn_decode_step: dk=%d dv=%d, supported: 64 or 128", dk, dv);
-    if (N < 1 || H < 1 || (long long)N * H > (1LL << 30))
-        return fail(GDN_ERR_INVALID_ARGUMENT, "gdn_decode_step: N=%d H=%d out of range", N, H);
-    if (!q || !k || !v || !log_alpha || !beta || !S_inout || !out)
-        return fail(GDN_ERR_INVALID_ARGUMENT, "gdn_decode_step: every pointer is required");
-    const void *ptrs[] = {q, k, v, log_alpha, beta, S_inout, out};
-    for (const void *p : ptrs)
-        if (!aligned16(p))
-            return fail(GDN_ERR_INVALID_ARGUMENT, "gdn_decode_step: pointer %p is not 16-byte aligned", p);
-    cudaError_t e = launch_decode(q, k, v, log_alpha, beta, S_inout, out, N, H, dk, dv, dtype,
-                                  static_cast<cudaStream_t>(stream));
-    if (e != cudaSuccess) return cuda_fail(e, "gdn_decode_step");
-    return GDN_OK;
+    return decode_common("gdn_decode_step", q, k, v, log_alpha, beta, S_inout, out, N, H, 1, dk, dv, dtype,
+                         stream);
+}
+
+int gdn_decode_step_gva(const void *q, const void *k, const void *v, const float *log_alpha,
+                        const float *beta, float *S_inout, void *out, int N, int Hk, int Hv, int dk,
+                        int dv, int dtype, void *stream)
+{
+    g_last_error[0] = 0;
+    const int rc = check_groups("gdn_decode_step_gva", Hk, Hv);
+    if (rc != GDN_OK) return rc;
+    return decode_common("gdn_decode_step_gva", q, k, v, log_alpha, beta, S_inout, out, N, Hv, Hv / Hk, dk,
+                         dv, dtype, stream);
+}
+
+int gdn_chunk_fwd_gva(const void *q, const void *k, const void *v, const float *log_alpha,
+                      const float *beta, const float *S0, void *out, float *S_final, int B, int T,
+                      int Hk, int Hv, int dk, int dv, int chunk, const int32_t *cu_seqlens, int dtype,
+                      void *workspace, size_t workspace_bytes, void *stream)
+{
+    g_last_error[0] = 0;
+    const int rc = check_groups("gdn_chunk_fwd_gva", Hk, Hv);
+    if (rc != GDN_OK) return rc;
+    return chunk_fwd_common("gdn_chunk_fwd_gva", q, k, v, log_alpha, beta, S0, out, S_final, B, T, Hv, dk, dv,
+                            chunk, cu_seqlens, dtype, 0, 0.f, 0.f, workspace, workspace_bytes, stream,
+                            Hv / Hk);
 }
 
 int gdn_device_status(void *stream)

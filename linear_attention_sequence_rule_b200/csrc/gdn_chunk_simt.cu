@@ -61,7 +61,7 @@ __global__ void __launch_bounds__(kThreads)
 chunk_simt_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const TIn *__restrict__ v,
                   const float *__restrict__ log_alpha, const float *__restrict__ beta,
                   const float *__restrict__ S0, TIn *__restrict__ out, float *__restrict__ S_final,
-                  const int32_t *__restrict__ cu_seqlens, int T, int H, int DV)
+                  const int32_t *__restrict__ cu_seqlens, int T, int H, int DV, int G)
 {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     SimtSmem<DK> &sm = *reinterpret_cast<SimtSmem<DK> *>(smem_raw);
@@ -92,7 +92,7 @@ chunk_simt_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const TI
             const int r = idx / DK, c = idx % DK;
             float qv = 0.f, kv = 0.f;
             if (r < n) {
-                const size_t off = ((size_t)(tok0 + c0 + r) * H + h) * DK + c;
+                const size_t off = ((size_t)(tok0 + c0 + r) * (H / G) + h / G) * DK + c;  // q/k head h / G
                 qv = ld_f32(q + off);
                 kv = ld_f32(k + off);
             }
@@ -233,7 +233,7 @@ cudaError_t launch_dk(const ChunkArgs &a, cudaStream_t st)
     kern<<<grid, kThreads, smem, st>>>(
         static_cast<const TIn *>(a.q), static_cast<const TIn *>(a.k), static_cast<const TIn *>(a.v),
         a.log_alpha, a.beta, a.S0, static_cast<TIn *>(a.out), a.S_final, a.cu_seqlens, a.T, a.H,
-        a.dv);
+        a.dv, a.G);
     return cudaGetLastError();
 }
 

@@ -404,7 +404,7 @@ __global__ void __launch_bounds__(TcCfg<DK, DV>::THREADS, 1)
                     const float *__restrict__ beta, const float *__restrict__ S0,
                     __nv_bfloat16 *__restrict__ out, float *__restrict__ S_final,
                     const int32_t *__restrict__ cu_seqlens, int T, int H, int flags, float a_scale,
-                    float b_scale)
+                    float b_scale, int G)
 {
     using L = TcCfg<DK, DV>;
     constexpr int NS = L::NS;
@@ -425,6 +425,7 @@ __global__ void __launch_bounds__(TcCfg<DK, DV>::THREADS, 1)
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int h = blockIdx.y, s = blockIdx.z;
+    const int hq = G == 1 ? h : h / G;  // q/k head of value head h (G value heads share one q/k head)
     long tok0, len;
     if (cu_seqlens) {
         tok0 = cu_seqlens[s];
@@ -470,8 +471,8 @@ __global__ void __launch_bounds__(TcCfg<DK, DV>::THREADS, 1)
             mbar_arrive_expect_tx(&bars[B::kq_full + st], (DK / 64) * 16384);
             unsigned char *kq = sm + L::KQ + st * L::KQ_STAGE;
             for (int kb = 0; kb < DK / 64; ++kb) {
-                tma_load_3d(kq + kb * 16384, &tmK, &bars[B::kq_full + st], kb * 64, h, (int)tk);
-                tma_load_3d(kq + kb * 16384 + 8192, &tmQ, &bars[B::kq_full + st], kb * 64, h, (int)tk);
+                tma_load_3d(kq + kb * 16384, &tmK, &bars[B::kq_full + st], kb * 64, hq, (int)tk);
+                tma_load_3d(kq + kb * 16384 + 8192, &tmQ, &bars[B::kq_full + st], kb * 64, hq, (int)tk);
             }
         }
     };
@@ -991,10 +992,11 @@ struct TcLaunch {
     void *out;
     float *S_final;
     const int32_t *cu;
-    int nseq, T, H;
+    int nseq, T, H;  // H value heads; H / G q/k heads
     long tokens;  // rows of the q/k/v tensors
     int flags;
     float a_scale, b_scale;  // fused prologue (kFlagPrologue)
+    int G;                   // value heads per q/k head
 };
 
 template <int DK, int DV>
@@ -1005,10 +1007,12 @@ cudaError_t launch_tc(const TcLaunch &a, cudaStream_t st)
     // a zero-token varlen call still launches so that S_final = S0 is written
     const long map_tokens = a.tokens > 0 ? a.tokens : 1;
     // with V taken as zero nothing is loaded through the V map; any valid map will do
+    // with V taken as zero the V map is never read: the k map (H / G heads) serves as a stand-in
     const void *vsrc = (a.flags & kFlagVZero) ? a.k : a.v;
     const int vdim = (a.flags & kFlagVZero) ? DK : DV;
-    if (!make_map(&mq, a.q, map_tokens, a.H, DK) || !make_map(&mk, a.k, map_tokens, a.H, DK) ||
-        !make_map(&mv, vsrc, map_tokens, a.H, vdim)) {
+    const int vheads = (a.flags & kFlagVZero) ? a.H / a.G : a.H;
+    if (!make_map(&mq, a.q, map_tokens, a.H / a.G, DK) || !make_map(&mk, a.k, map_tokens, a.H / a.G, DK) ||
+        !make_map(&mv, vsrc, map_tokens, vheads, vdim)) {
         set_error("cuTensorMapEncodeTiled failed");
         return cudaErrorInvalidValue;
     }
@@ -1019,7 +1023,7 @@ cudaError_t launch_tc(const TcLaunch &a, cudaStream_t st)
     const dim3 grid(1, a.H, a.nseq);
     kern<<<grid, L::THREADS, smem, st>>>(mq, mk, mv, a.log_alpha, a.beta, a.S0,
                                        static_cast<__nv_bfloat16 *>(a.out), a.S_final, a.cu, a.T, a.H,
-                                       a.flags, a.a_scale, a.b_scale);
+                                       a.flags, a.a_scale, a.b_scale, a.G);
     return cudaGetLastError();
 }
 
@@ -1168,7 +1172,7 @@ cudaError_t run_chunk(const ChunkArgs &a, cudaStream_t st)
     const float as = a.a_scale, bs = a.b_scale;
     if (p.G <= 1) {
         return launch_tc<DK, DV>(TcLaunch{a.q, a.k, a.v, a.log_alpha, a.beta, a.S0, a.out, a.S_final,
-                                          a.cu_seqlens, a.B, a.T, a.H, tokens, pf, as, bs},
+                                          a.cu_seqlens, a.B, a.T, a.H, tokens, pf, as, bs, a.G},
                                  st);
     }
     const SegWork w = seg_layout(a.workspace, a.B, a.H, DK, DV, p);
@@ -1178,11 +1182,11 @@ cudaError_t run_chunk(const ChunkArgs &a, cudaStream_t st)
     if (e != cudaSuccess) return e;
     // pass A: local states from zero, and transitions from the identity with V = 0
     e = launch_tc<DK, DV>(TcLaunch{a.q, a.k, a.v, a.log_alpha, a.beta, nullptr, nullptr, w.Sloc, w.cu, nseg,
-                                   a.T, a.H, tokens, pf, as, bs},
+                                   a.T, a.H, tokens, pf, as, bs, a.G},
                           st);
     if (e != cudaSuccess) return e;
     e = launch_tc<DK, DK>(TcLaunch{a.q, a.k, nullptr, a.log_alpha, a.beta, nullptr, nullptr, w.M, w.cu, nseg,
-                                   a.T, a.H, tokens, kFlagVZero | kFlagS0Identity | pf, as, bs},
+                                   a.T, a.H, tokens, kFlagVZero | kFlagS0Identity | pf, as, bs, a.G},
                           st);
     if (e != cudaSuccess) return e;
     // pass B: segment scan of the states
@@ -1193,7 +1197,7 @@ cudaError_t run_chunk(const ChunkArgs &a, cudaStream_t st)
     if (e != cudaSuccess) return e;
     // pass C: outputs of every segment from its entry state
     return launch_tc<DK, DV>(TcLaunch{a.q, a.k, a.v, a.log_alpha, a.beta, w.Sin, a.out, nullptr, w.cu, nseg,
-                                      a.T, a.H, tokens, pf, as, bs},
+                                      a.T, a.H, tokens, pf, as, bs, a.G},
                              st);
 }
 

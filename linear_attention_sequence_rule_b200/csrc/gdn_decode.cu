@@ -35,7 +35,7 @@ template <int DK, int DV, typename TIn>
 __global__ void __launch_bounds__(kThreads, 2)
 decode_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const TIn *__restrict__ v,
               const float *__restrict__ log_alpha, const float *__restrict__ beta,
-              float *__restrict__ S, TIn *__restrict__ out)
+              float *__restrict__ S, TIn *__restrict__ out, int H, int G)
 {
     constexpr int TPR = DV / 4;          // threads per state row (one float4 each)
     constexpr int RPP = kThreads / TPR;  // rows covered per pass
@@ -56,8 +56,10 @@ decode_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const TIn *_
 #pragma unroll
     for (int p = 0; p < R; ++p) s[p] = __ldcs(&Sp[(rg + p * RPP) * TPR + c4]);
 
-    const TIn *kp = k + u * DK;
-    const TIn *qp = q + u * DK;
+    // q/k of state (n, h) live at (n, h / G) among the H / G q/k heads (grouped value heads)
+    const size_t uq = G == 1 ? u : (size_t)((unsigned)u / (unsigned)H) * (unsigned)(H / G) + ((unsigned)u % (unsigned)H) / (unsigned)G;
+    const TIn *kp = k + uq * DK;
+    const TIn *qp = q + uq * DK;
     float kr[R], qr[R];
 #pragma unroll
     for (int p = 0; p < R; ++p) {
@@ -122,17 +124,17 @@ decode_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const TIn *_
 
 template <typename TIn>
 cudaError_t launch_typed(const void *q, const void *k, const void *v, const float *la,
-                         const float *be, float *S, void *out, int NH, int dk, int dv,
+                         const float *be, float *S, void *out, int NH, int H, int G, int dk, int dv,
                          cudaStream_t st)
 {
     const dim3 grid(NH), block(kThreads);
     const TIn *Q = static_cast<const TIn *>(q), *K = static_cast<const TIn *>(k),
               *V = static_cast<const TIn *>(v);
     TIn *O = static_cast<TIn *>(out);
-    if (dk == 128 && dv == 128) decode_kernel<128, 128, TIn><<<grid, block, 0, st>>>(Q, K, V, la, be, S, O);
-    else if (dk == 128 && dv == 64) decode_kernel<128, 64, TIn><<<grid, block, 0, st>>>(Q, K, V, la, be, S, O);
-    else if (dk == 64 && dv == 128) decode_kernel<64, 128, TIn><<<grid, block, 0, st>>>(Q, K, V, la, be, S, O);
-    else decode_kernel<64, 64, TIn><<<grid, block, 0, st>>>(Q, K, V, la, be, S, O);
+    if (dk == 128 && dv == 128) decode_kernel<128, 128, TIn><<<grid, block, 0, st>>>(Q, K, V, la, be, S, O, H, G);
+    else if (dk == 128 && dv == 64) decode_kernel<128, 64, TIn><<<grid, block, 0, st>>>(Q, K, V, la, be, S, O, H, G);
+    else if (dk == 64 && dv == 128) decode_kernel<64, 128, TIn><<<grid, block, 0, st>>>(Q, K, V, la, be, S, O, H, G);
+    else decode_kernel<64, 64, TIn><<<grid, block, 0, st>>>(Q, K, V, la, be, S, O, H, G);
     return cudaGetLastError();
 }
 
@@ -140,12 +142,12 @@ cudaError_t launch_typed(const void *q, const void *k, const void *v, const floa
 
 cudaError_t launch_decode(const void *q, const void *k, const void *v, const float *log_alpha,
                           const float *beta, float *S, void *out, int N, int H, int dk, int dv,
-                          int dtype, cudaStream_t stream)
+                          int dtype, cudaStream_t stream, int G)
 {
     const int NH = N * H;
     if (dtype == GDN_DTYPE_BF16)
-        return launch_typed<__nv_bfloat16>(q, k, v, log_alpha, beta, S, out, NH, dk, dv, stream);
-    return launch_typed<float>(q, k, v, log_alpha, beta, S, out, NH, dk, dv, stream);
+        return launch_typed<__nv_bfloat16>(q, k, v, log_alpha, beta, S, out, NH, H, G, dk, dv, stream);
+    return launch_typed<float>(q, k, v, log_alpha, beta, S, out, NH, H, G, dk, dv, stream);
 }
 
 }  // namespace gdn

@@ -15,7 +15,7 @@ void set_error(const char *fmt, ...);
 // C-ABI layer and return the cudaError_t of the launch.
 cudaError_t launch_decode(const void *q, const void *k, const void *v, const float *log_alpha,
                           const float *beta, float *S, void *out, int N, int H, int dk, int dv,
-                          int dtype, cudaStream_t stream);
+                          int dtype, cudaStream_t stream, int G = 1);
 
 struct ChunkArgs {
     const void *q, *k, *v;
@@ -29,6 +29,8 @@ struct ChunkArgs {
     // fused prologue (bf16 only): q, k unnormalised, log_alpha / beta hold the raw projections a, b
     int prologue = 0;
     float a_scale = 0.f, b_scale = 0.f;
+    // grouped value heads: H value heads, H / G q/k heads; value head h reads q/k head h / G
+    int G = 1;
 };
 
 // Chunk forward on CUDA cores, fp32 arithmetic throughout (fp32 inputs).

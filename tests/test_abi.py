@@ -90,6 +90,21 @@ def test_fused_chunk_fwd_rejects_bad_arguments(kw, code):
     assert "gdn_chunk_fwd" in gdn.gdn_last_error()
 
 
+def test_grouped_entries_reject_bad_head_counts():
+    base = dict(q=FAKE, k=FAKE, v=FAKE, log_alpha=FAKE, beta=FAKE, S0=None, out=FAKE, S_final=None,
+                B=1, T=64, dk=64, dv=64, chunk=64, cu_seqlens=None, dtype=gdn.GDN_DTYPE_BF16,
+                workspace=None, workspace_bytes=0, stream=None)
+    for Hk, Hv in ((2, 3), (0, 4), (4, 2), (2, 0)):
+        assert gdn.gdn_chunk_fwd_gva(Hk=Hk, Hv=Hv, **base) == gdn.GDN_ERR_INVALID_ARGUMENT
+        assert "gdn_chunk_fwd_gva" in gdn.gdn_last_error()
+        assert gdn.gdn_decode_step_gva(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, Hk, Hv, 64, 64,
+                                       gdn.GDN_DTYPE_BF16, None) == gdn.GDN_ERR_INVALID_ARGUMENT
+    # a valid grouping still meets the ordinary checks
+    assert gdn.gdn_chunk_fwd_gva(Hk=2, Hv=4, **(base | dict(dk=96))) == gdn.GDN_ERR_UNSUPPORTED
+    assert gdn.gdn_decode_step_gva(FAKE, FAKE + 4, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 2, 4, 64, 64,
+                                   gdn.GDN_DTYPE_BF16, None) == gdn.GDN_ERR_INVALID_ARGUMENT
+
+
 def test_workspace_query():
     assert gdn.gdn_chunk_fwd_workspace_bytes(1, 64, 1, 64, 64, 64, 0, 1) >= 0
     bad = ctypes.c_size_t(-1).value

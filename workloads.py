@@ -130,6 +130,34 @@ def config_raw_inputs(name: str, **overrides):
     return make_raw_chunk_inputs(**cfg)
 
 
+def make_gva_chunk_inputs(B=None, T=None, Hk=2, Hv=4, dk=64, dv=64, dtype="bf16", seed=0,
+                          beta_scale=1.0, la_std=1.0, la_scale=1.0, s0_std=0.0, lengths=None, **_ignored):
+    """Inputs for a grouped-value-head chunk forward: q,k [..., Hk, dk] L2-normalised as in
+    ``make_chunk_inputs``; v [..., Hv, dv]; gates [..., Hv]; S0 [B, Hv, dk, dv]."""
+    g = torch.Generator().manual_seed(int(seed))
+    dt = DTYPES[dtype]
+    if lengths is not None:
+        lengths = [int(x) for x in lengths]
+        cu = torch.zeros(len(lengths) + 1, dtype=torch.int32)
+        cu[1:] = torch.cumsum(torch.tensor(lengths, dtype=torch.int64), 0).to(torch.int32)
+        lead = (int(cu[-1]),)
+        nseq = len(lengths)
+    else:
+        cu = None
+        lead = (int(B), int(T))
+        nseq = int(B)
+    q = _unit_rows(torch.randn(*lead, Hk, dk, generator=g)).to(dt)
+    k = _unit_rows(torch.randn(*lead, Hk, dk, generator=g)).to(dt)
+    v = torch.randn(*lead, Hv, dv, generator=g).to(dt)
+    beta = (beta_scale * torch.sigmoid(torch.randn(*lead, Hv, generator=g))).float()
+    log_alpha = (-torch.nn.functional.softplus(la_std * torch.randn(*lead, Hv, generator=g))
+                 * la_scale).float()
+    S0 = (s0_std * torch.randn(nseq, Hv, dk, dv, generator=g)).float() if s0_std else None
+    return dict(q=q, k=k, v=v, log_alpha=log_alpha, beta=beta, S0=S0, cu_seqlens=cu, B=nseq,
+                T=(lead[0] if cu is not None else int(T)), Hk=Hk, H=Hv, dk=dk, dv=dv, dtype=dtype,
+                lengths=lengths)
+
+
 def config_inputs(name: str, **overrides):
     """Inputs of a named chunk workload (``tiny``, ``hybrid_lm``, ``long_context``, ``varlen``)."""
     cfg = dict(CONFIGS[name])
