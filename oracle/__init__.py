@@ -7,7 +7,8 @@ it; the only thing both sides use is the seeded input generator in ``workloads.p
 Two independent computations live here:
 
 * ``forward`` / ``decode_step`` -- the sequential definition (plain C, fp64, OpenMP over
-  independent (sequence, head) chains), ``gdn_oracle.c``.
+  independent (sequence, head) chains), ``gdn_oracle.c``; ``backward`` -- its gradients by
+  reverse mode over the same loop.
 * ``chunkwise.forward_chunkwise`` -- the chunkwise WY / UT-transform form in numpy fp64, written
   separately from the algebra, used only to pin the sequential oracle (and vice versa).
 
@@ -60,6 +61,8 @@ def _load():
                                                    ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                                    ctypes.c_int, ctypes.c_int]
             lib.gdn_oracle_decode_step.restype = ctypes.c_int
+            lib.gdn_oracle_backward.argtypes = [dp] * 14 + [ctypes.c_int] * 5 + [ip, ctypes.c_int]
+            lib.gdn_oracle_backward.restype = ctypes.c_int
             lib.gdn_oracle_max_threads.argtypes = []
             lib.gdn_oracle_max_threads.restype = ctypes.c_int
             _lib = lib
@@ -128,6 +131,40 @@ def forward(q, k, v, log_alpha, beta, S0=None, cu_seqlens=None, units=None, nthr
     if rc != 0:
         raise ValueError("gdn_oracle_forward rejected its arguments")
     return out, S_final
+
+
+def backward(q, k, v, log_alpha, beta, S0, dout, dS_final=None, cu_seqlens=None, nthreads=0):
+    """fp64 gradients of ``forward`` by reverse mode over the sequential definition.
+
+    ``dout`` is dL/dout (shaped like v), ``dS_final`` dL/dS_final or None.  Returns
+    (dq, dk, dv, dlog_alpha, dbeta, dS0) shaped like the inputs (dS0 [B,H,dk,dv] even when S0 is
+    None).  Keeps every state of a sequence in memory: for test-sized inputs.
+    """
+    lib = _load()
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    la, be = _f64(log_alpha), _f64(beta)
+    if cu_seqlens is not None:
+        cu = np.ascontiguousarray(np.asarray(
+            cu_seqlens.cpu() if hasattr(cu_seqlens, "cpu") else cu_seqlens, dtype=np.int32))
+        B = cu.shape[0] - 1
+        T = int(cu[-1])
+        H, dk = q.shape[-2], q.shape[-1]
+    else:
+        cu = None
+        B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    S0 = _f64(S0)
+    dout = _f64(dout)
+    dS_final = _f64(dS_final)
+    dq, dkk, dvv = np.zeros(q.shape), np.zeros(k.shape), np.zeros(v.shape)
+    dla, dbe = np.zeros(la.shape), np.zeros(be.shape)
+    dS0 = np.zeros((B, H, dk, dv))
+    rc = lib.gdn_oracle_backward(_dp(q), _dp(k), _dp(v), _dp(la), _dp(be), _dp(S0), _dp(dout),
+                                 _dp(dS_final), _dp(dq), _dp(dkk), _dp(dvv), _dp(dla), _dp(dbe),
+                                 _dp(dS0), B, T, H, dk, dv, _ip(cu), int(nthreads))
+    if rc != 0:
+        raise ValueError("gdn_oracle_backward rejected its arguments")
+    return dq, dkk, dvv, dla, dbe, dS0
 
 
 def decode_step(q, k, v, log_alpha, beta, S, nthreads=0):

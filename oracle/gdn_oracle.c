@@ -149,6 +149,125 @@ int gdn_oracle_forward(const double *q, const double *k, const double *v,
 }
 
 /*
+ * Gradients of the whole-sequence forward by reverse mode over the same sequential definition.
+ *   dout: dL/dout (layout of out); dS_final: dL/dS_final or NULL (zero).
+ *   Writes dq, dk, dv_ (layouts of q, k, v), dlog_alpha, dbeta (layouts of the gates) and dS0
+ *   (layout of S0; may be NULL).  Each unit keeps all of its states S_0 .. S_T (meant for the
+ *   short sequences of the tests).
+ * Per token, with G = dL/dS_t (after adding the read-out's q_t do_t^T), u = S_{t-1}^T k and
+ * r = G^T k, the chain rule through S_t = a (S - b k (k^T S)) + b k v^T gives
+ *     dq_t = S_t do_t,  dv_t = b r,  dbeta_t = r . (v - a u),
+ *     dlog_alpha_t = a <G, S_{t-1} - b k u^T>   (0 at an exact reset, a = 0),
+ *     dk_t = G b (v - a u) - a b S_{t-1} r,      dL/dS_{t-1} = a (G - b k r^T).
+ * Returns 0, or -1 for invalid sizes or a failed allocation.
+ */
+int gdn_oracle_backward(const double *q, const double *k, const double *v,
+                        const double *log_alpha, const double *beta, const double *S0,
+                        const double *dout, const double *dS_final, double *dq, double *dk,
+                        double *dv_, double *dlog_alpha, double *dbeta, double *dS0, int B, int T,
+                        int H, int dk_, int dv, const int32_t *cu_seqlens, int nthreads)
+{
+    const int DK = dk_;
+    if (B < 0 || T < 0 || H <= 0 || DK <= 0 || dv <= 0) return -1;
+    set_threads(nthreads);
+    const size_t state = (size_t)DK * dv;
+    int bad = 0;
+#pragma omp parallel
+    {
+        double *kS = (double *)malloc(sizeof(double) * (size_t)dv);
+        double *u = (double *)malloc(sizeof(double) * (size_t)dv);
+        double *r = (double *)malloc(sizeof(double) * (size_t)dv);
+        double *G = (double *)malloc(sizeof(double) * state);
+        if (!kS || !u || !r || !G) {
+#pragma omp atomic write
+            bad = 1;
+        }
+#pragma omp for schedule(dynamic, 1)
+        for (int un = 0; un < B * H; ++un) {
+            if (!kS || !u || !r || !G) continue;
+            const int s = un / H, h = un % H;
+            long tok0, ntok;
+            if (cu_seqlens) {
+                tok0 = cu_seqlens[s];
+                ntok = (long)cu_seqlens[s + 1] - cu_seqlens[s];
+            } else {
+                tok0 = (long)s * T;
+                ntok = T;
+            }
+            double *St = (double *)malloc(sizeof(double) * state * (size_t)(ntok + 1));
+            if (!St) {
+#pragma omp atomic write
+                bad = 1;
+                continue;
+            }
+            /* forward, keeping S_0 .. S_ntok */
+            if (S0) memcpy(St, S0 + (size_t)un * state, sizeof(double) * state);
+            else memset(St, 0, sizeof(double) * state);
+            for (long t = 0; t < ntok; ++t) {
+                const size_t th = (size_t)(tok0 + t) * H + h;
+                memcpy(St + (size_t)(t + 1) * state, St + (size_t)t * state, sizeof(double) * state);
+                oracle_token(St + (size_t)(t + 1) * state, q + th * DK, k + th * DK, v + th * dv,
+                             log_alpha[th], beta[th], NULL, kS, DK, dv);
+            }
+            /* reverse */
+            if (dS_final) memcpy(G, dS_final + (size_t)un * state, sizeof(double) * state);
+            else memset(G, 0, sizeof(double) * state);
+            for (long t = ntok - 1; t >= 0; --t) {
+                const size_t th = (size_t)(tok0 + t) * H + h;
+                const double *S_t = St + (size_t)(t + 1) * state, *Sp = St + (size_t)t * state;
+                const double *qt = q + th * DK, *kt = k + th * DK, *vt = v + th * dv, *dot = dout + th * dv;
+                const double a = exp(log_alpha[th]), b = beta[th];
+                /* read-out o_t = S_t^T q_t */
+                for (int i = 0; i < DK; ++i) {
+                    double acc = 0.0;
+                    for (int j = 0; j < dv; ++j) {
+                        acc += S_t[(size_t)i * dv + j] * dot[j];
+                        G[(size_t)i * dv + j] += qt[i] * dot[j];
+                    }
+                    dq[th * DK + i] = acc;
+                }
+                /* the update */
+                for (int j = 0; j < dv; ++j) {
+                    double uj = 0.0, rj = 0.0;
+                    for (int i = 0; i < DK; ++i) {
+                        uj += kt[i] * Sp[(size_t)i * dv + j];
+                        rj += kt[i] * G[(size_t)i * dv + j];
+                    }
+                    u[j] = uj;
+                    r[j] = rj;
+                }
+                double db = 0.0, da = 0.0;
+                for (int j = 0; j < dv; ++j) {
+                    dv_[th * dv + j] = b * r[j];
+                    db += r[j] * (vt[j] - a * u[j]);
+                }
+                for (int i = 0; i < DK; ++i) {
+                    double dki = 0.0;
+                    for (int j = 0; j < dv; ++j) {
+                        const double g = G[(size_t)i * dv + j];
+                        da += g * (Sp[(size_t)i * dv + j] - b * kt[i] * u[j]);
+                        dki += g * b * (vt[j] - a * u[j]) - a * b * Sp[(size_t)i * dv + j] * r[j];
+                    }
+                    dk[th * DK + i] = dki;
+                }
+                dbeta[th] = db;
+                dlog_alpha[th] = (a == 0.0) ? 0.0 : a * da;
+                for (int i = 0; i < DK; ++i)
+                    for (int j = 0; j < dv; ++j)
+                        G[(size_t)i * dv + j] = a * (G[(size_t)i * dv + j] - b * kt[i] * r[j]);
+            }
+            if (dS0) memcpy(dS0 + (size_t)un * state, G, sizeof(double) * state);
+            free(St);
+        }
+        free(kS);
+        free(u);
+        free(r);
+        free(G);
+    }
+    return bad ? -1 : 0;
+}
+
+/*
  * One decode step: every (n, h) state takes exactly one token, in place.
  * Returns 0, or -1 for invalid sizes.
  */
