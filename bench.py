@@ -455,6 +455,34 @@ def run_ours(args, world, rank, local):
                                   "ms": round(ms_g, 6), "tokens_per_s": round(8 * 4096 / (ms_g * 1e-3), 1),
                                   "launches_per_call": 1}
         del dg, outg, Sg
+        # backward of the hybrid-LM step (dq, dk, dv, gate and state gradients; fp32 CUDA cores)
+        dout = torch.randn(d["v"].shape, device="cuda").to(d["v"].dtype)
+        wsb = torch.empty(gdn.gdn_chunk_bwd_workspace_bytes(8, 4096, 12, 64, 64, 64, 0), dtype=torch.uint8,
+                          device="cuda")
+
+        def call_bwd():
+            gdn.chunk_bwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], dout, workspace=wsb, stream=stream)
+        with torch.cuda.stream(stream):
+            for _ in range(3):
+                flush.zero_()
+                call_bwd()
+            stream.synchronize()
+            evb = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(5)]
+            for a0, b0 in evb:
+                flush.zero_()
+                a0.record(stream)
+                call_bwd()
+                b0.record(stream)
+            stream.synchronize()
+        ms_b = statistics.mean(a0.elapsed_time(b0) for a0, b0 in evb)
+        # bytes per token-head: q, k, v, dout (bf16) and gates in; dq, dk, dv (fp32) and two gate grads out
+        by_b = 393216 * (4 * 64 * 2 + 8 + 3 * 64 * 4 + 8)
+        extra["hybrid_lm_backward"] = {"workload": "hybrid_lm backward: dq, dk, dv, dlog_alpha, dbeta (fp32) from dout",
+                                       "ms": round(ms_b, 6), "tokens_per_s": round(32768 / (ms_b * 1e-3), 1),
+                                       "launches_per_call": 4, "algo_bytes": by_b,
+                                       "gbs": round(by_b / (ms_b * 1e-3) / 1e9, 3),
+                                       "hbm_frac": round(by_b / (ms_b * 1e-3) / 1e9 / peaks["hbm_gbs"], 5)}
+        del dout, wsb
     cpu = None
     if rank == 0 and world == 1:
         cpu = cpu_oracle_baseline(inp)

@@ -168,6 +168,30 @@ GDN_API int gdn_chunk_fwd_noalloc(const void *q, const void *k, const void *v, c
                                   int dtype, void *stream);
 
 /*
+ * gdn_chunk_bwd -- gradients of gdn_chunk_fwd (the training path; Sykra README, "Architectural
+ * Highlights": chunk-parallel training through the WY / unit triangular transform), for
+ * dk = dv = 64 and chunk = 64.  Given the forward's inputs (same layouts, dtype for q, k, v and
+ * dout) and dout = dL/dout, dS_final = dL/dS_final (NULL: zero), it writes
+ *     dq, dk [.., H, 64], dv [.., H, 64], dlog_alpha, dbeta [.., H]   (fp32, always)
+ *     dS0 [B, H, 64, 64] fp32 (NULL: not written)
+ * Computed in fp32 on the CUDA cores from the chunk form: every chunk's state map
+ * S' = M S + Bm and gradient map dS = M^T dS' + (Q^T diag(gam) - W^T P^T) dO are formed in
+ * parallel, two scans over each sequence's chunks give the entry states and exit gradients, and
+ * every chunk's input gradients are then formed in parallel.  log_alpha = -inf (an exact reset)
+ * gets dlog_alpha = 0.  Workspace: gdn_chunk_bwd_workspace_bytes(...) bytes, 256-byte aligned
+ * (five 16 KB matrices per chunk and head).  Errors as gdn_chunk_fwd; other head sizes return
+ * GDN_ERR_UNSUPPORTED.
+ */
+GDN_API int gdn_chunk_bwd(const void *q, const void *k, const void *v, const float *log_alpha,
+                          const float *beta, const float *S0, const void *dout, const float *dS_final,
+                          float *dq, float *dk, float *dv, float *dlog_alpha, float *dbeta, float *dS0,
+                          int B, int T, int H, int dk_, int dv_, int chunk, const int32_t *cu_seqlens,
+                          int dtype, void *workspace, size_t workspace_bytes, void *stream);
+
+/* Workspace gdn_chunk_bwd needs for these sizes; (size_t)-1 for sizes it rejects. */
+GDN_API size_t gdn_chunk_bwd_workspace_bytes(int B, int T, int H, int dk, int dv, int chunk, int varlen);
+
+/*
  * gdn_decode_step -- one generation step: every (n, h) state takes exactly one token, in place
  * (Sykra README, "Architectural Highlights" and "Computational Complexity": an O(d^2) update of
  * a fixed d x d state per token).  With r = S^T k, s = S^T q (both from the state before the

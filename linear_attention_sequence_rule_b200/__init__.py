@@ -6,7 +6,8 @@ PyTorch provides device memory and streams.  The binding has two layers:
 * ``gdn_chunk_fwd``, ``gdn_chunk_fwd_noalloc``, ``gdn_decode_step``, ``gdn_chunk_fwd_workspace_bytes``,
   ``gdn_status_string``, ``gdn_last_error``, ``gdn_version`` -- the C-ABI entry points of
   ``include/gdn.h`` with the same names and arguments (pointers as Python ints);
-* ``chunk_fwd``, ``chunk_fwd_fused``, ``chunk_fwd_gva``, ``decode_step`` and ``decode_step_gva`` --
+* ``chunk_fwd``, ``chunk_fwd_fused``, ``chunk_fwd_gva``, ``chunk_bwd``, ``decode_step`` and
+  ``decode_step_gva`` --
   the same calls taking torch tensors; they check shapes,
   devices and dtypes, allocate outputs with torch when none are given, and raise ``GdnError``
   on a non-zero status.
@@ -24,9 +25,9 @@ __all__ = [
     "GdnError", "GDN_OK", "GDN_ERR_INVALID_ARGUMENT", "GDN_ERR_UNSUPPORTED", "GDN_ERR_WORKSPACE",
     "GDN_ERR_CUDA", "GDN_ERR_TIMEOUT", "GDN_DTYPE_F32", "GDN_DTYPE_BF16", "LIB_PATH",
     "gdn_chunk_fwd", "gdn_chunk_fwd_noalloc", "gdn_chunk_fwd_fused", "gdn_chunk_fwd_gva",
-    "gdn_decode_step", "gdn_decode_step_gva", "gdn_chunk_fwd_workspace_bytes", "gdn_status_string",
+    "gdn_decode_step", "gdn_decode_step_gva", "gdn_chunk_bwd", "gdn_chunk_bwd_workspace_bytes", "gdn_chunk_fwd_workspace_bytes", "gdn_status_string",
     "gdn_last_error", "gdn_version", "gdn_device_status", "device_status", "chunk_fwd", "chunk_fwd_fused",
-    "chunk_fwd_gva", "decode_step", "decode_step_gva", "workspace_bytes",
+    "chunk_fwd_gva", "chunk_bwd", "decode_step", "decode_step_gva", "workspace_bytes",
 ]
 
 GDN_OK = 0
@@ -59,6 +60,10 @@ _lib.gdn_chunk_fwd_gva.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _
 _lib.gdn_chunk_fwd_gva.restype = _i
 _lib.gdn_decode_step_gva.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp]
 _lib.gdn_decode_step_gva.restype = _i
+_lib.gdn_chunk_bwd.argtypes = [_vp] * 14 + [_i] * 6 + [_vp, _i, _vp, _sz, _vp]
+_lib.gdn_chunk_bwd.restype = _i
+_lib.gdn_chunk_bwd_workspace_bytes.argtypes = [_i] * 7
+_lib.gdn_chunk_bwd_workspace_bytes.restype = _sz
 _lib.gdn_chunk_fwd_noalloc.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i,
                                        _i, _vp, _i, _vp]
 _lib.gdn_chunk_fwd_noalloc.restype = _i
@@ -107,6 +112,17 @@ def gdn_decode_step_gva(q, k, v, log_alpha, beta, S_inout, out, N, Hk, Hv, dk, d
                         stream) -> int:
     return _lib.gdn_decode_step_gva(q, k, v, log_alpha, beta, S_inout, out, N, Hk, Hv, dk, dv, dtype,
                                     stream)
+
+
+def gdn_chunk_bwd(q, k, v, log_alpha, beta, S0, dout, dS_final, dq, dk, dv, dlog_alpha, dbeta, dS0, B, T,
+                  H, dk_, dv_, chunk, cu_seqlens, dtype, workspace, workspace_bytes, stream) -> int:
+    return _lib.gdn_chunk_bwd(q, k, v, log_alpha, beta, S0, dout, dS_final, dq, dk, dv, dlog_alpha, dbeta,
+                              dS0, B, T, H, dk_, dv_, chunk, cu_seqlens, dtype, workspace, workspace_bytes,
+                              stream)
+
+
+def gdn_chunk_bwd_workspace_bytes(B, T, H, dk, dv, chunk, varlen) -> int:
+    return _lib.gdn_chunk_bwd_workspace_bytes(B, T, H, dk, dv, chunk, varlen)
 
 
 def gdn_chunk_fwd_noalloc(q, k, v, log_alpha, beta, S0, out, S_final, B, T, H, dk, dv, chunk,
@@ -266,6 +282,49 @@ def chunk_fwd_gva(q, k, v, log_alpha, beta, S0=None, cu_seqlens=None, out=None, 
     if rc != GDN_OK:
         raise GdnError(rc, gdn_last_error())
     return p["out"], p["S_final"]
+
+
+def chunk_bwd(q, k, v, log_alpha, beta, dout, S0=None, dS_final=None, cu_seqlens=None, want_dS0=True,
+              workspace=None, chunk=64, stream=None):
+    """Gradients of ``chunk_fwd`` (dk = dv = 64): returns fp32 (dq, dk, dv, dlog_alpha, dbeta,
+    dS0 or None) for dout = dL/dout and dS_final = dL/dS_final (None: zero)."""
+    dt = q.dtype
+    if dt not in _DT:
+        raise ValueError(f"unsupported dtype {dt}")
+    dev = q.device
+    if cu_seqlens is not None:
+        T, H, dk = q.shape
+        B = cu_seqlens.shape[0] - 1
+        lead = (T,)
+        _need(cu_seqlens, "cu_seqlens", torch.int32, (B + 1,), dev)
+    else:
+        B, T, H, dk = q.shape
+        lead = (B, T)
+    dv = v.shape[-1]
+    for name, x, shp in (("q", q, (*lead, H, dk)), ("k", k, (*lead, H, dk)), ("v", v, (*lead, H, dv)),
+                         ("dout", dout, (*lead, H, dv))):
+        _need(x, name, dt, shp, dev)
+    _need(log_alpha, "log_alpha", torch.float32, (*lead, H), dev)
+    _need(beta, "beta", torch.float32, (*lead, H), dev)
+    for name, x in (("S0", S0), ("dS_final", dS_final)):
+        if x is not None:
+            _need(x, name, torch.float32, (B, H, dk, dv), dev)
+    f32 = dict(dtype=torch.float32, device=dev)
+    dq, dkk, dvv = torch.empty((*lead, H, dk), **f32), torch.empty((*lead, H, dk), **f32), torch.empty((*lead, H, dv), **f32)
+    dla, dbe = torch.empty((*lead, H), **f32), torch.empty((*lead, H), **f32)
+    dS0 = torch.empty((B, H, dk, dv), **f32) if want_dS0 else None
+    need = gdn_chunk_bwd_workspace_bytes(B, T, H, dk, dv, chunk, int(cu_seqlens is not None))
+    if need == (1 << 64) - 1:
+        raise GdnError(GDN_ERR_UNSUPPORTED, f"gdn_chunk_bwd does not take dk={dk} dv={dv} chunk={chunk}")
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    rc = gdn_chunk_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(S0), _ptr(dout),
+                       _ptr(dS_final), _ptr(dq), _ptr(dkk), _ptr(dvv), _ptr(dla), _ptr(dbe), _ptr(dS0), B, T,
+                       H, dk, dv, chunk, _ptr(cu_seqlens), _DT[dt], _ptr(workspace),
+                       workspace.numel() * workspace.element_size(), _stream_ptr(stream))
+    if rc != GDN_OK:
+        raise GdnError(rc, gdn_last_error())
+    return dq, dkk, dvv, dla, dbe, dS0
 
 
 def decode_step_gva(q, k, v, log_alpha, beta, S, out=None, stream=None):

@@ -248,3 +248,41 @@ int gdn_device_status(void *stream)
 }
 
 }  // extern "C"
+
+size_t gdn_chunk_bwd_workspace_bytes(int B, int T, int H, int dk, int dv, int chunk, int varlen)
+{
+    if (dk != 64 || dv != 64 || chunk != 64 || B < 1 || H < 1 || T < 0 || (!varlen && T < 1)) return (size_t)-1;
+    return chunk_bwd_workspace_bytes(B, T, H, varlen);
+}
+
+int gdn_chunk_bwd(const void *q, const void *k, const void *v, const float *log_alpha, const float *beta,
+                  const float *S0, const void *dout, const float *dS_final, float *dq, float *dk, float *dv,
+                  float *dlog_alpha, float *dbeta, float *dS0, int B, int T, int H, int dk_, int dv_, int chunk,
+                  const int32_t *cu_seqlens, int dtype, void *workspace, size_t workspace_bytes, void *stream)
+{
+    g_last_error[0] = 0;
+    const char *fn = "gdn_chunk_bwd";
+    const int varlen = cu_seqlens != nullptr;
+    int rc = check_chunk_shape(B, T, H, dk_, dv_, chunk, varlen, dtype);
+    if (rc != GDN_OK) return rc;
+    if (dk_ != 64 || dv_ != 64)
+        return fail(GDN_ERR_UNSUPPORTED, "%s: dk=%d dv=%d, supported: 64", fn, dk_, dv_);
+    if (!q || !k || !v || !log_alpha || !beta || !dout || !dq || !dk || !dv || !dlog_alpha || !dbeta)
+        return fail(GDN_ERR_INVALID_ARGUMENT, "%s: inputs, dout and every gradient output except dS0 are required",
+                    fn);
+    const void *ptrs[] = {q, k, v, log_alpha, beta, S0, dout, dS_final, dq, dk, dv, dlog_alpha, dbeta, dS0,
+                          cu_seqlens};
+    for (const void *p : ptrs)
+        if (p && !aligned16(p)) return fail(GDN_ERR_INVALID_ARGUMENT, "%s: pointer %p is not 16-byte aligned", fn, p);
+    const size_t need = chunk_bwd_workspace_bytes(B, T, H, varlen);
+    if (!workspace || workspace_bytes < need)
+        return fail(GDN_ERR_WORKSPACE, "%s: workspace of %zu bytes needed, %zu given", fn, need,
+                    workspace ? workspace_bytes : (size_t)0);
+    if (reinterpret_cast<uintptr_t>(workspace) & 255u)
+        return fail(GDN_ERR_INVALID_ARGUMENT, "%s: workspace must be 256-byte aligned", fn);
+    BwdArgs a{q, k, v, log_alpha, beta, S0, dout, dS_final, dq, dk, dv, dlog_alpha, dbeta, dS0, cu_seqlens,
+              B, T, H, dtype, workspace};
+    cudaError_t e = launch_chunk_bwd(a, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, fn);
+    return GDN_OK;
+}

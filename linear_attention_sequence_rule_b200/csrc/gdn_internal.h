@@ -46,4 +46,18 @@ size_t chunk_tc_workspace_bytes(int B, int T, int H, int dk, int dv, int varlen,
 // after synchronising the device.  Returns -1 when the read itself failed.
 int read_and_clear_tc_error();
 
+// Gradients of the chunk forward (fp32 CUDA-core kernels, dk = dv = 64); see gdn_chunk_bwd.cu.
+struct BwdArgs {
+    const void *q, *k, *v;
+    const float *log_alpha, *beta, *S0;
+    const void *dout;
+    const float *dS_final;
+    float *dq, *dk, *dv, *dlog_alpha, *dbeta, *dS0;
+    const int32_t *cu_seqlens;
+    int B, T, H, dtype;
+    void *workspace;
+};
+size_t chunk_bwd_workspace_bytes(int B, int T, int H, int varlen);
+cudaError_t launch_chunk_bwd(const BwdArgs &a, cudaStream_t stream);
+
 }  // namespace gdn

@@ -138,3 +138,16 @@ def test_torch_layer_checks_shapes_without_launching():
     q = torch.zeros(1, 64, 1, 64)
     with pytest.raises(ValueError):
         gdn.chunk_fwd(q, q, q[..., :32], torch.zeros(1, 64, 1), torch.zeros(1, 64, 2))
+
+
+def test_backward_entry_validation():
+    a = dict(q=FAKE, k=FAKE, v=FAKE, log_alpha=FAKE, beta=FAKE, S0=None, dout=FAKE, dS_final=None, dq=FAKE,
+             dk=FAKE, dv=FAKE, dlog_alpha=FAKE, dbeta=FAKE, dS0=None, B=1, T=64, H=1, dk_=64, dv_=64, chunk=64,
+             cu_seqlens=None, dtype=gdn.GDN_DTYPE_BF16, workspace=None, workspace_bytes=0, stream=None)
+    assert gdn.gdn_chunk_bwd(**(a | dict(dk_=128, dv_=128))) == gdn.GDN_ERR_UNSUPPORTED
+    assert gdn.gdn_chunk_bwd(**(a | dict(dq=None))) == gdn.GDN_ERR_INVALID_ARGUMENT
+    assert gdn.gdn_chunk_bwd(**(a | dict(dbeta=FAKE + 4))) == gdn.GDN_ERR_INVALID_ARGUMENT
+    assert gdn.gdn_chunk_bwd(**a) == gdn.GDN_ERR_WORKSPACE
+    assert "gdn_chunk_bwd" in gdn.gdn_last_error()
+    assert gdn.gdn_chunk_bwd_workspace_bytes(1, 64, 1, 128, 128, 64, 0) == (1 << 64) - 1
+    assert gdn.gdn_chunk_bwd_workspace_bytes(2, 128, 3, 64, 64, 64, 0) > 5 * 2 * 2 * 3 * 64 * 64 * 4 - 1
