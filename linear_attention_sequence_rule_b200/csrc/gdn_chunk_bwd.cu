@@ -11,11 +11,11 @@
 //   dS  = M^T dS' + R,           R  = (Q^T diag(gam) - W^T P^T) dO
 // Four kernels:
 //   bwd_prep   (chunk x head, parallel)  : T, W, U~, P  ->  M, Bm, R
-//   bwd_fscan  (sequence x head)         : S_c for every chunk, from S0
-//   bwd_bscan  (sequence x head, reverse): dS at every chunk's end, from dS_final; dS0
+//   bwd_scan<false> (sequence x head)    : S_c for every chunk, from S0
+//   bwd_scan<true>  (sequence x head, reverse): dS at every chunk's end, from dS_final; dS0
 //   bwd_grads  (chunk x head, parallel)  : with S_c and dS_{c+1}, every input gradient of the chunk
-// All matrices are 64 x 64 fp32 in shared memory (row stride 65); 256 threads; a matrix product
-// gives each thread a 4 x 4 block of the result.
+// All matrices are 64 x 64 fp32 in shared memory (swizzled 16-byte groups); 256 threads; a matrix
+// product gives each thread a 4 x 4 block of the result.
 #include <cuda_bf16.h>
 #include <math.h>
 
@@ -26,9 +26,16 @@ namespace gdn {
 namespace {
 
 constexpr int N = 64;          // chunk length = dk = dv
-constexpr int LD = 65;         // shared-memory row stride
-constexpr int MAT = N * LD;    // floats per matrix
+constexpr int MAT = N * N;     // floats per matrix
 constexpr int kThreads = 256;
+
+// Shared matrices are 64 x 64 fp32 with 64-float rows; the 16 groups of 4 floats of row r are
+// stored in the order group ^ ((r / 4) mod 16), so that the 16-byte loads of a matrix product
+// spread over the banks.  Element (r, c) lives at sw(r, c).
+__device__ __forceinline__ int sw(int r, int c)
+{
+    return r * N + ((((c >> 2) ^ (r >> 2)) & 15) << 2) + (c & 3);
+}
 
 __device__ __forceinline__ float ld_in(const float *p) { return *p; }
 __device__ __forceinline__ float ld_in(const __nv_bfloat16 *p) { return __bfloat162float(*p); }
@@ -70,7 +77,7 @@ __device__ ChunkRef chunk_ref(int e, const int32_t *cu, const int32_t *off, int 
 
 // C(r, c) = sum_k opA(r, k) ks[k] opB(k, c) for 64 x 64 operands (ks: optional diagonal, NULL = 1);
 // thread t gets rows 4 (t / 16) .. +3 and columns 4 (t % 16) .. +3 and hands each result to
-// emit(r, c, value).
+// emit(r, c, value).  Four steps of k at a time, every operand read as 16-byte groups.
 template <bool TA, bool TB, typename F>
 __device__ __forceinline__ void mm(const float *A, const float *B, int t, F &&emit, const float *ks = nullptr)
 {
@@ -80,18 +87,34 @@ __device__ __forceinline__ void mm(const float *A, const float *B, int t, F &&em
     for (int i = 0; i < 4; ++i)
 #pragma unroll
         for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
-#pragma unroll 4
-    for (int k = 0; k < N; ++k) {
-        float a[4], b[4];
-        const float sk = ks ? ks[k] : 1.f;  // optional scale of the summation index (a diagonal)
+#pragma unroll 2
+    for (int k0 = 0; k0 < N; k0 += 4) {
+        float a[4][4], b[4][4];  // a[i][kk] = opA(r0 + i, k0 + kk), b[kk][j] = opB(k0 + kk, c0 + j)
 #pragma unroll
-        for (int i = 0; i < 4; ++i) a[i] = (TA ? A[k * LD + r0 + i] : A[(r0 + i) * LD + k]) * sk;
+        for (int x = 0; x < 4; ++x) {
+            const float4 va = TA ? *reinterpret_cast<const float4 *>(&A[sw(k0 + x, r0)])
+                                 : *reinterpret_cast<const float4 *>(&A[sw(r0 + x, k0)]);
+            if (TA) { a[0][x] = va.x; a[1][x] = va.y; a[2][x] = va.z; a[3][x] = va.w; }
+            else { a[x][0] = va.x; a[x][1] = va.y; a[x][2] = va.z; a[x][3] = va.w; }
+            const float4 vb = TB ? *reinterpret_cast<const float4 *>(&B[sw(c0 + x, k0)])
+                                 : *reinterpret_cast<const float4 *>(&B[sw(k0 + x, c0)]);
+            if (TB) { b[0][x] = vb.x; b[1][x] = vb.y; b[2][x] = vb.z; b[3][x] = vb.w; }
+            else { b[x][0] = vb.x; b[x][1] = vb.y; b[x][2] = vb.z; b[x][3] = vb.w; }
+        }
+        if (ks) {
+            const float4 s4 = *reinterpret_cast<const float4 *>(&ks[k0]);
+            const float sv[4] = {s4.x, s4.y, s4.z, s4.w};
 #pragma unroll
-        for (int j = 0; j < 4; ++j) b[j] = TB ? B[(c0 + j) * LD + k] : B[k * LD + c0 + j];
+            for (int i = 0; i < 4; ++i)
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
+                for (int kk = 0; kk < 4; ++kk) a[i][kk] *= sv[kk];
+        }
 #pragma unroll
-            for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+        for (int kk = 0; kk < 4; ++kk)
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i][kk], b[kk][j], acc[i][j]);
     }
 #pragma unroll
     for (int i = 0; i < 4; ++i)
@@ -99,7 +122,49 @@ __device__ __forceinline__ void mm(const float *A, const float *B, int t, F &&em
         for (int j = 0; j < 4; ++j) emit(r0 + i, c0 + j, acc[i][j]);
 }
 
-// Gate vectors of one chunk (thread 0 computes them; the caller synchronises):
+// Thread t's 4 x 4 block of a product (the layout mm hands out) into the shared matrix C.
+__device__ __forceinline__ void put_block(float *C, const float (&x)[16], int t)
+{
+    const int r0 = (t >> 4) * 4, c0 = (t & 15) * 4;
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+        *reinterpret_cast<float4 *>(&C[sw(r0 + i, c0)]) = make_float4(x[4 * i], x[4 * i + 1], x[4 * i + 2], x[4 * i + 3]);
+}
+
+// Sum of a value over the 16 threads that share a row block (lanes l, l ^ 1, ..., l ^ 15 of a
+// half warp): every one of them gets the total.
+__device__ __forceinline__ float row_block_sum(float x)
+{
+#pragma unroll
+    for (int o = 1; o < 16; o <<= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+    return x;
+}
+
+// Inclusive sums of x over the 32 lanes of a warp, restarted at every lane whose f is set (f on
+// return: a restart lies at or before this lane).
+__device__ __forceinline__ void seg_scan32(float &x, int &f, int lane)
+{
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const float xo = __shfl_up_sync(0xffffffffu, x, o);
+        const int fo = __shfl_up_sync(0xffffffffu, f, o);
+        if (lane >= o) {
+            if (!f) x += xo;
+            f |= fo;
+        }
+    }
+}
+
+// The same over 64 positions, lane l holding positions l (x0, f0) and l + 32 (x1, f1).
+__device__ __forceinline__ void seg_scan64(float &x0, int f0, float &x1, int f1, int lane)
+{
+    seg_scan32(x0, f0, lane);
+    seg_scan32(x1, f1, lane);
+    const float carry = __shfl_sync(0xffffffffu, x0, 31);
+    if (!f1) x1 += carry;
+}
+
+// Gate vectors of one chunk (every thread of the block calls this; the caller synchronises after):
 // G[r] = sum of log_alpha over (last reset, r], last[r] = last exact reset at or before r (-1:
 // none), gam[r] = exp(G[r]) (0 after a reset), lam[i] = exp(G[63] - G[i]) (0 when a reset lies in
 // (i, 63]), bet[r]; padded rows get log_alpha = 0, beta = 0.
@@ -112,26 +177,36 @@ template <typename TIn>
 __device__ void chunk_gates(Gates &g, const float *log_alpha, const float *beta, const ChunkRef &c, int H, int h,
                             int t)
 {
-    if (t == 0) {
-        float acc = 0.f;
-        int lst = -1;
-        for (int r = 0; r < N; ++r) {
-            const size_t off = (size_t)(c.tok + r) * H + h;
-            const float la = r < c.n ? log_alpha[off] : 0.f;
-            g.bet[r] = r < c.n ? beta[off] : 0.f;
-            if (la == -INFINITY) {
-                lst = r;
-                acc = 0.f;
-            } else {
-                acc += la;
+    if (t < N) {
+        const size_t off = (size_t)(c.tok + t) * H + h;
+        g.G[t] = t < c.n ? log_alpha[off] : 0.f;
+        g.bet[t] = t < c.n ? beta[off] : 0.f;
+    }
+    __syncthreads();
+    if (t < 32) {
+        const float la0 = g.G[t], la1 = g.G[t + 32];
+        const int r0 = la0 == -INFINITY, r1 = la1 == -INFINITY;
+        float x0 = r0 ? 0.f : la0, x1 = r1 ? 0.f : la1;
+        seg_scan64(x0, r0, x1, r1, t);
+        int l0 = r0 ? t : -1, l1 = r1 ? t + 32 : -1;  // prefix maxima of the reset positions
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int a = __shfl_up_sync(0xffffffffu, l0, o), b = __shfl_up_sync(0xffffffffu, l1, o);
+            if (t >= o) {
+                l0 = max(l0, a);
+                l1 = max(l1, b);
             }
-            g.G[r] = acc;
-            g.last[r] = lst;
         }
-        for (int r = 0; r < N; ++r) {
-            g.gam[r] = g.last[r] >= 0 ? 0.f : expf(g.G[r]);
-            g.lam[r] = g.last[N - 1] > r ? 0.f : expf(g.G[N - 1] - g.G[r]);
-        }
+        l1 = max(l1, __shfl_sync(0xffffffffu, l0, 31));
+        g.G[t] = x0;
+        g.G[t + 32] = x1;
+        g.last[t] = l0;
+        g.last[t + 32] = l1;
+    }
+    __syncthreads();
+    if (t < N) {
+        g.gam[t] = g.last[t] >= 0 ? 0.f : expf(g.G[t]);
+        g.lam[t] = g.last[N - 1] > t ? 0.f : expf(g.G[N - 1] - g.G[t]);
     }
 }
 
@@ -141,13 +216,62 @@ __device__ __forceinline__ float decay(const Gates &g, int r, int i)
     return (i <= r && g.last[r] <= i) ? expf(g.G[r] - g.G[i]) : 0.f;
 }
 
-// Rows of a [tokens, H, 64] tensor into a 64 x LD shared matrix (zero past the chunk end).
+// One chunk's rows of a [tokens, H, 64] tensor in registers, as 16-byte pieces (zero past the
+// chunk end): fetch() issues every load, put() converts to fp32 into a shared matrix, so that the
+// loads of several tensors are in flight at once.
 template <typename TIn>
-__device__ void load_rows(float *M, const TIn *x, const ChunkRef &c, int H, int h, int t)
+struct RowTile {
+    static constexpr int V = 16 / (int)sizeof(TIn);      // elements per piece
+    static constexpr int PER_ROW = N / V;
+    static constexpr int ITER = N * PER_ROW / kThreads;  // pieces per thread
+    uint4 b[ITER];
+
+    __device__ __forceinline__ void fetch(const TIn *x, const ChunkRef &c, int H, int h, int t)
+    {
+#pragma unroll
+        for (int u = 0; u < ITER; ++u) {
+            const int e = t + u * kThreads, r = e / PER_ROW, j = (e % PER_ROW) * V;
+            b[u] = r < c.n ? __ldg(reinterpret_cast<const uint4 *>(x + ((size_t)(c.tok + r) * H + h) * N + j))
+                           : make_uint4(0u, 0u, 0u, 0u);
+        }
+    }
+    __device__ __forceinline__ void put(float *M, int t) const
+    {
+#pragma unroll
+        for (int u = 0; u < ITER; ++u) {
+            const int e = t + u * kThreads, r = e / PER_ROW, j = (e % PER_ROW) * V;
+            if constexpr (sizeof(TIn) == 4) {
+                *reinterpret_cast<float4 *>(&M[sw(r, j)]) = *reinterpret_cast<const float4 *>(&b[u]);
+            } else {
+                const __nv_bfloat162 *p = reinterpret_cast<const __nv_bfloat162 *>(&b[u]);
+                const float2 a0 = __bfloat1622float2(p[0]), a1 = __bfloat1622float2(p[1]),
+                             a2 = __bfloat1622float2(p[2]), a3 = __bfloat1622float2(p[3]);
+                *reinterpret_cast<float4 *>(&M[sw(r, j)]) = make_float4(a0.x, a0.y, a1.x, a1.y);
+                *reinterpret_cast<float4 *>(&M[sw(r, j + 4)]) = make_float4(a2.x, a2.y, a3.x, a3.y);
+            }
+        }
+    }
+};
+
+// A dense 64 x 64 fp32 matrix from global memory (row-major) into a shared matrix, and back.
+__device__ __forceinline__ void mat_to_shared(float *M, const float *src, int t)
 {
-    for (int e = t; e < N * N; e += kThreads) {
-        const int r = e >> 6, j = e & 63;
-        M[r * LD + j] = r < c.n ? ld_in(x + ((size_t)(c.tok + r) * H + h) * N + j) : 0.f;
+    float4 b[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) b[u] = __ldg(reinterpret_cast<const float4 *>(src) + t + u * kThreads);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+        const int e = (t + u * kThreads) * 4;
+        *reinterpret_cast<float4 *>(&M[sw(e >> 6, e & 63)]) = b[u];
+    }
+}
+
+__device__ __forceinline__ void mat_from_shared(float *dst, const float *M, int t)
+{
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+        const int e = (t + u * kThreads) * 4;
+        reinterpret_cast<float4 *>(dst)[t + u * kThreads] = *reinterpret_cast<const float4 *>(&M[sw(e >> 6, e & 63)]);
     }
 }
 
@@ -162,11 +286,11 @@ __device__ void unit_lower_inverse(const float *A, float *Tm, int t)
         for (int r = 0; r < N; ++r) {
             float s = 0.f;
 #pragma unroll
-            for (int i = 0; i < r; ++i) s = fmaf(A[r * LD + i], x[i], s);
+            for (int i = 0; i < r; ++i) s = fmaf(A[sw(r, i)], x[i], s);
             x[r] = r < c ? 0.f : (r == c ? 1.f : -s);
         }
 #pragma unroll
-        for (int r = 0; r < N; ++r) Tm[r * LD + c] = x[r];
+        for (int r = 0; r < N; ++r) Tm[sw(r, c)] = x[r];
     }
 }
 
@@ -178,7 +302,7 @@ __global__ void __launch_bounds__(kThreads, 1)
              const int32_t *__restrict__ cu, const int32_t *__restrict__ off, int nseq, int T, int H,
              float *__restrict__ Mo, float *__restrict__ Bo, float *__restrict__ Ro)
 {
-    extern __shared__ float smf[];
+    extern __shared__ __align__(16) float smf[];
     float *K = smf, *Q = K + MAT, *V = Q + MAT, *dO = V + MAT, *A = dO + MAT, *Tm = A + MAT, *W = Tm + MAT,
           *Ut = W + MAT, *P = Ut + MAT;
     Gates &g = *reinterpret_cast<Gates *>(P + MAT);
@@ -186,29 +310,36 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int t = threadIdx.x, h = blockIdx.y, e = blockIdx.x;
     const ChunkRef c = chunk_ref(e, cu, off, nseq, T);
     if (c.n == 0) return;
-    load_rows(K, k, c, H, h, t);
-    load_rows(Q, q, c, H, h, t);
-    load_rows(V, v, c, H, h, t);
-    load_rows(dO, dout, c, H, h, t);
+    {
+        RowTile<TIn> tk, tq, tv, td;
+        tk.fetch(k, c, H, h, t);
+        tq.fetch(q, c, H, h, t);
+        tv.fetch(v, c, H, h, t);
+        td.fetch(dout, c, H, h, t);
+        tk.put(K, t);
+        tq.put(Q, t);
+        tv.put(V, t);
+        td.put(dO, t);
+    }
     chunk_gates<TIn>(g, log_alpha, beta, c, H, h, t);
     __syncthreads();
     if (t < N) bg[t] = g.bet[t] * g.gam[t];
-    mm<false, true>(K, K, t, [&](int r, int i, float x) { A[r * LD + i] = i < r ? g.bet[r] * decay(g, r, i) * x : 0.f; });
-    mm<false, true>(Q, K, t, [&](int r, int i, float x) { P[r * LD + i] = decay(g, r, i) * x; });
+    mm<false, true>(K, K, t, [&](int r, int i, float x) { A[sw(r, i)] = i < r ? g.bet[r] * decay(g, r, i) * x : 0.f; });
+    mm<false, true>(Q, K, t, [&](int r, int i, float x) { P[sw(r, i)] = decay(g, r, i) * x; });
     __syncthreads();
     unit_lower_inverse(A, Tm, t);
     __syncthreads();
-    mm<false, false>(Tm, K, t, [&](int r, int m, float x) { W[r * LD + m] = x; }, bg);
-    mm<false, false>(Tm, V, t, [&](int r, int j, float x) { Ut[r * LD + j] = x; }, g.bet);
-    mm<true, false>(P, dO, t, [&](int i, int j, float x) { A[i * LD + j] = x; });  // Y = P^T dO (A is free)
+    mm<false, false>(Tm, K, t, [&](int r, int m, float x) { W[sw(r, m)] = x; }, bg);
+    mm<false, false>(Tm, V, t, [&](int r, int j, float x) { Ut[sw(r, j)] = x; }, g.bet);
+    mm<true, false>(P, dO, t, [&](int i, int j, float x) { A[sw(i, j)] = x; });  // Y = P^T dO (A is free)
     __syncthreads();
     const size_t base = ((size_t)e * H + h) * (size_t)(N * N);
     const float gC = g.gam[N - 1];
     mm<true, false>(K, W, t, [&](int m, int n2, float x) { Mo[base + m * N + n2] = (m == n2 ? gC : 0.f) - x; }, g.lam);
     mm<true, false>(K, Ut, t, [&](int m, int j, float x) { Bo[base + m * N + j] = x; }, g.lam);
-    mm<true, false>(Q, dO, t, [&](int m, int j, float x) { Tm[m * LD + j] = x; }, g.gam);  // T is free
+    mm<true, false>(Q, dO, t, [&](int m, int j, float x) { Tm[sw(m, j)] = x; }, g.gam);  // T is free
     __syncthreads();
-    mm<true, false>(W, A, t, [&](int m, int j, float x) { Ro[base + m * N + j] = Tm[m * LD + j] - x; });
+    mm<true, false>(W, A, t, [&](int m, int j, float x) { Ro[base + m * N + j] = Tm[sw(m, j)] - x; });
 }
 
 // Number of chunks of sequence s and the table index of its first chunk.
@@ -223,67 +354,87 @@ __device__ __forceinline__ void seq_chunks(int s, const int32_t *cu, const int32
     }
 }
 
-// ---- bwd_fscan: S_c for every chunk of one (sequence, head), from S0 ------------------------
+// ---- bwd_scan: the chunk maps along one (sequence, head) ----------------------------------------
+// Forward (REV = false): X = S0, then X <- M_c X + Bm_c; Xc[c] = the state entering chunk c.
+// Reverse (REV = true):  X = dS_final, then X <- M_c^T X + R_c over the chunks from the last;
+// Xc[c] = dL/dS at the end of chunk c, Xend = dS0.
+// X is double-buffered in shared memory, and so is M_c; chunk c + 2's M and additive term are
+// loaded into registers while chunk c is multiplied, so one barrier per chunk remains.
+template <bool REV>
 __global__ void __launch_bounds__(kThreads, 1)
-    bwd_fscan(const float *__restrict__ Mo, const float *__restrict__ Bo, const float *__restrict__ S0,
-              const int32_t *__restrict__ cu, const int32_t *__restrict__ off, int T, int H, float *__restrict__ Sc)
+    bwd_scan(const float *__restrict__ Mo, const float *__restrict__ Add, const float *__restrict__ X0,
+             const int32_t *__restrict__ cu, const int32_t *__restrict__ off, int T, int H, float *__restrict__ Xc,
+             float *__restrict__ Xend)
 {
-    extern __shared__ float smf[];
-    float *S = smf, *Mm = S + MAT;
+    extern __shared__ __align__(16) float smf[];  // X[2], then M[2]
     const int t = threadIdx.x, h = blockIdx.x, s = blockIdx.y;
+    const int r0 = (t >> 4) * 4, c0 = (t & 15) * 4;
     int first, count;
     seq_chunks(s, cu, off, T, first, count);
-    const size_t st0 = ((size_t)s * H + h) * (size_t)(N * N);
-    for (int i = t; i < N * N; i += kThreads) S[(i >> 6) * LD + (i & 63)] = S0 ? S0[st0 + i] : 0.f;
+    const size_t st0 = ((size_t)s * H + h) * (size_t)MAT;
+    auto chunk_base = [&](int i) { return ((size_t)(first + (REV ? count - 1 - i : i)) * H + h) * (size_t)MAT; };
+    auto fetch_m = [&](int i, float4 (&m)[4]) {
+        const float4 *src = reinterpret_cast<const float4 *>(Mo + chunk_base(i));
+#pragma unroll
+        for (int u = 0; u < 4; ++u) m[u] = __ldg(src + t + u * kThreads);
+    };
+    auto fetch_a = [&](int i, float4 (&a)[4]) {
+        const float *src = Add + chunk_base(i);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) a[u] = __ldg(reinterpret_cast<const float4 *>(src + (r0 + u) * N + c0));
+    };
+    auto put_m = [&](float *M, const float4 (&m)[4]) {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int e = (t + u * kThreads) * 4;
+            *reinterpret_cast<float4 *>(&M[sw(e >> 6, e & 63)]) = m[u];
+        }
+    };
+    float4 pm[4], pa[4], pa2[4];
+    if (X0) {
+        mat_to_shared(smf, X0 + st0, t);
+    } else {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) reinterpret_cast<float4 *>(smf)[t + u * kThreads] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    if (count > 0) {
+        fetch_m(0, pm);
+        fetch_a(0, pa);
+        put_m(smf + 2 * MAT, pm);
+    }
+    if (count > 1) {
+        fetch_m(1, pm);
+        fetch_a(1, pa2);
+    }
     __syncthreads();
-    for (int cc = 0; cc < count; ++cc) {
-        const size_t base = ((size_t)(first + cc) * H + h) * (size_t)(N * N);
-        for (int i = t; i < N * N; i += kThreads) {
-            Sc[base + i] = S[(i >> 6) * LD + (i & 63)];
-            Mm[(i >> 6) * LD + (i & 63)] = Mo[base + i];
+    for (int i = 0; i < count; ++i) {
+        const int cur = i & 1;
+        float *Xcur = smf + cur * MAT, *Xnxt = smf + (cur ^ 1) * MAT, *Mcur = smf + (2 + cur) * MAT,
+              *Mnxt = smf + (3 - cur) * MAT;
+        mat_from_shared(Xc + chunk_base(i), Xcur, t);
+        float nx[16];
+        int id = 0;
+        mm<REV, false>(Mcur, Xcur, t, [&](int, int, float x) { nx[id++] = x; });
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            nx[4 * u] += pa[u].x;
+            nx[4 * u + 1] += pa[u].y;
+            nx[4 * u + 2] += pa[u].z;
+            nx[4 * u + 3] += pa[u].w;
+        }
+        put_block(Xnxt, nx, t);
+        if (i + 1 < count) {
+            put_m(Mnxt, pm);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) pa[u] = pa2[u];
+        }
+        if (i + 2 < count) {
+            fetch_m(i + 2, pm);
+            fetch_a(i + 2, pa2);
         }
         __syncthreads();
-        float nx[16];
-        int idx = 0;
-        mm<false, false>(Mm, S, t, [&](int r, int j, float x) { nx[idx++] = x + Bo[base + r * N + j]; });
-        __syncthreads();
-        idx = 0;
-        mm<false, false>(Mm, S, t, [&](int r, int j, float) { S[r * LD + j] = nx[idx++]; });
-        __syncthreads();
     }
-}
-
-// ---- bwd_bscan: dL/dS at the end of every chunk (reverse), and dS0 ---------------------------
-__global__ void __launch_bounds__(kThreads, 1)
-    bwd_bscan(const float *__restrict__ Mo, const float *__restrict__ Ro, const float *__restrict__ dS_final,
-              const int32_t *__restrict__ cu, const int32_t *__restrict__ off, int T, int H, float *__restrict__ dSn,
-              float *__restrict__ dS0)
-{
-    extern __shared__ float smf[];
-    float *D = smf, *Mm = D + MAT;
-    const int t = threadIdx.x, h = blockIdx.x, s = blockIdx.y;
-    int first, count;
-    seq_chunks(s, cu, off, T, first, count);
-    const size_t st0 = ((size_t)s * H + h) * (size_t)(N * N);
-    for (int i = t; i < N * N; i += kThreads) D[(i >> 6) * LD + (i & 63)] = dS_final ? dS_final[st0 + i] : 0.f;
-    __syncthreads();
-    for (int cc = count - 1; cc >= 0; --cc) {
-        const size_t base = ((size_t)(first + cc) * H + h) * (size_t)(N * N);
-        for (int i = t; i < N * N; i += kThreads) {
-            dSn[base + i] = D[(i >> 6) * LD + (i & 63)];
-            Mm[(i >> 6) * LD + (i & 63)] = Mo[base + i];
-        }
-        __syncthreads();
-        float nx[16];
-        int idx = 0;
-        mm<true, false>(Mm, D, t, [&](int r, int j, float x) { nx[idx++] = x + Ro[base + r * N + j]; });
-        __syncthreads();
-        idx = 0;
-        mm<true, false>(Mm, D, t, [&](int r, int j, float) { D[r * LD + j] = nx[idx++]; });
-        __syncthreads();
-    }
-    if (dS0)
-        for (int i = t; i < N * N; i += kThreads) dS0[st0 + i] = D[(i >> 6) * LD + (i & 63)];
+    if (Xend) mat_from_shared(Xend + st0, smf + (count & 1) * MAT, t);
 }
 
 // ---- bwd_grads: every input gradient of one (chunk, head) --------------------------------------
@@ -303,36 +454,45 @@ __global__ void __launch_bounds__(kThreads, 1)
               const int32_t *__restrict__ off, int nseq, int T, int H, float *__restrict__ dq,
               float *__restrict__ dk, float *__restrict__ dv, float *__restrict__ dla, float *__restrict__ dbe)
 {
-    extern __shared__ float smf[];
+    extern __shared__ __align__(16) float smf[];
     float *K = smf, *Q = K + MAT, *V = Q + MAT, *dO = V + MAT, *S = dO + MAT, *dSp = S + MAT, *KK = dSp + MAT,
           *Tm = KK + MAT, *X1 = Tm + MAT, *U = X1 + MAT, *QK = U + MAT, *dU = QK + MAT, *X2 = dU + MAT;
     Gates &g = *reinterpret_cast<Gates *>(X2 + MAT);
     float *vec = reinterpret_cast<float *>(&g + 1);
     float *bg = vec, *dG = vec + N, *dgam = vec + 2 * N, *dlam = vec + 3 * N, *dbet = vec + 4 * N, *dgC = vec + 5 * N;
+    float *colp = vec + 6 * N;  // 16 x 64 column partial sums
     const int t = threadIdx.x, h = blockIdx.y, e = blockIdx.x;
     const ChunkRef c = chunk_ref(e, cu, off, nseq, T);
     if (c.n == 0) return;
     const size_t base = ((size_t)e * H + h) * (size_t)(N * N);
-    load_rows(K, k, c, H, h, t);
-    load_rows(Q, q, c, H, h, t);
-    load_rows(V, v, c, H, h, t);
-    load_rows(dO, dout, c, H, h, t);
-    for (int i = t; i < N * N; i += kThreads) {
-        S[(i >> 6) * LD + (i & 63)] = Sc[base + i];
-        dSp[(i >> 6) * LD + (i & 63)] = dSn[base + i];
+    {
+        RowTile<TIn> tk, tq, tv, td;
+        tk.fetch(k, c, H, h, t);
+        tq.fetch(q, c, H, h, t);
+        tv.fetch(v, c, H, h, t);
+        td.fetch(dout, c, H, h, t);
+        mat_to_shared(S, Sc + base, t);
+        mat_to_shared(dSp, dSn + base, t);
+        tk.put(K, t);
+        tq.put(Q, t);
+        tv.put(V, t);
+        td.put(dO, t);
     }
-    vec[N + t] = 0.f;  // dG, dgam, dlam, dbet
     if (t == 0) dgC[0] = 0.f;
     chunk_gates<TIn>(g, log_alpha, beta, c, H, h, t);
     __syncthreads();
     if (t < N) bg[t] = g.bet[t] * g.gam[t];
+    const int r0 = (t >> 4) * 4, c0 = (t & 15) * 4;  // this thread's rows and columns in every product
     float aq[16], ak[16], av[16];  // this thread's 4 x 4 blocks of dQ, dK, dV
+    float pb[4], pg[4], pG[4], pc[4];  // partial d beta, d gam, dG over its rows; dG over its columns
 #pragma unroll
     for (int i = 0; i < 16; ++i) aq[i] = ak[i] = av[i] = 0.f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) pb[i] = pg[i] = pG[i] = pc[i] = 0.f;
     int id;
-    mm<false, true>(K, K, t, [&](int r, int i, float x) { KK[r * LD + i] = x; });
-    mm<false, true>(Q, K, t, [&](int r, int i, float x) { QK[r * LD + i] = x; });
-    mm<false, false>(K, dSp, t, [&](int i, int m, float x) { X2[i * LD + m] = x; });  // K dS'
+    mm<false, true>(K, K, t, [&](int r, int i, float x) { KK[sw(r, i)] = x; });
+    mm<false, true>(Q, K, t, [&](int r, int i, float x) { QK[sw(r, i)] = x; });
+    mm<false, false>(K, dSp, t, [&](int i, int m, float x) { X2[sw(i, m)] = x; });  // K dS'
     __syncthreads();
     // A (strictly lower) in dU for the solve; P in X1; d gam_C = <S, dS'>
     {
@@ -340,9 +500,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int idx = t; idx < N * N; idx += kThreads) {
             const int r = idx >> 6, i = idx & 63;
             const float gm = decay(g, r, i);
-            dU[r * LD + i] = i < r ? g.bet[r] * gm * KK[r * LD + i] : 0.f;
-            X1[r * LD + i] = gm * QK[r * LD + i];
-            part = fmaf(S[r * LD + i], dSp[r * LD + i], part);
+            dU[sw(r, i)] = i < r ? g.bet[r] * gm * KK[sw(r, i)] : 0.f;
+            X1[sw(r, i)] = gm * QK[sw(r, i)];
+            part = fmaf(S[sw(r, i)], dSp[sw(r, i)], part);
         }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
@@ -352,75 +512,80 @@ __global__ void __launch_bounds__(kThreads, 1)
     unit_lower_inverse(dU, Tm, t);
     __syncthreads();
     // U~ into U, W into dU (A is no longer needed)
-    mm<false, false>(Tm, V, t, [&](int r, int j, float x) { U[r * LD + j] = x; }, g.bet);
-    mm<false, false>(Tm, K, t, [&](int r, int m, float x) { dU[r * LD + m] = x; }, bg);
+    mm<false, false>(Tm, V, t, [&](int r, int j, float x) { U[sw(r, j)] = x; }, g.bet);
+    mm<false, false>(Tm, K, t, [&](int r, int m, float x) { dU[sw(r, m)] = x; }, bg);
     __syncthreads();
     // U = U~ - W S
-    mm<false, false>(dU, S, t, [&](int r, int j, float x) { U[r * LD + j] -= x; });
+    mm<false, false>(dU, S, t, [&](int r, int j, float x) { U[sw(r, j)] -= x; });
     __syncthreads();
-    // dU = P^T dO + diag(lam) K dS'; d lam_i = sum_j (K dS')_ij U_ij
-    mm<true, false>(X1, dO, t, [&](int i, int j, float x) {
-        dU[i * LD + j] = x + g.lam[i] * X2[i * LD + j];
-        atomicAdd(&dlam[i], X2[i * LD + j] * U[i * LD + j]);
+    // dU = P^T dO + diag(lam) K dS'; d lam_i = sum_j (K dS')_ij U_ij (the only term of d lam)
+    {
+        float pl[4] = {0.f, 0.f, 0.f, 0.f};
+        mm<true, false>(X1, dO, t, [&](int i, int j, float x) {
+            const float kd = X2[sw(i, j)];
+            dU[sw(i, j)] = x + g.lam[i] * kd;
+            pl[i - r0] = fmaf(kd, U[sw(i, j)], pl[i - r0]);
+        });
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float sum = row_block_sum(pl[i]);
+            if ((t & 15) == 0) dlam[r0 + i] = sum;
+        }
+    }
+    __syncthreads();
+    // dP = dO U^T (lower incl.), and at once D2 = dP o Gam into X1 (P is no longer needed) with the
+    // dG terms of Gam (P); dK += diag(lam) U dS'^T; d gam (O1) and dQ += diag(gam) dO S^T
+    mm<false, true>(dO, U, t, [&](int r, int i, float x) {
+        const float gm = decay(g, r, i), dp = i <= r ? x : 0.f;
+        X1[sw(r, i)] = dp * gm;
+        const float E = dp * QK[sw(r, i)] * gm;
+        pG[r - r0] += E;
+        pc[i - c0] -= E;
     });
-    __syncthreads();
-    // dP = dO U^T (lower incl.) over P; dK += diag(lam) U dS'^T; d gam (O1) and dQ += diag(gam) dO S^T
-    mm<false, true>(dO, U, t, [&](int r, int i, float x) { X1[r * LD + i] = i <= r ? x : 0.f; });
     id = 0;
     mm<false, true>(U, dSp, t, [&](int i, int m, float x) { ak[id++] += g.lam[i] * x; });
     id = 0;
     mm<false, true>(dO, S, t, [&](int r, int m, float x) { aq[id++] += g.gam[r] * x; });
-    mm<false, false>(Q, S, t, [&](int r, int j, float x) { atomicAdd(&dgam[r], dO[r * LD + j] * x); });
+    mm<false, false>(Q, S, t, [&](int r, int j, float x) { pg[r - r0] = fmaf(dO[sw(r, j)], x, pg[r - r0]); });
     __syncthreads();
     // dW = -dU S^T into U (U is no longer needed)
-    mm<false, true>(dU, S, t, [&](int r, int m, float x) { U[r * LD + m] = -x; });
+    mm<false, true>(dU, S, t, [&](int r, int m, float x) { U[sw(r, m)] = -x; });
     __syncthreads();
     // Y = T^T dU: dV, dbeta;  X = T^T dW: dK, dbeta, d gam
     id = 0;
     mm<true, false>(Tm, dU, t, [&](int i, int j, float x) {
         av[id++] += g.bet[i] * x;
-        atomicAdd(&dbet[i], x * V[i * LD + j]);
+        pb[i - r0] = fmaf(x, V[sw(i, j)], pb[i - r0]);
     });
     id = 0;
     mm<true, false>(Tm, U, t, [&](int i, int m, float x) {
         ak[id++] += bg[i] * x;
-        const float xk = x * K[i * LD + m];
-        atomicAdd(&dbet[i], g.gam[i] * xk);
-        atomicAdd(&dgam[i], g.bet[i] * xk);
+        const float xk = x * K[sw(i, m)];
+        pb[i - r0] = fmaf(g.gam[i], xk, pb[i - r0]);
+        pg[i - r0] = fmaf(g.bet[i], xk, pg[i - r0]);
     });
     // dT = dU (diag(b) V)^T + dW (diag(b gam) K)^T into X2 (K dS' is no longer needed); the
     // diagonals scale the result's column index
-    mm<false, true>(dU, V, t, [&](int r, int i, float x) { X2[r * LD + i] = g.bet[i] * x; });
-    mm<false, true>(U, K, t, [&](int r, int i, float x) { X2[r * LD + i] += bg[i] * x; });
+    mm<false, true>(dU, V, t, [&](int r, int i, float x) { X2[sw(r, i)] = g.bet[i] * x; });
+    mm<false, true>(U, K, t, [&](int r, int i, float x) { X2[sw(r, i)] += bg[i] * x; });
     __syncthreads();
     // Z = dT T^T into dU
-    mm<false, true>(X2, Tm, t, [&](int r, int i, float x) { dU[r * LD + i] = x; });
+    mm<false, true>(X2, Tm, t, [&](int r, int i, float x) { dU[sw(r, i)] = x; });
     __syncthreads();
     // dA = -T^T Z (strictly lower) -> D into U; dbeta (A); dG from Gam (A)
     mm<true, false>(Tm, dU, t, [&](int r, int i, float x) {
         float d = 0.f;
         if (i < r) {
-            const float dA = -x, gm = decay(g, r, i);
-            const float dAbar = g.bet[r] * dA;
-            d = dAbar * gm;
-            atomicAdd(&dbet[r], dA * gm * KK[r * LD + i]);
-            const float E = dAbar * KK[r * LD + i] * gm;
-            atomicAdd(&dG[r], E);
-            atomicAdd(&dG[i], -E);
+            const float gm = decay(g, r, i), kk = KK[sw(r, i)];
+            const float dAg = -x * gm;  // dA o Gam
+            d = g.bet[r] * dAg;
+            pb[r - r0] = fmaf(dAg, kk, pb[r - r0]);
+            const float E = d * kk;
+            pG[r - r0] += E;
+            pc[i - c0] -= E;
         }
-        U[r * LD + i] = d;
+        U[sw(r, i)] = d;
     });
-    // D2 = dP o Gam in X1; dG from Gam (P)
-    for (int idx = t; idx < N * N; idx += kThreads) {
-        const int r = idx >> 6, i = idx & 63;
-        const float gm = decay(g, r, i), dp = X1[r * LD + i];
-        X1[r * LD + i] = dp * gm;
-        const float E = dp * QK[r * LD + i] * gm;
-        if (E != 0.f) {
-            atomicAdd(&dG[r], E);
-            atomicAdd(&dG[i], -E);
-        }
-    }
     __syncthreads();
     // dK += D K + D^T K + D2^T Q;  dQ += D2 K
     id = 0;
@@ -431,39 +596,58 @@ __global__ void __launch_bounds__(kThreads, 1)
     mm<true, false>(X1, Q, t, [&](int i, int m, float x) { ak[id++] += x; });
     id = 0;
     mm<false, false>(X1, K, t, [&](int r, int m, float x) { aq[id++] += x; });
+    // the partial sums: rows over the 16 threads of a row block, columns over the 16 row blocks
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float sb = row_block_sum(pb[i]), sg = row_block_sum(pg[i]), sG = row_block_sum(pG[i]);
+        if ((t & 15) == 0) {
+            dbet[r0 + i] = sb;
+            dgam[r0 + i] = sg;
+            dG[r0 + i] = sG;
+        }
+        colp[(t >> 4) * N + c0 + i] = pc[i];
+    }
+    __syncthreads();
+    if (t < N) {
+        float sum = 0.f;
+#pragma unroll
+        for (int b = 0; b < 16; ++b) sum += colp[b * N + t];
+        dG[t] += sum;
+    }
     __syncthreads();
     // gate gradients: gam_r = exp(G_r), lam_i = exp(G_63 - G_i), gam_C = gam_63; then dlog_alpha_j =
-    // sum of dG_r over the rows r >= j of j's reset segment (0 at a reset itself)
-    if (t == 0) {
-        for (int r = 0; r < N; ++r) dG[r] += dgam[r] * g.gam[r];
-        float s63 = dgC[0] * g.gam[N - 1];
-        for (int i = 0; i < N; ++i) {
-            const float li = dlam[i] * g.lam[i];
-            s63 += li;
-            dG[i] -= li;
+    // sum of dG_r over the rows r >= j of j's reset segment (0 at a reset itself): a segmented sum
+    // over the reversed rows, restarting below every reset
+    if (t < 32) {
+        float x[2], li[2];
+        int f[2];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const int j = N - 1 - (t + 32 * u);
+            li[u] = dlam[j] * g.lam[j];
+            x[u] = dG[j] + dgam[j] * g.gam[j] - li[u];
+            f[u] = j < N - 1 && g.last[j + 1] == j + 1;
         }
-        dG[N - 1] += s63;
-        float acc = 0.f;
-        for (int j = N - 1; j >= 0; --j) {
-            acc += dG[j];
-            const bool reset = g.last[j] == j;
-            dlam[j] = reset ? 0.f : acc;  // reuse as dlog_alpha
-            if (reset) acc = 0.f;
+        float s63 = li[0] + li[1];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) s63 += __shfl_xor_sync(0xffffffffu, s63, o);
+        if (t == 0) x[0] += s63 + dgC[0] * g.gam[N - 1];  // row 63
+        seg_scan64(x[0], f[0], x[1], f[1], t);
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const int j = N - 1 - (t + 32 * u);
+            dlam[j] = g.last[j] == j ? 0.f : x[u];  // reuse as dlog_alpha
         }
     }
     __syncthreads();
-    const int r0 = (t >> 4) * 4, c0 = (t & 15) * 4;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
         const int r = r0 + i;
         if (r >= c.n) continue;
         const size_t row = ((size_t)(c.tok + r) * H + h) * N + c0;
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            dq[row + j] = aq[i * 4 + j];
-            dk[row + j] = ak[i * 4 + j];
-            dv[row + j] = av[i * 4 + j];
-        }
+        *reinterpret_cast<float4 *>(dq + row) = make_float4(aq[4 * i], aq[4 * i + 1], aq[4 * i + 2], aq[4 * i + 3]);
+        *reinterpret_cast<float4 *>(dk + row) = make_float4(ak[4 * i], ak[4 * i + 1], ak[4 * i + 2], ak[4 * i + 3]);
+        *reinterpret_cast<float4 *>(dv + row) = make_float4(av[4 * i], av[4 * i + 1], av[4 * i + 2], av[4 * i + 3]);
     }
     if (t < c.n) {
         const size_t o = (size_t)(c.tok + t) * H + h;
@@ -522,17 +706,21 @@ cudaError_t run_bwd(const BwdArgs &a, cudaStream_t st)
     const TIn *q = static_cast<const TIn *>(a.q), *k = static_cast<const TIn *>(a.k),
               *v = static_cast<const TIn *>(a.v), *dout = static_cast<const TIn *>(a.dout);
     const int smem_prep = (9 * MAT) * (int)sizeof(float) + (int)sizeof(Gates) + N * (int)sizeof(float);
-    const int smem_grads = (13 * MAT) * (int)sizeof(float) + (int)sizeof(Gates) + 6 * N * (int)sizeof(float);
-    const int smem_scan = 2 * MAT * (int)sizeof(float);
+    const int smem_grads = (13 * MAT) * (int)sizeof(float) + (int)sizeof(Gates) + (6 + 16) * N * (int)sizeof(float);
+    const int smem_scan = 4 * MAT * (int)sizeof(float);
     cudaError_t e = cudaFuncSetAttribute(bwd_prep<TIn>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_prep);
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(bwd_grads<TIn>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_grads);
     if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(bwd_scan<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_scan);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(bwd_scan<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_scan);
+    if (e != cudaSuccess) return e;
     const dim3 gc((unsigned)chunks, a.H), gs(a.H, a.B);
     bwd_prep<TIn><<<gc, kThreads, smem_prep, st>>>(q, k, v, a.log_alpha, a.beta, dout, a.cu_seqlens, offp, a.B, a.T,
                                                    a.H, Mo, Bo, Ro);
-    bwd_fscan<<<gs, kThreads, smem_scan, st>>>(Mo, Bo, a.S0, a.cu_seqlens, offp, a.T, a.H, Sc);
-    bwd_bscan<<<gs, kThreads, smem_scan, st>>>(Mo, Ro, a.dS_final, a.cu_seqlens, offp, a.T, a.H, dSn, a.dS0);
+    bwd_scan<false><<<gs, kThreads, smem_scan, st>>>(Mo, Bo, a.S0, a.cu_seqlens, offp, a.T, a.H, Sc, nullptr);
+    bwd_scan<true><<<gs, kThreads, smem_scan, st>>>(Mo, Ro, a.dS_final, a.cu_seqlens, offp, a.T, a.H, dSn, a.dS0);
     bwd_grads<TIn><<<gc, kThreads, smem_grads, st>>>(q, k, v, a.log_alpha, a.beta, dout, Sc, dSn, a.cu_seqlens, offp,
                                                      a.B, a.T, a.H, a.dq, a.dk, a.dv, a.dlog_alpha, a.dbeta);
     return cudaGetLastError();
