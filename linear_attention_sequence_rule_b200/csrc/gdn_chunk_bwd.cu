@@ -29,16 +29,14 @@ constexpr int N = 64;          // chunk length = dk = dv
 constexpr int MAT = N * N;     // floats per matrix
 constexpr int kThreads = 256;
 
-// Shared matrices are 64 x 64 fp32 with 64-float rows; the 16 groups of 4 floats of row r are
-// stored in the order group ^ ((r / 4) mod 16), so that the 16-byte loads of a matrix product
-// spread over the banks.  Element (r, c) lives at sw(r, c).
+// Shared matrices are 64 x 64 fp32 with 64-float rows; column c of row r is stored at position
+// c ^ 4 sigma(r mod 8), sigma = (0 2 4 6 1 3 5 7), which moves whole 16-byte groups.  Both access
+// patterns of the tensor-core fragments -- 8 rows x 4 columns and 4 rows x 8 columns -- then fall
+// on 32 different banks, and so do whole rows.  Element (r, c) lives at sw(r, c).
 __device__ __forceinline__ int sw(int r, int c)
 {
-    return r * N + ((((c >> 2) ^ (r >> 2)) & 15) << 2) + (c & 3);
+    return r * N + (c ^ (((r & 3) << 3) | (((r >> 2) & 1) << 2)));
 }
-
-__device__ __forceinline__ float ld_in(const float *p) { return *p; }
-__device__ __forceinline__ float ld_in(const __nv_bfloat16 *p) { return __bfloat162float(*p); }
 
 // One chunk's place: sequence, first token, valid rows, chunk index inside the sequence.
 struct ChunkRef {
@@ -75,70 +73,145 @@ __device__ ChunkRef chunk_ref(int e, const int32_t *cu, const int32_t *off, int 
     return r;
 }
 
-// C(r, c) = sum_k opA(r, k) ks[k] opB(k, c) for 64 x 64 operands (ks: optional diagonal, NULL = 1);
-// thread t gets rows 4 (t / 16) .. +3 and columns 4 (t % 16) .. +3 and hands each result to
-// emit(r, c, value).  Four steps of k at a time, every operand read as 16-byte groups.
+// fp32 x fp32 on the tensor cores: x = hi + lo with hi, lo tf32 (11 significant bits each), and
+// a b ~ hi_a hi_b + hi_a lo_b + lo_a hi_b (the dropped lo_a lo_b is below 2^-22 |a b|).
+__device__ __forceinline__ void split_tf32(float x, uint32_t &hi, uint32_t &lo)
+{
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(hi) : "f"(x));
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(lo) : "f"(x - __uint_as_float(hi)));
+}
+
+__device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1)
+{
+    asm volatile("mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+                 "{%0,%1,%2,%3};"
+                 : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+                 : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// The dynamic shared memory of every kernel in this file.
+extern __shared__ __align__(16) float smf[];
+
+// One thread's 16 results of a product, index u (see mm).
+struct Frag {
+    float v[16];
+};
+
+// C(r, c) = sum_k opA(r, k) ks[k] opB(k, c) for 64 x 64 operands (opA = A or A^T, opB = B or B^T;
+// ks: optional diagonal), on the tensor cores with the three-term tf32 split.  Warp w computes
+// rows 16 (w mod 4) .. +15 and columns 32 (w / 4) .. +31; lane l holds rows 16 (w mod 4) + l / 4 +
+// {0, 8} and columns 32 (w / 4) + 8 n + 2 (l mod 4) + {0, 1}, n = 0..3, as element
+// u = 4 n + 2 (row half) + (column parity) of its Frag -- the same u for the same (r, c) in every
+// product, so per-thread accumulators can be indexed by it.  The operands are given as offsets
+// into the shared memory.  Kept out of line: a kernel runs this loop some twenty times, and one
+// shared copy of it stays in the instruction cache.
+template <bool TA, bool TB, bool KS>
+__device__ __noinline__ Frag mm_core(int a_off, int b_off, int ks_off)
+{
+    const float *A = smf + a_off, *B = smf + b_off, *ks = smf + ks_off;
+    const int t = threadIdx.x, lane = t & 31, w = t >> 5, g = lane >> 2, q = lane & 3;
+    const int m0 = (w & 3) * 16, n0 = (w >> 2) * 32;
+    float acc[4][4], cor[4][4];  // hi x hi, and the two cross terms (independent chains)
+#pragma unroll
+    for (int n = 0; n < 4; ++n)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[n][j] = cor[n][j] = 0.f;
+#pragma unroll 1
+    for (int k0 = 0; k0 < N; k0 += 8) {
+        float a[4];  // opA at (m0 + g, k0 + q), (m0 + g + 8, k0 + q), (m0 + g, k0 + q + 4), (m0 + g + 8, k0 + q + 4)
+        a[0] = TA ? A[sw(k0 + q, m0 + g)] : A[sw(m0 + g, k0 + q)];
+        a[1] = TA ? A[sw(k0 + q, m0 + g + 8)] : A[sw(m0 + g + 8, k0 + q)];
+        a[2] = TA ? A[sw(k0 + q + 4, m0 + g)] : A[sw(m0 + g, k0 + q + 4)];
+        a[3] = TA ? A[sw(k0 + q + 4, m0 + g + 8)] : A[sw(m0 + g + 8, k0 + q + 4)];
+        if (KS) {
+            const float s0 = ks[k0 + q], s1 = ks[k0 + q + 4];
+            a[0] *= s0;
+            a[1] *= s0;
+            a[2] *= s1;
+            a[3] *= s1;
+        }
+        uint32_t ah[4], al[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) split_tf32(a[j], ah[j], al[j]);
+#pragma unroll
+        for (int n = 0; n < 4; ++n) {
+            const int col = n0 + 8 * n + g;  // opB at (k0 + q, col), (k0 + q + 4, col)
+            const float b0 = TB ? B[sw(col, k0 + q)] : B[sw(k0 + q, col)];
+            const float b1 = TB ? B[sw(col, k0 + q + 4)] : B[sw(k0 + q + 4, col)];
+            uint32_t bh0, bl0, bh1, bl1;
+            split_tf32(b0, bh0, bl0);
+            split_tf32(b1, bh1, bl1);
+            mma_tf32(cor[n], al, bh0, bh1);
+            mma_tf32(acc[n], ah, bh0, bh1);
+            mma_tf32(cor[n], ah, bl0, bl1);
+        }
+    }
+    Frag f;
+#pragma unroll
+    for (int n = 0; n < 4; ++n)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) f.v[4 * n + j] = acc[n][j] + cor[n][j];
+    return f;
+}
+
+// The product of mm_core, handed element by element to emit(r, c, value, u).  A, B and ks (NULL:
+// no diagonal) point into the shared memory.
 template <bool TA, bool TB, typename F>
 __device__ __forceinline__ void mm(const float *A, const float *B, int t, F &&emit, const float *ks = nullptr)
 {
-    const int r0 = (t >> 4) * 4, c0 = (t & 15) * 4;
-    float acc[4][4];
+    const int lane = t & 31, w = t >> 5, g = lane >> 2, q = lane & 3;
+    const int m0 = (w & 3) * 16, n0 = (w >> 2) * 32;
+    const Frag f = ks ? mm_core<TA, TB, true>((int)(A - smf), (int)(B - smf), (int)(ks - smf))
+                      : mm_core<TA, TB, false>((int)(A - smf), (int)(B - smf), 0);
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
+    for (int n = 0; n < 4; ++n)
 #pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
-#pragma unroll 2
-    for (int k0 = 0; k0 < N; k0 += 4) {
-        float a[4][4], b[4][4];  // a[i][kk] = opA(r0 + i, k0 + kk), b[kk][j] = opB(k0 + kk, c0 + j)
+        for (int hh = 0; hh < 2; ++hh)
 #pragma unroll
-        for (int x = 0; x < 4; ++x) {
-            const float4 va = TA ? *reinterpret_cast<const float4 *>(&A[sw(k0 + x, r0)])
-                                 : *reinterpret_cast<const float4 *>(&A[sw(r0 + x, k0)]);
-            if (TA) { a[0][x] = va.x; a[1][x] = va.y; a[2][x] = va.z; a[3][x] = va.w; }
-            else { a[x][0] = va.x; a[x][1] = va.y; a[x][2] = va.z; a[x][3] = va.w; }
-            const float4 vb = TB ? *reinterpret_cast<const float4 *>(&B[sw(c0 + x, k0)])
-                                 : *reinterpret_cast<const float4 *>(&B[sw(k0 + x, c0)]);
-            if (TB) { b[0][x] = vb.x; b[1][x] = vb.y; b[2][x] = vb.z; b[3][x] = vb.w; }
-            else { b[x][0] = vb.x; b[x][1] = vb.y; b[x][2] = vb.z; b[x][3] = vb.w; }
-        }
-        if (ks) {
-            const float4 s4 = *reinterpret_cast<const float4 *>(&ks[k0]);
-            const float sv[4] = {s4.x, s4.y, s4.z, s4.w};
+            for (int e = 0; e < 2; ++e)
+                emit(m0 + g + 8 * hh, n0 + 8 * n + 2 * q + e, f.v[4 * n + 2 * hh + e], 4 * n + 2 * hh + e);
+}
+
+// Per-thread partial sums over the rows and columns a thread holds in mm's layout, completed over
+// the block in two steps: *_put writes a thread's share to scratch shared memory (rows: two per
+// thread, u bit 1, summed over the 4 lanes of a row, 2 x 64 floats of scratch; columns: eight per
+// thread, u / 4 and u bit 0, summed over the 8 row groups of a warp, 4 x 64 floats), and after a
+// barrier *_get(j) returns the total of row or column j.
+__device__ __forceinline__ void row_put(const float (&p)[2], float *buf, int t)
+{
+    const int lane = t & 31, w = t >> 5, r = (w & 3) * 16 + (lane >> 2);
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk) a[i][kk] *= sv[kk];
-        }
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-#pragma unroll
-                for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i][kk], b[kk][j], acc[i][j]);
+    for (int hh = 0; hh < 2; ++hh) {
+        float x = p[hh];
+        x += __shfl_xor_sync(0xffffffffu, x, 1);
+        x += __shfl_xor_sync(0xffffffffu, x, 2);
+        if ((lane & 3) == 0) buf[(w >> 2) * N + r + 8 * hh] = x;
     }
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) emit(r0 + i, c0 + j, acc[i][j]);
 }
 
-// Thread t's 4 x 4 block of a product (the layout mm hands out) into the shared matrix C.
-__device__ __forceinline__ void put_block(float *C, const float (&x)[16], int t)
+__device__ __forceinline__ float row_get(const float *buf, int j) { return buf[j] + buf[N + j]; }
+
+__device__ __forceinline__ void col_put(const float (&p)[8], float *buf, int t)
 {
-    const int r0 = (t >> 4) * 4, c0 = (t & 15) * 4;
+    const int lane = t & 31, w = t >> 5;
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
-        *reinterpret_cast<float4 *>(&C[sw(r0 + i, c0)]) = make_float4(x[4 * i], x[4 * i + 1], x[4 * i + 2], x[4 * i + 3]);
+    for (int j = 0; j < 8; ++j) {
+        float x = p[j];
+        x += __shfl_xor_sync(0xffffffffu, x, 4);
+        x += __shfl_xor_sync(0xffffffffu, x, 8);
+        x += __shfl_xor_sync(0xffffffffu, x, 16);
+        if (lane < 4) buf[(w & 3) * N + (w >> 2) * 32 + 8 * (j >> 1) + 2 * lane + (j & 1)] = x;
+    }
 }
 
-// Sum of a value over the 16 threads that share a row block (lanes l, l ^ 1, ..., l ^ 15 of a
-// half warp): every one of them gets the total.
-__device__ __forceinline__ float row_block_sum(float x)
+__device__ __forceinline__ float col_get(const float *buf, int j)
 {
-#pragma unroll
-    for (int o = 1; o < 16; o <<= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
-    return x;
+    return buf[j] + buf[N + j] + buf[2 * N + j] + buf[3 * N + j];
 }
+
+// Row half (0, 1) and column slot (0..7) of mm's element index u.
+__device__ __forceinline__ constexpr int u_row(int u) { return (u >> 1) & 1; }
+__device__ __forceinline__ constexpr int u_col(int u) { return ((u >> 2) << 1) | (u & 1); }
 
 // Inclusive sums of x over the 32 lanes of a warp, restarted at every lane whose f is set (f on
 // return: a restart lies at or before this lane).
@@ -275,23 +348,28 @@ __device__ __forceinline__ void mat_from_shared(float *dst, const float *M, int 
     }
 }
 
-// T = (I + A)^{-1} for strictly lower A (only entries below the diagonal are read): column c by
-// forward substitution on thread c (threads 0..63); every entry of T is written.
-__device__ void unit_lower_inverse(const float *A, float *Tm, int t)
+// T = (I + A)^{-1} for strictly lower A, given transposed (At(i, r) = A(r, i); only i < r is read).
+// Column c of T is found by forward substitution on threads 4c .. 4c + 3, thread 4c + q holding
+// rows q, q + 4, ..., q + 60: once row j is final it is passed among the four and subtracted from
+// every later row, so one multiply-add lies between row j and row j + 1.  A warp holds columns
+// 8w .. 8w + 7, whose rows above 8w are zero, and skips those steps.  Every entry of T is written.
+__device__ void unit_lower_inverse(const float *At, float *Tm, int t)
 {
-    if (t < N) {
-        const int c = t;
-        float x[N];
+    const int c = t >> 2, q = t & 3, w8 = (t >> 5) * 8;
+    float s[16];
 #pragma unroll
-        for (int r = 0; r < N; ++r) {
-            float s = 0.f;
+    for (int m = 0; m < 16; ++m) s[m] = (4 * m + q == c) ? 1.f : 0.f;
 #pragma unroll
-            for (int i = 0; i < r; ++i) s = fmaf(A[sw(r, i)], x[i], s);
-            x[r] = r < c ? 0.f : (r == c ? 1.f : -s);
+    for (int j = 0; j < N; ++j) {
+        if (j >= w8) {
+            const float xj = __shfl_sync(0xffffffffu, s[j >> 2], j & 3, 4);
+#pragma unroll
+            for (int m = j >> 2; m < 16; ++m)
+                if (4 * m + q > j) s[m] = fmaf(-At[sw(j, 4 * m + q)], xj, s[m]);
         }
-#pragma unroll
-        for (int r = 0; r < N; ++r) Tm[sw(r, c)] = x[r];
     }
+#pragma unroll
+    for (int m = 0; m < 16; ++m) Tm[sw(4 * m + q, c)] = s[m];
 }
 
 // ---- bwd_prep: per (chunk, head) the forward map (M, Bm) and the output term R ----------------
@@ -302,7 +380,6 @@ __global__ void __launch_bounds__(kThreads, 1)
              const int32_t *__restrict__ cu, const int32_t *__restrict__ off, int nseq, int T, int H,
              float *__restrict__ Mo, float *__restrict__ Bo, float *__restrict__ Ro)
 {
-    extern __shared__ __align__(16) float smf[];
     float *K = smf, *Q = K + MAT, *V = Q + MAT, *dO = V + MAT, *A = dO + MAT, *Tm = A + MAT, *W = Tm + MAT,
           *Ut = W + MAT, *P = Ut + MAT;
     Gates &g = *reinterpret_cast<Gates *>(P + MAT);
@@ -324,22 +401,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     chunk_gates<TIn>(g, log_alpha, beta, c, H, h, t);
     __syncthreads();
     if (t < N) bg[t] = g.bet[t] * g.gam[t];
-    mm<false, true>(K, K, t, [&](int r, int i, float x) { A[sw(r, i)] = i < r ? g.bet[r] * decay(g, r, i) * x : 0.f; });
-    mm<false, true>(Q, K, t, [&](int r, int i, float x) { P[sw(r, i)] = decay(g, r, i) * x; });
+    // A transposed: At(i, r) = b_r Gam_ri (K K^T)_ri for i < r (K K^T is symmetric)
+    mm<false, true>(K, K, t, [&](int i, int r, float x, int) { A[sw(i, r)] = i < r ? g.bet[r] * decay(g, r, i) * x : 0.f; });
+    mm<false, true>(Q, K, t, [&](int r, int i, float x, int) { P[sw(r, i)] = decay(g, r, i) * x; });
     __syncthreads();
     unit_lower_inverse(A, Tm, t);
     __syncthreads();
-    mm<false, false>(Tm, K, t, [&](int r, int m, float x) { W[sw(r, m)] = x; }, bg);
-    mm<false, false>(Tm, V, t, [&](int r, int j, float x) { Ut[sw(r, j)] = x; }, g.bet);
-    mm<true, false>(P, dO, t, [&](int i, int j, float x) { A[sw(i, j)] = x; });  // Y = P^T dO (A is free)
+    mm<false, false>(Tm, K, t, [&](int r, int m, float x, int) { W[sw(r, m)] = x; }, bg);
+    mm<false, false>(Tm, V, t, [&](int r, int j, float x, int) { Ut[sw(r, j)] = x; }, g.bet);
+    mm<true, false>(P, dO, t, [&](int i, int j, float x, int) { A[sw(i, j)] = x; });  // Y = P^T dO (A is free)
     __syncthreads();
     const size_t base = ((size_t)e * H + h) * (size_t)(N * N);
     const float gC = g.gam[N - 1];
-    mm<true, false>(K, W, t, [&](int m, int n2, float x) { Mo[base + m * N + n2] = (m == n2 ? gC : 0.f) - x; }, g.lam);
-    mm<true, false>(K, Ut, t, [&](int m, int j, float x) { Bo[base + m * N + j] = x; }, g.lam);
-    mm<true, false>(Q, dO, t, [&](int m, int j, float x) { Tm[sw(m, j)] = x; }, g.gam);  // T is free
+    mm<true, false>(K, W, t, [&](int m, int n2, float x, int) { Mo[base + m * N + n2] = (m == n2 ? gC : 0.f) - x; }, g.lam);
+    mm<true, false>(K, Ut, t, [&](int m, int j, float x, int) { Bo[base + m * N + j] = x; }, g.lam);
+    mm<true, false>(Q, dO, t, [&](int m, int j, float x, int) { Tm[sw(m, j)] = x; }, g.gam);  // T is free
     __syncthreads();
-    mm<true, false>(W, A, t, [&](int m, int j, float x) { Ro[base + m * N + j] = Tm[sw(m, j)] - x; });
+    mm<true, false>(W, A, t, [&](int m, int j, float x, int) { Ro[base + m * N + j] = Tm[sw(m, j)] - x; });
 }
 
 // Number of chunks of sequence s and the table index of its first chunk.
@@ -366,9 +444,9 @@ __global__ void __launch_bounds__(kThreads, 1)
              const int32_t *__restrict__ cu, const int32_t *__restrict__ off, int T, int H, float *__restrict__ Xc,
              float *__restrict__ Xend)
 {
-    extern __shared__ __align__(16) float smf[];  // X[2], then M[2]
+    // shared memory: X[2], then M[2]
     const int t = threadIdx.x, h = blockIdx.x, s = blockIdx.y;
-    const int r0 = (t >> 4) * 4, c0 = (t & 15) * 4;
+    const int g = (t & 31) >> 2, q = t & 3, m0 = ((t >> 5) & 3) * 16, n0 = (t >> 7) * 32;
     int first, count;
     seq_chunks(s, cu, off, T, first, count);
     const size_t st0 = ((size_t)s * H + h) * (size_t)MAT;
@@ -378,10 +456,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int u = 0; u < 4; ++u) m[u] = __ldg(src + t + u * kThreads);
     };
-    auto fetch_a = [&](int i, float4 (&a)[4]) {
+    auto fetch_a = [&](int i, float2 (&a)[8]) {  // the additive term in mm's layout
         const float *src = Add + chunk_base(i);
 #pragma unroll
-        for (int u = 0; u < 4; ++u) a[u] = __ldg(reinterpret_cast<const float4 *>(src + (r0 + u) * N + c0));
+        for (int n = 0; n < 4; ++n)
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh)
+                a[2 * n + hh] = __ldg(reinterpret_cast<const float2 *>(src + (m0 + g + 8 * hh) * N + n0 + 8 * n + 2 * q));
     };
     auto put_m = [&](float *M, const float4 (&m)[4]) {
 #pragma unroll
@@ -390,7 +471,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             *reinterpret_cast<float4 *>(&M[sw(e >> 6, e & 63)]) = m[u];
         }
     };
-    float4 pm[4], pa[4], pa2[4];
+    float4 pm[4];
+    float2 pa[8], pa2[8];
     if (X0) {
         mat_to_shared(smf, X0 + st0, t);
     } else {
@@ -412,21 +494,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         float *Xcur = smf + cur * MAT, *Xnxt = smf + (cur ^ 1) * MAT, *Mcur = smf + (2 + cur) * MAT,
               *Mnxt = smf + (3 - cur) * MAT;
         mat_from_shared(Xc + chunk_base(i), Xcur, t);
-        float nx[16];
-        int id = 0;
-        mm<REV, false>(Mcur, Xcur, t, [&](int, int, float x) { nx[id++] = x; });
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            nx[4 * u] += pa[u].x;
-            nx[4 * u + 1] += pa[u].y;
-            nx[4 * u + 2] += pa[u].z;
-            nx[4 * u + 3] += pa[u].w;
-        }
-        put_block(Xnxt, nx, t);
+        mm<REV, false>(Mcur, Xcur, t, [&](int r, int c, float x, int u) {
+            const float2 a = pa[2 * (u >> 2) + u_row(u)];
+            Xnxt[sw(r, c)] = x + ((u & 1) ? a.y : a.x);
+        });
         if (i + 1 < count) {
             put_m(Mnxt, pm);
 #pragma unroll
-            for (int u = 0; u < 4; ++u) pa[u] = pa2[u];
+            for (int u = 0; u < 8; ++u) pa[u] = pa2[u];
         }
         if (i + 2 < count) {
             fetch_m(i + 2, pm);
@@ -454,13 +529,11 @@ __global__ void __launch_bounds__(kThreads, 1)
               const int32_t *__restrict__ off, int nseq, int T, int H, float *__restrict__ dq,
               float *__restrict__ dk, float *__restrict__ dv, float *__restrict__ dla, float *__restrict__ dbe)
 {
-    extern __shared__ __align__(16) float smf[];
     float *K = smf, *Q = K + MAT, *V = Q + MAT, *dO = V + MAT, *S = dO + MAT, *dSp = S + MAT, *KK = dSp + MAT,
           *Tm = KK + MAT, *X1 = Tm + MAT, *U = X1 + MAT, *QK = U + MAT, *dU = QK + MAT, *X2 = dU + MAT;
     Gates &g = *reinterpret_cast<Gates *>(X2 + MAT);
     float *vec = reinterpret_cast<float *>(&g + 1);
     float *bg = vec, *dG = vec + N, *dgam = vec + 2 * N, *dlam = vec + 3 * N, *dbet = vec + 4 * N, *dgC = vec + 5 * N;
-    float *colp = vec + 6 * N;  // 16 x 64 column partial sums
     const int t = threadIdx.x, h = blockIdx.y, e = blockIdx.x;
     const ChunkRef c = chunk_ref(e, cu, off, nseq, T);
     if (c.n == 0) return;
@@ -482,26 +555,26 @@ __global__ void __launch_bounds__(kThreads, 1)
     chunk_gates<TIn>(g, log_alpha, beta, c, H, h, t);
     __syncthreads();
     if (t < N) bg[t] = g.bet[t] * g.gam[t];
-    const int r0 = (t >> 4) * 4, c0 = (t & 15) * 4;  // this thread's rows and columns in every product
-    float aq[16], ak[16], av[16];  // this thread's 4 x 4 blocks of dQ, dK, dV
-    float pb[4], pg[4], pG[4], pc[4];  // partial d beta, d gam, dG over its rows; dG over its columns
+    // per thread, in mm's layout (index u): the dQ, dK, dV accumulators; partial d beta, d gam, dG
+    // and d lam over its two rows; partial dG over its eight columns
+    float aq[16], ak[16], av[16];
+    float pb[2] = {0.f, 0.f}, pg[2] = {0.f, 0.f}, pG[2] = {0.f, 0.f}, pl[2] = {0.f, 0.f};
+    float pc[8];
 #pragma unroll
     for (int i = 0; i < 16; ++i) aq[i] = ak[i] = av[i] = 0.f;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) pb[i] = pg[i] = pG[i] = pc[i] = 0.f;
-    int id;
-    mm<false, true>(K, K, t, [&](int r, int i, float x) { KK[sw(r, i)] = x; });
-    mm<false, true>(Q, K, t, [&](int r, int i, float x) { QK[sw(r, i)] = x; });
-    mm<false, false>(K, dSp, t, [&](int i, int m, float x) { X2[sw(i, m)] = x; });  // K dS'
+    for (int i = 0; i < 8; ++i) pc[i] = 0.f;
+    mm<false, true>(K, K, t, [&](int r, int i, float x, int) { KK[sw(r, i)] = x; });
+    mm<false, true>(Q, K, t, [&](int r, int i, float x, int) { QK[sw(r, i)] = x; });
+    mm<false, false>(K, dSp, t, [&](int i, int m, float x, int) { X2[sw(i, m)] = x; });  // K dS'
     __syncthreads();
-    // A (strictly lower) in dU for the solve; P in X1; d gam_C = <S, dS'>
+    // A (strictly lower) transposed in dU for the solve; P in X1; d gam_C = <S, dS'>
     {
         float part = 0.f;
         for (int idx = t; idx < N * N; idx += kThreads) {
             const int r = idx >> 6, i = idx & 63;
-            const float gm = decay(g, r, i);
-            dU[sw(r, i)] = i < r ? g.bet[r] * gm * KK[sw(r, i)] : 0.f;
-            X1[sw(r, i)] = gm * QK[sw(r, i)];
+            dU[sw(r, i)] = r < i ? g.bet[i] * decay(g, i, r) * KK[sw(r, i)] : 0.f;  // A(i, r), KK symmetric
+            X1[sw(r, i)] = decay(g, r, i) * QK[sw(r, i)];
             part = fmaf(S[sw(r, i)], dSp[sw(r, i)], part);
         }
 #pragma unroll
@@ -512,107 +585,87 @@ __global__ void __launch_bounds__(kThreads, 1)
     unit_lower_inverse(dU, Tm, t);
     __syncthreads();
     // U~ into U, W into dU (A is no longer needed)
-    mm<false, false>(Tm, V, t, [&](int r, int j, float x) { U[sw(r, j)] = x; }, g.bet);
-    mm<false, false>(Tm, K, t, [&](int r, int m, float x) { dU[sw(r, m)] = x; }, bg);
+    mm<false, false>(Tm, V, t, [&](int r, int j, float x, int) { U[sw(r, j)] = x; }, g.bet);
+    mm<false, false>(Tm, K, t, [&](int r, int m, float x, int) { dU[sw(r, m)] = x; }, bg);
     __syncthreads();
     // U = U~ - W S
-    mm<false, false>(dU, S, t, [&](int r, int j, float x) { U[sw(r, j)] -= x; });
+    mm<false, false>(dU, S, t, [&](int r, int j, float x, int) { U[sw(r, j)] -= x; });
     __syncthreads();
     // dU = P^T dO + diag(lam) K dS'; d lam_i = sum_j (K dS')_ij U_ij (the only term of d lam)
-    {
-        float pl[4] = {0.f, 0.f, 0.f, 0.f};
-        mm<true, false>(X1, dO, t, [&](int i, int j, float x) {
-            const float kd = X2[sw(i, j)];
-            dU[sw(i, j)] = x + g.lam[i] * kd;
-            pl[i - r0] = fmaf(kd, U[sw(i, j)], pl[i - r0]);
-        });
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const float sum = row_block_sum(pl[i]);
-            if ((t & 15) == 0) dlam[r0 + i] = sum;
-        }
-    }
+    mm<true, false>(X1, dO, t, [&](int i, int j, float x, int u) {
+        const float kd = X2[sw(i, j)];
+        dU[sw(i, j)] = x + g.lam[i] * kd;
+        pl[u_row(u)] = fmaf(kd, U[sw(i, j)], pl[u_row(u)]);
+    });
     __syncthreads();
     // dP = dO U^T (lower incl.), and at once D2 = dP o Gam into X1 (P is no longer needed) with the
     // dG terms of Gam (P); dK += diag(lam) U dS'^T; d gam (O1) and dQ += diag(gam) dO S^T
-    mm<false, true>(dO, U, t, [&](int r, int i, float x) {
+    mm<false, true>(dO, U, t, [&](int r, int i, float x, int u) {
         const float gm = decay(g, r, i), dp = i <= r ? x : 0.f;
         X1[sw(r, i)] = dp * gm;
         const float E = dp * QK[sw(r, i)] * gm;
-        pG[r - r0] += E;
-        pc[i - c0] -= E;
+        pG[u_row(u)] += E;
+        pc[u_col(u)] -= E;
     });
-    id = 0;
-    mm<false, true>(U, dSp, t, [&](int i, int m, float x) { ak[id++] += g.lam[i] * x; });
-    id = 0;
-    mm<false, true>(dO, S, t, [&](int r, int m, float x) { aq[id++] += g.gam[r] * x; });
-    mm<false, false>(Q, S, t, [&](int r, int j, float x) { pg[r - r0] = fmaf(dO[sw(r, j)], x, pg[r - r0]); });
+    mm<false, true>(U, dSp, t, [&](int i, int m, float x, int u) { ak[u] += g.lam[i] * x; });
+    mm<false, true>(dO, S, t, [&](int r, int m, float x, int u) { aq[u] += g.gam[r] * x; });
+    mm<false, false>(Q, S, t,
+                     [&](int r, int j, float x, int u) { pg[u_row(u)] = fmaf(dO[sw(r, j)], x, pg[u_row(u)]); });
     __syncthreads();
     // dW = -dU S^T into U (U is no longer needed)
-    mm<false, true>(dU, S, t, [&](int r, int m, float x) { U[sw(r, m)] = -x; });
+    mm<false, true>(dU, S, t, [&](int r, int m, float x, int) { U[sw(r, m)] = -x; });
     __syncthreads();
     // Y = T^T dU: dV, dbeta;  X = T^T dW: dK, dbeta, d gam
-    id = 0;
-    mm<true, false>(Tm, dU, t, [&](int i, int j, float x) {
-        av[id++] += g.bet[i] * x;
-        pb[i - r0] = fmaf(x, V[sw(i, j)], pb[i - r0]);
+    mm<true, false>(Tm, dU, t, [&](int i, int j, float x, int u) {
+        av[u] += g.bet[i] * x;
+        pb[u_row(u)] = fmaf(x, V[sw(i, j)], pb[u_row(u)]);
     });
-    id = 0;
-    mm<true, false>(Tm, U, t, [&](int i, int m, float x) {
-        ak[id++] += bg[i] * x;
+    mm<true, false>(Tm, U, t, [&](int i, int m, float x, int u) {
+        ak[u] += bg[i] * x;
         const float xk = x * K[sw(i, m)];
-        pb[i - r0] = fmaf(g.gam[i], xk, pb[i - r0]);
-        pg[i - r0] = fmaf(g.bet[i], xk, pg[i - r0]);
+        pb[u_row(u)] = fmaf(g.gam[i], xk, pb[u_row(u)]);
+        pg[u_row(u)] = fmaf(g.bet[i], xk, pg[u_row(u)]);
     });
     // dT = dU (diag(b) V)^T + dW (diag(b gam) K)^T into X2 (K dS' is no longer needed); the
     // diagonals scale the result's column index
-    mm<false, true>(dU, V, t, [&](int r, int i, float x) { X2[sw(r, i)] = g.bet[i] * x; });
-    mm<false, true>(U, K, t, [&](int r, int i, float x) { X2[sw(r, i)] += bg[i] * x; });
+    mm<false, true>(dU, V, t, [&](int r, int i, float x, int) { X2[sw(r, i)] = g.bet[i] * x; });
+    mm<false, true>(U, K, t, [&](int r, int i, float x, int) { X2[sw(r, i)] += bg[i] * x; });
     __syncthreads();
     // Z = dT T^T into dU
-    mm<false, true>(X2, Tm, t, [&](int r, int i, float x) { dU[sw(r, i)] = x; });
+    mm<false, true>(X2, Tm, t, [&](int r, int i, float x, int) { dU[sw(r, i)] = x; });
     __syncthreads();
     // dA = -T^T Z (strictly lower) -> D into U; dbeta (A); dG from Gam (A)
-    mm<true, false>(Tm, dU, t, [&](int r, int i, float x) {
+    mm<true, false>(Tm, dU, t, [&](int r, int i, float x, int u) {
         float d = 0.f;
         if (i < r) {
             const float gm = decay(g, r, i), kk = KK[sw(r, i)];
             const float dAg = -x * gm;  // dA o Gam
             d = g.bet[r] * dAg;
-            pb[r - r0] = fmaf(dAg, kk, pb[r - r0]);
+            pb[u_row(u)] = fmaf(dAg, kk, pb[u_row(u)]);
             const float E = d * kk;
-            pG[r - r0] += E;
-            pc[i - c0] -= E;
+            pG[u_row(u)] += E;
+            pc[u_col(u)] -= E;
         }
         U[sw(r, i)] = d;
     });
     __syncthreads();
     // dK += D K + D^T K + D2^T Q;  dQ += D2 K
-    id = 0;
-    mm<false, false>(U, K, t, [&](int r, int m, float x) { ak[id++] += x; });
-    id = 0;
-    mm<true, false>(U, K, t, [&](int i, int m, float x) { ak[id++] += x; });
-    id = 0;
-    mm<true, false>(X1, Q, t, [&](int i, int m, float x) { ak[id++] += x; });
-    id = 0;
-    mm<false, false>(X1, K, t, [&](int r, int m, float x) { aq[id++] += x; });
-    // the partial sums: rows over the 16 threads of a row block, columns over the 16 row blocks
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const float sb = row_block_sum(pb[i]), sg = row_block_sum(pg[i]), sG = row_block_sum(pG[i]);
-        if ((t & 15) == 0) {
-            dbet[r0 + i] = sb;
-            dgam[r0 + i] = sg;
-            dG[r0 + i] = sG;
-        }
-        colp[(t >> 4) * N + c0 + i] = pc[i];
-    }
+    mm<false, false>(U, K, t, [&](int, int, float x, int u) { ak[u] += x; });
+    mm<true, false>(U, K, t, [&](int, int, float x, int u) { ak[u] += x; });
+    mm<true, false>(X1, Q, t, [&](int, int, float x, int u) { ak[u] += x; });
+    mm<false, false>(X1, K, t, [&](int, int, float x, int u) { aq[u] += x; });
+    // the partial sums over the block (X2 is free scratch now: its last reader is two barriers back)
+    row_put(pb, X2, t);
+    row_put(pg, X2 + 2 * N, t);
+    row_put(pG, X2 + 4 * N, t);
+    row_put(pl, X2 + 6 * N, t);
+    col_put(pc, X2 + 8 * N, t);
     __syncthreads();
     if (t < N) {
-        float sum = 0.f;
-#pragma unroll
-        for (int b = 0; b < 16; ++b) sum += colp[b * N + t];
-        dG[t] += sum;
+        dbet[t] = row_get(X2, t);
+        dgam[t] = row_get(X2 + 2 * N, t);
+        dG[t] = row_get(X2 + 4 * N, t) + col_get(X2 + 8 * N, t);
+        dlam[t] = row_get(X2 + 6 * N, t);
     }
     __syncthreads();
     // gate gradients: gam_r = exp(G_r), lam_i = exp(G_63 - G_i), gam_C = gam_63; then dlog_alpha_j =
@@ -640,14 +693,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     }
     __syncthreads();
+    {
+        const int lane = t & 31, w = t >> 5, gq = lane >> 2, qq = lane & 3;
+        const int m0 = (w & 3) * 16, n0 = (w >> 2) * 32;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const int r = r0 + i;
-        if (r >= c.n) continue;
-        const size_t row = ((size_t)(c.tok + r) * H + h) * N + c0;
-        *reinterpret_cast<float4 *>(dq + row) = make_float4(aq[4 * i], aq[4 * i + 1], aq[4 * i + 2], aq[4 * i + 3]);
-        *reinterpret_cast<float4 *>(dk + row) = make_float4(ak[4 * i], ak[4 * i + 1], ak[4 * i + 2], ak[4 * i + 3]);
-        *reinterpret_cast<float4 *>(dv + row) = make_float4(av[4 * i], av[4 * i + 1], av[4 * i + 2], av[4 * i + 3]);
+        for (int hh = 0; hh < 2; ++hh) {
+            const int r = m0 + gq + 8 * hh;
+            if (r >= c.n) continue;
+            const size_t row = ((size_t)(c.tok + r) * H + h) * N + n0 + 2 * qq;
+#pragma unroll
+            for (int n = 0; n < 4; ++n) {
+                const int u = 4 * n + 2 * hh;
+                *reinterpret_cast<float2 *>(dq + row + 8 * n) = make_float2(aq[u], aq[u + 1]);
+                *reinterpret_cast<float2 *>(dk + row + 8 * n) = make_float2(ak[u], ak[u + 1]);
+                *reinterpret_cast<float2 *>(dv + row + 8 * n) = make_float2(av[u], av[u + 1]);
+            }
+        }
     }
     if (t < c.n) {
         const size_t o = (size_t)(c.tok + t) * H + h;
@@ -706,7 +767,7 @@ cudaError_t run_bwd(const BwdArgs &a, cudaStream_t st)
     const TIn *q = static_cast<const TIn *>(a.q), *k = static_cast<const TIn *>(a.k),
               *v = static_cast<const TIn *>(a.v), *dout = static_cast<const TIn *>(a.dout);
     const int smem_prep = (9 * MAT) * (int)sizeof(float) + (int)sizeof(Gates) + N * (int)sizeof(float);
-    const int smem_grads = (13 * MAT) * (int)sizeof(float) + (int)sizeof(Gates) + (6 + 16) * N * (int)sizeof(float);
+    const int smem_grads = (13 * MAT) * (int)sizeof(float) + (int)sizeof(Gates) + 6 * N * (int)sizeof(float);
     const int smem_scan = 4 * MAT * (int)sizeof(float);
     cudaError_t e = cudaFuncSetAttribute(bwd_prep<TIn>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_prep);
     if (e != cudaSuccess) return e;
