@@ -56,6 +56,11 @@ def algo_flops(token_heads, dk, dv, C=64):
 DECODE_BYTES_PER_STATE = lambda dk, dv, e: 8 * dk * dv + e * (2 * dk + 2 * dv) + 8
 
 
+# dense tf32 : bf16 tensor throughput, nominal (1.1 and 2.25 PFLOP/s per GPU): the tf32 peak is the
+# measured bf16 peak scaled by it
+TF32_PER_BF16 = 1.1 / 2.25
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -455,7 +460,8 @@ def run_ours(args, world, rank, local):
                                   "ms": round(ms_g, 6), "tokens_per_s": round(8 * 4096 / (ms_g * 1e-3), 1),
                                   "launches_per_call": 1}
         del dg, outg, Sg
-        # backward of the hybrid-LM step (dq, dk, dv, gate and state gradients; fp32 CUDA cores)
+        # backward of the hybrid-LM step (dq, dk, dv, gate and state gradients; fp32-accurate products
+        # on the tensor cores as three tf32 terms)
         dout = torch.randn(d["v"].shape, device="cuda").to(d["v"].dtype)
         wsb = torch.empty(gdn.gdn_chunk_bwd_workspace_bytes(8, 4096, 12, 64, 64, 64, 0), dtype=torch.uint8,
                           device="cuda")
@@ -477,11 +483,20 @@ def run_ours(args, world, rank, local):
         ms_b = statistics.mean(a0.elapsed_time(b0) for a0, b0 in evb)
         # bytes per token-head: q, k, v, dout (bf16) and gates in; dq, dk, dv (fp32) and two gate grads out
         by_b = 393216 * (4 * 64 * 2 + 8 + 3 * 64 * 4 + 8)
+        # products per (chunk, head): 9 (prep) + 22 (grads) + 1 in each scan, each 2 * 64^3 flops in
+        # fp32; the tensor cores execute three tf32 products for each
+        fl_b = 6144 * 33 * 2 * 64 ** 3
+        tf32_peak = peaks["bf16_tflops"] * TF32_PER_BF16
         extra["hybrid_lm_backward"] = {"workload": "hybrid_lm backward: dq, dk, dv, dlog_alpha, dbeta (fp32) from dout",
                                        "ms": round(ms_b, 6), "tokens_per_s": round(32768 / (ms_b * 1e-3), 1),
                                        "launches_per_call": 4, "algo_bytes": by_b,
                                        "gbs": round(by_b / (ms_b * 1e-3) / 1e9, 3),
-                                       "hbm_frac": round(by_b / (ms_b * 1e-3) / 1e9 / peaks["hbm_gbs"], 5)}
+                                       "hbm_frac": round(by_b / (ms_b * 1e-3) / 1e9 / peaks["hbm_gbs"], 5),
+                                       "algo_flops_fp32": fl_b,
+                                       "fp32_tflops": round(fl_b / (ms_b * 1e-3) / 1e12, 3),
+                                       "tf32_mma_tflops": round(3 * fl_b / (ms_b * 1e-3) / 1e12, 3),
+                                       "tf32_peak_tflops": round(tf32_peak, 1),
+                                       "tensor_frac": round(3 * fl_b / (ms_b * 1e-3) / 1e12 / tf32_peak, 5)}
         del dout, wsb
     cpu = None
     if rank == 0 and world == 1:

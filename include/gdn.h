@@ -174,7 +174,9 @@ GDN_API int gdn_chunk_fwd_noalloc(const void *q, const void *k, const void *v, c
  * dout) and dout = dL/dout, dS_final = dL/dS_final (NULL: zero), it writes
  *     dq, dk [.., H, 64], dv [.., H, 64], dlog_alpha, dbeta [.., H]   (fp32, always)
  *     dS0 [B, H, 64, 64] fp32 (NULL: not written)
- * Computed in fp32 on the CUDA cores from the chunk form: every chunk's state map
+ * Computed from the chunk form with fp32-level accuracy: the 64 x 64 products run on the tensor
+ * cores as three tf32 products (x = hi + lo; a b ~ hi hi + hi lo + lo hi), everything else in
+ * fp32.  Every chunk's state map
  * S' = M S + Bm and gradient map dS = M^T dS' + (Q^T diag(gam) - W^T P^T) dO are formed in
  * parallel, two scans over each sequence's chunks give the entry states and exit gradients, and
  * every chunk's input gradients are then formed in parallel.  log_alpha = -inf (an exact reset)

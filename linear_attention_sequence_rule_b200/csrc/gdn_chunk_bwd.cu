@@ -1,6 +1,7 @@
-// gdn_chunk_bwd.cu -- gradients of the chunk forward (dq, dk, dv, dlog_alpha, dbeta, dS0) on the
-// CUDA cores in fp32, for dk = dv = 64 (the training path; Sykra README, "Architectural
-// Highlights": chunk-parallel training through the WY / UT transform).
+// gdn_chunk_bwd.cu -- gradients of the chunk forward (dq, dk, dv, dlog_alpha, dbeta, dS0) with
+// fp32-level accuracy, for dk = dv = 64 (the training path; Sykra README, "Architectural
+// Highlights": chunk-parallel training through the WY / UT transform).  The 64 x 64 products run
+// on the tensor cores as three tf32 products each; the rest is fp32 on the CUDA cores.
 //
 // Per chunk of C = 64 tokens with entry state S (the forward's chunk form):
 //   A = strictly_lower(diag(b) (Gam o K K^T)),  T = (I + A)^{-1}
@@ -14,8 +15,8 @@
 //   bwd_scan<false> (sequence x head)    : S_c for every chunk, from S0
 //   bwd_scan<true>  (sequence x head, reverse): dS at every chunk's end, from dS_final; dS0
 //   bwd_grads  (chunk x head, parallel)  : with S_c and dS_{c+1}, every input gradient of the chunk
-// All matrices are 64 x 64 fp32 in shared memory (swizzled 16-byte groups); 256 threads; a matrix
-// product gives each thread a 4 x 4 block of the result.
+// All matrices are 64 x 64 fp32 in shared memory (XOR-swizzled rows); 256 threads; a product
+// leaves each thread 16 results in the tensor cores' fragment layout (see mm_core).
 #include <cuda_bf16.h>
 #include <math.h>
 

@@ -2,9 +2,10 @@
 finite differences) on the same inputs: dense and varlen (ragged, empty and one-token sequences),
 exact resets, beta in (0, 2], with and without S0 and dS_final, bf16 and fp32 inputs.
 
-The kernels compute in fp32 from the stored input values (the oracle reads the same values in
-fp64), so the bound is relative to each gradient's scale: max |g - g_ref| <= 1e-5 *
-(1 + max |g_ref|) per tensor (a few 1e-7 is what fp32 gives on these sizes)."""
+The kernels compute with fp32-level accuracy from the stored input values (fp32 on the CUDA
+cores, products as three tf32 tensor-core terms with a relative error below 2^-21; the oracle
+reads the same values in fp64), so the bound is relative to each gradient's scale:
+max |g - g_ref| <= 1e-5 * (1 + max |g_ref|) per tensor (a few 1e-7 is what these sizes give)."""
 import numpy as np
 import pytest
 import torch
