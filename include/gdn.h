@@ -20,9 +20,11 @@
  * normalise q or k.
  *
  * Conventions shared by every entry point
- *   - Every tensor pointer is a DEVICE pointer owned by the caller.  The library allocates no
- *     memory, keeps no state between calls and may be called from several host threads (the
- *     one exception, gdn_chunk_fwd_noalloc, owns a fixed scratch array per device).
+ *   - Every tensor pointer is a DEVICE pointer owned by the caller (the exception:
+ *     gdn_chunk_fwd_host, which takes host buffers).  The library allocates no memory, keeps no
+ *     state between calls and may be called from several host threads (the exceptions:
+ *     gdn_chunk_fwd_noalloc owns a fixed scratch array per device; gdn_chunk_fwd_host keeps two
+ *     copy streams and a few events per device, made on its first call).
  *   - Calls are asynchronous: they validate on the host, enqueue kernels on `stream` (a
  *     cudaStream_t; NULL = the legacy default stream) and return.  Errors found on the host are
  *     returned before anything is enqueued, so a failed call writes nothing.
@@ -166,6 +168,33 @@ GDN_API int gdn_chunk_fwd_noalloc(const void *q, const void *k, const void *v, c
                                   const float *beta, const float *S0, void *out, float *S_final, int B,
                                   int T, int H, int dk, int dv, int chunk, const int32_t *cu_seqlens,
                                   int dtype, void *stream);
+
+/*
+ * gdn_chunk_fwd_host -- gdn_chunk_fwd from and to HOST buffers: q, k, v, log_alpha, beta, S0 (may
+ * be NULL), cu_seqlens (may be NULL) are read from host memory and out, S_final (may be NULL) are
+ * written to host memory, in gdn_chunk_fwd's layouts; the arithmetic is gdn_chunk_fwd's.  The
+ * batch is cut into at most 4 parts of whole sequences (varlen: about equal token counts); each
+ * part's inputs are copied up on a side stream, the part runs on `stream` once they have arrived,
+ * and its outputs are copied down on a second side stream, so copies in both directions overlap
+ * each other and the compute.  Host buffers in page-locked memory (cudaHostAlloc, or a pinned
+ * torch tensor) make the copies asynchronous; pageable buffers work, with the copies serialised.
+ * `workspace`: DEVICE memory of gdn_chunk_fwd_host_workspace_bytes(...) bytes, 256-byte
+ * aligned, holding device copies of every input and output and the device entry's own scratch.
+ * Asynchronous like every entry: the outputs are in host memory once `stream` has completed (the
+ * side streams are joined back into it), and the host input buffers must stay unchanged until
+ * then.  cu_seqlens is read on the host during the call (it decides the parts) and must run from
+ * 0 to T without decreasing.  Errors as gdn_chunk_fwd; GDN_ERR_CUDA if the copy streams cannot be
+ * made.  Nothing in the pages corresponds to this entry: it is the host-memory interface a
+ * serving process without device tensors of its own would call.
+ */
+GDN_API int gdn_chunk_fwd_host(const void *q, const void *k, const void *v, const float *log_alpha,
+                               const float *beta, const float *S0, void *out, float *S_final, int B, int T,
+                               int H, int dk, int dv, int chunk, const int32_t *cu_seqlens, int dtype,
+                               void *workspace, size_t workspace_bytes, void *stream);
+
+/* Device workspace gdn_chunk_fwd_host needs for these sizes; (size_t)-1 for sizes it rejects. */
+GDN_API size_t gdn_chunk_fwd_host_workspace_bytes(int B, int T, int H, int dk, int dv, int chunk, int varlen,
+                                                  int dtype);
 
 /*
  * gdn_chunk_bwd -- gradients of gdn_chunk_fwd (the training path; Sykra README, "Architectural

@@ -3,11 +3,12 @@
 Argument marshalling only: every step of the computation runs in the library's CUDA kernels.
 PyTorch provides device memory and streams.  The binding has two layers:
 
-* ``gdn_chunk_fwd``, ``gdn_chunk_fwd_noalloc``, ``gdn_decode_step``, ``gdn_chunk_fwd_workspace_bytes``,
+* ``gdn_chunk_fwd``, ``gdn_chunk_fwd_noalloc``, ``gdn_chunk_fwd_host``, ``gdn_decode_step``,
+  ``gdn_chunk_fwd_workspace_bytes``, ``gdn_chunk_fwd_host_workspace_bytes``,
   ``gdn_status_string``, ``gdn_last_error``, ``gdn_version`` -- the C-ABI entry points of
   ``include/gdn.h`` with the same names and arguments (pointers as Python ints);
-* ``chunk_fwd``, ``chunk_fwd_fused``, ``chunk_fwd_gva``, ``chunk_bwd``, ``decode_step`` and
-  ``decode_step_gva`` --
+* ``chunk_fwd``, ``chunk_fwd_host``, ``chunk_fwd_fused``, ``chunk_fwd_gva``, ``chunk_bwd``,
+  ``decode_step`` and ``decode_step_gva`` --
   the same calls taking torch tensors; they check shapes,
   devices and dtypes, allocate outputs with torch when none are given, and raise ``GdnError``
   on a non-zero status.
@@ -25,6 +26,7 @@ __all__ = [
     "GdnError", "GDN_OK", "GDN_ERR_INVALID_ARGUMENT", "GDN_ERR_UNSUPPORTED", "GDN_ERR_WORKSPACE",
     "GDN_ERR_CUDA", "GDN_ERR_TIMEOUT", "GDN_DTYPE_F32", "GDN_DTYPE_BF16", "LIB_PATH",
     "gdn_chunk_fwd", "gdn_chunk_fwd_noalloc", "gdn_chunk_fwd_fused", "gdn_chunk_fwd_gva",
+    "gdn_chunk_fwd_host", "gdn_chunk_fwd_host_workspace_bytes", "chunk_fwd_host",
     "gdn_decode_step", "gdn_decode_step_gva", "gdn_chunk_bwd", "gdn_chunk_bwd_workspace_bytes", "gdn_chunk_fwd_workspace_bytes", "gdn_status_string",
     "gdn_last_error", "gdn_version", "gdn_device_status", "device_status", "chunk_fwd", "chunk_fwd_fused",
     "chunk_fwd_gva", "chunk_bwd", "decode_step", "decode_step_gva", "workspace_bytes",
@@ -67,6 +69,10 @@ _lib.gdn_chunk_bwd_workspace_bytes.restype = _sz
 _lib.gdn_chunk_fwd_noalloc.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i,
                                        _i, _vp, _i, _vp]
 _lib.gdn_chunk_fwd_noalloc.restype = _i
+_lib.gdn_chunk_fwd_host.argtypes = list(_lib.gdn_chunk_fwd.argtypes)
+_lib.gdn_chunk_fwd_host.restype = _i
+_lib.gdn_chunk_fwd_host_workspace_bytes.argtypes = [_i, _i, _i, _i, _i, _i, _i, _i]
+_lib.gdn_chunk_fwd_host_workspace_bytes.restype = _sz
 _lib.gdn_chunk_fwd_workspace_bytes.argtypes = [_i, _i, _i, _i, _i, _i, _i, _i]
 _lib.gdn_chunk_fwd_workspace_bytes.restype = _sz
 _lib.gdn_decode_step.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp]
@@ -129,6 +135,16 @@ def gdn_chunk_fwd_noalloc(q, k, v, log_alpha, beta, S0, out, S_final, B, T, H, d
                           cu_seqlens, dtype, stream) -> int:
     return _lib.gdn_chunk_fwd_noalloc(q, k, v, log_alpha, beta, S0, out, S_final, B, T, H, dk, dv,
                                       chunk, cu_seqlens, dtype, stream)
+
+
+def gdn_chunk_fwd_host(q, k, v, log_alpha, beta, S0, out, S_final, B, T, H, dk, dv, chunk, cu_seqlens,
+                       dtype, workspace, workspace_bytes, stream) -> int:
+    return _lib.gdn_chunk_fwd_host(q, k, v, log_alpha, beta, S0, out, S_final, B, T, H, dk, dv, chunk,
+                                   cu_seqlens, dtype, workspace, workspace_bytes, stream)
+
+
+def gdn_chunk_fwd_host_workspace_bytes(B, T, H, dk, dv, chunk, varlen, dtype) -> int:
+    return _lib.gdn_chunk_fwd_host_workspace_bytes(B, T, H, dk, dv, chunk, varlen, dtype)
 
 
 def gdn_chunk_fwd_workspace_bytes(B, T, H, dk, dv, chunk, varlen, dtype) -> int:
@@ -249,6 +265,55 @@ def chunk_fwd(q, k, v, log_alpha, beta, S0=None, cu_seqlens=None, out=None, S_fi
     if rc != GDN_OK:
         raise GdnError(rc, gdn_last_error())
     return p["out"], p["S_final"]
+
+
+def chunk_fwd_host(q, k, v, log_alpha, beta, S0=None, cu_seqlens=None, out=None, S_final=None,
+                   output_final_state=True, workspace=None, chunk=64, stream=None):
+    """``chunk_fwd`` from and to host memory (``gdn_chunk_fwd_host``): q, k, v, gates, S0 and
+    cu_seqlens are CPU tensors (page-locked ones let the copies overlap), out and S_final are
+    written to CPU tensors (allocated page-locked when not given), workspace is a CUDA uint8
+    tensor of ``gdn_chunk_fwd_host_workspace_bytes`` bytes (allocated on the current device when
+    not given).  Asynchronous: the outputs are complete once ``stream`` has completed."""
+    dt = q.dtype
+    if dt not in _DT:
+        raise ValueError(f"unsupported dtype {dt}")
+    cpu = torch.device("cpu")
+    if cu_seqlens is not None:
+        T, H, dk = q.shape
+        B = cu_seqlens.shape[0] - 1
+        lead = (T,)
+        _need(cu_seqlens, "cu_seqlens", torch.int32, (B + 1,), cpu)
+    else:
+        B, T, H, dk = q.shape
+        lead = (B, T)
+    dv = v.shape[-1]
+    _need(q, "q", dt, (*lead, H, dk), cpu)
+    _need(k, "k", dt, (*lead, H, dk), cpu)
+    _need(v, "v", dt, (*lead, H, dv), cpu)
+    _need(log_alpha, "log_alpha", torch.float32, (*lead, H), cpu)
+    _need(beta, "beta", torch.float32, (*lead, H), cpu)
+    if S0 is not None:
+        _need(S0, "S0", torch.float32, (B, H, dk, dv), cpu)
+    if out is None:
+        out = torch.empty((*lead, H, dv), dtype=dt).pin_memory()
+    _need(out, "out", dt, (*lead, H, dv), cpu)
+    if S_final is None and output_final_state:
+        S_final = torch.empty((B, H, dk, dv), dtype=torch.float32).pin_memory()
+    if S_final is not None:
+        _need(S_final, "S_final", torch.float32, (B, H, dk, dv), cpu)
+    need = gdn_chunk_fwd_host_workspace_bytes(B, T, H, dk, dv, chunk, int(cu_seqlens is not None), _DT[dt])
+    if need == ctypes.c_size_t(-1).value:
+        raise GdnError(GDN_ERR_INVALID_ARGUMENT, gdn_last_error())
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device="cuda")
+    if not workspace.is_cuda:
+        raise ValueError("workspace must be a CUDA tensor")
+    rc = gdn_chunk_fwd_host(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(S0), _ptr(out),
+                            _ptr(S_final), B, T, H, dk, dv, chunk, _ptr(cu_seqlens), _DT[dt], _ptr(workspace),
+                            workspace.numel(), _stream_ptr(stream))
+    if rc != GDN_OK:
+        raise GdnError(rc, gdn_last_error())
+    return out, S_final
 
 
 def chunk_fwd_fused(q_raw, k_raw, v, a_raw, b_raw, a_scale, b_scale, S0=None, cu_seqlens=None,

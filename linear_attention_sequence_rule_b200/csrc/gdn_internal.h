@@ -46,7 +46,7 @@ size_t chunk_tc_workspace_bytes(int B, int T, int H, int dk, int dv, int varlen,
 // after synchronising the device.  Returns -1 when the read itself failed.
 int read_and_clear_tc_error();
 
-// Gradients of the chunk forward (fp32 CUDA-core kernels, dk = dv = 64); see gdn_chunk_bwd.cu.
+// Gradients of the chunk forward (fp32-level accuracy, dk = dv = 64); see gdn_chunk_bwd.cu.
 struct BwdArgs {
     const void *q, *k, *v;
     const float *log_alpha, *beta, *S0;

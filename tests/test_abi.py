@@ -151,3 +151,42 @@ def test_backward_entry_validation():
     assert "gdn_chunk_bwd" in gdn.gdn_last_error()
     assert gdn.gdn_chunk_bwd_workspace_bytes(1, 64, 1, 128, 128, 64, 0) == (1 << 64) - 1
     assert gdn.gdn_chunk_bwd_workspace_bytes(2, 128, 3, 64, 64, 64, 0) > 5 * 2 * 2 * 3 * 64 * 64 * 4 - 1
+
+
+def host_chunk(**kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, log_alpha=FAKE, beta=FAKE, S0=None, out=FAKE, S_final=None,
+             B=2, T=64, H=1, dk=64, dv=64, chunk=64, cu_seqlens=None, dtype=gdn.GDN_DTYPE_BF16,
+             workspace=FAKE * 256, workspace_bytes=1 << 40, stream=None)
+    a.update(kw)
+    return gdn.gdn_chunk_fwd_host(**a)
+
+
+def _cu(*vals):
+    arr = (ctypes.c_int32 * len(vals))(*vals)
+    return ctypes.cast(arr, ctypes.c_void_p).value, arr
+
+
+def test_host_entry_workspace_covers_every_input_and_output():
+    # bf16 dense, no segment scan needed for one-sequence parts this short
+    n = gdn.gdn_chunk_fwd_host_workspace_bytes(2, 64, 1, 64, 64, 64, 0, gdn.GDN_DTYPE_BF16)
+    tokens = 2 * 64
+    assert n >= 3 * tokens * 64 * 2 + 2 * tokens * 4 + 2 * 2 * 64 * 64 * 4 + tokens * 64 * 2
+    assert gdn.gdn_chunk_fwd_host_workspace_bytes(2, 64, 1, 96, 64, 64, 0, gdn.GDN_DTYPE_BF16) == \
+        ctypes.c_size_t(-1).value
+
+
+def test_host_entry_rejects_before_any_copy():
+    assert host_chunk(dk=96) == gdn.GDN_ERR_UNSUPPORTED
+    assert host_chunk(B=0) == gdn.GDN_ERR_INVALID_ARGUMENT
+    assert host_chunk(out=None) == gdn.GDN_ERR_INVALID_ARGUMENT
+    assert host_chunk(q=None) == gdn.GDN_ERR_INVALID_ARGUMENT
+    assert host_chunk(workspace=None) == gdn.GDN_ERR_WORKSPACE
+    assert host_chunk(workspace_bytes=16) == gdn.GDN_ERR_WORKSPACE
+    assert host_chunk(workspace=FAKE * 256 + 16) == gdn.GDN_ERR_INVALID_ARGUMENT
+    p, keep = _cu(0, 10, 5)  # decreasing
+    assert host_chunk(T=5, cu_seqlens=p) == gdn.GDN_ERR_INVALID_ARGUMENT
+    assert "decreases" in gdn.gdn_last_error()
+    p, keep = _cu(1, 3, 5)  # does not start at 0
+    assert host_chunk(T=5, cu_seqlens=p) == gdn.GDN_ERR_INVALID_ARGUMENT
+    p, keep = _cu(0, 3, 5)  # does not end at T
+    assert host_chunk(T=6, cu_seqlens=p) == gdn.GDN_ERR_INVALID_ARGUMENT
