@@ -28,7 +28,14 @@ namespace {
 
 constexpr int N = 64;          // chunk length = dk = dv
 constexpr int MAT = N * N;     // floats per matrix
-constexpr int kThreads = 256;
+constexpr int kThreads = 256;               // 8 warps (16 measured slower: 4.5 against 4.1 ms)
+constexpr int kColBlocks = kThreads / 128;  // a product's warps: 4 row blocks of 16 x this many column blocks
+constexpr int kNT = N / (8 * kColBlocks);   // 8-column MMA tiles per warp
+constexpr int kFrag = 4 * kNT;              // results per thread of a product
+constexpr int kColSlots = 2 * kNT;          // distinct columns among them
+constexpr int kSolveLanes = kThreads / N;   // threads per column in the triangular solve
+constexpr int kSolveRows = N / kSolveLanes; // rows per thread there
+static_assert(kNT >= 1 && 8 * kNT * kColBlocks == N && kSolveLanes * N == kThreads, "thread layout");
 
 // Shared matrices are 64 x 64 fp32 with 64-float rows; column c of row r is stored at position
 // c ^ 4 sigma(r mod 8), sigma = (0 2 4 6 1 3 5 7), which moves whole 16-byte groups.  Both access
@@ -95,15 +102,15 @@ extern __shared__ __align__(16) float smf[];
 
 // One thread's 16 results of a product, index u (see mm).
 struct Frag {
-    float v[16];
+    float v[kFrag];
 };
 
 // C(r, c) = sum_k opA(r, k) ks[k] opB(k, c) for 64 x 64 operands (opA = A or A^T, opB = B or B^T;
 // ks: optional diagonal), on the tensor cores with the three-term tf32 split.  Warp w computes
-// rows 16 (w mod 4) .. +15 and columns 32 (w / 4) .. +31; lane l holds rows 16 (w mod 4) + l / 4 +
-// {0, 8} and columns 32 (w / 4) + 8 n + 2 (l mod 4) + {0, 1}, n = 0..3, as element
-// u = 4 n + 2 (row half) + (column parity) of its Frag -- the same u for the same (r, c) in every
-// product, so per-thread accumulators can be indexed by it.  The operands are given as offsets
+// rows 16 (w mod 4) .. +15 and the W = 8 kNT columns from W (w / 4); lane l holds rows
+// 16 (w mod 4) + l / 4 + {0, 8} and columns W (w / 4) + 8 n + 2 (l mod 4) + {0, 1}, n < kNT, as
+// element u = 4 n + 2 (row half) + (column parity) of its Frag -- the same u for the same (r, c)
+// in every product, so per-thread accumulators can be indexed by it.  The operands are given as offsets
 // into the shared memory.  Kept out of line: a kernel runs this loop some twenty times, and one
 // shared copy of it stays in the instruction cache.
 template <bool TA, bool TB, bool KS>
@@ -111,13 +118,13 @@ __device__ __noinline__ Frag mm_core(int a_off, int b_off, int ks_off)
 {
     const float *A = smf + a_off, *B = smf + b_off, *ks = smf + ks_off;
     const int t = threadIdx.x, lane = t & 31, w = t >> 5, g = lane >> 2, q = lane & 3;
-    const int m0 = (w & 3) * 16, n0 = (w >> 2) * 32;
-    float acc[4][4], cor[4][4];  // hi x hi, and the two cross terms (independent chains)
+    const int m0 = (w & 3) * 16, n0 = (w >> 2) * 8 * kNT;
+    float acc[kNT][4], cor[kNT][4];  // hi x hi, and the two cross terms (independent chains)
 #pragma unroll
-    for (int n = 0; n < 4; ++n)
+    for (int n = 0; n < kNT; ++n)
 #pragma unroll
         for (int j = 0; j < 4; ++j) acc[n][j] = cor[n][j] = 0.f;
-#pragma unroll 1
+#pragma unroll 2
     for (int k0 = 0; k0 < N; k0 += 8) {
         float a[4];  // opA at (m0 + g, k0 + q), (m0 + g + 8, k0 + q), (m0 + g, k0 + q + 4), (m0 + g + 8, k0 + q + 4)
         a[0] = TA ? A[sw(k0 + q, m0 + g)] : A[sw(m0 + g, k0 + q)];
@@ -135,7 +142,7 @@ __device__ __noinline__ Frag mm_core(int a_off, int b_off, int ks_off)
 #pragma unroll
         for (int j = 0; j < 4; ++j) split_tf32(a[j], ah[j], al[j]);
 #pragma unroll
-        for (int n = 0; n < 4; ++n) {
+        for (int n = 0; n < kNT; ++n) {
             const int col = n0 + 8 * n + g;  // opB at (k0 + q, col), (k0 + q + 4, col)
             const float b0 = TB ? B[sw(col, k0 + q)] : B[sw(k0 + q, col)];
             const float b1 = TB ? B[sw(col, k0 + q + 4)] : B[sw(k0 + q + 4, col)];
@@ -149,7 +156,7 @@ __device__ __noinline__ Frag mm_core(int a_off, int b_off, int ks_off)
     }
     Frag f;
 #pragma unroll
-    for (int n = 0; n < 4; ++n)
+    for (int n = 0; n < kNT; ++n)
 #pragma unroll
         for (int j = 0; j < 4; ++j) f.v[4 * n + j] = acc[n][j] + cor[n][j];
     return f;
@@ -161,11 +168,11 @@ template <bool TA, bool TB, typename F>
 __device__ __forceinline__ void mm(const float *A, const float *B, int t, F &&emit, const float *ks = nullptr)
 {
     const int lane = t & 31, w = t >> 5, g = lane >> 2, q = lane & 3;
-    const int m0 = (w & 3) * 16, n0 = (w >> 2) * 32;
+    const int m0 = (w & 3) * 16, n0 = (w >> 2) * 8 * kNT;
     const Frag f = ks ? mm_core<TA, TB, true>((int)(A - smf), (int)(B - smf), (int)(ks - smf))
                       : mm_core<TA, TB, false>((int)(A - smf), (int)(B - smf), 0);
 #pragma unroll
-    for (int n = 0; n < 4; ++n)
+    for (int n = 0; n < kNT; ++n)
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh)
 #pragma unroll
@@ -175,9 +182,9 @@ __device__ __forceinline__ void mm(const float *A, const float *B, int t, F &&em
 
 // Per-thread partial sums over the rows and columns a thread holds in mm's layout, completed over
 // the block in two steps: *_put writes a thread's share to scratch shared memory (rows: two per
-// thread, u bit 1, summed over the 4 lanes of a row, 2 x 64 floats of scratch; columns: eight per
-// thread, u / 4 and u bit 0, summed over the 8 row groups of a warp, 4 x 64 floats), and after a
-// barrier *_get(j) returns the total of row or column j.
+// thread, u bit 1, summed over the 4 lanes of a row, kColBlocks x 64 floats of scratch; columns:
+// kColSlots per thread, u / 4 and u bit 0, summed over the 8 row groups of a warp, 4 x 64 floats),
+// and after a barrier *_get(j) returns the total of row or column j.
 __device__ __forceinline__ void row_put(const float (&p)[2], float *buf, int t)
 {
     const int lane = t & 31, w = t >> 5, r = (w & 3) * 16 + (lane >> 2);
@@ -190,18 +197,24 @@ __device__ __forceinline__ void row_put(const float (&p)[2], float *buf, int t)
     }
 }
 
-__device__ __forceinline__ float row_get(const float *buf, int j) { return buf[j] + buf[N + j]; }
+__device__ __forceinline__ float row_get(const float *buf, int j)
+{
+    float x = 0.f;
+#pragma unroll
+    for (int b = 0; b < kColBlocks; ++b) x += buf[b * N + j];
+    return x;
+}
 
-__device__ __forceinline__ void col_put(const float (&p)[8], float *buf, int t)
+__device__ __forceinline__ void col_put(const float (&p)[kColSlots], float *buf, int t)
 {
     const int lane = t & 31, w = t >> 5;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
+    for (int j = 0; j < kColSlots; ++j) {
         float x = p[j];
         x += __shfl_xor_sync(0xffffffffu, x, 4);
         x += __shfl_xor_sync(0xffffffffu, x, 8);
         x += __shfl_xor_sync(0xffffffffu, x, 16);
-        if (lane < 4) buf[(w & 3) * N + (w >> 2) * 32 + 8 * (j >> 1) + 2 * lane + (j & 1)] = x;
+        if (lane < 4) buf[(w & 3) * N + (w >> 2) * 8 * kNT + 8 * (j >> 1) + 2 * lane + (j & 1)] = x;
     }
 }
 
@@ -330,11 +343,12 @@ struct RowTile {
 // A dense 64 x 64 fp32 matrix from global memory (row-major) into a shared matrix, and back.
 __device__ __forceinline__ void mat_to_shared(float *M, const float *src, int t)
 {
-    float4 b[4];
+    constexpr int PER = MAT / 4 / kThreads;  // float4 pieces per thread
+    float4 b[PER];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) b[u] = __ldg(reinterpret_cast<const float4 *>(src) + t + u * kThreads);
+    for (int u = 0; u < PER; ++u) b[u] = __ldg(reinterpret_cast<const float4 *>(src) + t + u * kThreads);
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
+    for (int u = 0; u < PER; ++u) {
         const int e = (t + u * kThreads) * 4;
         *reinterpret_cast<float4 *>(&M[sw(e >> 6, e & 63)]) = b[u];
     }
@@ -343,34 +357,35 @@ __device__ __forceinline__ void mat_to_shared(float *M, const float *src, int t)
 __device__ __forceinline__ void mat_from_shared(float *dst, const float *M, int t)
 {
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
+    for (int u = 0; u < MAT / 4 / kThreads; ++u) {
         const int e = (t + u * kThreads) * 4;
         reinterpret_cast<float4 *>(dst)[t + u * kThreads] = *reinterpret_cast<const float4 *>(&M[sw(e >> 6, e & 63)]);
     }
 }
 
 // T = (I + A)^{-1} for strictly lower A, given transposed (At(i, r) = A(r, i); only i < r is read).
-// Column c of T is found by forward substitution on threads 4c .. 4c + 3, thread 4c + q holding
-// rows q, q + 4, ..., q + 60: once row j is final it is passed among the four and subtracted from
-// every later row, so one multiply-add lies between row j and row j + 1.  A warp holds columns
-// 8w .. 8w + 7, whose rows above 8w are zero, and skips those steps.  Every entry of T is written.
+// Column c of T is found by forward substitution on the kSolveLanes = L threads Lc .. Lc + L - 1,
+// thread Lc + q holding rows q, q + L, q + 2L, ...: once row j is final it is passed among the L
+// and subtracted from every later row, so one multiply-add lies between row j and row j + 1.  Every warp runs all 64
+// steps (a column's rows above its diagonal stay zero; skipping them per warp would put a branch
+// between the steps and keep the next step's loads from being issued early).  Every entry of T is
+// written.
 __device__ void unit_lower_inverse(const float *At, float *Tm, int t)
 {
-    const int c = t >> 2, q = t & 3, w8 = (t >> 5) * 8;
-    float s[16];
+    constexpr int L = kSolveLanes;
+    const int c = t / L, q = t % L;
+    float s[kSolveRows];
 #pragma unroll
-    for (int m = 0; m < 16; ++m) s[m] = (4 * m + q == c) ? 1.f : 0.f;
+    for (int m = 0; m < kSolveRows; ++m) s[m] = (L * m + q == c) ? 1.f : 0.f;
 #pragma unroll
     for (int j = 0; j < N; ++j) {
-        if (j >= w8) {
-            const float xj = __shfl_sync(0xffffffffu, s[j >> 2], j & 3, 4);
+        const float xj = __shfl_sync(0xffffffffu, s[j / L], j % L, L);
 #pragma unroll
-            for (int m = j >> 2; m < 16; ++m)
-                if (4 * m + q > j) s[m] = fmaf(-At[sw(j, 4 * m + q)], xj, s[m]);
-        }
+        for (int m = j / L; m < kSolveRows; ++m)
+            if (L * m + q > j) s[m] = fmaf(-At[sw(j, L * m + q)], xj, s[m]);
     }
 #pragma unroll
-    for (int m = 0; m < 16; ++m) Tm[sw(4 * m + q, c)] = s[m];
+    for (int m = 0; m < kSolveRows; ++m) Tm[sw(L * m + q, c)] = s[m];
 }
 
 // ---- bwd_prep: per (chunk, head) the forward map (M, Bm) and the output term R ----------------
@@ -447,38 +462,39 @@ __global__ void __launch_bounds__(kThreads, 1)
 {
     // shared memory: X[2], then M[2]
     const int t = threadIdx.x, h = blockIdx.x, s = blockIdx.y;
-    const int g = (t & 31) >> 2, q = t & 3, m0 = ((t >> 5) & 3) * 16, n0 = (t >> 7) * 32;
+    const int g = (t & 31) >> 2, q = t & 3, m0 = ((t >> 5) & 3) * 16, n0 = (t >> 7) * 8 * kNT;
+    constexpr int PER = MAT / 4 / kThreads;  // float4 pieces of a matrix per thread
     int first, count;
     seq_chunks(s, cu, off, T, first, count);
     const size_t st0 = ((size_t)s * H + h) * (size_t)MAT;
     auto chunk_base = [&](int i) { return ((size_t)(first + (REV ? count - 1 - i : i)) * H + h) * (size_t)MAT; };
-    auto fetch_m = [&](int i, float4 (&m)[4]) {
+    auto fetch_m = [&](int i, float4 (&m)[PER]) {
         const float4 *src = reinterpret_cast<const float4 *>(Mo + chunk_base(i));
 #pragma unroll
-        for (int u = 0; u < 4; ++u) m[u] = __ldg(src + t + u * kThreads);
+        for (int u = 0; u < PER; ++u) m[u] = __ldg(src + t + u * kThreads);
     };
-    auto fetch_a = [&](int i, float2 (&a)[8]) {  // the additive term in mm's layout
+    auto fetch_a = [&](int i, float2 (&a)[2 * kNT]) {  // the additive term in mm's layout
         const float *src = Add + chunk_base(i);
 #pragma unroll
-        for (int n = 0; n < 4; ++n)
+        for (int n = 0; n < kNT; ++n)
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh)
                 a[2 * n + hh] = __ldg(reinterpret_cast<const float2 *>(src + (m0 + g + 8 * hh) * N + n0 + 8 * n + 2 * q));
     };
-    auto put_m = [&](float *M, const float4 (&m)[4]) {
+    auto put_m = [&](float *M, const float4 (&m)[PER]) {
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
+        for (int u = 0; u < PER; ++u) {
             const int e = (t + u * kThreads) * 4;
             *reinterpret_cast<float4 *>(&M[sw(e >> 6, e & 63)]) = m[u];
         }
     };
-    float4 pm[4];
-    float2 pa[8], pa2[8];
+    float4 pm[PER];
+    float2 pa[2 * kNT], pa2[2 * kNT];
     if (X0) {
         mat_to_shared(smf, X0 + st0, t);
     } else {
 #pragma unroll
-        for (int u = 0; u < 4; ++u) reinterpret_cast<float4 *>(smf)[t + u * kThreads] = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int u = 0; u < PER; ++u) reinterpret_cast<float4 *>(smf)[t + u * kThreads] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
     if (count > 0) {
         fetch_m(0, pm);
@@ -502,7 +518,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (i + 1 < count) {
             put_m(Mnxt, pm);
 #pragma unroll
-            for (int u = 0; u < 8; ++u) pa[u] = pa2[u];
+            for (int u = 0; u < 2 * kNT; ++u) pa[u] = pa2[u];
         }
         if (i + 2 < count) {
             fetch_m(i + 2, pm);
@@ -557,14 +573,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     if (t < N) bg[t] = g.bet[t] * g.gam[t];
     // per thread, in mm's layout (index u): the dQ, dK, dV accumulators; partial d beta, d gam, dG
-    // and d lam over its two rows; partial dG over its eight columns
-    float aq[16], ak[16], av[16];
+    // and d lam over its two rows; partial dG over its columns
+    float aq[kFrag], ak[kFrag], av[kFrag];
     float pb[2] = {0.f, 0.f}, pg[2] = {0.f, 0.f}, pG[2] = {0.f, 0.f}, pl[2] = {0.f, 0.f};
-    float pc[8];
+    float pc[kColSlots];
 #pragma unroll
-    for (int i = 0; i < 16; ++i) aq[i] = ak[i] = av[i] = 0.f;
+    for (int i = 0; i < kFrag; ++i) aq[i] = ak[i] = av[i] = 0.f;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) pc[i] = 0.f;
+    for (int i = 0; i < kColSlots; ++i) pc[i] = 0.f;
     mm<false, true>(K, K, t, [&](int r, int i, float x, int) { KK[sw(r, i)] = x; });
     mm<false, true>(Q, K, t, [&](int r, int i, float x, int) { QK[sw(r, i)] = x; });
     mm<false, false>(K, dSp, t, [&](int i, int m, float x, int) { X2[sw(i, m)] = x; });  // K dS'
@@ -656,17 +672,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     mm<true, false>(X1, Q, t, [&](int, int, float x, int u) { ak[u] += x; });
     mm<false, false>(X1, K, t, [&](int, int, float x, int u) { aq[u] += x; });
     // the partial sums over the block (X2 is free scratch now: its last reader is two barriers back)
+    constexpr int RB = kColBlocks * N;  // scratch of one row sum
     row_put(pb, X2, t);
-    row_put(pg, X2 + 2 * N, t);
-    row_put(pG, X2 + 4 * N, t);
-    row_put(pl, X2 + 6 * N, t);
-    col_put(pc, X2 + 8 * N, t);
+    row_put(pg, X2 + RB, t);
+    row_put(pG, X2 + 2 * RB, t);
+    row_put(pl, X2 + 3 * RB, t);
+    col_put(pc, X2 + 4 * RB, t);
     __syncthreads();
     if (t < N) {
         dbet[t] = row_get(X2, t);
-        dgam[t] = row_get(X2 + 2 * N, t);
-        dG[t] = row_get(X2 + 4 * N, t) + col_get(X2 + 8 * N, t);
-        dlam[t] = row_get(X2 + 6 * N, t);
+        dgam[t] = row_get(X2 + RB, t);
+        dG[t] = row_get(X2 + 2 * RB, t) + col_get(X2 + 4 * RB, t);
+        dlam[t] = row_get(X2 + 3 * RB, t);
     }
     __syncthreads();
     // gate gradients: gam_r = exp(G_r), lam_i = exp(G_63 - G_i), gam_C = gam_63; then dlog_alpha_j =
@@ -696,14 +713,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     {
         const int lane = t & 31, w = t >> 5, gq = lane >> 2, qq = lane & 3;
-        const int m0 = (w & 3) * 16, n0 = (w >> 2) * 32;
+        const int m0 = (w & 3) * 16, n0 = (w >> 2) * 8 * kNT;
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
             const int r = m0 + gq + 8 * hh;
             if (r >= c.n) continue;
             const size_t row = ((size_t)(c.tok + r) * H + h) * N + n0 + 2 * qq;
 #pragma unroll
-            for (int n = 0; n < 4; ++n) {
+            for (int n = 0; n < kNT; ++n) {
                 const int u = 4 * n + 2 * hh;
                 *reinterpret_cast<float2 *>(dq + row + 8 * n) = make_float2(aq[u], aq[u + 1]);
                 *reinterpret_cast<float2 *>(dk + row + 8 * n) = make_float2(ak[u], ak[u + 1]);
