@@ -1,0 +1,148 @@
+"""fp64 oracle of the complex-phase delta memory (DeltaPhase README, section 2 "Complex Phase Matrix
+Delta Memory", with its gated-decay form; section 5 "Delta-Laplace Phase Memory Core" for keys
+e^{s dt}, Re s <= 0).
+
+TEST INFRASTRUCTURE ONLY (see ``oracle/__init__.py``): only tests/, the package's smoke check and
+bench.py's CPU baseline may import this module.
+
+Per (sequence, head) a complex state M in C^{dv x dk}; per token t, with complex key K_t and query
+Q_t (dk), real value V_t (dv), and scalars lam_t = exp(log_lam_t) in (0, 1] and beta_t:
+
+    v_old = (1/dk) Re(M_{t-1} conj(K_t))       read-out of the key from the previous state
+    e_t   = V_t - v_old                         error signal
+    M_t   = lam_t M_{t-1} + beta_t e_t K_t^T    decayed state plus the rank-one correction
+    o_t   = (1/dk) Re(M_t conj(Q_t))            read-out of the query
+
+The first three lines are the section's three steps with the gated decay; the read-out of the
+query (post-update state, the key's 1/dk scale) and lam_t as one scalar per (token, head) are
+readings (the section prints no query read-out; the Laplace core's per-row decay is not taken).
+
+``forward`` is that definition token by token in complex128.  ``forward_chunkwise`` is the chunk
+form derived separately (a unit-lower triangular solve per chunk for the errors), used as a pin.
+
+Inputs: K, Q complex arrays [..., H, dk] or real arrays [..., H, dk, 2] (re, im); V [..., H, dv];
+log_lam, beta [..., H]; M0 [B, H, dv, dk] complex (or [..., 2] real) or None (zero).  Dense
+tensors have leading [B, T]; with cu_seqlens they are packed [T_total, ...].
+Returns (out [..., H, dv] float64, M_final [B, H, dv, dk] complex128).
+"""
+from __future__ import annotations
+
+import numpy as np
+from scipy.linalg import solve_triangular
+
+
+def _np(x):
+    if x is None:
+        return None
+    if hasattr(x, "detach"):
+        x = x.detach().to("cpu")
+        x = x.double() if not x.is_complex() else x.to(dtype=__import__("torch").complex128)
+        x = x.numpy()
+    return np.asarray(x)
+
+
+def as_complex(x):
+    """Complex128 view of a complex array or of a real array whose last axis is (re, im)."""
+    x = _np(x)
+    if x is None:
+        return None
+    if np.iscomplexobj(x):
+        return x.astype(np.complex128)
+    assert x.shape[-1] == 2, x.shape
+    x = x.astype(np.float64)
+    return x[..., 0] + 1j * x[..., 1]
+
+
+def _real(x):
+    x = _np(x)
+    return None if x is None else x.astype(np.float64)
+
+
+def _sequences(n_lead, cu_seqlens, T_dense):
+    """(sequence index, token slice) for dense [B, T] or packed inputs."""
+    if cu_seqlens is None:
+        return [(b, None) for b in range(n_lead)]
+    cu = np.asarray(_np(cu_seqlens), dtype=np.int64)
+    return [(s, slice(int(cu[s]), int(cu[s + 1]))) for s in range(len(cu) - 1)]
+
+
+def forward(K, Q, V, log_lam, beta, M0=None, cu_seqlens=None):
+    """The definition, token by token (all (sequence, head) chains of a dense batch at once)."""
+    K, Q, M0 = as_complex(K), as_complex(Q), as_complex(M0)
+    V, la, be = _real(V), _real(log_lam), _real(beta)
+    dk, dv = K.shape[-1], V.shape[-1]
+    H = V.shape[-2]
+    out = np.zeros(V.shape)
+    if cu_seqlens is None:
+        B, T = V.shape[:2]
+        M = np.zeros((B, H, dv, dk), np.complex128) if M0 is None else M0.copy()
+        for t in range(T):
+            k, q = K[:, t], Q[:, t]                      # [B, H, dk]
+            v_old = np.einsum("bhji,bhi->bhj", M, np.conj(k)).real / dk
+            e = V[:, t] - v_old                          # [B, H, dv]
+            lam = np.exp(la[:, t])[..., None, None]
+            M = lam * M + (be[:, t, :, None] * e)[..., :, None] * k[..., None, :]
+            out[:, t] = np.einsum("bhji,bhi->bhj", M, np.conj(q)).real / dk
+        return out, M
+    seqs = _sequences(None, cu_seqlens, None)
+    Mf = np.zeros((len(seqs), H, dv, dk), np.complex128)
+    for s, sl in seqs:
+        M = np.zeros((H, dv, dk), np.complex128) if M0 is None else M0[s].copy()
+        for t in range(sl.start, sl.stop):
+            v_old = np.einsum("hji,hi->hj", M, np.conj(K[t])).real / dk
+            e = V[t] - v_old
+            M = np.exp(la[t])[:, None, None] * M + (be[t][:, None] * e)[:, :, None] * K[t][:, None, :]
+            out[t] = np.einsum("hji,hi->hj", M, np.conj(Q[t])).real / dk
+        Mf[s] = M
+    return out, Mf
+
+
+def _chunk(M0, K, Q, V, la, be):
+    """One chunk of one (sequence, head): M0 [dv, dk]; K, Q [C, dk]; V [C, dv]; la, be [C].
+
+    With g_t the sum of log_lam over the chunk's tokens up to t (g_{-1} = 0), the state before
+    token t is M_{t-1} = e^{g_{t-1}} M0 + sum_{s<t} e^{g_{t-1} - g_s} beta_s e_s K_s^T, so the errors
+    solve (I + A) E = V - (1/dk) diag(e^{g_{t-1}}) Re(conj(K) M0^T) with
+    A_ts = (1/dk) e^{g_{t-1} - g_s} beta_s Re(K_s . conj K_t) for s < t; then the outputs and the
+    exit state follow from E in closed form.
+    """
+    C, dk = K.shape
+    g = np.cumsum(la)
+    g_prev = np.concatenate([[0.0], g[:-1]])
+    gram_k = (K @ np.conj(K).T).real               # [s, t] -> Re(K_s . conj K_t)
+    gram_q = (K @ np.conj(Q).T).real               # [s, t] -> Re(K_s . conj Q_t)
+    t_idx, s_idx = np.meshgrid(np.arange(C), np.arange(C), indexing="ij")
+    A = np.where(s_idx < t_idx, np.exp(g_prev[:, None] - g[None, :]) * be[None, :] * gram_k.T, 0.0) / dk
+    rhs = V - np.exp(g_prev)[:, None] * (np.conj(K) @ M0.T).real / dk
+    E = solve_triangular(np.eye(C) + A, rhs, lower=True, unit_diagonal=True)
+    P = np.where(s_idx <= t_idx, np.exp(g[:, None] - g[None, :]) * be[None, :] * gram_q.T, 0.0)
+    O = (np.exp(g)[:, None] * (np.conj(Q) @ M0.T).real + P @ E) / dk
+    w = be * np.exp(g[-1] - g)
+    M_end = np.exp(g[-1]) * M0 + (E * w[:, None]).T @ K
+    return O, M_end
+
+
+def forward_chunkwise(K, Q, V, log_lam, beta, M0=None, chunk=64, cu_seqlens=None):
+    """The chunk form: the same results as ``forward`` up to rounding."""
+    K, Q, M0 = as_complex(K), as_complex(Q), as_complex(M0)
+    V, la, be = _real(V), _real(log_lam), _real(beta)
+    dk, dv = K.shape[-1], V.shape[-1]
+    H = V.shape[-2]
+    out = np.zeros(V.shape)
+    if cu_seqlens is None:
+        B, T = V.shape[:2]
+        runs = [(b, (b, slice(0, T))) for b in range(B)]
+    else:
+        runs = [(s, (sl,)) for s, sl in _sequences(None, cu_seqlens, None)]
+    Mf = np.zeros((len(runs), H, dv, dk), np.complex128)
+    for s, idx in runs:
+        sl = idx[-1]
+        for h in range(H):
+            M = np.zeros((dv, dk), np.complex128) if M0 is None else M0[s, h].copy()
+            for c0 in range(sl.start, sl.stop, chunk):
+                c1 = min(c0 + chunk, sl.stop)
+                rows = (*idx[:-1], slice(c0, c1), h)
+                O, M = _chunk(M, K[rows], Q[rows], V[rows], la[rows], be[rows])
+                out[rows] = O
+            Mf[s, h] = M
+    return out, Mf
