@@ -498,6 +498,40 @@ def run_ours(args, world, rank, local):
                                        "tf32_peak_tflops": round(tf32_peak, 1),
                                        "tensor_frac": round(3 * fl_b / (ms_b * 1e-3) / 1e12 / tf32_peak, 5)}
         del dout, wsb
+        # the complex-phase delta memory at the hybrid-LM shape (dk = 32 complex = 64 real, dv = 64)
+        ph = workloads.make_phase_inputs(B=8, T=4096, H=12, dk=32, dv=64, dtype="bf16", seed=530)
+        dph = {k: (v.cuda() if torch.is_tensor(v) else v) for k, v in ph.items()}
+        Kp, Qp = torch.view_as_real(dph["K"]).contiguous(), torch.view_as_real(dph["Q"]).contiguous()
+        out_p = torch.empty_like(dph["v"])
+        Mf_p = torch.empty(8, 12, 64, 32, 2, device="cuda")
+        need_p = gdn.gdn_phase_fwd_workspace_bytes(8, 4096, 12, 32, 64, 0, gdn.GDN_DTYPE_BF16)
+        wsp = torch.empty(need_p, dtype=torch.uint8, device="cuda")
+
+        def call_phase():
+            gdn.phase_fwd(Kp, Qp, dph["v"], dph["log_lam"], dph["beta"], out=out_p, M_final=Mf_p, workspace=wsp,
+                          stream=stream)
+        with torch.cuda.stream(stream):
+            for _ in range(3):
+                flush.zero_()
+                call_phase()
+            stream.synchronize()
+            evp = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(5)]
+            for a0, b0 in evp:
+                flush.zero_()
+                a0.record(stream)
+                call_phase()
+                b0.record(stream)
+            stream.synchronize()
+        ms_p = statistics.mean(a0.elapsed_time(b0) for a0, b0 in evp)
+        # bytes per token-head: K, Q (complex fp32), v and out (bf16), log_lam and beta; plus M_final
+        by_p = 393216 * (2 * 32 * 8 + 2 * 64 * 2 + 8) + 96 * 64 * 32 * 8
+        extra["phase_memory"] = {"workload": "complex-phase delta memory, hybrid_lm shape: B=8 T=4096 H=12, "
+                                             "dk=32 complex (64 real), dv=64, bf16 values, fp32 phasors",
+                                 "ms": round(ms_p, 6), "tokens_per_s": round(32768 / (ms_p * 1e-3), 1),
+                                 "launches_per_call": 3, "algo_bytes": by_p,
+                                 "gbs": round(by_p / (ms_p * 1e-3) / 1e9, 3),
+                                 "hbm_frac": round(by_p / (ms_p * 1e-3) / 1e9 / peaks["hbm_gbs"], 5)}
+        del dph, Kp, Qp, out_p, Mf_p, wsp
     cpu = None
     if rank == 0 and world == 1:
         cpu = cpu_oracle_baseline(inp)

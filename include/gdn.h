@@ -197,6 +197,31 @@ GDN_API size_t gdn_chunk_fwd_host_workspace_bytes(int B, int T, int H, int dk, i
                                                   int dtype);
 
 /*
+ * gdn_phase_fwd -- the complex-phase delta memory (DeltaPhase README, section 2 "Complex Phase
+ * Matrix Delta Memory" in its gated-decay form; keys e^{s dt} with Re s <= 0 as in section 5).
+ * Per (sequence, head) a complex state M in C^{dv x dk}; per token t, with complex key K_t and
+ * query Q_t (dk), real value V_t (dv) and scalars lam_t = exp(log_lam_t), beta_t:
+ *     e_t = V_t - (1/dk) Re(M_{t-1} conj K_t)          (read-out before the update)
+ *     M_t = lam_t M_{t-1} + beta_t e_t K_t^T
+ *     o_t = (1/dk) Re(M_t conj Q_t)                     (reading: the query reads the new state)
+ * Layouts (dense [B, T, ...] or packed with cu_seqlens, as gdn_chunk_fwd):
+ *     K, Q [.., H, dk, 2] fp32 (re, im pairs); v, out [.., H, dv] in dtype;
+ *     log_lam, beta [.., H] fp32; M0, M_final [B, H, dv, dk, 2] fp32 (re, im), either may be NULL.
+ * log_lam must be finite (lam > 0): the computation runs the real gated delta rule at head size
+ * 2 dk with a = lam and b = beta / lam (see gdn_phase.cu), on the tcgen05 kernel for bf16 and
+ * the fp32 CUDA-core kernel for fp32.  dk in {32, 64}, dv in {64, 128}.  Workspace:
+ * gdn_phase_fwd_workspace_bytes(...) bytes of device memory, 256-byte aligned.  Errors as
+ * gdn_chunk_fwd (the library's own scratch only is written before a late CUDA error).
+ */
+GDN_API int gdn_phase_fwd(const float *K, const float *Q, const void *v, const float *log_lam, const float *beta,
+                          const float *M0, void *out, float *M_final, int B, int T, int H, int dk, int dv,
+                          const int32_t *cu_seqlens, int dtype, void *workspace, size_t workspace_bytes,
+                          void *stream);
+
+/* Workspace gdn_phase_fwd needs for these sizes; (size_t)-1 for sizes it rejects. */
+GDN_API size_t gdn_phase_fwd_workspace_bytes(int B, int T, int H, int dk, int dv, int varlen, int dtype);
+
+/*
  * gdn_chunk_bwd -- gradients of gdn_chunk_fwd (the training path; Sykra README, "Architectural
  * Highlights": chunk-parallel training through the WY / unit triangular transform), for
  * dk = dv = 64 and chunk = 64.  Given the forward's inputs (same layouts, dtype for q, k, v and

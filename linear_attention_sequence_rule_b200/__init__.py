@@ -3,12 +3,12 @@
 Argument marshalling only: every step of the computation runs in the library's CUDA kernels.
 PyTorch provides device memory and streams.  The binding has two layers:
 
-* ``gdn_chunk_fwd``, ``gdn_chunk_fwd_noalloc``, ``gdn_chunk_fwd_host``, ``gdn_decode_step``,
+* ``gdn_chunk_fwd``, ``gdn_chunk_fwd_noalloc``, ``gdn_chunk_fwd_host``, ``gdn_phase_fwd``, ``gdn_decode_step``,
   ``gdn_chunk_fwd_workspace_bytes``, ``gdn_chunk_fwd_host_workspace_bytes``,
   ``gdn_status_string``, ``gdn_last_error``, ``gdn_version`` -- the C-ABI entry points of
   ``include/gdn.h`` with the same names and arguments (pointers as Python ints);
 * ``chunk_fwd``, ``chunk_fwd_host``, ``chunk_fwd_fused``, ``chunk_fwd_gva``, ``chunk_bwd``,
-  ``decode_step`` and ``decode_step_gva`` --
+  ``phase_fwd``, ``decode_step`` and ``decode_step_gva`` --
   the same calls taking torch tensors; they check shapes,
   devices and dtypes, allocate outputs with torch when none are given, and raise ``GdnError``
   on a non-zero status.
@@ -27,6 +27,7 @@ __all__ = [
     "GDN_ERR_CUDA", "GDN_ERR_TIMEOUT", "GDN_DTYPE_F32", "GDN_DTYPE_BF16", "LIB_PATH",
     "gdn_chunk_fwd", "gdn_chunk_fwd_noalloc", "gdn_chunk_fwd_fused", "gdn_chunk_fwd_gva",
     "gdn_chunk_fwd_host", "gdn_chunk_fwd_host_workspace_bytes", "chunk_fwd_host",
+    "gdn_phase_fwd", "gdn_phase_fwd_workspace_bytes", "phase_fwd",
     "gdn_decode_step", "gdn_decode_step_gva", "gdn_chunk_bwd", "gdn_chunk_bwd_workspace_bytes", "gdn_chunk_fwd_workspace_bytes", "gdn_status_string",
     "gdn_last_error", "gdn_version", "gdn_device_status", "device_status", "chunk_fwd", "chunk_fwd_fused",
     "chunk_fwd_gva", "chunk_bwd", "decode_step", "decode_step_gva", "workspace_bytes",
@@ -73,6 +74,10 @@ _lib.gdn_chunk_fwd_host.argtypes = list(_lib.gdn_chunk_fwd.argtypes)
 _lib.gdn_chunk_fwd_host.restype = _i
 _lib.gdn_chunk_fwd_host_workspace_bytes.argtypes = [_i, _i, _i, _i, _i, _i, _i, _i]
 _lib.gdn_chunk_fwd_host_workspace_bytes.restype = _sz
+_lib.gdn_phase_fwd.argtypes = [_vp] * 8 + [_i] * 5 + [_vp, _i, _vp, _sz, _vp]
+_lib.gdn_phase_fwd.restype = _i
+_lib.gdn_phase_fwd_workspace_bytes.argtypes = [_i] * 7
+_lib.gdn_phase_fwd_workspace_bytes.restype = _sz
 _lib.gdn_chunk_fwd_workspace_bytes.argtypes = [_i, _i, _i, _i, _i, _i, _i, _i]
 _lib.gdn_chunk_fwd_workspace_bytes.restype = _sz
 _lib.gdn_decode_step.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp]
@@ -145,6 +150,16 @@ def gdn_chunk_fwd_host(q, k, v, log_alpha, beta, S0, out, S_final, B, T, H, dk, 
 
 def gdn_chunk_fwd_host_workspace_bytes(B, T, H, dk, dv, chunk, varlen, dtype) -> int:
     return _lib.gdn_chunk_fwd_host_workspace_bytes(B, T, H, dk, dv, chunk, varlen, dtype)
+
+
+def gdn_phase_fwd(K, Q, v, log_lam, beta, M0, out, M_final, B, T, H, dk, dv, cu_seqlens, dtype, workspace,
+                  workspace_bytes, stream) -> int:
+    return _lib.gdn_phase_fwd(K, Q, v, log_lam, beta, M0, out, M_final, B, T, H, dk, dv, cu_seqlens, dtype,
+                              workspace, workspace_bytes, stream)
+
+
+def gdn_phase_fwd_workspace_bytes(B, T, H, dk, dv, varlen, dtype) -> int:
+    return _lib.gdn_phase_fwd_workspace_bytes(B, T, H, dk, dv, varlen, dtype)
 
 
 def gdn_chunk_fwd_workspace_bytes(B, T, H, dk, dv, chunk, varlen, dtype) -> int:
@@ -314,6 +329,68 @@ def chunk_fwd_host(q, k, v, log_alpha, beta, S0=None, cu_seqlens=None, out=None,
     if rc != GDN_OK:
         raise GdnError(rc, gdn_last_error())
     return out, S_final
+
+
+def _as_pairs(x, name):
+    """A complex tensor as contiguous fp32 (re, im) pairs; real tensors must already end in 2."""
+    if x is None:
+        return None
+    if x.is_complex():
+        x = torch.view_as_real(x.to(torch.complex64).contiguous())
+    if x.dtype != torch.float32 or x.shape[-1] != 2:
+        raise ValueError(f"{name} must be complex64 or float32 [..., 2]")
+    return x.contiguous()
+
+
+def phase_fwd(K, Q, v, log_lam, beta, M0=None, cu_seqlens=None, out=None, M_final=None,
+              output_final_state=True, workspace=None, stream=None):
+    """Complex-phase delta memory (``gdn_phase_fwd``).  K, Q complex [B,T,H,dk] (or packed [T,H,dk]
+    with cu_seqlens), complex64 or float32 [..., 2]; v [.., H, dv] bf16 (tensor-core path) or fp32;
+    log_lam, beta [.., H] fp32; M0 complex [B, H, dv, dk] or None.  Returns (out, M_final complex64
+    or None)."""
+    Kp, Qp = _as_pairs(K, "K"), _as_pairs(Q, "Q")
+    dt = v.dtype
+    if dt not in _DT:
+        raise ValueError(f"unsupported dtype {dt}")
+    dev = v.device
+    if cu_seqlens is not None:
+        T, H, dk = Kp.shape[:3]
+        B = cu_seqlens.shape[0] - 1
+        lead = (T,)
+        _need(cu_seqlens, "cu_seqlens", torch.int32, (B + 1,), dev)
+    else:
+        B, T, H, dk = Kp.shape[:4]
+        lead = (B, T)
+    dv = v.shape[-1]
+    _need(Kp, "K", torch.float32, (*lead, H, dk, 2), dev)
+    _need(Qp, "Q", torch.float32, (*lead, H, dk, 2), dev)
+    _need(v, "v", dt, (*lead, H, dv), dev)
+    _need(log_lam, "log_lam", torch.float32, (*lead, H), dev)
+    _need(beta, "beta", torch.float32, (*lead, H), dev)
+    M0p = _as_pairs(M0, "M0")
+    if M0p is not None:
+        _need(M0p, "M0", torch.float32, (B, H, dv, dk, 2), dev)
+    if out is None:
+        out = torch.empty((*lead, H, dv), dtype=dt, device=dev)
+    _need(out, "out", dt, (*lead, H, dv), dev)
+    Mf = None
+    if M_final is not None:
+        Mf = torch.view_as_real(M_final) if M_final.is_complex() else M_final
+    elif output_final_state:
+        Mf = torch.empty((B, H, dv, dk, 2), dtype=torch.float32, device=dev)
+    if Mf is not None:
+        _need(Mf, "M_final", torch.float32, (B, H, dv, dk, 2), dev)
+    need = gdn_phase_fwd_workspace_bytes(B, T, H, dk, dv, int(cu_seqlens is not None), _DT[dt])
+    if need == ctypes.c_size_t(-1).value:
+        raise GdnError(GDN_ERR_UNSUPPORTED, f"gdn_phase_fwd: unsupported sizes dk={dk} dv={dv}")
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    rc = gdn_phase_fwd(_ptr(Kp), _ptr(Qp), _ptr(v), _ptr(log_lam), _ptr(beta), _ptr(M0p), _ptr(out), _ptr(Mf),
+                       B, T, H, dk, dv, _ptr(cu_seqlens), _DT[dt], _ptr(workspace), workspace.numel(),
+                       _stream_ptr(stream))
+    if rc != GDN_OK:
+        raise GdnError(rc, gdn_last_error())
+    return out, (None if Mf is None else torch.view_as_complex(Mf))
 
 
 def chunk_fwd_fused(q_raw, k_raw, v, a_raw, b_raw, a_scale, b_scale, S0=None, cu_seqlens=None,

@@ -1,0 +1,222 @@
+// gdn_phase.cu -- gdn_phase_fwd: the complex-phase delta memory (DeltaPhase README, section 2
+// "Complex Phase Matrix Delta Memory", gated-decay form; section 5 for keys e^{s dt}) on the
+// chunk kernels of the real gated delta rule.
+//
+// Per (sequence, head) the state is M in C^{dv x dk}; per token
+//     e_t = V_t - (1/dk) Re(M_{t-1} conj K_t),   M_t = lam_t M_{t-1} + beta_t e_t K_t^T,
+//     o_t = (1/dk) Re(M_t conj Q_t).
+// Written over the real vector space C^dk = R^{2dk} with S = [Re M | Im M]^T (2dk x dv), this is
+//     S_t = lam_t S_{t-1} - (beta_t/dk) k~ k~^T S_{t-1} + beta_t k~ V_t^T,   o_t = (1/dk) S_t^T q~
+// with k~ = (Re K, Im K), q~ = (Re Q, Im Q): the real gated delta rule
+//     S_t = a_t (I - b_t k k^T) S_{t-1} + b_t k v^T,   o_t = S_t^T q
+// at head size 2dk with a = lam, b = beta / lam, k = k~ / sqrt(dk), v = lam sqrt(dk) V, q = q~ / dk
+// (lam > 0).  So one prologue kernel writes those inputs, the chunk kernel runs unchanged, and the
+// complex state is converted on the way in and out.
+#include <cuda_bf16.h>
+
+#include "gdn_internal.h"
+#include "../../include/gdn.h"
+
+namespace gdn {
+namespace {
+
+__device__ __forceinline__ float to_f(float x) { return x; }
+__device__ __forceinline__ float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }
+template <typename T> __device__ __forceinline__ T from_f(float x);
+template <> __device__ __forceinline__ float from_f<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float x) { return __float2bfloat16_rn(x); }
+
+// 1 / sqrt(DK) and sqrt(DK) for the two key sizes
+template <int DK> struct KeyScale;
+template <> struct KeyScale<32> {
+    static constexpr float inv_sqrt = 0.17677669529663688f, sqrt = 5.656854249492381f;
+};
+template <> struct KeyScale<64> {
+    static constexpr float inv_sqrt = 0.125f, sqrt = 8.0f;
+};
+
+// One thread per (token-head th, key element i): the real recurrence's inputs of token-head th.
+//   k[th] = (Re K, Im K) / sqrt(DK),  q[th] = (Re Q, Im Q) / DK     (2 DK elements each)
+//   v[th] = lam sqrt(DK) V[th]  (DV elements, threads i, i + DK, ...),  b[th] = beta / lam
+template <int DK, typename TV>
+__global__ void phase_prologue(const float2 *__restrict__ K, const float2 *__restrict__ Q, const TV *__restrict__ V,
+                               const float *__restrict__ log_lam, const float *__restrict__ beta, int DV,
+                               long token_heads, TV *__restrict__ kr, TV *__restrict__ qr, TV *__restrict__ vr,
+                               float *__restrict__ br)
+{
+    const long idx = (long)blockIdx.x * blockDim.x + threadIdx.x;
+    const long th = idx / DK;
+    const int i = (int)(idx % DK);
+    if (th >= token_heads) return;
+    const float ll = log_lam[th];
+    const float lam = expf(ll);
+    const float2 k = K[th * DK + i], q = Q[th * DK + i];
+    kr[th * 2 * DK + i] = from_f<TV>(k.x * KeyScale<DK>::inv_sqrt);
+    kr[th * 2 * DK + DK + i] = from_f<TV>(k.y * KeyScale<DK>::inv_sqrt);
+    qr[th * 2 * DK + i] = from_f<TV>(q.x * (1.0f / DK));
+    qr[th * 2 * DK + DK + i] = from_f<TV>(q.y * (1.0f / DK));
+    const float vs = lam * KeyScale<DK>::sqrt;
+    for (int j = i; j < DV; j += DK) vr[th * DV + j] = from_f<TV>(vs * to_f(V[th * DV + j]));
+    if (i == 0) br[th] = beta[th] * expf(-ll);
+}
+
+// Complex state [n, dv, dk] (re, im pairs) -> real state [n, 2dk, dv]: S[a][j] = Re M[j][a] (a < dk),
+// Im M[j][a - dk] (a >= dk); one thread per element of S.
+__global__ void phase_state_in(const float2 *__restrict__ M, float *__restrict__ S, int dk, int dv, long states)
+{
+    const long idx = (long)blockIdx.x * blockDim.x + threadIdx.x;
+    const long per = 2L * dk * dv;
+    if (idx >= states * per) return;
+    const long n = idx / per;
+    const int a = (int)((idx % per) / dv), j = (int)(idx % dv);
+    const float2 m = M[n * dk * dv + (long)j * dk + (a < dk ? a : a - dk)];
+    S[idx] = a < dk ? m.x : m.y;
+}
+
+// The reverse: one thread per complex element of M.
+__global__ void phase_state_out(const float *__restrict__ S, float2 *__restrict__ M, int dk, int dv, long states)
+{
+    const long idx = (long)blockIdx.x * blockDim.x + threadIdx.x;
+    const long per = (long)dk * dv;
+    if (idx >= states * per) return;
+    const long n = idx / per;
+    const int j = (int)((idx % per) / dk), a = (int)(idx % dk);
+    const float *s = S + n * 2 * per;
+    M[idx] = make_float2(s[(long)a * dv + j], s[(long)(a + dk) * dv + j]);
+}
+
+size_t al256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+struct PhasePlan {
+    size_t kr, qr, vr, br, s0, sf, ws, total, ws_bytes;
+};
+
+// Workspace: the real recurrence's k, q, v (element type of v), b (fp32), its states, and the
+// chunk forward's own scratch.
+bool phase_plan(PhasePlan &p, int B, int T, int H, int dk, int dv, int varlen, int dtype)
+{
+    const size_t ws = gdn_chunk_fwd_workspace_bytes(B, T, H, 2 * dk, dv, 64, varlen, dtype);
+    if (ws == (size_t)-1) return false;
+    const size_t es = dtype == GDN_DTYPE_BF16 ? 2 : 4;
+    const size_t th = (varlen ? (size_t)T : (size_t)B * T) * H;
+    size_t o = 0;
+    auto take = [&](size_t bytes) {
+        const size_t at = o;
+        o += al256(bytes);
+        return at;
+    };
+    p.kr = take(th * 2 * dk * es);
+    p.qr = take(th * 2 * dk * es);
+    p.vr = take(th * dv * es);
+    p.br = take(th * 4);
+    p.s0 = take((size_t)B * H * 2 * dk * dv * 4);
+    p.sf = take((size_t)B * H * 2 * dk * dv * 4);
+    p.ws_bytes = ws;
+    p.ws = take(ws);
+    p.total = o;
+    return true;
+}
+
+template <int DK, typename TV>
+cudaError_t launch_prologue(const float *K, const float *Q, const void *V, const float *log_lam, const float *beta,
+                            int dv, long token_heads, char *w, const PhasePlan &p, cudaStream_t st)
+{
+    const long threads = token_heads * DK;
+    const unsigned blocks = (unsigned)((threads + 255) / 256);
+    if (blocks)
+        phase_prologue<DK, TV><<<blocks, 256, 0, st>>>(
+            reinterpret_cast<const float2 *>(K), reinterpret_cast<const float2 *>(Q), static_cast<const TV *>(V),
+            log_lam, beta, dv, token_heads, reinterpret_cast<TV *>(w + p.kr), reinterpret_cast<TV *>(w + p.qr),
+            reinterpret_cast<TV *>(w + p.vr), reinterpret_cast<float *>(w + p.br));
+    return cudaGetLastError();
+}
+
+}  // namespace
+}  // namespace gdn
+
+using namespace gdn;
+
+extern "C" {
+
+size_t gdn_phase_fwd_workspace_bytes(int B, int T, int H, int dk, int dv, int varlen, int dtype)
+{
+    if (dk != 32 && dk != 64) return (size_t)-1;
+    PhasePlan p;
+    if (!phase_plan(p, B, T, H, dk, dv, varlen, dtype)) return (size_t)-1;
+    return p.total;
+}
+
+int gdn_phase_fwd(const float *K, const float *Q, const void *v, const float *log_lam, const float *beta,
+                  const float *M0, void *out, float *M_final, int B, int T, int H, int dk, int dv,
+                  const int32_t *cu_seqlens, int dtype, void *workspace, size_t workspace_bytes, void *stream)
+{
+    const int varlen = cu_seqlens != nullptr;
+    if (dk != 32 && dk != 64) {
+        set_error("gdn_phase_fwd: dk=%d, supported: 32 or 64 (the real recurrence runs at 2 dk)", dk);
+        return GDN_ERR_UNSUPPORTED;
+    }
+    PhasePlan p;
+    if (!phase_plan(p, B, T, H, dk, dv, varlen, dtype))  // the chunk forward's shape check gives the reason
+        return gdn_chunk_fwd(nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, B, T, H, 2 * dk,
+                             dv, 64, cu_seqlens, dtype, nullptr, 0, stream);
+    if (!K || !Q || !v || !log_lam || !beta || !out) {
+        set_error("gdn_phase_fwd: K, Q, v, log_lam, beta and out are required");
+        return GDN_ERR_INVALID_ARGUMENT;
+    }
+    const void *ptrs[] = {K, Q, v, log_lam, beta, M0, out, M_final, cu_seqlens};
+    for (const void *ptr : ptrs)
+        if (ptr && (reinterpret_cast<uintptr_t>(ptr) & 15u)) {
+            set_error("gdn_phase_fwd: pointer %p is not 16-byte aligned", ptr);
+            return GDN_ERR_INVALID_ARGUMENT;
+        }
+    if (!workspace || workspace_bytes < p.total) {
+        set_error("gdn_phase_fwd: workspace of %zu bytes needed, %zu given", p.total,
+                  workspace ? workspace_bytes : (size_t)0);
+        return GDN_ERR_WORKSPACE;
+    }
+    if (reinterpret_cast<uintptr_t>(workspace) & 255u) {
+        set_error("gdn_phase_fwd: workspace must be 256-byte aligned");
+        return GDN_ERR_INVALID_ARGUMENT;
+    }
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    char *w = static_cast<char *>(workspace);
+    const long token_heads = (varlen ? (long)T : (long)B * T) * H;
+    const long states = (long)B * H;
+    cudaError_t e;
+    if (dtype == GDN_DTYPE_BF16)
+        e = dk == 64 ? launch_prologue<64, __nv_bfloat16>(K, Q, v, log_lam, beta, dv, token_heads, w, p, st)
+                     : launch_prologue<32, __nv_bfloat16>(K, Q, v, log_lam, beta, dv, token_heads, w, p, st);
+    else
+        e = dk == 64 ? launch_prologue<64, float>(K, Q, v, log_lam, beta, dv, token_heads, w, p, st)
+                     : launch_prologue<32, float>(K, Q, v, log_lam, beta, dv, token_heads, w, p, st);
+    if (e == cudaSuccess && M0) {
+        const long n = states * 2 * dk * dv;
+        phase_state_in<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(reinterpret_cast<const float2 *>(M0),
+                                                                     reinterpret_cast<float *>(w + p.s0), dk, dv,
+                                                                     states);
+        e = cudaGetLastError();
+    }
+    if (e != cudaSuccess) {
+        set_error("gdn_phase_fwd: launch: %s", cudaGetErrorString(e));
+        return GDN_ERR_CUDA;
+    }
+    const int rc = gdn_chunk_fwd(w + p.qr, w + p.kr, w + p.vr, log_lam, reinterpret_cast<const float *>(w + p.br),
+                                 M0 ? reinterpret_cast<const float *>(w + p.s0) : nullptr, out,
+                                 M_final ? reinterpret_cast<float *>(w + p.sf) : nullptr, B, T, H, 2 * dk, dv, 64,
+                                 cu_seqlens, dtype, p.ws_bytes ? w + p.ws : nullptr, p.ws_bytes, stream);
+    if (rc != GDN_OK) return rc;
+    if (M_final) {
+        const long n = states * dk * dv;
+        phase_state_out<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(reinterpret_cast<const float *>(w + p.sf),
+                                                                      reinterpret_cast<float2 *>(M_final), dk, dv,
+                                                                      states);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) {
+            set_error("gdn_phase_fwd: launch: %s", cudaGetErrorString(e));
+            return GDN_ERR_CUDA;
+        }
+    }
+    return GDN_OK;
+}
+
+}  // extern "C"

@@ -190,3 +190,27 @@ def test_host_entry_rejects_before_any_copy():
     assert host_chunk(T=5, cu_seqlens=p) == gdn.GDN_ERR_INVALID_ARGUMENT
     p, keep = _cu(0, 3, 5)  # does not end at T
     assert host_chunk(T=6, cu_seqlens=p) == gdn.GDN_ERR_INVALID_ARGUMENT
+
+
+def phase_call(**kw):
+    a = dict(K=FAKE, Q=FAKE, v=FAKE, log_lam=FAKE, beta=FAKE, M0=None, out=FAKE, M_final=None, B=1, T=64, H=1,
+             dk=32, dv=64, cu_seqlens=None, dtype=gdn.GDN_DTYPE_BF16, workspace=FAKE * 256, workspace_bytes=1 << 40,
+             stream=None)
+    a.update(kw)
+    return gdn.gdn_phase_fwd(**a)
+
+
+def test_phase_entry_rejects_before_any_launch():
+    assert phase_call(dk=48) == gdn.GDN_ERR_UNSUPPORTED
+    assert phase_call(dk=128) == gdn.GDN_ERR_UNSUPPORTED   # 2 dk = 256 real columns
+    assert phase_call(dv=96) == gdn.GDN_ERR_UNSUPPORTED
+    assert phase_call(B=0) == gdn.GDN_ERR_INVALID_ARGUMENT
+    assert phase_call(K=None) == gdn.GDN_ERR_INVALID_ARGUMENT
+    assert phase_call(out=None) == gdn.GDN_ERR_INVALID_ARGUMENT
+    assert phase_call(Q=FAKE + 8) == gdn.GDN_ERR_INVALID_ARGUMENT
+    assert phase_call(workspace=None) == gdn.GDN_ERR_WORKSPACE
+    assert phase_call(workspace_bytes=1024) == gdn.GDN_ERR_WORKSPACE
+    assert gdn.gdn_phase_fwd_workspace_bytes(1, 64, 1, 48, 64, 0, gdn.GDN_DTYPE_BF16) == ctypes.c_size_t(-1).value
+    n = gdn.gdn_phase_fwd_workspace_bytes(2, 64, 3, 32, 64, 0, gdn.GDN_DTYPE_BF16)
+    token_heads = 2 * 64 * 3
+    assert n >= token_heads * (2 * 64 * 2 + 2 * 64 * 2 + 64 * 2 + 4)

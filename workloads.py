@@ -158,6 +158,41 @@ def make_gva_chunk_inputs(B=None, T=None, Hk=2, Hv=4, dk=64, dv=64, dtype="bf16"
                 lengths=lengths)
 
 
+def make_phase_inputs(B=None, T=None, H=2, dk=32, dv=64, dtype="bf16", seed=0, beta_scale=1.0, la_scale=0.1,
+                      m0_std=0.0, laplace=False, lengths=None, **_ignored):
+    """Inputs of the complex-phase delta memory: K, Q complex64 [..., H, dk] unit phasors e^{i theta},
+    theta ~ U[0, 2 pi) (K scaled by e^{sigma}, sigma ~ U[-0.5, 0] when ``laplace``); v [..., H, dv]
+    N(0, 1) in dtype; beta = beta_scale * sigmoid(N(0, 1)); log_lam = -softplus(N(0, 1)) * la_scale
+    (finite: lam > 0); M0 complex64 [B, H, dv, dk] with N(0, m0_std) parts, or None."""
+    g = torch.Generator().manual_seed(int(seed))
+    dt = DTYPES[dtype]
+    if lengths is not None:
+        lengths = [int(x) for x in lengths]
+        cu = torch.zeros(len(lengths) + 1, dtype=torch.int32)
+        cu[1:] = torch.cumsum(torch.tensor(lengths, dtype=torch.int64), 0).to(torch.int32)
+        lead = (int(cu[-1]),)
+        nseq = len(lengths)
+    else:
+        cu = None
+        lead = (int(B), int(T))
+        nseq = int(B)
+    two_pi = 6.283185307179586
+    th_k = two_pi * torch.rand(*lead, H, dk, generator=g)
+    th_q = two_pi * torch.rand(*lead, H, dk, generator=g)
+    mag = torch.exp(-0.5 * torch.rand(*lead, H, dk, generator=g)) if laplace else torch.ones(*lead, H, dk)
+    K = torch.polar(mag, th_k).to(torch.complex64)
+    Q = torch.polar(torch.ones_like(th_q), th_q).to(torch.complex64)
+    v = torch.randn(*lead, H, dv, generator=g).to(dt)
+    beta = (beta_scale * torch.sigmoid(torch.randn(*lead, H, generator=g))).float()
+    log_lam = (-torch.nn.functional.softplus(torch.randn(*lead, H, generator=g)) * la_scale).float()
+    M0 = None
+    if m0_std:
+        M0 = torch.complex(m0_std * torch.randn(nseq, H, dv, dk, generator=g),
+                           m0_std * torch.randn(nseq, H, dv, dk, generator=g)).to(torch.complex64)
+    return dict(K=K, Q=Q, v=v, log_lam=log_lam, beta=beta, M0=M0, cu_seqlens=cu, B=nseq,
+                T=(lead[0] if cu is not None else int(T)), H=H, dk=dk, dv=dv, dtype=dtype, lengths=lengths)
+
+
 def config_inputs(name: str, **overrides):
     """Inputs of a named chunk workload (``tiny``, ``hybrid_lm``, ``long_context``, ``varlen``)."""
     cfg = dict(CONFIGS[name])
