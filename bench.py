@@ -460,78 +460,8 @@ def run_ours(args, world, rank, local):
                                   "ms": round(ms_g, 6), "tokens_per_s": round(8 * 4096 / (ms_g * 1e-3), 1),
                                   "launches_per_call": 1}
         del dg, outg, Sg
-        # backward of the hybrid-LM step (dq, dk, dv, gate and state gradients; fp32-accurate products
-        # on the tensor cores as three tf32 terms)
-        dout = torch.randn(d["v"].shape, device="cuda").to(d["v"].dtype)
-        wsb = torch.empty(gdn.gdn_chunk_bwd_workspace_bytes(8, 4096, 12, 64, 64, 64, 0), dtype=torch.uint8,
-                          device="cuda")
-
-        def call_bwd():
-            gdn.chunk_bwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], dout, workspace=wsb, stream=stream)
-        with torch.cuda.stream(stream):
-            for _ in range(3):
-                flush.zero_()
-                call_bwd()
-            stream.synchronize()
-            evb = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(5)]
-            for a0, b0 in evb:
-                flush.zero_()
-                a0.record(stream)
-                call_bwd()
-                b0.record(stream)
-            stream.synchronize()
-        ms_b = statistics.mean(a0.elapsed_time(b0) for a0, b0 in evb)
-        # bytes per token-head: q, k, v, dout (bf16) and gates in; dq, dk, dv (fp32) and two gate grads out
-        by_b = 393216 * (4 * 64 * 2 + 8 + 3 * 64 * 4 + 8)
-        # products per (chunk, head): 9 (prep) + 22 (grads) + 1 in each scan, each 2 * 64^3 flops in
-        # fp32; the tensor cores execute three tf32 products for each
-        fl_b = 6144 * 33 * 2 * 64 ** 3
-        tf32_peak = peaks["bf16_tflops"] * TF32_PER_BF16
-        extra["hybrid_lm_backward"] = {"workload": "hybrid_lm backward: dq, dk, dv, dlog_alpha, dbeta (fp32) from dout",
-                                       "ms": round(ms_b, 6), "tokens_per_s": round(32768 / (ms_b * 1e-3), 1),
-                                       "launches_per_call": 4, "algo_bytes": by_b,
-                                       "gbs": round(by_b / (ms_b * 1e-3) / 1e9, 3),
-                                       "hbm_frac": round(by_b / (ms_b * 1e-3) / 1e9 / peaks["hbm_gbs"], 5),
-                                       "algo_flops_fp32": fl_b,
-                                       "fp32_tflops": round(fl_b / (ms_b * 1e-3) / 1e12, 3),
-                                       "tf32_mma_tflops": round(3 * fl_b / (ms_b * 1e-3) / 1e12, 3),
-                                       "tf32_peak_tflops": round(tf32_peak, 1),
-                                       "tensor_frac": round(3 * fl_b / (ms_b * 1e-3) / 1e12 / tf32_peak, 5)}
-        del dout, wsb
-        # the complex-phase delta memory at the hybrid-LM shape (dk = 32 complex = 64 real, dv = 64)
-        ph = workloads.make_phase_inputs(B=8, T=4096, H=12, dk=32, dv=64, dtype="bf16", seed=530)
-        dph = {k: (v.cuda() if torch.is_tensor(v) else v) for k, v in ph.items()}
-        Kp, Qp = torch.view_as_real(dph["K"]).contiguous(), torch.view_as_real(dph["Q"]).contiguous()
-        out_p = torch.empty_like(dph["v"])
-        Mf_p = torch.empty(8, 12, 64, 32, 2, device="cuda")
-        need_p = gdn.gdn_phase_fwd_workspace_bytes(8, 4096, 12, 32, 64, 0, gdn.GDN_DTYPE_BF16)
-        wsp = torch.empty(need_p, dtype=torch.uint8, device="cuda")
-
-        def call_phase():
-            gdn.phase_fwd(Kp, Qp, dph["v"], dph["log_lam"], dph["beta"], out=out_p, M_final=Mf_p, workspace=wsp,
-                          stream=stream)
-        with torch.cuda.stream(stream):
-            for _ in range(3):
-                flush.zero_()
-                call_phase()
-            stream.synchronize()
-            evp = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(5)]
-            for a0, b0 in evp:
-                flush.zero_()
-                a0.record(stream)
-                call_phase()
-                b0.record(stream)
-            stream.synchronize()
-        ms_p = statistics.mean(a0.elapsed_time(b0) for a0, b0 in evp)
-        # bytes per token-head: K, Q (complex fp32), v and out (bf16), log_lam and beta; plus M_final
-        by_p = 393216 * (2 * 32 * 8 + 2 * 64 * 2 + 8) + 96 * 64 * 32 * 8
-        extra["phase_memory"] = {"workload": "complex-phase delta memory, hybrid_lm shape: B=8 T=4096 H=12, "
-                                             "dk=32 complex (64 real), dv=64, bf16 values, fp32 phasors",
-                                 "ms": round(ms_p, 6), "tokens_per_s": round(32768 / (ms_p * 1e-3), 1),
-                                 "launches_per_call": 3, "algo_bytes": by_p,
-                                 "gbs": round(by_p / (ms_p * 1e-3) / 1e9, 3),
-                                 "hbm_frac": round(by_p / (ms_p * 1e-3) / 1e9 / peaks["hbm_gbs"], 5)}
-        del dph, Kp, Qp, out_p, Mf_p, wsp
+        extra["hybrid_lm_backward"] = backward_numbers(gdn, d, 5, 3, flush, stream, peaks)
+        extra["phase_memory"] = phase_numbers(gdn, 5, 3, flush, stream, peaks)
     cpu = None
     if rank == 0 and world == 1:
         cpu = cpu_oracle_baseline(inp)
@@ -577,6 +507,77 @@ def run_ours(args, world, rank, local):
     print(json.dumps(line), flush=True)
 
 
+def _time_loop(call, steps, warmup, flush, stream):
+    """Mean CUDA-event time (ms) of `call` on `stream` over `steps` calls after `warmup`, L2 flushed
+    before each."""
+    with torch.cuda.stream(stream):
+        for _ in range(warmup):
+            flush.zero_()
+            call()
+        stream.synchronize()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+        for a0, b0 in ev:
+            flush.zero_()
+            a0.record(stream)
+            call()
+            b0.record(stream)
+        stream.synchronize()
+    return statistics.mean(a0.elapsed_time(b0) for a0, b0 in ev)
+
+
+def backward_numbers(gdn, d, steps, warmup, flush, stream, peaks):
+    """The backward of the hybrid-LM step (dq, dk, dv, gate and state gradients; fp32-accurate
+    products on the tensor cores as three tf32 terms) from a seeded dout; `d` holds the hybrid-LM
+    inputs on the device."""
+    dout = torch.randn(d["v"].shape, device="cuda", generator=torch.Generator("cuda").manual_seed(7)).to(d["v"].dtype)
+    wsb = torch.empty(gdn.gdn_chunk_bwd_workspace_bytes(8, 4096, 12, 64, 64, 64, 0), dtype=torch.uint8,
+                      device="cuda")
+
+    def call():
+        gdn.chunk_bwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], dout, workspace=wsb, stream=stream)
+    ms_b = _time_loop(call, steps, warmup, flush, stream)
+    # bytes per token-head: q, k, v, dout (bf16) and gates in; dq, dk, dv (fp32) and two gate grads out
+    by_b = 393216 * (4 * 64 * 2 + 8 + 3 * 64 * 4 + 8)
+    # products per (chunk, head): 9 (prep) + 22 (grads) + 1 in each scan, each 2 * 64^3 flops in
+    # fp32; the tensor cores execute three tf32 products for each
+    fl_b = 6144 * 33 * 2 * 64 ** 3
+    tf32_peak = peaks["bf16_tflops"] * TF32_PER_BF16
+    return {"workload": "hybrid_lm backward: dq, dk, dv, dlog_alpha, dbeta (fp32) from dout",
+            "ms": round(ms_b, 6), "tokens_per_s": round(32768 / (ms_b * 1e-3), 1),
+            "launches_per_call": 4, "algo_bytes": by_b,
+            "gbs": round(by_b / (ms_b * 1e-3) / 1e9, 3),
+            "hbm_frac": round(by_b / (ms_b * 1e-3) / 1e9 / peaks["hbm_gbs"], 5),
+            "algo_flops_fp32": fl_b,
+            "fp32_tflops": round(fl_b / (ms_b * 1e-3) / 1e12, 3),
+            "tf32_mma_tflops": round(3 * fl_b / (ms_b * 1e-3) / 1e12, 3),
+            "tf32_peak_tflops": round(tf32_peak, 1),
+            "tensor_frac": round(3 * fl_b / (ms_b * 1e-3) / 1e12 / tf32_peak, 5)}
+
+
+def phase_numbers(gdn, steps, warmup, flush, stream, peaks):
+    """The complex-phase delta memory at the hybrid-LM shape (dk = 32 complex = 64 real, dv = 64)."""
+    ph = workloads.make_phase_inputs(B=8, T=4096, H=12, dk=32, dv=64, dtype="bf16", seed=530)
+    dph = {k: (v.cuda() if torch.is_tensor(v) else v) for k, v in ph.items()}
+    Kp, Qp = torch.view_as_real(dph["K"]).contiguous(), torch.view_as_real(dph["Q"]).contiguous()
+    out_p = torch.empty_like(dph["v"])
+    Mf_p = torch.empty(8, 12, 64, 32, 2, device="cuda")
+    wsp = torch.empty(gdn.gdn_phase_fwd_workspace_bytes(8, 4096, 12, 32, 64, 0, gdn.GDN_DTYPE_BF16),
+                      dtype=torch.uint8, device="cuda")
+
+    def call():
+        gdn.phase_fwd(Kp, Qp, dph["v"], dph["log_lam"], dph["beta"], out=out_p, M_final=Mf_p, workspace=wsp,
+                      stream=stream)
+    ms_p = _time_loop(call, steps, warmup, flush, stream)
+    # bytes per token-head: K, Q (complex fp32), v and out (bf16), log_lam and beta; plus M_final
+    by_p = 393216 * (2 * 32 * 8 + 2 * 64 * 2 + 8) + 96 * 64 * 32 * 8
+    return {"workload": "complex-phase delta memory, hybrid_lm shape: B=8 T=4096 H=12, "
+                        "dk=32 complex (64 real), dv=64, bf16 values, fp32 phasors",
+            "ms": round(ms_p, 6), "tokens_per_s": round(32768 / (ms_p * 1e-3), 1),
+            "launches_per_call": 3, "algo_bytes": by_p,
+            "gbs": round(by_p / (ms_p * 1e-3) / 1e9, 3),
+            "hbm_frac": round(by_p / (ms_p * 1e-3) / 1e9 / peaks["hbm_gbs"], 5)}
+
+
 def run_only(args):
     """One workload's timing loop, no e2e / CPU baseline; prints that workload's numbers."""
     import linear_attention_sequence_rule_b200 as gdn
@@ -585,6 +586,13 @@ def run_only(args):
     if args.only == "decode":
         r = time_decode(gdn, args.steps, args.warmup, stream)
         r["hbm_frac"] = r["gbs"] / peaks["hbm_gbs"]
+    elif args.only == "hybrid_lm_backward":
+        flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device="cuda")
+        r = backward_numbers(gdn, to_dev(workloads.config_inputs("hybrid_lm")), args.steps, args.warmup, flush,
+                             stream, peaks)
+    elif args.only == "phase_memory":
+        flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device="cuda")
+        r = phase_numbers(gdn, args.steps, args.warmup, flush, stream, peaks)
     elif args.only in ("hybrid_lm_fused", "hybrid_lm_unfused"):
         flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device="cuda")
         d = to_dev(workloads.config_raw_inputs("hybrid_lm"))
@@ -659,7 +667,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--quick", action="store_true", help="main workload only")
     ap.add_argument("--only", choices=["hybrid_lm", "long_context", "varlen", "tiny", "decode", "hybrid_lm_fused",
-                                             "hybrid_lm_unfused"],
+                                             "hybrid_lm_unfused", "hybrid_lm_backward", "phase_memory"],
                     help="time one workload's kernel loop only (for profiler runs)")
     args = ap.parse_args()
     if args.warmup < 3:

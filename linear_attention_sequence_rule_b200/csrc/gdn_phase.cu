@@ -22,9 +22,6 @@ namespace {
 
 __device__ __forceinline__ float to_f(float x) { return x; }
 __device__ __forceinline__ float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }
-template <typename T> __device__ __forceinline__ T from_f(float x);
-template <> __device__ __forceinline__ float from_f<float>(float x) { return x; }
-template <> __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float x) { return __float2bfloat16_rn(x); }
 
 // 1 / sqrt(DK) and sqrt(DK) for the two key sizes
 template <int DK> struct KeyScale;
@@ -35,28 +32,58 @@ template <> struct KeyScale<64> {
     static constexpr float inv_sqrt = 0.125f, sqrt = 8.0f;
 };
 
-// One thread per (token-head th, key element i): the real recurrence's inputs of token-head th.
+// The real recurrence's inputs of token-head th, written by DK / 4 threads, thread i taking key
+// elements 4i .. 4i + 3 (two 16-byte loads each of K and Q) and value elements i DV' .. (i + 1) DV'
+// - 1, DV' = 4 DV / DK:
 //   k[th] = (Re K, Im K) / sqrt(DK),  q[th] = (Re Q, Im Q) / DK     (2 DK elements each)
-//   v[th] = lam sqrt(DK) V[th]  (DV elements, threads i, i + DK, ...),  b[th] = beta / lam
-template <int DK, typename TV>
-__global__ void phase_prologue(const float2 *__restrict__ K, const float2 *__restrict__ Q, const TV *__restrict__ V,
-                               const float *__restrict__ log_lam, const float *__restrict__ beta, int DV,
-                               long token_heads, TV *__restrict__ kr, TV *__restrict__ qr, TV *__restrict__ vr,
-                               float *__restrict__ br)
+//   v[th] = lam sqrt(DK) V[th],  b[th] = beta / lam
+template <typename TV> struct Pack4;  // four elements as one store
+template <> struct Pack4<float> {
+    using type = float4;
+    __device__ static float4 make(float a, float b, float c, float d) { return make_float4(a, b, c, d); }
+};
+template <> struct Pack4<__nv_bfloat16> {
+    using type = uint2;
+    __device__ static uint2 make(float a, float b, float c, float d)
+    {
+        const __nv_bfloat162 lo = __floats2bfloat162_rn(a, b), hi = __floats2bfloat162_rn(c, d);
+        return make_uint2(*reinterpret_cast<const uint32_t *>(&lo), *reinterpret_cast<const uint32_t *>(&hi));
+    }
+};
+
+template <int DK, int DV, typename TV>
+__global__ void __launch_bounds__(256) phase_prologue(const float4 *__restrict__ K, const float4 *__restrict__ Q,
+                                                      const TV *__restrict__ V, const float *__restrict__ log_lam,
+                                                      const float *__restrict__ beta, long token_heads,
+                                                      TV *__restrict__ kr, TV *__restrict__ qr, TV *__restrict__ vr,
+                                                      float *__restrict__ br)
 {
+    constexpr int TPT = DK / 4;       // threads per token-head
+    constexpr int VPT = DV / TPT;     // value elements per thread
+    using P = Pack4<TV>;
     const long idx = (long)blockIdx.x * blockDim.x + threadIdx.x;
-    const long th = idx / DK;
-    const int i = (int)(idx % DK);
+    const long th = idx / TPT;
+    const int i = (int)(idx % TPT);
     if (th >= token_heads) return;
     const float ll = log_lam[th];
+    // complex elements 4i .. 4i + 3 = float4 pieces 2i, 2i + 1 of the token-head's (re, im) row
+    const float4 k0 = K[th * (DK / 2) + 2 * i], k1 = K[th * (DK / 2) + 2 * i + 1];
+    const float4 q0 = Q[th * (DK / 2) + 2 * i], q1 = Q[th * (DK / 2) + 2 * i + 1];
+    TV vin[VPT];
+#pragma unroll
+    for (int e = 0; e < VPT; ++e) vin[e] = V[th * DV + i * VPT + e];
     const float lam = expf(ll);
-    const float2 k = K[th * DK + i], q = Q[th * DK + i];
-    kr[th * 2 * DK + i] = from_f<TV>(k.x * KeyScale<DK>::inv_sqrt);
-    kr[th * 2 * DK + DK + i] = from_f<TV>(k.y * KeyScale<DK>::inv_sqrt);
-    qr[th * 2 * DK + i] = from_f<TV>(q.x * (1.0f / DK));
-    qr[th * 2 * DK + DK + i] = from_f<TV>(q.y * (1.0f / DK));
+    constexpr float ks = KeyScale<DK>::inv_sqrt, qs = 1.0f / DK;
+    using S = typename P::type;
+    reinterpret_cast<S *>(kr + th * 2 * DK)[i] = P::make(k0.x * ks, k0.z * ks, k1.x * ks, k1.z * ks);
+    reinterpret_cast<S *>(kr + th * 2 * DK + DK)[i] = P::make(k0.y * ks, k0.w * ks, k1.y * ks, k1.w * ks);
+    reinterpret_cast<S *>(qr + th * 2 * DK)[i] = P::make(q0.x * qs, q0.z * qs, q1.x * qs, q1.z * qs);
+    reinterpret_cast<S *>(qr + th * 2 * DK + DK)[i] = P::make(q0.y * qs, q0.w * qs, q1.y * qs, q1.w * qs);
     const float vs = lam * KeyScale<DK>::sqrt;
-    for (int j = i; j < DV; j += DK) vr[th * DV + j] = from_f<TV>(vs * to_f(V[th * DV + j]));
+#pragma unroll
+    for (int e = 0; e < VPT; e += 4)
+        reinterpret_cast<S *>(vr + th * DV + i * VPT + e)[0] =
+            P::make(vs * to_f(vin[e]), vs * to_f(vin[e + 1]), vs * to_f(vin[e + 2]), vs * to_f(vin[e + 3]));
     if (i == 0) br[th] = beta[th] * expf(-ll);
 }
 
@@ -117,18 +144,29 @@ bool phase_plan(PhasePlan &p, int B, int T, int H, int dk, int dv, int varlen, i
     return true;
 }
 
-template <int DK, typename TV>
+template <int DK, int DV, typename TV>
 cudaError_t launch_prologue(const float *K, const float *Q, const void *V, const float *log_lam, const float *beta,
-                            int dv, long token_heads, char *w, const PhasePlan &p, cudaStream_t st)
+                            long token_heads, char *w, const PhasePlan &p, cudaStream_t st)
 {
-    const long threads = token_heads * DK;
+    const long threads = token_heads * (DK / 4);
     const unsigned blocks = (unsigned)((threads + 255) / 256);
     if (blocks)
-        phase_prologue<DK, TV><<<blocks, 256, 0, st>>>(
-            reinterpret_cast<const float2 *>(K), reinterpret_cast<const float2 *>(Q), static_cast<const TV *>(V),
-            log_lam, beta, dv, token_heads, reinterpret_cast<TV *>(w + p.kr), reinterpret_cast<TV *>(w + p.qr),
+        phase_prologue<DK, DV, TV><<<blocks, 256, 0, st>>>(
+            reinterpret_cast<const float4 *>(K), reinterpret_cast<const float4 *>(Q), static_cast<const TV *>(V),
+            log_lam, beta, token_heads, reinterpret_cast<TV *>(w + p.kr), reinterpret_cast<TV *>(w + p.qr),
             reinterpret_cast<TV *>(w + p.vr), reinterpret_cast<float *>(w + p.br));
     return cudaGetLastError();
+}
+
+template <typename TV>
+cudaError_t prologue_for(int dk, int dv, const float *K, const float *Q, const void *V, const float *log_lam,
+                         const float *beta, long token_heads, char *w, const PhasePlan &p, cudaStream_t st)
+{
+    if (dk == 64)
+        return dv == 128 ? launch_prologue<64, 128, TV>(K, Q, V, log_lam, beta, token_heads, w, p, st)
+                         : launch_prologue<64, 64, TV>(K, Q, V, log_lam, beta, token_heads, w, p, st);
+    return dv == 128 ? launch_prologue<32, 128, TV>(K, Q, V, log_lam, beta, token_heads, w, p, st)
+                     : launch_prologue<32, 64, TV>(K, Q, V, log_lam, beta, token_heads, w, p, st);
 }
 
 }  // namespace
@@ -140,7 +178,7 @@ extern "C" {
 
 size_t gdn_phase_fwd_workspace_bytes(int B, int T, int H, int dk, int dv, int varlen, int dtype)
 {
-    if (dk != 32 && dk != 64) return (size_t)-1;
+    if ((dk != 32 && dk != 64) || (dv != 64 && dv != 128)) return (size_t)-1;
     PhasePlan p;
     if (!phase_plan(p, B, T, H, dk, dv, varlen, dtype)) return (size_t)-1;
     return p.total;
@@ -151,8 +189,9 @@ int gdn_phase_fwd(const float *K, const float *Q, const void *v, const float *lo
                   const int32_t *cu_seqlens, int dtype, void *workspace, size_t workspace_bytes, void *stream)
 {
     const int varlen = cu_seqlens != nullptr;
-    if (dk != 32 && dk != 64) {
-        set_error("gdn_phase_fwd: dk=%d, supported: 32 or 64 (the real recurrence runs at 2 dk)", dk);
+    if ((dk != 32 && dk != 64) || (dv != 64 && dv != 128)) {
+        set_error("gdn_phase_fwd: dk=%d dv=%d, supported: dk 32 or 64 (the real recurrence runs at 2 dk), dv 64 or "
+                  "128", dk, dv);
         return GDN_ERR_UNSUPPORTED;
     }
     PhasePlan p;
@@ -183,12 +222,9 @@ int gdn_phase_fwd(const float *K, const float *Q, const void *v, const float *lo
     const long token_heads = (varlen ? (long)T : (long)B * T) * H;
     const long states = (long)B * H;
     cudaError_t e;
-    if (dtype == GDN_DTYPE_BF16)
-        e = dk == 64 ? launch_prologue<64, __nv_bfloat16>(K, Q, v, log_lam, beta, dv, token_heads, w, p, st)
-                     : launch_prologue<32, __nv_bfloat16>(K, Q, v, log_lam, beta, dv, token_heads, w, p, st);
-    else
-        e = dk == 64 ? launch_prologue<64, float>(K, Q, v, log_lam, beta, dv, token_heads, w, p, st)
-                     : launch_prologue<32, float>(K, Q, v, log_lam, beta, dv, token_heads, w, p, st);
+    e = dtype == GDN_DTYPE_BF16
+            ? prologue_for<__nv_bfloat16>(dk, dv, K, Q, v, log_lam, beta, token_heads, w, p, st)
+            : prologue_for<float>(dk, dv, K, Q, v, log_lam, beta, token_heads, w, p, st);
     if (e == cudaSuccess && M0) {
         const long n = states * 2 * dk * dv;
         phase_state_in<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(reinterpret_cast<const float2 *>(M0),
