@@ -71,3 +71,23 @@ def test_varlen_ragged_with_resets_and_beta_two():
 def test_hybrid_lm_heads_on_a_short_sequence():
     inp = workloads.make_chunk_inputs(B=2, T=512, H=12, dk=64, dv=64, dtype="bf16", seed=14, la_scale=0.1)
     check(inp, 4)
+
+
+def test_hybrid_lm_full_size_sampled_sequences():
+    # the benchmark's launch: all 8 x 4096 tokens x 12 heads on the GPU; the oracle checks two of
+    # the eight sequences (every head), which depend on nothing outside themselves
+    import linear_attention_sequence_rule_b200 as gdn
+    inp = workloads.config_inputs("hybrid_lm")
+    g = torch.Generator().manual_seed(15)
+    dout = torch.randn(inp["v"].shape, generator=g).to(inp["v"].dtype)
+    d = {k2: (v2.cuda() if torch.is_tensor(v2) else v2) for k2, v2 in inp.items()}
+    got = gdn.chunk_bwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], dout.cuda())
+    gdn.device_status()
+    for s in (0, 7):
+        sl = slice(s, s + 1)
+        ref = oracle.backward(inp["q"][sl], inp["k"][sl], inp["v"][sl], inp["log_alpha"][sl], inp["beta"][sl], None,
+                              dout[sl], None)
+        for name, a, b in zip(("dq", "dk", "dv", "dlog_alpha", "dbeta"), got, ref):
+            a = f64(a[sl])
+            err = float(np.max(np.abs(a - b)) / (1.0 + np.max(np.abs(b))))
+            assert err <= RTOL, (s, name, err)
