@@ -62,6 +62,10 @@ constexpr int kFlagS0Identity = 2;
 // beta = b_scale sigmoid(b) (DeltaPhase README, section 1: beta = 2 sigmoid(W_beta x)).
 constexpr int kFlagPrologue = 4;
 constexpr float kNormEps = 1e-6f;
+// Longest sequence first (varlen launches of at most THREADS sequences): CTA z takes the sequence
+// of rank z by length (ties by index), so that the longest chains, which set the launch's length,
+// start in the first wave instead of wherever the packing put them.
+constexpr int kFlagLongestFirst = 8;
 
 template <int DK, int DV>
 struct TcCfg {
@@ -424,7 +428,23 @@ __global__ void __launch_bounds__(TcCfg<DK, DV>::THREADS, 1)
     const Ctl ctl{bars, abort_flag};
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int h = blockIdx.y, s = blockIdx.z;
+    const int h = blockIdx.y;
+    int s = blockIdx.z;
+    if (flags & kFlagLongestFirst) {  // gridDim.z <= THREADS sequences: thread i ranks sequence i
+        int *pick = reinterpret_cast<int *>(sm + L::MISC + 8);
+        const int nseq = (int)gridDim.z;
+        if (tid < nseq) {
+            const int mine = cu_seqlens[tid + 1] - cu_seqlens[tid];
+            int rank = 0;
+            for (int o = 0; o < nseq; ++o) {
+                const int other = cu_seqlens[o + 1] - cu_seqlens[o];
+                rank += (other > mine) || (other == mine && o < tid);
+            }
+            if (rank == (int)blockIdx.z) *pick = tid;
+        }
+        __syncthreads();
+        s = *pick;
+    }
     const int hq = G == 1 ? h : h / G;  // q/k head of value head h (G value heads share one q/k head)
     long tok0, len;
     if (cu_seqlens) {
@@ -1171,8 +1191,9 @@ cudaError_t run_chunk(const ChunkArgs &a, cudaStream_t st)
     const int pf = a.prologue ? kFlagPrologue : 0;
     const float as = a.a_scale, bs = a.b_scale;
     if (p.G <= 1) {
+        const int lf = (a.cu_seqlens && a.B <= TcCfg<DK, DV>::THREADS) ? kFlagLongestFirst : 0;
         return launch_tc<DK, DV>(TcLaunch{a.q, a.k, a.v, a.log_alpha, a.beta, a.S0, a.out, a.S_final,
-                                          a.cu_seqlens, a.B, a.T, a.H, tokens, pf, as, bs, a.G},
+                                          a.cu_seqlens, a.B, a.T, a.H, tokens, pf | lf, as, bs, a.G},
                                  st);
     }
     const SegWork w = seg_layout(a.workspace, a.B, a.H, DK, DV, p);
