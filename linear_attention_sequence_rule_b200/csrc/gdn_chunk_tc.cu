@@ -1131,52 +1131,58 @@ __global__ void seg_table_kernel(int32_t *cu, int B, int T, int G, int L)
     }
 }
 
-// Pass B: one CTA of 256 threads per (32 value columns, head, sequence).  S (dk x 32, fp32) is
-// kept in shared memory; S_in of every segment is written out, then S <- M_g S + S_loc,g.
+// Pass B: one CTA of 256 threads per (32 value columns, head, sequence).  S (DK x 32, fp32) is
+// kept in shared memory; S_in of every segment is written out, then S <- M_g S + S_loc,g with M_g
+// staged in shared memory first (coalesced 8-byte loads; row stride DK + 2 so that the rows the
+// threads of a warp read at one k fall on different banks).
+template <int DK>
 __global__ void __launch_bounds__(256) seg_combine_kernel(const float *__restrict__ M, const float *__restrict__ Sloc,
                                                           const float *__restrict__ S0, float *__restrict__ Sin,
-                                                          float *__restrict__ S_final, int G, int H, int dk, int dv)
+                                                          float *__restrict__ S_final, int G, int H, int dv)
 {
-    extern __shared__ float sh[];  // two dk x 32 buffers
+    constexpr int LDM = DK + 2;
+    constexpr int PER = DK * 32 / 256;  // outputs per thread, all in one row: 8 (DK = 64) or 16 (DK = 128)
+    extern __shared__ float sh[];       // M_g [DK][LDM], then two DK x 32 state buffers
+    float *Ms = sh, *cur = sh + DK * LDM, *nxt = cur + DK * 32;
     const int cb = blockIdx.x, h = blockIdx.y, b = blockIdx.z, t = threadIdx.x;
     const int c0 = cb * 32;
-    float *cur = sh, *nxt = sh + dk * 32;
-    const size_t st0 = ((size_t)b * H + h) * dk * dv;
-    for (int i = t; i < dk * 32; i += 256) {
+    const size_t st0 = ((size_t)b * H + h) * DK * dv;
+    for (int i = t; i < DK * 32; i += 256) {
         const int r = i / 32, c = i % 32;
         cur[i] = S0 ? S0[st0 + (size_t)r * dv + c0 + c] : 0.f;
     }
-    __syncthreads();
-    const int per = dk * 32 / 256;  // outputs per thread, all in one row: 8 (dk = 64) or 16 (dk = 128)
-    const int first = t * per, r = first / 32, cc = first % 32;
+    const int first = t * PER, r = first / 32, cc = first % 32;
     for (int g = 0; g < G; ++g) {
         const size_t seg = (size_t)b * G + g;
-        const size_t sv = (seg * H + h) * (size_t)dk * dv;
-        const size_t smi = (seg * H + h) * (size_t)dk * dk;
-        for (int i = t; i < dk * 32; i += 256) {
+        const size_t sv = (seg * H + h) * (size_t)DK * dv;
+        const float2 *mg = reinterpret_cast<const float2 *>(M + (seg * H + h) * (size_t)DK * DK);
+        for (int i = t; i < DK * DK / 2; i += 256) {
+            const int rr = (2 * i) / DK, k = (2 * i) % DK;
+            *reinterpret_cast<float2 *>(&Ms[rr * LDM + k]) = mg[i];
+        }
+        __syncthreads();  // M_g staged; cur complete (previous step or the initial load)
+        for (int i = t; i < DK * 32; i += 256) {
             const int rr = i / 32, c = i % 32;
             Sin[sv + (size_t)rr * dv + c0 + c] = cur[i];
         }
-        float acc[16];
+        float acc[PER];
 #pragma unroll
-        for (int e = 0; e < 16; ++e) acc[e] = 0.f;
-        const float *mrow = M + smi + (size_t)r * dk;
-        for (int k = 0; k < dk; ++k) {
-            const float m = mrow[k];
+        for (int e = 0; e < PER; ++e) acc[e] = 0.f;
+#pragma unroll 8
+        for (int k = 0; k < DK; ++k) {
+            const float m = Ms[r * LDM + k];
 #pragma unroll
-            for (int e = 0; e < 16; ++e)
-                if (e < per) acc[e] = fmaf(m, cur[k * 32 + cc + e], acc[e]);
+            for (int e = 0; e < PER; ++e) acc[e] = fmaf(m, cur[k * 32 + cc + e], acc[e]);
         }
 #pragma unroll
-        for (int e = 0; e < 16; ++e)
-            if (e < per) nxt[r * 32 + cc + e] = acc[e] + Sloc[sv + (size_t)r * dv + c0 + cc + e];
-        __syncthreads();
+        for (int e = 0; e < PER; ++e) nxt[r * 32 + cc + e] = acc[e] + Sloc[sv + (size_t)r * dv + c0 + cc + e];
+        __syncthreads();  // every read of Ms and cur done
         float *tmp = cur;
         cur = nxt;
         nxt = tmp;
     }
     if (S_final) {
-        for (int i = t; i < dk * 32; i += 256) {
+        for (int i = t; i < DK * 32; i += 256) {
             const int rr = i / 32, c = i % 32;
             S_final[st0 + (size_t)rr * dv + c0 + c] = cur[i];
         }
@@ -1211,9 +1217,11 @@ cudaError_t run_chunk(const ChunkArgs &a, cudaStream_t st)
                           st);
     if (e != cudaSuccess) return e;
     // pass B: segment scan of the states
-    const size_t shm = 2 * (size_t)DK * 32 * sizeof(float);
-    seg_combine_kernel<<<dim3(DV / 32, a.H, a.B), 256, shm, st>>>(w.M, w.Sloc, a.S0, w.Sin, a.S_final, p.G,
-                                                                  a.H, DK, DV);
+    const int shm = (DK * (DK + 2) + 2 * DK * 32) * (int)sizeof(float);
+    e = cudaFuncSetAttribute(seg_combine_kernel<DK>, cudaFuncAttributeMaxDynamicSharedMemorySize, shm);
+    if (e != cudaSuccess) return e;
+    seg_combine_kernel<DK><<<dim3(DV / 32, a.H, a.B), 256, shm, st>>>(w.M, w.Sloc, a.S0, w.Sin, a.S_final, p.G,
+                                                                      a.H, DV);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     // pass C: outputs of every segment from its entry state
