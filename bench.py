@@ -538,9 +538,9 @@ def backward_numbers(gdn, d, steps, warmup, flush, stream, peaks):
     ms_b = _time_loop(call, steps, warmup, flush, stream)
     # bytes per token-head: q, k, v, dout (bf16) and gates in; dq, dk, dv (fp32) and two gate grads out
     by_b = 393216 * (4 * 64 * 2 + 8 + 3 * 64 * 4 + 8)
-    # products per (chunk, head): 9 (prep) + 22 (grads) + 1 in each scan, each 2 * 64^3 flops in
+    # products per (chunk, head): 8 (prep) + 20 (grads) + 1 in each scan, each 2 * 64^3 flops in
     # fp32; the tensor cores execute three tf32 products for each
-    fl_b = 6144 * 33 * 2 * 64 ** 3
+    fl_b = 6144 * 30 * 2 * 64 ** 3
     tf32_peak = peaks["bf16_tflops"] * TF32_PER_BF16
     return {"workload": "hybrid_lm backward: dq, dk, dv, dlog_alpha, dbeta (fp32) from dout",
             "ms": round(ms_b, 6), "tokens_per_s": round(32768 / (ms_b * 1e-3), 1),

@@ -425,15 +425,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     mm<false, false>(Tm, K, t, [&](int r, int m, float x, int) { W[sw(r, m)] = x; }, bg);
     mm<false, false>(Tm, V, t, [&](int r, int j, float x, int) { Ut[sw(r, j)] = x; }, g.bet);
-    mm<true, false>(P, dO, t, [&](int i, int j, float x, int) { A[sw(i, j)] = x; });  // Y = P^T dO (A is free)
     __syncthreads();
     const size_t base = ((size_t)e * H + h) * (size_t)(N * N);
     const float gC = g.gam[N - 1];
     mm<true, false>(K, W, t, [&](int m, int n2, float x, int) { Mo[base + m * N + n2] = (m == n2 ? gC : 0.f) - x; }, g.lam);
     mm<true, false>(K, Ut, t, [&](int m, int j, float x, int) { Bo[base + m * N + j] = x; }, g.lam);
-    mm<true, false>(Q, dO, t, [&](int m, int j, float x, int) { Tm[sw(m, j)] = x; }, g.gam);  // T is free
+    // R = (Q^T diag(gam) - W^T P^T) dO = X^T dO with X = diag(gam) Q - P W (into A, free since the solve)
+    mm<false, false>(P, W, t, [&](int r, int m, float x, int) { A[sw(r, m)] = g.gam[r] * Q[sw(r, m)] - x; });
     __syncthreads();
-    mm<true, false>(W, A, t, [&](int m, int j, float x, int) { Ro[base + m * N + j] = Tm[sw(m, j)] - x; });
+    mm<true, false>(A, dO, t, [&](int m, int j, float x, int) { Ro[base + m * N + j] = x; });
 }
 
 // Number of chunks of sequence s and the table index of its first chunk.
@@ -625,9 +625,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         pc[u_col(u)] -= E;
     });
     mm<false, true>(U, dSp, t, [&](int i, int m, float x, int u) { ak[u] += g.lam[i] * x; });
-    mm<false, true>(dO, S, t, [&](int r, int m, float x, int u) { aq[u] += g.gam[r] * x; });
-    mm<false, false>(Q, S, t,
-                     [&](int r, int j, float x, int u) { pg[u_row(u)] = fmaf(dO[sw(r, j)], x, pg[u_row(u)]); });
+    // dQ += diag(gam) dO S^T, and d gam_r (O1) = sum_j dO_rj (Q S)_rj = sum_m Q_rm (dO S^T)_rm
+    mm<false, true>(dO, S, t, [&](int r, int m, float x, int u) {
+        aq[u] += g.gam[r] * x;
+        pg[u_row(u)] = fmaf(Q[sw(r, m)], x, pg[u_row(u)]);
+    });
     __syncthreads();
     // dW = -dU S^T into U (U is no longer needed)
     mm<false, true>(dU, S, t, [&](int r, int m, float x, int) { U[sw(r, m)] = -x; });
@@ -666,9 +668,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         U[sw(r, i)] = d;
     });
     __syncthreads();
-    // dK += D K + D^T K + D2^T Q;  dQ += D2 K
-    mm<false, false>(U, K, t, [&](int, int, float x, int u) { ak[u] += x; });
-    mm<true, false>(U, K, t, [&](int, int, float x, int u) { ak[u] += x; });
+    // D + D^T into dU (Z is no longer needed), so that D K + D^T K is one product
+    for (int idx = t; idx < N * N; idx += kThreads) {
+        const int r = idx >> 6, i = idx & 63;
+        dU[sw(r, i)] = U[sw(r, i)] + U[sw(i, r)];
+    }
+    __syncthreads();
+    // dK += (D + D^T) K + D2^T Q;  dQ += D2 K
+    mm<false, false>(dU, K, t, [&](int, int, float x, int u) { ak[u] += x; });
     mm<true, false>(X1, Q, t, [&](int, int, float x, int u) { ak[u] += x; });
     mm<false, false>(X1, K, t, [&](int, int, float x, int u) { aq[u] += x; });
     // the partial sums over the block (X2 is free scratch now: its last reader is two barriers back)
