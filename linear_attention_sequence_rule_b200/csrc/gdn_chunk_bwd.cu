@@ -11,7 +11,7 @@
 //   S'  = M S + Bm,              M  = gam_C I - K^T diag(lam) W,   Bm = K^T diag(lam) U~
 //   dS  = M^T dS' + R,           R  = (Q^T diag(gam) - W^T P^T) dO
 // Four kernels:
-//   bwd_prep   (chunk x head, parallel)  : T, W, U~, P  ->  M, Bm, R
+//   bwd_prep   (chunk x head, parallel)  : T, W, U~, P  ->  M, Bm, R, and T for bwd_grads
 //   bwd_scan<false> (sequence x head)    : S_c for every chunk, from S0
 //   bwd_scan<true>  (sequence x head, reverse): dS at every chunk's end, from dS_final; dS0
 //   bwd_grads  (chunk x head, parallel)  : with S_c and dS_{c+1}, every input gradient of the chunk
@@ -394,7 +394,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     bwd_prep(const TIn *__restrict__ q, const TIn *__restrict__ k, const TIn *__restrict__ v,
              const float *__restrict__ log_alpha, const float *__restrict__ beta, const TIn *__restrict__ dout,
              const int32_t *__restrict__ cu, const int32_t *__restrict__ off, int nseq, int T, int H,
-             float *__restrict__ Mo, float *__restrict__ Bo, float *__restrict__ Ro)
+             float *__restrict__ Mo, float *__restrict__ Bo, float *__restrict__ Ro, float *__restrict__ Tw)
 {
     float *K = smf, *Q = K + MAT, *V = Q + MAT, *dO = V + MAT, *A = dO + MAT, *Tm = A + MAT, *W = Tm + MAT,
           *Ut = W + MAT, *P = Ut + MAT;
@@ -423,10 +423,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     unit_lower_inverse(A, Tm, t);
     __syncthreads();
+    const size_t base = ((size_t)e * H + h) * (size_t)(N * N);
+    mat_from_shared(Tw + base, Tm, t);  // T for the gradient kernel
     mm<false, false>(Tm, K, t, [&](int r, int m, float x, int) { W[sw(r, m)] = x; }, bg);
     mm<false, false>(Tm, V, t, [&](int r, int j, float x, int) { Ut[sw(r, j)] = x; }, g.bet);
     __syncthreads();
-    const size_t base = ((size_t)e * H + h) * (size_t)(N * N);
     const float gC = g.gam[N - 1];
     mm<true, false>(K, W, t, [&](int m, int n2, float x, int) { Mo[base + m * N + n2] = (m == n2 ? gC : 0.f) - x; }, g.lam);
     mm<true, false>(K, Ut, t, [&](int m, int j, float x, int) { Bo[base + m * N + j] = x; }, g.lam);
@@ -542,7 +543,8 @@ template <typename TIn>
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_grads(const TIn *__restrict__ q, const TIn *__restrict__ k, const TIn *__restrict__ v,
               const float *__restrict__ log_alpha, const float *__restrict__ beta, const TIn *__restrict__ dout,
-              const float *__restrict__ Sc, const float *__restrict__ dSn, const int32_t *__restrict__ cu,
+              const float *__restrict__ Sc, const float *__restrict__ dSn, const float *__restrict__ Tw,
+              const int32_t *__restrict__ cu,
               const int32_t *__restrict__ off, int nseq, int T, int H, float *__restrict__ dq,
               float *__restrict__ dk, float *__restrict__ dv, float *__restrict__ dla, float *__restrict__ dbe)
 {
@@ -563,6 +565,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         td.fetch(dout, c, H, h, t);
         mat_to_shared(S, Sc + base, t);
         mat_to_shared(dSp, dSn + base, t);
+        mat_to_shared(Tm, Tw + base, t);  // T = (I + A)^{-1}, from the prep kernel
         tk.put(K, t);
         tq.put(Q, t);
         tv.put(V, t);
@@ -585,12 +588,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     mm<false, true>(Q, K, t, [&](int r, int i, float x, int) { QK[sw(r, i)] = x; });
     mm<false, false>(K, dSp, t, [&](int i, int m, float x, int) { X2[sw(i, m)] = x; });  // K dS'
     __syncthreads();
-    // A (strictly lower) transposed in dU for the solve; P in X1; d gam_C = <S, dS'>
+    // P in X1; d gam_C = <S, dS'>
     {
         float part = 0.f;
         for (int idx = t; idx < N * N; idx += kThreads) {
             const int r = idx >> 6, i = idx & 63;
-            dU[sw(r, i)] = r < i ? g.bet[i] * decay(g, i, r) * KK[sw(r, i)] : 0.f;  // A(i, r), KK symmetric
             X1[sw(r, i)] = decay(g, r, i) * QK[sw(r, i)];
             part = fmaf(S[sw(r, i)], dSp[sw(r, i)], part);
         }
@@ -598,8 +600,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
         if ((t & 31) == 0) atomicAdd(dgC, part);
     }
-    __syncthreads();
-    unit_lower_inverse(dU, Tm, t);
     __syncthreads();
     // U~ into U, W into dU (A is no longer needed)
     mm<false, false>(Tm, V, t, [&](int r, int j, float x, int) { U[sw(r, j)] = x; }, g.bet);
@@ -783,6 +783,7 @@ cudaError_t run_bwd(const BwdArgs &a, cudaStream_t st)
     float *Ro = reinterpret_cast<float *>(w + 2 * align256b(mats));
     float *Sc = reinterpret_cast<float *>(w + 3 * align256b(mats));
     float *dSn = reinterpret_cast<float *>(w + 4 * align256b(mats));
+    float *Tw = reinterpret_cast<float *>(w + 5 * align256b(mats));
     const int32_t *offp = varlen ? off : nullptr;
     if (varlen) {
         bwd_offsets<<<1, 1, 0, st>>>(a.cu_seqlens, a.B, off);
@@ -804,10 +805,10 @@ cudaError_t run_bwd(const BwdArgs &a, cudaStream_t st)
     if (e != cudaSuccess) return e;
     const dim3 gc((unsigned)chunks, a.H), gs(a.H, a.B);
     bwd_prep<TIn><<<gc, kThreads, smem_prep, st>>>(q, k, v, a.log_alpha, a.beta, dout, a.cu_seqlens, offp, a.B, a.T,
-                                                   a.H, Mo, Bo, Ro);
+                                                   a.H, Mo, Bo, Ro, Tw);
     bwd_scan<false><<<gs, kThreads, smem_scan, st>>>(Mo, Bo, a.S0, a.cu_seqlens, offp, a.T, a.H, Sc, nullptr);
     bwd_scan<true><<<gs, kThreads, smem_scan, st>>>(Mo, Ro, a.dS_final, a.cu_seqlens, offp, a.T, a.H, dSn, a.dS0);
-    bwd_grads<TIn><<<gc, kThreads, smem_grads, st>>>(q, k, v, a.log_alpha, a.beta, dout, Sc, dSn, a.cu_seqlens, offp,
+    bwd_grads<TIn><<<gc, kThreads, smem_grads, st>>>(q, k, v, a.log_alpha, a.beta, dout, Sc, dSn, Tw, a.cu_seqlens, offp,
                                                      a.B, a.T, a.H, a.dq, a.dk, a.dv, a.dlog_alpha, a.dbeta);
     return cudaGetLastError();
 }
@@ -817,7 +818,7 @@ cudaError_t run_bwd(const BwdArgs &a, cudaStream_t st)
 size_t chunk_bwd_workspace_bytes(int B, int T, int H, int varlen)
 {
     const size_t mats = (size_t)bwd_chunks(B, T, varlen) * H * N * N * sizeof(float);
-    return align256b((size_t)(B + 1) * sizeof(int32_t)) + 5 * align256b(mats);
+    return align256b((size_t)(B + 1) * sizeof(int32_t)) + 6 * align256b(mats);
 }
 
 cudaError_t launch_chunk_bwd(const BwdArgs &a, cudaStream_t stream)
