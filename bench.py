@@ -538,9 +538,11 @@ def backward_numbers(gdn, d, steps, warmup, flush, stream, peaks):
     ms_b = _time_loop(call, steps, warmup, flush, stream)
     # bytes per token-head: q, k, v, dout (bf16) and gates in; dq, dk, dv (fp32) and two gate grads out
     by_b = 393216 * (4 * 64 * 2 + 8 + 3 * 64 * 4 + 8)
-    # products per (chunk, head): 8 (prep) + 20 (grads) + 1 in each scan, each 2 * 64^3 flops in
-    # fp32; the tensor cores execute three tf32 products for each
-    fl_b = 6144 * 30 * 2 * 64 ** 3
+    # algorithmic work: the 26 distinct 64 x 64 x 64 products the chunk-form backward needs per
+    # (chunk, head), each counted once -- 8 forming T, W, U~, M, Bm, R; 1 in each scan; 16 for the
+    # gradients -- at 2 * 64^3 fp32 flops each (the gradient kernel's recomputed K K^T and Q K^T are
+    # not counted); the tensor cores execute three tf32 products for each
+    fl_b = 6144 * 26 * 2 * 64 ** 3
     tf32_peak = peaks["bf16_tflops"] * TF32_PER_BF16
     return {"workload": "hybrid_lm backward: dq, dk, dv, dlog_alpha, dbeta (fp32) from dout",
             "ms": round(ms_b, 6), "tokens_per_s": round(32768 / (ms_b * 1e-3), 1),

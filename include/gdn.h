@@ -235,7 +235,7 @@ GDN_API size_t gdn_phase_fwd_workspace_bytes(int B, int T, int H, int dk, int dv
  * parallel, two scans over each sequence's chunks give the entry states and exit gradients, and
  * every chunk's input gradients are then formed in parallel.  log_alpha = -inf (an exact reset)
  * gets dlog_alpha = 0.  Workspace: gdn_chunk_bwd_workspace_bytes(...) bytes, 256-byte aligned
- * (six 16 KB matrices per chunk and head).  Errors as gdn_chunk_fwd; other head sizes return
+ * (eight 16 KB matrices per chunk and head).  Errors as gdn_chunk_fwd; other head sizes return
  * GDN_ERR_UNSUPPORTED.
  */
 GDN_API int gdn_chunk_bwd(const void *q, const void *k, const void *v, const float *log_alpha,

@@ -11,7 +11,7 @@
 //   S'  = M S + Bm,              M  = gam_C I - K^T diag(lam) W,   Bm = K^T diag(lam) U~
 //   dS  = M^T dS' + R,           R  = (Q^T diag(gam) - W^T P^T) dO
 // Four kernels:
-//   bwd_prep   (chunk x head, parallel)  : T, W, U~, P  ->  M, Bm, R, and T for bwd_grads
+//   bwd_prep   (chunk x head, parallel)  : T, W, U~, P  ->  M, Bm, R, and T, W, U~ for bwd_grads
 //   bwd_scan<false> (sequence x head)    : S_c for every chunk, from S0
 //   bwd_scan<true>  (sequence x head, reverse): dS at every chunk's end, from dS_final; dS0
 //   bwd_grads  (chunk x head, parallel)  : with S_c and dS_{c+1}, every input gradient of the chunk
@@ -394,7 +394,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     bwd_prep(const TIn *__restrict__ q, const TIn *__restrict__ k, const TIn *__restrict__ v,
              const float *__restrict__ log_alpha, const float *__restrict__ beta, const TIn *__restrict__ dout,
              const int32_t *__restrict__ cu, const int32_t *__restrict__ off, int nseq, int T, int H,
-             float *__restrict__ Mo, float *__restrict__ Bo, float *__restrict__ Ro, float *__restrict__ Tw)
+             float *__restrict__ Mo, float *__restrict__ Bo, float *__restrict__ Ro, float *__restrict__ Tw,
+             float *__restrict__ Ww, float *__restrict__ Uw)
 {
     float *K = smf, *Q = K + MAT, *V = Q + MAT, *dO = V + MAT, *A = dO + MAT, *Tm = A + MAT, *W = Tm + MAT,
           *Ut = W + MAT, *P = Ut + MAT;
@@ -428,6 +429,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     mm<false, false>(Tm, K, t, [&](int r, int m, float x, int) { W[sw(r, m)] = x; }, bg);
     mm<false, false>(Tm, V, t, [&](int r, int j, float x, int) { Ut[sw(r, j)] = x; }, g.bet);
     __syncthreads();
+    mat_from_shared(Ww + base, W, t);  // W and U~ for the gradient kernel
+    mat_from_shared(Uw + base, Ut, t);
     const float gC = g.gam[N - 1];
     mm<true, false>(K, W, t, [&](int m, int n2, float x, int) { Mo[base + m * N + n2] = (m == n2 ? gC : 0.f) - x; }, g.lam);
     mm<true, false>(K, Ut, t, [&](int m, int j, float x, int) { Bo[base + m * N + j] = x; }, g.lam);
@@ -544,7 +547,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     bwd_grads(const TIn *__restrict__ q, const TIn *__restrict__ k, const TIn *__restrict__ v,
               const float *__restrict__ log_alpha, const float *__restrict__ beta, const TIn *__restrict__ dout,
               const float *__restrict__ Sc, const float *__restrict__ dSn, const float *__restrict__ Tw,
-              const int32_t *__restrict__ cu,
+              const float *__restrict__ Ww, const float *__restrict__ Uw, const int32_t *__restrict__ cu,
               const int32_t *__restrict__ off, int nseq, int T, int H, float *__restrict__ dq,
               float *__restrict__ dk, float *__restrict__ dv, float *__restrict__ dla, float *__restrict__ dbe)
 {
@@ -565,7 +568,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         td.fetch(dout, c, H, h, t);
         mat_to_shared(S, Sc + base, t);
         mat_to_shared(dSp, dSn + base, t);
-        mat_to_shared(Tm, Tw + base, t);  // T = (I + A)^{-1}, from the prep kernel
+        mat_to_shared(Tm, Tw + base, t);  // T = (I + A)^{-1}, W and U~ from the prep kernel
+        mat_to_shared(dU, Ww + base, t);
+        mat_to_shared(U, Uw + base, t);
         tk.put(K, t);
         tq.put(Q, t);
         tv.put(V, t);
@@ -601,11 +606,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if ((t & 31) == 0) atomicAdd(dgC, part);
     }
     __syncthreads();
-    // U~ into U, W into dU (A is no longer needed)
-    mm<false, false>(Tm, V, t, [&](int r, int j, float x, int) { U[sw(r, j)] = x; }, g.bet);
-    mm<false, false>(Tm, K, t, [&](int r, int m, float x, int) { dU[sw(r, m)] = x; }, bg);
-    __syncthreads();
-    // U = U~ - W S
+    // U = U~ - W S (U~ in U, W in dU, both loaded)
     mm<false, false>(dU, S, t, [&](int r, int j, float x, int) { U[sw(r, j)] -= x; });
     __syncthreads();
     // dU = P^T dO + diag(lam) K dS'; d lam_i = sum_j (K dS')_ij U_ij (the only term of d lam)
@@ -784,6 +785,8 @@ cudaError_t run_bwd(const BwdArgs &a, cudaStream_t st)
     float *Sc = reinterpret_cast<float *>(w + 3 * align256b(mats));
     float *dSn = reinterpret_cast<float *>(w + 4 * align256b(mats));
     float *Tw = reinterpret_cast<float *>(w + 5 * align256b(mats));
+    float *Ww = reinterpret_cast<float *>(w + 6 * align256b(mats));
+    float *Uw = reinterpret_cast<float *>(w + 7 * align256b(mats));
     const int32_t *offp = varlen ? off : nullptr;
     if (varlen) {
         bwd_offsets<<<1, 1, 0, st>>>(a.cu_seqlens, a.B, off);
@@ -805,10 +808,11 @@ cudaError_t run_bwd(const BwdArgs &a, cudaStream_t st)
     if (e != cudaSuccess) return e;
     const dim3 gc((unsigned)chunks, a.H), gs(a.H, a.B);
     bwd_prep<TIn><<<gc, kThreads, smem_prep, st>>>(q, k, v, a.log_alpha, a.beta, dout, a.cu_seqlens, offp, a.B, a.T,
-                                                   a.H, Mo, Bo, Ro, Tw);
+                                                   a.H, Mo, Bo, Ro, Tw, Ww, Uw);
     bwd_scan<false><<<gs, kThreads, smem_scan, st>>>(Mo, Bo, a.S0, a.cu_seqlens, offp, a.T, a.H, Sc, nullptr);
     bwd_scan<true><<<gs, kThreads, smem_scan, st>>>(Mo, Ro, a.dS_final, a.cu_seqlens, offp, a.T, a.H, dSn, a.dS0);
-    bwd_grads<TIn><<<gc, kThreads, smem_grads, st>>>(q, k, v, a.log_alpha, a.beta, dout, Sc, dSn, Tw, a.cu_seqlens, offp,
+    bwd_grads<TIn><<<gc, kThreads, smem_grads, st>>>(q, k, v, a.log_alpha, a.beta, dout, Sc, dSn, Tw, Ww, Uw,
+                                                     a.cu_seqlens, offp,
                                                      a.B, a.T, a.H, a.dq, a.dk, a.dv, a.dlog_alpha, a.dbeta);
     return cudaGetLastError();
 }
@@ -818,7 +822,7 @@ cudaError_t run_bwd(const BwdArgs &a, cudaStream_t st)
 size_t chunk_bwd_workspace_bytes(int B, int T, int H, int varlen)
 {
     const size_t mats = (size_t)bwd_chunks(B, T, varlen) * H * N * N * sizeof(float);
-    return align256b((size_t)(B + 1) * sizeof(int32_t)) + 6 * align256b(mats);
+    return align256b((size_t)(B + 1) * sizeof(int32_t)) + 8 * align256b(mats);
 }
 
 cudaError_t launch_chunk_bwd(const BwdArgs &a, cudaStream_t stream)
