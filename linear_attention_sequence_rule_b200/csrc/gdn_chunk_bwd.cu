@@ -12,8 +12,8 @@
 //   dS  = M^T dS' + R,           R  = (Q^T diag(gam) - W^T P^T) dO
 // Four kernels:
 //   bwd_prep   (chunk x head, parallel)  : T, W, U~, P  ->  M, Bm, R, and T, W, U~ for bwd_grads
-//   bwd_scan<false> (sequence x head)    : S_c for every chunk, from S0
-//   bwd_scan<true>  (sequence x head, reverse): dS at every chunk's end, from dS_final; dS0
+//   bwd_scans  (sequence x head x 2)     : forward, S_c for every chunk from S0; reverse, dS at every
+//                                          chunk's end from dS_final, and dS0 (one launch, both at once)
 //   bwd_grads  (chunk x head, parallel)  : with S_c and dS_{c+1}, every input gradient of the chunk
 // All matrices are 64 x 64 fp32 in shared memory (XOR-swizzled rows); 256 threads; a product
 // leaves each thread 16 results in the tensor cores' fragment layout (see mm_core).
@@ -452,17 +452,17 @@ __device__ __forceinline__ void seq_chunks(int s, const int32_t *cu, const int32
     }
 }
 
-// ---- bwd_scan: the chunk maps along one (sequence, head) ----------------------------------------
+// ---- the scans: the chunk maps along one (sequence, head) ---------------------------------------
 // Forward (REV = false): X = S0, then X <- M_c X + Bm_c; Xc[c] = the state entering chunk c.
 // Reverse (REV = true):  X = dS_final, then X <- M_c^T X + R_c over the chunks from the last;
 // Xc[c] = dL/dS at the end of chunk c, Xend = dS0.
 // X is double-buffered in shared memory, and so is M_c; chunk c + 2's M and additive term are
 // loaded into registers while chunk c is multiplied, so one barrier per chunk remains.
 template <bool REV>
-__global__ void __launch_bounds__(kThreads, 1)
-    bwd_scan(const float *__restrict__ Mo, const float *__restrict__ Add, const float *__restrict__ X0,
-             const int32_t *__restrict__ cu, const int32_t *__restrict__ off, int T, int H, float *__restrict__ Xc,
-             float *__restrict__ Xend)
+__device__ __forceinline__ void scan_body(const float *__restrict__ Mo, const float *__restrict__ Add,
+                                          const float *__restrict__ X0, const int32_t *__restrict__ cu,
+                                          const int32_t *__restrict__ off, int T, int H, float *__restrict__ Xc,
+                                          float *__restrict__ Xend)
 {
     // shared memory: X[2], then M[2]
     const int t = threadIdx.x, h = blockIdx.x, s = blockIdx.y;
@@ -531,6 +531,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncthreads();
     }
     if (Xend) mat_from_shared(Xend + st0, smf + (count & 1) * MAT, t);
+}
+
+// Both scans in one launch, blockIdx.z = 0 forward and 1 reverse: they are independent, and with
+// 64 KB of shared memory two CTAs share an SM, so all 2 B H chains run at once.
+__global__ void __launch_bounds__(kThreads, 2)
+    bwd_scans(const float *__restrict__ Mo, const float *__restrict__ Bo, const float *__restrict__ Ro,
+              const float *__restrict__ S0, const float *__restrict__ dS_final, const int32_t *__restrict__ cu,
+              const int32_t *__restrict__ off, int T, int H, float *__restrict__ Sc, float *__restrict__ dSn,
+              float *__restrict__ dS0)
+{
+    if (blockIdx.z == 0) scan_body<false>(Mo, Bo, S0, cu, off, T, H, Sc, nullptr);
+    else scan_body<true>(Mo, Ro, dS_final, cu, off, T, H, dSn, dS0);
 }
 
 // ---- bwd_grads: every input gradient of one (chunk, head) --------------------------------------
@@ -802,15 +814,13 @@ cudaError_t run_bwd(const BwdArgs &a, cudaStream_t st)
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(bwd_grads<TIn>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_grads);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(bwd_scan<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_scan);
+    e = cudaFuncSetAttribute(bwd_scans, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_scan);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(bwd_scan<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_scan);
-    if (e != cudaSuccess) return e;
-    const dim3 gc((unsigned)chunks, a.H), gs(a.H, a.B);
+    const dim3 gc((unsigned)chunks, a.H);
     bwd_prep<TIn><<<gc, kThreads, smem_prep, st>>>(q, k, v, a.log_alpha, a.beta, dout, a.cu_seqlens, offp, a.B, a.T,
                                                    a.H, Mo, Bo, Ro, Tw, Ww, Uw);
-    bwd_scan<false><<<gs, kThreads, smem_scan, st>>>(Mo, Bo, a.S0, a.cu_seqlens, offp, a.T, a.H, Sc, nullptr);
-    bwd_scan<true><<<gs, kThreads, smem_scan, st>>>(Mo, Ro, a.dS_final, a.cu_seqlens, offp, a.T, a.H, dSn, a.dS0);
+    bwd_scans<<<dim3(a.H, a.B, 2), kThreads, smem_scan, st>>>(Mo, Bo, Ro, a.S0, a.dS_final, a.cu_seqlens, offp, a.T,
+                                                             a.H, Sc, dSn, a.dS0);
     bwd_grads<TIn><<<gc, kThreads, smem_grads, st>>>(q, k, v, a.log_alpha, a.beta, dout, Sc, dSn, Tw, Ww, Uw,
                                                      a.cu_seqlens, offp,
                                                      a.B, a.T, a.H, a.dq, a.dk, a.dv, a.dlog_alpha, a.dbeta);
