@@ -61,3 +61,30 @@ def forward_fused(q_raw, k_raw, v, a_raw, b_raw, S0, a_scale, b_scale, cu_seqlen
     log_alpha, beta = gates(a_raw, b_raw, a_scale, b_scale)
     return oracle.forward(l2_normalize(q_raw), l2_normalize(k_raw), v, log_alpha, beta, S0,
                           cu_seqlens=cu_seqlens, units=units)
+
+
+def backward_fused(q_raw, k_raw, v, a_raw, b_raw, S0, dout, a_scale, b_scale, dS_final=None, cu_seqlens=None):
+    """fp64 gradients of ``forward_fused`` with respect to its raw inputs: the backward oracle on the
+    prologue's outputs, then the chain rule through the prologue, elementwise:
+      q = x / n with n = sqrt(|x|^2 + EPS):   dx = (dq - q (q . dq)) / n   (the same for k);
+      log alpha = -a_scale softplus(a):       da = -a_scale sigmoid(a) dlog_alpha;
+      beta = b_scale sigmoid(b):              db = b_scale sigmoid(b) (1 - sigmoid(b)) dbeta.
+    Returns (dq_raw, dk_raw, dv, da_raw, db_raw, dS0)."""
+    import oracle
+    xq, xk = _f64(q_raw), _f64(k_raw)
+    q, k = l2_normalize(xq), l2_normalize(xk)
+    log_alpha, beta = gates(a_raw, b_raw, a_scale, b_scale)
+    dq, dk, dv, dla, dbe, dS0 = oracle.backward(q, k, v, log_alpha, beta, S0, dout, dS_final,
+                                                cu_seqlens=cu_seqlens)
+
+    def through_norm(x, y, dy):
+        n = np.sqrt(np.sum(x * x, axis=-1, keepdims=True) + EPS)
+        return (dy - y * np.sum(y * dy, axis=-1, keepdims=True)) / n
+
+    a = _f64(a_raw)
+    sa = sigmoid(a)
+    sb = sigmoid(b_raw)
+    with np.errstate(invalid="ignore"):
+        da = np.where(np.isposinf(a), 0.0, -float(a_scale) * sa * dla)
+    db = float(b_scale) * sb * (1.0 - sb) * dbe
+    return through_norm(xq, q, dq), through_norm(xk, k, dk), dv, da, db, dS0
