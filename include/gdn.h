@@ -248,6 +248,29 @@ GDN_API int gdn_chunk_bwd(const void *q, const void *k, const void *v, const flo
 GDN_API size_t gdn_chunk_bwd_workspace_bytes(int B, int T, int H, int dk, int dv, int chunk, int varlen);
 
 /*
+ * gdn_chunk_bwd_fused -- gradients of gdn_chunk_fwd_fused with respect to its RAW inputs: given
+ * q_raw, k_raw, v (dtype), a_raw, b_raw (fp32), S0, a_scale, b_scale as passed to the forward,
+ * dout = dL/dout (dtype) and dS_final = dL/dS_final (NULL: zero), it writes fp32
+ *     dq_raw, dk_raw [.., H, 64], dv [.., H, 64], da_raw, db_raw [.., H], dS0 (NULL: not written).
+ * The prologue (rows divided by sqrt(|x|^2 + 1e-6), log alpha = -a_scale softplus(a),
+ * beta = b_scale sigmoid(b)) is formed again in fp32, the recurrence's backward runs in fp32 on
+ * it (as gdn_chunk_bwd with fp32 inputs), and the chain rule through the prologue follows:
+ * dx = (dq - q (q . dq)) / |x|_eps, da = -a_scale sigmoid(a) dlog_alpha (0 at a = +inf),
+ * db = b_scale sigmoid(b) (1 - sigmoid(b)) dbeta.  dk = dv = 64, chunk = 64.  Workspace:
+ * gdn_chunk_bwd_fused_workspace_bytes(...) bytes of device memory, 256-byte aligned.  Errors as
+ * gdn_chunk_bwd; a_scale must be finite and >= 0, b_scale in [0, 2].
+ */
+GDN_API int gdn_chunk_bwd_fused(const void *q_raw, const void *k_raw, const void *v, const float *a_raw,
+                                const float *b_raw, const float *S0, const void *dout, const float *dS_final,
+                                float *dq_raw, float *dk_raw, float *dv, float *da_raw, float *db_raw, float *dS0,
+                                int B, int T, int H, int dk, int dv_, int chunk, const int32_t *cu_seqlens,
+                                int dtype, float a_scale, float b_scale, void *workspace, size_t workspace_bytes,
+                                void *stream);
+
+/* Workspace gdn_chunk_bwd_fused needs for these sizes; (size_t)-1 for sizes it rejects. */
+GDN_API size_t gdn_chunk_bwd_fused_workspace_bytes(int B, int T, int H, int dk, int dv, int chunk, int varlen);
+
+/*
  * gdn_decode_step -- one generation step: every (n, h) state takes exactly one token, in place
  * (Sykra README, "Architectural Highlights" and "Computational Complexity": an O(d^2) update of
  * a fixed d x d state per token).  With r = S^T k, s = S^T q (both from the state before the

@@ -8,7 +8,7 @@ PyTorch provides device memory and streams.  The binding has two layers:
   ``gdn_status_string``, ``gdn_last_error``, ``gdn_version`` -- the C-ABI entry points of
   ``include/gdn.h`` with the same names and arguments (pointers as Python ints);
 * ``chunk_fwd``, ``chunk_fwd_host``, ``chunk_fwd_fused``, ``chunk_fwd_gva``, ``chunk_bwd``,
-  ``phase_fwd``, ``decode_step`` and ``decode_step_gva`` --
+  ``chunk_bwd_fused``, ``phase_fwd``, ``decode_step`` and ``decode_step_gva`` --
   the same calls taking torch tensors; they check shapes,
   devices and dtypes, allocate outputs with torch when none are given, and raise ``GdnError``
   on a non-zero status.
@@ -28,6 +28,7 @@ __all__ = [
     "gdn_chunk_fwd", "gdn_chunk_fwd_noalloc", "gdn_chunk_fwd_fused", "gdn_chunk_fwd_gva",
     "gdn_chunk_fwd_host", "gdn_chunk_fwd_host_workspace_bytes", "chunk_fwd_host",
     "gdn_phase_fwd", "gdn_phase_fwd_workspace_bytes", "phase_fwd",
+    "gdn_chunk_bwd_fused", "gdn_chunk_bwd_fused_workspace_bytes", "chunk_bwd_fused",
     "gdn_decode_step", "gdn_decode_step_gva", "gdn_chunk_bwd", "gdn_chunk_bwd_workspace_bytes", "gdn_chunk_fwd_workspace_bytes", "gdn_status_string",
     "gdn_last_error", "gdn_version", "gdn_device_status", "device_status", "chunk_fwd", "chunk_fwd_fused",
     "chunk_fwd_gva", "chunk_bwd", "decode_step", "decode_step_gva", "workspace_bytes",
@@ -65,6 +66,10 @@ _lib.gdn_decode_step_gva.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, 
 _lib.gdn_decode_step_gva.restype = _i
 _lib.gdn_chunk_bwd.argtypes = [_vp] * 14 + [_i] * 6 + [_vp, _i, _vp, _sz, _vp]
 _lib.gdn_chunk_bwd.restype = _i
+_lib.gdn_chunk_bwd_fused.argtypes = [_vp] * 14 + [_i] * 6 + [_vp, _i, ctypes.c_float, ctypes.c_float, _vp, _sz, _vp]
+_lib.gdn_chunk_bwd_fused.restype = _i
+_lib.gdn_chunk_bwd_fused_workspace_bytes.argtypes = [_i] * 7
+_lib.gdn_chunk_bwd_fused_workspace_bytes.restype = _sz
 _lib.gdn_chunk_bwd_workspace_bytes.argtypes = [_i] * 7
 _lib.gdn_chunk_bwd_workspace_bytes.restype = _sz
 _lib.gdn_chunk_fwd_noalloc.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i,
@@ -467,6 +472,61 @@ def chunk_bwd(q, k, v, log_alpha, beta, dout, S0=None, dS_final=None, cu_seqlens
     if rc != GDN_OK:
         raise GdnError(rc, gdn_last_error())
     return dq, dkk, dvv, dla, dbe, dS0
+
+
+def gdn_chunk_bwd_fused(q_raw, k_raw, v, a_raw, b_raw, S0, dout, dS_final, dq_raw, dk_raw, dv, da_raw, db_raw,
+                        dS0, B, T, H, dk, dv_, chunk, cu_seqlens, dtype, a_scale, b_scale, workspace,
+                        workspace_bytes, stream) -> int:
+    return _lib.gdn_chunk_bwd_fused(q_raw, k_raw, v, a_raw, b_raw, S0, dout, dS_final, dq_raw, dk_raw, dv, da_raw,
+                                    db_raw, dS0, B, T, H, dk, dv_, chunk, cu_seqlens, dtype, a_scale, b_scale,
+                                    workspace, workspace_bytes, stream)
+
+
+def gdn_chunk_bwd_fused_workspace_bytes(B, T, H, dk, dv, chunk, varlen) -> int:
+    return _lib.gdn_chunk_bwd_fused_workspace_bytes(B, T, H, dk, dv, chunk, varlen)
+
+
+def chunk_bwd_fused(q_raw, k_raw, v, a_raw, b_raw, dout, a_scale, b_scale, S0=None, dS_final=None,
+                    cu_seqlens=None, want_dS0=True, workspace=None, chunk=64, stream=None):
+    """Gradients of ``chunk_fwd_fused`` with respect to its raw inputs (dk = dv = 64): returns fp32
+    (dq_raw, dk_raw, dv, da_raw, db_raw, dS0 or None)."""
+    dt = q_raw.dtype
+    if dt not in _DT:
+        raise ValueError(f"unsupported dtype {dt}")
+    dev = q_raw.device
+    if cu_seqlens is not None:
+        T, H, dk = q_raw.shape
+        B = cu_seqlens.shape[0] - 1
+        lead = (T,)
+        _need(cu_seqlens, "cu_seqlens", torch.int32, (B + 1,), dev)
+    else:
+        B, T, H, dk = q_raw.shape
+        lead = (B, T)
+    dv = v.shape[-1]
+    for name, x, shp in (("q_raw", q_raw, (*lead, H, dk)), ("k_raw", k_raw, (*lead, H, dk)),
+                         ("v", v, (*lead, H, dv)), ("dout", dout, (*lead, H, dv))):
+        _need(x, name, dt, shp, dev)
+    _need(a_raw, "a_raw", torch.float32, (*lead, H), dev)
+    _need(b_raw, "b_raw", torch.float32, (*lead, H), dev)
+    for name, x in (("S0", S0), ("dS_final", dS_final)):
+        if x is not None:
+            _need(x, name, torch.float32, (B, H, dk, dv), dev)
+    f32 = dict(dtype=torch.float32, device=dev)
+    dq, dkk, dvv = torch.empty((*lead, H, dk), **f32), torch.empty((*lead, H, dk), **f32), torch.empty((*lead, H, dv), **f32)
+    da, db = torch.empty((*lead, H), **f32), torch.empty((*lead, H), **f32)
+    dS0 = torch.empty((B, H, dk, dv), **f32) if want_dS0 else None
+    need = gdn_chunk_bwd_fused_workspace_bytes(B, T, H, dk, dv, chunk, int(cu_seqlens is not None))
+    if need == ctypes.c_size_t(-1).value:
+        raise GdnError(GDN_ERR_UNSUPPORTED, f"gdn_chunk_bwd_fused does not take dk={dk} dv={dv} chunk={chunk}")
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    rc = gdn_chunk_bwd_fused(_ptr(q_raw), _ptr(k_raw), _ptr(v), _ptr(a_raw), _ptr(b_raw), _ptr(S0), _ptr(dout),
+                             _ptr(dS_final), _ptr(dq), _ptr(dkk), _ptr(dvv), _ptr(da), _ptr(db), _ptr(dS0), B, T, H,
+                             dk, dv, chunk, _ptr(cu_seqlens), _DT[dt], float(a_scale), float(b_scale),
+                             _ptr(workspace), workspace.numel() * workspace.element_size(), _stream_ptr(stream))
+    if rc != GDN_OK:
+        raise GdnError(rc, gdn_last_error())
+    return dq, dkk, dvv, da, db, dS0
 
 
 def decode_step_gva(q, k, v, log_alpha, beta, S, out=None, stream=None):

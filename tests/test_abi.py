@@ -214,3 +214,21 @@ def test_phase_entry_rejects_before_any_launch():
     n = gdn.gdn_phase_fwd_workspace_bytes(2, 64, 3, 32, 64, 0, gdn.GDN_DTYPE_BF16)
     token_heads = 2 * 64 * 3
     assert n >= token_heads * (2 * 64 * 2 + 2 * 64 * 2 + 64 * 2 + 4)
+
+
+def test_fused_backward_rejects_before_any_launch():
+    a = dict(q_raw=FAKE, k_raw=FAKE, v=FAKE, a_raw=FAKE, b_raw=FAKE, S0=None, dout=FAKE, dS_final=None, dq_raw=FAKE,
+             dk_raw=FAKE, dv=FAKE, da_raw=FAKE, db_raw=FAKE, dS0=None, B=1, T=64, H=1, dk=64, dv_=64, chunk=64,
+             cu_seqlens=None, dtype=gdn.GDN_DTYPE_BF16, a_scale=1.0, b_scale=1.0, workspace=FAKE * 256,
+             workspace_bytes=1 << 40, stream=None)
+
+    def call(**kw):
+        return gdn.gdn_chunk_bwd_fused(**dict(a, **kw))
+    assert call(dk=128) == gdn.GDN_ERR_UNSUPPORTED
+    assert call(dtype=9) == gdn.GDN_ERR_UNSUPPORTED
+    assert call(b_scale=2.5) == gdn.GDN_ERR_INVALID_ARGUMENT
+    assert call(a_scale=-1.0) == gdn.GDN_ERR_INVALID_ARGUMENT
+    assert call(db_raw=None) == gdn.GDN_ERR_INVALID_ARGUMENT
+    assert call(dout=FAKE + 4) == gdn.GDN_ERR_INVALID_ARGUMENT
+    assert call(workspace=None) == gdn.GDN_ERR_WORKSPACE
+    assert gdn.gdn_chunk_bwd_fused_workspace_bytes(1, 64, 1, 128, 64, 64, 0) == ctypes.c_size_t(-1).value
