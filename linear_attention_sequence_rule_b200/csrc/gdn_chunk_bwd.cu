@@ -389,55 +389,63 @@ __device__ void unit_lower_inverse(const float *At, float *Tm, int t)
 }
 
 // ---- bwd_prep: per (chunk, head) the forward map (M, Bm) and the output term R ----------------
+// Six shared matrices, reused as their contents die, so that two CTAs share an SM:
+//   B0 K | B1 Q, then V, then Q again | B2 A^T, then W | B3 P | B4 T, then dO | B5 U~, then X.
 template <typename TIn>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, 2)
     bwd_prep(const TIn *__restrict__ q, const TIn *__restrict__ k, const TIn *__restrict__ v,
              const float *__restrict__ log_alpha, const float *__restrict__ beta, const TIn *__restrict__ dout,
              const int32_t *__restrict__ cu, const int32_t *__restrict__ off, int nseq, int T, int H,
              float *__restrict__ Mo, float *__restrict__ Bo, float *__restrict__ Ro, float *__restrict__ Tw,
              float *__restrict__ Ww, float *__restrict__ Uw)
 {
-    float *K = smf, *Q = K + MAT, *V = Q + MAT, *dO = V + MAT, *A = dO + MAT, *Tm = A + MAT, *W = Tm + MAT,
-          *Ut = W + MAT, *P = Ut + MAT;
-    Gates &g = *reinterpret_cast<Gates *>(P + MAT);
+    float *K = smf, *B1 = K + MAT, *B2 = B1 + MAT, *P = B2 + MAT, *B4 = P + MAT, *B5 = B4 + MAT;
+    Gates &g = *reinterpret_cast<Gates *>(B5 + MAT);
     float *bg = reinterpret_cast<float *>(&g + 1);  // beta gam
     const int t = threadIdx.x, h = blockIdx.y, e = blockIdx.x;
     const ChunkRef c = chunk_ref(e, cu, off, nseq, T);
     if (c.n == 0) return;
+    RowTile<TIn> tv;
     {
-        RowTile<TIn> tk, tq, tv, td;
+        RowTile<TIn> tk, tq;
         tk.fetch(k, c, H, h, t);
         tq.fetch(q, c, H, h, t);
         tv.fetch(v, c, H, h, t);
-        td.fetch(dout, c, H, h, t);
         tk.put(K, t);
-        tq.put(Q, t);
-        tv.put(V, t);
-        td.put(dO, t);
+        tq.put(B1, t);  // Q
     }
     chunk_gates<TIn>(g, log_alpha, beta, c, H, h, t);
     __syncthreads();
     if (t < N) bg[t] = g.bet[t] * g.gam[t];
     // A transposed: At(i, r) = b_r Gam_ri (K K^T)_ri for i < r (K K^T is symmetric)
-    mm<false, true>(K, K, t, [&](int i, int r, float x, int) { A[sw(i, r)] = i < r ? g.bet[r] * decay(g, r, i) * x : 0.f; });
-    mm<false, true>(Q, K, t, [&](int r, int i, float x, int) { P[sw(r, i)] = decay(g, r, i) * x; });
+    mm<false, true>(K, K, t, [&](int i, int r, float x, int) { B2[sw(i, r)] = i < r ? g.bet[r] * decay(g, r, i) * x : 0.f; });
+    mm<false, true>(B1, K, t, [&](int r, int i, float x, int) { P[sw(r, i)] = decay(g, r, i) * x; });
     __syncthreads();
-    unit_lower_inverse(A, Tm, t);
+    tv.put(B1, t);  // V over Q (Q comes back for X)
+    unit_lower_inverse(B2, B4, t);  // T in B4
     __syncthreads();
     const size_t base = ((size_t)e * H + h) * (size_t)(N * N);
-    mat_from_shared(Tw + base, Tm, t);  // T for the gradient kernel
-    mm<false, false>(Tm, K, t, [&](int r, int m, float x, int) { W[sw(r, m)] = x; }, bg);
-    mm<false, false>(Tm, V, t, [&](int r, int j, float x, int) { Ut[sw(r, j)] = x; }, g.bet);
+    mat_from_shared(Tw + base, B4, t);  // T for the gradient kernel
+    mm<false, false>(B4, K, t, [&](int r, int m, float x, int) { B2[sw(r, m)] = x; }, bg);       // W over A^T
+    mm<false, false>(B4, B1, t, [&](int r, int j, float x, int) { B5[sw(r, j)] = x; }, g.bet);   // U~
     __syncthreads();
-    mat_from_shared(Ww + base, W, t);  // W and U~ for the gradient kernel
-    mat_from_shared(Uw + base, Ut, t);
+    {
+        RowTile<TIn> tq, td;
+        tq.fetch(q, c, H, h, t);
+        td.fetch(dout, c, H, h, t);
+        mat_from_shared(Ww + base, B2, t);  // W and U~ for the gradient kernel
+        mat_from_shared(Uw + base, B5, t);
+        tq.put(B1, t);  // Q again, over V
+        td.put(B4, t);  // dO over T
+    }
     const float gC = g.gam[N - 1];
-    mm<true, false>(K, W, t, [&](int m, int n2, float x, int) { Mo[base + m * N + n2] = (m == n2 ? gC : 0.f) - x; }, g.lam);
-    mm<true, false>(K, Ut, t, [&](int m, int j, float x, int) { Bo[base + m * N + j] = x; }, g.lam);
-    // R = (Q^T diag(gam) - W^T P^T) dO = X^T dO with X = diag(gam) Q - P W (into A, free since the solve)
-    mm<false, false>(P, W, t, [&](int r, int m, float x, int) { A[sw(r, m)] = g.gam[r] * Q[sw(r, m)] - x; });
+    mm<true, false>(K, B2, t, [&](int m, int n2, float x, int) { Mo[base + m * N + n2] = (m == n2 ? gC : 0.f) - x; }, g.lam);
+    mm<true, false>(K, B5, t, [&](int m, int j, float x, int) { Bo[base + m * N + j] = x; }, g.lam);
     __syncthreads();
-    mm<true, false>(A, dO, t, [&](int m, int j, float x, int) { Ro[base + m * N + j] = x; });
+    // R = (Q^T diag(gam) - W^T P^T) dO = X^T dO with X = diag(gam) Q - P W (over U~)
+    mm<false, false>(P, B2, t, [&](int r, int m, float x, int) { B5[sw(r, m)] = g.gam[r] * B1[sw(r, m)] - x; });
+    __syncthreads();
+    mm<true, false>(B5, B4, t, [&](int m, int j, float x, int) { Ro[base + m * N + j] = x; });
 }
 
 // Number of chunks of sequence s and the table index of its first chunk.
@@ -807,7 +815,7 @@ cudaError_t run_bwd(const BwdArgs &a, cudaStream_t st)
     }
     const TIn *q = static_cast<const TIn *>(a.q), *k = static_cast<const TIn *>(a.k),
               *v = static_cast<const TIn *>(a.v), *dout = static_cast<const TIn *>(a.dout);
-    const int smem_prep = (9 * MAT) * (int)sizeof(float) + (int)sizeof(Gates) + N * (int)sizeof(float);
+    const int smem_prep = (6 * MAT) * (int)sizeof(float) + (int)sizeof(Gates) + N * (int)sizeof(float);
     const int smem_grads = (13 * MAT) * (int)sizeof(float) + (int)sizeof(Gates) + 6 * N * (int)sizeof(float);
     const int smem_scan = 4 * MAT * (int)sizeof(float);
     cudaError_t e = cudaFuncSetAttribute(bwd_prep<TIn>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_prep);
