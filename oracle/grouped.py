@@ -32,3 +32,17 @@ def decode_step_gva(q, k, v, log_alpha, beta, S):
     """q,k [N, Hk, dk]; v [N, Hv, dv]; gates [N, Hv]; S [N, Hv, dk, dv] (fp64, not modified)."""
     G = v.shape[-2] // q.shape[-2]
     return oracle.decode_step(_expand(q, G), _expand(k, G), v, log_alpha, beta, S)
+
+
+def backward_gva(q, k, v, log_alpha, beta, S0, dout, dS_final=None, cu_seqlens=None):
+    """fp64 gradients of ``forward_gva``: the backward oracle on the Hv heads with q/k repeated,
+    then dq, dk of each q/k head summed over the G value heads that read it (the chain rule of
+    the repeat).  Returns (dq, dk [.., Hk, dk], dv, dlog_alpha, dbeta [.., Hv], dS0)."""
+    Hk, Hv = q.shape[-2], v.shape[-2]
+    G = Hv // Hk
+    dq, dk, dv, dla, dbe, dS0 = oracle.backward(_expand(q, G), _expand(k, G), v, log_alpha, beta, S0, dout,
+                                                dS_final, cu_seqlens=cu_seqlens)
+    lead = dq.shape[:-2]
+    dq = dq.reshape(*lead, Hk, G, dq.shape[-1]).sum(axis=-2)
+    dk = dk.reshape(*lead, Hk, G, dk.shape[-1]).sum(axis=-2)
+    return dq, dk, dv, dla, dbe, dS0
