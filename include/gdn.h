@@ -248,6 +248,23 @@ GDN_API int gdn_chunk_bwd(const void *q, const void *k, const void *v, const flo
 GDN_API size_t gdn_chunk_bwd_workspace_bytes(int B, int T, int H, int dk, int dv, int chunk, int varlen);
 
 /*
+ * gdn_chunk_bwd_gva -- gdn_chunk_bwd with grouped value heads (see gdn_chunk_fwd_gva): q, k
+ * [.., Hk, 64]; v, dout [.., Hv, 64]; gates [.., Hv]; states [B, Hv, 64, 64]; value head h reads
+ * q/k head h / (Hv / Hk).  dq, dk [.., Hk, 64] are the sums over each q/k head's Hv / Hk value
+ * heads; dv, dlog_alpha, dbeta, dS0 stay per value head.  Workspace:
+ * gdn_chunk_bwd_gva_workspace_bytes(...) (gdn_chunk_bwd's plus per-value-head dq and dk).
+ */
+GDN_API int gdn_chunk_bwd_gva(const void *q, const void *k, const void *v, const float *log_alpha,
+                              const float *beta, const float *S0, const void *dout, const float *dS_final,
+                              float *dq, float *dk, float *dv, float *dlog_alpha, float *dbeta, float *dS0, int B,
+                              int T, int Hk, int Hv, int dk_, int dv_, int chunk, const int32_t *cu_seqlens,
+                              int dtype, void *workspace, size_t workspace_bytes, void *stream);
+
+/* Workspace gdn_chunk_bwd_gva needs for these sizes; (size_t)-1 for sizes it rejects. */
+GDN_API size_t gdn_chunk_bwd_gva_workspace_bytes(int B, int T, int Hk, int Hv, int dk, int dv, int chunk,
+                                                 int varlen);
+
+/*
  * gdn_chunk_bwd_fused -- gradients of gdn_chunk_fwd_fused with respect to its RAW inputs: given
  * q_raw, k_raw, v (dtype), a_raw, b_raw (fp32), S0, a_scale, b_scale as passed to the forward,
  * dout = dL/dout (dtype) and dS_final = dL/dS_final (NULL: zero), it writes fp32

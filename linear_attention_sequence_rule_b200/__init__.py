@@ -8,7 +8,7 @@ PyTorch provides device memory and streams.  The binding has two layers:
   ``gdn_status_string``, ``gdn_last_error``, ``gdn_version`` -- the C-ABI entry points of
   ``include/gdn.h`` with the same names and arguments (pointers as Python ints);
 * ``chunk_fwd``, ``chunk_fwd_host``, ``chunk_fwd_fused``, ``chunk_fwd_gva``, ``chunk_bwd``,
-  ``chunk_bwd_fused``, ``phase_fwd``, ``decode_step`` and ``decode_step_gva`` --
+  ``chunk_bwd_fused``, ``chunk_bwd_gva``, ``phase_fwd``, ``decode_step`` and ``decode_step_gva`` --
   the same calls taking torch tensors; they check shapes,
   devices and dtypes, allocate outputs with torch when none are given, and raise ``GdnError``
   on a non-zero status.
@@ -29,6 +29,7 @@ __all__ = [
     "gdn_chunk_fwd_host", "gdn_chunk_fwd_host_workspace_bytes", "chunk_fwd_host",
     "gdn_phase_fwd", "gdn_phase_fwd_workspace_bytes", "phase_fwd",
     "gdn_chunk_bwd_fused", "gdn_chunk_bwd_fused_workspace_bytes", "chunk_bwd_fused",
+    "gdn_chunk_bwd_gva", "gdn_chunk_bwd_gva_workspace_bytes", "chunk_bwd_gva",
     "gdn_decode_step", "gdn_decode_step_gva", "gdn_chunk_bwd", "gdn_chunk_bwd_workspace_bytes", "gdn_chunk_fwd_workspace_bytes", "gdn_status_string",
     "gdn_last_error", "gdn_version", "gdn_device_status", "device_status", "chunk_fwd", "chunk_fwd_fused",
     "chunk_fwd_gva", "chunk_bwd", "decode_step", "decode_step_gva", "workspace_bytes",
@@ -70,6 +71,10 @@ _lib.gdn_chunk_bwd_fused.argtypes = [_vp] * 14 + [_i] * 6 + [_vp, _i, ctypes.c_f
 _lib.gdn_chunk_bwd_fused.restype = _i
 _lib.gdn_chunk_bwd_fused_workspace_bytes.argtypes = [_i] * 7
 _lib.gdn_chunk_bwd_fused_workspace_bytes.restype = _sz
+_lib.gdn_chunk_bwd_gva.argtypes = [_vp] * 14 + [_i] * 7 + [_vp, _i, _vp, _sz, _vp]
+_lib.gdn_chunk_bwd_gva.restype = _i
+_lib.gdn_chunk_bwd_gva_workspace_bytes.argtypes = [_i] * 8
+_lib.gdn_chunk_bwd_gva_workspace_bytes.restype = _sz
 _lib.gdn_chunk_bwd_workspace_bytes.argtypes = [_i] * 7
 _lib.gdn_chunk_bwd_workspace_bytes.restype = _sz
 _lib.gdn_chunk_fwd_noalloc.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i,
@@ -469,6 +474,61 @@ def chunk_bwd(q, k, v, log_alpha, beta, dout, S0=None, dS_final=None, cu_seqlens
                        _ptr(dS_final), _ptr(dq), _ptr(dkk), _ptr(dvv), _ptr(dla), _ptr(dbe), _ptr(dS0), B, T,
                        H, dk, dv, chunk, _ptr(cu_seqlens), _DT[dt], _ptr(workspace),
                        workspace.numel() * workspace.element_size(), _stream_ptr(stream))
+    if rc != GDN_OK:
+        raise GdnError(rc, gdn_last_error())
+    return dq, dkk, dvv, dla, dbe, dS0
+
+
+def gdn_chunk_bwd_gva(q, k, v, log_alpha, beta, S0, dout, dS_final, dq, dk, dv, dlog_alpha, dbeta, dS0, B, T, Hk,
+                      Hv, dk_, dv_, chunk, cu_seqlens, dtype, workspace, workspace_bytes, stream) -> int:
+    return _lib.gdn_chunk_bwd_gva(q, k, v, log_alpha, beta, S0, dout, dS_final, dq, dk, dv, dlog_alpha, dbeta, dS0,
+                                  B, T, Hk, Hv, dk_, dv_, chunk, cu_seqlens, dtype, workspace, workspace_bytes,
+                                  stream)
+
+
+def gdn_chunk_bwd_gva_workspace_bytes(B, T, Hk, Hv, dk, dv, chunk, varlen) -> int:
+    return _lib.gdn_chunk_bwd_gva_workspace_bytes(B, T, Hk, Hv, dk, dv, chunk, varlen)
+
+
+def chunk_bwd_gva(q, k, v, log_alpha, beta, dout, S0=None, dS_final=None, cu_seqlens=None, want_dS0=True,
+                  workspace=None, chunk=64, stream=None):
+    """Gradients of ``chunk_fwd_gva`` (dk = dv = 64): q, k [.., Hk, 64]; v, dout [.., Hv, 64]; returns
+    fp32 (dq, dk [.., Hk, 64], dv, dlog_alpha, dbeta, dS0 or None), dq and dk summed over each q/k
+    head's value heads."""
+    dt = q.dtype
+    if dt not in _DT:
+        raise ValueError(f"unsupported dtype {dt}")
+    dev = q.device
+    if cu_seqlens is not None:
+        T, Hk, dk = q.shape
+        B = cu_seqlens.shape[0] - 1
+        lead = (T,)
+        _need(cu_seqlens, "cu_seqlens", torch.int32, (B + 1,), dev)
+    else:
+        B, T, Hk, dk = q.shape
+        lead = (B, T)
+    Hv, dv = v.shape[-2], v.shape[-1]
+    for name, x, shp in (("q", q, (*lead, Hk, dk)), ("k", k, (*lead, Hk, dk)), ("v", v, (*lead, Hv, dv)),
+                         ("dout", dout, (*lead, Hv, dv))):
+        _need(x, name, dt, shp, dev)
+    _need(log_alpha, "log_alpha", torch.float32, (*lead, Hv), dev)
+    _need(beta, "beta", torch.float32, (*lead, Hv), dev)
+    for name, x in (("S0", S0), ("dS_final", dS_final)):
+        if x is not None:
+            _need(x, name, torch.float32, (B, Hv, dk, dv), dev)
+    f32 = dict(dtype=torch.float32, device=dev)
+    dq, dkk, dvv = torch.empty((*lead, Hk, dk), **f32), torch.empty((*lead, Hk, dk), **f32), torch.empty((*lead, Hv, dv), **f32)
+    dla, dbe = torch.empty((*lead, Hv), **f32), torch.empty((*lead, Hv), **f32)
+    dS0 = torch.empty((B, Hv, dk, dv), **f32) if want_dS0 else None
+    need = gdn_chunk_bwd_gva_workspace_bytes(B, T, Hk, Hv, dk, dv, chunk, int(cu_seqlens is not None))
+    if need == ctypes.c_size_t(-1).value:
+        raise GdnError(GDN_ERR_UNSUPPORTED, f"gdn_chunk_bwd_gva does not take Hk={Hk} Hv={Hv} dk={dk} dv={dv}")
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    rc = gdn_chunk_bwd_gva(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(S0), _ptr(dout),
+                           _ptr(dS_final), _ptr(dq), _ptr(dkk), _ptr(dvv), _ptr(dla), _ptr(dbe), _ptr(dS0), B, T,
+                           Hk, Hv, dk, dv, chunk, _ptr(cu_seqlens), _DT[dt], _ptr(workspace),
+                           workspace.numel() * workspace.element_size(), _stream_ptr(stream))
     if rc != GDN_OK:
         raise GdnError(rc, gdn_last_error())
     return dq, dkk, dvv, dla, dbe, dS0

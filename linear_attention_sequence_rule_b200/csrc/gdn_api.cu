@@ -255,13 +255,22 @@ size_t gdn_chunk_bwd_workspace_bytes(int B, int T, int H, int dk, int dv, int ch
     return chunk_bwd_workspace_bytes(B, T, H, varlen);
 }
 
-int gdn_chunk_bwd(const void *q, const void *k, const void *v, const float *log_alpha, const float *beta,
-                  const float *S0, const void *dout, const float *dS_final, float *dq, float *dk, float *dv,
-                  float *dlog_alpha, float *dbeta, float *dS0, int B, int T, int H, int dk_, int dv_, int chunk,
-                  const int32_t *cu_seqlens, int dtype, void *workspace, size_t workspace_bytes, void *stream)
+size_t gdn_chunk_bwd_gva_workspace_bytes(int B, int T, int Hk, int Hv, int dk, int dv, int chunk, int varlen)
 {
-    g_last_error[0] = 0;
-    const char *fn = "gdn_chunk_bwd";
+    if (Hk < 1 || Hv < 1 || Hv % Hk != 0) return (size_t)-1;
+    if (dk != 64 || dv != 64 || chunk != 64 || B < 1 || T < 0 || (!varlen && T < 1)) return (size_t)-1;
+    return chunk_bwd_workspace_bytes(B, T, Hv, varlen, Hv / Hk);
+}
+
+namespace gdn {
+
+// Validation and launch shared by the plain (G = 1) and the grouped-value-head backward.
+static int chunk_bwd_common(const char *fn, const void *q, const void *k, const void *v, const float *log_alpha,
+                            const float *beta, const float *S0, const void *dout, const float *dS_final, float *dq,
+                            float *dk, float *dv, float *dlog_alpha, float *dbeta, float *dS0, int B, int T, int H,
+                            int G, int dk_, int dv_, int chunk, const int32_t *cu_seqlens, int dtype,
+                            void *workspace, size_t workspace_bytes, void *stream)
+{
     const int varlen = cu_seqlens != nullptr;
     int rc = check_chunk_shape(B, T, H, dk_, dv_, chunk, varlen, dtype);
     if (rc != GDN_OK) return rc;
@@ -274,15 +283,42 @@ int gdn_chunk_bwd(const void *q, const void *k, const void *v, const float *log_
                           cu_seqlens};
     for (const void *p : ptrs)
         if (p && !aligned16(p)) return fail(GDN_ERR_INVALID_ARGUMENT, "%s: pointer %p is not 16-byte aligned", fn, p);
-    const size_t need = chunk_bwd_workspace_bytes(B, T, H, varlen);
+    const size_t need = chunk_bwd_workspace_bytes(B, T, H, varlen, G);
     if (!workspace || workspace_bytes < need)
         return fail(GDN_ERR_WORKSPACE, "%s: workspace of %zu bytes needed, %zu given", fn, need,
                     workspace ? workspace_bytes : (size_t)0);
     if (reinterpret_cast<uintptr_t>(workspace) & 255u)
         return fail(GDN_ERR_INVALID_ARGUMENT, "%s: workspace must be 256-byte aligned", fn);
     BwdArgs a{q, k, v, log_alpha, beta, S0, dout, dS_final, dq, dk, dv, dlog_alpha, dbeta, dS0, cu_seqlens,
-              B, T, H, dtype, workspace};
+              B, T, H, dtype, workspace, G};
     cudaError_t e = launch_chunk_bwd(a, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, fn);
     return GDN_OK;
+}
+
+}  // namespace gdn
+
+int gdn_chunk_bwd(const void *q, const void *k, const void *v, const float *log_alpha, const float *beta,
+                  const float *S0, const void *dout, const float *dS_final, float *dq, float *dk, float *dv,
+                  float *dlog_alpha, float *dbeta, float *dS0, int B, int T, int H, int dk_, int dv_, int chunk,
+                  const int32_t *cu_seqlens, int dtype, void *workspace, size_t workspace_bytes, void *stream)
+{
+    g_last_error[0] = 0;
+    return chunk_bwd_common("gdn_chunk_bwd", q, k, v, log_alpha, beta, S0, dout, dS_final, dq, dk, dv, dlog_alpha,
+                            dbeta, dS0, B, T, H, 1, dk_, dv_, chunk, cu_seqlens, dtype, workspace, workspace_bytes,
+                            stream);
+}
+
+int gdn_chunk_bwd_gva(const void *q, const void *k, const void *v, const float *log_alpha, const float *beta,
+                      const float *S0, const void *dout, const float *dS_final, float *dq, float *dk, float *dv,
+                      float *dlog_alpha, float *dbeta, float *dS0, int B, int T, int Hk, int Hv, int dk_, int dv_,
+                      int chunk, const int32_t *cu_seqlens, int dtype, void *workspace, size_t workspace_bytes,
+                      void *stream)
+{
+    g_last_error[0] = 0;
+    const int rc = check_groups("gdn_chunk_bwd_gva", Hk, Hv);
+    if (rc != GDN_OK) return rc;
+    return chunk_bwd_common("gdn_chunk_bwd_gva", q, k, v, log_alpha, beta, S0, dout, dS_final, dq, dk, dv,
+                            dlog_alpha, dbeta, dS0, B, T, Hv, Hv / Hk, dk_, dv_, chunk, cu_seqlens, dtype, workspace,
+                            workspace_bytes, stream);
 }

@@ -395,7 +395,7 @@ template <typename TIn>
 __global__ void __launch_bounds__(kThreads, 2)
     bwd_prep(const TIn *__restrict__ q, const TIn *__restrict__ k, const TIn *__restrict__ v,
              const float *__restrict__ log_alpha, const float *__restrict__ beta, const TIn *__restrict__ dout,
-             const int32_t *__restrict__ cu, const int32_t *__restrict__ off, int nseq, int T, int H,
+             const int32_t *__restrict__ cu, const int32_t *__restrict__ off, int nseq, int T, int H, int G,
              float *__restrict__ Mo, float *__restrict__ Bo, float *__restrict__ Ro, float *__restrict__ Tw,
              float *__restrict__ Ww, float *__restrict__ Uw)
 {
@@ -405,11 +405,13 @@ __global__ void __launch_bounds__(kThreads, 2)
     const int t = threadIdx.x, h = blockIdx.y, e = blockIdx.x;
     const ChunkRef c = chunk_ref(e, cu, off, nseq, T);
     if (c.n == 0) return;
+    // grouped value heads: value head h reads q/k head h / G of H / G
+    const int Hq = G == 1 ? H : H / G, hq = G == 1 ? h : h / G;
     RowTile<TIn> tv;
     {
         RowTile<TIn> tk, tq;
-        tk.fetch(k, c, H, h, t);
-        tq.fetch(q, c, H, h, t);
+        tk.fetch(k, c, Hq, hq, t);
+        tq.fetch(q, c, Hq, hq, t);
         tv.fetch(v, c, H, h, t);
         tk.put(K, t);
         tq.put(B1, t);  // Q
@@ -431,7 +433,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     __syncthreads();
     {
         RowTile<TIn> tq, td;
-        tq.fetch(q, c, H, h, t);
+        tq.fetch(q, c, Hq, hq, t);
         td.fetch(dout, c, H, h, t);
         mat_from_shared(Ww + base, B2, t);  // W and U~ for the gradient kernel
         mat_from_shared(Uw + base, B5, t);
@@ -568,7 +570,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               const float *__restrict__ log_alpha, const float *__restrict__ beta, const TIn *__restrict__ dout,
               const float *__restrict__ Sc, const float *__restrict__ dSn, const float *__restrict__ Tw,
               const float *__restrict__ Ww, const float *__restrict__ Uw, const int32_t *__restrict__ cu,
-              const int32_t *__restrict__ off, int nseq, int T, int H, float *__restrict__ dq,
+              const int32_t *__restrict__ off, int nseq, int T, int H, int G, float *__restrict__ dq,
               float *__restrict__ dk, float *__restrict__ dv, float *__restrict__ dla, float *__restrict__ dbe)
 {
     float *K = smf, *Q = K + MAT, *V = Q + MAT, *dO = V + MAT, *S = dO + MAT, *dSp = S + MAT, *KK = dSp + MAT,
@@ -581,9 +583,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (c.n == 0) return;
     const size_t base = ((size_t)e * H + h) * (size_t)(N * N);
     {
+        // grouped value heads: value head h reads q/k head h / G of H / G (dq, dk per value head)
+        const int Hq = G == 1 ? H : H / G, hq = G == 1 ? h : h / G;
         RowTile<TIn> tk, tq, tv, td;
-        tk.fetch(k, c, H, h, t);
-        tq.fetch(q, c, H, h, t);
+        tk.fetch(k, c, Hq, hq, t);
+        tq.fetch(q, c, Hq, hq, t);
         tv.fetch(v, c, H, h, t);
         td.fetch(dout, c, H, h, t);
         mat_to_shared(S, Sc + base, t);
@@ -763,6 +767,24 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
+// Grouped value heads: dq, dk of q/k head j = the sum over its G value heads (rows of 64 fp32,
+// [rows, Hv, 64] -> [rows, Hv / G, 64]); one thread per output element.
+__global__ void bwd_group_sum(const float *__restrict__ gq, const float *__restrict__ gk, float *__restrict__ dq,
+                              float *__restrict__ dk, long out_elems, int G)
+{
+    const long i = (long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= out_elems) return;
+    const long row = i / N, col = i % N;  // row = token * Hk + j
+    const float *a = gq + row * G * N + col, *b = gk + row * G * N + col;
+    float sq = 0.f, sk = 0.f;
+    for (int u = 0; u < G; ++u) {
+        sq += a[u * N];
+        sk += b[u * N];
+    }
+    dq[i] = sq;
+    dk[i] = sk;
+}
+
 // chunk offsets of varlen sequences: off[s] = sum over s' < s of ceil(len / 64); off[nseq] = total
 __global__ void bwd_offsets(const int32_t *__restrict__ cu, int nseq, int32_t *__restrict__ off)
 {
@@ -807,6 +829,10 @@ cudaError_t run_bwd(const BwdArgs &a, cudaStream_t st)
     float *Tw = reinterpret_cast<float *>(w + 5 * align256b(mats));
     float *Ww = reinterpret_cast<float *>(w + 6 * align256b(mats));
     float *Uw = reinterpret_cast<float *>(w + 7 * align256b(mats));
+    // grouped value heads: per-value-head dq, dk here, summed per group at the end
+    const size_t rows = (varlen ? (size_t)a.T : (size_t)a.B * a.T) * a.H;
+    float *gq = a.G > 1 ? reinterpret_cast<float *>(w + 8 * align256b(mats)) : a.dq;
+    float *gk = a.G > 1 ? reinterpret_cast<float *>(w + 8 * align256b(mats) + align256b(rows * N * 4)) : a.dk;
     const int32_t *offp = varlen ? off : nullptr;
     if (varlen) {
         bwd_offsets<<<1, 1, 0, st>>>(a.cu_seqlens, a.B, off);
@@ -826,21 +852,31 @@ cudaError_t run_bwd(const BwdArgs &a, cudaStream_t st)
     if (e != cudaSuccess) return e;
     const dim3 gc((unsigned)chunks, a.H);
     bwd_prep<TIn><<<gc, kThreads, smem_prep, st>>>(q, k, v, a.log_alpha, a.beta, dout, a.cu_seqlens, offp, a.B, a.T,
-                                                   a.H, Mo, Bo, Ro, Tw, Ww, Uw);
+                                                   a.H, a.G, Mo, Bo, Ro, Tw, Ww, Uw);
     bwd_scans<<<dim3(a.H, a.B, 2), kThreads, smem_scan, st>>>(Mo, Bo, Ro, a.S0, a.dS_final, a.cu_seqlens, offp, a.T,
                                                              a.H, Sc, dSn, a.dS0);
     bwd_grads<TIn><<<gc, kThreads, smem_grads, st>>>(q, k, v, a.log_alpha, a.beta, dout, Sc, dSn, Tw, Ww, Uw,
-                                                     a.cu_seqlens, offp,
-                                                     a.B, a.T, a.H, a.dq, a.dk, a.dv, a.dlog_alpha, a.dbeta);
+                                                     a.cu_seqlens, offp, a.B, a.T, a.H, a.G, gq, gk, a.dv,
+                                                     a.dlog_alpha, a.dbeta);
+    if (a.G > 1) {
+        const long out_elems = (long)(rows / a.G) * N;
+        if (out_elems > 0)
+            bwd_group_sum<<<(unsigned)((out_elems + 255) / 256), 256, 0, st>>>(gq, gk, a.dq, a.dk, out_elems, a.G);
+    }
     return cudaGetLastError();
 }
 
 }  // namespace
 
-size_t chunk_bwd_workspace_bytes(int B, int T, int H, int varlen)
+size_t chunk_bwd_workspace_bytes(int B, int T, int H, int varlen, int G)
 {
     const size_t mats = (size_t)bwd_chunks(B, T, varlen) * H * N * N * sizeof(float);
-    return align256b((size_t)(B + 1) * sizeof(int32_t)) + 8 * align256b(mats);
+    size_t bytes = align256b((size_t)(B + 1) * sizeof(int32_t)) + 8 * align256b(mats);
+    if (G > 1) {  // per-value-head dq and dk before the group sums
+        const size_t rows = (varlen ? (size_t)T : (size_t)B * T) * H;
+        bytes += 2 * align256b(rows * N * 4);
+    }
+    return bytes;
 }
 
 cudaError_t launch_chunk_bwd(const BwdArgs &a, cudaStream_t stream)

@@ -54,10 +54,11 @@ struct BwdArgs {
     const float *dS_final;
     float *dq, *dk, *dv, *dlog_alpha, *dbeta, *dS0;
     const int32_t *cu_seqlens;
-    int B, T, H, dtype;
+    int B, T, H, dtype;  // H value heads
     void *workspace;
+    int G = 1;  // grouped value heads: H / G q/k heads, value head h reads q/k head h / G
 };
-size_t chunk_bwd_workspace_bytes(int B, int T, int H, int varlen);
+size_t chunk_bwd_workspace_bytes(int B, int T, int H, int varlen, int G = 1);
 cudaError_t launch_chunk_bwd(const BwdArgs &a, cudaStream_t stream);
 
 }  // namespace gdn

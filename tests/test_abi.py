@@ -232,3 +232,15 @@ def test_fused_backward_rejects_before_any_launch():
     assert call(dout=FAKE + 4) == gdn.GDN_ERR_INVALID_ARGUMENT
     assert call(workspace=None) == gdn.GDN_ERR_WORKSPACE
     assert gdn.gdn_chunk_bwd_fused_workspace_bytes(1, 64, 1, 128, 64, 64, 0) == ctypes.c_size_t(-1).value
+
+
+def test_grouped_backward_rejects_bad_groups():
+    a = dict(q=FAKE, k=FAKE, v=FAKE, log_alpha=FAKE, beta=FAKE, S0=None, dout=FAKE, dS_final=None, dq=FAKE, dk=FAKE,
+             dv=FAKE, dlog_alpha=FAKE, dbeta=FAKE, dS0=None, B=1, T=64, Hk=2, Hv=5, dk_=64, dv_=64, chunk=64,
+             cu_seqlens=None, dtype=gdn.GDN_DTYPE_BF16, workspace=FAKE * 256, workspace_bytes=1 << 40, stream=None)
+    assert gdn.gdn_chunk_bwd_gva(**a) == gdn.GDN_ERR_INVALID_ARGUMENT        # 5 value heads on 2 q/k heads
+    assert gdn.gdn_chunk_bwd_gva(**dict(a, Hv=4, dk_=128)) == gdn.GDN_ERR_UNSUPPORTED
+    assert gdn.gdn_chunk_bwd_gva(**dict(a, Hv=4, workspace=None)) == gdn.GDN_ERR_WORKSPACE
+    assert gdn.gdn_chunk_bwd_gva_workspace_bytes(1, 64, 2, 5, 64, 64, 64, 0) == ctypes.c_size_t(-1).value
+    plain = gdn.gdn_chunk_bwd_workspace_bytes(1, 64, 4, 64, 64, 64, 0)
+    assert gdn.gdn_chunk_bwd_gva_workspace_bytes(1, 64, 2, 4, 64, 64, 64, 0) >= plain + 2 * 64 * 4 * 64 * 4
