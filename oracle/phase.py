@@ -146,3 +146,36 @@ def forward_chunkwise(K, Q, V, log_lam, beta, M0=None, chunk=64, cu_seqlens=None
                 out[rows] = O
             Mf[s, h] = M
     return out, Mf
+
+
+def backward(K, Q, V, log_lam, beta, M0, dout, dM_final=None, cu_seqlens=None):
+    """fp64 gradients of ``forward`` with respect to (K, Q, V, log_lam, beta, M0) for the loss
+    gradients dout (dL/d out) and dM_final (dL/d M_final, complex: d/dRe + i d/dIm; None = 0).
+    Complex gradients are returned the same way (d/dRe + i d/dIm).
+
+    Through the real form of the recurrence (the module doc: S = [Re M | Im M]^T, head size 2 dk,
+    a = lam, b = beta / lam, k = (Re K, Im K) / sqrt(dk), v = lam sqrt(dk) V, q = (Re Q, Im Q) / dk):
+    the real backward oracle, then the chain rule of that map --
+    dK = dk / sqrt(dk), dQ = dq / dk, dV = lam sqrt(dk) dv, dbeta = db / lam,
+    dlog_lam = dlog_a + sum_j dv_j v_j - db b.  Pinned against finite differences of ``forward``."""
+    import oracle
+    K, Q, M0, dMf = as_complex(K), as_complex(Q), as_complex(M0), as_complex(dM_final)
+    V, la, be, dO = _real(V), _real(log_lam), _real(beta), _real(dout)
+    dk = K.shape[-1]
+    lam = np.exp(la)
+    k = np.concatenate([K.real, K.imag], axis=-1) / np.sqrt(dk)
+    q = np.concatenate([Q.real, Q.imag], axis=-1) / dk
+    v = lam[..., None] * np.sqrt(dk) * V
+    b = be / lam
+
+    def to_real_state(M):
+        return None if M is None else np.concatenate([M.real, M.imag], axis=-1).swapaxes(-1, -2)
+    dq, dkr, dv, dla, db, dS0 = oracle.backward(q, k, v, la, b, to_real_state(M0), dO, to_real_state(dMf),
+                                                cu_seqlens=cu_seqlens)
+    dK = (dkr[..., :dk] + 1j * dkr[..., dk:]) / np.sqrt(dk)
+    dQ = (dq[..., :dk] + 1j * dq[..., dk:]) / dk
+    dV = lam[..., None] * np.sqrt(dk) * dv
+    dlog_lam = dla + np.sum(dv * v, axis=-1) - db * b
+    dS0 = dS0.swapaxes(-1, -2)
+    dM0 = dS0[..., :dk] + 1j * dS0[..., dk:]
+    return dK, dQ, dV, dlog_lam, db / lam, dM0

@@ -164,3 +164,38 @@ def test_reduces_to_the_real_gated_delta_rule():
         np.testing.assert_allclose(o_r, o, atol=1e-10)
         np.testing.assert_allclose(S_r[:, :, :dk, :].transpose(0, 1, 3, 2), M.real, atol=1e-10)
         np.testing.assert_allclose(S_r[:, :, dk:, :].transpose(0, 1, 3, 2), M.imag, atol=1e-10)
+
+
+def test_backward_matches_finite_differences():
+    # the backward oracle (through the real form) against central differences of the complex
+    # definition, for every real input component: Re / Im of K, Q, M0; V; log_lam; beta
+    rng = np.random.default_rng(40)
+    for lengths in (None, [3, 0, 6]):
+        c = rand_case(rng, B=2, T=7, H=2, dk=3, dv=2, laplace=True, beta_max=2.0, lengths=lengths)
+        Go = rng.normal(size=c["V"].shape)
+        Wm = rng.normal(size=c["M0"].shape) + 1j * rng.normal(size=c["M0"].shape)
+
+        def loss():
+            o, M = run(c)
+            return float(np.sum(o * Go) + np.sum(M.real * Wm.real + M.imag * Wm.imag))
+        got = dict(zip(("K", "Q", "V", "log_lam", "beta", "M0"),
+                       phase.backward(c["K"], c["Q"], c["V"], c["log_lam"], c["beta"], c["M0"], Go, Wm,
+                                      cu_seqlens=c["cu_seqlens"])))
+        h = 1e-6
+        for name in ("K", "Q", "V", "log_lam", "beta", "M0"):
+            x = c[name]
+            parts = (1.0, 1j) if np.iscomplexobj(x) else (1.0,)
+            for part in parts:
+                fd = np.zeros(x.shape)
+                for i in np.ndindex(x.shape):
+                    old = x[i]
+                    x[i] = old + h * part
+                    lp = loss()
+                    x[i] = old - h * part
+                    lm = loss()
+                    x[i] = old
+                    fd[i] = (lp - lm) / (2 * h)
+                g = got[name].real if part == 1.0 else got[name].imag
+                if not np.iscomplexobj(x):
+                    g = got[name]
+                assert np.max(np.abs(fd - g)) / (1.0 + np.max(np.abs(fd))) < 1e-6, (name, part)
