@@ -222,6 +222,24 @@ GDN_API int gdn_phase_fwd(const float *K, const float *Q, const void *v, const f
 GDN_API size_t gdn_phase_fwd_workspace_bytes(int B, int T, int H, int dk, int dv, int varlen, int dtype);
 
 /*
+ * gdn_phase_bwd -- gradients of gdn_phase_fwd for dk = 32 complex (64 real) and dv = 64: given the
+ * forward's inputs, dout = dL/dout (dtype) and dM_final = dL/dM_final ((re, im) pairs, NULL: zero),
+ * it writes fp32
+ *     dK, dQ [.., H, 32, 2] (d/dRe, d/dIm pairs), dv [.., H, 64], dlog_lam, dbeta [.., H],
+ *     dM0 [B, H, 64, 32, 2] (NULL: not written).
+ * The fp32 backward of the real recurrence runs on the map gdn_phase_fwd uses (see gdn_phase.cu),
+ * followed by its chain rule.  Workspace: gdn_phase_bwd_workspace_bytes(...), 256-byte aligned.
+ */
+GDN_API int gdn_phase_bwd(const float *K, const float *Q, const void *v, const float *log_lam, const float *beta,
+                          const float *M0, const void *dout, const float *dM_final, float *dK, float *dQ,
+                          float *dv_out, float *dlog_lam, float *dbeta, float *dM0, int B, int T, int H, int dk,
+                          int dv, const int32_t *cu_seqlens, int dtype, void *workspace, size_t workspace_bytes,
+                          void *stream);
+
+/* Workspace gdn_phase_bwd needs for these sizes; (size_t)-1 for sizes it rejects. */
+GDN_API size_t gdn_phase_bwd_workspace_bytes(int B, int T, int H, int dk, int dv, int varlen);
+
+/*
  * gdn_chunk_bwd -- gradients of gdn_chunk_fwd (the training path; Sykra README, "Architectural
  * Highlights": chunk-parallel training through the WY / unit triangular transform), for
  * dk = dv = 64 and chunk = 64.  Given the forward's inputs (same layouts, dtype for q, k, v and

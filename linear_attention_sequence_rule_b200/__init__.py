@@ -8,7 +8,8 @@ PyTorch provides device memory and streams.  The binding has two layers:
   ``gdn_status_string``, ``gdn_last_error``, ``gdn_version`` -- the C-ABI entry points of
   ``include/gdn.h`` with the same names and arguments (pointers as Python ints);
 * ``chunk_fwd``, ``chunk_fwd_host``, ``chunk_fwd_fused``, ``chunk_fwd_gva``, ``chunk_bwd``,
-  ``chunk_bwd_fused``, ``chunk_bwd_gva``, ``phase_fwd``, ``decode_step`` and ``decode_step_gva`` --
+  ``chunk_bwd_fused``, ``chunk_bwd_gva``, ``phase_fwd``, ``phase_bwd``, ``decode_step`` and
+  ``decode_step_gva`` --
   the same calls taking torch tensors; they check shapes,
   devices and dtypes, allocate outputs with torch when none are given, and raise ``GdnError``
   on a non-zero status.
@@ -28,6 +29,7 @@ __all__ = [
     "gdn_chunk_fwd", "gdn_chunk_fwd_noalloc", "gdn_chunk_fwd_fused", "gdn_chunk_fwd_gva",
     "gdn_chunk_fwd_host", "gdn_chunk_fwd_host_workspace_bytes", "chunk_fwd_host",
     "gdn_phase_fwd", "gdn_phase_fwd_workspace_bytes", "phase_fwd",
+    "gdn_phase_bwd", "gdn_phase_bwd_workspace_bytes", "phase_bwd",
     "gdn_chunk_bwd_fused", "gdn_chunk_bwd_fused_workspace_bytes", "chunk_bwd_fused",
     "gdn_chunk_bwd_gva", "gdn_chunk_bwd_gva_workspace_bytes", "chunk_bwd_gva",
     "gdn_decode_step", "gdn_decode_step_gva", "gdn_chunk_bwd", "gdn_chunk_bwd_workspace_bytes", "gdn_chunk_fwd_workspace_bytes", "gdn_status_string",
@@ -87,6 +89,10 @@ _lib.gdn_chunk_fwd_host_workspace_bytes.restype = _sz
 _lib.gdn_phase_fwd.argtypes = [_vp] * 8 + [_i] * 5 + [_vp, _i, _vp, _sz, _vp]
 _lib.gdn_phase_fwd.restype = _i
 _lib.gdn_phase_fwd_workspace_bytes.argtypes = [_i] * 7
+_lib.gdn_phase_bwd.argtypes = [_vp] * 14 + [_i] * 5 + [_vp, _i, _vp, _sz, _vp]
+_lib.gdn_phase_bwd.restype = _i
+_lib.gdn_phase_bwd_workspace_bytes.argtypes = [_i] * 6
+_lib.gdn_phase_bwd_workspace_bytes.restype = _sz
 _lib.gdn_phase_fwd_workspace_bytes.restype = _sz
 _lib.gdn_chunk_fwd_workspace_bytes.argtypes = [_i, _i, _i, _i, _i, _i, _i, _i]
 _lib.gdn_chunk_fwd_workspace_bytes.restype = _sz
@@ -170,6 +176,16 @@ def gdn_phase_fwd(K, Q, v, log_lam, beta, M0, out, M_final, B, T, H, dk, dv, cu_
 
 def gdn_phase_fwd_workspace_bytes(B, T, H, dk, dv, varlen, dtype) -> int:
     return _lib.gdn_phase_fwd_workspace_bytes(B, T, H, dk, dv, varlen, dtype)
+
+
+def gdn_phase_bwd(K, Q, v, log_lam, beta, M0, dout, dM_final, dK, dQ, dv_out, dlog_lam, dbeta, dM0, B, T, H, dk,
+                  dv, cu_seqlens, dtype, workspace, workspace_bytes, stream) -> int:
+    return _lib.gdn_phase_bwd(K, Q, v, log_lam, beta, M0, dout, dM_final, dK, dQ, dv_out, dlog_lam, dbeta, dM0, B,
+                              T, H, dk, dv, cu_seqlens, dtype, workspace, workspace_bytes, stream)
+
+
+def gdn_phase_bwd_workspace_bytes(B, T, H, dk, dv, varlen) -> int:
+    return _lib.gdn_phase_bwd_workspace_bytes(B, T, H, dk, dv, varlen)
 
 
 def gdn_chunk_fwd_workspace_bytes(B, T, H, dk, dv, chunk, varlen, dtype) -> int:
@@ -401,6 +417,53 @@ def phase_fwd(K, Q, v, log_lam, beta, M0=None, cu_seqlens=None, out=None, M_fina
     if rc != GDN_OK:
         raise GdnError(rc, gdn_last_error())
     return out, (None if Mf is None else torch.view_as_complex(Mf))
+
+
+def phase_bwd(K, Q, v, log_lam, beta, dout, M0=None, dM_final=None, cu_seqlens=None, want_dM0=True,
+              workspace=None, stream=None):
+    """Gradients of ``phase_fwd`` (dk = 32 complex, dv = 64): returns (dK, dQ complex64, dv fp32,
+    dlog_lam, dbeta fp32, dM0 complex64 or None); complex gradients as d/dRe + i d/dIm."""
+    Kp, Qp = _as_pairs(K, "K"), _as_pairs(Q, "Q")
+    dt = v.dtype
+    if dt not in _DT:
+        raise ValueError(f"unsupported dtype {dt}")
+    dev = v.device
+    if cu_seqlens is not None:
+        T, H, dk = Kp.shape[:3]
+        B = cu_seqlens.shape[0] - 1
+        lead = (T,)
+        _need(cu_seqlens, "cu_seqlens", torch.int32, (B + 1,), dev)
+    else:
+        B, T, H, dk = Kp.shape[:4]
+        lead = (B, T)
+    dv = v.shape[-1]
+    _need(Kp, "K", torch.float32, (*lead, H, dk, 2), dev)
+    _need(Qp, "Q", torch.float32, (*lead, H, dk, 2), dev)
+    _need(v, "v", dt, (*lead, H, dv), dev)
+    _need(dout, "dout", dt, (*lead, H, dv), dev)
+    _need(log_lam, "log_lam", torch.float32, (*lead, H), dev)
+    _need(beta, "beta", torch.float32, (*lead, H), dev)
+    M0p, dMp = _as_pairs(M0, "M0"), _as_pairs(dM_final, "dM_final")
+    for name, x in (("M0", M0p), ("dM_final", dMp)):
+        if x is not None:
+            _need(x, name, torch.float32, (B, H, dv, dk, 2), dev)
+    f32 = dict(dtype=torch.float32, device=dev)
+    dK, dQ = torch.empty((*lead, H, dk, 2), **f32), torch.empty((*lead, H, dk, 2), **f32)
+    dV = torch.empty((*lead, H, dv), **f32)
+    dla, dbe = torch.empty((*lead, H), **f32), torch.empty((*lead, H), **f32)
+    dM0 = torch.empty((B, H, dv, dk, 2), **f32) if want_dM0 else None
+    need = gdn_phase_bwd_workspace_bytes(B, T, H, dk, dv, int(cu_seqlens is not None))
+    if need == ctypes.c_size_t(-1).value:
+        raise GdnError(GDN_ERR_UNSUPPORTED, f"gdn_phase_bwd: unsupported sizes dk={dk} dv={dv}")
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    rc = gdn_phase_bwd(_ptr(Kp), _ptr(Qp), _ptr(v), _ptr(log_lam), _ptr(beta), _ptr(M0p), _ptr(dout), _ptr(dMp),
+                       _ptr(dK), _ptr(dQ), _ptr(dV), _ptr(dla), _ptr(dbe), _ptr(dM0), B, T, H, dk, dv,
+                       _ptr(cu_seqlens), _DT[dt], _ptr(workspace), workspace.numel(), _stream_ptr(stream))
+    if rc != GDN_OK:
+        raise GdnError(rc, gdn_last_error())
+    return (torch.view_as_complex(dK), torch.view_as_complex(dQ), dV, dla, dbe,
+            None if dM0 is None else torch.view_as_complex(dM0))
 
 
 def chunk_fwd_fused(q_raw, k_raw, v, a_raw, b_raw, a_scale, b_scale, S0=None, cu_seqlens=None,

@@ -51,16 +51,16 @@ template <> struct Pack4<__nv_bfloat16> {
     }
 };
 
-template <int DK, int DV, typename TV>
+template <int DK, int DV, typename TV, typename TO>
 __global__ void __launch_bounds__(256) phase_prologue(const float4 *__restrict__ K, const float4 *__restrict__ Q,
                                                       const TV *__restrict__ V, const float *__restrict__ log_lam,
                                                       const float *__restrict__ beta, long token_heads,
-                                                      TV *__restrict__ kr, TV *__restrict__ qr, TV *__restrict__ vr,
+                                                      TO *__restrict__ kr, TO *__restrict__ qr, TO *__restrict__ vr,
                                                       float *__restrict__ br)
 {
     constexpr int TPT = DK / 4;       // threads per token-head
     constexpr int VPT = DV / TPT;     // value elements per thread
-    using P = Pack4<TV>;
+    using P = Pack4<TO>;
     const long idx = (long)blockIdx.x * blockDim.x + threadIdx.x;
     const long th = idx / TPT;
     const int i = (int)(idx % TPT);
@@ -144,17 +144,18 @@ bool phase_plan(PhasePlan &p, int B, int T, int H, int dk, int dv, int varlen, i
     return true;
 }
 
-template <int DK, int DV, typename TV>
+// The prologue into the workspace regions p.kr, p.qr, p.vr, p.br; v read as TV, written as TO.
+template <int DK, int DV, typename TV, typename TO = TV>
 cudaError_t launch_prologue(const float *K, const float *Q, const void *V, const float *log_lam, const float *beta,
                             long token_heads, char *w, const PhasePlan &p, cudaStream_t st)
 {
     const long threads = token_heads * (DK / 4);
     const unsigned blocks = (unsigned)((threads + 255) / 256);
     if (blocks)
-        phase_prologue<DK, DV, TV><<<blocks, 256, 0, st>>>(
+        phase_prologue<DK, DV, TV, TO><<<blocks, 256, 0, st>>>(
             reinterpret_cast<const float4 *>(K), reinterpret_cast<const float4 *>(Q), static_cast<const TV *>(V),
-            log_lam, beta, token_heads, reinterpret_cast<TV *>(w + p.kr), reinterpret_cast<TV *>(w + p.qr),
-            reinterpret_cast<TV *>(w + p.vr), reinterpret_cast<float *>(w + p.br));
+            log_lam, beta, token_heads, reinterpret_cast<TO *>(w + p.kr), reinterpret_cast<TO *>(w + p.qr),
+            reinterpret_cast<TO *>(w + p.vr), reinterpret_cast<float *>(w + p.br));
     return cudaGetLastError();
 }
 
@@ -167,6 +168,87 @@ cudaError_t prologue_for(int dk, int dv, const float *K, const float *Q, const v
                          : launch_prologue<64, 64, TV>(K, Q, V, log_lam, beta, token_heads, w, p, st);
     return dv == 128 ? launch_prologue<32, 128, TV>(K, Q, V, log_lam, beta, token_heads, w, p, st)
                      : launch_prologue<32, 64, TV>(K, Q, V, log_lam, beta, token_heads, w, p, st);
+}
+
+// ---- backward ---------------------------------------------------------------------------------
+// gdn_phase_bwd runs the fp32 backward of the real recurrence (head size 2 dk = 64, dv = 64) on the
+// same map and applies its chain rule: dK = dk_r / sqrt(dk), dQ = dq_r / dk, dV = lam sqrt(dk) dv_r,
+// dbeta = db_r / lam, dlog_lam = dlog_a + sum_j dv_r,j v_r,j - db_r b_r, dM0 from the real dS0.
+
+// dout in fp32 (a copy when it arrives in bf16); one thread per element.
+template <typename TV>
+__global__ void phase_widen(const TV *__restrict__ x, float *__restrict__ y, long n)
+{
+    const long i = (long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i < n) y[i] = to_f(x[i]);
+}
+
+// One warp per token-head (DK = 32 complex key elements: one per lane; DV = 64: two per lane).
+__global__ void __launch_bounds__(256) phase_bwd_epilogue(const float *__restrict__ dq_r,
+                                                          const float *__restrict__ dk_r,
+                                                          const float *__restrict__ dv_r,
+                                                          const float *__restrict__ v_r, const float *__restrict__ dla,
+                                                          const float *__restrict__ db_r,
+                                                          const float *__restrict__ b_r,
+                                                          const float *__restrict__ log_lam, long token_heads,
+                                                          float2 *__restrict__ dK, float2 *__restrict__ dQ,
+                                                          float *__restrict__ dV, float *__restrict__ dlog_lam,
+                                                          float *__restrict__ dbeta)
+{
+    constexpr int DK = 32, DV = 64;
+    const long th = ((long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    if (th >= token_heads) return;
+    const float lam = expf(log_lam[th]);
+    dK[th * DK + lane] = make_float2(dk_r[th * 2 * DK + lane] * KeyScale<DK>::inv_sqrt,
+                                     dk_r[th * 2 * DK + DK + lane] * KeyScale<DK>::inv_sqrt);
+    dQ[th * DK + lane] = make_float2(dq_r[th * 2 * DK + lane] * (1.0f / DK), dq_r[th * 2 * DK + DK + lane] * (1.0f / DK));
+    const float g0 = dv_r[th * DV + lane], g1 = dv_r[th * DV + lane + 32];
+    const float vs = lam * KeyScale<DK>::sqrt;
+    dV[th * DV + lane] = vs * g0;
+    dV[th * DV + lane + 32] = vs * g1;
+    float dot = g0 * v_r[th * DV + lane] + g1 * v_r[th * DV + lane + 32];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+    if (lane == 0) {
+        dlog_lam[th] = dla[th] + dot - db_r[th] * b_r[th];
+        dbeta[th] = db_r[th] / lam;
+    }
+}
+
+struct PhaseBwdPlan {
+    size_t kr, qr, vr, br, d32, s0, sf, dq, dk, dv, dla, db, ds0, ws, ws_bytes, total;
+};
+
+bool phase_bwd_plan(PhaseBwdPlan &p, int B, int T, int H, int varlen)
+{
+    constexpr int DK = 32, DV = 64;
+    const size_t ws = gdn_chunk_bwd_workspace_bytes(B, T, H, 2 * DK, DV, 64, varlen);
+    if (ws == (size_t)-1) return false;
+    const size_t th = (varlen ? (size_t)T : (size_t)B * T) * H, st = (size_t)B * H * 2 * DK * DV * 4;
+    size_t o = 0;
+    auto take = [&](size_t bytes) {
+        const size_t at = o;
+        o += al256(bytes);
+        return at;
+    };
+    p.kr = take(th * 2 * DK * 4);
+    p.qr = take(th * 2 * DK * 4);
+    p.vr = take(th * DV * 4);
+    p.br = take(th * 4);
+    p.d32 = take(th * DV * 4);
+    p.s0 = take(st);
+    p.sf = take(st);
+    p.dq = take(th * 2 * DK * 4);
+    p.dk = take(th * 2 * DK * 4);
+    p.dv = take(th * DV * 4);
+    p.dla = take(th * 4);
+    p.db = take(th * 4);
+    p.ds0 = take(st);
+    p.ws_bytes = ws;
+    p.ws = take(ws);
+    p.total = o;
+    return true;
 }
 
 }  // namespace
@@ -252,6 +334,113 @@ int gdn_phase_fwd(const float *K, const float *Q, const void *v, const float *lo
             return GDN_ERR_CUDA;
         }
     }
+    return GDN_OK;
+}
+
+
+size_t gdn_phase_bwd_workspace_bytes(int B, int T, int H, int dk, int dv, int varlen)
+{
+    if (dk != 32 || dv != 64) return (size_t)-1;
+    PhaseBwdPlan p;
+    if (!phase_bwd_plan(p, B, T, H, varlen)) return (size_t)-1;
+    return p.total;
+}
+
+int gdn_phase_bwd(const float *K, const float *Q, const void *v, const float *log_lam, const float *beta,
+                  const float *M0, const void *dout, const float *dM_final, float *dK, float *dQ, float *dv_out,
+                  float *dlog_lam, float *dbeta, float *dM0, int B, int T, int H, int dk, int dv,
+                  const int32_t *cu_seqlens, int dtype, void *workspace, size_t workspace_bytes, void *stream)
+{
+    const int varlen = cu_seqlens != nullptr;
+    if (dk != 32 || dv != 64 || (dtype != GDN_DTYPE_BF16 && dtype != GDN_DTYPE_F32)) {
+        set_error("gdn_phase_bwd: dk=%d dv=%d dtype=%d, supported: dk 32 (64 real), dv 64, bf16 or fp32", dk, dv,
+                  dtype);
+        return GDN_ERR_UNSUPPORTED;
+    }
+    PhaseBwdPlan p;
+    if (!phase_bwd_plan(p, B, T, H, varlen))  // the backward's own checks give the reason
+        return gdn_chunk_bwd(nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr,
+                             nullptr, nullptr, nullptr, nullptr, nullptr, B, T, H, 2 * dk, dv, 64, cu_seqlens,
+                             GDN_DTYPE_F32, nullptr, 0, stream);
+    if (!K || !Q || !v || !log_lam || !beta || !dout || !dK || !dQ || !dv_out || !dlog_lam || !dbeta) {
+        set_error("gdn_phase_bwd: inputs, dout and every gradient output except dM0 are required");
+        return GDN_ERR_INVALID_ARGUMENT;
+    }
+    const void *ptrs[] = {K, Q, v, log_lam, beta, M0, dout, dM_final, dK, dQ, dv_out, dlog_lam, dbeta, dM0,
+                          cu_seqlens};
+    for (const void *ptr : ptrs)
+        if (ptr && (reinterpret_cast<uintptr_t>(ptr) & 15u)) {
+            set_error("gdn_phase_bwd: pointer %p is not 16-byte aligned", ptr);
+            return GDN_ERR_INVALID_ARGUMENT;
+        }
+    if (!workspace || workspace_bytes < p.total) {
+        set_error("gdn_phase_bwd: workspace of %zu bytes needed, %zu given", p.total,
+                  workspace ? workspace_bytes : (size_t)0);
+        return GDN_ERR_WORKSPACE;
+    }
+    if (reinterpret_cast<uintptr_t>(workspace) & 255u) {
+        set_error("gdn_phase_bwd: workspace must be 256-byte aligned");
+        return GDN_ERR_INVALID_ARGUMENT;
+    }
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    char *w = static_cast<char *>(workspace);
+    const long th = (varlen ? (long)T : (long)B * T) * H, states = (long)B * H;
+    auto fail_launch = [](cudaError_t err) {
+        set_error("gdn_phase_bwd: launch: %s", cudaGetErrorString(err));
+        return GDN_ERR_CUDA;
+    };
+    // the forward's prologue, written in fp32: k, q, v, b of the real recurrence
+    PhasePlan fp{};
+    fp.kr = p.kr;
+    fp.qr = p.qr;
+    fp.vr = p.vr;
+    fp.br = p.br;
+    cudaError_t e = dtype == GDN_DTYPE_BF16
+                        ? launch_prologue<32, 64, __nv_bfloat16, float>(K, Q, v, log_lam, beta, th, w, fp, st)
+                        : launch_prologue<32, 64, float, float>(K, Q, v, log_lam, beta, th, w, fp, st);
+    if (e != cudaSuccess) return fail_launch(e);
+    const long nv = th * dv;
+    float *d32 = reinterpret_cast<float *>(w + p.d32);
+    if (dtype == GDN_DTYPE_BF16) {
+        if (nv) phase_widen<__nv_bfloat16><<<(unsigned)((nv + 255) / 256), 256, 0, st>>>(
+                static_cast<const __nv_bfloat16 *>(dout), d32, nv);
+        e = cudaGetLastError();
+    } else if (nv) {
+        e = cudaMemcpyAsync(d32, dout, (size_t)nv * 4, cudaMemcpyDeviceToDevice, st);
+    }
+    if (e != cudaSuccess) return fail_launch(e);
+    const long ns = states * 2 * dk * dv;
+    if (M0) phase_state_in<<<(unsigned)((ns + 255) / 256), 256, 0, st>>>(reinterpret_cast<const float2 *>(M0),
+                                                                          reinterpret_cast<float *>(w + p.s0), dk, dv,
+                                                                          states);
+    if (dM_final)
+        phase_state_in<<<(unsigned)((ns + 255) / 256), 256, 0, st>>>(reinterpret_cast<const float2 *>(dM_final),
+                                                                     reinterpret_cast<float *>(w + p.sf), dk, dv,
+                                                                     states);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return fail_launch(e);
+    float *dq = reinterpret_cast<float *>(w + p.dq), *dkr = reinterpret_cast<float *>(w + p.dk),
+          *dvr = reinterpret_cast<float *>(w + p.dv), *dla = reinterpret_cast<float *>(w + p.dla),
+          *dbr = reinterpret_cast<float *>(w + p.db);
+    const int rc = gdn_chunk_bwd(w + p.qr, w + p.kr, w + p.vr, log_lam, reinterpret_cast<const float *>(w + p.br),
+                                 M0 ? reinterpret_cast<const float *>(w + p.s0) : nullptr, d32,
+                                 dM_final ? reinterpret_cast<const float *>(w + p.sf) : nullptr, dq, dkr, dvr, dla,
+                                 dbr, dM0 ? reinterpret_cast<float *>(w + p.ds0) : nullptr, B, T, H, 2 * dk, dv, 64,
+                                 cu_seqlens, GDN_DTYPE_F32, w + p.ws, p.ws_bytes, stream);
+    if (rc != GDN_OK) return rc;
+    if (th)
+        phase_bwd_epilogue<<<(unsigned)((th * 32 + 255) / 256), 256, 0, st>>>(
+            dq, dkr, dvr, reinterpret_cast<const float *>(w + p.vr), dla, dbr,
+            reinterpret_cast<const float *>(w + p.br), log_lam, th, reinterpret_cast<float2 *>(dK),
+            reinterpret_cast<float2 *>(dQ), dv_out, dlog_lam, dbeta);
+    if (dM0) {
+        const long nm = states * dk * dv;
+        phase_state_out<<<(unsigned)((nm + 255) / 256), 256, 0, st>>>(reinterpret_cast<const float *>(w + p.ds0),
+                                                                       reinterpret_cast<float2 *>(dM0), dk, dv,
+                                                                       states);
+    }
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return fail_launch(e);
     return GDN_OK;
 }
 

@@ -244,3 +244,15 @@ def test_grouped_backward_rejects_bad_groups():
     assert gdn.gdn_chunk_bwd_gva_workspace_bytes(1, 64, 2, 5, 64, 64, 64, 0) == ctypes.c_size_t(-1).value
     plain = gdn.gdn_chunk_bwd_workspace_bytes(1, 64, 4, 64, 64, 64, 0)
     assert gdn.gdn_chunk_bwd_gva_workspace_bytes(1, 64, 2, 4, 64, 64, 64, 0) >= plain + 2 * 64 * 4 * 64 * 4
+
+
+def test_phase_backward_rejects_before_any_launch():
+    a = dict(K=FAKE, Q=FAKE, v=FAKE, log_lam=FAKE, beta=FAKE, M0=None, dout=FAKE, dM_final=None, dK=FAKE, dQ=FAKE,
+             dv_out=FAKE, dlog_lam=FAKE, dbeta=FAKE, dM0=None, B=1, T=64, H=1, dk=32, dv=64, cu_seqlens=None,
+             dtype=gdn.GDN_DTYPE_BF16, workspace=FAKE * 256, workspace_bytes=1 << 40, stream=None)
+    assert gdn.gdn_phase_bwd(**dict(a, dk=64)) == gdn.GDN_ERR_UNSUPPORTED   # the backward takes 64 real columns
+    assert gdn.gdn_phase_bwd(**dict(a, dv=128)) == gdn.GDN_ERR_UNSUPPORTED
+    assert gdn.gdn_phase_bwd(**dict(a, dQ=None)) == gdn.GDN_ERR_INVALID_ARGUMENT
+    assert gdn.gdn_phase_bwd(**dict(a, K=FAKE + 4)) == gdn.GDN_ERR_INVALID_ARGUMENT
+    assert gdn.gdn_phase_bwd(**dict(a, workspace=None)) == gdn.GDN_ERR_WORKSPACE
+    assert gdn.gdn_phase_bwd_workspace_bytes(1, 64, 1, 64, 64, 0) == ctypes.c_size_t(-1).value
