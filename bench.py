@@ -462,6 +462,7 @@ def run_ours(args, world, rank, local):
         del dg, outg, Sg
         extra["hybrid_lm_backward"] = backward_numbers(gdn, d, 5, 3, flush, stream, peaks)
         extra["phase_memory"] = phase_numbers(gdn, 5, 3, flush, stream, peaks)
+        extra["decode_small_batch_graph"] = decode_graph_numbers(gdn)
     cpu = None
     if rank == 0 and world == 1:
         cpu = cpu_oracle_baseline(inp)
@@ -578,6 +579,45 @@ def phase_numbers(gdn, steps, warmup, flush, stream, peaks):
             "launches_per_call": 3, "algo_bytes": by_p,
             "gbs": round(by_p / (ms_p * 1e-3) / 1e9, 3),
             "hbm_frac": round(by_p / (ms_p * 1e-3) / 1e9 / peaks["hbm_gbs"], 5)}
+
+
+def decode_graph_numbers(gdn, steps=100):
+    """Small-batch decode (16 sequences x 8 heads, d = 128), where launch overhead rivals the
+    kernel: 100 steps launched one by one from Python versus the same steps captured once in a
+    CUDA graph and replayed; per-step time from CUDA events around the 100 steps."""
+    N, H, d = 16, 8, 128
+    xs = [to_dev(workloads.make_decode_step_inputs(N, H, d, d, "bf16", seed=9, step=i)) for i in range(steps)]
+    S = workloads.make_decode_state(N, H, d, d, seed=9).cuda()
+    outs = [torch.empty(N, H, d, dtype=torch.bfloat16, device="cuda") for _ in range(steps)]
+
+    def run_steps():
+        for x, o in zip(xs, outs):
+            gdn.decode_step(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], S, out=o)
+    side = torch.cuda.Stream()
+    with torch.cuda.stream(side):
+        run_steps()  # first calls outside the capture
+        side.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(side)
+        run_steps()
+        e1.record(side)
+        side.synchronize()
+    eager = e0.elapsed_time(e1) / steps
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        run_steps()
+    g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    graph.replay()
+    torch.cuda.synchronize()
+    g0.record()
+    graph.replay()
+    g1.record()
+    torch.cuda.synchronize()
+    replay = g0.elapsed_time(g1) / steps
+    del graph
+    return {"workload": "decode, 16 x 8 states of 128 x 128, 100 steps per measurement",
+            "eager_us_per_step": round(eager * 1e3, 3), "graph_us_per_step": round(replay * 1e3, 3),
+            "launches_per_step": 1}
 
 
 def run_only(args):
