@@ -339,6 +339,16 @@ GDN_API int gdn_decode_step_gva(const void *q, const void *k, const void *v, con
  */
 GDN_API int gdn_device_status(void *stream);
 
+/*
+ * gdn_selftest_wait_timeout -- exercise the failure path of the bounded waits: enqueues on `stream`
+ * one kernel whose wait on an mbarrier that nothing arrives on runs out after limit_ms (1..2000)
+ * milliseconds; the kernel records it in the device error word the other kernels use and returns.
+ * The next gdn_device_status(stream) then reports GDN_ERR_TIMEOUT (and clears the record); the
+ * context stays usable.  Nothing is faulted or hung: the wait is bounded.  The pages have no
+ * counterpart of it; it exists for the library's own failure-detection test.
+ */
+GDN_API int gdn_selftest_wait_timeout(int limit_ms, void *stream);
+
 /* Static text for a status code. */
 GDN_API const char *gdn_status_string(int status);
 

@@ -33,7 +33,7 @@ __all__ = [
     "gdn_chunk_bwd_fused", "gdn_chunk_bwd_fused_workspace_bytes", "chunk_bwd_fused",
     "gdn_chunk_bwd_gva", "gdn_chunk_bwd_gva_workspace_bytes", "chunk_bwd_gva",
     "gdn_decode_step", "gdn_decode_step_gva", "gdn_chunk_bwd", "gdn_chunk_bwd_workspace_bytes", "gdn_chunk_fwd_workspace_bytes", "gdn_status_string",
-    "gdn_last_error", "gdn_version", "gdn_device_status", "device_status", "chunk_fwd", "chunk_fwd_fused",
+    "gdn_last_error", "gdn_version", "gdn_device_status", "gdn_selftest_wait_timeout", "device_status", "chunk_fwd", "chunk_fwd_fused",
     "chunk_fwd_gva", "chunk_bwd", "decode_step", "decode_step_gva", "workspace_bytes",
 ]
 
@@ -98,6 +98,8 @@ _lib.gdn_chunk_fwd_workspace_bytes.argtypes = [_i, _i, _i, _i, _i, _i, _i, _i]
 _lib.gdn_chunk_fwd_workspace_bytes.restype = _sz
 _lib.gdn_decode_step.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp]
 _lib.gdn_decode_step.restype = _i
+_lib.gdn_selftest_wait_timeout.argtypes = [_i, _vp]
+_lib.gdn_selftest_wait_timeout.restype = _i
 _lib.gdn_device_status.argtypes = [_vp]
 _lib.gdn_device_status.restype = _i
 _lib.gdn_status_string.argtypes = [_i]
@@ -194,6 +196,10 @@ def gdn_chunk_fwd_workspace_bytes(B, T, H, dk, dv, chunk, varlen, dtype) -> int:
 
 def gdn_decode_step(q, k, v, log_alpha, beta, S_inout, out, N, H, dk, dv, dtype, stream) -> int:
     return _lib.gdn_decode_step(q, k, v, log_alpha, beta, S_inout, out, N, H, dk, dv, dtype, stream)
+
+
+def gdn_selftest_wait_timeout(limit_ms, stream) -> int:
+    return _lib.gdn_selftest_wait_timeout(limit_ms, stream)
 
 
 def gdn_device_status(stream) -> int:

@@ -236,6 +236,17 @@ int gdn_chunk_fwd_gva(const void *q, const void *k, const void *v, const float *
                             Hv / Hk);
 }
 
+int gdn_selftest_wait_timeout(int limit_ms, void *stream)
+{
+    g_last_error[0] = 0;
+    if (limit_ms < 1 || limit_ms > 2000)
+        return fail(GDN_ERR_INVALID_ARGUMENT, "gdn_selftest_wait_timeout: limit_ms=%d, must lie in [1, 2000]",
+                    limit_ms);
+    cudaError_t e = launch_wait_probe(limit_ms, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "gdn_selftest_wait_timeout");
+    return GDN_OK;
+}
+
 int gdn_device_status(void *stream)
 {
     g_last_error[0] = 0;

@@ -1247,6 +1247,25 @@ cudaError_t launch_chunk_tc(const ChunkArgs &a, cudaStream_t stream)
     return run_chunk<64, 64>(a, stream);
 }
 
+// Self-test of the failure path: one thread waits, bounded by limit_ns, on an mbarrier that nothing
+// arrives on; the wait runs out, the thread records it in the same device error word the kernels
+// use, and the kernel returns (it holds no TMEM and has no copies in flight).
+__global__ void wait_probe_kernel(uint64_t limit_ns)
+{
+    __shared__ __align__(8) uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        fence_mbar_init();
+        if (!mbar_wait_bounded(&bar, 0, limit_ns)) atomicOr(&g_tc_device_error, 2);
+    }
+}
+
+cudaError_t launch_wait_probe(int limit_ms, cudaStream_t stream)
+{
+    wait_probe_kernel<<<1, 32, 0, stream>>>((uint64_t)limit_ms * 1000000ull);
+    return cudaGetLastError();
+}
+
 int read_and_clear_tc_error()
 {
     int v = 0, z = 0;

@@ -46,6 +46,10 @@ size_t chunk_tc_workspace_bytes(int B, int T, int H, int dk, int dv, int varlen,
 // after synchronising the device.  Returns -1 when the read itself failed.
 int read_and_clear_tc_error();
 
+// Self-test of the bounded waits: a kernel whose wait on an mbarrier nothing arrives on runs out
+// after limit_ms and records it in that error word (see gdn_selftest_wait_timeout).
+cudaError_t launch_wait_probe(int limit_ms, cudaStream_t stream);
+
 // Gradients of the chunk forward (fp32-level accuracy, dk = dv = 64); see gdn_chunk_bwd.cu.
 struct BwdArgs {
     const void *q, *k, *v;
