@@ -292,6 +292,15 @@ def chunk_numbers(name, d, times_ms, peaks):
                 tflops=tfs, tensor_frac=tfs / peaks["bf16_tflops"])
 
 
+WIDE_VALUE = "hybrid_lm tokens and heads (B=8 T=4096 H=12) at dk=128, dv=256: two 128-column CTAs per chain"
+
+
+def wide_value_inputs(seed=0):
+    """The hybrid-LM token and head counts at head sizes dk=128, dv=256 (bf16), on the device."""
+    return to_dev(workloads.make_chunk_inputs(B=8, T=4096, H=12, dk=128, dv=256, dtype="bf16", seed=seed,
+                                              la_scale=0.1))
+
+
 def time_decode(gdn, steps, warmup, stream, pool=32):
     cfg = workloads.CONFIGS["decode"]
     N, H, dk, dv = cfg["N"], cfg["H"], cfg["dk"], cfg["dv"]
@@ -418,12 +427,18 @@ def run_ours(args, world, rank, local):
     if not args.quick:
         decode = time_decode(gdn, 1000, 10, stream)
         decode["hbm_frac"] = decode["gbs"] / peaks["hbm_gbs"]
+        # DRAM bytes per step from the ncu record of the current decode source (null once it changed)
+        decode["traffic"] = ncu_traffic("decode", "decode")
         for w in ("long_context", "varlen"):
             dw = to_dev(workloads.config_inputs(w))
             tw = time_chunk(gdn, dw, max(3, args.steps // 20), 2, flush, stream)
             nums = chunk_numbers(w, dw, tw, peaks)
             extra[w] = {k: (round(v, 6) if isinstance(v, float) else v) for k, v in nums.items()}
             del dw
+        dw = wide_value_inputs(rank_seed(cfg["seed"], rank))
+        nums = chunk_numbers(WIDE_VALUE, dw, time_chunk(gdn, dw, max(3, args.steps // 2), 3, flush, stream), peaks)
+        extra["hybrid_lm_dv256"] = {k: (round(v, 6) if isinstance(v, float) else v) for k, v in nums.items()}
+        del dw
         # the same hybrid-LM step from raw projections: fused prologue vs PyTorch prologue + call
         dr = to_dev(workloads.config_raw_inputs(name, seed=rank_seed(cfg["seed"], rank)))
         for key, fused in (("hybrid_lm_fused_prologue", True), ("hybrid_lm_pytorch_prologue", False)):
@@ -635,6 +650,10 @@ def run_only(args):
     elif args.only == "phase_memory":
         flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device="cuda")
         r = phase_numbers(gdn, args.steps, args.warmup, flush, stream, peaks)
+    elif args.only == "hybrid_lm_dv256":
+        flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device="cuda")
+        d = wide_value_inputs()
+        r = chunk_numbers(WIDE_VALUE, d, time_chunk(gdn, d, args.steps, args.warmup, flush, stream), peaks)
     elif args.only in ("hybrid_lm_fused", "hybrid_lm_unfused"):
         flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device="cuda")
         d = to_dev(workloads.config_raw_inputs("hybrid_lm"))
@@ -709,7 +728,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--quick", action="store_true", help="main workload only")
     ap.add_argument("--only", choices=["hybrid_lm", "long_context", "varlen", "tiny", "decode", "hybrid_lm_fused",
-                                             "hybrid_lm_unfused", "hybrid_lm_backward", "phase_memory"],
+                                             "hybrid_lm_unfused", "hybrid_lm_backward", "phase_memory",
+                                             "hybrid_lm_dv256"],
                     help="time one workload's kernel loop only (for profiler runs)")
     args = ap.parse_args()
     if args.warmup < 3:

@@ -53,7 +53,7 @@ extern "C" {
 enum gdn_status {
     GDN_OK = 0,
     GDN_ERR_INVALID_ARGUMENT = -1, /* null required pointer, bad size, misaligned pointer      */
-    GDN_ERR_UNSUPPORTED = -2,      /* dk/dv not in {64,128}, chunk != 64, unknown dtype        */
+    GDN_ERR_UNSUPPORTED = -2,      /* head size, chunk or dtype outside an entry's support      */
     GDN_ERR_WORKSPACE = -3,        /* workspace NULL or smaller than the query function says   */
     GDN_ERR_CUDA = -4,             /* a CUDA launch or driver call failed (see gdn_last_error) */
     GDN_ERR_TIMEOUT = -5           /* reserved: a bounded device-side wait ran out             */
@@ -85,7 +85,8 @@ enum gdn_dtype {
  *          written.  S_final == S0 (same pointer) is allowed (in-place carry); no other
  *          overlap between any output and any input is allowed.
  * Arguments
- *   B >= 1, T >= 0 (T == 0 only with cu_seqlens), H >= 1; dk, dv in {64, 128}; chunk == 64.
+ *   B >= 1, T >= 0 (T == 0 only with cu_seqlens), H >= 1; dk in {64, 128}; dv in {64, 128},
+ *   or 256 with bf16 (run as two 128-column blocks: value columns do not interact); chunk == 64.
  *   log_alpha <= 0 expected (-inf allowed: an exact reset); positive values are accepted but
  *   may overflow.  beta in [0, 2].
  *   workspace / workspace_bytes: device scratch of at least gdn_chunk_fwd_workspace_bytes(...)
@@ -314,8 +315,8 @@ GDN_API size_t gdn_chunk_bwd_fused_workspace_bytes(int B, int T, int H, int dk, 
  *     out = a s + (k . q) u
  *     S  <- a S + k u^T
  *   q,k [N,H,dk]; v,out [N,H,dv] in dtype; log_alpha,beta [N,H] fp32; S_inout [N,H,dk,dv] fp32,
- *   read and overwritten.  N >= 1, H >= 1, dk and dv in {64, 128}.  No overlap between S_inout
- *   and the other arguments.
+ *   read and overwritten.  N >= 1, H >= 1, dk in {64, 128}, dv in {64, 128, 256} (256 runs as two
+ *   128-column blocks per state).  No overlap between S_inout and the other arguments.
  */
 GDN_API int gdn_decode_step(const void *q, const void *k, const void *v, const float *log_alpha,
                     const float *beta, float *S_inout, void *out, int N, int H, int dk, int dv,

@@ -43,8 +43,9 @@ static int check_chunk_shape(int B, int T, int H, int dk, int dv, int chunk, int
 {
     if (dtype != GDN_DTYPE_BF16 && dtype != GDN_DTYPE_F32)
         return fail(GDN_ERR_UNSUPPORTED, "gdn_chunk_fwd: unknown dtype %d", dtype);
-    if (!head_dim_ok(dk) || !head_dim_ok(dv))
-        return fail(GDN_ERR_UNSUPPORTED, "gdn_chunk_fwd: dk=%d dv=%d, supported: 64 or 128", dk, dv);
+    if (!head_dim_ok(dk) || !(head_dim_ok(dv) || (dv == 256 && dtype == GDN_DTYPE_BF16)))
+        return fail(GDN_ERR_UNSUPPORTED,
+                    "gdn_chunk_fwd: dk=%d dv=%d, supported: dk 64 or 128, dv 64 or 128 (256 with bf16)", dk, dv);
     if (chunk != 64)
         return fail(GDN_ERR_UNSUPPORTED, "gdn_chunk_fwd: chunk=%d, supported: 64", chunk);
     if (B < 1 || H < 1)
@@ -176,8 +177,9 @@ static int decode_common(const char *fn, const void *q, const void *k, const voi
 {
     if (dtype != GDN_DTYPE_BF16 && dtype != GDN_DTYPE_F32)
         return fail(GDN_ERR_UNSUPPORTED, "%s: unknown dtype %d", fn, dtype);
-    if (!head_dim_ok(dk) || !head_dim_ok(dv))
-        return fail(GDN_ERR_UNSUPPORTED, "%s: dk=%d dv=%d, supported: 64 or 128", fn, dk, dv);
+    if (!head_dim_ok(dk) || !(head_dim_ok(dv) || dv == 256))
+        return fail(GDN_ERR_UNSUPPORTED, "%s: dk=%d dv=%d, supported: dk 64 or 128, dv 64, 128 or 256", fn, dk,
+                    dv);
     if (N < 1 || H < 1 || (long long)N * H > (1LL << 30))
         return fail(GDN_ERR_INVALID_ARGUMENT, "%s: N=%d H=%d out of range", fn, N, H);
     if (!q || !k || !v || !log_alpha || !beta || !S_inout || !out)

@@ -455,7 +455,11 @@ __global__ void __launch_bounds__(TcCfg<DK, DV>::THREADS, 1)
         len = T;
     }
     const int nchunks = (int)((len + CH - 1) / CH);
-    const size_t sbase = ((size_t)s * H + h) * (size_t)DK * DV;
+    // value columns col0 .. col0 + DV - 1 of a row of ldv: a wider value head runs as gridDim.x
+    // column blocks, one CTA each (value columns do not interact in the recurrence)
+    const int col0 = (int)blockIdx.x * DV;
+    const size_t ldv = (size_t)gridDim.x * DV;
+    const size_t sbase = ((size_t)s * H + h) * (size_t)DK * ldv + col0;
 
     if (tid == 0) {
         for (int i = 0; i < L::NBAR; ++i) mbar_init(&bars[i], (i >= B::gfull && i < B::gfull + NS) ? 32 : 1);
@@ -505,7 +509,7 @@ __global__ void __launch_bounds__(TcCfg<DK, DV>::THREADS, 1)
         uint64_t *vb_bar = &bars[B::v_full + c % NB];
         mbar_arrive_expect_tx(vb_bar, L::V_BUF);
         for (int vb = 0; vb < DV / 64; ++vb)
-            tma_load_3d(sm + L::V + (c % NB) * L::V_BUF + vb * 8192, &tmV, vb_bar, vb * 64, h, tk);
+            tma_load_3d(sm + L::V + (c % NB) * L::V_BUF + vb * 8192, &tmV, vb_bar, col0 + vb * 64, h, tk);
     };
     if (warp == 0) {
         if (lane == 0) {
@@ -783,7 +787,7 @@ __global__ void __launch_bounds__(TcCfg<DK, DV>::THREADS, 1)
                 tc_fence_after();
                 if (tid == 0) ctl.arrive(B::cdone + (c % NS));
                 const int r = 16 * warp + (lane & 15);
-                __nv_bfloat16 *op = out + ((size_t)(tk + r) * H + h) * DV + (lane >> 4) * (DV / 2);
+                __nv_bfloat16 *op = out + ((size_t)(tk + r) * H + h) * ldv + col0 + (lane >> 4) * (DV / 2);
 #pragma unroll 1
                 for (int cb = 0; cb < DV / 64; ++cb) {
                     float o[32];
@@ -819,7 +823,7 @@ __global__ void __launch_bounds__(TcCfg<DK, DV>::THREADS, 1)
 #pragma unroll
                 for (int i = 0; i < 32; ++i)
                     x[i] = (flags & kFlagS0Identity) ? ((cb * 32 + i == j) ? 1.f : 0.f)
-                                                     : (S0 ? S0[sbase + (size_t)(cb * 32 + i) * DV + j] : 0.f);
+                                                     : (S0 ? S0[sbase + (size_t)(cb * 32 + i) * ldv + j] : 0.f);
                 store_state_bf16(0, cb, x);
 #pragma unroll
                 for (int i = 0; i < 32; ++i) x[i] *= g0;
@@ -955,12 +959,12 @@ __global__ void __launch_bounds__(TcCfg<DK, DV>::THREADS, 1)
                     ld_state(k, x);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) S_final[sbase + (size_t)(cb * 32 + i) * DV + j] = x[i];
+                    for (int i = 0; i < 32; ++i) S_final[sbase + (size_t)(cb * 32 + i) * ldv + j] = x[i];
                 }
             } else if (hh == 0) {
                 for (int c2 = 0; c2 < DK; ++c2)
-                    S_final[sbase + (size_t)c2 * DV + j] =
-                        (flags & kFlagS0Identity) ? (c2 == j ? 1.f : 0.f) : (S0 ? S0[sbase + (size_t)c2 * DV + j] : 0.f);
+                    S_final[sbase + (size_t)c2 * ldv + j] =
+                        (flags & kFlagS0Identity) ? (c2 == j ? 1.f : 0.f) : (S0 ? S0[sbase + (size_t)c2 * ldv + j] : 0.f);
             }
         }
     }
@@ -1017,6 +1021,7 @@ struct TcLaunch {
     int flags;
     float a_scale, b_scale;  // fused prologue (kFlagPrologue)
     int G;                   // value heads per q/k head
+    int vblocks = 1;         // value head size = vblocks x DV, one CTA per column block
 };
 
 template <int DK, int DV>
@@ -1029,7 +1034,7 @@ cudaError_t launch_tc(const TcLaunch &a, cudaStream_t st)
     // with V taken as zero nothing is loaded through the V map; any valid map will do
     // with V taken as zero the V map is never read: the k map (H / G heads) serves as a stand-in
     const void *vsrc = (a.flags & kFlagVZero) ? a.k : a.v;
-    const int vdim = (a.flags & kFlagVZero) ? DK : DV;
+    const int vdim = (a.flags & kFlagVZero) ? DK : DV * a.vblocks;
     const int vheads = (a.flags & kFlagVZero) ? a.H / a.G : a.H;
     if (!make_map(&mq, a.q, map_tokens, a.H / a.G, DK) || !make_map(&mk, a.k, map_tokens, a.H / a.G, DK) ||
         !make_map(&mv, vsrc, map_tokens, vheads, vdim)) {
@@ -1040,7 +1045,7 @@ cudaError_t launch_tc(const TcLaunch &a, cudaStream_t st)
     auto kern = (a.flags & kFlagPrologue) ? chunk_tc_kernel<DK, DV, true> : chunk_tc_kernel<DK, DV, false>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    const dim3 grid(1, a.H, a.nseq);
+    const dim3 grid(a.vblocks, a.H, a.nseq);
     kern<<<grid, L::THREADS, smem, st>>>(mq, mk, mv, a.log_alpha, a.beta, a.S0,
                                        static_cast<__nv_bfloat16 *>(a.out), a.S_final, a.cu, a.T, a.H,
                                        a.flags, a.a_scale, a.b_scale, a.G);
@@ -1189,18 +1194,21 @@ __global__ void __launch_bounds__(256) seg_combine_kernel(const float *__restric
     }
 }
 
+// vblocks > 1: a value head of vblocks x DV columns, one CTA per column block (no segment scan;
+// the column blocks already multiply the CTAs per chain)
 template <int DK, int DV>
-cudaError_t run_chunk(const ChunkArgs &a, cudaStream_t st)
+cudaError_t run_chunk(const ChunkArgs &a, cudaStream_t st, int vblocks = 1)
 {
     const long tokens = a.cu_seqlens ? (long)a.T : (long)a.B * a.T;
-    const SegPlan p = plan_segments(a.B, a.T, a.H, a.cu_seqlens != nullptr, a.dtype);
+    const SegPlan p = vblocks > 1 ? SegPlan{} : plan_segments(a.B, a.T, a.H, a.cu_seqlens != nullptr, a.dtype);
     const int pf = a.prologue ? kFlagPrologue : 0;
     const float as = a.a_scale, bs = a.b_scale;
     if (p.G <= 1) {
         const int lf = (a.cu_seqlens && a.B <= TcCfg<DK, DV>::THREADS) ? kFlagLongestFirst : 0;
-        return launch_tc<DK, DV>(TcLaunch{a.q, a.k, a.v, a.log_alpha, a.beta, a.S0, a.out, a.S_final,
-                                          a.cu_seqlens, a.B, a.T, a.H, tokens, pf | lf, as, bs, a.G},
-                                 st);
+        TcLaunch t{a.q, a.k, a.v, a.log_alpha, a.beta, a.S0, a.out, a.S_final,
+                   a.cu_seqlens, a.B, a.T, a.H, tokens, pf | lf, as, bs, a.G};
+        t.vblocks = vblocks;
+        return launch_tc<DK, DV>(t, st);
     }
     const SegWork w = seg_layout(a.workspace, a.B, a.H, DK, DV, p);
     const int nseg = a.B * p.G;
@@ -1234,6 +1242,7 @@ cudaError_t run_chunk(const ChunkArgs &a, cudaStream_t st)
 
 size_t chunk_tc_workspace_bytes(int B, int T, int H, int dk, int dv, int varlen, int dtype)
 {
+    if (dv > 128) return 0;  // column blocks, no segment scan
     const SegPlan p = plan_segments(B, T, H, varlen, dtype);
     if (p.G <= 1) return 0;
     return seg_layout(nullptr, B, H, dk, dv, p).bytes;
@@ -1241,6 +1250,7 @@ size_t chunk_tc_workspace_bytes(int B, int T, int H, int dk, int dv, int varlen,
 
 cudaError_t launch_chunk_tc(const ChunkArgs &a, cudaStream_t stream)
 {
+    if (a.dv == 256) return a.dk == 128 ? run_chunk<128, 128>(a, stream, 2) : run_chunk<64, 128>(a, stream, 2);
     if (a.dk == 128 && a.dv == 128) return run_chunk<128, 128>(a, stream);
     if (a.dk == 128 && a.dv == 64) return run_chunk<128, 64>(a, stream);
     if (a.dk == 64 && a.dv == 128) return run_chunk<64, 128>(a, stream);

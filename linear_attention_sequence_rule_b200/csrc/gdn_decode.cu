@@ -13,6 +13,8 @@
 // arithmetic (dk*dv*4 bytes in flight per CTA), the two column sums S^T k and S^T q are reduced
 // across row groups through shared memory, and the updated state is written back with
 // streaming stores.  The state is touched by no other CTA, so there is no inter-CTA traffic.
+// A value head of VB x DV columns runs as VB CTAs per state (blockIdx.y = column block): value
+// columns do not interact in the step, so each CTA updates its own columns of every row.
 #include <cuda_bf16.h>
 
 #include "gdn_internal.h"
@@ -31,7 +33,7 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(flo
 
 constexpr int kThreads = 256;
 
-template <int DK, int DV, typename TIn>
+template <int DK, int DV, int VB, typename TIn>
 __global__ void __launch_bounds__(kThreads, 2)
 decode_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const TIn *__restrict__ v,
               const float *__restrict__ log_alpha, const float *__restrict__ beta,
@@ -41,6 +43,7 @@ decode_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const TIn *_
     constexpr int RPP = kThreads / TPR;  // rows covered per pass
     constexpr int R = DK / RPP;          // rows per thread
     static_assert(R * RPP == DK, "row split");
+    constexpr int LDV = VB * DV;         // row length of v, out and the state
 
     __shared__ float4 red_r[RPP][TPR];
     __shared__ float4 red_s[RPP][TPR];
@@ -50,11 +53,12 @@ decode_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const TIn *_
     const int tid = threadIdx.x;
     const int c4 = tid % TPR;
     const int rg = tid / TPR;  // row group: rows rg, rg + RPP, ...
+    const int col0 = VB == 1 ? 0 : (int)blockIdx.y * DV;
 
-    float4 *Sp = reinterpret_cast<float4 *>(S + u * (size_t)(DK * DV));
+    float4 *Sp = reinterpret_cast<float4 *>(S + u * (size_t)(DK * LDV) + col0);
     float4 s[R];
 #pragma unroll
-    for (int p = 0; p < R; ++p) s[p] = __ldcs(&Sp[(rg + p * RPP) * TPR + c4]);
+    for (int p = 0; p < R; ++p) s[p] = __ldcs(&Sp[(rg + p * RPP) * (LDV / 4) + c4]);
 
     // q/k of state (n, h) live at (n, h / G) among the H / G q/k heads (grouped value heads)
     const size_t uq = G == 1 ? u : (size_t)((unsigned)u / (unsigned)H) * (unsigned)(H / G) + ((unsigned)u % (unsigned)H) / (unsigned)G;
@@ -70,7 +74,7 @@ decode_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const TIn *_
     const float b = beta[u];
     float vv[4];
     {
-        const TIn *vp = v + u * DV + 4 * c4;
+        const TIn *vp = v + u * LDV + col0 + 4 * c4;
 #pragma unroll
         for (int j = 0; j < 4; ++j) vv[j] = to_f32(vp[j]);
     }
@@ -111,10 +115,10 @@ decode_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const TIn *_
         t.y = fmaf(a, s[p].y, kr[p] * u1);
         t.z = fmaf(a, s[p].z, kr[p] * u2);
         t.w = fmaf(a, s[p].w, kr[p] * u3);
-        __stcs(&Sp[(rg + p * RPP) * TPR + c4], t);
+        __stcs(&Sp[(rg + p * RPP) * (LDV / 4) + c4], t);
     }
     if (rg == 0) {
-        TIn *op = out + u * DV + 4 * c4;
+        TIn *op = out + u * LDV + col0 + 4 * c4;
         op[0] = from_f32<TIn>(fmaf(a, sq.x, kq * u0));
         op[1] = from_f32<TIn>(fmaf(a, sq.y, kq * u1));
         op[2] = from_f32<TIn>(fmaf(a, sq.z, kq * u2));
@@ -131,10 +135,13 @@ cudaError_t launch_typed(const void *q, const void *k, const void *v, const floa
     const TIn *Q = static_cast<const TIn *>(q), *K = static_cast<const TIn *>(k),
               *V = static_cast<const TIn *>(v);
     TIn *O = static_cast<TIn *>(out);
-    if (dk == 128 && dv == 128) decode_kernel<128, 128, TIn><<<grid, block, 0, st>>>(Q, K, V, la, be, S, O, H, G);
-    else if (dk == 128 && dv == 64) decode_kernel<128, 64, TIn><<<grid, block, 0, st>>>(Q, K, V, la, be, S, O, H, G);
-    else if (dk == 64 && dv == 128) decode_kernel<64, 128, TIn><<<grid, block, 0, st>>>(Q, K, V, la, be, S, O, H, G);
-    else decode_kernel<64, 64, TIn><<<grid, block, 0, st>>>(Q, K, V, la, be, S, O, H, G);
+    const dim3 grid2(NH, 2);  // dv = 256: two 128-column blocks per state
+    if (dk == 128 && dv == 256) decode_kernel<128, 128, 2, TIn><<<grid2, block, 0, st>>>(Q, K, V, la, be, S, O, H, G);
+    else if (dk == 64 && dv == 256) decode_kernel<64, 128, 2, TIn><<<grid2, block, 0, st>>>(Q, K, V, la, be, S, O, H, G);
+    else if (dk == 128 && dv == 128) decode_kernel<128, 128, 1, TIn><<<grid, block, 0, st>>>(Q, K, V, la, be, S, O, H, G);
+    else if (dk == 128 && dv == 64) decode_kernel<128, 64, 1, TIn><<<grid, block, 0, st>>>(Q, K, V, la, be, S, O, H, G);
+    else if (dk == 64 && dv == 128) decode_kernel<64, 128, 1, TIn><<<grid, block, 0, st>>>(Q, K, V, la, be, S, O, H, G);
+    else decode_kernel<64, 64, 1, TIn><<<grid, block, 0, st>>>(Q, K, V, la, be, S, O, H, G);
     return cudaGetLastError();
 }
 

@@ -48,7 +48,9 @@ def chunk(**kw):
 @pytest.mark.parametrize("kw,code", [
     (dict(dtype=7), gdn.GDN_ERR_UNSUPPORTED),
     (dict(dk=96), gdn.GDN_ERR_UNSUPPORTED),
-    (dict(dv=256), gdn.GDN_ERR_UNSUPPORTED),
+    (dict(dv=192), gdn.GDN_ERR_UNSUPPORTED),
+    (dict(dv=256, dtype=gdn.GDN_DTYPE_F32), gdn.GDN_ERR_UNSUPPORTED),
+    (dict(dv=512), gdn.GDN_ERR_UNSUPPORTED),
     (dict(chunk=32), gdn.GDN_ERR_UNSUPPORTED),
     (dict(B=0), gdn.GDN_ERR_INVALID_ARGUMENT),
     (dict(H=0), gdn.GDN_ERR_INVALID_ARGUMENT),
@@ -111,6 +113,9 @@ def test_workspace_query():
     assert gdn.gdn_chunk_fwd_workspace_bytes(1, 64, 1, 96, 64, 64, 0, 1) == bad
     assert gdn.gdn_chunk_fwd_workspace_bytes(0, 64, 1, 64, 64, 64, 0, 1) == bad
     assert gdn.gdn_chunk_fwd_workspace_bytes(1, 64, 1, 64, 64, 128, 0, 1) == bad
+    # value head size 256: bf16 only, as column blocks (no segment scan, so no workspace)
+    assert gdn.gdn_chunk_fwd_workspace_bytes(1, 4096, 1, 128, 256, 64, 0, 1) == 0
+    assert gdn.gdn_chunk_fwd_workspace_bytes(1, 64, 1, 128, 256, 64, 0, 0) == bad
 
 
 def decode(**kw):
@@ -123,6 +128,8 @@ def decode(**kw):
 @pytest.mark.parametrize("kw,code", [
     (dict(dtype=3), gdn.GDN_ERR_UNSUPPORTED),
     (dict(dk=32), gdn.GDN_ERR_UNSUPPORTED),
+    (dict(dk=256), gdn.GDN_ERR_UNSUPPORTED),
+    (dict(dv=192), gdn.GDN_ERR_UNSUPPORTED),
     (dict(N=0), gdn.GDN_ERR_INVALID_ARGUMENT),
     (dict(H=-1), gdn.GDN_ERR_INVALID_ARGUMENT),
     (dict(S_inout=None), gdn.GDN_ERR_INVALID_ARGUMENT),
