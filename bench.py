@@ -476,6 +476,10 @@ def run_ours(args, world, rank, local):
                                   "launches_per_call": 1}
         del dg, outg, Sg
         extra["hybrid_lm_backward"] = backward_numbers(gdn, d, 5, 3, flush, stream, peaks)
+        dw = to_dev(workloads.make_chunk_inputs(B=8, T=4096, H=12, dk=64, dv=128, dtype="bf16",
+                                                seed=rank_seed(cfg["seed"], rank), la_scale=0.1))
+        extra["hybrid_lm_backward_dv128"] = backward_numbers(gdn, dw, 3, 3, flush, stream, peaks)
+        del dw
         extra["phase_memory"] = phase_numbers(gdn, 5, 3, flush, stream, peaks)
         extra["decode_small_batch_graph"] = decode_graph_numbers(gdn)
     cpu = None
@@ -543,26 +547,31 @@ def _time_loop(call, steps, warmup, flush, stream):
 
 def backward_numbers(gdn, d, steps, warmup, flush, stream, peaks):
     """The backward of the hybrid-LM step (dq, dk, dv, gate and state gradients; fp32-accurate
-    products on the tensor cores as three tf32 terms) from a seeded dout; `d` holds the hybrid-LM
-    inputs on the device."""
+    products on the tensor cores as three tf32 terms) from a seeded dout; `d` holds inputs of the
+    hybrid-LM token and head counts (B=8 T=4096 H=12, dk=64) on the device, dv = 64 VS."""
+    dv = d["v"].shape[-1]
+    VS = dv // 64
     dout = torch.randn(d["v"].shape, device="cuda", generator=torch.Generator("cuda").manual_seed(7)).to(d["v"].dtype)
-    wsb = torch.empty(gdn.gdn_chunk_bwd_workspace_bytes(8, 4096, 12, 64, 64, 64, 0), dtype=torch.uint8,
+    wsb = torch.empty(gdn.gdn_chunk_bwd_workspace_bytes(8, 4096, 12, 64, dv, 64, 0), dtype=torch.uint8,
                       device="cuda")
 
     def call():
         gdn.chunk_bwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], dout, workspace=wsb, stream=stream)
     ms_b = _time_loop(call, steps, warmup, flush, stream)
     # bytes per token-head: q, k, v, dout (bf16) and gates in; dq, dk, dv (fp32) and two gate grads out
-    by_b = 393216 * (4 * 64 * 2 + 8 + 3 * 64 * 4 + 8)
+    by_b = 393216 * (2 * 64 * 2 + 2 * dv * 2 + 8 + 2 * 64 * 4 + dv * 4 + 8)
     # algorithmic work: the 26 distinct 64 x 64 x 64 products the chunk-form backward needs per
-    # (chunk, head), each counted once -- 8 forming T, W, U~, M, Bm, R; 1 in each scan; 16 for the
-    # gradients -- at 2 * 64^3 fp32 flops each (the gradient kernel's recomputed K K^T and Q K^T are
-    # not counted); the tensor cores execute three tf32 products for each
-    fl_b = 6144 * 26 * 2 * 64 ** 3
+    # (chunk, head) at dv = 64, each counted once -- 8 forming T, W, U~, M, Bm, R; 1 in each scan; 16
+    # for the gradients -- at 2 * 64^3 fp32 flops each (the gradient kernel's recomputed K K^T and
+    # Q K^T are not counted); the tensor cores execute three tf32 products for each.  14 of them
+    # have a value dimension and scale with dv / 64, 12 do not (value splits recompute those per
+    # 64-column block: executed work is 26 VS products, counted here once)
+    fl_b = 6144 * (12 + 14 * VS) * 2 * 64 ** 3
+    launches = 3 + (2 if VS > 1 else 0)
     tf32_peak = peaks["bf16_tflops"] * TF32_PER_BF16
-    return {"workload": "hybrid_lm backward: dq, dk, dv, dlog_alpha, dbeta (fp32) from dout",
+    return {"workload": f"hybrid_lm backward: dq, dk, dv, dlog_alpha, dbeta (fp32) from dout; dk=64, dv={dv}",
             "ms": round(ms_b, 6), "tokens_per_s": round(32768 / (ms_b * 1e-3), 1),
-            "launches_per_call": 3, "algo_bytes": by_b,
+            "launches_per_call": launches, "algo_bytes": by_b,
             "gbs": round(by_b / (ms_b * 1e-3) / 1e9, 3),
             "hbm_frac": round(by_b / (ms_b * 1e-3) / 1e9 / peaks["hbm_gbs"], 5),
             "algo_flops_fp32": fl_b,
@@ -647,6 +656,10 @@ def run_only(args):
         flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device="cuda")
         r = backward_numbers(gdn, to_dev(workloads.config_inputs("hybrid_lm")), args.steps, args.warmup, flush,
                              stream, peaks)
+    elif args.only == "hybrid_lm_backward_dv128":
+        flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device="cuda")
+        d = to_dev(workloads.make_chunk_inputs(B=8, T=4096, H=12, dk=64, dv=128, dtype="bf16", seed=0, la_scale=0.1))
+        r = backward_numbers(gdn, d, args.steps, args.warmup, flush, stream, peaks)
     elif args.only == "phase_memory":
         flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device="cuda")
         r = phase_numbers(gdn, args.steps, args.warmup, flush, stream, peaks)
@@ -729,7 +742,7 @@ def main():
     ap.add_argument("--quick", action="store_true", help="main workload only")
     ap.add_argument("--only", choices=["hybrid_lm", "long_context", "varlen", "tiny", "decode", "hybrid_lm_fused",
                                              "hybrid_lm_unfused", "hybrid_lm_backward", "phase_memory",
-                                             "hybrid_lm_dv256"],
+                                             "hybrid_lm_dv256", "hybrid_lm_backward_dv128"],
                     help="time one workload's kernel loop only (for profiler runs)")
     args = ap.parse_args()
     if args.warmup < 3:

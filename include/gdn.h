@@ -223,11 +223,11 @@ GDN_API int gdn_phase_fwd(const float *K, const float *Q, const void *v, const f
 GDN_API size_t gdn_phase_fwd_workspace_bytes(int B, int T, int H, int dk, int dv, int varlen, int dtype);
 
 /*
- * gdn_phase_bwd -- gradients of gdn_phase_fwd for dk = 32 complex (64 real) and dv = 64: given the
- * forward's inputs, dout = dL/dout (dtype) and dM_final = dL/dM_final ((re, im) pairs, NULL: zero),
- * it writes fp32
- *     dK, dQ [.., H, 32, 2] (d/dRe, d/dIm pairs), dv [.., H, 64], dlog_lam, dbeta [.., H],
- *     dM0 [B, H, 64, 32, 2] (NULL: not written).
+ * gdn_phase_bwd -- gradients of gdn_phase_fwd for dk = 32 complex (64 real) and dv in {64, 128}:
+ * given the forward's inputs, dout = dL/dout (dtype) and dM_final = dL/dM_final ((re, im) pairs,
+ * NULL: zero), it writes fp32
+ *     dK, dQ [.., H, 32, 2] (d/dRe, d/dIm pairs), dv [.., H, dv], dlog_lam, dbeta [.., H],
+ *     dM0 [B, H, dv, 32, 2] (NULL: not written).
  * The fp32 backward of the real recurrence runs on the map gdn_phase_fwd uses (see gdn_phase.cu),
  * followed by its chain rule.  Workspace: gdn_phase_bwd_workspace_bytes(...), 256-byte aligned.
  */
@@ -243,10 +243,12 @@ GDN_API size_t gdn_phase_bwd_workspace_bytes(int B, int T, int H, int dk, int dv
 /*
  * gdn_chunk_bwd -- gradients of gdn_chunk_fwd (the training path; Sykra README, "Architectural
  * Highlights": chunk-parallel training through the WY / unit triangular transform), for
- * dk = dv = 64 and chunk = 64.  Given the forward's inputs (same layouts, dtype for q, k, v and
- * dout) and dout = dL/dout, dS_final = dL/dS_final (NULL: zero), it writes
- *     dq, dk [.., H, 64], dv [.., H, 64], dlog_alpha, dbeta [.., H]   (fp32, always)
- *     dS0 [B, H, 64, 64] fp32 (NULL: not written)
+ * dk = 64, dv in {64, 128, 256} and chunk = 64.  Given the forward's inputs (same layouts, dtype
+ * for q, k, v and dout) and dout = dL/dout, dS_final = dL/dS_final (NULL: zero), it writes
+ *     dq, dk [.., H, 64], dv [.., H, dv], dlog_alpha, dbeta [.., H]   (fp32, always)
+ *     dS0 [B, H, 64, dv] fp32 (NULL: not written)
+ * A value head of dv = 64 VS columns runs as VS heads of 64 columns that share q, k and the gates
+ * (value columns never interact); their dq, dk, dlog_alpha and dbeta are summed.
  * Computed from the chunk form with fp32-level accuracy: the 64 x 64 products run on the tensor
  * cores as three tf32 products (x = hi + lo; a b ~ hi hi + hi lo + lo hi), everything else in
  * fp32.  Every chunk's state map
@@ -254,7 +256,8 @@ GDN_API size_t gdn_phase_bwd_workspace_bytes(int B, int T, int H, int dk, int dv
  * parallel, two scans over each sequence's chunks give the entry states and exit gradients, and
  * every chunk's input gradients are then formed in parallel.  log_alpha = -inf (an exact reset)
  * gets dlog_alpha = 0.  Workspace: gdn_chunk_bwd_workspace_bytes(...) bytes, 256-byte aligned
- * (eight 16 KB matrices per chunk and head).  Errors as gdn_chunk_fwd; other head sizes return
+ * (eight 16 KB matrices per chunk, head and 64-column value block, plus the partial q/k and
+ * gate gradients when dv > 64).  Errors as gdn_chunk_fwd; other head sizes return
  * GDN_ERR_UNSUPPORTED.
  */
 GDN_API int gdn_chunk_bwd(const void *q, const void *k, const void *v, const float *log_alpha,
@@ -268,7 +271,7 @@ GDN_API size_t gdn_chunk_bwd_workspace_bytes(int B, int T, int H, int dk, int dv
 
 /*
  * gdn_chunk_bwd_gva -- gdn_chunk_bwd with grouped value heads (see gdn_chunk_fwd_gva): q, k
- * [.., Hk, 64]; v, dout [.., Hv, 64]; gates [.., Hv]; states [B, Hv, 64, 64]; value head h reads
+ * [.., Hk, 64]; v, dout [.., Hv, dv]; gates [.., Hv]; states [B, Hv, 64, dv]; value head h reads
  * q/k head h / (Hv / Hk).  dq, dk [.., Hk, 64] are the sums over each q/k head's Hv / Hk value
  * heads; dv, dlog_alpha, dbeta, dS0 stay per value head.  Workspace:
  * gdn_chunk_bwd_gva_workspace_bytes(...) (gdn_chunk_bwd's plus per-value-head dq and dk).

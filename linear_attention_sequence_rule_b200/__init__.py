@@ -427,7 +427,7 @@ def phase_fwd(K, Q, v, log_lam, beta, M0=None, cu_seqlens=None, out=None, M_fina
 
 def phase_bwd(K, Q, v, log_lam, beta, dout, M0=None, dM_final=None, cu_seqlens=None, want_dM0=True,
               workspace=None, stream=None):
-    """Gradients of ``phase_fwd`` (dk = 32 complex, dv = 64): returns (dK, dQ complex64, dv fp32,
+    """Gradients of ``phase_fwd`` (dk = 32 complex, dv 64 or 128): returns (dK, dQ complex64, dv fp32,
     dlog_lam, dbeta fp32, dM0 complex64 or None); complex gradients as d/dRe + i d/dIm."""
     Kp, Qp = _as_pairs(K, "K"), _as_pairs(Q, "Q")
     dt = v.dtype
@@ -507,7 +507,7 @@ def chunk_fwd_gva(q, k, v, log_alpha, beta, S0=None, cu_seqlens=None, out=None, 
 
 def chunk_bwd(q, k, v, log_alpha, beta, dout, S0=None, dS_final=None, cu_seqlens=None, want_dS0=True,
               workspace=None, chunk=64, stream=None):
-    """Gradients of ``chunk_fwd`` (dk = dv = 64): returns fp32 (dq, dk, dv, dlog_alpha, dbeta,
+    """Gradients of ``chunk_fwd`` (dk = 64, dv in {64, 128, 256}): returns fp32 (dq, dk, dv, dlog_alpha, dbeta,
     dS0 or None) for dout = dL/dout and dS_final = dL/dS_final (None: zero)."""
     dt = q.dtype
     if dt not in _DT:

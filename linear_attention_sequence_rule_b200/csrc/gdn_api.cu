@@ -38,12 +38,14 @@ static int cuda_fail(cudaError_t e, const char *where)
 
 static bool head_dim_ok(int d) { return d == 64 || d == 128; }
 
-// Shared shape/type checks of the chunk forward; returns GDN_OK or an error code.
-static int check_chunk_shape(int B, int T, int H, int dk, int dv, int chunk, int varlen, int dtype)
+// Shared shape/type checks of the chunk forward (and, without the forward's head sizes, of the
+// backward); returns GDN_OK or an error code.
+static int check_chunk_shape(int B, int T, int H, int dk, int dv, int chunk, int varlen, int dtype,
+                             bool fwd_heads = true)
 {
     if (dtype != GDN_DTYPE_BF16 && dtype != GDN_DTYPE_F32)
         return fail(GDN_ERR_UNSUPPORTED, "gdn_chunk_fwd: unknown dtype %d", dtype);
-    if (!head_dim_ok(dk) || !(head_dim_ok(dv) || (dv == 256 && dtype == GDN_DTYPE_BF16)))
+    if (fwd_heads && (!head_dim_ok(dk) || !(head_dim_ok(dv) || (dv == 256 && dtype == GDN_DTYPE_BF16))))
         return fail(GDN_ERR_UNSUPPORTED,
                     "gdn_chunk_fwd: dk=%d dv=%d, supported: dk 64 or 128, dv 64 or 128 (256 with bf16)", dk, dv);
     if (chunk != 64)
@@ -262,17 +264,20 @@ int gdn_device_status(void *stream)
 
 }  // extern "C"
 
+// Head sizes of the backward: dk = 64, dv = 64 VS with VS in {1, 2, 4} (value splits).
+static bool bwd_heads_ok(int dk, int dv) { return dk == 64 && (dv == 64 || dv == 128 || dv == 256); }
+
 size_t gdn_chunk_bwd_workspace_bytes(int B, int T, int H, int dk, int dv, int chunk, int varlen)
 {
-    if (dk != 64 || dv != 64 || chunk != 64 || B < 1 || H < 1 || T < 0 || (!varlen && T < 1)) return (size_t)-1;
-    return chunk_bwd_workspace_bytes(B, T, H, varlen);
+    if (!bwd_heads_ok(dk, dv) || chunk != 64 || B < 1 || H < 1 || T < 0 || (!varlen && T < 1)) return (size_t)-1;
+    return chunk_bwd_workspace_bytes(B, T, H, varlen, 1, dv / 64);
 }
 
 size_t gdn_chunk_bwd_gva_workspace_bytes(int B, int T, int Hk, int Hv, int dk, int dv, int chunk, int varlen)
 {
     if (Hk < 1 || Hv < 1 || Hv % Hk != 0) return (size_t)-1;
-    if (dk != 64 || dv != 64 || chunk != 64 || B < 1 || T < 0 || (!varlen && T < 1)) return (size_t)-1;
-    return chunk_bwd_workspace_bytes(B, T, Hv, varlen, Hv / Hk);
+    if (!bwd_heads_ok(dk, dv) || chunk != 64 || B < 1 || T < 0 || (!varlen && T < 1)) return (size_t)-1;
+    return chunk_bwd_workspace_bytes(B, T, Hv, varlen, Hv / Hk, dv / 64);
 }
 
 namespace gdn {
@@ -285,10 +290,10 @@ static int chunk_bwd_common(const char *fn, const void *q, const void *k, const 
                             void *workspace, size_t workspace_bytes, void *stream)
 {
     const int varlen = cu_seqlens != nullptr;
-    int rc = check_chunk_shape(B, T, H, dk_, dv_, chunk, varlen, dtype);
+    if (!bwd_heads_ok(dk_, dv_))
+        return fail(GDN_ERR_UNSUPPORTED, "%s: dk=%d dv=%d, supported: dk 64, dv 64, 128 or 256", fn, dk_, dv_);
+    int rc = check_chunk_shape(B, T, H, dk_, dv_, chunk, varlen, dtype, false);
     if (rc != GDN_OK) return rc;
-    if (dk_ != 64 || dv_ != 64)
-        return fail(GDN_ERR_UNSUPPORTED, "%s: dk=%d dv=%d, supported: 64", fn, dk_, dv_);
     if (!q || !k || !v || !log_alpha || !beta || !dout || !dq || !dk || !dv || !dlog_alpha || !dbeta)
         return fail(GDN_ERR_INVALID_ARGUMENT, "%s: inputs, dout and every gradient output except dS0 are required",
                     fn);
@@ -296,14 +301,15 @@ static int chunk_bwd_common(const char *fn, const void *q, const void *k, const 
                           cu_seqlens};
     for (const void *p : ptrs)
         if (p && !aligned16(p)) return fail(GDN_ERR_INVALID_ARGUMENT, "%s: pointer %p is not 16-byte aligned", fn, p);
-    const size_t need = chunk_bwd_workspace_bytes(B, T, H, varlen, G);
+    const int VS = dv_ / 64;
+    const size_t need = chunk_bwd_workspace_bytes(B, T, H, varlen, G, VS);
     if (!workspace || workspace_bytes < need)
         return fail(GDN_ERR_WORKSPACE, "%s: workspace of %zu bytes needed, %zu given", fn, need,
                     workspace ? workspace_bytes : (size_t)0);
     if (reinterpret_cast<uintptr_t>(workspace) & 255u)
         return fail(GDN_ERR_INVALID_ARGUMENT, "%s: workspace must be 256-byte aligned", fn);
     BwdArgs a{q, k, v, log_alpha, beta, S0, dout, dS_final, dq, dk, dv, dlog_alpha, dbeta, dS0, cu_seqlens,
-              B, T, H, dtype, workspace, G};
+              B, T, H, dtype, workspace, G, VS};
     cudaError_t e = launch_chunk_bwd(a, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, fn);
     return GDN_OK;

@@ -1,6 +1,6 @@
 // gdn_chunk_bwd.cu -- gradients of the chunk forward (dq, dk, dv, dlog_alpha, dbeta, dS0) with
-// fp32-level accuracy, for dk = dv = 64 (the training path; Sykra README, "Architectural
-// Highlights": chunk-parallel training through the WY / UT transform).  The 64 x 64 products run
+// fp32-level accuracy, for dk = 64 and dv = 64 VS, VS in {1, 2, 4} (the training path; Sykra
+// README, "Architectural Highlights": chunk-parallel training through the WY / UT transform).  The 64 x 64 products run
 // on the tensor cores as three tf32 products each; the rest is fp32 on the CUDA cores.
 //
 // Per chunk of C = 64 tokens with entry state S (the forward's chunk form):
@@ -17,6 +17,11 @@
 //   bwd_grads  (chunk x head, parallel)  : with S_c and dS_{c+1}, every input gradient of the chunk
 // All matrices are 64 x 64 fp32 in shared memory (XOR-swizzled rows); 256 threads; a product
 // leaves each thread 16 results in the tensor cores' fragment layout (see mm_core).
+// Value splits: the recurrence never mixes value columns (column j of S, O and dS follows from
+// column j of V, S0 and dO alone), so a value head of 64 VS columns runs as VS virtual heads of 64
+// columns, hx = h VS + block, that share q, k and the gates.  Their dv and dS0 are disjoint column
+// blocks of the outputs; their dq, dk, dbeta and dlog_alpha are partial sums, added up at the end
+// (with the grouped-value-head sums when value heads also share q/k heads).
 #include <cuda_bf16.h>
 #include <math.h>
 
@@ -363,6 +368,34 @@ __device__ __forceinline__ void mat_from_shared(float *dst, const float *M, int 
     }
 }
 
+// A 64 x 64 block of a row-major fp32 matrix whose rows are `ld` floats apart, to and from a
+// shared matrix (ld = 64: the dense forms above).
+__device__ __forceinline__ void mat_to_shared_ld(float *M, const float *src, int ld, int t)
+{
+    constexpr int PER = MAT / 4 / kThreads;
+    float4 b[PER];
+#pragma unroll
+    for (int u = 0; u < PER; ++u) {
+        const int e = (t + u * kThreads) * 4;
+        b[u] = __ldg(reinterpret_cast<const float4 *>(src + (size_t)(e >> 6) * ld + (e & 63)));
+    }
+#pragma unroll
+    for (int u = 0; u < PER; ++u) {
+        const int e = (t + u * kThreads) * 4;
+        *reinterpret_cast<float4 *>(&M[sw(e >> 6, e & 63)]) = b[u];
+    }
+}
+
+__device__ __forceinline__ void mat_from_shared_ld(float *dst, const float *M, int ld, int t)
+{
+#pragma unroll
+    for (int u = 0; u < MAT / 4 / kThreads; ++u) {
+        const int e = (t + u * kThreads) * 4;
+        *reinterpret_cast<float4 *>(dst + (size_t)(e >> 6) * ld + (e & 63)) =
+            *reinterpret_cast<const float4 *>(&M[sw(e >> 6, e & 63)]);
+    }
+}
+
 // T = (I + A)^{-1} for strictly lower A, given transposed (At(i, r) = A(r, i); only i < r is read).
 // Column c of T is found by forward substitution on the kSolveLanes = L threads Lc .. Lc + L - 1,
 // thread Lc + q holding rows q, q + L, q + 2L, ...: once row j is final it is passed among the L
@@ -395,14 +428,15 @@ template <typename TIn>
 __global__ void __launch_bounds__(kThreads, 2)
     bwd_prep(const TIn *__restrict__ q, const TIn *__restrict__ k, const TIn *__restrict__ v,
              const float *__restrict__ log_alpha, const float *__restrict__ beta, const TIn *__restrict__ dout,
-             const int32_t *__restrict__ cu, const int32_t *__restrict__ off, int nseq, int T, int H, int G,
+             const int32_t *__restrict__ cu, const int32_t *__restrict__ off, int nseq, int T, int H, int G, int VS,
              float *__restrict__ Mo, float *__restrict__ Bo, float *__restrict__ Ro, float *__restrict__ Tw,
              float *__restrict__ Ww, float *__restrict__ Uw)
 {
     float *K = smf, *B1 = K + MAT, *B2 = B1 + MAT, *P = B2 + MAT, *B4 = P + MAT, *B5 = B4 + MAT;
     Gates &g = *reinterpret_cast<Gates *>(B5 + MAT);
     float *bg = reinterpret_cast<float *>(&g + 1);  // beta gam
-    const int t = threadIdx.x, h = blockIdx.y, e = blockIdx.x;
+    // virtual head hx = h VS + value block; v, dout are [tokens, H VS, 64] in these terms
+    const int t = threadIdx.x, hx = blockIdx.y, Hx = H * VS, h = VS == 1 ? hx : hx / VS, e = blockIdx.x;
     const ChunkRef c = chunk_ref(e, cu, off, nseq, T);
     if (c.n == 0) return;
     // grouped value heads: value head h reads q/k head h / G of H / G
@@ -412,7 +446,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         RowTile<TIn> tk, tq;
         tk.fetch(k, c, Hq, hq, t);
         tq.fetch(q, c, Hq, hq, t);
-        tv.fetch(v, c, H, h, t);
+        tv.fetch(v, c, Hx, hx, t);
         tk.put(K, t);
         tq.put(B1, t);  // Q
     }
@@ -426,7 +460,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     tv.put(B1, t);  // V over Q (Q comes back for X)
     unit_lower_inverse(B2, B4, t);  // T in B4
     __syncthreads();
-    const size_t base = ((size_t)e * H + h) * (size_t)(N * N);
+    const size_t base = ((size_t)e * Hx + hx) * (size_t)(N * N);
     mat_from_shared(Tw + base, B4, t);  // T for the gradient kernel
     mm<false, false>(B4, K, t, [&](int r, int m, float x, int) { B2[sw(r, m)] = x; }, bg);       // W over A^T
     mm<false, false>(B4, B1, t, [&](int r, int j, float x, int) { B5[sw(r, j)] = x; }, g.bet);   // U~
@@ -434,7 +468,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     {
         RowTile<TIn> tq, td;
         tq.fetch(q, c, Hq, hq, t);
-        td.fetch(dout, c, H, h, t);
+        td.fetch(dout, c, Hx, hx, t);
         mat_from_shared(Ww + base, B2, t);  // W and U~ for the gradient kernel
         mat_from_shared(Uw + base, B5, t);
         tq.put(B1, t);  // Q again, over V
@@ -468,20 +502,23 @@ __device__ __forceinline__ void seq_chunks(int s, const int32_t *cu, const int32
 // Xc[c] = dL/dS at the end of chunk c, Xend = dS0.
 // X is double-buffered in shared memory, and so is M_c; chunk c + 2's M and additive term are
 // loaded into registers while chunk c is multiplied, so one barrier per chunk remains.
+// X0 and Xend are [B, H, 64, 64 VS] (the caller's states); this chain takes the 64 columns of
+// value block hx mod VS.
 template <bool REV>
 __device__ __forceinline__ void scan_body(const float *__restrict__ Mo, const float *__restrict__ Add,
                                           const float *__restrict__ X0, const int32_t *__restrict__ cu,
-                                          const int32_t *__restrict__ off, int T, int H, float *__restrict__ Xc,
-                                          float *__restrict__ Xend)
+                                          const int32_t *__restrict__ off, int T, int H, int VS,
+                                          float *__restrict__ Xc, float *__restrict__ Xend)
 {
     // shared memory: X[2], then M[2]
-    const int t = threadIdx.x, h = blockIdx.x, s = blockIdx.y;
+    const int t = threadIdx.x, hx = blockIdx.x, s = blockIdx.y, Hx = H * VS;
     const int g = (t & 31) >> 2, q = t & 3, m0 = ((t >> 5) & 3) * 16, n0 = (t >> 7) * 8 * kNT;
     constexpr int PER = MAT / 4 / kThreads;  // float4 pieces of a matrix per thread
     int first, count;
     seq_chunks(s, cu, off, T, first, count);
-    const size_t st0 = ((size_t)s * H + h) * (size_t)MAT;
-    auto chunk_base = [&](int i) { return ((size_t)(first + (REV ? count - 1 - i : i)) * H + h) * (size_t)MAT; };
+    const int ld = N * VS;  // row stride of the caller's states
+    const size_t st0 = ((size_t)s * H + hx / VS) * (size_t)N * ld + (size_t)(hx % VS) * N;
+    auto chunk_base = [&](int i) { return ((size_t)(first + (REV ? count - 1 - i : i)) * Hx + hx) * (size_t)MAT; };
     auto fetch_m = [&](int i, float4 (&m)[PER]) {
         const float4 *src = reinterpret_cast<const float4 *>(Mo + chunk_base(i));
 #pragma unroll
@@ -505,7 +542,7 @@ __device__ __forceinline__ void scan_body(const float *__restrict__ Mo, const fl
     float4 pm[PER];
     float2 pa[2 * kNT], pa2[2 * kNT];
     if (X0) {
-        mat_to_shared(smf, X0 + st0, t);
+        mat_to_shared_ld(smf, X0 + st0, ld, t);
     } else {
 #pragma unroll
         for (int u = 0; u < PER; ++u) reinterpret_cast<float4 *>(smf)[t + u * kThreads] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -540,7 +577,7 @@ __device__ __forceinline__ void scan_body(const float *__restrict__ Mo, const fl
         }
         __syncthreads();
     }
-    if (Xend) mat_from_shared(Xend + st0, smf + (count & 1) * MAT, t);
+    if (Xend) mat_from_shared_ld(Xend + st0, smf + (count & 1) * MAT, ld, t);
 }
 
 // Both scans in one launch, blockIdx.z = 0 forward and 1 reverse: they are independent, and with
@@ -548,11 +585,11 @@ __device__ __forceinline__ void scan_body(const float *__restrict__ Mo, const fl
 __global__ void __launch_bounds__(kThreads, 2)
     bwd_scans(const float *__restrict__ Mo, const float *__restrict__ Bo, const float *__restrict__ Ro,
               const float *__restrict__ S0, const float *__restrict__ dS_final, const int32_t *__restrict__ cu,
-              const int32_t *__restrict__ off, int T, int H, float *__restrict__ Sc, float *__restrict__ dSn,
-              float *__restrict__ dS0)
+              const int32_t *__restrict__ off, int T, int H, int VS, float *__restrict__ Sc,
+              float *__restrict__ dSn, float *__restrict__ dS0)
 {
-    if (blockIdx.z == 0) scan_body<false>(Mo, Bo, S0, cu, off, T, H, Sc, nullptr);
-    else scan_body<true>(Mo, Ro, dS_final, cu, off, T, H, dSn, dS0);
+    if (blockIdx.z == 0) scan_body<false>(Mo, Bo, S0, cu, off, T, H, VS, Sc, nullptr);
+    else scan_body<true>(Mo, Ro, dS_final, cu, off, T, H, VS, dSn, dS0);
 }
 
 // ---- bwd_grads: every input gradient of one (chunk, head) --------------------------------------
@@ -570,7 +607,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               const float *__restrict__ log_alpha, const float *__restrict__ beta, const TIn *__restrict__ dout,
               const float *__restrict__ Sc, const float *__restrict__ dSn, const float *__restrict__ Tw,
               const float *__restrict__ Ww, const float *__restrict__ Uw, const int32_t *__restrict__ cu,
-              const int32_t *__restrict__ off, int nseq, int T, int H, int G, float *__restrict__ dq,
+              const int32_t *__restrict__ off, int nseq, int T, int H, int G, int VS, float *__restrict__ dq,
               float *__restrict__ dk, float *__restrict__ dv, float *__restrict__ dla, float *__restrict__ dbe)
 {
     float *K = smf, *Q = K + MAT, *V = Q + MAT, *dO = V + MAT, *S = dO + MAT, *dSp = S + MAT, *KK = dSp + MAT,
@@ -578,18 +615,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     Gates &g = *reinterpret_cast<Gates *>(X2 + MAT);
     float *vec = reinterpret_cast<float *>(&g + 1);
     float *bg = vec, *dG = vec + N, *dgam = vec + 2 * N, *dlam = vec + 3 * N, *dbet = vec + 4 * N, *dgC = vec + 5 * N;
-    const int t = threadIdx.x, h = blockIdx.y, e = blockIdx.x;
+    // virtual head hx = h VS + value block (see the file's head); dq, dk, dv are written as
+    // [tokens, H VS, 64] and dlog_alpha, dbeta as [tokens, H VS]
+    const int t = threadIdx.x, hx = blockIdx.y, Hx = H * VS, h = VS == 1 ? hx : hx / VS, e = blockIdx.x;
     const ChunkRef c = chunk_ref(e, cu, off, nseq, T);
     if (c.n == 0) return;
-    const size_t base = ((size_t)e * H + h) * (size_t)(N * N);
+    const size_t base = ((size_t)e * Hx + hx) * (size_t)(N * N);
     {
         // grouped value heads: value head h reads q/k head h / G of H / G (dq, dk per value head)
         const int Hq = G == 1 ? H : H / G, hq = G == 1 ? h : h / G;
         RowTile<TIn> tk, tq, tv, td;
         tk.fetch(k, c, Hq, hq, t);
         tq.fetch(q, c, Hq, hq, t);
-        tv.fetch(v, c, H, h, t);
-        td.fetch(dout, c, H, h, t);
+        tv.fetch(v, c, Hx, hx, t);
+        td.fetch(dout, c, Hx, hx, t);
         mat_to_shared(S, Sc + base, t);
         mat_to_shared(dSp, dSn + base, t);
         mat_to_shared(Tm, Tw + base, t);  // T = (I + A)^{-1}, W and U~ from the prep kernel
@@ -600,7 +639,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         tv.put(V, t);
         td.put(dO, t);
     }
-    if (t == 0) dgC[0] = 0.f;
     chunk_gates<TIn>(g, log_alpha, beta, c, H, h, t);
     __syncthreads();
     if (t < N) bg[t] = g.bet[t] * g.gam[t];
@@ -627,7 +665,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
-        if ((t & 31) == 0) atomicAdd(dgC, part);
+        if ((t & 31) == 0) dgC[t >> 5] = part;  // per warp, summed in warp order below (reproducible)
     }
     __syncthreads();
     // U = U~ - W S (U~ in U, W in dU, both loaded)
@@ -734,7 +772,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         float s63 = li[0] + li[1];
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) s63 += __shfl_xor_sync(0xffffffffu, s63, o);
-        if (t == 0) x[0] += s63 + dgC[0] * g.gam[N - 1];  // row 63
+        if (t == 0) {  // row 63
+            float dgc = 0.f;
+            for (int w = 0; w < kThreads / 32; ++w) dgc += dgC[w];
+            x[0] += s63 + dgc * g.gam[N - 1];
+        }
         seg_scan64(x[0], f[0], x[1], f[1], t);
 #pragma unroll
         for (int u = 0; u < 2; ++u) {
@@ -750,7 +792,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int hh = 0; hh < 2; ++hh) {
             const int r = m0 + gq + 8 * hh;
             if (r >= c.n) continue;
-            const size_t row = ((size_t)(c.tok + r) * H + h) * N + n0 + 2 * qq;
+            const size_t row = ((size_t)(c.tok + r) * Hx + hx) * N + n0 + 2 * qq;
 #pragma unroll
             for (int n = 0; n < kNT; ++n) {
                 const int u = 4 * n + 2 * hh;
@@ -761,7 +803,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     }
     if (t < c.n) {
-        const size_t o = (size_t)(c.tok + t) * H + h;
+        const size_t o = (size_t)(c.tok + t) * Hx + hx;
         dla[o] = dlam[t];
         dbe[o] = dbet[t];
     }
@@ -783,6 +825,22 @@ __global__ void bwd_group_sum(const float *__restrict__ gq, const float *__restr
     }
     dq[i] = sq;
     dk[i] = sk;
+}
+
+// Value splits: dlog_alpha, dbeta of value head i = the sum over its VS virtual heads
+// ([rows, H VS] -> [rows, H]); one thread per output element.
+__global__ void bwd_gate_sum(const float *__restrict__ pla, const float *__restrict__ pbe, float *__restrict__ dla,
+                             float *__restrict__ dbe, long out_elems, int VS)
+{
+    const long i = (long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= out_elems) return;
+    float sa = 0.f, sb = 0.f;
+    for (int u = 0; u < VS; ++u) {
+        sa += pla[i * VS + u];
+        sb += pbe[i * VS + u];
+    }
+    dla[i] = sa;
+    dbe[i] = sb;
 }
 
 // chunk offsets of varlen sequences: off[s] = sum over s' < s of ceil(len / 64); off[nseq] = total
@@ -812,27 +870,53 @@ long bwd_chunks(int B, int T, int varlen)
     return varlen ? (long)(T + N - 1) / N + B : (long)B * ((T + N - 1) / N);
 }
 
+// Workspace: chunk offsets, then eight matrices per (chunk, virtual head) -- M, Bm, R, S_c, dS_{c+1},
+// T, W, U~ -- then, when the q/k gradients are partial (G VS > 1), per-virtual-head dq and dk, and
+// when the gate gradients are partial (VS > 1), per-virtual-head dlog_alpha and dbeta.
+struct BwdLayout {
+    size_t off, mats, qk, gates, bytes;
+};
+
+BwdLayout bwd_layout(int B, int T, int H, int varlen, int G, int VS)
+{
+    BwdLayout l;
+    const size_t Hx = (size_t)H * VS, tokens = varlen ? (size_t)T : (size_t)B * T;
+    l.off = align256b((size_t)(B + 1) * sizeof(int32_t));
+    l.mats = align256b((size_t)bwd_chunks(B, T, varlen) * Hx * N * N * sizeof(float));
+    l.qk = G * VS > 1 ? align256b(tokens * Hx * N * sizeof(float)) : 0;
+    l.gates = VS > 1 ? align256b(tokens * Hx * sizeof(float)) : 0;
+    l.bytes = l.off + 8 * l.mats + 2 * l.qk + 2 * l.gates;
+    return l;
+}
+
 template <typename TIn>
 cudaError_t run_bwd(const BwdArgs &a, cudaStream_t st)
 {
     const int varlen = a.cu_seqlens != nullptr;
     const long chunks = bwd_chunks(a.B, a.T, varlen);
-    const size_t mats = (size_t)chunks * a.H * N * N * sizeof(float);
+    const int VS = a.VS, Hx = a.H * VS;
+    const BwdLayout l = bwd_layout(a.B, a.T, a.H, varlen, a.G, VS);
+    const size_t mats = l.mats;
     char *w = static_cast<char *>(a.workspace);
     int32_t *off = reinterpret_cast<int32_t *>(w);
-    w += align256b((size_t)(a.B + 1) * sizeof(int32_t));
+    w += l.off;
     float *Mo = reinterpret_cast<float *>(w);
-    float *Bo = reinterpret_cast<float *>(w + align256b(mats));
-    float *Ro = reinterpret_cast<float *>(w + 2 * align256b(mats));
-    float *Sc = reinterpret_cast<float *>(w + 3 * align256b(mats));
-    float *dSn = reinterpret_cast<float *>(w + 4 * align256b(mats));
-    float *Tw = reinterpret_cast<float *>(w + 5 * align256b(mats));
-    float *Ww = reinterpret_cast<float *>(w + 6 * align256b(mats));
-    float *Uw = reinterpret_cast<float *>(w + 7 * align256b(mats));
-    // grouped value heads: per-value-head dq, dk here, summed per group at the end
-    const size_t rows = (varlen ? (size_t)a.T : (size_t)a.B * a.T) * a.H;
-    float *gq = a.G > 1 ? reinterpret_cast<float *>(w + 8 * align256b(mats)) : a.dq;
-    float *gk = a.G > 1 ? reinterpret_cast<float *>(w + 8 * align256b(mats) + align256b(rows * N * 4)) : a.dk;
+    float *Bo = reinterpret_cast<float *>(w + mats);
+    float *Ro = reinterpret_cast<float *>(w + 2 * mats);
+    float *Sc = reinterpret_cast<float *>(w + 3 * mats);
+    float *dSn = reinterpret_cast<float *>(w + 4 * mats);
+    float *Tw = reinterpret_cast<float *>(w + 5 * mats);
+    float *Ww = reinterpret_cast<float *>(w + 6 * mats);
+    float *Uw = reinterpret_cast<float *>(w + 7 * mats);
+    // grouped value heads and value splits: per-virtual-head dq, dk (and dlog_alpha, dbeta) here,
+    // summed at the end
+    const size_t tokens = varlen ? (size_t)a.T : (size_t)a.B * a.T;
+    const int GQ = a.G * VS;  // virtual heads per q/k head
+    char *pw = w + 8 * mats;
+    float *gq = GQ > 1 ? reinterpret_cast<float *>(pw) : a.dq;
+    float *gk = GQ > 1 ? reinterpret_cast<float *>(pw + l.qk) : a.dk;
+    float *gla = VS > 1 ? reinterpret_cast<float *>(pw + 2 * l.qk) : a.dlog_alpha;
+    float *gbe = VS > 1 ? reinterpret_cast<float *>(pw + 2 * l.qk + l.gates) : a.dbeta;
     const int32_t *offp = varlen ? off : nullptr;
     if (varlen) {
         bwd_offsets<<<1, 1, 0, st>>>(a.cu_seqlens, a.B, off);
@@ -850,33 +934,33 @@ cudaError_t run_bwd(const BwdArgs &a, cudaStream_t st)
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(bwd_scans, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_scan);
     if (e != cudaSuccess) return e;
-    const dim3 gc((unsigned)chunks, a.H);
+    const dim3 gc((unsigned)chunks, Hx);
     bwd_prep<TIn><<<gc, kThreads, smem_prep, st>>>(q, k, v, a.log_alpha, a.beta, dout, a.cu_seqlens, offp, a.B, a.T,
-                                                   a.H, a.G, Mo, Bo, Ro, Tw, Ww, Uw);
-    bwd_scans<<<dim3(a.H, a.B, 2), kThreads, smem_scan, st>>>(Mo, Bo, Ro, a.S0, a.dS_final, a.cu_seqlens, offp, a.T,
-                                                             a.H, Sc, dSn, a.dS0);
+                                                   a.H, a.G, VS, Mo, Bo, Ro, Tw, Ww, Uw);
+    bwd_scans<<<dim3(Hx, a.B, 2), kThreads, smem_scan, st>>>(Mo, Bo, Ro, a.S0, a.dS_final, a.cu_seqlens, offp, a.T,
+                                                            a.H, VS, Sc, dSn, a.dS0);
     bwd_grads<TIn><<<gc, kThreads, smem_grads, st>>>(q, k, v, a.log_alpha, a.beta, dout, Sc, dSn, Tw, Ww, Uw,
-                                                     a.cu_seqlens, offp, a.B, a.T, a.H, a.G, gq, gk, a.dv,
-                                                     a.dlog_alpha, a.dbeta);
-    if (a.G > 1) {
-        const long out_elems = (long)(rows / a.G) * N;
+                                                     a.cu_seqlens, offp, a.B, a.T, a.H, a.G, VS, gq, gk, a.dv, gla,
+                                                     gbe);
+    if (GQ > 1) {
+        const long out_elems = (long)(tokens * (a.H / a.G)) * N;
         if (out_elems > 0)
-            bwd_group_sum<<<(unsigned)((out_elems + 255) / 256), 256, 0, st>>>(gq, gk, a.dq, a.dk, out_elems, a.G);
+            bwd_group_sum<<<(unsigned)((out_elems + 255) / 256), 256, 0, st>>>(gq, gk, a.dq, a.dk, out_elems, GQ);
+    }
+    if (VS > 1) {
+        const long out_elems = (long)(tokens * a.H);
+        if (out_elems > 0)
+            bwd_gate_sum<<<(unsigned)((out_elems + 255) / 256), 256, 0, st>>>(gla, gbe, a.dlog_alpha, a.dbeta,
+                                                                              out_elems, VS);
     }
     return cudaGetLastError();
 }
 
 }  // namespace
 
-size_t chunk_bwd_workspace_bytes(int B, int T, int H, int varlen, int G)
+size_t chunk_bwd_workspace_bytes(int B, int T, int H, int varlen, int G, int VS)
 {
-    const size_t mats = (size_t)bwd_chunks(B, T, varlen) * H * N * N * sizeof(float);
-    size_t bytes = align256b((size_t)(B + 1) * sizeof(int32_t)) + 8 * align256b(mats);
-    if (G > 1) {  // per-value-head dq and dk before the group sums
-        const size_t rows = (varlen ? (size_t)T : (size_t)B * T) * H;
-        bytes += 2 * align256b(rows * N * 4);
-    }
-    return bytes;
+    return bwd_layout(B, T, H, varlen, G, VS).bytes;
 }
 
 cudaError_t launch_chunk_bwd(const BwdArgs &a, cudaStream_t stream)

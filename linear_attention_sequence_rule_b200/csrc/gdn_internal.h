@@ -50,7 +50,7 @@ int read_and_clear_tc_error();
 // after limit_ms and records it in that error word (see gdn_selftest_wait_timeout).
 cudaError_t launch_wait_probe(int limit_ms, cudaStream_t stream);
 
-// Gradients of the chunk forward (fp32-level accuracy, dk = dv = 64); see gdn_chunk_bwd.cu.
+// Gradients of the chunk forward (fp32-level accuracy, dk = 64, dv = 64 VS); see gdn_chunk_bwd.cu.
 struct BwdArgs {
     const void *q, *k, *v;
     const float *log_alpha, *beta, *S0;
@@ -60,9 +60,10 @@ struct BwdArgs {
     const int32_t *cu_seqlens;
     int B, T, H, dtype;  // H value heads
     void *workspace;
-    int G = 1;  // grouped value heads: H / G q/k heads, value head h reads q/k head h / G
+    int G = 1;   // grouped value heads: H / G q/k heads, value head h reads q/k head h / G
+    int VS = 1;  // value splits: dv = 64 VS, each value head run as VS heads of 64 columns
 };
-size_t chunk_bwd_workspace_bytes(int B, int T, int H, int varlen, int G = 1);
+size_t chunk_bwd_workspace_bytes(int B, int T, int H, int varlen, int G = 1, int VS = 1);
 cudaError_t launch_chunk_bwd(const BwdArgs &a, cudaStream_t stream);
 
 }  // namespace gdn

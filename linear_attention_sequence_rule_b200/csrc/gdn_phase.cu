@@ -183,7 +183,8 @@ __global__ void phase_widen(const TV *__restrict__ x, float *__restrict__ y, lon
     if (i < n) y[i] = to_f(x[i]);
 }
 
-// One warp per token-head (DK = 32 complex key elements: one per lane; DV = 64: two per lane).
+// One warp per token-head (DK = 32 complex key elements: one per lane; DV / 32 values per lane).
+template <int DV>
 __global__ void __launch_bounds__(256) phase_bwd_epilogue(const float *__restrict__ dq_r,
                                                           const float *__restrict__ dk_r,
                                                           const float *__restrict__ dv_r,
@@ -195,7 +196,7 @@ __global__ void __launch_bounds__(256) phase_bwd_epilogue(const float *__restric
                                                           float *__restrict__ dV, float *__restrict__ dlog_lam,
                                                           float *__restrict__ dbeta)
 {
-    constexpr int DK = 32, DV = 64;
+    constexpr int DK = 32;
     const long th = ((long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int lane = threadIdx.x & 31;
     if (th >= token_heads) return;
@@ -203,11 +204,14 @@ __global__ void __launch_bounds__(256) phase_bwd_epilogue(const float *__restric
     dK[th * DK + lane] = make_float2(dk_r[th * 2 * DK + lane] * KeyScale<DK>::inv_sqrt,
                                      dk_r[th * 2 * DK + DK + lane] * KeyScale<DK>::inv_sqrt);
     dQ[th * DK + lane] = make_float2(dq_r[th * 2 * DK + lane] * (1.0f / DK), dq_r[th * 2 * DK + DK + lane] * (1.0f / DK));
-    const float g0 = dv_r[th * DV + lane], g1 = dv_r[th * DV + lane + 32];
     const float vs = lam * KeyScale<DK>::sqrt;
-    dV[th * DV + lane] = vs * g0;
-    dV[th * DV + lane + 32] = vs * g1;
-    float dot = g0 * v_r[th * DV + lane] + g1 * v_r[th * DV + lane + 32];
+    float dot = 0.f;
+#pragma unroll
+    for (int j = lane; j < DV; j += 32) {
+        const float gj = dv_r[th * DV + j];
+        dV[th * DV + j] = vs * gj;
+        dot = fmaf(gj, v_r[th * DV + j], dot);
+    }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
     if (lane == 0) {
@@ -220,9 +224,9 @@ struct PhaseBwdPlan {
     size_t kr, qr, vr, br, d32, s0, sf, dq, dk, dv, dla, db, ds0, ws, ws_bytes, total;
 };
 
-bool phase_bwd_plan(PhaseBwdPlan &p, int B, int T, int H, int varlen)
+bool phase_bwd_plan(PhaseBwdPlan &p, int B, int T, int H, int DV, int varlen)
 {
-    constexpr int DK = 32, DV = 64;
+    constexpr int DK = 32;
     const size_t ws = gdn_chunk_bwd_workspace_bytes(B, T, H, 2 * DK, DV, 64, varlen);
     if (ws == (size_t)-1) return false;
     const size_t th = (varlen ? (size_t)T : (size_t)B * T) * H, st = (size_t)B * H * 2 * DK * DV * 4;
@@ -340,9 +344,9 @@ int gdn_phase_fwd(const float *K, const float *Q, const void *v, const float *lo
 
 size_t gdn_phase_bwd_workspace_bytes(int B, int T, int H, int dk, int dv, int varlen)
 {
-    if (dk != 32 || dv != 64) return (size_t)-1;
+    if (dk != 32 || (dv != 64 && dv != 128)) return (size_t)-1;
     PhaseBwdPlan p;
-    if (!phase_bwd_plan(p, B, T, H, varlen)) return (size_t)-1;
+    if (!phase_bwd_plan(p, B, T, H, dv, varlen)) return (size_t)-1;
     return p.total;
 }
 
@@ -352,13 +356,13 @@ int gdn_phase_bwd(const float *K, const float *Q, const void *v, const float *lo
                   const int32_t *cu_seqlens, int dtype, void *workspace, size_t workspace_bytes, void *stream)
 {
     const int varlen = cu_seqlens != nullptr;
-    if (dk != 32 || dv != 64 || (dtype != GDN_DTYPE_BF16 && dtype != GDN_DTYPE_F32)) {
-        set_error("gdn_phase_bwd: dk=%d dv=%d dtype=%d, supported: dk 32 (64 real), dv 64, bf16 or fp32", dk, dv,
-                  dtype);
+    if (dk != 32 || (dv != 64 && dv != 128) || (dtype != GDN_DTYPE_BF16 && dtype != GDN_DTYPE_F32)) {
+        set_error("gdn_phase_bwd: dk=%d dv=%d dtype=%d, supported: dk 32 (64 real), dv 64 or 128, bf16 or fp32",
+                  dk, dv, dtype);
         return GDN_ERR_UNSUPPORTED;
     }
     PhaseBwdPlan p;
-    if (!phase_bwd_plan(p, B, T, H, varlen))  // the backward's own checks give the reason
+    if (!phase_bwd_plan(p, B, T, H, dv, varlen))  // the backward's own checks give the reason
         return gdn_chunk_bwd(nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr,
                              nullptr, nullptr, nullptr, nullptr, nullptr, B, T, H, 2 * dk, dv, 64, cu_seqlens,
                              GDN_DTYPE_F32, nullptr, 0, stream);
@@ -395,9 +399,13 @@ int gdn_phase_bwd(const float *K, const float *Q, const void *v, const float *lo
     fp.qr = p.qr;
     fp.vr = p.vr;
     fp.br = p.br;
-    cudaError_t e = dtype == GDN_DTYPE_BF16
-                        ? launch_prologue<32, 64, __nv_bfloat16, float>(K, Q, v, log_lam, beta, th, w, fp, st)
-                        : launch_prologue<32, 64, float, float>(K, Q, v, log_lam, beta, th, w, fp, st);
+    cudaError_t e;
+    if (dv == 64)
+        e = dtype == GDN_DTYPE_BF16 ? launch_prologue<32, 64, __nv_bfloat16, float>(K, Q, v, log_lam, beta, th, w, fp, st)
+                                    : launch_prologue<32, 64, float, float>(K, Q, v, log_lam, beta, th, w, fp, st);
+    else
+        e = dtype == GDN_DTYPE_BF16 ? launch_prologue<32, 128, __nv_bfloat16, float>(K, Q, v, log_lam, beta, th, w, fp, st)
+                                    : launch_prologue<32, 128, float, float>(K, Q, v, log_lam, beta, th, w, fp, st);
     if (e != cudaSuccess) return fail_launch(e);
     const long nv = th * dv;
     float *d32 = reinterpret_cast<float *>(w + p.d32);
@@ -428,11 +436,13 @@ int gdn_phase_bwd(const float *K, const float *Q, const void *v, const float *lo
                                  dbr, dM0 ? reinterpret_cast<float *>(w + p.ds0) : nullptr, B, T, H, 2 * dk, dv, 64,
                                  cu_seqlens, GDN_DTYPE_F32, w + p.ws, p.ws_bytes, stream);
     if (rc != GDN_OK) return rc;
-    if (th)
-        phase_bwd_epilogue<<<(unsigned)((th * 32 + 255) / 256), 256, 0, st>>>(
+    if (th) {
+        auto epi = dv == 64 ? phase_bwd_epilogue<64> : phase_bwd_epilogue<128>;
+        epi<<<(unsigned)((th * 32 + 255) / 256), 256, 0, st>>>(
             dq, dkr, dvr, reinterpret_cast<const float *>(w + p.vr), dla, dbr,
             reinterpret_cast<const float *>(w + p.br), log_lam, th, reinterpret_cast<float2 *>(dK),
             reinterpret_cast<float2 *>(dQ), dv_out, dlog_lam, dbeta);
+    }
     if (dM0) {
         const long nm = states * dk * dv;
         phase_state_out<<<(unsigned)((nm + 255) / 256), 256, 0, st>>>(reinterpret_cast<const float *>(w + p.ds0),

@@ -158,6 +158,14 @@ def test_backward_entry_validation():
     assert "gdn_chunk_bwd" in gdn.gdn_last_error()
     assert gdn.gdn_chunk_bwd_workspace_bytes(1, 64, 1, 128, 128, 64, 0) == (1 << 64) - 1
     assert gdn.gdn_chunk_bwd_workspace_bytes(2, 128, 3, 64, 64, 64, 0) > 5 * 2 * 2 * 3 * 64 * 64 * 4 - 1
+    # value head sizes 128 and 256 (64-column value splits): more workspace; other sizes rejected
+    w64 = gdn.gdn_chunk_bwd_workspace_bytes(2, 128, 3, 64, 64, 64, 0)
+    assert gdn.gdn_chunk_bwd_workspace_bytes(2, 128, 3, 64, 128, 64, 0) > 2 * w64 - 4096
+    assert gdn.gdn_chunk_bwd_workspace_bytes(2, 128, 3, 64, 256, 64, 1) > 4 * w64 - 4096
+    assert gdn.gdn_chunk_bwd_workspace_bytes(2, 128, 3, 64, 96, 64, 0) == (1 << 64) - 1
+    assert gdn.gdn_chunk_bwd_workspace_bytes(2, 128, 3, 128, 64, 64, 0) == (1 << 64) - 1
+    assert gdn.gdn_chunk_bwd(**(a | dict(dv_=128))) == gdn.GDN_ERR_WORKSPACE
+    assert gdn.gdn_chunk_bwd(**(a | dict(dv_=512))) == gdn.GDN_ERR_UNSUPPORTED
 
 
 def host_chunk(**kw):
@@ -258,7 +266,8 @@ def test_phase_backward_rejects_before_any_launch():
              dv_out=FAKE, dlog_lam=FAKE, dbeta=FAKE, dM0=None, B=1, T=64, H=1, dk=32, dv=64, cu_seqlens=None,
              dtype=gdn.GDN_DTYPE_BF16, workspace=FAKE * 256, workspace_bytes=1 << 40, stream=None)
     assert gdn.gdn_phase_bwd(**dict(a, dk=64)) == gdn.GDN_ERR_UNSUPPORTED   # the backward takes 64 real columns
-    assert gdn.gdn_phase_bwd(**dict(a, dv=128)) == gdn.GDN_ERR_UNSUPPORTED
+    assert gdn.gdn_phase_bwd(**dict(a, dv=256)) == gdn.GDN_ERR_UNSUPPORTED
+    assert gdn.gdn_phase_bwd_workspace_bytes(1, 64, 1, 32, 128, 0) > gdn.gdn_phase_bwd_workspace_bytes(1, 64, 1, 32, 64, 0)
     assert gdn.gdn_phase_bwd(**dict(a, dQ=None)) == gdn.GDN_ERR_INVALID_ARGUMENT
     assert gdn.gdn_phase_bwd(**dict(a, K=FAKE + 4)) == gdn.GDN_ERR_INVALID_ARGUMENT
     assert gdn.gdn_phase_bwd(**dict(a, workspace=None)) == gdn.GDN_ERR_WORKSPACE

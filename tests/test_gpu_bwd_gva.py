@@ -1,7 +1,7 @@
 """GPU parity of gdn_chunk_bwd_gva (grouped value heads: Hv value heads reading Hk q/k heads)
 against the fp64 oracle (oracle/grouped.py backward_gva, pinned by finite differences in
 tests/test_oracle_grouped_backward.py): dense and varlen, G = 2 and 3, with and without S0 and
-dS_final.  Bound as the plain backward: max |g - g_ref| <= 1e-5 * (1 + max |g_ref|) per tensor."""
+dS_final, value head sizes 64 and 128.  Bound as the plain backward: max |g - g_ref| <= 1e-5 * (1 + max |g_ref|) per tensor."""
 import numpy as np
 import pytest
 import torch
@@ -48,3 +48,8 @@ def test_dense_groups_of_three():
 def test_varlen_groups_of_two_fp32():
     check(workloads.make_gva_chunk_inputs(Hk=2, Hv=4, dk=64, dv=64, dtype="f32", seed=82,
                                           lengths=[1, 64, 0, 130, 7]), 2, with_dsf=False)
+
+
+def test_dense_groups_of_two_value_head_128():
+    check(workloads.make_gva_chunk_inputs(B=2, T=150, Hk=1, Hv=2, dk=64, dv=128, dtype="bf16", seed=83, s0_std=0.1,
+                                          la_scale=0.3), 3)

@@ -1,5 +1,5 @@
 """GPU parity of gdn_phase_bwd (gradients of the complex-phase delta memory, dk = 32 complex,
-dv = 64) against the fp64 phase backward oracle (oracle/phase.py backward, pinned by finite
+dv = 64 and 128) against the fp64 phase backward oracle (oracle/phase.py backward, pinned by finite
 differences of the complex definition in tests/test_oracle_phase.py): dense and varlen, bf16 and
 fp32 values, unit and Laplace keys, with and without M0 and dM_final.  The backward runs in fp32
 on the stored inputs, so the bound is the plain backward's: max |g - g_ref| <= 1e-5 *
@@ -66,3 +66,8 @@ def test_dense_fp32_laplace_keys():
 def test_varlen_ragged_beta_two():
     check(workloads.make_phase_inputs(H=2, dk=32, dv=64, dtype="bf16", seed=603, beta_scale=2.0,
                                       lengths=[0, 1, 63, 64, 65, 200, 7]), 3, with_dm=False)
+
+
+def test_value_head_128_varlen():
+    check(workloads.make_phase_inputs(H=2, dk=32, dv=128, dtype="bf16", seed=604, m0_std=0.05,
+                                      lengths=[70, 0, 129, 1]), 4)
