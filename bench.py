@@ -301,16 +301,23 @@ def wide_value_inputs(seed=0):
                                               la_scale=0.1))
 
 
-def time_decode(gdn, steps, warmup, stream, pool=32):
+def time_decode(gdn, steps, warmup, stream, pool=32, fused=False):
+    """The decode workload's steps (CUDA events per step); fused: from raw projections through
+    gdn_decode_step_fused (same bytes: raw q/k and gates replace the prepared ones)."""
     cfg = workloads.CONFIGS["decode"]
     N, H, dk, dv = cfg["N"], cfg["H"], cfg["dk"], cfg["dv"]
     S = workloads.make_decode_state(N, H, dk, dv, cfg["seed"]).cuda()
-    xs = [to_dev(workloads.make_decode_step_inputs(N, H, dk, dv, cfg["dtype"], seed=cfg["seed"],
-                                                   step=i, la_scale=cfg["la_scale"]))
+    make = workloads.make_raw_decode_step_inputs if fused else workloads.make_decode_step_inputs
+    xs = [{k: (v.cuda() if torch.is_tensor(v) else v)
+           for k, v in make(N, H, dk, dv, cfg["dtype"], seed=cfg["seed"], step=i, la_scale=cfg["la_scale"]).items()}
           for i in range(pool)]
     out = torch.empty((N, H, dv), dtype=torch.bfloat16, device="cuda")
-    call = lambda x: gdn.decode_step(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], S,
-                                     out=out, stream=stream)
+    if fused:
+        call = lambda x: gdn.decode_step_fused(x["q_raw"], x["k_raw"], x["v"], x["a_raw"], x["b_raw"], x["a_scale"],
+                                               x["b_scale"], S, out=out, stream=stream)
+    else:
+        call = lambda x: gdn.decode_step(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], S,
+                                         out=out, stream=stream)
     with torch.cuda.stream(stream):
         for i in range(warmup):
             call(xs[i % pool])
@@ -325,7 +332,8 @@ def time_decode(gdn, steps, warmup, stream, pool=32):
     t = [s.elapsed_time(e) for s, e in ev]
     ms = statistics.mean(t)
     by = N * H * DECODE_BYTES_PER_STATE(dk, dv, 2)
-    return dict(workload=f"decode N={N} H={H} dk=dv={dk} bf16, fp32 state", steps=steps,
+    name = f"decode N={N} H={H} dk=dv={dk} bf16, fp32 state" + (", from raw projections (fused entry)" if fused else "")
+    return dict(workload=name, steps=steps,
                 input_pool=pool, ms_per_step=ms, state_updates_per_s=N * H / (ms * 1e-3),
                 tokens_per_s=N / (ms * 1e-3), algo_bytes_per_step=by,
                 gbs=by / (ms * 1e-3) / 1e9)
@@ -429,6 +437,9 @@ def run_ours(args, world, rank, local):
         decode["hbm_frac"] = decode["gbs"] / peaks["hbm_gbs"]
         # DRAM bytes per step from the ncu record of the current decode source (null once it changed)
         decode["traffic"] = ncu_traffic("decode", "decode")
+        dfu = time_decode(gdn, 300, 10, stream, fused=True)
+        extra["decode_fused"] = {k: (round(v, 6) if isinstance(v, float) else v) for k, v in dfu.items()}
+        extra["decode_fused"]["hbm_frac"] = round(dfu["gbs"] / peaks["hbm_gbs"], 5)
         for w in ("long_context", "varlen"):
             dw = to_dev(workloads.config_inputs(w))
             tw = time_chunk(gdn, dw, max(3, args.steps // 20), 2, flush, stream)
@@ -649,8 +660,8 @@ def run_only(args):
     import linear_attention_sequence_rule_b200 as gdn
     peaks, _ = load_peaks()
     stream = torch.cuda.Stream()
-    if args.only == "decode":
-        r = time_decode(gdn, args.steps, args.warmup, stream)
+    if args.only in ("decode", "decode_fused"):
+        r = time_decode(gdn, args.steps, args.warmup, stream, fused=args.only == "decode_fused")
         r["hbm_frac"] = r["gbs"] / peaks["hbm_gbs"]
     elif args.only == "hybrid_lm_backward":
         flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device="cuda")
@@ -742,7 +753,7 @@ def main():
     ap.add_argument("--quick", action="store_true", help="main workload only")
     ap.add_argument("--only", choices=["hybrid_lm", "long_context", "varlen", "tiny", "decode", "hybrid_lm_fused",
                                              "hybrid_lm_unfused", "hybrid_lm_backward", "phase_memory",
-                                             "hybrid_lm_dv256", "hybrid_lm_backward_dv128"],
+                                             "hybrid_lm_dv256", "hybrid_lm_backward_dv128", "decode_fused"],
                     help="time one workload's kernel loop only (for profiler runs)")
     args = ap.parse_args()
     if args.warmup < 3:

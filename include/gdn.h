@@ -290,12 +290,12 @@ GDN_API size_t gdn_chunk_bwd_gva_workspace_bytes(int B, int T, int Hk, int Hv, i
  * gdn_chunk_bwd_fused -- gradients of gdn_chunk_fwd_fused with respect to its RAW inputs: given
  * q_raw, k_raw, v (dtype), a_raw, b_raw (fp32), S0, a_scale, b_scale as passed to the forward,
  * dout = dL/dout (dtype) and dS_final = dL/dS_final (NULL: zero), it writes fp32
- *     dq_raw, dk_raw [.., H, 64], dv [.., H, 64], da_raw, db_raw [.., H], dS0 (NULL: not written).
+ *     dq_raw, dk_raw [.., H, 64], dv [.., H, dv], da_raw, db_raw [.., H], dS0 (NULL: not written).
  * The prologue (rows divided by sqrt(|x|^2 + 1e-6), log alpha = -a_scale softplus(a),
  * beta = b_scale sigmoid(b)) is formed again in fp32, the recurrence's backward runs in fp32 on
  * it (as gdn_chunk_bwd with fp32 inputs), and the chain rule through the prologue follows:
  * dx = (dq - q (q . dq)) / |x|_eps, da = -a_scale sigmoid(a) dlog_alpha (0 at a = +inf),
- * db = b_scale sigmoid(b) (1 - sigmoid(b)) dbeta.  dk = dv = 64, chunk = 64.  Workspace:
+ * db = b_scale sigmoid(b) (1 - sigmoid(b)) dbeta.  dk = 64, dv in {64, 128, 256}, chunk = 64.  Workspace:
  * gdn_chunk_bwd_fused_workspace_bytes(...) bytes of device memory, 256-byte aligned.  Errors as
  * gdn_chunk_bwd; a_scale must be finite and >= 0, b_scale in [0, 2].
  */
@@ -324,6 +324,18 @@ GDN_API size_t gdn_chunk_bwd_fused_workspace_bytes(int B, int T, int H, int dk, 
 GDN_API int gdn_decode_step(const void *q, const void *k, const void *v, const float *log_alpha,
                     const float *beta, float *S_inout, void *out, int N, int H, int dk, int dv,
                     int dtype, void *stream);
+
+/*
+ * gdn_decode_step_fused -- gdn_decode_step from raw projections, the prologue of
+ * gdn_chunk_fwd_fused formed inside the step (one launch; the state is still read and written
+ * once): q_raw, k_raw [N,H,dk] in dtype are divided by sqrt(|x|^2 + 1e-6) over their dk elements,
+ * a_raw, b_raw [N,H] fp32 become log alpha = -a_scale softplus(a) (a = +inf: an exact reset) and
+ * beta = b_scale sigmoid(b); v, out, S_inout and the head sizes as gdn_decode_step.  a_scale must
+ * be finite and >= 0, b_scale in [0, 2] (GDN_ERR_INVALID_ARGUMENT otherwise).
+ */
+GDN_API int gdn_decode_step_fused(const void *q_raw, const void *k_raw, const void *v, const float *a_raw,
+                                  const float *b_raw, float *S_inout, void *out, int N, int H, int dk, int dv,
+                                  int dtype, float a_scale, float b_scale, void *stream);
 
 /*
  * gdn_decode_step_gva -- gdn_decode_step with grouped value heads (see gdn_chunk_fwd_gva):

@@ -8,8 +8,8 @@ PyTorch provides device memory and streams.  The binding has two layers:
   ``gdn_status_string``, ``gdn_last_error``, ``gdn_version`` -- the C-ABI entry points of
   ``include/gdn.h`` with the same names and arguments (pointers as Python ints);
 * ``chunk_fwd``, ``chunk_fwd_host``, ``chunk_fwd_fused``, ``chunk_fwd_gva``, ``chunk_bwd``,
-  ``chunk_bwd_fused``, ``chunk_bwd_gva``, ``phase_fwd``, ``phase_bwd``, ``decode_step`` and
-  ``decode_step_gva`` --
+  ``chunk_bwd_fused``, ``chunk_bwd_gva``, ``phase_fwd``, ``phase_bwd``, ``decode_step``,
+  ``decode_step_fused`` and ``decode_step_gva`` --
   the same calls taking torch tensors; they check shapes,
   devices and dtypes, allocate outputs with torch when none are given, and raise ``GdnError``
   on a non-zero status.
@@ -32,7 +32,7 @@ __all__ = [
     "gdn_phase_bwd", "gdn_phase_bwd_workspace_bytes", "phase_bwd",
     "gdn_chunk_bwd_fused", "gdn_chunk_bwd_fused_workspace_bytes", "chunk_bwd_fused",
     "gdn_chunk_bwd_gva", "gdn_chunk_bwd_gva_workspace_bytes", "chunk_bwd_gva",
-    "gdn_decode_step", "gdn_decode_step_gva", "gdn_chunk_bwd", "gdn_chunk_bwd_workspace_bytes", "gdn_chunk_fwd_workspace_bytes", "gdn_status_string",
+    "gdn_decode_step", "gdn_decode_step_fused", "decode_step_fused", "gdn_decode_step_gva", "gdn_chunk_bwd", "gdn_chunk_bwd_workspace_bytes", "gdn_chunk_fwd_workspace_bytes", "gdn_status_string",
     "gdn_last_error", "gdn_version", "gdn_device_status", "gdn_selftest_wait_timeout", "device_status", "chunk_fwd", "chunk_fwd_fused",
     "chunk_fwd_gva", "chunk_bwd", "decode_step", "decode_step_gva", "workspace_bytes",
 ]
@@ -98,6 +98,8 @@ _lib.gdn_chunk_fwd_workspace_bytes.argtypes = [_i, _i, _i, _i, _i, _i, _i, _i]
 _lib.gdn_chunk_fwd_workspace_bytes.restype = _sz
 _lib.gdn_decode_step.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp]
 _lib.gdn_decode_step.restype = _i
+_lib.gdn_decode_step_fused.argtypes = [_vp] * 7 + [_i] * 5 + [ctypes.c_float, ctypes.c_float, _vp]
+_lib.gdn_decode_step_fused.restype = _i
 _lib.gdn_selftest_wait_timeout.argtypes = [_i, _vp]
 _lib.gdn_selftest_wait_timeout.restype = _i
 _lib.gdn_device_status.argtypes = [_vp]
@@ -196,6 +198,12 @@ def gdn_chunk_fwd_workspace_bytes(B, T, H, dk, dv, chunk, varlen, dtype) -> int:
 
 def gdn_decode_step(q, k, v, log_alpha, beta, S_inout, out, N, H, dk, dv, dtype, stream) -> int:
     return _lib.gdn_decode_step(q, k, v, log_alpha, beta, S_inout, out, N, H, dk, dv, dtype, stream)
+
+
+def gdn_decode_step_fused(q_raw, k_raw, v, a_raw, b_raw, S_inout, out, N, H, dk, dv, dtype, a_scale, b_scale,
+                          stream) -> int:
+    return _lib.gdn_decode_step_fused(q_raw, k_raw, v, a_raw, b_raw, S_inout, out, N, H, dk, dv, dtype, a_scale,
+                                      b_scale, stream)
 
 
 def gdn_selftest_wait_timeout(limit_ms, stream) -> int:
@@ -617,7 +625,7 @@ def gdn_chunk_bwd_fused_workspace_bytes(B, T, H, dk, dv, chunk, varlen) -> int:
 
 def chunk_bwd_fused(q_raw, k_raw, v, a_raw, b_raw, dout, a_scale, b_scale, S0=None, dS_final=None,
                     cu_seqlens=None, want_dS0=True, workspace=None, chunk=64, stream=None):
-    """Gradients of ``chunk_fwd_fused`` with respect to its raw inputs (dk = dv = 64): returns fp32
+    """Gradients of ``chunk_fwd_fused`` with respect to its raw inputs (dk = 64, dv in {64, 128, 256}): returns fp32
     (dq_raw, dk_raw, dv, da_raw, db_raw, dS0 or None)."""
     dt = q_raw.dtype
     if dt not in _DT:
@@ -702,6 +710,32 @@ def decode_step(q, k, v, log_alpha, beta, S, out=None, stream=None):
     _need(out, "out", dt, (N, H, dv), dev)
     rc = gdn_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(S), _ptr(out),
                          N, H, dk, dv, _DT[dt], _stream_ptr(stream))
+    if rc != GDN_OK:
+        raise GdnError(rc, gdn_last_error())
+    return out
+
+
+def decode_step_fused(q_raw, k_raw, v, a_raw, b_raw, a_scale, b_scale, S, out=None, stream=None):
+    """One decode step from raw projections (``gdn_decode_step_fused``): q_raw, k_raw [N,H,dk]
+    unnormalised, a_raw, b_raw [N,H] fp32 raw gate projections; S [N,H,dk,dv] fp32 updated in
+    place.  Returns out [N,H,dv]."""
+    dt = q_raw.dtype
+    if dt not in _DT:
+        raise ValueError(f"unsupported dtype {dt}")
+    dev = q_raw.device
+    N, H, dk = q_raw.shape
+    dv = v.shape[-1]
+    _need(q_raw, "q_raw", dt, (N, H, dk), dev)
+    _need(k_raw, "k_raw", dt, (N, H, dk), dev)
+    _need(v, "v", dt, (N, H, dv), dev)
+    _need(a_raw, "a_raw", torch.float32, (N, H), dev)
+    _need(b_raw, "b_raw", torch.float32, (N, H), dev)
+    _need(S, "S", torch.float32, (N, H, dk, dv), dev)
+    if out is None:
+        out = torch.empty((N, H, dv), dtype=dt, device=dev)
+    _need(out, "out", dt, (N, H, dv), dev)
+    rc = gdn_decode_step_fused(_ptr(q_raw), _ptr(k_raw), _ptr(v), _ptr(a_raw), _ptr(b_raw), _ptr(S), _ptr(out),
+                               N, H, dk, dv, _DT[dt], float(a_scale), float(b_scale), _stream_ptr(stream))
     if rc != GDN_OK:
         raise GdnError(rc, gdn_last_error())
     return out

@@ -175,7 +175,7 @@ namespace gdn {
 
 static int decode_common(const char *fn, const void *q, const void *k, const void *v, const float *log_alpha,
                          const float *beta, float *S_inout, void *out, int N, int H, int G, int dk, int dv,
-                         int dtype, void *stream)
+                         int dtype, void *stream, int prologue = 0, float a_scale = 0.f, float b_scale = 0.f)
 {
     if (dtype != GDN_DTYPE_BF16 && dtype != GDN_DTYPE_F32)
         return fail(GDN_ERR_UNSUPPORTED, "%s: unknown dtype %d", fn, dtype);
@@ -190,8 +190,11 @@ static int decode_common(const char *fn, const void *q, const void *k, const voi
     for (const void *p : ptrs)
         if (!aligned16(p))
             return fail(GDN_ERR_INVALID_ARGUMENT, "%s: pointer %p is not 16-byte aligned", fn, p);
+    if (prologue && (!(a_scale >= 0.f) || !(a_scale < INFINITY) || !(b_scale >= 0.f && b_scale <= 2.f)))
+        return fail(GDN_ERR_INVALID_ARGUMENT, "%s: a_scale %g (finite, >= 0) or b_scale %g (in [0, 2]) out of range",
+                    fn, (double)a_scale, (double)b_scale);
     cudaError_t e = launch_decode(q, k, v, log_alpha, beta, S_inout, out, N, H, dk, dv, dtype,
-                                  static_cast<cudaStream_t>(stream), G);
+                                  static_cast<cudaStream_t>(stream), G, prologue, a_scale, b_scale);
     if (e != cudaSuccess) return cuda_fail(e, fn);
     return GDN_OK;
 }
@@ -214,6 +217,15 @@ int gdn_decode_step(const void *q, const void *k, const void *v, const float *lo
     g_last_error[0] = 0;
     return decode_common("gdn_decode_step", q, k, v, log_alpha, beta, S_inout, out, N, H, 1, dk, dv, dtype,
                          stream);
+}
+
+int gdn_decode_step_fused(const void *q_raw, const void *k_raw, const void *v, const float *a_raw,
+                          const float *b_raw, float *S_inout, void *out, int N, int H, int dk, int dv, int dtype,
+                          float a_scale, float b_scale, void *stream)
+{
+    g_last_error[0] = 0;
+    return decode_common("gdn_decode_step_fused", q_raw, k_raw, v, a_raw, b_raw, S_inout, out, N, H, 1, dk, dv,
+                         dtype, stream, 1, a_scale, b_scale);
 }
 
 int gdn_decode_step_gva(const void *q, const void *k, const void *v, const float *log_alpha,

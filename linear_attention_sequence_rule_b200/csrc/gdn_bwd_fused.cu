@@ -17,7 +17,7 @@
 namespace gdn {
 namespace {
 
-constexpr int D = 64;              // head size (the backward supports dk = dv = 64)
+constexpr int D = 64;              // key head size (the backward supports dk = 64, dv = 64, 128, 256)
 constexpr float kEps = 1e-6f;      // the forward prologue's normalisation epsilon
 
 __device__ __forceinline__ float to_f(float x) { return x; }
@@ -38,13 +38,14 @@ __device__ __forceinline__ float warp_sum(float x)
     return x;
 }
 
-// One warp per (token, head): normalised q and k rows, v and dout widened to fp32, the gates.
+// One warp per (token, head): normalised q and k rows, v and dout (dv values) widened to fp32, the
+// gates.
 template <typename TIn>
 __global__ void __launch_bounds__(256) fused_bwd_prologue(const TIn *__restrict__ q_raw, const TIn *__restrict__ k_raw,
                                                           const TIn *__restrict__ v, const TIn *__restrict__ dout,
                                                           const float *__restrict__ a_raw,
                                                           const float *__restrict__ b_raw, float a_scale,
-                                                          float b_scale, long rows, float *__restrict__ qn,
+                                                          float b_scale, long rows, int dv, float *__restrict__ qn,
                                                           float *__restrict__ kn, float *__restrict__ v32,
                                                           float *__restrict__ d32, float *__restrict__ la,
                                                           float *__restrict__ be)
@@ -61,10 +62,11 @@ __global__ void __launch_bounds__(256) fused_bwd_prologue(const TIn *__restrict_
     qn[o + lane + 32] = q1 * rq;
     kn[o + lane] = k0 * rk;
     kn[o + lane + 32] = k1 * rk;
-    v32[o + lane] = to_f(v[o + lane]);
-    v32[o + lane + 32] = to_f(v[o + lane + 32]);
-    d32[o + lane] = to_f(dout[o + lane]);
-    d32[o + lane + 32] = to_f(dout[o + lane + 32]);
+    const size_t ov = (size_t)row * dv;
+    for (int j = lane; j < dv; j += 32) {
+        v32[ov + j] = to_f(v[ov + j]);
+        d32[ov + j] = to_f(dout[ov + j]);
+    }
     if (lane == 0) {
         const float a = a_raw[row];
         la[row] = a == INFINITY ? -INFINITY : -a_scale * softplusf_(a);
@@ -116,9 +118,9 @@ struct FusedBwdPlan {
     size_t qn, kn, v32, d32, la, be, dla, dbe, ws, ws_bytes, total;
 };
 
-bool fused_bwd_plan(FusedBwdPlan &p, int B, int T, int H, int varlen)
+bool fused_bwd_plan(FusedBwdPlan &p, int B, int T, int H, int dv, int varlen)
 {
-    const size_t ws = gdn_chunk_bwd_workspace_bytes(B, T, H, D, D, 64, varlen);
+    const size_t ws = gdn_chunk_bwd_workspace_bytes(B, T, H, D, dv, 64, varlen);
     if (ws == (size_t)-1) return false;
     const size_t rows = (varlen ? (size_t)T : (size_t)B * T) * H;
     size_t o = 0;
@@ -129,8 +131,8 @@ bool fused_bwd_plan(FusedBwdPlan &p, int B, int T, int H, int varlen)
     };
     p.qn = take(rows * D * 4);
     p.kn = take(rows * D * 4);
-    p.v32 = take(rows * D * 4);
-    p.d32 = take(rows * D * 4);
+    p.v32 = take(rows * dv * 4);
+    p.d32 = take(rows * dv * 4);
     p.la = take(rows * 4);
     p.be = take(rows * 4);
     p.dla = take(rows * 4);
@@ -144,7 +146,7 @@ bool fused_bwd_plan(FusedBwdPlan &p, int B, int T, int H, int varlen)
 template <typename TIn>
 int run_fused_bwd(const void *q_raw, const void *k_raw, const void *v, const float *a_raw, const float *b_raw,
                   const float *S0, const void *dout, const float *dS_final, float *dq_raw, float *dk_raw, float *dv,
-                  float *da_raw, float *db_raw, float *dS0, int B, int T, int H, const int32_t *cu_seqlens,
+                  float *da_raw, float *db_raw, float *dS0, int B, int T, int H, int dv_, const int32_t *cu_seqlens,
                   float a_scale, float b_scale, char *w, const FusedBwdPlan &p, void *stream)
 {
     cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -155,7 +157,7 @@ int run_fused_bwd(const void *q_raw, const void *k_raw, const void *v, const flo
     if (blocks)
         fused_bwd_prologue<TIn><<<blocks, 256, 0, st>>>(
             static_cast<const TIn *>(q_raw), static_cast<const TIn *>(k_raw), static_cast<const TIn *>(v),
-            static_cast<const TIn *>(dout), a_raw, b_raw, a_scale, b_scale, rows, qn, kn,
+            static_cast<const TIn *>(dout), a_raw, b_raw, a_scale, b_scale, rows, dv_, qn, kn,
             reinterpret_cast<float *>(w + p.v32), reinterpret_cast<float *>(w + p.d32),
             reinterpret_cast<float *>(w + p.la), reinterpret_cast<float *>(w + p.be));
     cudaError_t e = cudaGetLastError();
@@ -165,7 +167,7 @@ int run_fused_bwd(const void *q_raw, const void *k_raw, const void *v, const flo
     }
     const int rc = gdn_chunk_bwd(qn, kn, w + p.v32, reinterpret_cast<const float *>(w + p.la),
                                  reinterpret_cast<const float *>(w + p.be), S0, w + p.d32, dS_final, dq_raw, dk_raw,
-                                 dv, dla, dbe, dS0, B, T, H, D, D, 64, cu_seqlens, GDN_DTYPE_F32, w + p.ws,
+                                 dv, dla, dbe, dS0, B, T, H, D, dv_, 64, cu_seqlens, GDN_DTYPE_F32, w + p.ws,
                                  p.ws_bytes, stream);
     if (rc != GDN_OK) return rc;
     if (blocks)
@@ -190,9 +192,9 @@ extern "C" {
 
 size_t gdn_chunk_bwd_fused_workspace_bytes(int B, int T, int H, int dk, int dv, int chunk, int varlen)
 {
-    if (dk != D || dv != D || chunk != 64) return (size_t)-1;
+    if (dk != D || (dv != 64 && dv != 128 && dv != 256) || chunk != 64) return (size_t)-1;
     FusedBwdPlan p;
-    if (!fused_bwd_plan(p, B, T, H, varlen)) return (size_t)-1;
+    if (!fused_bwd_plan(p, B, T, H, dv, varlen)) return (size_t)-1;
     return p.total;
 }
 
@@ -207,8 +209,9 @@ int gdn_chunk_bwd_fused(const void *q_raw, const void *k_raw, const void *v, con
         set_error("gdn_chunk_bwd_fused: unknown dtype %d", dtype);
         return GDN_ERR_UNSUPPORTED;
     }
-    if (dk != D || dv_ != D || chunk != 64) {
-        set_error("gdn_chunk_bwd_fused: dk=%d dv=%d chunk=%d, supported: 64, 64, 64", dk, dv_, chunk);
+    if (dk != D || (dv_ != 64 && dv_ != 128 && dv_ != 256) || chunk != 64) {
+        set_error("gdn_chunk_bwd_fused: dk=%d dv=%d chunk=%d, supported: dk 64, dv 64, 128 or 256, chunk 64", dk,
+                  dv_, chunk);
         return GDN_ERR_UNSUPPORTED;
     }
     if (!(a_scale >= 0.f) || !(a_scale < INFINITY) || !(b_scale >= 0.f && b_scale <= 2.f)) {
@@ -217,7 +220,7 @@ int gdn_chunk_bwd_fused(const void *q_raw, const void *k_raw, const void *v, con
         return GDN_ERR_INVALID_ARGUMENT;
     }
     FusedBwdPlan p;
-    if (!fused_bwd_plan(p, B, T, H, varlen))  // the backward's own checks give the reason
+    if (!fused_bwd_plan(p, B, T, H, dv_, varlen))  // the backward's own checks give the reason
         return gdn_chunk_bwd(nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr,
                              nullptr, nullptr, nullptr, nullptr, nullptr, B, T, H, dk, dv_, chunk, cu_seqlens,
                              GDN_DTYPE_F32, nullptr, 0, stream);
@@ -244,10 +247,10 @@ int gdn_chunk_bwd_fused(const void *q_raw, const void *k_raw, const void *v, con
     char *w = static_cast<char *>(workspace);
     return dtype == GDN_DTYPE_BF16
                ? run_fused_bwd<__nv_bfloat16>(q_raw, k_raw, v, a_raw, b_raw, S0, dout, dS_final, dq_raw, dk_raw,
-                                              dv, da_raw, db_raw, dS0, B, T, H, cu_seqlens, a_scale, b_scale, w, p,
-                                              stream)
+                                              dv, da_raw, db_raw, dS0, B, T, H, dv_, cu_seqlens, a_scale, b_scale, w,
+                                              p, stream)
                : run_fused_bwd<float>(q_raw, k_raw, v, a_raw, b_raw, S0, dout, dS_final, dq_raw, dk_raw, dv,
-                                      da_raw, db_raw, dS0, B, T, H, cu_seqlens, a_scale, b_scale, w, p, stream);
+                                      da_raw, db_raw, dS0, B, T, H, dv_, cu_seqlens, a_scale, b_scale, w, p, stream);
 }
 
 }  // extern "C"

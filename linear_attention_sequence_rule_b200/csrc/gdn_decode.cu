@@ -15,6 +15,11 @@
 // streaming stores.  The state is touched by no other CTA, so there is no inter-CTA traffic.
 // A value head of VB x DV columns runs as VB CTAs per state (blockIdx.y = column block): value
 // columns do not interact in the step, so each CTA updates its own columns of every row.
+// PRO (gdn_decode_step_fused): q, k are raw rows and log_alpha, beta hold the raw gate projections
+// a, b; the kernel forms k / sqrt(|k|^2 + 1e-6), q likewise, log alpha = -a_scale softplus(a)
+// (a = +inf: an exact reset) and beta = b_scale sigmoid(b).  The norms come out of the same
+// block reduction as k . q, and the scales are applied to the reduced sums, so the state is still
+// read and written once.
 #include <cuda_bf16.h>
 
 #include "gdn_internal.h"
@@ -22,6 +27,14 @@
 
 namespace gdn {
 namespace {
+
+__device__ __forceinline__ float sigmoid_f(float x)
+{
+    const float e = expf(-fabsf(x));
+    return x >= 0.f ? 1.f / (1.f + e) : e / (1.f + e);
+}
+
+__device__ __forceinline__ float softplus_f(float x) { return x > 0.f ? x + log1pf(expf(-x)) : log1pf(expf(x)); }
 
 __device__ __forceinline__ float to_f32(float x) { return x; }
 __device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
@@ -33,11 +46,11 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(flo
 
 constexpr int kThreads = 256;
 
-template <int DK, int DV, int VB, typename TIn>
+template <int DK, int DV, int VB, typename TIn, bool PRO>
 __global__ void __launch_bounds__(kThreads, 2)
 decode_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const TIn *__restrict__ v,
               const float *__restrict__ log_alpha, const float *__restrict__ beta,
-              float *__restrict__ S, TIn *__restrict__ out, int H, int G)
+              float *__restrict__ S, TIn *__restrict__ out, int H, int G, float a_scale, float b_scale)
 {
     constexpr int TPR = DV / 4;          // threads per state row (one float4 each)
     constexpr int RPP = kThreads / TPR;  // rows covered per pass
@@ -48,6 +61,7 @@ decode_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const TIn *_
     __shared__ float4 red_r[RPP][TPR];
     __shared__ float4 red_s[RPP][TPR];
     __shared__ float red_kq[RPP];
+    __shared__ float red_kk[PRO ? RPP : 1], red_qq[PRO ? RPP : 1];
 
     const size_t u = blockIdx.x;  // state index n * H + h
     const int tid = threadIdx.x;
@@ -70,8 +84,15 @@ decode_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const TIn *_
         kr[p] = to_f32(kp[rg + p * RPP]);
         qr[p] = to_f32(qp[rg + p * RPP]);
     }
-    const float a = expf(log_alpha[u]);
-    const float b = beta[u];
+    float a, b;
+    if constexpr (PRO) {
+        const float ar = log_alpha[u];
+        a = ar == INFINITY ? 0.f : expf(-a_scale * softplus_f(ar));
+        b = b_scale * sigmoid_f(beta[u]);
+    } else {
+        a = expf(log_alpha[u]);
+        b = beta[u];
+    }
     float vv[4];
     {
         const TIn *vp = v + u * LDV + col0 + 4 * c4;
@@ -81,9 +102,13 @@ decode_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const TIn *_
 
     // partial column sums over this thread's rows
     float4 pr = make_float4(0.f, 0.f, 0.f, 0.f), ps = pr;
-    float pkq = 0.f;
+    float pkq = 0.f, pkk = 0.f, pqq = 0.f;
 #pragma unroll
     for (int p = 0; p < R; ++p) {
+        if constexpr (PRO) {
+            pkk = fmaf(kr[p], kr[p], pkk);
+            pqq = fmaf(qr[p], qr[p], pqq);
+        }
         pr.x = fmaf(s[p].x, kr[p], pr.x); pr.y = fmaf(s[p].y, kr[p], pr.y);
         pr.z = fmaf(s[p].z, kr[p], pr.z); pr.w = fmaf(s[p].w, kr[p], pr.w);
         ps.x = fmaf(s[p].x, qr[p], ps.x); ps.y = fmaf(s[p].y, qr[p], ps.y);
@@ -92,7 +117,13 @@ decode_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const TIn *_
     }
     red_r[rg][c4] = pr;
     red_s[rg][c4] = ps;
-    if (c4 == 0) red_kq[rg] = pkq;
+    if (c4 == 0) {
+        red_kq[rg] = pkq;
+        if constexpr (PRO) {
+            red_kk[rg] = pkk;
+            red_qq[rg] = pqq;
+        }
+    }
     __syncthreads();
 
     float4 r = make_float4(0.f, 0.f, 0.f, 0.f), sq = r;
@@ -103,6 +134,20 @@ decode_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const TIn *_
         r.x += x.x; r.y += x.y; r.z += x.z; r.w += x.w;
         sq.x += y.x; sq.y += y.y; sq.z += y.z; sq.w += y.w;
         kq += red_kq[g];
+    }
+    if constexpr (PRO) {  // S^T k, S^T q and k . q of the normalised rows from the raw sums
+        float kk = 0.f, qq = 0.f;
+#pragma unroll
+        for (int g = 0; g < RPP; ++g) {
+            kk += red_kk[g];
+            qq += red_qq[g];
+        }
+        const float rk = 1.f / sqrtf(kk + 1e-6f), rq = 1.f / sqrtf(qq + 1e-6f);
+        r.x *= rk; r.y *= rk; r.z *= rk; r.w *= rk;
+        sq.x *= rq; sq.y *= rq; sq.z *= rq; sq.w *= rq;
+        kq *= rk * rq;
+#pragma unroll
+        for (int p = 0; p < R; ++p) kr[p] *= rk;
     }
     // u = b (v - a r)
     const float u0 = b * (vv[0] - a * r.x), u1 = b * (vv[1] - a * r.y);
@@ -126,22 +171,22 @@ decode_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const TIn *_
     }
 }
 
-template <typename TIn>
+template <typename TIn, bool PRO>
 cudaError_t launch_typed(const void *q, const void *k, const void *v, const float *la,
                          const float *be, float *S, void *out, int NH, int H, int G, int dk, int dv,
-                         cudaStream_t st)
+                         float as, float bs, cudaStream_t st)
 {
     const dim3 grid(NH), block(kThreads);
     const TIn *Q = static_cast<const TIn *>(q), *K = static_cast<const TIn *>(k),
               *V = static_cast<const TIn *>(v);
     TIn *O = static_cast<TIn *>(out);
     const dim3 grid2(NH, 2);  // dv = 256: two 128-column blocks per state
-    if (dk == 128 && dv == 256) decode_kernel<128, 128, 2, TIn><<<grid2, block, 0, st>>>(Q, K, V, la, be, S, O, H, G);
-    else if (dk == 64 && dv == 256) decode_kernel<64, 128, 2, TIn><<<grid2, block, 0, st>>>(Q, K, V, la, be, S, O, H, G);
-    else if (dk == 128 && dv == 128) decode_kernel<128, 128, 1, TIn><<<grid, block, 0, st>>>(Q, K, V, la, be, S, O, H, G);
-    else if (dk == 128 && dv == 64) decode_kernel<128, 64, 1, TIn><<<grid, block, 0, st>>>(Q, K, V, la, be, S, O, H, G);
-    else if (dk == 64 && dv == 128) decode_kernel<64, 128, 1, TIn><<<grid, block, 0, st>>>(Q, K, V, la, be, S, O, H, G);
-    else decode_kernel<64, 64, 1, TIn><<<grid, block, 0, st>>>(Q, K, V, la, be, S, O, H, G);
+    if (dk == 128 && dv == 256) decode_kernel<128, 128, 2, TIn, PRO><<<grid2, block, 0, st>>>(Q, K, V, la, be, S, O, H, G, as, bs);
+    else if (dk == 64 && dv == 256) decode_kernel<64, 128, 2, TIn, PRO><<<grid2, block, 0, st>>>(Q, K, V, la, be, S, O, H, G, as, bs);
+    else if (dk == 128 && dv == 128) decode_kernel<128, 128, 1, TIn, PRO><<<grid, block, 0, st>>>(Q, K, V, la, be, S, O, H, G, as, bs);
+    else if (dk == 128 && dv == 64) decode_kernel<128, 64, 1, TIn, PRO><<<grid, block, 0, st>>>(Q, K, V, la, be, S, O, H, G, as, bs);
+    else if (dk == 64 && dv == 128) decode_kernel<64, 128, 1, TIn, PRO><<<grid, block, 0, st>>>(Q, K, V, la, be, S, O, H, G, as, bs);
+    else decode_kernel<64, 64, 1, TIn, PRO><<<grid, block, 0, st>>>(Q, K, V, la, be, S, O, H, G, as, bs);
     return cudaGetLastError();
 }
 
@@ -149,12 +194,19 @@ cudaError_t launch_typed(const void *q, const void *k, const void *v, const floa
 
 cudaError_t launch_decode(const void *q, const void *k, const void *v, const float *log_alpha,
                           const float *beta, float *S, void *out, int N, int H, int dk, int dv,
-                          int dtype, cudaStream_t stream, int G)
+                          int dtype, cudaStream_t stream, int G, int prologue, float a_scale, float b_scale)
 {
     const int NH = N * H;
+    if (prologue)
+        return dtype == GDN_DTYPE_BF16
+                   ? launch_typed<__nv_bfloat16, true>(q, k, v, log_alpha, beta, S, out, NH, H, G, dk, dv, a_scale,
+                                                       b_scale, stream)
+                   : launch_typed<float, true>(q, k, v, log_alpha, beta, S, out, NH, H, G, dk, dv, a_scale, b_scale,
+                                               stream);
     if (dtype == GDN_DTYPE_BF16)
-        return launch_typed<__nv_bfloat16>(q, k, v, log_alpha, beta, S, out, NH, H, G, dk, dv, stream);
-    return launch_typed<float>(q, k, v, log_alpha, beta, S, out, NH, H, G, dk, dv, stream);
+        return launch_typed<__nv_bfloat16, false>(q, k, v, log_alpha, beta, S, out, NH, H, G, dk, dv, 0.f, 0.f,
+                                                  stream);
+    return launch_typed<float, false>(q, k, v, log_alpha, beta, S, out, NH, H, G, dk, dv, 0.f, 0.f, stream);
 }
 
 }  // namespace gdn

@@ -15,7 +15,8 @@ void set_error(const char *fmt, ...);
 // C-ABI layer and return the cudaError_t of the launch.
 cudaError_t launch_decode(const void *q, const void *k, const void *v, const float *log_alpha,
                           const float *beta, float *S, void *out, int N, int H, int dk, int dv,
-                          int dtype, cudaStream_t stream, int G = 1);
+                          int dtype, cudaStream_t stream, int G = 1, int prologue = 0, float a_scale = 0.f,
+                          float b_scale = 0.f);
 
 struct ChunkArgs {
     const void *q, *k, *v;

@@ -140,6 +140,17 @@ def test_decode_rejects_bad_arguments(kw, code):
     assert gdn.gdn_last_error() != ""
 
 
+def test_fused_decode_rejects_bad_arguments():
+    a = dict(q_raw=FAKE, k_raw=FAKE, v=FAKE, a_raw=FAKE, b_raw=FAKE, S_inout=FAKE, out=FAKE, N=1, H=1, dk=128,
+             dv=128, dtype=gdn.GDN_DTYPE_BF16, a_scale=1.0, b_scale=1.0, stream=None)
+    assert gdn.gdn_decode_step_fused(**(a | dict(dk=96))) == gdn.GDN_ERR_UNSUPPORTED
+    assert gdn.gdn_decode_step_fused(**(a | dict(b_scale=2.5))) == gdn.GDN_ERR_INVALID_ARGUMENT
+    assert gdn.gdn_decode_step_fused(**(a | dict(a_scale=-1.0))) == gdn.GDN_ERR_INVALID_ARGUMENT
+    assert gdn.gdn_decode_step_fused(**(a | dict(a_scale=float("inf")))) == gdn.GDN_ERR_INVALID_ARGUMENT
+    assert gdn.gdn_decode_step_fused(**(a | dict(out=FAKE + 2))) == gdn.GDN_ERR_INVALID_ARGUMENT
+    assert "gdn_decode_step_fused" in gdn.gdn_last_error()
+
+
 def test_torch_layer_checks_shapes_without_launching():
     import torch
     q = torch.zeros(1, 64, 1, 64)
@@ -247,6 +258,9 @@ def test_fused_backward_rejects_before_any_launch():
     assert call(dout=FAKE + 4) == gdn.GDN_ERR_INVALID_ARGUMENT
     assert call(workspace=None) == gdn.GDN_ERR_WORKSPACE
     assert gdn.gdn_chunk_bwd_fused_workspace_bytes(1, 64, 1, 128, 64, 64, 0) == ctypes.c_size_t(-1).value
+    assert call(dv_=96) == gdn.GDN_ERR_UNSUPPORTED
+    assert gdn.gdn_chunk_bwd_fused_workspace_bytes(1, 64, 1, 64, 256, 64, 0) > \
+        gdn.gdn_chunk_bwd_fused_workspace_bytes(1, 64, 1, 64, 64, 64, 0)
 
 
 def test_grouped_backward_rejects_bad_groups():

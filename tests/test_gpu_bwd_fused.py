@@ -2,7 +2,7 @@
 raw projections) against the fp64 oracle (oracle/prologue.py backward_fused, pinned by finite
 differences in tests/test_oracle_prologue_backward.py), on the same seeded raw inputs: dense and
 varlen, bf16 and fp32 inputs, an exact reset (a = +inf), b_scale 1 and 2, with and without S0 and
-dS_final.
+dS_final, value head sizes 64, 128 and 256.
 
 The prologue and the recurrence's backward run in fp32 on the stored input values (the oracle
 reads the same values in fp64), so the bound is the plain backward's: max |g - g_ref| <= 1e-5 *
@@ -60,3 +60,11 @@ def test_varlen_reset_and_beta_scale_two():
     inp["a_raw"][70, 1] = float("inf")  # log alpha = -inf: an exact reset
     errs = check(inp, 2, with_dsf=False)
     assert errs["da_raw"] <= RTOL
+
+
+@pytest.mark.parametrize("dv,lengths", [(128, None), (256, [70, 0, 129])])
+def test_value_heads_128_and_256(dv, lengths):
+    kw = dict(lengths=lengths) if lengths else dict(B=2, T=150)
+    inp = workloads.make_raw_chunk_inputs(H=2, dk=64, dv=dv, dtype="bf16", seed=63 + dv, s0_std=0.1, la_scale=0.3,
+                                          **kw)
+    check(inp, 3)

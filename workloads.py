@@ -223,3 +223,20 @@ def make_decode_step_inputs(N, H, dk, dv, dtype="bf16", seed=0, step=0, beta_sca
     log_alpha = (-torch.nn.functional.softplus(la_std * torch.randn(N, H, generator=g))
                  * la_scale).float()
     return dict(q=q, k=k, v=v, log_alpha=log_alpha, beta=beta)
+
+
+def make_raw_decode_step_inputs(N, H, dk, dv, dtype="bf16", seed=0, step=0, beta_scale=1.0, la_std=1.0,
+                                la_scale=1.0, **_ignored):
+    """Raw-projection inputs of decode step ``step`` for the fused decode entry: q_raw, k_raw
+    ~ N(0, 1) [N,H,dk] and v ~ N(0, 1) [N,H,dv] in dtype; b_raw ~ N(0, 1) and a_raw ~ N(0, la_std)
+    [N,H] fp32; a_scale = la_scale, b_scale = beta_scale.  One generator per step, as
+    ``make_decode_step_inputs``."""
+    g = torch.Generator().manual_seed(int(seed) * 1_000_003 + int(step) + 1)
+    dt = DTYPES[dtype]
+    q_raw = torch.randn(N, H, dk, generator=g).to(dt)
+    k_raw = torch.randn(N, H, dk, generator=g).to(dt)
+    v = torch.randn(N, H, dv, generator=g).to(dt)
+    b_raw = torch.randn(N, H, generator=g).float()
+    a_raw = (la_std * torch.randn(N, H, generator=g)).float()
+    return dict(q_raw=q_raw, k_raw=k_raw, v=v, a_raw=a_raw, b_raw=b_raw, a_scale=float(la_scale),
+                b_scale=float(beta_scale))
