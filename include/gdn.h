@@ -210,7 +210,7 @@ GDN_API size_t gdn_chunk_fwd_host_workspace_bytes(int B, int T, int H, int dk, i
  *     log_lam, beta [.., H] fp32; M0, M_final [B, H, dv, dk, 2] fp32 (re, im), either may be NULL.
  * log_lam must be finite (lam > 0): the computation runs the real gated delta rule at head size
  * 2 dk with a = lam and b = beta / lam (see gdn_phase.cu), on the tcgen05 kernel for bf16 and
- * the fp32 CUDA-core kernel for fp32.  dk in {32, 64}, dv in {64, 128}.  Workspace:
+ * the fp32 CUDA-core kernel for fp32.  dk in {32, 64}, dv in {64, 128}, or 256 with bf16.  Workspace:
  * gdn_phase_fwd_workspace_bytes(...) bytes of device memory, 256-byte aligned.  Errors as
  * gdn_chunk_fwd (the library's own scratch only is written before a late CUDA error).
  */
@@ -223,7 +223,7 @@ GDN_API int gdn_phase_fwd(const float *K, const float *Q, const void *v, const f
 GDN_API size_t gdn_phase_fwd_workspace_bytes(int B, int T, int H, int dk, int dv, int varlen, int dtype);
 
 /*
- * gdn_phase_bwd -- gradients of gdn_phase_fwd for dk = 32 complex (64 real) and dv in {64, 128}:
+ * gdn_phase_bwd -- gradients of gdn_phase_fwd for dk = 32 complex (64 real) and dv in {64, 128, 256}:
  * given the forward's inputs, dout = dL/dout (dtype) and dM_final = dL/dM_final ((re, im) pairs,
  * NULL: zero), it writes fp32
  *     dK, dQ [.., H, 32, 2] (d/dRe, d/dIm pairs), dv [.., H, dv], dlog_lam, dbeta [.., H],

@@ -435,7 +435,7 @@ def phase_fwd(K, Q, v, log_lam, beta, M0=None, cu_seqlens=None, out=None, M_fina
 
 def phase_bwd(K, Q, v, log_lam, beta, dout, M0=None, dM_final=None, cu_seqlens=None, want_dM0=True,
               workspace=None, stream=None):
-    """Gradients of ``phase_fwd`` (dk = 32 complex, dv 64 or 128): returns (dK, dQ complex64, dv fp32,
+    """Gradients of ``phase_fwd`` (dk = 32 complex, dv 64, 128 or 256): returns (dK, dQ complex64, dv fp32,
     dlog_lam, dbeta fp32, dM0 complex64 or None); complex gradients as d/dRe + i d/dIm."""
     Kp, Qp = _as_pairs(K, "K"), _as_pairs(Q, "Q")
     dt = v.dtype

@@ -164,10 +164,12 @@ cudaError_t prologue_for(int dk, int dv, const float *K, const float *Q, const v
                          const float *beta, long token_heads, char *w, const PhasePlan &p, cudaStream_t st)
 {
     if (dk == 64)
-        return dv == 128 ? launch_prologue<64, 128, TV>(K, Q, V, log_lam, beta, token_heads, w, p, st)
-                         : launch_prologue<64, 64, TV>(K, Q, V, log_lam, beta, token_heads, w, p, st);
-    return dv == 128 ? launch_prologue<32, 128, TV>(K, Q, V, log_lam, beta, token_heads, w, p, st)
-                     : launch_prologue<32, 64, TV>(K, Q, V, log_lam, beta, token_heads, w, p, st);
+        return dv == 256   ? launch_prologue<64, 256, TV>(K, Q, V, log_lam, beta, token_heads, w, p, st)
+               : dv == 128 ? launch_prologue<64, 128, TV>(K, Q, V, log_lam, beta, token_heads, w, p, st)
+                           : launch_prologue<64, 64, TV>(K, Q, V, log_lam, beta, token_heads, w, p, st);
+    return dv == 256   ? launch_prologue<32, 256, TV>(K, Q, V, log_lam, beta, token_heads, w, p, st)
+           : dv == 128 ? launch_prologue<32, 128, TV>(K, Q, V, log_lam, beta, token_heads, w, p, st)
+                       : launch_prologue<32, 64, TV>(K, Q, V, log_lam, beta, token_heads, w, p, st);
 }
 
 // ---- backward ---------------------------------------------------------------------------------
@@ -264,7 +266,7 @@ extern "C" {
 
 size_t gdn_phase_fwd_workspace_bytes(int B, int T, int H, int dk, int dv, int varlen, int dtype)
 {
-    if ((dk != 32 && dk != 64) || (dv != 64 && dv != 128)) return (size_t)-1;
+    if ((dk != 32 && dk != 64) || (dv != 64 && dv != 128 && dv != 256)) return (size_t)-1;
     PhasePlan p;
     if (!phase_plan(p, B, T, H, dk, dv, varlen, dtype)) return (size_t)-1;
     return p.total;
@@ -275,9 +277,9 @@ int gdn_phase_fwd(const float *K, const float *Q, const void *v, const float *lo
                   const int32_t *cu_seqlens, int dtype, void *workspace, size_t workspace_bytes, void *stream)
 {
     const int varlen = cu_seqlens != nullptr;
-    if ((dk != 32 && dk != 64) || (dv != 64 && dv != 128)) {
-        set_error("gdn_phase_fwd: dk=%d dv=%d, supported: dk 32 or 64 (the real recurrence runs at 2 dk), dv 64 or "
-                  "128", dk, dv);
+    if ((dk != 32 && dk != 64) || (dv != 64 && dv != 128 && dv != 256)) {
+        set_error("gdn_phase_fwd: dk=%d dv=%d, supported: dk 32 or 64 (the real recurrence runs at 2 dk), dv 64, "
+                  "128 or 256 (256 with bf16)", dk, dv);
         return GDN_ERR_UNSUPPORTED;
     }
     PhasePlan p;
@@ -344,7 +346,7 @@ int gdn_phase_fwd(const float *K, const float *Q, const void *v, const float *lo
 
 size_t gdn_phase_bwd_workspace_bytes(int B, int T, int H, int dk, int dv, int varlen)
 {
-    if (dk != 32 || (dv != 64 && dv != 128)) return (size_t)-1;
+    if (dk != 32 || (dv != 64 && dv != 128 && dv != 256)) return (size_t)-1;
     PhaseBwdPlan p;
     if (!phase_bwd_plan(p, B, T, H, dv, varlen)) return (size_t)-1;
     return p.total;
@@ -356,8 +358,8 @@ int gdn_phase_bwd(const float *K, const float *Q, const void *v, const float *lo
                   const int32_t *cu_seqlens, int dtype, void *workspace, size_t workspace_bytes, void *stream)
 {
     const int varlen = cu_seqlens != nullptr;
-    if (dk != 32 || (dv != 64 && dv != 128) || (dtype != GDN_DTYPE_BF16 && dtype != GDN_DTYPE_F32)) {
-        set_error("gdn_phase_bwd: dk=%d dv=%d dtype=%d, supported: dk 32 (64 real), dv 64 or 128, bf16 or fp32",
+    if (dk != 32 || (dv != 64 && dv != 128 && dv != 256) || (dtype != GDN_DTYPE_BF16 && dtype != GDN_DTYPE_F32)) {
+        set_error("gdn_phase_bwd: dk=%d dv=%d dtype=%d, supported: dk 32 (64 real), dv 64, 128 or 256, bf16 or fp32",
                   dk, dv, dtype);
         return GDN_ERR_UNSUPPORTED;
     }
@@ -403,9 +405,12 @@ int gdn_phase_bwd(const float *K, const float *Q, const void *v, const float *lo
     if (dv == 64)
         e = dtype == GDN_DTYPE_BF16 ? launch_prologue<32, 64, __nv_bfloat16, float>(K, Q, v, log_lam, beta, th, w, fp, st)
                                     : launch_prologue<32, 64, float, float>(K, Q, v, log_lam, beta, th, w, fp, st);
-    else
+    else if (dv == 128)
         e = dtype == GDN_DTYPE_BF16 ? launch_prologue<32, 128, __nv_bfloat16, float>(K, Q, v, log_lam, beta, th, w, fp, st)
                                     : launch_prologue<32, 128, float, float>(K, Q, v, log_lam, beta, th, w, fp, st);
+    else
+        e = dtype == GDN_DTYPE_BF16 ? launch_prologue<32, 256, __nv_bfloat16, float>(K, Q, v, log_lam, beta, th, w, fp, st)
+                                    : launch_prologue<32, 256, float, float>(K, Q, v, log_lam, beta, th, w, fp, st);
     if (e != cudaSuccess) return fail_launch(e);
     const long nv = th * dv;
     float *d32 = reinterpret_cast<float *>(w + p.d32);
@@ -437,7 +442,7 @@ int gdn_phase_bwd(const float *K, const float *Q, const void *v, const float *lo
                                  cu_seqlens, GDN_DTYPE_F32, w + p.ws, p.ws_bytes, stream);
     if (rc != GDN_OK) return rc;
     if (th) {
-        auto epi = dv == 64 ? phase_bwd_epilogue<64> : phase_bwd_epilogue<128>;
+        auto epi = dv == 64 ? phase_bwd_epilogue<64> : dv == 128 ? phase_bwd_epilogue<128> : phase_bwd_epilogue<256>;
         epi<<<(unsigned)((th * 32 + 255) / 256), 256, 0, st>>>(
             dq, dkr, dvr, reinterpret_cast<const float *>(w + p.vr), dla, dbr,
             reinterpret_cast<const float *>(w + p.br), log_lam, th, reinterpret_cast<float2 *>(dK),

@@ -230,6 +230,8 @@ def test_phase_entry_rejects_before_any_launch():
     assert phase_call(dk=48) == gdn.GDN_ERR_UNSUPPORTED
     assert phase_call(dk=128) == gdn.GDN_ERR_UNSUPPORTED   # 2 dk = 256 real columns
     assert phase_call(dv=96) == gdn.GDN_ERR_UNSUPPORTED
+    assert phase_call(dv=256, dtype=gdn.GDN_DTYPE_F32) == gdn.GDN_ERR_UNSUPPORTED  # 256 with bf16 only
+    assert gdn.gdn_phase_fwd_workspace_bytes(1, 64, 1, 32, 256, 0, gdn.GDN_DTYPE_BF16) != ctypes.c_size_t(-1).value
     assert phase_call(B=0) == gdn.GDN_ERR_INVALID_ARGUMENT
     assert phase_call(K=None) == gdn.GDN_ERR_INVALID_ARGUMENT
     assert phase_call(out=None) == gdn.GDN_ERR_INVALID_ARGUMENT
@@ -280,7 +282,7 @@ def test_phase_backward_rejects_before_any_launch():
              dv_out=FAKE, dlog_lam=FAKE, dbeta=FAKE, dM0=None, B=1, T=64, H=1, dk=32, dv=64, cu_seqlens=None,
              dtype=gdn.GDN_DTYPE_BF16, workspace=FAKE * 256, workspace_bytes=1 << 40, stream=None)
     assert gdn.gdn_phase_bwd(**dict(a, dk=64)) == gdn.GDN_ERR_UNSUPPORTED   # the backward takes 64 real columns
-    assert gdn.gdn_phase_bwd(**dict(a, dv=256)) == gdn.GDN_ERR_UNSUPPORTED
+    assert gdn.gdn_phase_bwd(**dict(a, dv=512)) == gdn.GDN_ERR_UNSUPPORTED
     assert gdn.gdn_phase_bwd_workspace_bytes(1, 64, 1, 32, 128, 0) > gdn.gdn_phase_bwd_workspace_bytes(1, 64, 1, 32, 64, 0)
     assert gdn.gdn_phase_bwd(**dict(a, dQ=None)) == gdn.GDN_ERR_INVALID_ARGUMENT
     assert gdn.gdn_phase_bwd(**dict(a, K=FAKE + 4)) == gdn.GDN_ERR_INVALID_ARGUMENT

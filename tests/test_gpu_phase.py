@@ -45,7 +45,7 @@ def check(inp):
     return errs
 
 
-@pytest.mark.parametrize("dk,dv", [(32, 64), (64, 64), (64, 128), (32, 128)])
+@pytest.mark.parametrize("dk,dv", [(32, 64), (64, 64), (64, 128), (32, 128), (32, 256), (64, 256)])
 def test_dense_bf16_with_initial_state(dk, dv):
     check(workloads.make_phase_inputs(B=2, T=300, H=3, dk=dk, dv=dv, dtype="bf16", seed=500 + dk + dv, m0_std=0.05))
 

@@ -1,5 +1,5 @@
 """GPU parity of gdn_phase_bwd (gradients of the complex-phase delta memory, dk = 32 complex,
-dv = 64 and 128) against the fp64 phase backward oracle (oracle/phase.py backward, pinned by finite
+dv = 64, 128 and 256) against the fp64 phase backward oracle (oracle/phase.py backward, pinned by finite
 differences of the complex definition in tests/test_oracle_phase.py): dense and varlen, bf16 and
 fp32 values, unit and Laplace keys, with and without M0 and dM_final.  The backward runs in fp32
 on the stored inputs, so the bound is the plain backward's: max |g - g_ref| <= 1e-5 *
@@ -71,3 +71,7 @@ def test_varlen_ragged_beta_two():
 def test_value_head_128_varlen():
     check(workloads.make_phase_inputs(H=2, dk=32, dv=128, dtype="bf16", seed=604, m0_std=0.05,
                                       lengths=[70, 0, 129, 1]), 4)
+
+
+def test_value_head_256_dense_fp32():
+    check(workloads.make_phase_inputs(B=1, T=150, H=2, dk=32, dv=256, dtype="f32", seed=605, m0_std=0.05), 5)

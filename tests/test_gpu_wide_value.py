@@ -120,3 +120,23 @@ def test_decode_equals_two_column_halves_bitwise(dtype):
         assert torch.equal(o, torch.cat(o_h, dim=-1)), step
     gdn.device_status()
     assert torch.equal(S, torch.cat(S_halves, dim=-1))
+
+
+def test_decode_grouped_value_heads():
+    import linear_attention_sequence_rule_b200 as gdn
+    from tests.parity import TOL
+    N, Hk, Hv, dk = 2, 1, 3, 128
+    S = workloads.make_decode_state(N, Hv, dk, DV, seed=31)
+    S_dev, S_ref = S.cuda(), S.double().numpy()
+    g = torch.Generator().manual_seed(31)
+    for step in range(6):
+        q = torch.nn.functional.normalize(torch.randn(N, Hk, dk, generator=g), dim=-1).to(torch.bfloat16)
+        k = torch.nn.functional.normalize(torch.randn(N, Hk, dk, generator=g), dim=-1).to(torch.bfloat16)
+        v = torch.randn(N, Hv, DV, generator=g).to(torch.bfloat16)
+        la = (-0.3 * torch.nn.functional.softplus(torch.randn(N, Hv, generator=g))).float()
+        be = torch.sigmoid(torch.randn(N, Hv, generator=g)).float()
+        o = gdn.decode_step_gva(q.cuda(), k.cuda(), v.cuda(), la.cuda(), be.cuda(), S_dev)
+        o_ref, S_ref = grouped.decode_step_gva(q, k, v, la, be, S_ref)
+        assert max_abs(f64(o), o_ref) <= TOL["bf16"], step
+    gdn.device_status()
+    assert max_abs(f64(S_dev), S_ref) <= TOL["bf16"]
