@@ -1194,13 +1194,14 @@ __global__ void __launch_bounds__(256) seg_combine_kernel(const float *__restric
     }
 }
 
-// vblocks > 1: a value head of vblocks x DV columns, one CTA per column block (no segment scan;
-// the column blocks already multiply the CTAs per chain)
+// vblocks > 1: a value head of vblocks x DV columns, one CTA per column block in every pass (the
+// transitions of the segment scan do not depend on V and run once per chain)
 template <int DK, int DV>
 cudaError_t run_chunk(const ChunkArgs &a, cudaStream_t st, int vblocks = 1)
 {
     const long tokens = a.cu_seqlens ? (long)a.T : (long)a.B * a.T;
-    const SegPlan p = vblocks > 1 ? SegPlan{} : plan_segments(a.B, a.T, a.H, a.cu_seqlens != nullptr, a.dtype);
+    const int dv = DV * vblocks;
+    const SegPlan p = plan_segments(a.B, a.T, a.H * vblocks, a.cu_seqlens != nullptr, a.dtype);
     const int pf = a.prologue ? kFlagPrologue : 0;
     const float as = a.a_scale, bs = a.b_scale;
     if (p.G <= 1) {
@@ -1210,15 +1211,16 @@ cudaError_t run_chunk(const ChunkArgs &a, cudaStream_t st, int vblocks = 1)
         t.vblocks = vblocks;
         return launch_tc<DK, DV>(t, st);
     }
-    const SegWork w = seg_layout(a.workspace, a.B, a.H, DK, DV, p);
+    const SegWork w = seg_layout(a.workspace, a.B, a.H, DK, dv, p);
     const int nseg = a.B * p.G;
     seg_table_kernel<<<(nseg + 256) / 256, 256, 0, st>>>(w.cu, a.B, a.T, p.G, p.L);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     // pass A: local states from zero, and transitions from the identity with V = 0
-    e = launch_tc<DK, DV>(TcLaunch{a.q, a.k, a.v, a.log_alpha, a.beta, nullptr, nullptr, w.Sloc, w.cu, nseg,
-                                   a.T, a.H, tokens, pf, as, bs, a.G},
-                          st);
+    TcLaunch ta{a.q, a.k, a.v, a.log_alpha, a.beta, nullptr, nullptr, w.Sloc, w.cu, nseg, a.T, a.H, tokens, pf, as, bs,
+                a.G};
+    ta.vblocks = vblocks;
+    e = launch_tc<DK, DV>(ta, st);
     if (e != cudaSuccess) return e;
     e = launch_tc<DK, DK>(TcLaunch{a.q, a.k, nullptr, a.log_alpha, a.beta, nullptr, nullptr, w.M, w.cu, nseg,
                                    a.T, a.H, tokens, kFlagVZero | kFlagS0Identity | pf, as, bs, a.G},
@@ -1228,22 +1230,22 @@ cudaError_t run_chunk(const ChunkArgs &a, cudaStream_t st, int vblocks = 1)
     const int shm = (DK * (DK + 2) + 2 * DK * 32) * (int)sizeof(float);
     e = cudaFuncSetAttribute(seg_combine_kernel<DK>, cudaFuncAttributeMaxDynamicSharedMemorySize, shm);
     if (e != cudaSuccess) return e;
-    seg_combine_kernel<DK><<<dim3(DV / 32, a.H, a.B), 256, shm, st>>>(w.M, w.Sloc, a.S0, w.Sin, a.S_final, p.G,
-                                                                      a.H, DV);
+    seg_combine_kernel<DK><<<dim3(dv / 32, a.H, a.B), 256, shm, st>>>(w.M, w.Sloc, a.S0, w.Sin, a.S_final, p.G,
+                                                                      a.H, dv);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     // pass C: outputs of every segment from its entry state
-    return launch_tc<DK, DV>(TcLaunch{a.q, a.k, a.v, a.log_alpha, a.beta, w.Sin, a.out, nullptr, w.cu, nseg,
-                                      a.T, a.H, tokens, pf, as, bs, a.G},
-                             st);
+    TcLaunch tc{a.q, a.k, a.v, a.log_alpha, a.beta, w.Sin, a.out, nullptr, w.cu, nseg, a.T, a.H, tokens, pf, as, bs,
+                a.G};
+    tc.vblocks = vblocks;
+    return launch_tc<DK, DV>(tc, st);
 }
 
 }  // namespace
 
 size_t chunk_tc_workspace_bytes(int B, int T, int H, int dk, int dv, int varlen, int dtype)
 {
-    if (dv > 128) return 0;  // column blocks, no segment scan
-    const SegPlan p = plan_segments(B, T, H, varlen, dtype);
+    const SegPlan p = plan_segments(B, T, H * (dv > 128 ? dv / 128 : 1), varlen, dtype);
     if (p.G <= 1) return 0;
     return seg_layout(nullptr, B, H, dk, dv, p).bytes;
 }

@@ -140,3 +140,22 @@ def test_decode_grouped_value_heads():
         assert max_abs(f64(o), o_ref) <= TOL["bf16"], step
     gdn.device_status()
     assert max_abs(f64(S_dev), S_ref) <= TOL["bf16"]
+
+
+def test_segment_scan_path():
+    # one sequence, two heads, 40 chunks: 4 column-block chains, so the long sequence is cut into
+    # segments (a workspace is needed); parity against the oracle, and bit identity with two
+    # 128-column calls, which cut the sequence the same way
+    import linear_attention_sequence_rule_b200 as gdn
+    inp = workloads.make_chunk_inputs(B=1, T=40 * 64, H=2, dk=128, dv=DV, dtype="bf16", seed=37, s0_std=0.1,
+                                      la_scale=0.1)
+    assert gdn.workspace_bytes(1, 40 * 64, 2, 128, DV) > 0
+    out, Sf = run_gpu_chunk(inp)
+    e_o, e_s = compare_chunk(inp, out, Sf)
+    assert e_o <= TOL["bf16"] and e_s <= TOL["bf16"], (e_o, e_s)
+    d = {k: (v.cuda() if torch.is_tensor(v) else v) for k, v in inp.items()}
+    halves = [gdn.chunk_fwd(d["q"], d["k"], d["v"][..., c].contiguous(), d["log_alpha"], d["beta"],
+                            S0=d["S0"][..., c].contiguous()) for c in (slice(0, 128), slice(128, 256))]
+    gdn.device_status()
+    assert torch.equal(out, torch.cat([h[0] for h in halves], dim=-1))
+    assert torch.equal(Sf, torch.cat([h[1] for h in halves], dim=-1))
