@@ -23,7 +23,8 @@ namespace {
 // 32 MiB.  The segment scan keeps per (segment, head) a local state and an entry state
 // (dk x dv fp32) and a transition (dk x dk fp32), with segments x heads bounded by the SM count,
 // plus a small offset table: 3 * 148 * 128 * 128 * 4 B = 29.1 MB for dk = dv = 128 on a 148-SM
-// device, the largest case there.
+// device, the largest case there (dv = 256 counts its two column blocks as chains, which halves
+// segments x heads: 74 * (2 * 128 * 256 + 128 * 128) * 4 B = 24.2 MB).
 constexpr size_t kScratchBytes = size_t(32) << 20;
 constexpr int kMaxDevices = 64;
 
