@@ -1,0 +1,52 @@
+"""The benchmark's roofline arithmetic against counts made from first principles (CPU only).
+
+The algorithmic flops of the chunk forward are counted here product by product over one chunk of
+C tokens -- the multiply-adds of each triangular product enumerated row by row, the dense products
+as 2 C dk dv each, the unit-lower inverse at its standard C^3/3 -- and compared with
+``bench.algo_flops`` per token-head. Bytes are the tensors each call must move once.  The figures quoted with the results (46,357 and
+140,501 flops per token-head; 132,104 bytes per decode state at d = 128) are checked as well."""
+import bench
+
+
+def macs_lower(C, inclusive):
+    """Multiply-adds of one output column of a (strictly or inclusively) lower C x C product."""
+    return sum(r + 1 if inclusive else r for r in range(C))
+
+
+def chunk_flops_per_token(C, dk, dv):
+    f = 0
+    f += 2 * dk * macs_lower(C, False)        # K K^T, strictly lower
+    f += 2 * dk * macs_lower(C, True)         # Q K^T, lower inclusive
+    f += 2 * dk * macs_lower(C, False)        # W = T diag(b gam) K with T unit lower
+    f += 2 * dv * macs_lower(C, False)        # U~ = T diag(b) V
+    f += 2 * dv * macs_lower(C, True)         # P U, P lower inclusive
+    f += C ** 3 / 3                           # T = (I + A)^{-1}
+    f += 3 * 2 * C * dk * dv                  # W S, (gam Q) S, K^T diag(lam) U
+    return f / C
+
+
+def test_chunk_flops_match_the_product_count():
+    for dk, dv in ((64, 64), (128, 128), (64, 128), (128, 64), (128, 256)):
+        assert abs(bench.algo_flops(1, dk, dv) - chunk_flops_per_token(64, dk, dv)) < 1e-9, (dk, dv)
+    assert round(bench.algo_flops(1, 64, 64)) == 46357
+    assert round(bench.algo_flops(1, 128, 128)) == 140501
+    assert bench.algo_flops(7, 64, 64) == 7 * bench.algo_flops(1, 64, 64)
+
+
+def test_chunk_bytes_are_each_tensor_once():
+    th, n_states = 1000, 10
+    for dk, dv, e in ((64, 64, 2), (128, 256, 2), (64, 64, 4)):
+        q = k = th * dk * e
+        v = out = th * dv * e
+        gates = th * 2 * 4
+        state = n_states * dk * dv * 4
+        assert bench.algo_bytes(th, n_states, dk, dv, e, False, False) == q + k + v + out + gates
+        assert bench.algo_bytes(th, n_states, dk, dv, e, True, True) == q + k + v + out + gates + 2 * state
+        assert bench.algo_bytes(th, n_states, dk, dv, e, True, False) == q + k + v + out + gates + state
+
+
+def test_decode_bytes_per_state():
+    dk = dv = 128
+    state_read_and_write = 2 * dk * dv * 4
+    q_k_v_out = (dk + dk + dv + dv) * 2
+    assert bench.DECODE_BYTES_PER_STATE(dk, dv, 2) == state_read_and_write + q_k_v_out + 8 == 132104
