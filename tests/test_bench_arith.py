@@ -3,8 +3,9 @@
 The algorithmic flops of the chunk forward are counted here product by product over one chunk of
 C tokens -- the multiply-adds of each triangular product enumerated row by row, the dense products
 as 2 C dk dv each, the unit-lower inverse at its standard C^3/3 -- and compared with
-``bench.algo_flops`` per token-head. Bytes are the tensors each call must move once.  The figures quoted with the results (46,357 and
-140,501 flops per token-head; 132,104 bytes per decode state at d = 128) are checked as well."""
+``bench.algo_flops`` per token-head. Bytes are the tensors each call must move once. The figures
+quoted with the results (46,357 and 140,501 flops per token-head; 132,104 bytes per decode state
+at d = 128) are checked as well."""
 import bench
 
 
