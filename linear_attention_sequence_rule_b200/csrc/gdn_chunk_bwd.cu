@@ -1,7 +1,8 @@
 // gdn_chunk_bwd.cu -- gradients of the chunk forward (dq, dk, dv, dlog_alpha, dbeta, dS0) with
 // fp32-level accuracy, for dk = 64 and dv = 64 VS, VS in {1, 2, 4} (the training path; Sykra
-// README, "Architectural Highlights": chunk-parallel training through the WY / UT transform).  The 64 x 64 products run
-// on the tensor cores as three tf32 products each; the rest is fp32 on the CUDA cores.
+// README, "Architectural Highlights": chunk-parallel training through the WY / UT transform).
+// The 64 x 64 products run on the tensor cores as three tf32 products each; the rest is fp32 on
+// the CUDA cores.
 //
 // Per chunk of C = 64 tokens with entry state S (the forward's chunk form):
 //   A = strictly_lower(diag(b) (Gam o K K^T)),  T = (I + A)^{-1}
@@ -10,7 +11,7 @@
 // so the chunk maps states and state gradients affinely:
 //   S'  = M S + Bm,              M  = gam_C I - K^T diag(lam) W,   Bm = K^T diag(lam) U~
 //   dS  = M^T dS' + R,           R  = (Q^T diag(gam) - W^T P^T) dO
-// Four kernels:
+// Three kernels (plus the varlen chunk offsets and, when gradients are partial, their sums):
 //   bwd_prep   (chunk x head, parallel)  : T, W, U~, P  ->  M, Bm, R, and T, W, U~ for bwd_grads
 //   bwd_scans  (sequence x head x 2)     : forward, S_c for every chunk from S0; reverse, dS at every
 //                                          chunk's end from dS_final, and dS0 (one launch, both at once)
