@@ -493,6 +493,16 @@ def run_ours(args, world, rank, local):
         del dw
         extra["phase_memory"] = phase_numbers(gdn, 5, 3, flush, stream, peaks)
         extra["decode_small_batch_graph"] = decode_graph_numbers(gdn)
+        # key head size 128 (two key blocks), the hybrid-LM token and head counts at dk = dv = 128;
+        # last of the device work and guarded, so that a failure here is reported in the line
+        # rather than losing it
+        try:
+            dw = to_dev(workloads.make_chunk_inputs(B=8, T=4096, H=12, dk=128, dv=128, dtype="bf16",
+                                                    seed=rank_seed(cfg["seed"], rank), la_scale=0.1))
+            extra["hybrid_lm_backward_dk128"] = backward_numbers(gdn, dw, 3, 3, flush, stream, peaks)
+            del dw
+        except Exception as exc:  # noqa: BLE001  (reported, not hidden)
+            extra["hybrid_lm_backward_dk128"] = {"error": f"{type(exc).__name__}: {exc}"[:300]}
     cpu = None
     if rank == 0 and world == 1:
         cpu = cpu_oracle_baseline(inp)
@@ -556,31 +566,40 @@ def _time_loop(call, steps, warmup, flush, stream):
     return statistics.mean(a0.elapsed_time(b0) for a0, b0 in ev)
 
 
+def bwd_products(KB, VS):
+    """Distinct 64 x 64 x 64 products of the chunk-form backward per (chunk, head) at dk = 64 KB,
+    dv = 64 VS, each counted once: forming T, W, U~, M, Bm, R (4 KB + VS + KB^2 + 2 KB VS, with
+    K K^T, Q K^T, W and P W per key block), the two scans (2 KB^2 VS), and the gradients
+    (5 KB VS + 4 VS + 5 KB + 2: K dS', W S, U dS'^T, dO S^T, dU S^T per key and value block;
+    P^T dO, dO U^T, T^T dU, dU (b V)^T per value block; T^T dW, dW (b gam K)^T, (D + D^T) K, D2^T Q,
+    D2 K per key block; dT T^T and T^T Z).  The gradient kernel's recomputed K K^T and Q K^T are
+    not counted."""
+    return (4 * KB + VS + KB * KB + 2 * KB * VS) + 2 * KB * KB * VS + (5 * KB * VS + 4 * VS + 5 * KB + 2)
+
+
 def backward_numbers(gdn, d, steps, warmup, flush, stream, peaks):
     """The backward of the hybrid-LM step (dq, dk, dv, gate and state gradients; fp32-accurate
     products on the tensor cores as three tf32 terms) from a seeded dout; `d` holds inputs of the
-    hybrid-LM token and head counts (B=8 T=4096 H=12, dk=64) on the device, dv = 64 VS."""
-    dv = d["v"].shape[-1]
-    VS = dv // 64
+    hybrid-LM token and head counts (B=8 T=4096 H=12) on the device, dk = 64 KB, dv = 64 VS."""
+    dk, dv = d["q"].shape[-1], d["v"].shape[-1]
+    KB, VS = dk // 64, dv // 64
     dout = torch.randn(d["v"].shape, device="cuda", generator=torch.Generator("cuda").manual_seed(7)).to(d["v"].dtype)
-    wsb = torch.empty(gdn.gdn_chunk_bwd_workspace_bytes(8, 4096, 12, 64, dv, 64, 0), dtype=torch.uint8,
+    wsb = torch.empty(gdn.gdn_chunk_bwd_workspace_bytes(8, 4096, 12, dk, dv, 64, 0), dtype=torch.uint8,
                       device="cuda")
 
     def call():
         gdn.chunk_bwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], dout, workspace=wsb, stream=stream)
     ms_b = _time_loop(call, steps, warmup, flush, stream)
     # bytes per token-head: q, k, v, dout (bf16) and gates in; dq, dk, dv (fp32) and two gate grads out
-    by_b = 393216 * (2 * 64 * 2 + 2 * dv * 2 + 8 + 2 * 64 * 4 + dv * 4 + 8)
-    # algorithmic work: the 26 distinct 64 x 64 x 64 products the chunk-form backward needs per
-    # (chunk, head) at dv = 64, each counted once -- 8 forming T, W, U~, M, Bm, R; 1 in each scan; 16
-    # for the gradients -- at 2 * 64^3 fp32 flops each (the gradient kernel's recomputed K K^T and
-    # Q K^T are not counted); the tensor cores execute three tf32 products for each.  14 of them
-    # have a value dimension and scale with dv / 64, 12 do not (value splits recompute those per
-    # 64-column block: executed work is 26 VS products, counted here once)
-    fl_b = 6144 * (12 + 14 * VS) * 2 * 64 ** 3
+    by_b = 393216 * (2 * dk * 2 + 2 * dv * 2 + 8 + 2 * dk * 4 + dv * 4 + 8)
+    # algorithmic work: the distinct 64 x 64 x 64 products per (chunk, head) (bwd_products: 26 at
+    # dk = dv = 64), at 2 * 64^3 fp32 flops each; the tensor cores execute three tf32 products for
+    # each.  Value splits recompute the value-independent ones per 64-column block; those are
+    # counted once here
+    fl_b = 6144 * bwd_products(KB, VS) * 2 * 64 ** 3
     launches = 3 + (2 if VS > 1 else 0)
     tf32_peak = peaks["bf16_tflops"] * TF32_PER_BF16
-    return {"workload": f"hybrid_lm backward: dq, dk, dv, dlog_alpha, dbeta (fp32) from dout; dk=64, dv={dv}",
+    return {"workload": f"hybrid_lm backward: dq, dk, dv, dlog_alpha, dbeta (fp32) from dout; dk={dk}, dv={dv}",
             "ms": round(ms_b, 6), "tokens_per_s": round(32768 / (ms_b * 1e-3), 1),
             "launches_per_call": launches, "algo_bytes": by_b,
             "gbs": round(by_b / (ms_b * 1e-3) / 1e9, 3),
@@ -667,9 +686,10 @@ def run_only(args):
         flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device="cuda")
         r = backward_numbers(gdn, to_dev(workloads.config_inputs("hybrid_lm")), args.steps, args.warmup, flush,
                              stream, peaks)
-    elif args.only == "hybrid_lm_backward_dv128":
+    elif args.only in ("hybrid_lm_backward_dv128", "hybrid_lm_backward_dk128"):
         flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device="cuda")
-        d = to_dev(workloads.make_chunk_inputs(B=8, T=4096, H=12, dk=64, dv=128, dtype="bf16", seed=0, la_scale=0.1))
+        dk = 128 if args.only.endswith("dk128") else 64
+        d = to_dev(workloads.make_chunk_inputs(B=8, T=4096, H=12, dk=dk, dv=128, dtype="bf16", seed=0, la_scale=0.1))
         r = backward_numbers(gdn, d, args.steps, args.warmup, flush, stream, peaks)
     elif args.only == "phase_memory":
         flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device="cuda")
@@ -753,7 +773,8 @@ def main():
     ap.add_argument("--quick", action="store_true", help="main workload only")
     ap.add_argument("--only", choices=["hybrid_lm", "long_context", "varlen", "tiny", "decode", "hybrid_lm_fused",
                                              "hybrid_lm_unfused", "hybrid_lm_backward", "phase_memory",
-                                             "hybrid_lm_dv256", "hybrid_lm_backward_dv128", "decode_fused"],
+                                             "hybrid_lm_dv256", "hybrid_lm_backward_dv128", "decode_fused",
+                                             "hybrid_lm_backward_dk128"],
                     help="time one workload's kernel loop only (for profiler runs)")
     args = ap.parse_args()
     if args.warmup < 3:

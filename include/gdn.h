@@ -243,10 +243,12 @@ GDN_API size_t gdn_phase_bwd_workspace_bytes(int B, int T, int H, int dk, int dv
 /*
  * gdn_chunk_bwd -- gradients of gdn_chunk_fwd (the training path; Sykra README, "Architectural
  * Highlights": chunk-parallel training through the WY / unit triangular transform), for
- * dk = 64, dv in {64, 128, 256} and chunk = 64.  Given the forward's inputs (same layouts, dtype
- * for q, k, v and dout) and dout = dL/dout, dS_final = dL/dS_final (NULL: zero), it writes
- *     dq, dk [.., H, 64], dv [.., H, dv], dlog_alpha, dbeta [.., H]   (fp32, always)
- *     dS0 [B, H, 64, dv] fp32 (NULL: not written)
+ * dk in {64, 128}, dv in {64, 128, 256} and chunk = 64.  Given the forward's inputs (same layouts,
+ * dtype for q, k, v and dout) and dout = dL/dout, dS_final = dL/dS_final (NULL: zero), it writes
+ *     dq, dk [.., H, dk], dv [.., H, dv], dlog_alpha, dbeta [.., H]   (fp32, always)
+ *     dS0 [B, H, dk, dv] fp32 (NULL: not written)
+ * dk = 128 runs the key dimension as two 64-column blocks (sums of block products; the chunk
+ * transition M as four 64 x 64 blocks).
  * A value head of dv = 64 VS columns runs as VS heads of 64 columns that share q, k and the gates
  * (value columns never interact); their dq, dk, dlog_alpha and dbeta are summed.
  * Computed from the chunk form with fp32-level accuracy: the 64 x 64 products run on the tensor
@@ -256,8 +258,8 @@ GDN_API size_t gdn_phase_bwd_workspace_bytes(int B, int T, int H, int dk, int dv
  * parallel, two scans over each sequence's chunks give the entry states and exit gradients, and
  * every chunk's input gradients are then formed in parallel.  log_alpha = -inf (an exact reset)
  * gets dlog_alpha = 0.  Workspace: gdn_chunk_bwd_workspace_bytes(...) bytes, 256-byte aligned
- * (eight 16 KB matrices per chunk, head and 64-column value block, plus the partial q/k and
- * gate gradients when dv > 64).  Errors as gdn_chunk_fwd; other head sizes return
+ * (eight 16 KB matrices per chunk, head and 64-column value block, sixteen at dk = 128, plus
+ * the partial q/k and gate gradients when dv > 64).  Errors as gdn_chunk_fwd; other head sizes return
  * GDN_ERR_UNSUPPORTED.
  */
 GDN_API int gdn_chunk_bwd(const void *q, const void *k, const void *v, const float *log_alpha,
@@ -271,7 +273,7 @@ GDN_API size_t gdn_chunk_bwd_workspace_bytes(int B, int T, int H, int dk, int dv
 
 /*
  * gdn_chunk_bwd_gva -- gdn_chunk_bwd with grouped value heads (see gdn_chunk_fwd_gva): q, k
- * [.., Hk, 64]; v, dout [.., Hv, dv]; gates [.., Hv]; states [B, Hv, 64, dv]; value head h reads
+ * [.., Hk, dk]; v, dout [.., Hv, dv]; gates [.., Hv]; states [B, Hv, dk, dv]; value head h reads
  * q/k head h / (Hv / Hk).  dq, dk [.., Hk, 64] are the sums over each q/k head's Hv / Hk value
  * heads; dv, dlog_alpha, dbeta, dS0 stay per value head.  Workspace:
  * gdn_chunk_bwd_gva_workspace_bytes(...) (gdn_chunk_bwd's plus per-value-head dq and dk).

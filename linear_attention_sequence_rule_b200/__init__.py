@@ -515,7 +515,7 @@ def chunk_fwd_gva(q, k, v, log_alpha, beta, S0=None, cu_seqlens=None, out=None, 
 
 def chunk_bwd(q, k, v, log_alpha, beta, dout, S0=None, dS_final=None, cu_seqlens=None, want_dS0=True,
               workspace=None, chunk=64, stream=None):
-    """Gradients of ``chunk_fwd`` (dk = 64, dv in {64, 128, 256}): returns fp32 (dq, dk, dv, dlog_alpha, dbeta,
+    """Gradients of ``chunk_fwd`` (dk in {64, 128}, dv in {64, 128, 256}): returns fp32 (dq, dk, dv, dlog_alpha, dbeta,
     dS0 or None) for dout = dL/dout and dS_final = dL/dS_final (None: zero)."""
     dt = q.dtype
     if dt not in _DT:

@@ -276,20 +276,21 @@ int gdn_device_status(void *stream)
 
 }  // extern "C"
 
-// Head sizes of the backward: dk = 64, dv = 64 VS with VS in {1, 2, 4} (value splits).
-static bool bwd_heads_ok(int dk, int dv) { return dk == 64 && (dv == 64 || dv == 128 || dv == 256); }
+// Head sizes of the backward: dk = 64 KB with KB in {1, 2} (key blocks), dv = 64 VS with VS in
+// {1, 2, 4} (value splits).
+static bool bwd_heads_ok(int dk, int dv) { return (dk == 64 || dk == 128) && (dv == 64 || dv == 128 || dv == 256); }
 
 size_t gdn_chunk_bwd_workspace_bytes(int B, int T, int H, int dk, int dv, int chunk, int varlen)
 {
     if (!bwd_heads_ok(dk, dv) || chunk != 64 || B < 1 || H < 1 || T < 0 || (!varlen && T < 1)) return (size_t)-1;
-    return chunk_bwd_workspace_bytes(B, T, H, varlen, 1, dv / 64);
+    return chunk_bwd_workspace_bytes(B, T, H, varlen, 1, dv / 64, dk / 64);
 }
 
 size_t gdn_chunk_bwd_gva_workspace_bytes(int B, int T, int Hk, int Hv, int dk, int dv, int chunk, int varlen)
 {
     if (Hk < 1 || Hv < 1 || Hv % Hk != 0) return (size_t)-1;
     if (!bwd_heads_ok(dk, dv) || chunk != 64 || B < 1 || T < 0 || (!varlen && T < 1)) return (size_t)-1;
-    return chunk_bwd_workspace_bytes(B, T, Hv, varlen, Hv / Hk, dv / 64);
+    return chunk_bwd_workspace_bytes(B, T, Hv, varlen, Hv / Hk, dv / 64, dk / 64);
 }
 
 namespace gdn {
@@ -303,7 +304,8 @@ static int chunk_bwd_common(const char *fn, const void *q, const void *k, const 
 {
     const int varlen = cu_seqlens != nullptr;
     if (!bwd_heads_ok(dk_, dv_))
-        return fail(GDN_ERR_UNSUPPORTED, "%s: dk=%d dv=%d, supported: dk 64, dv 64, 128 or 256", fn, dk_, dv_);
+        return fail(GDN_ERR_UNSUPPORTED, "%s: dk=%d dv=%d, supported: dk 64 or 128, dv 64, 128 or 256", fn, dk_,
+                    dv_);
     int rc = check_chunk_shape(B, T, H, dk_, dv_, chunk, varlen, dtype, false);
     if (rc != GDN_OK) return rc;
     if (!q || !k || !v || !log_alpha || !beta || !dout || !dq || !dk || !dv || !dlog_alpha || !dbeta)
@@ -313,15 +315,15 @@ static int chunk_bwd_common(const char *fn, const void *q, const void *k, const 
                           cu_seqlens};
     for (const void *p : ptrs)
         if (p && !aligned16(p)) return fail(GDN_ERR_INVALID_ARGUMENT, "%s: pointer %p is not 16-byte aligned", fn, p);
-    const int VS = dv_ / 64;
-    const size_t need = chunk_bwd_workspace_bytes(B, T, H, varlen, G, VS);
+    const int VS = dv_ / 64, KB = dk_ / 64;
+    const size_t need = chunk_bwd_workspace_bytes(B, T, H, varlen, G, VS, KB);
     if (!workspace || workspace_bytes < need)
         return fail(GDN_ERR_WORKSPACE, "%s: workspace of %zu bytes needed, %zu given", fn, need,
                     workspace ? workspace_bytes : (size_t)0);
     if (reinterpret_cast<uintptr_t>(workspace) & 255u)
         return fail(GDN_ERR_INVALID_ARGUMENT, "%s: workspace must be 256-byte aligned", fn);
     BwdArgs a{q, k, v, log_alpha, beta, S0, dout, dS_final, dq, dk, dv, dlog_alpha, dbeta, dS0, cu_seqlens,
-              B, T, H, dtype, workspace, G, VS};
+              B, T, H, dtype, workspace, G, VS, KB};
     cudaError_t e = launch_chunk_bwd(a, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, fn);
     return GDN_OK;

@@ -857,6 +857,479 @@ __global__ void bwd_offsets(const int32_t *__restrict__ cu, int nseq, int32_t *_
     }
 }
 
+
+// ==== dk = 128: the key dimension as two 64-column blocks (KB = 2) ==============================
+// Every formula of the dk = 64 kernels with the key dimension split into blocks a in {0, 1}: q and
+// k rows of 128 are read as two heads of 64 ([tokens, 2 Hq, 64]); K K^T, Q K^T, K dS' and
+// sum_a W_a S_a are sums of two products; M is four tiles (M_ab = gam_C delta_ab I -
+// K_a^T diag(lam) W_b), Bm, R, W, S_c and dS are two.  Value splits apply unchanged (VS heads of
+// 64 value columns).
+
+// The sum of two products of mm_core, handed out as mm does.
+template <bool TA, bool TB, typename F>
+__device__ __forceinline__ void mm2(const float *A0, const float *B0, const float *A1, const float *B1, int t,
+                                    F &&emit)
+{
+    const int lane = t & 31, w = t >> 5, g = lane >> 2, q = lane & 3;
+    const int m0 = (w & 3) * 16, n0 = (w >> 2) * 8 * kNT;
+    Frag f = mm_core<TA, TB, false>((int)(A0 - smf), (int)(B0 - smf), 0);
+    const Frag f1 = mm_core<TA, TB, false>((int)(A1 - smf), (int)(B1 - smf), 0);
+#pragma unroll
+    for (int i = 0; i < kFrag; ++i) f.v[i] += f1.v[i];
+#pragma unroll
+    for (int n = 0; n < kNT; ++n)
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh)
+#pragma unroll
+            for (int e = 0; e < 2; ++e)
+                emit(m0 + g + 8 * hh, n0 + 8 * n + 2 * q + e, f.v[4 * n + 2 * hh + e], 4 * n + 2 * hh + e);
+}
+
+// Per (chunk, virtual head) unit u: T and U~ one matrix each at u; W, Bm, R, S_c, dS two at 2u + a;
+// M four at 4u + 2a + b.
+// Ten shared matrices: K0 K1 | Q0 Q1 (then X0 X1) | A^T (then V, then dO) | P | T | U~ | W0 W1.
+template <typename TIn>
+__global__ void __launch_bounds__(kThreads, 1)
+    bwd_prep2(const TIn *__restrict__ q, const TIn *__restrict__ k, const TIn *__restrict__ v,
+              const float *__restrict__ log_alpha, const float *__restrict__ beta, const TIn *__restrict__ dout,
+              const int32_t *__restrict__ cu, const int32_t *__restrict__ off, int nseq, int T, int H, int G, int VS,
+              float *__restrict__ Mo, float *__restrict__ Bo, float *__restrict__ Ro, float *__restrict__ Tw,
+              float *__restrict__ Ww, float *__restrict__ Uw)
+{
+    float *K0 = smf, *K1 = K0 + MAT, *Q0 = K1 + MAT, *Q1 = Q0 + MAT, *AT = Q1 + MAT, *P = AT + MAT, *Tm = P + MAT,
+          *Ub = Tm + MAT, *W0 = Ub + MAT, *W1 = W0 + MAT;
+    Gates &g = *reinterpret_cast<Gates *>(W1 + MAT);
+    float *bg = reinterpret_cast<float *>(&g + 1);
+    const int t = threadIdx.x, hx = blockIdx.y, Hx = H * VS, h = VS == 1 ? hx : hx / VS, e = blockIdx.x;
+    const ChunkRef c = chunk_ref(e, cu, off, nseq, T);
+    if (c.n == 0) return;
+    const int Hq = G == 1 ? H : H / G, hq = G == 1 ? h : h / G;
+    RowTile<TIn> tv;
+    {
+        RowTile<TIn> tk0, tk1, tq0, tq1;
+        tk0.fetch(k, c, 2 * Hq, 2 * hq, t);
+        tk1.fetch(k, c, 2 * Hq, 2 * hq + 1, t);
+        tq0.fetch(q, c, 2 * Hq, 2 * hq, t);
+        tq1.fetch(q, c, 2 * Hq, 2 * hq + 1, t);
+        tv.fetch(v, c, Hx, hx, t);
+        tk0.put(K0, t);
+        tk1.put(K1, t);
+        tq0.put(Q0, t);
+        tq1.put(Q1, t);
+    }
+    chunk_gates<TIn>(g, log_alpha, beta, c, H, h, t);
+    __syncthreads();
+    if (t < N) bg[t] = g.bet[t] * g.gam[t];
+    mm2<false, true>(K0, K0, K1, K1, t,
+                     [&](int i, int r, float x, int) { AT[sw(i, r)] = i < r ? g.bet[r] * decay(g, r, i) * x : 0.f; });
+    mm2<false, true>(Q0, K0, Q1, K1, t, [&](int r, int i, float x, int) { P[sw(r, i)] = decay(g, r, i) * x; });
+    __syncthreads();
+    unit_lower_inverse(AT, Tm, t);
+    __syncthreads();
+    tv.put(AT, t);  // V over A^T
+    const size_t u = (size_t)e * Hx + hx;
+    mat_from_shared(Tw + u * MAT, Tm, t);
+    __syncthreads();
+    mm<false, false>(Tm, K0, t, [&](int r, int m, float x, int) { W0[sw(r, m)] = x; }, bg);
+    mm<false, false>(Tm, K1, t, [&](int r, int m, float x, int) { W1[sw(r, m)] = x; }, bg);
+    mm<false, false>(Tm, AT, t, [&](int r, int j, float x, int) { Ub[sw(r, j)] = x; }, g.bet);
+    __syncthreads();
+    RowTile<TIn> td;
+    td.fetch(dout, c, Hx, hx, t);
+    mat_from_shared(Ww + (2 * u) * MAT, W0, t);
+    mat_from_shared(Ww + (2 * u + 1) * MAT, W1, t);
+    mat_from_shared(Uw + u * MAT, Ub, t);
+    const float gC = g.gam[N - 1];
+    float *Mb = Mo + 4 * u * MAT;
+    mm<true, false>(K0, W0, t, [&](int m, int n2, float x, int) { Mb[m * N + n2] = (m == n2 ? gC : 0.f) - x; }, g.lam);
+    mm<true, false>(K0, W1, t, [&](int m, int n2, float x, int) { Mb[MAT + m * N + n2] = -x; }, g.lam);
+    mm<true, false>(K1, W0, t, [&](int m, int n2, float x, int) { Mb[2 * MAT + m * N + n2] = -x; }, g.lam);
+    mm<true, false>(K1, W1, t,
+                    [&](int m, int n2, float x, int) { Mb[3 * MAT + m * N + n2] = (m == n2 ? gC : 0.f) - x; }, g.lam);
+    mm<true, false>(K0, Ub, t, [&](int m, int j, float x, int) { Bo[(2 * u) * MAT + m * N + j] = x; }, g.lam);
+    mm<true, false>(K1, Ub, t, [&](int m, int j, float x, int) { Bo[(2 * u + 1) * MAT + m * N + j] = x; }, g.lam);
+    // X_a = diag(gam) Q_a - P W_a in place over Q_a (each element read and written by one thread)
+    mm<false, false>(P, W0, t, [&](int r, int m, float x, int) { Q0[sw(r, m)] = g.gam[r] * Q0[sw(r, m)] - x; });
+    mm<false, false>(P, W1, t, [&](int r, int m, float x, int) { Q1[sw(r, m)] = g.gam[r] * Q1[sw(r, m)] - x; });
+    td.put(AT, t);  // dO over V (its last reader, the U~ product, is behind the barrier above)
+    __syncthreads();
+    // R_a = X_a^T dO
+    mm<true, false>(Q0, AT, t, [&](int m, int j, float x, int) { Ro[(2 * u) * MAT + m * N + j] = x; });
+    mm<true, false>(Q1, AT, t, [&](int m, int j, float x, int) { Ro[(2 * u + 1) * MAT + m * N + j] = x; });
+}
+
+// The scans for KB = 2: the state is two 64 x 64 blocks (rows 0..63 and 64..127 of the 128-row
+// state); forward X_a <- sum_b M_ab X_b + Bm_a, reverse X_a <- sum_b M_ba^T X_b + R_a.  Shared
+// memory: X[2][2], then M[2][4] (192 KB, one CTA per SM).
+template <bool REV>
+__device__ __forceinline__ void scan_body2(const float *__restrict__ Mo, const float *__restrict__ Add,
+                                           const float *__restrict__ X0, const int32_t *__restrict__ cu,
+                                           const int32_t *__restrict__ off, int T, int H, int VS,
+                                           float *__restrict__ Xc, float *__restrict__ Xend)
+{
+    const int t = threadIdx.x, hx = blockIdx.x, s = blockIdx.y, Hx = H * VS;
+    const int g = (t & 31) >> 2, q = t & 3, m0 = ((t >> 5) & 3) * 16, n0 = (t >> 7) * 8 * kNT;
+    constexpr int PER = MAT / 4 / kThreads;
+    int first, count;
+    seq_chunks(s, cu, off, T, first, count);
+    const int ld = N * VS;  // row stride of the caller's states [B, H, 128, 64 VS]
+    const size_t st0 = ((size_t)s * H + hx / VS) * (size_t)(2 * N) * ld + (size_t)(hx % VS) * N;
+    auto unit = [&](int i) { return (size_t)(first + (REV ? count - 1 - i : i)) * Hx + hx; };
+    auto fetch_m = [&](int i, float4 (&m)[4][PER]) {
+        const float4 *src = reinterpret_cast<const float4 *>(Mo + 4 * unit(i) * MAT);
+#pragma unroll
+        for (int bb = 0; bb < 4; ++bb)
+#pragma unroll
+            for (int uu = 0; uu < PER; ++uu) m[bb][uu] = __ldg(src + bb * (MAT / 4) + t + uu * kThreads);
+    };
+    auto fetch_a = [&](int i, float2 (&a)[2][2 * kNT]) {
+#pragma unroll
+        for (int blk = 0; blk < 2; ++blk) {
+            const float *src = Add + (2 * unit(i) + blk) * MAT;
+#pragma unroll
+            for (int n = 0; n < kNT; ++n)
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh)
+                    a[blk][2 * n + hh] =
+                        __ldg(reinterpret_cast<const float2 *>(src + (m0 + g + 8 * hh) * N + n0 + 8 * n + 2 * q));
+        }
+    };
+    auto put_m = [&](float *M, const float4 (&m)[4][PER]) {
+#pragma unroll
+        for (int bb = 0; bb < 4; ++bb)
+#pragma unroll
+            for (int uu = 0; uu < PER; ++uu) {
+                const int e = (t + uu * kThreads) * 4;
+                *reinterpret_cast<float4 *>(&M[bb * MAT + sw(e >> 6, e & 63)]) = m[bb][uu];
+            }
+    };
+    float *Xs = smf, *Ms = smf + 4 * MAT;
+    float4 pm[4][PER];
+    float2 pa[2][2 * kNT], pa2[2][2 * kNT];
+#pragma unroll
+    for (int blk = 0; blk < 2; ++blk) {
+        if (X0) {
+            mat_to_shared_ld(Xs + blk * MAT, X0 + st0 + (size_t)blk * N * ld, ld, t);
+        } else {
+#pragma unroll
+            for (int uu = 0; uu < PER; ++uu)
+                reinterpret_cast<float4 *>(Xs + blk * MAT)[t + uu * kThreads] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+    }
+    if (count > 0) {
+        fetch_m(0, pm);
+        fetch_a(0, pa);
+        put_m(Ms, pm);
+    }
+    if (count > 1) {
+        fetch_m(1, pm);
+        fetch_a(1, pa2);
+    }
+    __syncthreads();
+    for (int i = 0; i < count; ++i) {
+        const int cur = i & 1;
+        float *Xcur = Xs + cur * 2 * MAT, *Xnxt = Xs + (cur ^ 1) * 2 * MAT, *Mcur = Ms + cur * 4 * MAT,
+              *Mnxt = Ms + (cur ^ 1) * 4 * MAT;
+        mat_from_shared(Xc + (2 * unit(i)) * MAT, Xcur, t);
+        mat_from_shared(Xc + (2 * unit(i) + 1) * MAT, Xcur + MAT, t);
+#pragma unroll
+        for (int a = 0; a < 2; ++a) {
+            const float *A0 = Mcur + (REV ? a : 2 * a) * MAT;      // M_0a (reverse) or M_a0
+            const float *A1 = Mcur + (REV ? 2 + a : 2 * a + 1) * MAT;  // M_1a (reverse) or M_a1
+            mm2<REV, false>(A0, Xcur, A1, Xcur + MAT, t, [&](int r, int cc, float x, int uu) {
+                const float2 av = pa[a][2 * (uu >> 2) + u_row(uu)];
+                Xnxt[a * MAT + sw(r, cc)] = x + ((uu & 1) ? av.y : av.x);
+            });
+        }
+        if (i + 1 < count) {
+            put_m(Mnxt, pm);
+#pragma unroll
+            for (int blk = 0; blk < 2; ++blk)
+#pragma unroll
+                for (int uu = 0; uu < 2 * kNT; ++uu) pa[blk][uu] = pa2[blk][uu];
+        }
+        if (i + 2 < count) {
+            fetch_m(i + 2, pm);
+            fetch_a(i + 2, pa2);
+        }
+        __syncthreads();
+    }
+    if (Xend) {
+#pragma unroll
+        for (int blk = 0; blk < 2; ++blk)
+            mat_from_shared_ld(Xend + st0 + (size_t)blk * N * ld, Xs + (count & 1) * 2 * MAT + blk * MAT, ld, t);
+    }
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    bwd_scans2(const float *__restrict__ Mo, const float *__restrict__ Bo, const float *__restrict__ Ro,
+               const float *__restrict__ S0, const float *__restrict__ dS_final, const int32_t *__restrict__ cu,
+               const int32_t *__restrict__ off, int T, int H, int VS, float *__restrict__ Sc,
+               float *__restrict__ dSn, float *__restrict__ dS0)
+{
+    if (blockIdx.z == 0) scan_body2<false>(Mo, Bo, S0, cu, off, T, H, VS, Sc, nullptr);
+    else scan_body2<true>(Mo, Ro, dS_final, cu, off, T, H, VS, dSn, dS0);
+}
+
+// Gradients for KB = 2.  Thirteen shared matrices, reused as their contents die:
+//   K0 K1 | B0 B1: Q, then W, then dW, then Q again | S0 S1: S, then dT (S0), Z (S1), D + D^T (S0) |
+//   D0 D1: dS', then T (D0), V (D1) | KK | X1: P, then D2 | Ub: U~, then U, then D | X2: K dS', then dU,
+//   then scratch | dO.
+template <typename TIn>
+__global__ void __launch_bounds__(kThreads, 1)
+    bwd_grads2(const TIn *__restrict__ q, const TIn *__restrict__ k, const TIn *__restrict__ v,
+               const float *__restrict__ log_alpha, const float *__restrict__ beta, const TIn *__restrict__ dout,
+               const float *__restrict__ Sc, const float *__restrict__ dSn, const float *__restrict__ Tw,
+               const float *__restrict__ Ww, const float *__restrict__ Uw, const int32_t *__restrict__ cu,
+               const int32_t *__restrict__ off, int nseq, int T, int H, int G, int VS, float *__restrict__ dq,
+               float *__restrict__ dk, float *__restrict__ dv, float *__restrict__ dla, float *__restrict__ dbe)
+{
+    float *K0 = smf, *K1 = K0 + MAT, *B0 = K1 + MAT, *B1 = B0 + MAT, *S0s = B1 + MAT, *S1s = S0s + MAT,
+          *D0 = S1s + MAT, *D1 = D0 + MAT, *KK = D1 + MAT, *X1 = KK + MAT, *Ub = X1 + MAT, *X2 = Ub + MAT,
+          *dO = X2 + MAT;
+    Gates &g = *reinterpret_cast<Gates *>(dO + MAT);
+    float *vec = reinterpret_cast<float *>(&g + 1);
+    float *bg = vec, *dG = vec + N, *dgam = vec + 2 * N, *dlam = vec + 3 * N, *dbet = vec + 4 * N, *dgC = vec + 5 * N;
+    const int t = threadIdx.x, hx = blockIdx.y, Hx = H * VS, h = VS == 1 ? hx : hx / VS, e = blockIdx.x;
+    const ChunkRef c = chunk_ref(e, cu, off, nseq, T);
+    if (c.n == 0) return;
+    const size_t u1 = (size_t)e * Hx + hx;
+    const int Hq = G == 1 ? H : H / G, hq = G == 1 ? h : h / G;
+    {
+        RowTile<TIn> tk0, tk1, tq0, tq1, td;
+        tk0.fetch(k, c, 2 * Hq, 2 * hq, t);
+        tk1.fetch(k, c, 2 * Hq, 2 * hq + 1, t);
+        tq0.fetch(q, c, 2 * Hq, 2 * hq, t);
+        tq1.fetch(q, c, 2 * Hq, 2 * hq + 1, t);
+        td.fetch(dout, c, Hx, hx, t);
+        mat_to_shared(S0s, Sc + (2 * u1) * MAT, t);
+        mat_to_shared(S1s, Sc + (2 * u1 + 1) * MAT, t);
+        mat_to_shared(D0, dSn + (2 * u1) * MAT, t);
+        mat_to_shared(D1, dSn + (2 * u1 + 1) * MAT, t);
+        mat_to_shared(Ub, Uw + u1 * MAT, t);
+        tk0.put(K0, t);
+        tk1.put(K1, t);
+        tq0.put(B0, t);
+        tq1.put(B1, t);
+        td.put(dO, t);
+    }
+    chunk_gates<TIn>(g, log_alpha, beta, c, H, h, t);
+    __syncthreads();
+    if (t < N) bg[t] = g.bet[t] * g.gam[t];
+    float aq0[kFrag], aq1[kFrag], ak0[kFrag], ak1[kFrag], av[kFrag];
+    float pb[2] = {0.f, 0.f}, pg[2] = {0.f, 0.f}, pG[2] = {0.f, 0.f}, pl[2] = {0.f, 0.f};
+    float pc[kColSlots];
+#pragma unroll
+    for (int i = 0; i < kFrag; ++i) aq0[i] = aq1[i] = ak0[i] = ak1[i] = av[i] = 0.f;
+#pragma unroll
+    for (int i = 0; i < kColSlots; ++i) pc[i] = 0.f;
+    // K K^T; P = Gam o Q K^T; K dS'
+    mm2<false, true>(K0, K0, K1, K1, t, [&](int r, int i, float x, int) { KK[sw(r, i)] = x; });
+    mm2<false, true>(B0, K0, B1, K1, t, [&](int r, int i, float x, int) { X1[sw(r, i)] = decay(g, r, i) * x; });
+    mm2<false, false>(K0, D0, K1, D1, t, [&](int i, int m, float x, int) { X2[sw(i, m)] = x; });
+    // dQ_a += diag(gam) dO S_a^T, and d gam_r (O1) = sum_a sum_m Q_a(r, m) (dO S_a^T)(r, m)
+    mm<false, true>(dO, S0s, t, [&](int r, int m, float x, int uu) {
+        aq0[uu] += g.gam[r] * x;
+        pg[u_row(uu)] = fmaf(B0[sw(r, m)], x, pg[u_row(uu)]);
+    });
+    mm<false, true>(dO, S1s, t, [&](int r, int m, float x, int uu) {
+        aq1[uu] += g.gam[r] * x;
+        pg[u_row(uu)] = fmaf(B1[sw(r, m)], x, pg[u_row(uu)]);
+    });
+    // d gam_C = <S, dS'>, per warp (summed in warp order with the gate gradients)
+    {
+        float part = 0.f;
+        for (int idx = t; idx < N * N; idx += kThreads) {
+            const int r = idx >> 6, i = idx & 63;
+            part = fmaf(S0s[sw(r, i)], D0[sw(r, i)], part);
+            part = fmaf(S1s[sw(r, i)], D1[sw(r, i)], part);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+        if ((t & 31) == 0) dgC[t >> 5] = part;
+    }
+    __syncthreads();
+    mat_to_shared(B0, Ww + (2 * u1) * MAT, t);  // W over Q
+    mat_to_shared(B1, Ww + (2 * u1 + 1) * MAT, t);
+    __syncthreads();
+    // U = U~ - sum_a W_a S_a
+    mm2<false, false>(B0, S0s, B1, S1s, t, [&](int r, int j, float x, int) { Ub[sw(r, j)] -= x; });
+    __syncthreads();
+    // dU = P^T dO + diag(lam) K dS' over K dS'; d lam_i = sum_j (K dS')_ij U_ij
+    mm<true, false>(X1, dO, t, [&](int i, int j, float x, int uu) {
+        const float kd = X2[sw(i, j)];
+        X2[sw(i, j)] = x + g.lam[i] * kd;
+        pl[u_row(uu)] = fmaf(kd, Ub[sw(i, j)], pl[u_row(uu)]);
+    });
+    __syncthreads();
+    // dP = dO U^T (lower incl.) -> D2 = dP o Gam over P, with the dG terms of Gam (P): E = dP o P
+    mm<false, true>(dO, Ub, t, [&](int r, int i, float x, int uu) {
+        const float gm = decay(g, r, i), dp = i <= r ? x : 0.f;
+        const float E = dp * X1[sw(r, i)];
+        X1[sw(r, i)] = dp * gm;
+        pG[u_row(uu)] += E;
+        pc[u_col(uu)] -= E;
+    });
+    // dK_a += diag(lam) U dS'_a^T
+    mm<false, true>(Ub, D0, t, [&](int i, int, float x, int uu) { ak0[uu] += g.lam[i] * x; });
+    mm<false, true>(Ub, D1, t, [&](int i, int, float x, int uu) { ak1[uu] += g.lam[i] * x; });
+    __syncthreads();
+    {
+        RowTile<TIn> tv;
+        tv.fetch(v, c, Hx, hx, t);
+        mat_to_shared(D0, Tw + u1 * MAT, t);  // T over dS'_0
+        tv.put(D1, t);                         // V over dS'_1
+    }
+    // dW_a = -dU S_a^T over W_a
+    mm<false, true>(X2, S0s, t, [&](int r, int m, float x, int) { B0[sw(r, m)] = -x; });
+    mm<false, true>(X2, S1s, t, [&](int r, int m, float x, int) { B1[sw(r, m)] = -x; });
+    __syncthreads();
+    // Y = T^T dU: dV, dbeta;  X_a = T^T dW_a: dK_a, dbeta, d gam
+    mm<true, false>(D0, X2, t, [&](int i, int j, float x, int uu) {
+        av[uu] += g.bet[i] * x;
+        pb[u_row(uu)] = fmaf(x, D1[sw(i, j)], pb[u_row(uu)]);
+    });
+    mm<true, false>(D0, B0, t, [&](int i, int m, float x, int uu) {
+        ak0[uu] += bg[i] * x;
+        const float xk = x * K0[sw(i, m)];
+        pb[u_row(uu)] = fmaf(g.gam[i], xk, pb[u_row(uu)]);
+        pg[u_row(uu)] = fmaf(g.bet[i], xk, pg[u_row(uu)]);
+    });
+    mm<true, false>(D0, B1, t, [&](int i, int m, float x, int uu) {
+        ak1[uu] += bg[i] * x;
+        const float xk = x * K1[sw(i, m)];
+        pb[u_row(uu)] = fmaf(g.gam[i], xk, pb[u_row(uu)]);
+        pg[u_row(uu)] = fmaf(g.bet[i], xk, pg[u_row(uu)]);
+    });
+    // dT = dU (diag(b) V)^T + sum_a dW_a (diag(b gam) K_a)^T over S_0; the diagonals scale the
+    // result's column index
+    mm<false, true>(X2, D1, t, [&](int r, int i, float x, int) { S0s[sw(r, i)] = g.bet[i] * x; });
+    mm2<false, true>(B0, K0, B1, K1, t, [&](int r, int i, float x, int) { S0s[sw(r, i)] += bg[i] * x; });
+    __syncthreads();
+    // Z = dT T^T over S_1
+    mm<false, true>(S0s, D0, t, [&](int r, int i, float x, int) { S1s[sw(r, i)] = x; });
+    __syncthreads();
+    // dA = -T^T Z (strictly lower) -> D over U; dbeta (A); dG from Gam (A)
+    mm<true, false>(D0, S1s, t, [&](int r, int i, float x, int uu) {
+        float d = 0.f;
+        if (i < r) {
+            const float gm = decay(g, r, i), kk = KK[sw(r, i)];
+            const float dAg = -x * gm;
+            d = g.bet[r] * dAg;
+            pb[u_row(uu)] = fmaf(dAg, kk, pb[u_row(uu)]);
+            const float E = d * kk;
+            pG[u_row(uu)] += E;
+            pc[u_col(uu)] -= E;
+        }
+        Ub[sw(r, i)] = d;
+    });
+    __syncthreads();
+    // D + D^T over dT, and Q again over dW
+    {
+        RowTile<TIn> tq0, tq1;
+        tq0.fetch(q, c, 2 * Hq, 2 * hq, t);
+        tq1.fetch(q, c, 2 * Hq, 2 * hq + 1, t);
+        for (int idx = t; idx < N * N; idx += kThreads) {
+            const int r = idx >> 6, i = idx & 63;
+            S0s[sw(r, i)] = Ub[sw(r, i)] + Ub[sw(i, r)];
+        }
+        tq0.put(B0, t);
+        tq1.put(B1, t);
+    }
+    __syncthreads();
+    // dK_a += (D + D^T) K_a + D2^T Q_a;  dQ_a += D2 K_a
+    mm<false, false>(S0s, K0, t, [&](int, int, float x, int uu) { ak0[uu] += x; });
+    mm<false, false>(S0s, K1, t, [&](int, int, float x, int uu) { ak1[uu] += x; });
+    mm<true, false>(X1, B0, t, [&](int, int, float x, int uu) { ak0[uu] += x; });
+    mm<true, false>(X1, B1, t, [&](int, int, float x, int uu) { ak1[uu] += x; });
+    mm<false, false>(X1, K0, t, [&](int, int, float x, int uu) { aq0[uu] += x; });
+    mm<false, false>(X1, K1, t, [&](int, int, float x, int uu) { aq1[uu] += x; });
+    // the partial sums over the block (X2 is free scratch: its last reader is behind two barriers)
+    constexpr int RB = kColBlocks * N;
+    row_put(pb, X2, t);
+    row_put(pg, X2 + RB, t);
+    row_put(pG, X2 + 2 * RB, t);
+    row_put(pl, X2 + 3 * RB, t);
+    col_put(pc, X2 + 4 * RB, t);
+    __syncthreads();
+    if (t < N) {
+        dbet[t] = row_get(X2, t);
+        dgam[t] = row_get(X2 + RB, t);
+        dG[t] = row_get(X2 + 2 * RB, t) + col_get(X2 + 4 * RB, t);
+        dlam[t] = row_get(X2 + 3 * RB, t);
+    }
+    __syncthreads();
+    if (t < 32) {
+        float x[2], li[2];
+        int f[2];
+#pragma unroll
+        for (int w2 = 0; w2 < 2; ++w2) {
+            const int j = N - 1 - (t + 32 * w2);
+            li[w2] = dlam[j] * g.lam[j];
+            x[w2] = dG[j] + dgam[j] * g.gam[j] - li[w2];
+            f[w2] = j < N - 1 && g.last[j + 1] == j + 1;
+        }
+        float s63 = li[0] + li[1];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) s63 += __shfl_xor_sync(0xffffffffu, s63, o);
+        if (t == 0) {  // row 63
+            float dgc = 0.f;
+            for (int w2 = 0; w2 < kThreads / 32; ++w2) dgc += dgC[w2];
+            x[0] += s63 + dgc * g.gam[N - 1];
+        }
+        seg_scan64(x[0], f[0], x[1], f[1], t);
+#pragma unroll
+        for (int w2 = 0; w2 < 2; ++w2) {
+            const int j = N - 1 - (t + 32 * w2);
+            dlam[j] = g.last[j] == j ? 0.f : x[w2];  // reuse as dlog_alpha
+        }
+    }
+    __syncthreads();
+    {
+        const int lane = t & 31, w = t >> 5, gq = lane >> 2, qq = lane & 3;
+        const int m0 = (w & 3) * 16, n0 = (w >> 2) * 8 * kNT;
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+            const int r = m0 + gq + 8 * hh;
+            if (r >= c.n) continue;
+            const size_t rowk = ((size_t)(c.tok + r) * Hx + hx) * (2 * N) + n0 + 2 * qq;  // dq, dk rows of 128
+            const size_t rowv = ((size_t)(c.tok + r) * Hx + hx) * N + n0 + 2 * qq;
+#pragma unroll
+            for (int n = 0; n < kNT; ++n) {
+                const int uu = 4 * n + 2 * hh;
+                *reinterpret_cast<float2 *>(dq + rowk + 8 * n) = make_float2(aq0[uu], aq0[uu + 1]);
+                *reinterpret_cast<float2 *>(dq + rowk + N + 8 * n) = make_float2(aq1[uu], aq1[uu + 1]);
+                *reinterpret_cast<float2 *>(dk + rowk + 8 * n) = make_float2(ak0[uu], ak0[uu + 1]);
+                *reinterpret_cast<float2 *>(dk + rowk + N + 8 * n) = make_float2(ak1[uu], ak1[uu + 1]);
+                *reinterpret_cast<float2 *>(dv + rowv + 8 * n) = make_float2(av[uu], av[uu + 1]);
+            }
+        }
+    }
+    if (t < c.n) {
+        const size_t o = (size_t)(c.tok + t) * Hx + hx;
+        dla[o] = dlam[t];
+        dbe[o] = dbet[t];
+    }
+}
+
+// Grouped sums over rows of width W (dq, dk of KB = 2 have rows of 128): out[row][col] =
+// sum_u in[row G + u][col]; one thread per output element.
+__global__ void bwd_group_sum_w(const float *__restrict__ gq, const float *__restrict__ gk, float *__restrict__ dq,
+                                float *__restrict__ dk, long out_elems, int G, int W)
+{
+    const long i = (long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= out_elems) return;
+    const long row = i / W, col = i % W;
+    const float *a = gq + row * G * W + col, *b = gk + row * G * W + col;
+    float sq = 0.f, sk = 0.f;
+    for (int u = 0; u < G; ++u) {
+        sq += a[u * W];
+        sk += b[u * W];
+    }
+    dq[i] = sq;
+    dk[i] = sk;
+}
+
 }  // namespace
 
 // ---- host side -------------------------------------------------------------------------------
@@ -878,16 +1351,84 @@ struct BwdLayout {
     size_t off, mats, qk, gates, bytes;
 };
 
-BwdLayout bwd_layout(int B, int T, int H, int varlen, int G, int VS)
+BwdLayout bwd_layout(int B, int T, int H, int varlen, int G, int VS, int KB = 1)
 {
     BwdLayout l;
     const size_t Hx = (size_t)H * VS, tokens = varlen ? (size_t)T : (size_t)B * T;
     l.off = align256b((size_t)(B + 1) * sizeof(int32_t));
     l.mats = align256b((size_t)bwd_chunks(B, T, varlen) * Hx * N * N * sizeof(float));
-    l.qk = G * VS > 1 ? align256b(tokens * Hx * N * sizeof(float)) : 0;
+    l.qk = G * VS > 1 ? align256b(tokens * Hx * N * KB * sizeof(float)) : 0;
     l.gates = VS > 1 ? align256b(tokens * Hx * sizeof(float)) : 0;
-    l.bytes = l.off + 8 * l.mats + 2 * l.qk + 2 * l.gates;
+    // KB = 1: M, Bm, R, S_c, dS, T, W, U~; KB = 2: M four, Bm, R, S_c, dS, W two, T and U~ one
+    l.bytes = l.off + (KB == 1 ? 8 : 16) * l.mats + 2 * l.qk + 2 * l.gates;
     return l;
+}
+
+// dk = 128: the same plan with the KB = 2 kernels.
+template <typename TIn>
+cudaError_t run_bwd2(const BwdArgs &a, cudaStream_t st)
+{
+    const int varlen = a.cu_seqlens != nullptr;
+    const long chunks = bwd_chunks(a.B, a.T, varlen);
+    const int VS = a.VS, Hx = a.H * VS;
+    const BwdLayout l = bwd_layout(a.B, a.T, a.H, varlen, a.G, VS, 2);
+    const size_t mats = l.mats;
+    char *w = static_cast<char *>(a.workspace);
+    int32_t *off = reinterpret_cast<int32_t *>(w);
+    w += l.off;
+    float *Mo = reinterpret_cast<float *>(w);
+    float *Bo = reinterpret_cast<float *>(w + 4 * mats);
+    float *Ro = reinterpret_cast<float *>(w + 6 * mats);
+    float *Sc = reinterpret_cast<float *>(w + 8 * mats);
+    float *dSn = reinterpret_cast<float *>(w + 10 * mats);
+    float *Tw = reinterpret_cast<float *>(w + 12 * mats);
+    float *Ww = reinterpret_cast<float *>(w + 13 * mats);
+    float *Uw = reinterpret_cast<float *>(w + 15 * mats);
+    const size_t tokens = varlen ? (size_t)a.T : (size_t)a.B * a.T;
+    const int GQ = a.G * VS;
+    char *pw = w + 16 * mats;
+    float *gq = GQ > 1 ? reinterpret_cast<float *>(pw) : a.dq;
+    float *gk = GQ > 1 ? reinterpret_cast<float *>(pw + l.qk) : a.dk;
+    float *gla = VS > 1 ? reinterpret_cast<float *>(pw + 2 * l.qk) : a.dlog_alpha;
+    float *gbe = VS > 1 ? reinterpret_cast<float *>(pw + 2 * l.qk + l.gates) : a.dbeta;
+    const int32_t *offp = varlen ? off : nullptr;
+    if (varlen) {
+        bwd_offsets<<<1, 1, 0, st>>>(a.cu_seqlens, a.B, off);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    const TIn *q = static_cast<const TIn *>(a.q), *k = static_cast<const TIn *>(a.k),
+              *v = static_cast<const TIn *>(a.v), *dout = static_cast<const TIn *>(a.dout);
+    const int smem_prep = (10 * MAT) * (int)sizeof(float) + (int)sizeof(Gates) + N * (int)sizeof(float);
+    const int smem_grads = (13 * MAT) * (int)sizeof(float) + (int)sizeof(Gates) + 6 * N * (int)sizeof(float);
+    const int smem_scan = 12 * MAT * (int)sizeof(float);
+    cudaError_t e = cudaFuncSetAttribute(bwd_prep2<TIn>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_prep);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(bwd_grads2<TIn>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_grads);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(bwd_scans2, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_scan);
+    if (e != cudaSuccess) return e;
+    const dim3 gc((unsigned)chunks, Hx);
+    bwd_prep2<TIn><<<gc, kThreads, smem_prep, st>>>(q, k, v, a.log_alpha, a.beta, dout, a.cu_seqlens, offp, a.B, a.T,
+                                                    a.H, a.G, VS, Mo, Bo, Ro, Tw, Ww, Uw);
+    bwd_scans2<<<dim3(Hx, a.B, 2), kThreads, smem_scan, st>>>(Mo, Bo, Ro, a.S0, a.dS_final, a.cu_seqlens, offp, a.T,
+                                                             a.H, VS, Sc, dSn, a.dS0);
+    bwd_grads2<TIn><<<gc, kThreads, smem_grads, st>>>(q, k, v, a.log_alpha, a.beta, dout, Sc, dSn, Tw, Ww, Uw,
+                                                      a.cu_seqlens, offp, a.B, a.T, a.H, a.G, VS, gq, gk, a.dv, gla,
+                                                      gbe);
+    if (GQ > 1) {
+        const long out_elems = (long)(tokens * (a.H / a.G)) * 2 * N;
+        if (out_elems > 0)
+            bwd_group_sum_w<<<(unsigned)((out_elems + 255) / 256), 256, 0, st>>>(gq, gk, a.dq, a.dk, out_elems, GQ,
+                                                                                 2 * N);
+    }
+    if (VS > 1) {
+        const long out_elems = (long)(tokens * a.H);
+        if (out_elems > 0)
+            bwd_gate_sum<<<(unsigned)((out_elems + 255) / 256), 256, 0, st>>>(gla, gbe, a.dlog_alpha, a.dbeta,
+                                                                              out_elems, VS);
+    }
+    return cudaGetLastError();
 }
 
 template <typename TIn>
@@ -959,13 +1500,15 @@ cudaError_t run_bwd(const BwdArgs &a, cudaStream_t st)
 
 }  // namespace
 
-size_t chunk_bwd_workspace_bytes(int B, int T, int H, int varlen, int G, int VS)
+size_t chunk_bwd_workspace_bytes(int B, int T, int H, int varlen, int G, int VS, int KB)
 {
-    return bwd_layout(B, T, H, varlen, G, VS).bytes;
+    return bwd_layout(B, T, H, varlen, G, VS, KB).bytes;
 }
 
 cudaError_t launch_chunk_bwd(const BwdArgs &a, cudaStream_t stream)
 {
+    if (a.KB == 2)
+        return a.dtype == GDN_DTYPE_BF16 ? run_bwd2<__nv_bfloat16>(a, stream) : run_bwd2<float>(a, stream);
     return a.dtype == GDN_DTYPE_BF16 ? run_bwd<__nv_bfloat16>(a, stream) : run_bwd<float>(a, stream);
 }
 

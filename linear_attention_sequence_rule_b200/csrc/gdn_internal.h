@@ -63,8 +63,9 @@ struct BwdArgs {
     void *workspace;
     int G = 1;   // grouped value heads: H / G q/k heads, value head h reads q/k head h / G
     int VS = 1;  // value splits: dv = 64 VS, each value head run as VS heads of 64 columns
+    int KB = 1;  // key blocks: dk = 64 KB
 };
-size_t chunk_bwd_workspace_bytes(int B, int T, int H, int varlen, int G = 1, int VS = 1);
+size_t chunk_bwd_workspace_bytes(int B, int T, int H, int varlen, int G = 1, int VS = 1, int KB = 1);
 cudaError_t launch_chunk_bwd(const BwdArgs &a, cudaStream_t stream);
 
 }  // namespace gdn

@@ -162,19 +162,21 @@ def test_backward_entry_validation():
     a = dict(q=FAKE, k=FAKE, v=FAKE, log_alpha=FAKE, beta=FAKE, S0=None, dout=FAKE, dS_final=None, dq=FAKE,
              dk=FAKE, dv=FAKE, dlog_alpha=FAKE, dbeta=FAKE, dS0=None, B=1, T=64, H=1, dk_=64, dv_=64, chunk=64,
              cu_seqlens=None, dtype=gdn.GDN_DTYPE_BF16, workspace=None, workspace_bytes=0, stream=None)
-    assert gdn.gdn_chunk_bwd(**(a | dict(dk_=128, dv_=128))) == gdn.GDN_ERR_UNSUPPORTED
+    assert gdn.gdn_chunk_bwd(**(a | dict(dk_=96, dv_=128))) == gdn.GDN_ERR_UNSUPPORTED
+    assert gdn.gdn_chunk_bwd(**(a | dict(dk_=256, dv_=64))) == gdn.GDN_ERR_UNSUPPORTED
     assert gdn.gdn_chunk_bwd(**(a | dict(dq=None))) == gdn.GDN_ERR_INVALID_ARGUMENT
     assert gdn.gdn_chunk_bwd(**(a | dict(dbeta=FAKE + 4))) == gdn.GDN_ERR_INVALID_ARGUMENT
     assert gdn.gdn_chunk_bwd(**a) == gdn.GDN_ERR_WORKSPACE
     assert "gdn_chunk_bwd" in gdn.gdn_last_error()
-    assert gdn.gdn_chunk_bwd_workspace_bytes(1, 64, 1, 128, 128, 64, 0) == (1 << 64) - 1
+    assert gdn.gdn_chunk_bwd_workspace_bytes(1, 64, 1, 256, 128, 64, 0) == (1 << 64) - 1
     assert gdn.gdn_chunk_bwd_workspace_bytes(2, 128, 3, 64, 64, 64, 0) > 5 * 2 * 2 * 3 * 64 * 64 * 4 - 1
     # value head sizes 128 and 256 (64-column value splits): more workspace; other sizes rejected
     w64 = gdn.gdn_chunk_bwd_workspace_bytes(2, 128, 3, 64, 64, 64, 0)
     assert gdn.gdn_chunk_bwd_workspace_bytes(2, 128, 3, 64, 128, 64, 0) > 2 * w64 - 4096
     assert gdn.gdn_chunk_bwd_workspace_bytes(2, 128, 3, 64, 256, 64, 1) > 4 * w64 - 4096
     assert gdn.gdn_chunk_bwd_workspace_bytes(2, 128, 3, 64, 96, 64, 0) == (1 << 64) - 1
-    assert gdn.gdn_chunk_bwd_workspace_bytes(2, 128, 3, 128, 64, 64, 0) == (1 << 64) - 1
+    # key head size 128 (two key blocks): sixteen matrices per unit instead of eight
+    assert gdn.gdn_chunk_bwd_workspace_bytes(2, 128, 3, 128, 64, 64, 0) > 2 * w64 - 4096
     assert gdn.gdn_chunk_bwd(**(a | dict(dv_=128))) == gdn.GDN_ERR_WORKSPACE
     assert gdn.gdn_chunk_bwd(**(a | dict(dv_=512))) == gdn.GDN_ERR_UNSUPPORTED
 
@@ -270,7 +272,7 @@ def test_grouped_backward_rejects_bad_groups():
              dv=FAKE, dlog_alpha=FAKE, dbeta=FAKE, dS0=None, B=1, T=64, Hk=2, Hv=5, dk_=64, dv_=64, chunk=64,
              cu_seqlens=None, dtype=gdn.GDN_DTYPE_BF16, workspace=FAKE * 256, workspace_bytes=1 << 40, stream=None)
     assert gdn.gdn_chunk_bwd_gva(**a) == gdn.GDN_ERR_INVALID_ARGUMENT        # 5 value heads on 2 q/k heads
-    assert gdn.gdn_chunk_bwd_gva(**dict(a, Hv=4, dk_=128)) == gdn.GDN_ERR_UNSUPPORTED
+    assert gdn.gdn_chunk_bwd_gva(**dict(a, Hv=4, dk_=96)) == gdn.GDN_ERR_UNSUPPORTED
     assert gdn.gdn_chunk_bwd_gva(**dict(a, Hv=4, workspace=None)) == gdn.GDN_ERR_WORKSPACE
     assert gdn.gdn_chunk_bwd_gva_workspace_bytes(1, 64, 2, 5, 64, 64, 64, 0) == ctypes.c_size_t(-1).value
     plain = gdn.gdn_chunk_bwd_workspace_bytes(1, 64, 4, 64, 64, 64, 0)

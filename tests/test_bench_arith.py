@@ -51,3 +51,13 @@ def test_decode_bytes_per_state():
     state_read_and_write = 2 * dk * dv * 4
     q_k_v_out = (dk + dk + dv + dv) * 2
     assert bench.DECODE_BYTES_PER_STATE(dk, dv, 2) == state_read_and_write + q_k_v_out + 8 == 132104
+
+
+def test_backward_product_count():
+    # 26 distinct products at dk = dv = 64 (8 forming the chunk maps, 1 per scan, 16 for the
+    # gradients); 14 of them carry a value dimension, so dv = 128 adds 14; every product of the
+    # chunk form grows with each key or value block it contracts over or produces
+    assert bench.bwd_products(1, 1) == 26
+    assert bench.bwd_products(1, 2) == 26 + 14
+    assert bench.bwd_products(1, 4) == 26 + 3 * 14
+    assert bench.bwd_products(2, 2) > bench.bwd_products(1, 2) + 26
