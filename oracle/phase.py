@@ -15,7 +15,13 @@ Q_t (dk), real value V_t (dv), and scalars lam_t = exp(log_lam_t) in (0, 1] and 
 
 The first three lines are the section's three steps with the gated decay; the read-out of the
 query (post-update state, the key's 1/dk scale) and lam_t as one scalar per (token, head) are
-readings (the section prints no query read-out; the Laplace core's per-row decay is not taken).
+readings (the section prints no query read-out).
+
+``forward_rowdecay`` is the Laplace core's per-row form (section 5, "Exact Chunkwise-Parallel
+Scan"): the decay is diag(r_t), one factor r_t,j = exp(log_r_t,j) per output row j of M (value
+channel), M_t = diag(r_t) M_{t-1} + beta_t e_t K_t^T with e_t and o_t as above.  Reading: r_t is
+an input per (token, head, channel), as lam_t is in the scalar form, and finite in log (r > 0).  ``forward_rowdecay_chunkwise``
+is its chunk form, with the per-channel triangular solve the section describes.
 
 ``forward`` is that definition token by token in complex128.  ``forward_chunkwise`` is the chunk
 form derived separately (a unit-lower triangular solve per chunk for the errors), used as a pin.
@@ -179,3 +185,84 @@ def backward(K, Q, V, log_lam, beta, M0, dout, dM_final=None, cu_seqlens=None):
     dS0 = dS0.swapaxes(-1, -2)
     dM0 = dS0[..., :dk] + 1j * dS0[..., dk:]
     return dK, dQ, dV, dlog_lam, db / lam, dM0
+
+
+def forward_rowdecay(K, Q, V, log_r, beta, M0=None, cu_seqlens=None):
+    """The per-row-decay definition, token by token: log_r [..., H, dv] (one decay per value
+    channel); otherwise as ``forward``."""
+    K, Q, M0 = as_complex(K), as_complex(Q), as_complex(M0)
+    V, lr, be = _real(V), _real(log_r), _real(beta)
+    dk, dv = K.shape[-1], V.shape[-1]
+    H = V.shape[-2]
+    out = np.zeros(V.shape)
+    if cu_seqlens is None:
+        B, T = V.shape[:2]
+        runs = [(b, [(b, t) for t in range(T)]) for b in range(B)]
+    else:
+        runs = [(s, [(t,) for t in range(sl.start, sl.stop)]) for s, sl in _sequences(None, cu_seqlens, None)]
+    Mf = np.zeros((len(runs), H, dv, dk), np.complex128)
+    for s, toks in runs:
+        M = np.zeros((H, dv, dk), np.complex128) if M0 is None else M0[s].copy()
+        for idx in toks:
+            k, q = K[idx], Q[idx]                                   # [H, dk]
+            e = V[idx] - np.einsum("hji,hi->hj", M, np.conj(k)).real / dk
+            M = np.exp(lr[idx])[:, :, None] * M + (be[idx][:, None] * e)[:, :, None] * k[:, None, :]
+            out[idx] = np.einsum("hji,hi->hj", M, np.conj(q)).real / dk
+        Mf[s] = M
+    return out, Mf
+
+
+def _chunk_rowdecay(M0, K, Q, V, lr, be):
+    """One chunk of one (sequence, head) with per-channel decays: M0 [dv, dk]; K, Q [C, dk]; V, lr
+    [C, dv]; be [C].  With g_t,j the sum of log_r over the chunk's tokens up to t (g_-1 = 0), channel
+    j's errors solve its own unit-lower system (I + A_j) e_j = v_j - (1/dk) e^{g_{t-1},j}
+    Re(conj(K) M0^T)[:, j], A_j[t, s] = (1/dk) e^{g_{t-1},j - g_s,j} beta_s Re(K_s . conj K_t) for
+    s < t: the phasor Gram is shared, the decay weighting is the channel's own."""
+    C, dk = K.shape
+    dv = V.shape[1]
+    g = np.cumsum(lr, axis=0)                                        # [C, dv]
+    g_prev = np.concatenate([np.zeros((1, dv)), g[:-1]])
+    gram_k = (K @ np.conj(K).T).real                                 # [s, t]
+    gram_q = (K @ np.conj(Q).T).real
+    read0 = (np.conj(K) @ M0.T).real / dk                            # [C, dv]
+    readq = (np.conj(Q) @ M0.T).real / dk
+    E = np.zeros((C, dv))
+    O = np.zeros((C, dv))
+    M_end = np.zeros_like(M0)
+    lower = np.tril(np.ones((C, C)), -1) > 0
+    incl = np.tril(np.ones((C, C))) > 0
+    for j in range(dv):
+        A = np.where(lower, np.exp(g_prev[:, j][:, None] - g[:, j][None, :]) * be[None, :] * gram_k.T, 0.0) / dk
+        E[:, j] = solve_triangular(np.eye(C) + A, V[:, j] - np.exp(g_prev[:, j]) * read0[:, j], lower=True,
+                                   unit_diagonal=True)
+        P = np.where(incl, np.exp(g[:, j][:, None] - g[:, j][None, :]) * be[None, :] * gram_q.T, 0.0) / dk
+        O[:, j] = np.exp(g[:, j]) * readq[:, j] + P @ E[:, j]
+        w = be * np.exp(g[-1, j] - g[:, j])
+        M_end[j] = np.exp(g[-1, j]) * M0[j] + (E[:, j] * w) @ K
+    return O, M_end
+
+
+def forward_rowdecay_chunkwise(K, Q, V, log_r, beta, M0=None, chunk=64, cu_seqlens=None):
+    """The per-row-decay chunk form: the same results as ``forward_rowdecay`` up to rounding."""
+    K, Q, M0 = as_complex(K), as_complex(Q), as_complex(M0)
+    V, lr, be = _real(V), _real(log_r), _real(beta)
+    dk, dv = K.shape[-1], V.shape[-1]
+    H = V.shape[-2]
+    out = np.zeros(V.shape)
+    if cu_seqlens is None:
+        B, T = V.shape[:2]
+        runs = [(b, (b, slice(0, T))) for b in range(B)]
+    else:
+        runs = [(s, (sl,)) for s, sl in _sequences(None, cu_seqlens, None)]
+    Mf = np.zeros((len(runs), H, dv, dk), np.complex128)
+    for s, idx in runs:
+        sl = idx[-1]
+        for h in range(H):
+            M = np.zeros((dv, dk), np.complex128) if M0 is None else M0[s, h].copy()
+            for c0 in range(sl.start, sl.stop, chunk):
+                c1 = min(c0 + chunk, sl.stop)
+                rows = (*idx[:-1], slice(c0, c1), h)
+                O, M = _chunk_rowdecay(M, K[rows], Q[rows], V[rows], lr[rows], be[rows])
+                out[rows] = O
+            Mf[s, h] = M
+    return out, Mf

@@ -10,7 +10,10 @@
   1e-12 for several chunk sizes, dense and varlen, Laplace keys |K| < 1, beta up to 2, M0 != 0;
 * the reduction to the real gated delta rule that the CUDA path runs on: with S = [Re M | Im M]^T,
   k = (Re K, Im K) / sqrt(dk), q = (Re Q, Im Q) / dk, v = lam sqrt(dk) V, alpha = lam and
-  beta' = beta / lam, the (separately pinned) real oracle returns the same outputs and state.
+  beta' = beta / lam, the (separately pinned) real oracle returns the same outputs and state;
+* the per-row decay form (one decay per value channel): with equal rows it is the scalar memory,
+  each channel is the scalar memory with that channel's decay, beta = 0 is pure per-row decay in
+  closed form, and its chunk form (a triangular solve per channel) equals the definition.
 """
 import json
 import os
@@ -199,3 +202,71 @@ def test_backward_matches_finite_differences():
                 if not np.iscomplexobj(x):
                     g = got[name]
                 assert np.max(np.abs(fd - g)) / (1.0 + np.max(np.abs(fd))) < 1e-6, (name, part)
+
+
+# ---- the per-row decay (the Laplace core's diag(r_t) on the output rows of M) ------------------
+
+def with_row_decays(c, rng, spread=0.4):
+    """The case with one finite log-decay per (token, head, value channel); some decays are strong
+    (r down to about 1e-3), as finite as the phase memory requires (r > 0, like lam)."""
+    dv = c["V"].shape[-1]
+    lr = -np.log1p(np.exp(rng.normal(size=(*c["log_lam"].shape, dv)))) * spread
+    lr.reshape(-1)[5] = -7.0
+    return dict(c, log_r=lr)
+
+
+def run_rd(c, fn=phase.forward_rowdecay, **kw):
+    return fn(c["K"], c["Q"], c["V"], c["log_r"], c["beta"], c["M0"], cu_seqlens=c["cu_seqlens"], **kw)
+
+
+def test_rowdecay_with_equal_rows_is_the_scalar_memory():
+    rng = np.random.default_rng(50)
+    for c in (rand_case(rng, B=2, T=40, H=2, dk=6, dv=4, laplace=True, beta_max=2.0),
+              rand_case(rng, H=2, dk=5, dv=3, lengths=[7, 0, 30, 1])):
+        c = dict(c, log_r=np.repeat(c["log_lam"][..., None], c["V"].shape[-1], axis=-1))
+        o, M = run_rd(c)
+        o2, M2 = run(c)
+        np.testing.assert_allclose(o, o2, atol=1e-13)
+        np.testing.assert_allclose(M, M2, atol=1e-13)
+
+
+def test_rowdecay_is_one_scalar_memory_per_channel():
+    # channel j of the per-row memory is the scalar-decay memory with value V[..., j], decay
+    # log_r[..., j] and initial rows M0[:, :, j] (the separately pinned ``forward``)
+    rng = np.random.default_rng(51)
+    for lengths in (None, [9, 0, 33, 2]):
+        c = with_row_decays(rand_case(rng, B=2, T=37, H=2, dk=6, dv=4, laplace=True, beta_max=2.0,
+                                      lengths=lengths), rng)
+        o, M = run_rd(c)
+        assert np.abs(np.diff(c["log_r"], axis=-1)).max() > 0.1  # the channels' decays do differ
+        for j in range(c["V"].shape[-1]):
+            cj = dict(c, V=c["V"][..., j:j + 1], log_lam=c["log_r"][..., j], M0=c["M0"][:, :, j:j + 1])
+            oj, Mj = run(cj)
+            np.testing.assert_allclose(o[..., j], oj[..., 0], atol=1e-12)
+            np.testing.assert_allclose(M[:, :, j], Mj[:, :, 0], atol=1e-12)
+
+
+def test_rowdecay_beta_zero_is_pure_row_decay():
+    rng = np.random.default_rng(52)
+    c = with_row_decays(rand_case(rng, B=1, T=15, H=2, dk=4, dv=3), rng)
+    c["beta"] = np.zeros_like(c["beta"])
+    o, M = run_rd(c)
+    G = np.cumsum(c["log_r"][0], axis=0)  # [T, H, dv]
+    dk = c["K"].shape[-1]
+    for t in range(15):
+        for h in range(2):
+            Mt = np.exp(G[t, h])[:, None] * c["M0"][0, h]
+            np.testing.assert_allclose(o[0, t, h], (Mt @ np.conj(c["Q"][0, t, h])).real / dk, atol=1e-12)
+    np.testing.assert_allclose(M[0], np.exp(G[-1])[:, :, None] * c["M0"][0], atol=1e-12)
+
+
+@pytest.mark.parametrize("chunk", [1, 5, 16, 64])
+def test_rowdecay_chunk_form_equals_definition(chunk):
+    rng = np.random.default_rng(60 + chunk)
+    for lengths in (None, [0, 1, 63, 64, 65, 20]):
+        c = with_row_decays(rand_case(rng, B=2, T=90, H=2, dk=6, dv=5, laplace=True, beta_max=2.0,
+                                      lengths=lengths), rng)
+        o, M = run_rd(c)
+        o2, M2 = run_rd(c, phase.forward_rowdecay_chunkwise, chunk=chunk)
+        np.testing.assert_allclose(o2, o, atol=1e-12)
+        np.testing.assert_allclose(M2, M, atol=1e-12)
