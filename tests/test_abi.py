@@ -290,3 +290,39 @@ def test_phase_backward_rejects_before_any_launch():
     assert gdn.gdn_phase_bwd(**dict(a, K=FAKE + 4)) == gdn.GDN_ERR_INVALID_ARGUMENT
     assert gdn.gdn_phase_bwd(**dict(a, workspace=None)) == gdn.GDN_ERR_WORKSPACE
     assert gdn.gdn_phase_bwd_workspace_bytes(1, 64, 1, 64, 64, 0) == ctypes.c_size_t(-1).value
+
+
+def declared_prototypes():
+    """name -> (return type, [parameter types]) for every GDN_API declaration in include/."""
+    protos = {}
+    for hdr in os.listdir(os.path.join(ROOT, "include")):
+        if not hdr.endswith(".h"):
+            continue
+        text = re.sub(r"/\*.*?\*/", " ", open(os.path.join(ROOT, "include", hdr)).read(), flags=re.S)
+        for ret, name, params in re.findall(r"GDN_API\s+([^;(]*?)\b(gdn_\w+)\s*\(([^)]*)\)\s*;", text):
+            plist = [p.strip() for p in params.split(",") if p.strip() and p.strip() != "void"]
+            protos[name] = (" ".join(ret.split()), plist)
+    return protos
+
+
+def ctype_of(decl):
+    """The ctypes type a C parameter or return type must be marshalled as."""
+    if "*" in decl:
+        return ctypes.c_char_p if decl.replace(" ", "").startswith("constchar*") else ctypes.c_void_p
+    words = decl.replace("const", "").split()
+    base = words[0]
+    return {"int": ctypes.c_int, "size_t": ctypes.c_size_t, "float": ctypes.c_float}[base]
+
+
+def test_binding_signatures_match_the_header():
+    # every entry's ctypes argtypes and restype agree with its C prototype, parameter by parameter
+    # (a shifted or mistyped argument would reach a kernel as a wrong pointer or size)
+    protos = declared_prototypes()
+    assert len(protos) >= 20
+    for name, (ret, params) in sorted(protos.items()):
+        fn = getattr(gdn._lib, name)
+        assert fn.argtypes is not None, f"{name}: no argtypes"
+        got = list(fn.argtypes)
+        want = [ctype_of(p) for p in params]
+        assert got == want, f"{name}: argtypes {got} != header {want}"
+        assert fn.restype == ctype_of(ret), f"{name}: restype {fn.restype} != header {ret}"
