@@ -2,13 +2,16 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--quick]
 
-One step = one gdn_chunk_fwd over the hybrid-LM prefill batch (B=8, T=4096, H=12, dk=dv=64,
-chunk 64, bf16 q/k/v, fp32 gates and state): the whole chunkwise path (gates, intra-chunk
-products, triangular inverse, state chain, outputs, final state) in the library's kernels.
-Inputs are synthetic (seeded, see workloads.py) and resident in HBM before timing; L2 is flushed
-(a 256 MB device write) between timed steps because the batch is smaller than L2.  Rank 0 prints
-one JSON line.  Extra objects report the decode workload (N=256, H=32, d=128, 1000 steps;
-state-updates/s, HBM fraction) and the long-context and varlen prefill workloads.
+One step = one gdn_chunk_fwd over the varlen packed prefill batch (32 sequences with lengths
+uniform in [128, 8192], H=16, dk=dv=128, chunk 64, bf16 q/k/v, beta in (0, 2), strong decays
+log_alpha = -softplus(N(0, 2)) with some alpha near 0, fp32 gates and state), the largest of the single-GPU prefill
+workloads: the whole chunkwise path (gates, intra-chunk products, triangular inverse, state
+chain, outputs, final states) in the library's kernels.  Inputs are synthetic (seeded, see
+workloads.py) and resident in HBM before timing; the inputs are larger than L2 and L2 is flushed
+(a 256 MB device write) between timed steps as well.  Rank 0 prints one JSON line.  The line
+also reports, each with its own roofline and CPU baseline, the hybrid-LM prefill batch (B=8,
+T=4096, H=12, d=64), the long-context prefill (B=1, T=65536, H=16, d=128) and the decode workload
+(N=256, H=32, d=128, 1000 steps; state-updates/s, HBM fraction by algorithmic and by DRAM bytes).
 
 With --gpus N (under torchrun) every rank runs its own batch (independent sequences need no
 exchange): weak scaling, time = max over ranks.  --impl reference times the fp64 CPU oracle on
@@ -395,14 +398,77 @@ def cpu_oracle_baseline(inp, budget_s=12.0):
     oracle.forward(inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["beta"], inp["S0"],
                    cu_seqlens=inp["cu_seqlens"], units=units)
     dt = time.perf_counter() - t0
-    if inp["cu_seqlens"] is None:
-        th = n * inp["T"]
-    else:
-        cu = inp["cu_seqlens"]
-        th = sum(int(cu[u // H + 1] - cu[u // H]) for u in units)
+    th = chain_token_heads(inp, units)
     return dict(value=(th / H) / dt, unit="tokens/s", cores=threads, kind="oracle",
                 sample=f"{n} of {n_units} (sequence, head) chains, each in full "
-                       f"({th} token-heads, {dt:.2f} s, fp64 sequential recurrence)")
+                       f"({th} token-heads = {th / H:.0f} tokens, {dt:.2f} s, fp64 sequential recurrence)")
+
+
+def chain_token_heads(inp, units):
+    """Token-heads of the given (sequence * H + head) chains: each chain's sequence length."""
+    H = inp["H"]
+    if inp["cu_seqlens"] is None:
+        return len(units) * inp["T"]
+    cu = inp["cu_seqlens"]
+    return sum(int(cu[u // H + 1] - cu[u // H]) for u in units)
+
+
+def cpu_decode_baseline(states=64, steps=100):
+    """The fp64 decode oracle, as it stands, on the host cores: `steps` steps of a sample of
+    `states` of the decode workload's states; returns state-updates/s and the sample."""
+    import oracle
+    cfg = workloads.CONFIGS["decode"]
+    N, H, dk, dv = cfg["N"], cfg["H"], cfg["dk"], cfg["dv"]
+    sel = list(range(states))
+    S = workloads.make_decode_state(N, H, dk, dv, cfg["seed"]).double().numpy().reshape(N * H, dk, dv)
+    S = S[sel][:, None]
+    xs = []
+    for step in range(steps):
+        x = workloads.make_decode_step_inputs(N, H, dk, dv, cfg["dtype"], seed=cfg["seed"], step=step,
+                                              la_scale=cfg["la_scale"])
+        xs.append({k: v.reshape(N * H, *v.shape[2:])[sel][:, None] for k, v in x.items()})
+    t0 = time.perf_counter()
+    for x in xs:
+        _, S = oracle.decode_step(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], S)
+    dt = time.perf_counter() - t0
+    return dict(value=states * steps / dt, unit="state-updates/s", cores=oracle.max_threads(), kind="oracle",
+                sample=f"{states} of {N * H} states x {steps} of {cfg['steps']} steps "
+                       f"({dt:.2f} s, fp64 sequential update)")
+
+
+HEADLINE = "varlen"
+WORKLOAD_TEXT = {
+    "varlen": "varlen packed prefill chunk forward: 32 sequences, lengths U[128,8192] (seeded draw), "
+              "H=16 dk=dv=128 chunk=64, bf16 q/k/v/out, fp32 gates and state, beta=2 sigmoid(N(0,1)), "
+              "log_alpha=-softplus(N(0,2)), S0=0",
+    "hybrid_lm": "hybrid_lm prefill chunk forward: B=8 T=4096 H=12 dk=dv=64 chunk=64, bf16 q/k/v/out, "
+                 "fp32 gates and state, beta=sigmoid(N(0,1)), log_alpha=-0.1 softplus(N(0,1)), S0=0",
+    "long_context": "long-context prefill chunk forward: B=1 T=65536 H=16 dk=dv=128 chunk=64, bf16 q/k/v/out, "
+                    "fp32 gates and state, beta=sigmoid(N(0,1)), log_alpha=-0.1 softplus(N(0,1)), "
+                    "S0~N(0,0.02), final state returned",
+}
+
+
+def headline_config(world):
+    """The `config` object of the JSON line, identical in both arms."""
+    cfg = workloads.CONFIGS[HEADLINE]
+    return {"workload": WORKLOAD_TEXT[HEADLINE],
+            "global_batch": cfg["n_seqs"] * world, "seq_len": f"U[{cfg['len_lo']},{cfg['len_hi']}]",
+            "heads": cfg["H"], "head_dim": cfg["dk"],
+            "parallelism": f"dp{world} (independent sequences per rank)",
+            "l2": "inputs larger than L2 (126 MB); the GPU arm also flushes L2 (256 MB device write) "
+                  "between timed steps"}
+
+
+def roofline_obj(nums, peaks, peak_kind, traffic):
+    return {"bound": "hbm", "achieved": nums["gbs"], "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": nums["gbs"] / peaks["hbm_gbs"], "traffic": traffic,
+            "peak_source": f"{peak_kind} hbm_gbs", "algo_bytes_per_launch": nums["algo_bytes"]}
+
+
+def tensor_obj(nums, peaks):
+    return {"achieved_tflops": nums["tflops"], "peak_tflops": peaks["bf16_tflops"],
+            "frac": nums["tensor_frac"], "algo_flops_per_launch": nums["algo_flops"]}
 
 
 def run_ours(args, world, rank, local):
@@ -410,7 +476,7 @@ def run_ours(args, world, rank, local):
     peaks, peak_kind = load_peaks()
     stream = torch.cuda.Stream()
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device="cuda")
-    name = "hybrid_lm"
+    name = HEADLINE
     cfg = workloads.CONFIGS[name]
     inp = workloads.config_inputs(name, seed=rank_seed(cfg["seed"], rank))
     d = to_dev(inp)
@@ -426,69 +492,76 @@ def run_ours(args, world, rank, local):
     main = chunk_numbers(name, d, times, peaks)
     tokens_all = main["tokens"] * world
     value = aggregate_tokens_per_s(main["tokens"], world, ms)
+    del d
 
-    e2e_ms, h2d, d2h = e2e_chunk(gdn, inp, max(3, args.steps // 10), 2, stream)
+    e2e_ms, h2d, d2h = e2e_chunk(gdn, inp, max(3, args.steps // 10), 3, stream)
     e2e_ms = max_over_ranks(e2e_ms, world)
 
-    extra = {}
+    others = {}
     decode = None
+    extra = {}
     if not args.quick:
+        # the other prefill workloads, each with its own roofline (CPU baselines below)
+        for w in ("hybrid_lm", "long_context"):
+            cw = workloads.CONFIGS[w]
+            dw = to_dev(workloads.config_inputs(w, seed=rank_seed(cw["seed"], rank)))
+            tw = time_chunk(gdn, dw, max(3, args.steps // 2 if w == "hybrid_lm" else args.steps // 4), 3,
+                            flush, stream)
+            nums = chunk_numbers(w, dw, tw, peaks)
+            nums["workload"] = WORKLOAD_TEXT[w]
+            nums["roofline"] = roofline_obj(nums, peaks, peak_kind, ncu_traffic("chunk", w))
+            nums["tensor"] = tensor_obj(nums, peaks)
+            others[w] = {k: (round(v, 6) if isinstance(v, float) else v) for k, v in nums.items()}
+            del dw
         decode = time_decode(gdn, 1000, 10, stream)
         decode["hbm_frac"] = decode["gbs"] / peaks["hbm_gbs"]
-        # DRAM bytes per step from the ncu record of the current decode source (null once it changed)
+        # DRAM bytes per step from the ncu record of the current decode source (null once it
+        # changed): part of the state stream is served by L2, so the DRAM-side fraction is lower
         decode["traffic"] = ncu_traffic("decode", "decode")
+        if decode["traffic"]:
+            decode["dram_gbs"] = decode["traffic"] / (decode["ms_per_step"] * 1e-3) / 1e9
+            decode["dram_hbm_frac"] = decode["dram_gbs"] / peaks["hbm_gbs"]
+        decode["roofline"] = {"bound": "hbm", "achieved": decode["gbs"], "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                              "frac": decode["hbm_frac"], "traffic": decode["traffic"],
+                              "peak_source": f"{peak_kind} hbm_gbs",
+                              "algo_bytes_per_launch": decode["algo_bytes_per_step"],
+                              "frac_by_dram_bytes": decode.get("dram_hbm_frac")}
         dfu = time_decode(gdn, 300, 10, stream, fused=True)
         extra["decode_fused"] = {k: (round(v, 6) if isinstance(v, float) else v) for k, v in dfu.items()}
         extra["decode_fused"]["hbm_frac"] = round(dfu["gbs"] / peaks["hbm_gbs"], 5)
-        for w in ("long_context", "varlen"):
-            dw = to_dev(workloads.config_inputs(w))
-            tw = time_chunk(gdn, dw, max(3, args.steps // 20), 2, flush, stream)
-            nums = chunk_numbers(w, dw, tw, peaks)
-            extra[w] = {k: (round(v, 6) if isinstance(v, float) else v) for k, v in nums.items()}
-            del dw
-        dw = wide_value_inputs(rank_seed(cfg["seed"], rank))
+        hl = workloads.CONFIGS["hybrid_lm"]
+        dw = wide_value_inputs(rank_seed(hl["seed"], rank))
         nums = chunk_numbers(WIDE_VALUE, dw, time_chunk(gdn, dw, max(3, args.steps // 2), 3, flush, stream), peaks)
         extra["hybrid_lm_dv256"] = {k: (round(v, 6) if isinstance(v, float) else v) for k, v in nums.items()}
         del dw
-        # the same hybrid-LM step from raw projections: fused prologue vs PyTorch prologue + call
-        dr = to_dev(workloads.config_raw_inputs(name, seed=rank_seed(cfg["seed"], rank)))
+        # the hybrid-LM step from raw projections: fused prologue vs PyTorch prologue + call
+        dr = to_dev(workloads.config_raw_inputs("hybrid_lm", seed=rank_seed(hl["seed"], rank)))
         for key, fused in (("hybrid_lm_fused_prologue", True), ("hybrid_lm_pytorch_prologue", False)):
             tw = time_prologue(gdn, dr, max(3, args.steps // 2), 3, flush, stream, fused)
             ms_w = statistics.mean(tw)
             extra[key] = {"workload": f"hybrid_lm from raw projections ({'fused entry' if fused else 'PyTorch normalisation and activations, then the plain entry'})",
-                          "ms": round(ms_w, 6), "tokens_per_s": round(main["tokens"] / (ms_w * 1e-3), 1),
+                          "ms": round(ms_w, 6), "tokens_per_s": round(8 * 4096 / (ms_w * 1e-3), 1),
                           "launches_per_call": 1 if fused else None}
         del dr
         # grouped value heads: the hybrid-LM shape with 6 q/k heads for its 12 value heads
         dg = to_dev(workloads.make_gva_chunk_inputs(B=8, T=4096, Hk=6, Hv=12, dk=64, dv=64, dtype="bf16",
-                                                    seed=rank_seed(cfg["seed"], rank), la_scale=0.1))
+                                                    seed=rank_seed(hl["seed"], rank), la_scale=0.1))
         outg = torch.empty_like(dg["v"])
         Sg = torch.empty((8, 12, 64, 64), dtype=torch.float32, device="cuda")
 
         def call_gva():
             gdn.chunk_fwd_gva(dg["q"], dg["k"], dg["v"], dg["log_alpha"], dg["beta"], out=outg, S_final=Sg,
                               stream=stream)
-        with torch.cuda.stream(stream):
-            for _ in range(3):
-                flush.zero_()
-                call_gva()
-            stream.synchronize()
-            evg = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                   for _ in range(max(3, args.steps // 2))]
-            for a0, b0 in evg:
-                flush.zero_()
-                a0.record(stream)
-                call_gva()
-                b0.record(stream)
-            stream.synchronize()
-        ms_g = statistics.mean(a0.elapsed_time(b0) for a0, b0 in evg)
+        ms_g = _time_loop(call_gva, max(3, args.steps // 2), 3, flush, stream)
         extra["hybrid_lm_gva"] = {"workload": "hybrid_lm shape, grouped value heads: Hk=6 q/k heads, Hv=12 value heads",
                                   "ms": round(ms_g, 6), "tokens_per_s": round(8 * 4096 / (ms_g * 1e-3), 1),
                                   "launches_per_call": 1}
         del dg, outg, Sg
-        extra["hybrid_lm_backward"] = backward_numbers(gdn, d, 5, 3, flush, stream, peaks)
+        dh = to_dev(workloads.config_inputs("hybrid_lm", seed=rank_seed(hl["seed"], rank)))
+        extra["hybrid_lm_backward"] = backward_numbers(gdn, dh, 5, 3, flush, stream, peaks)
+        del dh
         dw = to_dev(workloads.make_chunk_inputs(B=8, T=4096, H=12, dk=64, dv=128, dtype="bf16",
-                                                seed=rank_seed(cfg["seed"], rank), la_scale=0.1))
+                                                seed=rank_seed(hl["seed"], rank), la_scale=0.1))
         extra["hybrid_lm_backward_dv128"] = backward_numbers(gdn, dw, 3, 3, flush, stream, peaks)
         del dw
         extra["phase_memory"] = phase_numbers(gdn, 5, 3, flush, stream, peaks)
@@ -498,7 +571,7 @@ def run_ours(args, world, rank, local):
         # rather than losing it
         try:
             dw = to_dev(workloads.make_chunk_inputs(B=8, T=4096, H=12, dk=128, dv=128, dtype="bf16",
-                                                    seed=rank_seed(cfg["seed"], rank), la_scale=0.1))
+                                                    seed=rank_seed(hl["seed"], rank), la_scale=0.1))
             extra["hybrid_lm_backward_dk128"] = backward_numbers(gdn, dw, 3, 3, flush, stream, peaks)
             del dw
         except Exception as exc:  # noqa: BLE001  (reported, not hidden)
@@ -506,6 +579,12 @@ def run_ours(args, world, rank, local):
     cpu = None
     if rank == 0 and world == 1:
         cpu = cpu_oracle_baseline(inp)
+        if not args.quick:
+            for w in ("hybrid_lm", "long_context"):
+                cw = workloads.CONFIGS[w]
+                others[w]["cpu_baseline"] = cpu_oracle_baseline(
+                    workloads.config_inputs(w, seed=rank_seed(cw["seed"], rank)), budget_s=6.0)
+            decode["cpu_baseline"] = cpu_decode_baseline()
 
     if rank != 0:
         return
@@ -522,25 +601,20 @@ def run_ours(args, world, rank, local):
         "scaling": "weak",
         "vs_baseline": None,
         "dtype": "bf16",
-        "data": "synthetic (seeded; q,k L2-normalised N(0,1), v N(0,1), beta=sigmoid(N(0,1)), "
-                "log_alpha=-0.1*softplus(N(0,1)), S0=0)",
-        "config": {"workload": "hybrid_lm prefill chunk forward: B=8 T=4096 H=12 dk=dv=64 "
-                               "chunk=64, bf16 q/k/v/out, fp32 gates and state",
-                   "global_batch": 8 * world, "seq_len": 4096, "heads": 12, "head_dim": 64,
-                   "parallelism": f"dp{world} (independent sequences per rank)",
-                   "l2": "flushed between timed steps (256 MB device write)"},
-        "roofline": {"bound": "hbm", "achieved": main["gbs"], "peak": peaks["hbm_gbs"],
-                     "unit": "GB/s", "frac": main["gbs"] / peaks["hbm_gbs"],
-                     "traffic": traffic, "peak_source": f"{peak_kind} hbm_gbs",
-                     "algo_bytes_per_launch": main["algo_bytes"]},
-        "tensor": {"achieved_tflops": main["tflops"], "peak_tflops": peaks["bf16_tflops"],
-                   "frac": main["tensor_frac"], "algo_flops_per_launch": main["algo_flops"]},
+        "data": "synthetic (seeded; varlen lengths U[128,8192]; q,k L2-normalised N(0,1), v N(0,1), "
+                "beta=2 sigmoid(N(0,1)), log_alpha=-softplus(N(0,2)), S0=0)",
+        "config": headline_config(world),
+        "roofline": roofline_obj(main, peaks, peak_kind, traffic),
+        "tensor": tensor_obj(main, peaks),
         "e2e": {"value": tokens_all / (e2e_ms * 1e-3), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         "gpu_launches": args.steps * main["launches_per_call"],
         "clocks": clk.result(),
         "cpu_baseline": cpu,
+        "tokens_per_step": main["tokens"],
     }
+    if others:
+        line.update(others)
     if decode is not None:
         line["decode"] = decode
     if extra:
@@ -714,30 +788,36 @@ def run_only(args):
 
 # ---- reference arm: the fp64 oracle on the host cores ----------------------------------------
 
-def run_reference(args, world, rank):
+def run_reference(args, world, rank, inp=None):
+    """The reference arm: the fp64 oracle on the host cores over a bounded sample of the headline
+    workload's chains per step; returns the JSON line (rank 0) or None."""
     if rank != 0:
-        return
+        return None
     import oracle
-    name = "hybrid_lm"
-    inp = workloads.config_inputs(name)
+    if inp is None:
+        inp = workloads.config_inputs(HEADLINE)
     H = inp["H"]
     n_units = inp["B"] * H
     threads = oracle.max_threads()
-    # each step: a bounded sample of whole chains, sized so the whole run takes a few minutes
+    # each step: a bounded sample of whole chains (one per host thread), taken in turn over the
+    # workload's chains, so that the whole run takes a few minutes
     per_step = max(threads, 8)
-    times = []
+    times, token_heads = [], []
     for i in range(args.warmup + args.steps):
         units = [(i * per_step + j) % n_units for j in range(per_step)]
         t0 = time.perf_counter()
         oracle.forward(inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["beta"], inp["S0"],
-                       units=units)
+                       cu_seqlens=inp["cu_seqlens"], units=units)
         dt = time.perf_counter() - t0
         if i >= args.warmup:
             times.append(dt)
+            token_heads.append(chain_token_heads(inp, units))
     s = statistics.mean(times)
-    value = (per_step * inp["T"]) / s
+    # tokens, not token-heads: a token of the workload is all H of its heads
+    value = (sum(token_heads) / H) / sum(times)
     sample = (f"{per_step} of {n_units} (sequence, head) chains per step, each in full "
-              f"({per_step * inp['T']} token-heads), fp64 sequential recurrence")
+              f"({sum(token_heads) // len(token_heads)} token-heads per step on average, "
+              f"counted as token-heads / {H} tokens), fp64 sequential recurrence")
     line = {
         "impl": "reference",
         "metric": METRIC,
@@ -752,16 +832,14 @@ def run_reference(args, world, rank):
         "vs_baseline": None,
         "dtype": "f64",
         "data": "synthetic (seeded, same inputs as the GPU arm)",
-        "config": {"workload": "hybrid_lm prefill chunk forward: B=8 T=4096 H=12 dk=dv=64 "
-                               "chunk=64, bf16 q/k/v/out, fp32 gates and state",
-                   "global_batch": 8, "seq_len": 4096, "heads": 12, "head_dim": 64,
-                   "parallelism": "host cores (OpenMP over chains)"},
+        "config": headline_config(world),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
+        "token_heads_timed": sum(token_heads), "seconds_timed": sum(times),
     }
-    print(json.dumps(line), flush=True)
+    return line
 
 
 def main():
@@ -782,7 +860,9 @@ def main():
     if args.impl == "reference":
         world = int(os.environ.get("WORLD_SIZE", "1"))
         rank = int(os.environ.get("RANK", "0"))
-        run_reference(args, world, rank)
+        line = run_reference(args, world, rank)
+        if line is not None:
+            print(json.dumps(line), flush=True)
         return
     world, rank, local = dist_setup(args.gpus)
     try:

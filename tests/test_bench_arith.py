@@ -61,3 +61,24 @@ def test_backward_product_count():
     assert bench.bwd_products(1, 2) == 26 + 14
     assert bench.bwd_products(1, 4) == 26 + 3 * 14
     assert bench.bwd_products(2, 2) > bench.bwd_products(1, 2) + 26
+
+
+def test_reference_arm_counts_tokens_not_token_heads():
+    """The reference arm's tokens/s is token-heads / H over the timed seconds, on a varlen pack
+    whose chains differ in length, and agrees with the CPU-baseline leg's count of the same
+    chains."""
+    import argparse
+    import workloads
+    inp = workloads.make_chunk_inputs(H=3, dk=64, dv=64, dtype="bf16", seed=5, lengths=[70, 5, 130])
+    args = argparse.Namespace(steps=2, warmup=3)
+    line = bench.run_reference(args, 1, 0, inp=inp)
+    th, s = line["token_heads_timed"], line["seconds_timed"]
+    assert line["unit"] == "tokens/s"
+    assert abs(line["value"] - th / 3 / s) <= 1e-9 * line["value"]
+    # every chain of the pack, in full: 3 heads x (70 + 5 + 130) token-heads
+    assert bench.chain_token_heads(inp, range(9)) == 3 * 205
+    assert bench.chain_token_heads(inp, [0, 1, 2]) == 3 * 70
+    dense = workloads.make_chunk_inputs(B=2, T=40, H=3, dk=64, dv=64, dtype="bf16", seed=5)
+    assert bench.chain_token_heads(dense, range(6)) == 6 * 40
+    assert bench.run_reference(args, 1, 1, inp=inp) is None
+    assert line["config"] == bench.headline_config(1)
