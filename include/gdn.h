@@ -158,8 +158,14 @@ GDN_API size_t gdn_chunk_fwd_workspace_bytes(int B, int T, int H, int dk, int dv
  * that has reserved its device memory up front and admits no call-time allocation, or a C host
  * program without a device allocator).  Arguments, layouts and results are those of
  * gdn_chunk_fwd.
- *   - The first call on each device looks up the array's address there (and loads the module);
- *     make that first call before any stream capture on that device.
+ *   - Every call looks up the array's address in the current context.  The first call on a
+ *     device also loads the module that holds it; make that first call before any stream
+ *     capture on that device.
+ *   - Footprint: the array takes 32 MiB of device memory on every device where its module is
+ *     loaded -- with CUDA's default lazy module loading, from the first gdn_chunk_fwd_noalloc
+ *     call on that device; with CUDA_MODULE_LOADING=EAGER, from the CUDA runtime's
+ *     initialisation of the device -- until the process exits.  Callers that reserve device
+ *     memory up front should budget for it.
  *   - Calls on the same device must not overlap in time (two streams, two host threads): they
  *     share the one array.  Nothing in it needs to start at zero.
  *   - Sizes whose scratch would exceed 32 MiB return GDN_ERR_WORKSPACE (about 3 * SMs * dk * dv
@@ -354,6 +360,14 @@ GDN_API int gdn_decode_step_gva(const void *q, const void *k, const void *v, con
  * out, after which the kernel stopped issuing work and returned): GDN_ERR_TIMEOUT if so, GDN_OK
  * if not, GDN_ERR_CUDA if the synchronisation itself failed.  The record is per device and is
  * cleared by this call.
+ *   - After GDN_ERR_TIMEOUT the outputs of every call enqueued since the previous status check
+ *     are undefined (the kernel that gave up skipped the rest of its work, and tensor-core or
+ *     copy operations it had already issued may have finished after it stopped waiting for
+ *     them).  Discard those results and run the calls again.  Only a wait that ran out is
+ *     recorded -- no memory access is made out of bounds -- so the context itself stays usable;
+ *     a caller that cannot tell why a wait ran out (a wait runs out only when an operation did
+ *     not complete within 2 s) should synchronise, check for CUDA errors, and recreate the
+ *     context if any is reported.
  */
 GDN_API int gdn_device_status(void *stream);
 

@@ -1,6 +1,8 @@
 // gdn_api.cu -- the C-ABI of libgdn (declared in include/gdn.h): argument validation on the
-// host, choice of kernel, and launch on the caller's stream.  No device memory is allocated here
-// or anywhere else in the library.
+// host, choice of kernel, and launch on the caller's stream.  No call allocates device memory.
+// The one fixed device footprint of the library is the 32 MiB scratch array of
+// gdn_chunk_fwd_noalloc (gdn_noalloc.cu), held on each device where its module is loaded (with
+// CUDA's default lazy loading: from that entry point's first call on the device).
 #include <stdarg.h>
 #include <stdio.h>
 #include <string.h>

@@ -13,8 +13,6 @@
 // results.  Calls whose scratch would exceed kScratchBytes are rejected with GDN_ERR_WORKSPACE.
 // Nothing in the scratch has to start at zero: the segment scan writes every byte it reads
 // (offset table, local states, transitions, entry states) earlier in the same call.
-#include <mutex>
-
 #include "gdn_internal.h"
 #include "../../include/gdn.h"
 
@@ -26,41 +24,29 @@ namespace {
 // device, the largest case there (dv = 256 counts its two column blocks as chains, which halves
 // segments x heads: 74 * (2 * 128 * 256 + 128 * 128) * 4 B = 24.2 MB).
 constexpr size_t kScratchBytes = size_t(32) << 20;
-constexpr int kMaxDevices = 64;
-
-std::mutex g_mu;
-void *g_scratch_ptr[kMaxDevices];
 
 }  // namespace
 
+// The array takes 32 MiB on every device where the module that holds it is loaded: with CUDA's
+// default lazy module loading that happens the first time gdn_chunk_fwd_noalloc runs on the
+// device; with CUDA_MODULE_LOADING=EAGER, when the CUDA runtime initialises the device.  It stays
+// until the process exits (or the context is destroyed).
 static __device__ __align__(256) unsigned char g_scratch[kScratchBytes];
 
-// Device address of g_scratch on the current device, looked up once per device with that device
-// current.  The first call on a device loads this module there, so make it before any stream
-// capture on that device.
+// Device address of g_scratch in the current context, looked up on every call with the target
+// device current.  The lookup is cheap once the module is loaded, and taking it afresh each time
+// keeps it valid when the context changes under the library (a cudaDeviceReset, or a driver-API
+// context the caller made current), where a cached address could point at unmapped memory.  The
+// first call on a device loads the module there, so make it before any stream capture.
 static int scratch_on_current_device(void **ptr)
 {
-    int dev = -1;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) {
-        gdn::set_error("gdn_chunk_fwd_noalloc: cudaGetDevice: %s", cudaGetErrorString(e));
+    void *p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_scratch);
+    if (e != cudaSuccess || p == nullptr) {
+        gdn::set_error("gdn_chunk_fwd_noalloc: cudaGetSymbolAddress: %s", cudaGetErrorString(e));
         return GDN_ERR_CUDA;
     }
-    if (dev < 0 || dev >= kMaxDevices) {
-        gdn::set_error("gdn_chunk_fwd_noalloc: device %d beyond the %d supported", dev, kMaxDevices);
-        return GDN_ERR_UNSUPPORTED;
-    }
-    std::lock_guard<std::mutex> lock(g_mu);
-    if (!g_scratch_ptr[dev]) {
-        void *p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_scratch);
-        if (e != cudaSuccess || p == nullptr) {
-            gdn::set_error("gdn_chunk_fwd_noalloc: cudaGetSymbolAddress: %s", cudaGetErrorString(e));
-            return GDN_ERR_CUDA;
-        }
-        g_scratch_ptr[dev] = p;
-    }
-    *ptr = g_scratch_ptr[dev];
+    *ptr = p;
     return GDN_OK;
 }
 

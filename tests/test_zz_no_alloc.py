@@ -9,7 +9,6 @@ import pytest
 import torch
 
 import workloads
-from tests.parity import TOL
 
 pytestmark = pytest.mark.gpu
 
@@ -27,10 +26,14 @@ def _p(t):
 
 CASES = {
     # the segment scan runs (scratch in use): one long sequence, both head sizes
-    "segmented_d128": dict(B=1, T=81 * 64 - 45, H=2, d=128, seed=901),
-    "segmented_d64_two_seqs": dict(B=2, T=2100, H=3, d=64, seed=902),
+    "segmented_d128": dict(B=1, T=81 * 64 - 45, H=2, dk=128, dv=128, seed=901),
+    "segmented_d64_two_seqs": dict(B=2, T=2100, H=3, dk=64, dv=64, seed=902),
+    # plans near the array's limit: 74 segments x 2 chains fill 148 SMs (29.1 MB at dk = dv = 128;
+    # 24.2 MB at dv = 256, whose two column blocks count as the chains)
+    "segmented_d128_full": dict(B=1, T=74 * 16 * 64 - 17, H=2, dk=128, dv=128, seed=904, min_mb=28),
+    "segmented_dv256_full": dict(B=1, T=74 * 16 * 64, H=1, dk=128, dv=256, seed=905, min_mb=23),
     # no scratch needed: many chains
-    "single_pass": dict(B=4, T=300, H=8, d=64, seed=903),
+    "single_pass": dict(B=4, T=300, H=8, dk=64, dv=64, seed=903),
 }
 
 
@@ -38,16 +41,18 @@ CASES = {
 def test_noalloc_matches_workspace_entry(name):
     import linear_attention_sequence_rule_b200 as gdn
     c = CASES[name]
-    inp = workloads.make_chunk_inputs(B=c["B"], T=c["T"], H=c["H"], dk=c["d"], dv=c["d"],
+    inp = workloads.make_chunk_inputs(B=c["B"], T=c["T"], H=c["H"], dk=c["dk"], dv=c["dv"],
                                       dtype="bf16", seed=c["seed"], s0_std=0.05, la_scale=0.1)
     d = {k: (v.cuda() if torch.is_tensor(v) else v) for k, v in inp.items()}
-    B, T, H, dk, dv = c["B"], c["T"], c["H"], c["d"], c["d"]
+    B, T, H, dk, dv = c["B"], c["T"], c["H"], c["dk"], c["dv"]
     stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
     head = (_p(d["q"]), _p(d["k"]), _p(d["v"]), _p(d["log_alpha"]), _p(d["beta"]), _p(d["S0"]))
     dims = (B, T, H, dk, dv, 64, None, gdn.GDN_DTYPE_BF16)
 
     need = gdn.gdn_chunk_fwd_workspace_bytes(B, T, H, dk, dv, 64, 0, gdn.GDN_DTYPE_BF16)
     assert (need > 0) == name.startswith("segmented")
+    if "min_mb" in c and torch.cuda.get_device_properties(0).multi_processor_count == 148:
+        assert c["min_mb"] * 1e6 <= need <= 32 * 2 ** 20, need
     ws = torch.empty(max(need, 1), dtype=torch.uint8, device="cuda")
     out_ref = torch.empty_like(d["v"])
     Sf_ref = torch.empty(B, H, dk, dv, device="cuda")
@@ -61,5 +66,7 @@ def test_noalloc_matches_workspace_entry(name):
         rc = gdn.gdn_chunk_fwd_noalloc(*head, _p(out), _p(Sf), *dims, stream)
         assert rc == gdn.GDN_OK, gdn.gdn_last_error()
         assert gdn.gdn_device_status(stream) == gdn.GDN_OK
-        assert (out.float() - out_ref.float()).abs().max().item() <= TOL["bf16"]
-        assert (Sf - Sf_ref).abs().max().item() <= TOL["bf16"]
+        # the same kernels on the same segment plan: identical bits, so a partly overwritten or
+        # stale scratch array would show here
+        assert torch.equal(out, out_ref)
+        assert torch.equal(Sf, Sf_ref)
