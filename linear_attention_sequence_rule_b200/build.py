@@ -30,9 +30,8 @@ NVCC_FLAGS = [
 ]
 
 
-# per-file extra flags: the tensor-core kernel runs 288 threads (9 warps), for which 224 registers
-# per thread fit the register file; without the cap the compiler assumes 12 warps (168 registers).
-FILE_FLAGS = {"gdn_chunk_tc.cu": ["-maxrregcount=224"]}
+# per-file extra flags (none at present: each kernel's __launch_bounds__ sets its register cap)
+FILE_FLAGS = {}
 
 
 def sources():

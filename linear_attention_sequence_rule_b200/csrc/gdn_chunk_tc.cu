@@ -11,20 +11,21 @@
 //   O  = diag(gam) Q S + lower_incl(Gam o Q K^T) U
 //   S' = gam_C S + K^T diag(lam) U
 //
-// One CTA of 256 threads per (sequence, head); two warpgroups work concurrently:
-//   intra warpgroup (warps 4-7), one chunk ahead of the state: gate sums (warp-shuffle segmented
-//       scan), Gram matrices [K;Q] K^T (tcgen05, M=128), decays, A = diag(b)(Gam o K K^T) and
-//       P = Gam o Q K^T, then T = (I+A)^{-1} (8x8 diagonal blocks by substitution on CUDA cores,
-//       8->16->32->64 merges on CUDA cores / mma.sync TF32), written as T diag(b) and
-//       T diag(b gam) in bf16.
+// One CTA of 384 threads per (sequence, head, value-column block); three warpgroups work
+// concurrently:
+//   two intra warpgroups (warps 4-7 and 8-11) take alternate chunks, ahead of the state chain:
+//       gate sums (warp-shuffle segmented scan), Gram matrices [K;Q] K^T (tcgen05, M=128),
+//       decays, A = diag(b)(Gam o K K^T) and P = Gam o Q K^T, T = (I+A)^{-1} (8x8 diagonal
+//       blocks by substitution on CUDA cores, 16->32->64 merges on mma.sync TF32), written as
+//       T diag(b) and T diag(b gam) in bf16, then the WY products U~^T = V^T (T diag b)^T and
+//       W^T = K^T (T diag(b gam))^T (tcgen05) and W^T to shared memory.
 //   chain warpgroup (warps 0-3), thread j = value column j, for chunk c:
 //       U^T   = U~^T - S^T W^T           (accumulated onto U~^T, A operand negated)
 //       O     = (gam Q) S + P U          (M = 64 token rows, 16-byte row stores)
 //       S'^T  = gam_C S^T + U^T (lam K)  (accumulated onto the pre-scaled fp32 state in TMEM)
-//     and, in the shadow of those MMAs, the WY part of chunk c+1: U~^T = V^T (T diag b)^T and
-//     W^T = K^T (T diag(b gam))^T (tcgen05), W^T to shared memory, gam Q and lam K in place.
-//   Loads: K/Q through a TMA stage ring (reissued as soon as a stage's last MMA completes), V
-//   single-buffered, gates by cp.async onto an mbarrier.
+//   Loads: K/Q through a TMA stage ring (NS stages, reissued as soon as a stage's last MMA
+//   completes), V through NB buffers (two where TMEM holds two output buffers), gates by cp.async
+//   onto an mbarrier.
 // The state chain's critical path per chunk is two MMA round trips plus their epilogues.
 //
 // Gates: decays are exp of log_alpha sums taken from the last exact reset (log_alpha = -inf)
