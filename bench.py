@@ -413,7 +413,7 @@ def chain_token_heads(inp, units):
     return sum(int(cu[u // H + 1] - cu[u // H]) for u in units)
 
 
-def cpu_decode_baseline(states=64, steps=100):
+def cpu_decode_baseline(states=512, steps=200):
     """The fp64 decode oracle, as it stands, on the host cores: `steps` steps of a sample of
     `states` of the decode workload's states; returns state-updates/s and the sample."""
     import oracle

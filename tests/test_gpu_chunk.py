@@ -3,8 +3,7 @@
 Small cases span several 64-token chunks, a ragged tail, both head sizes, both dtypes, varlen
 packs with empty / 1-token / boundary-length sequences, exact resets (log_alpha = -inf) and the
 extreme gates beta = 0 and beta = 2.  The named workloads run at full size in the launch
-configuration the benchmark times; where the oracle would take too long it checks a seeded
-sample of (sequence, head) chains, each chain computed in full.
+configuration the benchmark times, with every (sequence, head) chain compared.
 """
 import numpy as np
 import pytest
@@ -153,19 +152,20 @@ def test_hybrid_lm_full():
     assert e_o <= TOL["bf16"] and e_s <= TOL["bf16"], (e_o, e_s)
 
 
-def test_long_context_full_sampled_heads():
+def test_long_context_full_all_heads():
+    """The long-context workload in full (segment scan, five launches): every head's outputs and
+    final state against the oracle."""
     inp = workloads.config_inputs("long_context")
     out, Sf = run_gpu_chunk(inp)
-    units = sample_units(inp["B"] * inp["H"], 3, seed=1)
-    e_o, e_s = compare_chunk(inp, out, Sf, units)
-    assert e_o <= TOL["bf16"] and e_s <= TOL["bf16"], (e_o, e_s)
     assert torch.isfinite(out).all() and torch.isfinite(Sf).all()
+    e_o, e_s = compare_chunk(inp, out, Sf)  # all 16 heads
+    assert e_o <= TOL["bf16"] and e_s <= TOL["bf16"], (e_o, e_s)
 
 
-def test_varlen_full_sampled_chains():
+def test_varlen_full_all_chains():
+    """The varlen workload in full: all 512 (sequence, head) chains against the oracle."""
     inp = workloads.config_inputs("varlen")
     out, Sf = run_gpu_chunk(inp)
-    units = sample_units(inp["B"] * inp["H"], 12, seed=2)
-    e_o, e_s = compare_chunk(inp, out, Sf, units)
-    assert e_o <= TOL["bf16"] and e_s <= TOL["bf16"], (e_o, e_s)
     assert torch.isfinite(out).all() and torch.isfinite(Sf).all()
+    e_o, e_s = compare_chunk(inp, out, Sf)
+    assert e_o <= TOL["bf16"] and e_s <= TOL["bf16"], (e_o, e_s)
