@@ -565,6 +565,7 @@ def run_ours(args, world, rank, local):
         extra["hybrid_lm_backward_dv128"] = backward_numbers(gdn, dw, 3, 3, flush, stream, peaks)
         del dw
         extra["phase_memory"] = phase_numbers(gdn, 5, 3, flush, stream, peaks)
+        extra["phase_memory_rowdecay"] = rowdecay_numbers(gdn, 5, 3, flush, stream, peaks)
         extra["decode_small_batch_graph"] = decode_graph_numbers(gdn)
         # key head size 128 (two key blocks), the hybrid-LM token and head counts at dk = dv = 128;
         # last of the device work and guarded, so that a failure here is reported in the line
@@ -709,6 +710,29 @@ def phase_numbers(gdn, steps, warmup, flush, stream, peaks):
             "hbm_frac": round(by_p / (ms_p * 1e-3) / 1e9 / peaks["hbm_gbs"], 5)}
 
 
+def rowdecay_numbers(gdn, steps, warmup, flush, stream, peaks):
+    """The complex-phase memory with one decay per value channel (the Laplace core's diag(r_t)) at
+    the hybrid-LM shape (dk = 32 complex, dv = 64): gdn_phase_rowdecay_fwd."""
+    ph = workloads.make_phase_rowdecay_inputs(B=8, T=4096, H=12, dk=32, dv=64, dtype="bf16", seed=640)
+    d = {k: (v.cuda() if torch.is_tensor(v) else v) for k, v in ph.items()}
+    Kp, Qp = torch.view_as_real(d["K"]).contiguous(), torch.view_as_real(d["Q"]).contiguous()
+    out = torch.empty_like(d["v"])
+    Mf = torch.empty(8, 12, 64, 32, 2, device="cuda")
+
+    def call():
+        gdn.phase_rowdecay_fwd(Kp, Qp, d["v"], d["log_r"], d["beta"], out=out, M_final=Mf, stream=stream)
+    ms = _time_loop(call, steps, warmup, flush, stream)
+    # bytes per token-head: K, Q (complex fp32), v and out (bf16), log_r (fp32 per channel), beta;
+    # plus M_final
+    by = 393216 * (2 * 32 * 8 + 2 * 64 * 2 + 64 * 4 + 4) + 96 * 64 * 32 * 8
+    return {"workload": "complex-phase memory with per-channel decays, hybrid_lm shape: B=8 T=4096 H=12, "
+                        "dk=32 complex, dv=64, bf16 values, fp32 phasors and decays",
+            "ms": round(ms, 6), "tokens_per_s": round(32768 / (ms * 1e-3), 1),
+            "launches_per_call": 1, "algo_bytes": by,
+            "gbs": round(by / (ms * 1e-3) / 1e9, 3),
+            "hbm_frac": round(by / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 5)}
+
+
 def decode_graph_numbers(gdn, steps=100):
     """Small-batch decode (16 sequences x 8 heads, d = 128), where launch overhead rivals the
     kernel: 100 steps launched one by one from Python versus the same steps captured once in a
@@ -768,6 +792,9 @@ def run_only(args):
     elif args.only == "phase_memory":
         flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device="cuda")
         r = phase_numbers(gdn, args.steps, args.warmup, flush, stream, peaks)
+    elif args.only == "phase_memory_rowdecay":
+        flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device="cuda")
+        r = rowdecay_numbers(gdn, args.steps, args.warmup, flush, stream, peaks)
     elif args.only == "hybrid_lm_dv256":
         flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device="cuda")
         d = wide_value_inputs()
@@ -852,7 +879,7 @@ def main():
     ap.add_argument("--only", choices=["hybrid_lm", "long_context", "varlen", "tiny", "decode", "hybrid_lm_fused",
                                              "hybrid_lm_unfused", "hybrid_lm_backward", "phase_memory",
                                              "hybrid_lm_dv256", "hybrid_lm_backward_dv128", "decode_fused",
-                                             "hybrid_lm_backward_dk128"],
+                                             "hybrid_lm_backward_dk128", "phase_memory_rowdecay"],
                     help="time one workload's kernel loop only (for profiler runs)")
     args = ap.parse_args()
     if args.warmup < 3:

@@ -67,7 +67,7 @@ enum gdn_dtype {
 /*
  * gdn_chunk_fwd -- prefill / training forward of the recurrence over whole sequences, computed
  * chunk by chunk in the WY / UT-transform form (Sykra README, "Architectural Highlights";
- * DeltaPhase README, section 1 "Fast Triangular Solve").  Per chunk of C = 64 tokens:
+ * DeltaPhase README, section 1 "Fast Triangular Solve").  Per chunk of C = `chunk` tokens:
  *     A = strictly_lower(diag(b) (Gam o K K^T)),  T = (I + A)^{-1},
  *     W = T diag(b gam) K,  U~ = T diag(b) V,  U = U~ - W S,
  *     O = diag(gam) Q S + lower_incl(Gam o Q K^T) U,  S <- gam_C S + (diag(lam) K)^T U,
@@ -85,8 +85,11 @@ enum gdn_dtype {
  *          written.  S_final == S0 (same pointer) is allowed (in-place carry); no other
  *          overlap between any output and any input is allowed.
  * Arguments
- *   B >= 1, T >= 0 (T == 0 only with cu_seqlens), H >= 1; dk in {64, 128}; dv in {64, 128},
- *   or 256 with bf16 (run as two 128-column blocks: value columns do not interact); chunk == 64.
+ *   B >= 1, T >= 0 (T == 0 only with cu_seqlens), H >= 1; dk, dv in {64, 128, 256}; chunk in
+ *   {64, 128}.  Paths: dk, dv in {64, 128} at chunk 64 run the fused kernels (bf16: tcgen05;
+ *   fp32: CUDA cores), and bf16 at dv = 256 runs there as two 128-column blocks (value columns do
+ *   not interact); key head size 256, chunk 128 and fp32 at dv = 256 run the general path
+ *   (gdn_chunk_general.cu: fp32 on CUDA cores, the chunk factors through the workspace).
  *   log_alpha <= 0 expected (-inf allowed: an exact reset); positive values are accepted but
  *   may overflow.  beta in [0, 2].
  *   workspace / workspace_bytes: device scratch of at least gdn_chunk_fwd_workspace_bytes(...)
@@ -229,6 +232,24 @@ GDN_API int gdn_phase_fwd(const float *K, const float *Q, const void *v, const f
 GDN_API size_t gdn_phase_fwd_workspace_bytes(int B, int T, int H, int dk, int dv, int varlen, int dtype);
 
 /*
+ * gdn_phase_rowdecay_fwd -- the complex-phase delta memory with one decay per output row of the
+ * state, the Laplace core's diag(r_t) (DeltaPhase README, section 5 "Delta-Laplace Phase Memory
+ * Core", "Exact Chunkwise-Parallel Scan"; the delta steps of section 2).  Row j of M (value
+ * channel j) decays by its own r_t,j = exp(log_r_t,j):
+ *     e_t,j = V_t,j - (1/dk) Re(M_{t-1}[j] . conj K_t)
+ *     M_t[j] = r_t,j M_{t-1}[j] + beta_t e_t,j K_t
+ *     o_t,j = (1/dk) Re(M_t[j] . conj Q_t)
+ * Layouts as gdn_phase_fwd, with log_r [.., H, dv] fp32 (one decay per token, head and channel,
+ * finite) in place of log_lam.  dk in {32, 64} complex, any dv in 1 .. 4096, B and H up to 65535,
+ * dtype bf16 or fp32 for v and out (the arithmetic is fp32).  No workspace.  The channels are
+ * independent scans (gdn_phase_rowdecay.cu).  Errors as gdn_chunk_fwd; M0 == M_final (in-place
+ * carry) is allowed.
+ */
+GDN_API int gdn_phase_rowdecay_fwd(const float *K, const float *Q, const void *v, const float *log_r,
+                                   const float *beta, const float *M0, void *out, float *M_final, int B, int T,
+                                   int H, int dk, int dv, const int32_t *cu_seqlens, int dtype, void *stream);
+
+/*
  * gdn_phase_bwd -- gradients of gdn_phase_fwd for dk = 32 complex (64 real) and dv in {64, 128, 256}:
  * given the forward's inputs, dout = dL/dout (dtype) and dM_final = dL/dM_final ((re, im) pairs,
  * NULL: zero), it writes fp32
@@ -326,8 +347,9 @@ GDN_API size_t gdn_chunk_bwd_fused_workspace_bytes(int B, int T, int H, int dk, 
  *     out = a s + (k . q) u
  *     S  <- a S + k u^T
  *   q,k [N,H,dk]; v,out [N,H,dv] in dtype; log_alpha,beta [N,H] fp32; S_inout [N,H,dk,dv] fp32,
- *   read and overwritten.  N >= 1, H >= 1, dk in {64, 128}, dv in {64, 128, 256} (256 runs as two
- *   128-column blocks per state).  No overlap between S_inout and the other arguments.
+ *   read and overwritten.  N >= 1, H >= 1, dk, dv in {64, 128, 256} (dv = 256 runs as two
+ *   128-column blocks per state, and dk = 256 as dv / 64 blocks of 64 columns).  No overlap
+ *   between S_inout and the other arguments.
  */
 GDN_API int gdn_decode_step(const void *q, const void *k, const void *v, const float *log_alpha,
                     const float *beta, float *S_inout, void *out, int N, int H, int dk, int dv,

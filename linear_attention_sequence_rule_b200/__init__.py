@@ -3,12 +3,13 @@
 Argument marshalling only: every step of the computation runs in the library's CUDA kernels.
 PyTorch provides device memory and streams.  The binding has two layers:
 
-* ``gdn_chunk_fwd``, ``gdn_chunk_fwd_noalloc``, ``gdn_chunk_fwd_host``, ``gdn_phase_fwd``, ``gdn_decode_step``,
+* ``gdn_chunk_fwd``, ``gdn_chunk_fwd_noalloc``, ``gdn_chunk_fwd_host``, ``gdn_phase_fwd``,
+  ``gdn_phase_rowdecay_fwd``, ``gdn_decode_step``,
   ``gdn_chunk_fwd_workspace_bytes``, ``gdn_chunk_fwd_host_workspace_bytes``,
   ``gdn_status_string``, ``gdn_last_error``, ``gdn_version`` -- the C-ABI entry points of
   ``include/gdn.h`` with the same names and arguments (pointers as Python ints);
 * ``chunk_fwd``, ``chunk_fwd_host``, ``chunk_fwd_fused``, ``chunk_fwd_gva``, ``chunk_bwd``,
-  ``chunk_bwd_fused``, ``chunk_bwd_gva``, ``phase_fwd``, ``phase_bwd``, ``decode_step``,
+  ``chunk_bwd_fused``, ``chunk_bwd_gva``, ``phase_fwd``, ``phase_rowdecay_fwd``, ``phase_bwd``, ``decode_step``,
   ``decode_step_fused`` and ``decode_step_gva`` --
   the same calls taking torch tensors; they check shapes,
   devices and dtypes, allocate outputs with torch when none are given, and raise ``GdnError``
@@ -29,6 +30,7 @@ __all__ = [
     "gdn_chunk_fwd", "gdn_chunk_fwd_noalloc", "gdn_chunk_fwd_fused", "gdn_chunk_fwd_gva",
     "gdn_chunk_fwd_host", "gdn_chunk_fwd_host_workspace_bytes", "chunk_fwd_host",
     "gdn_phase_fwd", "gdn_phase_fwd_workspace_bytes", "phase_fwd",
+    "gdn_phase_rowdecay_fwd", "phase_rowdecay_fwd",
     "gdn_phase_bwd", "gdn_phase_bwd_workspace_bytes", "phase_bwd",
     "gdn_chunk_bwd_fused", "gdn_chunk_bwd_fused_workspace_bytes", "chunk_bwd_fused",
     "gdn_chunk_bwd_gva", "gdn_chunk_bwd_gva_workspace_bytes", "chunk_bwd_gva",
@@ -89,6 +91,8 @@ _lib.gdn_chunk_fwd_host_workspace_bytes.restype = _sz
 _lib.gdn_phase_fwd.argtypes = [_vp] * 8 + [_i] * 5 + [_vp, _i, _vp, _sz, _vp]
 _lib.gdn_phase_fwd.restype = _i
 _lib.gdn_phase_fwd_workspace_bytes.argtypes = [_i] * 7
+_lib.gdn_phase_rowdecay_fwd.argtypes = [_vp] * 8 + [_i] * 5 + [_vp, _i, _vp]
+_lib.gdn_phase_rowdecay_fwd.restype = _i
 _lib.gdn_phase_bwd.argtypes = [_vp] * 14 + [_i] * 5 + [_vp, _i, _vp, _sz, _vp]
 _lib.gdn_phase_bwd.restype = _i
 _lib.gdn_phase_bwd_workspace_bytes.argtypes = [_i] * 6
@@ -176,6 +180,12 @@ def gdn_phase_fwd(K, Q, v, log_lam, beta, M0, out, M_final, B, T, H, dk, dv, cu_
                   workspace_bytes, stream) -> int:
     return _lib.gdn_phase_fwd(K, Q, v, log_lam, beta, M0, out, M_final, B, T, H, dk, dv, cu_seqlens, dtype,
                               workspace, workspace_bytes, stream)
+
+
+def gdn_phase_rowdecay_fwd(K, Q, v, log_r, beta, M0, out, M_final, B, T, H, dk, dv, cu_seqlens, dtype,
+                           stream) -> int:
+    return _lib.gdn_phase_rowdecay_fwd(K, Q, v, log_r, beta, M0, out, M_final, B, T, H, dk, dv, cu_seqlens, dtype,
+                                       stream)
 
 
 def gdn_phase_fwd_workspace_bytes(B, T, H, dk, dv, varlen, dtype) -> int:
@@ -428,6 +438,50 @@ def phase_fwd(K, Q, v, log_lam, beta, M0=None, cu_seqlens=None, out=None, M_fina
     rc = gdn_phase_fwd(_ptr(Kp), _ptr(Qp), _ptr(v), _ptr(log_lam), _ptr(beta), _ptr(M0p), _ptr(out), _ptr(Mf),
                        B, T, H, dk, dv, _ptr(cu_seqlens), _DT[dt], _ptr(workspace), workspace.numel(),
                        _stream_ptr(stream))
+    if rc != GDN_OK:
+        raise GdnError(rc, gdn_last_error())
+    return out, (None if Mf is None else torch.view_as_complex(Mf))
+
+
+def phase_rowdecay_fwd(K, Q, v, log_r, beta, M0=None, cu_seqlens=None, out=None, M_final=None,
+                       output_final_state=True, stream=None):
+    """Complex-phase delta memory with one decay per value channel (``gdn_phase_rowdecay_fwd``):
+    as ``phase_fwd`` with log_r [.., H, dv] fp32 in place of log_lam.  Returns (out, M_final
+    complex64 or None)."""
+    Kp, Qp = _as_pairs(K, "K"), _as_pairs(Q, "Q")
+    dt = v.dtype
+    if dt not in _DT:
+        raise ValueError(f"unsupported dtype {dt}")
+    dev = v.device
+    if cu_seqlens is not None:
+        T, H, dk = Kp.shape[:3]
+        B = cu_seqlens.shape[0] - 1
+        lead = (T,)
+        _need(cu_seqlens, "cu_seqlens", torch.int32, (B + 1,), dev)
+    else:
+        B, T, H, dk = Kp.shape[:4]
+        lead = (B, T)
+    dv = v.shape[-1]
+    _need(Kp, "K", torch.float32, (*lead, H, dk, 2), dev)
+    _need(Qp, "Q", torch.float32, (*lead, H, dk, 2), dev)
+    _need(v, "v", dt, (*lead, H, dv), dev)
+    _need(log_r, "log_r", torch.float32, (*lead, H, dv), dev)
+    _need(beta, "beta", torch.float32, (*lead, H), dev)
+    M0p = _as_pairs(M0, "M0")
+    if M0p is not None:
+        _need(M0p, "M0", torch.float32, (B, H, dv, dk, 2), dev)
+    if out is None:
+        out = torch.empty((*lead, H, dv), dtype=dt, device=dev)
+    _need(out, "out", dt, (*lead, H, dv), dev)
+    Mf = None
+    if M_final is not None:
+        Mf = torch.view_as_real(M_final) if M_final.is_complex() else M_final
+    elif output_final_state:
+        Mf = torch.empty((B, H, dv, dk, 2), dtype=torch.float32, device=dev)
+    if Mf is not None:
+        _need(Mf, "M_final", torch.float32, (B, H, dv, dk, 2), dev)
+    rc = gdn_phase_rowdecay_fwd(_ptr(Kp), _ptr(Qp), _ptr(v), _ptr(log_r), _ptr(beta), _ptr(M0p), _ptr(out),
+                                _ptr(Mf), B, T, H, dk, dv, _ptr(cu_seqlens), _DT[dt], _stream_ptr(stream))
     if rc != GDN_OK:
         raise GdnError(rc, gdn_last_error())
     return out, (None if Mf is None else torch.view_as_complex(Mf))

@@ -40,18 +40,26 @@ static int cuda_fail(cudaError_t e, const char *where)
 
 static bool head_dim_ok(int d) { return d == 64 || d == 128; }
 
-// Shared shape/type checks of the chunk forward (and, without the forward's head sizes, of the
-// backward); returns GDN_OK or an error code.
+// Shapes of the chunk forward: the fused tensor-core kernel (bf16; dk, dv in {64, 128}, dv 256 as
+// two column blocks; chunk 64) and the fp32 CUDA-core kernel (fp32; dk, dv in {64, 128}; chunk
+// 64) cover the common sizes; key head size 256 and chunk 128 (and fp32 at dv 256) take the
+// general two-launch path of gdn_chunk_general.cu.
+static bool general_path(int dk, int dv, int chunk, int dtype)
+{
+    return chunk_general_needed(dk, dv, chunk) || (dv == 256 && dtype == GDN_DTYPE_F32);
+}
+
+// Shared shape/type checks of the chunk forward (and, with fwd = false, of the backward, which
+// keeps chunk 64 and its own head sizes); returns GDN_OK or an error code.
 static int check_chunk_shape(int B, int T, int H, int dk, int dv, int chunk, int varlen, int dtype,
-                             bool fwd_heads = true)
+                             bool fwd = true)
 {
     if (dtype != GDN_DTYPE_BF16 && dtype != GDN_DTYPE_F32)
         return fail(GDN_ERR_UNSUPPORTED, "gdn_chunk_fwd: unknown dtype %d", dtype);
-    if (fwd_heads && (!head_dim_ok(dk) || !(head_dim_ok(dv) || (dv == 256 && dtype == GDN_DTYPE_BF16))))
-        return fail(GDN_ERR_UNSUPPORTED,
-                    "gdn_chunk_fwd: dk=%d dv=%d, supported: dk 64 or 128, dv 64 or 128 (256 with bf16)", dk, dv);
-    if (chunk != 64)
-        return fail(GDN_ERR_UNSUPPORTED, "gdn_chunk_fwd: chunk=%d, supported: 64", chunk);
+    if (fwd && (!(head_dim_ok(dk) || dk == 256) || !(head_dim_ok(dv) || dv == 256)))
+        return fail(GDN_ERR_UNSUPPORTED, "gdn_chunk_fwd: dk=%d dv=%d, supported: dk and dv in {64, 128, 256}", dk, dv);
+    if (fwd ? (chunk != 64 && chunk != 128) : chunk != 64)
+        return fail(GDN_ERR_UNSUPPORTED, "gdn_chunk_fwd: chunk=%d, supported: %s", chunk, fwd ? "64 or 128" : "64");
     if (B < 1 || H < 1)
         return fail(GDN_ERR_INVALID_ARGUMENT, "gdn_chunk_fwd: B=%d H=%d must be >= 1", B, H);
     if (T < 0 || (!varlen && T < 1))
@@ -64,8 +72,9 @@ static int check_chunk_shape(int B, int T, int H, int dk, int dv, int chunk, int
     return GDN_OK;
 }
 
-static size_t chunk_workspace(int B, int T, int H, int dk, int dv, int varlen, int dtype)
+static size_t chunk_workspace(int B, int T, int H, int dk, int dv, int chunk, int varlen, int dtype)
 {
+    if (general_path(dk, dv, chunk, dtype)) return chunk_general_workspace_bytes(B, T, H, dk, dv, chunk, varlen);
     if (dtype != GDN_DTYPE_BF16) return 0;
     return chunk_tc_workspace_bytes(B, T, H, dk, dv, varlen, dtype);
 }
@@ -97,7 +106,7 @@ size_t gdn_chunk_fwd_workspace_bytes(int B, int T, int H, int dk, int dv, int ch
                                      int dtype)
 {
     if (check_chunk_shape(B, T, H, dk, dv, chunk, varlen, dtype) != GDN_OK) return (size_t)-1;
-    return chunk_workspace(B, T, H, dk, dv, varlen, dtype);
+    return chunk_workspace(B, T, H, dk, dv, chunk, varlen, dtype);
 }
 
 namespace gdn {
@@ -125,7 +134,10 @@ static int chunk_fwd_common(const char *fn, const void *q, const void *k, const 
         if (a0 < b0 + bytes && b0 < a0 + bytes)
             return fail(GDN_ERR_INVALID_ARGUMENT, "%s: S0 and S_final overlap partially", fn);
     }
-    const size_t need = chunk_workspace(B, T, H, dk, dv, varlen, dtype);
+    if (prologue && general_path(dk, dv, chunk, dtype))
+        return fail(GDN_ERR_UNSUPPORTED, "%s: the fused prologue takes dk, dv in {64, 128} (dv 256) and chunk 64",
+                    fn);
+    const size_t need = chunk_workspace(B, T, H, dk, dv, chunk, varlen, dtype);
     if (need > 0) {
         if (!workspace || workspace_bytes < need)
             return fail(GDN_ERR_WORKSPACE, "%s: workspace of %zu bytes needed, %zu given", fn, need,
@@ -136,7 +148,9 @@ static int chunk_fwd_common(const char *fn, const void *q, const void *k, const 
     ChunkArgs a{q, k, v, log_alpha, beta, S0, out, S_final, cu_seqlens, B, T, H, dk, dv, dtype,
                 workspace, workspace_bytes, prologue, a_scale, b_scale, G};
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    cudaError_t e = dtype == GDN_DTYPE_BF16 ? launch_chunk_tc(a, st) : launch_chunk_simt(a, st);
+    cudaError_t e = general_path(dk, dv, chunk, dtype) ? launch_chunk_general(a, chunk, st)
+                    : dtype == GDN_DTYPE_BF16                ? launch_chunk_tc(a, st)
+                                                             : launch_chunk_simt(a, st);
     if (e != cudaSuccess) return cuda_fail(e, fn);
     return GDN_OK;
 }
@@ -181,9 +195,8 @@ static int decode_common(const char *fn, const void *q, const void *k, const voi
 {
     if (dtype != GDN_DTYPE_BF16 && dtype != GDN_DTYPE_F32)
         return fail(GDN_ERR_UNSUPPORTED, "%s: unknown dtype %d", fn, dtype);
-    if (!head_dim_ok(dk) || !(head_dim_ok(dv) || dv == 256))
-        return fail(GDN_ERR_UNSUPPORTED, "%s: dk=%d dv=%d, supported: dk 64 or 128, dv 64, 128 or 256", fn, dk,
-                    dv);
+    if (!(head_dim_ok(dk) || dk == 256) || !(head_dim_ok(dv) || dv == 256))
+        return fail(GDN_ERR_UNSUPPORTED, "%s: dk=%d dv=%d, supported: dk and dv in {64, 128, 256}", fn, dk, dv);
     if (N < 1 || H < 1 || (long long)N * H > (1LL << 30))
         return fail(GDN_ERR_INVALID_ARGUMENT, "%s: N=%d H=%d out of range", fn, N, H);
     if (!q || !k || !v || !log_alpha || !beta || !S_inout || !out)
@@ -252,6 +265,39 @@ int gdn_chunk_fwd_gva(const void *q, const void *k, const void *v, const float *
     return chunk_fwd_common("gdn_chunk_fwd_gva", q, k, v, log_alpha, beta, S0, out, S_final, B, T, Hv, dk, dv,
                             chunk, cu_seqlens, dtype, 0, 0.f, 0.f, workspace, workspace_bytes, stream,
                             Hv / Hk);
+}
+
+int gdn_phase_rowdecay_fwd(const float *K, const float *Q, const void *v, const float *log_r, const float *beta,
+                           const float *M0, void *out, float *M_final, int B, int T, int H, int dk, int dv,
+                           const int32_t *cu_seqlens, int dtype, void *stream)
+{
+    g_last_error[0] = 0;
+    const char *fn = "gdn_phase_rowdecay_fwd";
+    if (dtype != GDN_DTYPE_BF16 && dtype != GDN_DTYPE_F32) return fail(GDN_ERR_UNSUPPORTED, "%s: unknown dtype %d", fn, dtype);
+    if (dk != 32 && dk != 64) return fail(GDN_ERR_UNSUPPORTED, "%s: dk=%d, supported: 32 or 64 (complex)", fn, dk);
+    if (dv < 1 || dv > 4096) return fail(GDN_ERR_UNSUPPORTED, "%s: dv=%d, supported: 1 .. 4096", fn, dv);
+    const int varlen = cu_seqlens != nullptr;
+    if (B < 1 || H < 1 || T < 0 || (!varlen && T < 1))
+        return fail(GDN_ERR_INVALID_ARGUMENT, "%s: B=%d T=%d H=%d (B, H >= 1; dense T >= 1)", fn, B, T, H);
+    const long long tokens = varlen ? (long long)T : (long long)B * T;
+    if (tokens * H * (dv > 2 * dk ? dv : 2 * dk) >= (1LL << 40) || (long long)B * H * dv >= (1LL << 31) ||
+        B > 65535 || H > 65535)
+        return fail(GDN_ERR_INVALID_ARGUMENT, "%s: problem too large (B and H at most 65535)", fn);
+    if (!K || !Q || !v || !log_r || !beta || !out)
+        return fail(GDN_ERR_INVALID_ARGUMENT, "%s: K, Q, v, log_r, beta and out are required", fn);
+    const void *ptrs[] = {K, Q, v, log_r, beta, M0, out, M_final, cu_seqlens};
+    for (const void *p : ptrs)
+        if (p && !aligned16(p)) return fail(GDN_ERR_INVALID_ARGUMENT, "%s: pointer %p is not 16-byte aligned", fn, p);
+    if (M0 && M_final && M0 != M_final) {
+        const size_t bytes = (size_t)B * H * dv * dk * 2 * sizeof(float);
+        const char *a0 = (const char *)M0, *b0 = (const char *)M_final;
+        if (a0 < b0 + bytes && b0 < a0 + bytes)
+            return fail(GDN_ERR_INVALID_ARGUMENT, "%s: M0 and M_final overlap partially", fn);
+    }
+    cudaError_t e = launch_phase_rowdecay(K, Q, v, log_r, beta, M0, out, M_final, cu_seqlens, B, T, H, dk, dv,
+                                          dtype == GDN_DTYPE_BF16, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, fn);
+    return GDN_OK;
 }
 
 int gdn_selftest_wait_timeout(int limit_ms, void *stream)

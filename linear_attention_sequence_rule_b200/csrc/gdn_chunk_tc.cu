@@ -74,7 +74,7 @@ struct TcCfg {
     static constexpr int NI = 2;
     static constexpr int THREADS = 128 * (1 + NI);
     static constexpr int NS = (DK == 128 || DV == 128) ? 2 : 3;  // K/Q stages
-    // buffers of V, of the bf16 S^T copy and of O: two where TMEM holds two O buffers (the V load
+    // buffers of V and of O: two where TMEM holds two O buffers (the V load
     // of a chunk then starts two chunks ahead, and the output epilogue overlaps the next state MMA)
     static constexpr int NB = (2 * DV + DK + NI * 64 + NS * 64 <= 512) ? 2 : 1;
     // shared memory byte offsets (swizzled tiles first, all 1024-aligned)
@@ -83,9 +83,11 @@ struct TcCfg {
     static constexpr int V = KQ + NS * KQ_STAGE;                 // per buffer: per 64-column block 8 KB
     static constexpr int V_BUF = (DV / 64) * 8192;
     static constexpr int PM = V + NB * V_BUF;                    // per stage: P bf16, 64 x 128 B
-    static constexpr int ST = PM + NS * 8192;                    // per buffer: S^T bf16, per 64-feature block DV x 128 B
+    static constexpr int ST = PM + NS * 8192;                    // S^T bf16, per 64-feature block DV x 128 B
     static constexpr int ST_BUF = (DK / 64) * DV * 128;
-    static constexpr int UT = ST + NB * ST_BUF;                  // U^T bf16, DV x 128 B
+    // one S^T copy: the copy of chunk c + 1 is written once the state MMA of chunk c has
+    // completed, and that MMA's commit also covers the U and O1 MMAs that read the copy of chunk c
+    static constexpr int UT = ST + ST_BUF;                       // U^T bf16, DV x 128 B
     static constexpr int WG0 = UT + DV * 128;                    // per intra warpgroup:
     static constexpr int W_TB = 0;                               //   T diag(b)      bf16 64 x 128 B
     static constexpr int W_TG = 8192;                            //   T diag(b gam)  bf16 64 x 128 B
@@ -416,9 +418,8 @@ __global__ void __launch_bounds__(TcCfg<DK, DV>::THREADS, 1)
     constexpr int NI = L::NI;
     constexpr int NB = L::NB;
     using B = Bars<NS, NI, NB>;
-    // gam Q and lam K are formed in place by the chain (dk = 128, whose chain has slack while the
-    // U MMA runs) or by the intra side (dk = 64, where the chain is the busier side)
-    constexpr bool kChainScales = DK == 128;
+    // gam Q and lam K are formed in place by the intra side, which runs ahead of the chain
+    constexpr bool kChainScales = false;
     extern __shared__ unsigned char smem_raw[];
     // 1024-aligned base by pointer arithmetic on the shared array, so that the compiler keeps
     // every access below in the shared address space
@@ -672,7 +673,10 @@ __global__ void __launch_bounds__(TcCfg<DK, DV>::THREADS, 1)
                     for (int i = 0; i < CH; i += 4)
                         *reinterpret_cast<float4 *>(&AT[r * LDF + i]) = make_float4(x[i], x[i + 1], x[i + 2], x[i + 3]);
                 }
-                if (!kChainScales) scale_row_bf16(Kt + 8192, r, gam[r], (t >> 6) * 4, (t >> 6) * 4 + 4);
+                if (!kChainScales) {
+                    if (DK == 64) scale_row_bf16(Kt + 8192, r, gam[r], (t >> 6) * 4, (t >> 6) * 4 + 4);
+                    else scale_row_bf16(Kt + (t >> 6) * 16384 + 8192, r, gam[r], 0, 8);
+                }
             }
             tc_fence_before();
             // this warpgroup's previous chunk: its W^T and T diag(b..) tiles must have been read
@@ -736,7 +740,10 @@ __global__ void __launch_bounds__(TcCfg<DK, DV>::THREADS, 1)
                     tmem_wait_ld();
                     st_half_row_bf16_sw128(WTs, wi * 16 + (t & 15), (t >> 4) & 1, x);
                 }
-                if (!kChainScales) scale_row_bf16(Kt, t & 63, lam[t & 63], (t >> 6) * 4, (t >> 6) * 4 + 4);
+                if (!kChainScales) {
+                    if (DK == 64) scale_row_bf16(Kt, t & 63, lam[t & 63], (t >> 6) * 4, (t >> 6) * 4 + 4);
+                    else scale_row_bf16(Kt + (t >> 6) * 16384, t & 63, lam[t & 63], 0, 8);
+                }
             }
             fence_proxy_async_smem();
             tc_fence_before();
@@ -763,9 +770,9 @@ __global__ void __launch_bounds__(TcCfg<DK, DV>::THREADS, 1)
             if (kHalf) tmem_st16x2_32<DK / 2>(tl + L::T_S + 32 * k, x);
             else tmem_st32(tl + L::T_S + 32 * k, x);
         };
-        // bf16 copy of S^T row j, features 32cb .. 32cb+31, into S^T buffer b
-        auto store_state_bf16 = [&](int b, int cb, const float (&x)[32]) {
-            unsigned char *stt = sm + L::ST + b * L::ST_BUF + (cb >> 1) * (DV * 128);
+        // bf16 copy of S^T row j, features 32cb .. 32cb+31
+        auto store_state_bf16 = [&](int cb, const float (&x)[32]) {
+            unsigned char *stt = sm + L::ST + (cb >> 1) * (DV * 128);
 #pragma unroll
             for (int cc = 0; cc < 4; ++cc) {
                 const int chunk = (cb & 1) * 4 + cc;
@@ -825,7 +832,7 @@ __global__ void __launch_bounds__(TcCfg<DK, DV>::THREADS, 1)
                 for (int i = 0; i < 32; ++i)
                     x[i] = (flags & kFlagS0Identity) ? ((cb * 32 + i == j) ? 1.f : 0.f)
                                                      : (S0 ? S0[sbase + (size_t)(cb * 32 + i) * ldv + j] : 0.f);
-                store_state_bf16(0, cb, x);
+                store_state_bf16(cb, x);
 #pragma unroll
                 for (int i = 0; i < 32; ++i) x[i] *= g0;
                 st_state(k, x);
@@ -838,7 +845,7 @@ __global__ void __launch_bounds__(TcCfg<DK, DV>::THREADS, 1)
         for (int c = 0; c < nchunks; ++c) {
             const int st = c % NS;
             const uint32_t tO = tmem + L::T_O + (c % NB) * DV;
-            const uint32_t stc = smem_u32(sm + L::ST + (c % NB) * L::ST_BUF);  // S_c^T, bf16
+            const uint32_t stc = smem_u32(sm + L::ST);  // S_c^T, bf16
             unsigned char *Kt = sm + L::KQ + st * L::KQ_STAGE;
             const unsigned char *WTc = sm + L::WG0 + (c % NI) * L::WG_BYTES + L::W_WT;
             // O = (gam Q) S: A = gam-scaled Q tile (K-major), B = S^T rows (K-major)
@@ -923,7 +930,7 @@ __global__ void __launch_bounds__(TcCfg<DK, DV>::THREADS, 1)
             tc_fence_after();
             if (warp == 0 && c + NS < nchunks) load_kq(c + NS);
             {
-                // S_{c+1} = gam_C(c) S_c + increment is in TMEM; keep a bf16 copy (buffer (c+1) % NB)
+                // S_{c+1} = gam_C(c) S_c + increment is in TMEM; keep a bf16 copy
                 // and pre-scale the fp32 state by gam_C of the next chunk
                 const bool more = c + 1 < nchunks;
                 float gn = 1.f;
@@ -936,7 +943,7 @@ __global__ void __launch_bounds__(TcCfg<DK, DV>::THREADS, 1)
                     float x[32];
                     ld_state(k, x);
                     tmem_wait_ld();
-                    store_state_bf16((c + 1) % NB, s_block(k), x);
+                    store_state_bf16(s_block(k), x);
                     if (more) {
 #pragma unroll
                         for (int i = 0; i < 32; ++i) x[i] *= gn;

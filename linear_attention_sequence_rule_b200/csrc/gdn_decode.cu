@@ -181,7 +181,14 @@ cudaError_t launch_typed(const void *q, const void *k, const void *v, const floa
               *V = static_cast<const TIn *>(v);
     TIn *O = static_cast<TIn *>(out);
     const dim3 grid2(NH, 2);  // dv = 256: two 128-column blocks per state
-    if (dk == 128 && dv == 256) decode_kernel<128, 128, 2, TIn, PRO><<<grid2, block, 0, st>>>(Q, K, V, la, be, S, O, H, G, as, bs);
+    if (dk == 256) {
+        // key head size 256: 64-column blocks (a thread then holds 16 float4 of the state, as at
+        // dk = dv = 128), dv / 64 CTAs per state
+        const dim3 gridk(NH, dv / 64);
+        if (dv == 64) decode_kernel<256, 64, 1, TIn, PRO><<<gridk, block, 0, st>>>(Q, K, V, la, be, S, O, H, G, as, bs);
+        else if (dv == 128) decode_kernel<256, 64, 2, TIn, PRO><<<gridk, block, 0, st>>>(Q, K, V, la, be, S, O, H, G, as, bs);
+        else decode_kernel<256, 64, 4, TIn, PRO><<<gridk, block, 0, st>>>(Q, K, V, la, be, S, O, H, G, as, bs);
+    } else if (dk == 128 && dv == 256) decode_kernel<128, 128, 2, TIn, PRO><<<grid2, block, 0, st>>>(Q, K, V, la, be, S, O, H, G, as, bs);
     else if (dk == 64 && dv == 256) decode_kernel<64, 128, 2, TIn, PRO><<<grid2, block, 0, st>>>(Q, K, V, la, be, S, O, H, G, as, bs);
     else if (dk == 128 && dv == 128) decode_kernel<128, 128, 1, TIn, PRO><<<grid, block, 0, st>>>(Q, K, V, la, be, S, O, H, G, as, bs);
     else if (dk == 128 && dv == 64) decode_kernel<128, 64, 1, TIn, PRO><<<grid, block, 0, st>>>(Q, K, V, la, be, S, O, H, G, as, bs);

@@ -32,7 +32,7 @@ struct HostPlan {
 
 int part_count(int B) { return B < kMaxParts ? B : kMaxParts; }
 
-void layout(HostPlan &p, int B, int T, int H, int dk, int dv, int varlen, int dtype)
+void layout(HostPlan &p, int B, int T, int H, int dk, int dv, int chunk, int varlen, int dtype)
 {
     const size_t es = dtype == GDN_DTYPE_BF16 ? 2 : 4;
     const size_t tokens = varlen ? (size_t)T : (size_t)B * T;
@@ -56,16 +56,20 @@ void layout(HostPlan &p, int B, int T, int H, int dk, int dv, int varlen, int dt
     // varlen: each part gets its own slice of cu_seqlens (absolute offsets), 256-byte aligned
     p.cu_stride = varlen ? al256((size_t)(B + 1) * 4) : 0;
     p.cu = take(p.cu_stride * part_count(B));
-    // the parts run one after another on the caller's stream, so one chunk workspace serves all;
-    // only dense parts can need one (the segment scan); parts hold floor(B / P) or ceil(B / P)
-    // sequences, and the larger need of the two sizes is kept
+    // the parts run one after another on the caller's stream, so one chunk workspace serves all.
+    // Dense parts hold floor(B / P) or ceil(B / P) sequences, and the larger need of the two sizes
+    // is kept; a varlen part indexes the whole packed buffer (T tokens) with at most B sequences,
+    // so the need of the whole batch bounds every part's
     size_t ws = 0;
     if (!varlen) {
         const int P = part_count(B);
         for (int bp : {B / P, (B + P - 1) / P}) {
-            const size_t need = gdn_chunk_fwd_workspace_bytes(bp, T, H, dk, dv, 64, 0, dtype);
+            const size_t need = gdn_chunk_fwd_workspace_bytes(bp, T, H, dk, dv, chunk, 0, dtype);
             if (need != (size_t)-1 && need > ws) ws = need;
         }
+    } else {
+        const size_t need = gdn_chunk_fwd_workspace_bytes(B, T, H, dk, dv, chunk, 1, dtype);
+        if (need != (size_t)-1) ws = need;
     }
     p.ws_bytes = ws;
     p.ws = take(ws);
@@ -143,7 +147,7 @@ size_t gdn_chunk_fwd_host_workspace_bytes(int B, int T, int H, int dk, int dv, i
 {
     if (gdn_chunk_fwd_workspace_bytes(B, T, H, dk, dv, chunk, varlen, dtype) == (size_t)-1) return (size_t)-1;
     HostPlan p;
-    layout(p, B, T, H, dk, dv, varlen, dtype);
+    layout(p, B, T, H, dk, dv, chunk, varlen, dtype);
     return p.total;
 }
 
@@ -182,7 +186,7 @@ int gdn_chunk_fwd_host(const void *q, const void *k, const void *v, const float 
             }
     }
     HostPlan p;
-    layout(p, B, T, H, dk, dv, varlen, dtype);
+    layout(p, B, T, H, dk, dv, chunk, varlen, dtype);
     if (varlen) cut_varlen(p, B, cu_seqlens);
     else cut_dense(p, B);
 

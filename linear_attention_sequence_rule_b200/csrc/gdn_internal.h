@@ -43,6 +43,13 @@ cudaError_t launch_chunk_simt(const ChunkArgs &a, cudaStream_t stream);
 cudaError_t launch_chunk_tc(const ChunkArgs &a, cudaStream_t stream);
 size_t chunk_tc_workspace_bytes(int B, int T, int H, int dk, int dv, int varlen, int dtype);
 
+// Chunk forward for key head size 256 and chunk 128 (gdn_chunk_general.cu): fp32 on CUDA cores in
+// two launches (per-chunk factors, then the state chain) through a workspace of
+// chunk_general_workspace_bytes(...) bytes.
+bool chunk_general_needed(int dk, int dv, int chunk);
+size_t chunk_general_workspace_bytes(int B, int T, int H, int dk, int dv, int chunk, int varlen);
+cudaError_t launch_chunk_general(const ChunkArgs &a, int chunk, cudaStream_t stream);
+
 // Device error word of the tensor-core kernels (bounded waits that ran out); read and cleared
 // after synchronising the device.  Returns -1 when the read itself failed.
 int read_and_clear_tc_error();
@@ -67,5 +74,12 @@ struct BwdArgs {
 };
 size_t chunk_bwd_workspace_bytes(int B, int T, int H, int varlen, int G = 1, int VS = 1, int KB = 1);
 cudaError_t launch_chunk_bwd(const BwdArgs &a, cudaStream_t stream);
+
+// Complex-phase memory with one decay per value channel (gdn_phase_rowdecay.cu): K, Q, M0,
+// M_final as (re, im) fp32 pairs; V and out bf16 (bf16 != 0) or fp32.
+cudaError_t launch_phase_rowdecay(const float *K, const float *Q, const void *V, const float *log_r,
+                                  const float *beta, const float *M0, void *out, float *M_final,
+                                  const int32_t *cu_seqlens, int nseq, int T, int H, int dk, int dv, int bf16,
+                                  cudaStream_t stream);
 
 }  // namespace gdn

@@ -122,6 +122,7 @@ struct PhasePlan {
 // chunk forward's own scratch.
 bool phase_plan(PhasePlan &p, int B, int T, int H, int dk, int dv, int varlen, int dtype)
 {
+    if (dv == 256 && dtype != GDN_DTYPE_BF16) return false;  // the prologue's fp32 forms stop at 128
     const size_t ws = gdn_chunk_fwd_workspace_bytes(B, T, H, 2 * dk, dv, 64, varlen, dtype);
     if (ws == (size_t)-1) return false;
     const size_t es = dtype == GDN_DTYPE_BF16 ? 2 : 4;
@@ -277,7 +278,7 @@ int gdn_phase_fwd(const float *K, const float *Q, const void *v, const float *lo
                   const int32_t *cu_seqlens, int dtype, void *workspace, size_t workspace_bytes, void *stream)
 {
     const int varlen = cu_seqlens != nullptr;
-    if ((dk != 32 && dk != 64) || (dv != 64 && dv != 128 && dv != 256)) {
+    if ((dk != 32 && dk != 64) || (dv != 64 && dv != 128 && dv != 256) || (dv == 256 && dtype != GDN_DTYPE_BF16)) {
         set_error("gdn_phase_fwd: dk=%d dv=%d, supported: dk 32 or 64 (the real recurrence runs at 2 dk), dv 64, "
                   "128 or 256 (256 with bf16)", dk, dv);
         return GDN_ERR_UNSUPPORTED;

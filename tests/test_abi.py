@@ -49,9 +49,12 @@ def chunk(**kw):
     (dict(dtype=7), gdn.GDN_ERR_UNSUPPORTED),
     (dict(dk=96), gdn.GDN_ERR_UNSUPPORTED),
     (dict(dv=192), gdn.GDN_ERR_UNSUPPORTED),
-    (dict(dv=256, dtype=gdn.GDN_DTYPE_F32), gdn.GDN_ERR_UNSUPPORTED),
+    (dict(dk=512), gdn.GDN_ERR_UNSUPPORTED),
     (dict(dv=512), gdn.GDN_ERR_UNSUPPORTED),
     (dict(chunk=32), gdn.GDN_ERR_UNSUPPORTED),
+    (dict(chunk=96), gdn.GDN_ERR_UNSUPPORTED),
+    (dict(chunk=128, workspace=None), gdn.GDN_ERR_WORKSPACE),   # the general path needs its scratch
+    (dict(dk=256, workspace=None), gdn.GDN_ERR_WORKSPACE),
     (dict(B=0), gdn.GDN_ERR_INVALID_ARGUMENT),
     (dict(H=0), gdn.GDN_ERR_INVALID_ARGUMENT),
     (dict(T=0), gdn.GDN_ERR_INVALID_ARGUMENT),
@@ -79,6 +82,8 @@ def fused(**kw):
 @pytest.mark.parametrize("kw,code", [
     (dict(dtype=gdn.GDN_DTYPE_F32), gdn.GDN_ERR_UNSUPPORTED),
     (dict(dk=96), gdn.GDN_ERR_UNSUPPORTED),
+    (dict(dk=256), gdn.GDN_ERR_UNSUPPORTED),
+    (dict(chunk=128), gdn.GDN_ERR_UNSUPPORTED),
     (dict(a_scale=-1.0), gdn.GDN_ERR_INVALID_ARGUMENT),
     (dict(a_scale=float("inf")), gdn.GDN_ERR_INVALID_ARGUMENT),
     (dict(a_scale=float("nan")), gdn.GDN_ERR_INVALID_ARGUMENT),
@@ -112,10 +117,18 @@ def test_workspace_query():
     bad = ctypes.c_size_t(-1).value
     assert gdn.gdn_chunk_fwd_workspace_bytes(1, 64, 1, 96, 64, 64, 0, 1) == bad
     assert gdn.gdn_chunk_fwd_workspace_bytes(0, 64, 1, 64, 64, 64, 0, 1) == bad
-    assert gdn.gdn_chunk_fwd_workspace_bytes(1, 64, 1, 64, 64, 128, 0, 1) == bad
-    # value head size 256: bf16 only, as column blocks (no segment scan, so no workspace)
+    assert gdn.gdn_chunk_fwd_workspace_bytes(1, 64, 1, 64, 64, 96, 0, 1) == bad
+    # value head size 256 with bf16: column blocks of the fused kernel (no segment scan, so no
+    # workspace)
     assert gdn.gdn_chunk_fwd_workspace_bytes(1, 4096, 1, 128, 256, 64, 0, 1) == 0
-    assert gdn.gdn_chunk_fwd_workspace_bytes(1, 64, 1, 128, 256, 64, 0, 0) == bad
+    # the general path (chunk 128, key head size 256, fp32 at dv 256) passes its per-chunk factors
+    # through the workspace: W, U~ (C x dk, C x dv), P (C x C) and two decay vectors per chunk and
+    # head, plus the chunk table
+    for B, T, H, dk, dv, C, varlen, dt in ((1, 64, 1, 64, 64, 128, 0, 1), (2, 300, 3, 256, 128, 64, 0, 1),
+                                           (3, 1000, 2, 128, 256, 128, 1, 0), (1, 64, 1, 128, 256, 64, 0, 0)):
+        n = gdn.gdn_chunk_fwd_workspace_bytes(B, T, H, dk, dv, C, varlen, dt)
+        chunks = (T // C + B) if varlen else B * ((T + C - 1) // C)
+        assert n >= chunks * H * C * (dk + dv + C + 2) * 4, (B, T, H, dk, dv, C)
 
 
 def decode(**kw):
@@ -128,7 +141,7 @@ def decode(**kw):
 @pytest.mark.parametrize("kw,code", [
     (dict(dtype=3), gdn.GDN_ERR_UNSUPPORTED),
     (dict(dk=32), gdn.GDN_ERR_UNSUPPORTED),
-    (dict(dk=256), gdn.GDN_ERR_UNSUPPORTED),
+    (dict(dk=512), gdn.GDN_ERR_UNSUPPORTED),
     (dict(dv=192), gdn.GDN_ERR_UNSUPPORTED),
     (dict(N=0), gdn.GDN_ERR_INVALID_ARGUMENT),
     (dict(H=-1), gdn.GDN_ERR_INVALID_ARGUMENT),
@@ -326,3 +339,26 @@ def test_binding_signatures_match_the_header():
         want = [ctype_of(p) for p in params]
         assert got == want, f"{name}: argtypes {got} != header {want}"
         assert fn.restype == ctype_of(ret), f"{name}: restype {fn.restype} != header {ret}"
+
+
+def rowdecay_call(**kw):
+    a = dict(K=FAKE, Q=FAKE, v=FAKE, log_r=FAKE, beta=FAKE, M0=None, out=FAKE, M_final=None, B=1, T=64, H=1,
+             dk=32, dv=64, cu_seqlens=None, dtype=gdn.GDN_DTYPE_BF16, stream=None)
+    a.update(kw)
+    return gdn.gdn_phase_rowdecay_fwd(**a)
+
+
+def test_rowdecay_entry_rejects_before_any_launch():
+    assert rowdecay_call(dk=48) == gdn.GDN_ERR_UNSUPPORTED
+    assert rowdecay_call(dk=128) == gdn.GDN_ERR_UNSUPPORTED
+    assert rowdecay_call(dv=0) == gdn.GDN_ERR_UNSUPPORTED
+    assert rowdecay_call(dv=5000) == gdn.GDN_ERR_UNSUPPORTED
+    assert rowdecay_call(dtype=7) == gdn.GDN_ERR_UNSUPPORTED
+    assert rowdecay_call(B=0) == gdn.GDN_ERR_INVALID_ARGUMENT
+    assert rowdecay_call(T=0) == gdn.GDN_ERR_INVALID_ARGUMENT          # dense needs T >= 1
+    assert rowdecay_call(log_r=None) == gdn.GDN_ERR_INVALID_ARGUMENT
+    assert rowdecay_call(out=None) == gdn.GDN_ERR_INVALID_ARGUMENT
+    assert rowdecay_call(K=FAKE + 8) == gdn.GDN_ERR_INVALID_ARGUMENT   # not 16-byte aligned
+    # M0 and M_final overlapping partially
+    assert rowdecay_call(M0=FAKE, M_final=FAKE + 256) == gdn.GDN_ERR_INVALID_ARGUMENT
+    assert "rowdecay" in gdn.gdn_last_error()

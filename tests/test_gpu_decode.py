@@ -44,7 +44,8 @@ def run_steps(N, H, dk, dv, dtype, steps, seed, units=None, la_scale=0.1, beta_s
 
 
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
-@pytest.mark.parametrize("dk,dv", [(128, 128), (64, 64), (64, 128), (128, 64), (128, 256), (64, 256)])
+@pytest.mark.parametrize("dk,dv", [(128, 128), (64, 64), (64, 128), (128, 64), (128, 256), (64, 256), (256, 64),
+                                   (256, 128), (256, 256)])
 def test_small(dtype, dk, dv):
     e_o, e_s = run_steps(3, 5, dk, dv, dtype, steps=40, seed=dk * 7 + dv)
     assert e_o <= TOL[dtype] and e_s <= TOL[dtype], (e_o, e_s)

@@ -193,6 +193,21 @@ def make_phase_inputs(B=None, T=None, H=2, dk=32, dv=64, dtype="bf16", seed=0, b
                 T=(lead[0] if cu is not None else int(T)), H=H, dk=dk, dv=dv, dtype=dtype, lengths=lengths)
 
 
+def make_phase_rowdecay_inputs(B=None, T=None, H=2, dk=32, dv=64, dtype="bf16", seed=0, beta_scale=1.0,
+                               la_scale=0.1, lr_std=1.0, m0_std=0.0, laplace=False, lengths=None, **_ignored):
+    """Inputs of the phase memory with one decay per value channel: the draws of
+    ``make_phase_inputs`` (same seed, same order), then log_r [..., H, dv] =
+    -softplus(N(0, lr_std)) * la_scale from the same generator (finite: r > 0).  The scalar
+    log_lam is kept in the dict but unused by the per-channel form."""
+    d = make_phase_inputs(B=B, T=T, H=H, dk=dk, dv=dv, dtype=dtype, seed=seed, beta_scale=beta_scale,
+                          la_scale=la_scale, m0_std=m0_std, laplace=laplace, lengths=lengths)
+    g = torch.Generator().manual_seed(int(seed) * 7 + 3)
+    lead = tuple(d["v"].shape[:-2])
+    d["log_r"] = (-torch.nn.functional.softplus(lr_std * torch.randn(*lead, H, dv, generator=g))
+                  * la_scale).float()
+    return d
+
+
 def config_inputs(name: str, **overrides):
     """Inputs of a named chunk workload (``tiny``, ``hybrid_lm``, ``long_context``, ``varlen``)."""
     cfg = dict(CONFIGS[name])
