@@ -67,16 +67,29 @@ constexpr float kNormEps = 1e-6f;
 // of rank z by length (ties by index), so that the longest chains, which set the launch's length,
 // start in the first wave instead of wherever the packing put them.
 constexpr int kFlagLongestFirst = 8;
+#ifndef GDN_U_SPLIT
+#define GDN_U_SPLIT 1
+#endif
 
 template <int DK, int DV>
 struct TcCfg {
     // Two intra warpgroups take alternate chunks.
     static constexpr int NI = 2;
     static constexpr int THREADS = 128 * (1 + NI);
-    static constexpr int NS = (DK == 128 || DV == 128) ? 2 : 3;  // K/Q stages
-    // buffers of V and of O: two where TMEM holds two O buffers (the V load
-    // of a chunk then starts two chunks ahead, and the output epilogue overlaps the next state MMA)
-    static constexpr int NB = (2 * DV + DK + NI * 64 + NS * 64 <= 512) ? 2 : 1;
+    // TA (value head 128): the chain keeps its MMA A operands -- the bf16 copy of S^T and U^T --
+    // in tensor memory and forms the outputs transposed (O^T, value columns on the TMEM lanes),
+    // which frees the shared S^T and U^T copies for a third K/Q stage.
+    static constexpr bool TA = DV == 128;
+    static constexpr int NS = TA ? 3 : ((DK == 128 || DV == 128) ? 2 : 3);  // K/Q stages
+    // U~^T / U^T slots in TMEM: one per intra warpgroup (TA) or per stage
+    static constexpr int NU = TA ? NI : NS;
+    // O buffers in TMEM (two: the output epilogue of a chunk overlaps the next state MMA); O^T
+    // takes 64 columns (TA), O (M = 64 token rows) DV columns
+    static constexpr int O_COLS = TA ? 64 : DV;
+    static constexpr int SB_COLS = TA ? DK / 2 : 0;  // bf16 S^T, two per column (TA)
+    static constexpr int NBO = (2 * O_COLS + DK + SB_COLS + NI * 64 + NU * 64 <= 512) ? 2 : 1;
+    // V buffers (two: the V load of a chunk starts two chunks ahead)
+    static constexpr int NB = TA ? (DK == 64 ? 2 : 1) : NBO;
     // shared memory byte offsets (swizzled tiles first, all 1024-aligned)
     static constexpr int KQ = 0;                                 // per stage: per 64-feature block K (8K) | Q (8K)
     static constexpr int KQ_STAGE = (DK / 64) * 16384;
@@ -84,11 +97,11 @@ struct TcCfg {
     static constexpr int V_BUF = (DV / 64) * 8192;
     static constexpr int PM = V + NB * V_BUF;                    // per stage: P bf16, 64 x 128 B
     static constexpr int ST = PM + NS * 8192;                    // S^T bf16, per 64-feature block DV x 128 B
-    static constexpr int ST_BUF = (DK / 64) * DV * 128;
     // one S^T copy: the copy of chunk c + 1 is written once the state MMA of chunk c has
     // completed, and that MMA's commit also covers the U and O1 MMAs that read the copy of chunk c
-    static constexpr int UT = ST + ST_BUF;                       // U^T bf16, DV x 128 B
-    static constexpr int WG0 = UT + DV * 128;                    // per intra warpgroup:
+    static constexpr int ST_BYTES = TA ? 0 : (DK / 64) * DV * 128;
+    static constexpr int UT = ST + ST_BYTES;                     // U^T bf16, DV x 128 B
+    static constexpr int WG0 = UT + (TA ? 0 : DV * 128);         // per intra warpgroup:
     static constexpr int W_TB = 0;                               //   T diag(b)      bf16 64 x 128 B
     static constexpr int W_TG = 8192;                            //   T diag(b gam)  bf16 64 x 128 B
     // W^T (DK rows x 128 B bf16) is written over T diag(b gam) (dk = 64) or over both T tiles
@@ -97,23 +110,28 @@ struct TcCfg {
     static constexpr int W_AT = 16384;                           //   decays, then A, then T: fp32 [64][LDF]
     static constexpr int W_XS = W_AT + CH * LDF * 4;             //   merge scratch, 4 x 256 fp32
     static constexpr int WG_BYTES = (W_XS + 4 * 256 * 4 + 1023) & ~1023;
-    static constexpr int GT = WG0 + NI * WG_BYTES;               // per stage: gate vectors
+    // TA with two O buffers: a bf16 tile [64 tokens][DV] through which the outputs leave (one
+    // O buffer: the chunk's own K/Q stage serves, once its state MMA has completed)
+    static constexpr int OT = WG0 + NI * WG_BYTES;
+    static constexpr int OT_BYTES = (TA && NBO == 2) ? CH * DV * 2 : 0;
+    static constexpr int GT = OT + OT_BYTES;                     // per stage: gate vectors
     static constexpr int GT_STAGE = 7 * CH * 4;                  //   graw, G2, gam, lam, bet, last, (gC)
     static constexpr int BAR = GT + NS * GT_STAGE;
-    static constexpr int NBAR = 5 * NS + 2 * NB + 2 + 3 * NI;
+    static constexpr int NBAR = 5 * NS + NB + NBO + 2 + 4 * NI;
     static constexpr int MISC = BAR + NBAR * 8;                  // TMEM slot, abort flag
     static constexpr int TOTAL = MISC + 16;
     // TMEM columns
-    static constexpr uint32_t T_O = 0;                            // NB x DV: output rows (M = 64 tokens)
-    static constexpr uint32_t T_S = NB * DV;                      // DK: fp32 state (transposed)
-    static constexpr uint32_t T_G = T_S + DK;                     // NI x 64: Gram, then W^T (intra)
-    static constexpr uint32_t T_U = T_G + NI * 64;                // NS x 64: U~^T, then U^T
-    static_assert(T_U + NS * 64 <= 512, "TMEM budget");
+    static constexpr uint32_t T_O = 0;                            // NBO x O_COLS: outputs
+    static constexpr uint32_t T_S = NBO * O_COLS;                 // DK: fp32 state (transposed)
+    static constexpr uint32_t T_SB = T_S + DK;                    // SB_COLS: bf16 S^T (TA)
+    static constexpr uint32_t T_G = T_SB + SB_COLS;               // NI x 64: Gram, then W^T (intra)
+    static constexpr uint32_t T_U = T_G + NI * 64;                // NU x 64: U~^T, then U^T
+    static_assert(T_U + NU * 64 <= 512, "TMEM budget");
     static_assert(TOTAL + 1024 <= 232448, "shared memory budget");
 };
 
 // barrier indices
-template <int NS, int NI, int NB> struct Bars {
+template <int NS, int NI, int NB, int NBO> struct Bars {
     static constexpr int kq_full = 0;            // [NS] K/Q tiles of a stage landed (TMA)
     static constexpr int gfull = NS;             // [NS] gates landed, 32 arrivals (cp.async of chain warp 0)
     static constexpr int gready = 2 * NS;        // [NS] gate vectors (gam, lam, gam_C) computed
@@ -122,10 +140,11 @@ template <int NS, int NI, int NB> struct Bars {
     static constexpr int v_full = 5 * NS;        // [NB] V tile landed
     static constexpr int u = 5 * NS + NB;
     static constexpr int s = 5 * NS + NB + 1;
-    static constexpr int o = 5 * NS + NB + 2;    // [NB] output MMAs of a chunk done
-    static constexpr int gram = 5 * NS + 2 * NB + 2;   // [NI] Gram MMA done
+    static constexpr int o = 5 * NS + NB + 2;    // [NBO] output MMAs of a chunk done
+    static constexpr int gram = 5 * NS + NB + NBO + 2;  // [NI] Gram MMA done
     static constexpr int uw = gram + NI;               // [NI] WY MMAs done
     static constexpr int tfree = uw + NI;              // [NI] chain -> intra: the U MMA has read W^T
+    static constexpr int ufree = tfree + NI;           // [NI] chain -> intra: the U slot has been read (TA)
 };
 
 // Thread roles inside an intra warpgroup (t = 0..127): the gate scan runs on warp scan_warp(wg)
@@ -417,7 +436,11 @@ __global__ void __launch_bounds__(TcCfg<DK, DV>::THREADS, 1)
     constexpr int NS = L::NS;
     constexpr int NI = L::NI;
     constexpr int NB = L::NB;
-    using B = Bars<NS, NI, NB>;
+    constexpr int NBO = L::NBO;
+    constexpr bool TA = L::TA;
+    // TA: U^T enters the state and output MMAs as two bf16 parts (hi + lo)
+    constexpr bool kUSplit = GDN_U_SPLIT;
+    using B = Bars<NS, NI, NB, NBO>;
     // gam Q and lam K are formed in place by the intra side, which runs ahead of the chain
     constexpr bool kChainScales = false;
     extern __shared__ unsigned char smem_raw[];
@@ -699,10 +722,13 @@ __global__ void __launch_bounds__(TcCfg<DK, DV>::THREADS, 1)
             fence_proxy_async_smem();
             tc_fence_before();
             named_bar(bar_id, 128);
-            // ---- WY products: U~^T = V^T (T diag b)^T into the stage's U slot and
+            // ---- WY products: U~^T = V^T (T diag b)^T into the chunk's U slot and
             //      W^T = K^T (T diag(b gam))^T over the Gram accumulator ----
             if (t == kIssuer) {
                 if (!v_zero) ctl.wait(B::v_full + c % NB, (c / NB) & 1);
+                // TA: the slot is this warpgroup's; the chain's state and output MMAs of its
+                // previous chunk read U^T from it
+                if (TA && kc >= 1) ctl.wait(B::ufree + wg, (kc - 1) & 1);
                 if (!ctl.aborted()) {
                     tc_fence_after();
                     constexpr uint32_t idU = idesc_bf16(DV, 64, 1, 0);
@@ -710,7 +736,7 @@ __global__ void __launch_bounds__(TcCfg<DK, DV>::THREADS, 1)
                     if (!v_zero) {
 #pragma unroll
                         for (int kk = 0; kk < 4; ++kk)
-                            mma_bf16(tmem + L::T_U + st * 64,
+                            mma_bf16(tmem + L::T_U + (TA ? wg : st) * 64,
                                      sdesc_sw128(smem_u32(sm + L::V + (c % NB) * L::V_BUF + kk * 2048), 8192, 1024),
                                      sdesc_sw128(smem_u32(TBs + kk * 32), 16, 1024), idU, kk > 0);
                     }
@@ -727,17 +753,28 @@ __global__ void __launch_bounds__(TcCfg<DK, DV>::THREADS, 1)
             {
                 // W^T rows (one per feature) to shared memory in bf16, then (unless the chain does
                 // it) lam K in place: the W MMA has read K unscaled
+                // TA: -W^T, so that the chain's U MMA (A operand in tensor memory) adds
+                // S^T (-W^T) onto U~^T without negating its A operand
+                constexpr float wsign = TA ? -1.f : 1.f;
                 if (DK == 128) {
                     float x[64];
                     tmem_ld32(tl + tG, *reinterpret_cast<float(*)[32]>(&x[0]));
                     tmem_ld32(tl + tG + 32, *reinterpret_cast<float(*)[32]>(&x[32]));
                     tmem_wait_ld();
+                    if (TA) {
+#pragma unroll
+                        for (int i = 0; i < 64; ++i) x[i] *= wsign;
+                    }
                     st_row_bf16_sw128(WTs, t, x);
                 } else {
                     // M = 64 layout: threads lane and lane + 16 take the two halves of a row
                     float x[32];
                     tmem_ld16x2_32<32>(tl + tG, x);
                     tmem_wait_ld();
+                    if (TA) {
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) x[i] *= wsign;
+                    }
                     st_half_row_bf16_sw128(WTs, wi * 16 + (t & 15), (t >> 4) & 1, x);
                 }
                 if (!kChainScales) {
@@ -791,7 +828,7 @@ __global__ void __launch_bounds__(TcCfg<DK, DV>::THREADS, 1)
             const long tk = tok0 + (long)c * CH;
             const int n = (int)min((long)CH, len - (long)c * CH);
             if (want_out) {
-                ctl.wait(B::o + c % NB, (c / NB) & 1);
+                ctl.wait(B::o + c % NBO, (c / NBO) & 1);
                 tc_fence_after();
                 if (tid == 0) ctl.arrive(B::cdone + (c % NS));
                 const int r = 16 * warp + (lane & 15);
@@ -799,7 +836,7 @@ __global__ void __launch_bounds__(TcCfg<DK, DV>::THREADS, 1)
 #pragma unroll 1
                 for (int cb = 0; cb < DV / 64; ++cb) {
                     float o[32];
-                    tmem_ld16x2_32<DV / 2>(tl + L::T_O + (c % NB) * DV + cb * 32, o);
+                    tmem_ld16x2_32<DV / 2>(tl + L::T_O + (c % NBO) * DV + cb * 32, o);
                     tmem_wait_ld();
                     if (r < n) {
                         uint4 *dst = reinterpret_cast<uint4 *>(op + cb * 32);
@@ -820,143 +857,326 @@ __global__ void __launch_bounds__(TcCfg<DK, DV>::THREADS, 1)
             }
             named_bar(1, 128);
         };
-        if (nchunks > 0) {
-            // initial state: S^T row j (fp32, pre-scaled by gam_C of chunk 0) and its bf16 copy
-            ctl.wait(B::gready + 0, 0);
-            const float g0 = gates(0)[6 * CH];
-#pragma unroll 1
-            for (int k = 0; k < kSB; ++k) {
-                const int cb = s_block(k);
-                float x[32];
+        if constexpr (TA) {
+            // ---- value head 128: thread j = value column = TMEM lane j.  The bf16 copy of S^T
+            //      and U^T are the A operands of the chain's MMAs, read from tensor memory; the
+            //      outputs are formed as O^T (64 token columns) ----
+            // S^T row j (64 features) as 32 packed bf16 pairs into the copy at column 32 kb
+            auto st_state_bf16 = [&](int kb, const float *x) {
+                float p[32];
 #pragma unroll
-                for (int i = 0; i < 32; ++i)
-                    x[i] = (flags & kFlagS0Identity) ? ((cb * 32 + i == j) ? 1.f : 0.f)
-                                                     : (S0 ? S0[sbase + (size_t)(cb * 32 + i) * ldv + j] : 0.f);
-                store_state_bf16(cb, x);
+                for (int i = 0; i < 32; ++i) p[i] = __uint_as_float(pack_bf16x2(x[2 * i], x[2 * i + 1]));
+                tmem_st32(tl + L::T_SB + 32 * kb, *reinterpret_cast<const float(*)[32]>(p));
+            };
+            // Outputs of chunk c: O^T row j holds column j of the chunk's 64 token rows.  They
+            // leave through a bf16 tile in shared memory -- thread j writes column j (16-byte
+            // units XOR-swizzled by row), then each thread stores half a row with 16-byte stores
+            // -- the chunk's own K/Q stage with one O buffer (free from its state MMA's
+            // completion until the next load is issued into it), a tile of its own with two.
+            auto out_epilogue_staged = [&](int c, unsigned char *buf) {
+                if (!want_out) return;
+                const long tk = tok0 + (long)c * CH;
+                const int n = (int)min((long)CH, len - (long)c * CH);
+                {
+                    float o[64];
+                    tmem_ld32(tl + L::T_O + (c % NBO) * 64, *reinterpret_cast<float(*)[32]>(&o[0]));
+                    tmem_ld32(tl + L::T_O + (c % NBO) * 64 + 32, *reinterpret_cast<float(*)[32]>(&o[32]));
+                    tmem_wait_ld();
 #pragma unroll
-                for (int i = 0; i < 32; ++i) x[i] *= g0;
-                st_state(k, x);
-            }
-            tmem_wait_st();
-            fence_proxy_async_smem();
-            tc_fence_before();
-            named_bar(1, 128);
-        }
-        for (int c = 0; c < nchunks; ++c) {
-            const int st = c % NS;
-            const uint32_t tO = tmem + L::T_O + (c % NB) * DV;
-            const uint32_t stc = smem_u32(sm + L::ST);  // S_c^T, bf16
-            unsigned char *Kt = sm + L::KQ + st * L::KQ_STAGE;
-            const unsigned char *WTc = sm + L::WG0 + (c % NI) * L::WG_BYTES + L::W_WT;
-            // O = (gam Q) S: A = gam-scaled Q tile (K-major), B = S^T rows (K-major)
-            auto issue_o1 = [&]() {
-                constexpr uint32_t idQ = idesc_bf16(64, DV, 0, 0);
+                    for (int r = 0; r < CH; ++r)
+                        *reinterpret_cast<__nv_bfloat16 *>(buf + r * 256 + (((j >> 3) ^ (r & 15)) << 4) + (j & 7) * 2) =
+                            __float2bfloat16_rn(o[r]);
+                }
+                named_bar(1, 128);
+                const int r = tid >> 1, hf = tid & 1;
+                if (r < n) {
+                    uint4 *dst = reinterpret_cast<uint4 *>(out + ((size_t)(tk + r) * H + h) * ldv + col0 + 64 * hf);
 #pragma unroll
-                for (int kk = 0; kk < DK / 16; ++kk) {
-                    const uint32_t a = smem_u32(Kt + (kk >> 2) * 16384 + 8192 + (kk & 3) * 32);
-                    mma_bf16(tO, sdesc_sw128(a, 16, 1024), sdesc_sw128(stc + (kk >> 2) * (DV * 128) + (kk & 3) * 32, 16, 1024),
-                             idQ, kk > 0);
+                    for (int i = 0; i < 8; ++i)
+                        dst[i] = *reinterpret_cast<const uint4 *>(buf + r * 256 + (((8 * hf + i) ^ (r & 15)) << 4));
                 }
             };
-            ctl.wait(B::tready + st, (c / NS) & 1);
-            if (tid == 0 && !ctl.aborted()) {
-                // U^T = U~^T - S^T W^T, accumulated onto U~^T (A operand negated)
-                tc_fence_after();
-                constexpr uint32_t idN = idesc_bf16(DV, 64, 0, 1, 1);
-#pragma unroll
-                for (int kk = 0; kk < DK / 16; ++kk) {
-                    const uint64_t a = sdesc_sw128(stc + (kk >> 2) * (DV * 128) + (kk & 3) * 32, 16, 1024);
-                    mma_bf16(tmem + L::T_U + st * 64, a, sdesc_sw128(smem_u32(WTc + kk * 2048), 16, 1024), idN,
-                             v_zero ? (kk > 0) : 1);
-                }
-                mma_commit(&bars[B::u]);
-            }
-            if (kChainScales) {
-                // while the U MMA runs: gam Q and lam K in place for O1 and the state MMA (every
-                // MMA that reads them unscaled, Gram and W, completed before the chunk was ready)
-                const float *gv = gates(st);
-                const int r = tid & 63;
-                scale_row_bf16(Kt + (tid >> 6) * 16384 + 8192, r, gv[2 * CH + r], 0, 8);
-                scale_row_bf16(Kt + (tid >> 6) * 16384, r, gv[3 * CH + r], 0, 8);
-                fence_proxy_async_smem();
-            }
-            // O1 goes before the state MMA's commit, so that its completion also covers O1's reads
-            // of the Q tile (reloaded right after) and of the S_c copy.  One O buffer: the previous
-            // chunk's outputs leave first, while the U MMA runs.
-            if (NB == 1 && c >= 1) out_epilogue(c - 1);
-            if (kChainScales) named_bar(1, 128);  // the scaled tiles are complete
-            if (tid == 0 && want_out && !ctl.aborted()) {
-                tc_fence_after();
-                issue_o1();
-            }
-            ctl.wait(B::u, c & 1);
-            tc_fence_after();
-            if (tid == 0) ctl.arrive(B::tfree + (c % NI));  // W^T of this chunk has been read
-            if (kHalf) {
-                float x[32];
-                tmem_ld16x2_32<32>(tl + L::T_U + st * 64, x);
-                tmem_wait_ld();
-                st_half_row_bf16_sw128(sm + L::UT, j, hh, x);
-            } else {
-                float x[64];
-                tmem_ld32(tl + L::T_U + st * 64, *reinterpret_cast<float(*)[32]>(&x[0]));
-                tmem_ld32(tl + L::T_U + st * 64 + 32, *reinterpret_cast<float(*)[32]>(&x[32]));
-                tmem_wait_ld();
-                st_row_bf16_sw128(sm + L::UT, j, x);
-            }
-            fence_proxy_async_smem();
-            tc_fence_before();
-            named_bar(1, 128);
-            if (tid == 0 && !ctl.aborted()) {
-                tc_fence_after();
-                constexpr uint32_t idS = idesc_bf16(DV, DK, 0, 1);
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk)  // S^T += U^T (lam K)
-                    mma_bf16(tmem + L::T_S, sdesc_sw128(smem_u32(sm + L::UT + kk * 32), 16, 1024),
-                             sdesc_sw128(smem_u32(Kt + kk * 2048), 16384, 1024), idS, 1);
-                mma_commit(&bars[B::s]);
-                if (want_out) {
-                    constexpr uint32_t idP = idesc_bf16(64, DV, 0, 0);
-#pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)  // O += P U: A = P rows (K-major), B = U^T rows (K-major)
-                        mma_bf16(tO, sdesc_sw128(smem_u32(sm + L::PM + st * 8192 + kk * 32), 16, 1024),
-                                 sdesc_sw128(smem_u32(sm + L::UT + kk * 32), 16, 1024), idP, 1);
-                    mma_commit(&bars[B::o + c % NB]);
-                }
-            }
-            // two O buffers: the previous chunk's outputs leave while the state MMA runs
-            if (NB == 2 && c >= 1) out_epilogue(c - 1);
-            ctl.wait(B::s, c & 1);
-            tc_fence_after();
-            if (warp == 0 && c + NS < nchunks) load_kq(c + NS);
-            {
-                // S_{c+1} = gam_C(c) S_c + increment is in TMEM; keep a bf16 copy
-                // and pre-scale the fp32 state by gam_C of the next chunk
-                const bool more = c + 1 < nchunks;
-                float gn = 1.f;
-                if (more) {
-                    ctl.wait(B::gready + (c + 1) % NS, ((c + 1) / NS) & 1);
-                    gn = gates((c + 1) % NS)[6 * CH];
-                }
+            if (nchunks > 0) {
+                // initial state: fp32 S^T row j pre-scaled by gam_C of chunk 0, and its bf16 copy
+                ctl.wait(B::gready + 0, 0);
+                const float g0 = gates(0)[6 * CH];
 #pragma unroll 1
-                for (int k = 0; k < kSB; ++k) {
-                    float x[32];
-                    ld_state(k, x);
-                    tmem_wait_ld();
-                    store_state_bf16(s_block(k), x);
-                    if (more) {
+                for (int kb = 0; kb < DK / 64; ++kb) {
+                    float x[64];
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) x[i] *= gn;
-                        st_state(k, x);
+                    for (int i = 0; i < 64; ++i) {
+                        const int f = kb * 64 + i;
+                        x[i] = (flags & kFlagS0Identity) ? (f == j ? 1.f : 0.f)
+                                                         : (S0 ? S0[sbase + (size_t)f * ldv + j] : 0.f);
                     }
+                    st_state_bf16(kb, x);
+#pragma unroll
+                    for (int i = 0; i < 64; ++i) x[i] *= g0;
+                    tmem_st32(tl + L::T_S + 64 * kb, *reinterpret_cast<const float(*)[32]>(&x[0]));
+                    tmem_st32(tl + L::T_S + 64 * kb + 32, *reinterpret_cast<const float(*)[32]>(&x[32]));
                 }
                 tmem_wait_st();
+                tc_fence_before();
+                named_bar(1, 128);
             }
-            fence_proxy_async_smem();
-            tc_fence_before();
-            named_bar(1, 128);
+            for (int c = 0; c < nchunks; ++c) {
+                const int st = c % NS, wu = c % NI;
+                const uint32_t tO = tmem + L::T_O + (c % NBO) * 64;
+                const uint32_t tU = tmem + L::T_U + wu * 64;  // lane 0: the MMAs' operand address
+                unsigned char *Kt = sm + L::KQ + st * L::KQ_STAGE;
+                const unsigned char *WTc = sm + L::WG0 + wu * L::WG_BYTES + L::W_WT;
+                constexpr uint32_t idU = idesc_bf16(128, 64, 0, 1);   // B = -W^T rows (MN-major)
+                constexpr uint32_t idO = idesc_bf16(128, 64, 0, 0);   // O^T: B = gam Q or P rows (K-major)
+                constexpr uint32_t idS = idesc_bf16(128, DK, 0, 1);   // B = lam K (MN-major)
+                ctl.wait(B::tready + st, (c / NS) & 1);
+                if (tid == 0 && !ctl.aborted()) {
+                    tc_fence_after();
+                    // U^T = U~^T + S^T (-W^T), accumulated onto U~^T
+#pragma unroll
+                    for (int kk = 0; kk < DK / 16; ++kk)
+                        mma_bf16_ta(tU, tmem + L::T_SB + 8 * kk, sdesc_sw128(smem_u32(WTc + kk * 2048), 16, 1024), idU,
+                                    v_zero ? (kk > 0) : 1);
+                    mma_commit(&bars[B::u]);
+                    // O^T = S^T (gam Q)^T; its completion is covered by the state MMA's commit
+                    if (want_out) {
+#pragma unroll
+                        for (int kk = 0; kk < DK / 16; ++kk)
+                            mma_bf16_ta(tO, tmem + L::T_SB + 8 * kk,
+                                        sdesc_sw128(smem_u32(Kt + (kk >> 2) * 16384 + 8192 + (kk & 3) * 32), 16, 1024),
+                                        idO, kk > 0);
+                    }
+                }
+                ctl.wait(B::u, c & 1);
+                tc_fence_after();
+                if (tid == 0) ctl.arrive(B::tfree + wu);  // W^T of this chunk has been read
+                {
+                    // U^T row j: 64 fp32 -> 32 packed bf16 pairs, over the slot's first 32 columns
+                    float x[64];
+                    tmem_ld32(tl + L::T_U + wu * 64, *reinterpret_cast<float(*)[32]>(&x[0]));
+                    tmem_ld32(tl + L::T_U + wu * 64 + 32, *reinterpret_cast<float(*)[32]>(&x[32]));
+                    tmem_wait_ld();
+                    // U^T = hi + lo in two bf16 parts (hi over columns 0-31, lo over 32-63): the
+                    // state and output MMAs then see U to about 16 bits instead of 8
+                    float p[32], pl[32];
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        const uint32_t hi = pack_bf16x2(x[2 * i], x[2 * i + 1]);
+                        p[i] = __uint_as_float(hi);
+                        const float h0 = __uint_as_float(hi << 16), h1 = __uint_as_float(hi & 0xffff0000u);
+                        pl[i] = __uint_as_float(pack_bf16x2(x[2 * i] - h0, x[2 * i + 1] - h1));
+                    }
+                    tmem_st32(tl + L::T_U + wu * 64, *reinterpret_cast<const float(*)[32]>(p));
+                    if (kUSplit) tmem_st32(tl + L::T_U + wu * 64 + 32, *reinterpret_cast<const float(*)[32]>(pl));
+                    tmem_wait_st();
+                }
+                tc_fence_before();
+                named_bar(1, 128);
+                if (tid == 0 && !ctl.aborted()) {
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < (kUSplit ? 8 : 4); ++kk)  // S^T += (U_hi + U_lo)^T (lam K)
+                        mma_bf16_ta(tmem + L::T_S, tU + 8 * kk,
+                                    sdesc_sw128(smem_u32(Kt + (kk & 3) * 2048), 16384, 1024), idS, 1);
+                    if (want_out) {
+#pragma unroll
+                        for (int kk = 0; kk < (kUSplit ? 8 : 4); ++kk)  // O^T += (U_hi + U_lo)^T P^T
+                            mma_bf16_ta(tO, tU + 8 * kk,
+                                        sdesc_sw128(smem_u32(sm + L::PM + st * 8192 + (kk & 3) * 32), 16, 1024), idO, 1);
+                    }
+                    mma_commit(&bars[B::s]);
+                    if (NBO == 2) mma_commit(&bars[B::o + c % NBO]);
+                }
+                // two O buffers: the previous chunk's outputs leave while the state MMA runs
+                if (NBO == 2 && c >= 1) {
+                    ctl.wait(B::o + (c - 1) % NBO, ((c - 1) / NBO) & 1);
+                    tc_fence_after();
+                    out_epilogue_staged(c - 1, sm + L::OT);
+                }
+                ctl.wait(B::s, c & 1);
+                tc_fence_after();
+                if (tid == 0) {
+                    ctl.arrive(B::cdone + st);  // P of this stage has been read
+                    ctl.arrive(B::ufree + wu);  // the U slot has been read
+                }
+                if (NBO == 1) {
+                    out_epilogue_staged(c, Kt);
+                    // every thread has read the tile before the stage is reloaded by TMA
+                    fence_proxy_async_smem();
+                    named_bar(1, 128);
+                }
+                if (warp == 0 && c + NS < nchunks) load_kq(c + NS);
+                {
+                    // S_{c+1} = gam_C(c) S_c + increment is in TMEM: its bf16 copy, and the fp32
+                    // state pre-scaled by gam_C of the next chunk
+                    const bool more = c + 1 < nchunks;
+                    float gn = 1.f;
+                    if (more) {
+                        ctl.wait(B::gready + (c + 1) % NS, ((c + 1) / NS) & 1);
+                        gn = gates((c + 1) % NS)[6 * CH];
+                    }
+#pragma unroll 1
+                    for (int kb = 0; kb < DK / 64; ++kb) {
+                        float x[64];
+                        tmem_ld32(tl + L::T_S + 64 * kb, *reinterpret_cast<float(*)[32]>(&x[0]));
+                        tmem_ld32(tl + L::T_S + 64 * kb + 32, *reinterpret_cast<float(*)[32]>(&x[32]));
+                        tmem_wait_ld();
+                        st_state_bf16(kb, x);
+                        if (more) {
+#pragma unroll
+                            for (int i = 0; i < 64; ++i) x[i] *= gn;
+                            tmem_st32(tl + L::T_S + 64 * kb, *reinterpret_cast<const float(*)[32]>(&x[0]));
+                            tmem_st32(tl + L::T_S + 64 * kb + 32, *reinterpret_cast<const float(*)[32]>(&x[32]));
+                        }
+                    }
+                    tmem_wait_st();
+                }
+                tc_fence_before();
+                named_bar(1, 128);
+            }
+            if (NBO == 2 && nchunks > 0) {
+                ctl.wait(B::o + (nchunks - 1) % NBO, ((nchunks - 1) / NBO) & 1);
+                tc_fence_after();
+                out_epilogue_staged(nchunks - 1, sm + L::OT);
+            }
+        } else {
+            if (nchunks > 0) {
+                // initial state: S^T row j (fp32, pre-scaled by gam_C of chunk 0) and its bf16 copy
+                ctl.wait(B::gready + 0, 0);
+                const float g0 = gates(0)[6 * CH];
+    #pragma unroll 1
+                for (int k = 0; k < kSB; ++k) {
+                    const int cb = s_block(k);
+                    float x[32];
+    #pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        x[i] = (flags & kFlagS0Identity) ? ((cb * 32 + i == j) ? 1.f : 0.f)
+                                                         : (S0 ? S0[sbase + (size_t)(cb * 32 + i) * ldv + j] : 0.f);
+                    store_state_bf16(cb, x);
+    #pragma unroll
+                    for (int i = 0; i < 32; ++i) x[i] *= g0;
+                    st_state(k, x);
+                }
+                tmem_wait_st();
+                fence_proxy_async_smem();
+                tc_fence_before();
+                named_bar(1, 128);
+            }
+            for (int c = 0; c < nchunks; ++c) {
+                const int st = c % NS;
+                const uint32_t tO = tmem + L::T_O + (c % NBO) * DV;
+                const uint32_t stc = smem_u32(sm + L::ST);  // S_c^T, bf16
+                unsigned char *Kt = sm + L::KQ + st * L::KQ_STAGE;
+                const unsigned char *WTc = sm + L::WG0 + (c % NI) * L::WG_BYTES + L::W_WT;
+                // O = (gam Q) S: A = gam-scaled Q tile (K-major), B = S^T rows (K-major)
+                auto issue_o1 = [&]() {
+                    constexpr uint32_t idQ = idesc_bf16(64, DV, 0, 0);
+    #pragma unroll
+                    for (int kk = 0; kk < DK / 16; ++kk) {
+                        const uint32_t a = smem_u32(Kt + (kk >> 2) * 16384 + 8192 + (kk & 3) * 32);
+                        mma_bf16(tO, sdesc_sw128(a, 16, 1024), sdesc_sw128(stc + (kk >> 2) * (DV * 128) + (kk & 3) * 32, 16, 1024),
+                                 idQ, kk > 0);
+                    }
+                };
+                ctl.wait(B::tready + st, (c / NS) & 1);
+                if (tid == 0 && !ctl.aborted()) {
+                    // U^T = U~^T - S^T W^T, accumulated onto U~^T (A operand negated)
+                    tc_fence_after();
+                    constexpr uint32_t idN = idesc_bf16(DV, 64, 0, 1, 1);
+    #pragma unroll
+                    for (int kk = 0; kk < DK / 16; ++kk) {
+                        const uint64_t a = sdesc_sw128(stc + (kk >> 2) * (DV * 128) + (kk & 3) * 32, 16, 1024);
+                        mma_bf16(tmem + L::T_U + st * 64, a, sdesc_sw128(smem_u32(WTc + kk * 2048), 16, 1024), idN,
+                                 v_zero ? (kk > 0) : 1);
+                    }
+                    mma_commit(&bars[B::u]);
+                }
+                if (kChainScales) {
+                    // while the U MMA runs: gam Q and lam K in place for O1 and the state MMA (every
+                    // MMA that reads them unscaled, Gram and W, completed before the chunk was ready)
+                    const float *gv = gates(st);
+                    const int r = tid & 63;
+                    scale_row_bf16(Kt + (tid >> 6) * 16384 + 8192, r, gv[2 * CH + r], 0, 8);
+                    scale_row_bf16(Kt + (tid >> 6) * 16384, r, gv[3 * CH + r], 0, 8);
+                    fence_proxy_async_smem();
+                }
+                // O1 goes before the state MMA's commit, so that its completion also covers O1's reads
+                // of the Q tile (reloaded right after) and of the S_c copy.  One O buffer: the previous
+                // chunk's outputs leave first, while the U MMA runs.
+                if (NBO == 1 && c >= 1) out_epilogue(c - 1);
+                if (kChainScales) named_bar(1, 128);  // the scaled tiles are complete
+                if (tid == 0 && want_out && !ctl.aborted()) {
+                    tc_fence_after();
+                    issue_o1();
+                }
+                ctl.wait(B::u, c & 1);
+                tc_fence_after();
+                if (tid == 0) ctl.arrive(B::tfree + (c % NI));  // W^T of this chunk has been read
+                if (kHalf) {
+                    float x[32];
+                    tmem_ld16x2_32<32>(tl + L::T_U + st * 64, x);
+                    tmem_wait_ld();
+                    st_half_row_bf16_sw128(sm + L::UT, j, hh, x);
+                } else {
+                    float x[64];
+                    tmem_ld32(tl + L::T_U + st * 64, *reinterpret_cast<float(*)[32]>(&x[0]));
+                    tmem_ld32(tl + L::T_U + st * 64 + 32, *reinterpret_cast<float(*)[32]>(&x[32]));
+                    tmem_wait_ld();
+                    st_row_bf16_sw128(sm + L::UT, j, x);
+                }
+                fence_proxy_async_smem();
+                tc_fence_before();
+                named_bar(1, 128);
+                if (tid == 0 && !ctl.aborted()) {
+                    tc_fence_after();
+                    constexpr uint32_t idS = idesc_bf16(DV, DK, 0, 1);
+    #pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)  // S^T += U^T (lam K)
+                        mma_bf16(tmem + L::T_S, sdesc_sw128(smem_u32(sm + L::UT + kk * 32), 16, 1024),
+                                 sdesc_sw128(smem_u32(Kt + kk * 2048), 16384, 1024), idS, 1);
+                    mma_commit(&bars[B::s]);
+                    if (want_out) {
+                        constexpr uint32_t idP = idesc_bf16(64, DV, 0, 0);
+    #pragma unroll
+                        for (int kk = 0; kk < 4; ++kk)  // O += P U: A = P rows (K-major), B = U^T rows (K-major)
+                            mma_bf16(tO, sdesc_sw128(smem_u32(sm + L::PM + st * 8192 + kk * 32), 16, 1024),
+                                     sdesc_sw128(smem_u32(sm + L::UT + kk * 32), 16, 1024), idP, 1);
+                        mma_commit(&bars[B::o + c % NBO]);
+                    }
+                }
+                // two O buffers: the previous chunk's outputs leave while the state MMA runs
+                if (NBO == 2 && c >= 1) out_epilogue(c - 1);
+                ctl.wait(B::s, c & 1);
+                tc_fence_after();
+                if (warp == 0 && c + NS < nchunks) load_kq(c + NS);
+                {
+                    // S_{c+1} = gam_C(c) S_c + increment is in TMEM; keep a bf16 copy
+                    // and pre-scale the fp32 state by gam_C of the next chunk
+                    const bool more = c + 1 < nchunks;
+                    float gn = 1.f;
+                    if (more) {
+                        ctl.wait(B::gready + (c + 1) % NS, ((c + 1) / NS) & 1);
+                        gn = gates((c + 1) % NS)[6 * CH];
+                    }
+    #pragma unroll 1
+                    for (int k = 0; k < kSB; ++k) {
+                        float x[32];
+                        ld_state(k, x);
+                        tmem_wait_ld();
+                        store_state_bf16(s_block(k), x);
+                        if (more) {
+    #pragma unroll
+                            for (int i = 0; i < 32; ++i) x[i] *= gn;
+                            st_state(k, x);
+                        }
+                    }
+                    tmem_wait_st();
+                }
+                fence_proxy_async_smem();
+                tc_fence_before();
+                named_bar(1, 128);
+            }
+            if (nchunks > 0) out_epilogue(nchunks - 1);
         }
-        if (nchunks > 0) out_epilogue(nchunks - 1);
         // final state
         if (S_final) {
             if (nchunks > 0) {
