@@ -876,7 +876,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--quick", action="store_true", help="main workload only")
-    ap.add_argument("--only", choices=["hybrid_lm", "long_context", "varlen", "tiny", "decode", "hybrid_lm_fused",
+    ap.add_argument("--only", choices=["hybrid_lm", "long_context", "varlen", "varlen_profile", "tiny", "decode",
+                                       "hybrid_lm_fused",
                                              "hybrid_lm_unfused", "hybrid_lm_backward", "phase_memory",
                                              "hybrid_lm_dv256", "hybrid_lm_backward_dv128", "decode_fused",
                                              "hybrid_lm_backward_dk128", "phase_memory_rowdecay"],

@@ -877,15 +877,29 @@ __global__ void __launch_bounds__(TcCfg<DK, DV>::THREADS, 1)
                 if (!want_out) return;
                 const long tk = tok0 + (long)c * CH;
                 const int n = (int)min((long)CH, len - (long)c * CH);
-                {
-                    float o[64];
-                    tmem_ld32(tl + L::T_O + (c % NBO) * 64, *reinterpret_cast<float(*)[32]>(&o[0]));
-                    tmem_ld32(tl + L::T_O + (c % NBO) * 64 + 32, *reinterpret_cast<float(*)[32]>(&o[32]));
+                // per warp: its 32 lanes as two halves of 16, the 64 token columns as four groups
+                // of 16; a 16 x 16 block is loaded in fragments and stored transposed as four
+                // 8 x 8 bf16 matrices (rows = tokens), thread `lane` addressing row lane % 8 of
+                // matrix lane / 8
+                const int mi = lane >> 3, mrow = lane & 7;
+#pragma unroll
+                for (int hf = 0; hf < 2; ++hf) {
+                    uint32_t f[4][8];  // the four loads first, then one wait
+#pragma unroll
+                    for (int g = 0; g < 4; ++g)
+                        tmem_ld16x256b_x2(tmem + ((uint32_t)(warp * 32 + 16 * hf) << 16) + L::T_O + (c % NBO) * 64 + 16 * g,
+                                          f[g]);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int r = 0; r < CH; ++r)
-                        *reinterpret_cast<__nv_bfloat16 *>(buf + r * 256 + (((j >> 3) ^ (r & 15)) << 4) + (j & 7) * 2) =
-                            __float2bfloat16_rn(o[r]);
+                    for (int g = 0; g < 4; ++g) {
+                        const int r = 16 * g + 8 * (mi >> 1) + mrow;        // token row of this address
+                        const int col = warp * 32 + 16 * hf + 8 * (mi & 1);  // first value column
+                        stmatrix_x4_trans(smem_u32(buf + r * 256 + (((col >> 3) ^ (r & 15)) << 4)),
+                                          pack_bf16x2(__uint_as_float(f[g][0]), __uint_as_float(f[g][1])),
+                                          pack_bf16x2(__uint_as_float(f[g][2]), __uint_as_float(f[g][3])),
+                                          pack_bf16x2(__uint_as_float(f[g][4]), __uint_as_float(f[g][5])),
+                                          pack_bf16x2(__uint_as_float(f[g][6]), __uint_as_float(f[g][7])));
+                    }
                 }
                 named_bar(1, 128);
                 const int r = tid >> 1, hf = tid & 1;

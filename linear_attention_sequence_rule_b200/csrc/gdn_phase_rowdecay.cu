@@ -14,8 +14,8 @@
 // registers; per token two reductions over the LPC lanes (log2 LPC shuffles) and a rank-one
 // update.  A CTA takes CB channels of one (sequence, head): its threads stage the inputs of TT
 // tokens at a time in shared memory by cp.async (K and Q rows once for all the CTA's channels,
-// the channels' values and decays), double-buffered, so the scans read every input from shared
-// memory while the next tile is in flight.
+// the channels' values and decays, the decays turned into factors once per tile), double
+// buffered, so the scans read every input from shared memory while the next tile is in flight.
 #include <cuda_bf16.h>
 #include <math.h>
 
@@ -24,9 +24,9 @@
 namespace gdn {
 namespace {
 
-constexpr int LPC = 8;              // lanes per channel
+constexpr int LPC = 4;              // lanes per channel
 constexpr int CPW = 32 / LPC;       // channels per warp
-constexpr int WARPS = 8;
+constexpr int WARPS = 4;
 constexpr int CB = CPW * WARPS;     // channels per CTA
 constexpr int TT = 32;              // tokens per staged tile
 
@@ -156,6 +156,13 @@ __global__ void __launch_bounds__(32 * WARPS) rowdecay_scan(const float2 *__rest
         __syncthreads();
         Tile<DK> &tl = tiles[buf];
         const int nt = (int)min((long)TT, t1 - tb);
+        // the decay factors r = exp(log r), once per (token, channel) instead of in every lane
+        for (int c = tid; c < TT * CB; c += 32 * WARPS) {
+            float &x = (&tl.lr[0][0])[c];
+            x = expf(x);
+        }
+        __syncthreads();
+#pragma unroll 2
         for (int r = 0; r < nt; ++r) {
             const long t = tb + r;
             float2 k[E], q[E];
@@ -165,7 +172,7 @@ __global__ void __launch_bounds__(32 * WARPS) rowdecay_scan(const float2 *__rest
                 q[e] = tl.q[r][i + LPC * e];
             }
             const float v = tl.v[r][jl];
-            const float rr = expf(tl.lr[r][jl]), b = tl.b[r];
+            const float rr = tl.lr[r][jl], b = tl.b[r];
             // e = v - (1/dk) Re(m . conj k), Re(m conj k) = Re m Re k + Im m Im k
             float rd0 = 0.f, rd1 = 0.f;
 #pragma unroll

@@ -283,6 +283,26 @@ __device__ __forceinline__ void tmem_st16x2_32(uint32_t taddr, const float (&v)[
         : "memory");
 }
 
+// Shape 16x256b, two repetitions: 16 lanes x 16 columns.  Thread t receives, for k = 0, 1 (the
+// two 8-column halves): r[4k] = (lane t/4, column 8k + 2(t%4)), r[4k+1] = (lane t/4, column
+// 8k + 2(t%4) + 1), r[4k+2] and r[4k+3] the same columns of lane 8 + t/4 -- the fragment layout
+// of the warp-level MMAs and of stmatrix.
+__device__ __forceinline__ void tmem_ld16x256b_x2(uint32_t taddr, uint32_t (&r)[8])
+{
+    asm volatile("tcgen05.ld.sync.aligned.16x256b.x2.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+                 : "r"(taddr));
+}
+
+// Four 8 x 8 bf16 matrices from fragments to shared memory, each transposed on the way: thread t
+// gives the address of row t % 8 of matrix t / 8 (a 16-byte row), a_i its fragment of matrix i.
+__device__ __forceinline__ void stmatrix_x4_trans(uint32_t saddr, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3)
+{
+    asm volatile("stmatrix.sync.aligned.m8n8.x4.trans.shared.b16 [%0], {%1, %2, %3, %4};" ::"r"(saddr), "r"(a0),
+                 "r"(a1), "r"(a2), "r"(a3)
+                 : "memory");
+}
+
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 

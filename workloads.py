@@ -38,6 +38,10 @@ CONFIGS = {
     "varlen": dict(kind="chunk", n_seqs=32, len_lo=128, len_hi=8192, H=16, dk=128, dv=128,
                    chunk=64, dtype="bf16", beta_scale=2.0, la_std=2.0, la_scale=1.0,
                    s0_std=0.0, seed=1004),
+    # a smaller pack of the varlen workload's kind (for profiler captures of a few GB at most)
+    "varlen_profile": dict(kind="chunk", n_seqs=32, len_lo=128, len_hi=2048, H=16, dk=128, dv=128,
+                           chunk=64, dtype="bf16", beta_scale=2.0, la_std=2.0, la_scale=1.0,
+                           s0_std=0.0, seed=1006),
     "decode": dict(kind="decode", N=256, H=32, dk=128, dv=128, steps=1000, dtype="bf16",
                    beta_scale=1.0, la_std=1.0, la_scale=0.1, s0_std=0.02, seed=1005),
 }
