@@ -33,7 +33,8 @@
 // their (finite) K/Q/V contents contribute nothing.
 //
 // Every mbarrier wait is bounded (2 s).  On timeout the kernel records an error word, stops
-// issuing work and skips all later waits, so it always reaches the end, frees TMEM and returns.
+// issuing work and skips all later waits; at the end each MMA-issuing thread waits (bounded) for
+// the MMAs it had issued before TMEM is freed.  The call's outputs are then undefined.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_bf16.h>
@@ -117,7 +118,7 @@ struct TcCfg {
     static constexpr int GT = OT + OT_BYTES;                     // per stage: gate vectors
     static constexpr int GT_STAGE = 7 * CH * 4;                  //   graw, G2, gam, lam, bet, last, (gC)
     static constexpr int BAR = GT + NS * GT_STAGE;
-    static constexpr int NBAR = 5 * NS + NB + NBO + 2 + 4 * NI;
+    static constexpr int NBAR = 5 * NS + NB + NBO + 2 + 4 * NI + 1 + NI;
     static constexpr int MISC = BAR + NBAR * 8;                  // TMEM slot, abort flag
     static constexpr int TOTAL = MISC + 16;
     // TMEM columns
@@ -145,6 +146,7 @@ template <int NS, int NI, int NB, int NBO> struct Bars {
     static constexpr int uw = gram + NI;               // [NI] WY MMAs done
     static constexpr int tfree = uw + NI;              // [NI] chain -> intra: the U MMA has read W^T
     static constexpr int ufree = tfree + NI;           // [NI] chain -> intra: the U slot has been read (TA)
+    static constexpr int drain = ufree + NI;           // [1 + NI] after a timeout: the MMAs of each issuer done
 };
 
 // Thread roles inside an intra warpgroup (t = 0..127): the gate scan runs on warp scan_warp(wg)
@@ -1208,6 +1210,16 @@ __global__ void __launch_bounds__(TcCfg<DK, DV>::THREADS, 1)
                     S_final[sbase + (size_t)c2 * ldv + j] =
                         (flags & kFlagS0Identity) ? (c2 == j ? 1.f : 0.f) : (S0 ? S0[sbase + (size_t)c2 * ldv + j] : 0.f);
             }
+        }
+    }
+    // After a wait ran out, MMAs already issued may still be running: each issuing thread (the
+    // chain's thread 0 and each intra warpgroup's issuer) commits once more and waits, bounded,
+    // for its MMAs to complete before the tensor memory is freed.
+    if (ctl.aborted()) {
+        const int who = tid == 0 ? 0 : (tid >= 128 && (tid - 128) % 128 == kIssuer ? 1 + (tid - 128) / 128 : -1);
+        if (who >= 0) {
+            mma_commit(&bars[B::drain + who]);
+            mbar_wait_bounded(&bars[B::drain + who], 0, 100000000ull);
         }
     }
     tc_fence_before();
