@@ -904,12 +904,19 @@ __global__ void __launch_bounds__(TcCfg<DK, DV>::THREADS, 1)
                     }
                 }
                 named_bar(1, 128);
-                const int r = tid >> 1, hf = tid & 1;
-                if (r < n) {
-                    uint4 *dst = reinterpret_cast<uint4 *>(out + ((size_t)(tk + r) * H + h) * ldv + col0 + 64 * hf);
+                // rows to global memory: eight threads per 256-byte row, each taking 16-byte units
+                // (tid & 7) and (tid & 7) + 8, so a warp stores four rows with full 128-byte runs
 #pragma unroll
-                    for (int i = 0; i < 8; ++i)
-                        dst[i] = *reinterpret_cast<const uint4 *>(buf + r * 256 + (((8 * hf + i) ^ (r & 15)) << 4));
+                for (int p = 0; p < 4; ++p) {
+                    const int r = 16 * p + (tid >> 3);
+                    if (r < n) {
+                        uint4 *dst = reinterpret_cast<uint4 *>(out + ((size_t)(tk + r) * H + h) * ldv + col0);
+#pragma unroll
+                        for (int s8 = 0; s8 < 2; ++s8) {
+                            const int u = (tid & 7) + 8 * s8;
+                            dst[u] = *reinterpret_cast<const uint4 *>(buf + r * 256 + ((u ^ (r & 15)) << 4));
+                        }
+                    }
                 }
             };
             if (nchunks > 0) {
