@@ -105,3 +105,40 @@ def test_chunk_invariance_on_the_gpu():
     o1, s1 = run(inp, 64)
     o2, s2 = run(inp, 128)
     assert float((o1 - o2).abs().max()) <= 1e-4 and float((s1 - s2).abs().max()) <= 1e-4
+
+
+@pytest.mark.parametrize("dk,chunk,lengths", [(256, 64, None), (128, 128, [0, 1, 130, 300, 64, 7])])
+def test_host_entry_on_the_general_path(dk, chunk, lengths):
+    # host buffers in and out, the batch cut into parts: each part runs the general path with the
+    # same per-sequence arithmetic as the device entry, so the results are bit-identical
+    import linear_attention_sequence_rule_b200 as gdn
+    if lengths is None:
+        inp = workloads.make_chunk_inputs(B=3, T=200, H=2, dk=dk, dv=128, dtype="bf16", seed=90, s0_std=0.05)
+    else:
+        inp = workloads.make_chunk_inputs(H=2, dk=dk, dv=128, dtype="bf16", seed=91, s0_std=0.05, lengths=lengths)
+    host = {k: (v.contiguous().pin_memory() if torch.is_tensor(v) else v) for k, v in inp.items()}
+    out_h, sf_h = gdn.chunk_fwd_host(host["q"], host["k"], host["v"], host["log_alpha"], host["beta"], S0=host["S0"],
+                                     cu_seqlens=host["cu_seqlens"], chunk=chunk)
+    torch.cuda.synchronize()
+    out_d, sf_d = run(inp, chunk)
+    assert torch.equal(out_h, out_d.cpu()) and torch.equal(sf_h, sf_d.cpu())
+
+
+def test_noalloc_entry_on_the_general_path():
+    # the general path's factors fit the fixed scratch array at these sizes; results bit-identical
+    import ctypes
+    import linear_attention_sequence_rule_b200 as gdn
+    inp = workloads.make_chunk_inputs(B=2, T=150, H=2, dk=256, dv=64, dtype="bf16", seed=92, s0_std=0.05)
+    d = {k: (v.cuda() if torch.is_tensor(v) else v) for k, v in inp.items()}
+    p = lambda t: None if t is None else ctypes.c_void_p(t.data_ptr())
+    need = gdn.gdn_chunk_fwd_workspace_bytes(2, 150, 2, 256, 64, 64, 0, gdn.GDN_DTYPE_BF16)
+    assert 0 < need <= 32 * 2 ** 20
+    out = torch.empty_like(d["v"])
+    Sf = torch.empty(2, 2, 256, 64, device="cuda")
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    rc = gdn.gdn_chunk_fwd_noalloc(p(d["q"]), p(d["k"]), p(d["v"]), p(d["log_alpha"]), p(d["beta"]), p(d["S0"]),
+                                   p(out), p(Sf), 2, 150, 2, 256, 64, 64, None, gdn.GDN_DTYPE_BF16, stream)
+    assert rc == gdn.GDN_OK, gdn.gdn_last_error()
+    assert gdn.gdn_device_status(stream) == gdn.GDN_OK
+    out_d, sf_d = run(inp, 64)
+    assert torch.equal(out, out_d) and torch.equal(Sf, sf_d)
