@@ -241,9 +241,11 @@ GDN_API size_t gdn_phase_fwd_workspace_bytes(int B, int T, int H, int dk, int dv
  *     o_t,j = (1/dk) Re(M_t[j] . conj Q_t)
  * Layouts as gdn_phase_fwd, with log_r [.., H, dv] fp32 (one decay per token, head and channel,
  * finite) in place of log_lam.  dk in {32, 64} complex, any dv in 1 .. 4096, B and H up to 65535,
- * dtype bf16 or fp32 for v and out (the arithmetic is fp32).  No workspace.  The channels are
- * independent scans (gdn_phase_rowdecay.cu).  Errors as gdn_chunk_fwd; M0 == M_final (in-place
- * carry) is allowed.
+ * dtype bf16 or fp32 for v and out (fp32-level arithmetic: the products shared by the channels
+ * run on the tensor cores as three tf32 products of hi / lo splits, about 2^-21 relative).  No
+ * workspace.  It runs in chunks of 32 tokens (gdn_phase_rowdecay.cu).  Errors as gdn_chunk_fwd; a
+ * device-side wait that runs out is reported by gdn_device_status; M0 == M_final (in-place carry)
+ * is allowed.
  */
 GDN_API int gdn_phase_rowdecay_fwd(const float *K, const float *Q, const void *v, const float *log_r,
                                    const float *beta, const float *M0, void *out, float *M_final, int B, int T,

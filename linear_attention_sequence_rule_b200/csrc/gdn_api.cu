@@ -316,8 +316,9 @@ int gdn_device_status(void *stream)
     g_last_error[0] = 0;
     cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "gdn_device_status");
-    const int v = read_and_clear_tc_error();
-    if (v < 0) return fail(GDN_ERR_CUDA, "gdn_device_status: reading the device record failed");
+    const int v1 = read_and_clear_tc_error(), v2 = read_and_clear_rowdecay_error();
+    if (v1 < 0 || v2 < 0) return fail(GDN_ERR_CUDA, "gdn_device_status: reading the device record failed");
+    const int v = v1 | v2;
     if (v) return fail(GDN_ERR_TIMEOUT, "a device-side wait ran out (record 0x%x)", v);
     return GDN_OK;
 }

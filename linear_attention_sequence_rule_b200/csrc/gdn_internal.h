@@ -81,5 +81,7 @@ cudaError_t launch_phase_rowdecay(const float *K, const float *Q, const void *V,
                                   const float *beta, const float *M0, void *out, float *M_final,
                                   const int32_t *cu_seqlens, int nseq, int T, int H, int dk, int dv, int bf16,
                                   cudaStream_t stream);
+// The row-decay kernel's device error record (bounded MMA waits that ran out), read and cleared.
+int read_and_clear_rowdecay_error();
 
 }  // namespace gdn
