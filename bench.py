@@ -705,7 +705,7 @@ def phase_numbers(gdn, steps, warmup, flush, stream, peaks):
     return {"workload": "complex-phase delta memory, hybrid_lm shape: B=8 T=4096 H=12, "
                         "dk=32 complex (64 real), dv=64, bf16 values, fp32 phasors",
             "ms": round(ms_p, 6), "tokens_per_s": round(32768 / (ms_p * 1e-3), 1),
-            "launches_per_call": 3, "algo_bytes": by_p,
+            "launches_per_call": 2, "algo_bytes": by_p,
             "gbs": round(by_p / (ms_p * 1e-3) / 1e9, 3),
             "hbm_frac": round(by_p / (ms_p * 1e-3) / 1e9 / peaks["hbm_gbs"], 5)}
 

@@ -218,8 +218,9 @@ GDN_API size_t gdn_chunk_fwd_host_workspace_bytes(int B, int T, int H, int dk, i
  *     K, Q [.., H, dk, 2] fp32 (re, im pairs); v, out [.., H, dv] in dtype;
  *     log_lam, beta [.., H] fp32; M0, M_final [B, H, dv, dk, 2] fp32 (re, im), either may be NULL.
  * log_lam must be finite (lam > 0): the computation runs the real gated delta rule at head size
- * 2 dk with a = lam and b = beta / lam (see gdn_phase.cu), on the tcgen05 kernel for bf16 and
- * the fp32 CUDA-core kernel for fp32.  dk in {32, 64}, dv in {64, 128}, or 256 with bf16.  Workspace:
+ * 2 dk with a = lam and b = beta / lam (see gdn_phase.cu), on the tcgen05 kernel for bf16 (at
+ * dk = 32, dv = 64 with the conversion of K, Q, beta and V inside it) and the fp32 CUDA-core
+ * kernel for fp32.  dk in {32, 64}, dv in {64, 128}, or 256 with bf16.  Workspace:
  * gdn_phase_fwd_workspace_bytes(...) bytes of device memory, 256-byte aligned.  Errors as
  * gdn_chunk_fwd (the library's own scratch only is written before a late CUDA error).
  */

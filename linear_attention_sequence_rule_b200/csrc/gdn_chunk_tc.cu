@@ -68,12 +68,20 @@ constexpr float kNormEps = 1e-6f;
 // of rank z by length (ties by index), so that the longest chains, which set the launch's length,
 // start in the first wave instead of wherever the packing put them.
 constexpr int kFlagLongestFirst = 8;
+// Complex-phase memory with its prologue fused (dk = 32 complex, the real recurrence at head size
+// 64): K and Q arrive as fp32 (re, im) pairs and are scaled (1 / sqrt(dk), 1 / dk), real parts
+// first, into the bf16 tiles in shared memory; beta arrives raw, b = beta / lam is formed in the
+// gate scan, and V enters unscaled with lam sqrt(dk) folded into T diag(.) of the U~ product
+// (b v = beta sqrt(dk) V); see gdn_phase.cu for the algebra.
+constexpr int kFlagPhase = 16;
+constexpr float kPhaseSqrtDk = 5.656854249492381f;  // sqrt(32)
 #ifndef GDN_U_SPLIT
 #define GDN_U_SPLIT 1
 #endif
 
-template <int DK, int DV>
+template <int DK, int DV, bool PH = false>
 struct TcCfg {
+    static_assert(!PH || (DK == 64 && DV == 64), "the fused phase prologue is built for dk = 32 complex, dv = 64");
     // Two intra warpgroups take alternate chunks.
     static constexpr int NI = 2;
     static constexpr int THREADS = 128 * (1 + NI);
@@ -90,10 +98,13 @@ struct TcCfg {
     static constexpr int SB_COLS = TA ? DK / 2 : 0;  // bf16 S^T, two per column (TA)
     static constexpr int NBO = (2 * O_COLS + DK + SB_COLS + NI * 64 + NU * 64 <= 512) ? 2 : 1;
     // V buffers (two: the V load of a chunk starts two chunks ahead)
-    static constexpr int NB = TA ? (DK == 64 ? 2 : 1) : NBO;
+    // (one with the fused phase prologue, whose K/Q stages are twice as large)
+    static constexpr int NB = PH ? 1 : (TA ? (DK == 64 ? 2 : 1) : NBO);
     // shared memory byte offsets (swizzled tiles first, all 1024-aligned)
     static constexpr int KQ = 0;                                 // per stage: per 64-feature block K (8K) | Q (8K)
-    static constexpr int KQ_STAGE = (DK / 64) * 16384;
+    // PH: a stage first holds the fp32 K and Q rows (two 32-float blocks each), which the intra
+    // warpgroup turns into the bf16 tiles in place
+    static constexpr int KQ_STAGE = (DK / 64) * 16384 * (PH ? 2 : 1);
     static constexpr int V = KQ + NS * KQ_STAGE;                 // per buffer: per 64-column block 8 KB
     static constexpr int V_BUF = (DV / 64) * 8192;
     static constexpr int PM = V + NB * V_BUF;                    // per stage: P bf16, 64 x 128 B
@@ -116,7 +127,7 @@ struct TcCfg {
     static constexpr int OT = WG0 + NI * WG_BYTES;
     static constexpr int OT_BYTES = (TA && NBO == 2) ? CH * DV * 2 : 0;
     static constexpr int GT = OT + OT_BYTES;                     // per stage: gate vectors
-    static constexpr int GT_STAGE = 7 * CH * 4;                  //   graw, G2, gam, lam, bet, last, (gC)
+    static constexpr int GT_STAGE = (PH ? 8 : 7) * CH * 4;       //   graw, G2, gam, lam, bet, last, (gC), (PH: bv)
     static constexpr int BAR = GT + NS * GT_STAGE;
     static constexpr int NBAR = 5 * NS + NB + NBO + 2 + 4 * NI + 1 + NI;
     static constexpr int MISC = BAR + NBAR * 8;                  // TMEM slot, abort flag
@@ -191,21 +202,25 @@ struct TOut {
     float *Tm;
     unsigned char *TB, *TG;
     const float *bet, *gam;
-    // (bc, gc) = bet/gam of column c, loaded once by the caller
-    __device__ __forceinline__ void put(int r, int c, float v, float bc, float gc) const
+    // the column factors of T diag(.) for the U~ product: bet, or (fused phase prologue) the
+    // per-token factor that also carries the scale of V
+    const float *bv;
+    __device__ __forceinline__ float vfac(int c, float bc) const { return bv ? bv[c] : bc; }
+    // (vc, bc, gc) = factors of column c, loaded once by the caller
+    __device__ __forceinline__ void put(int r, int c, float v, float vc, float bc, float gc) const
     {
         Tm[r * LDF + c] = v;
         const float b = v * bc;
-        *reinterpret_cast<__nv_bfloat16 *>(TB + sw128_off(r, c)) = __float2bfloat16_rn(b);
+        *reinterpret_cast<__nv_bfloat16 *>(TB + sw128_off(r, c)) = __float2bfloat16_rn(v * vc);
         *reinterpret_cast<__nv_bfloat16 *>(TG + sw128_off(r, c)) = __float2bfloat16_rn(b * gc);
     }
-    // c even; (b0, b1, g0, g1) = bet/gam of columns c, c+1; keep: also store the fp32 values
-    __device__ __forceinline__ void put2(int r, int c, float v0, float v1, float b0, float b1, float g0, float g1,
-                                         bool keep) const
+    // c even; (u0, u1, b0, b1, g0, g1) = factors of columns c, c+1; keep: also store the fp32 values
+    __device__ __forceinline__ void put2(int r, int c, float v0, float v1, float u0, float u1, float b0, float b1,
+                                         float g0, float g1, bool keep) const
     {
         if (keep) *reinterpret_cast<float2 *>(&Tm[r * LDF + c]) = make_float2(v0, v1);
         const float x0 = v0 * b0, x1 = v1 * b1;
-        *reinterpret_cast<uint32_t *>(TB + sw128_off(r, c)) = pack_bf16x2(x0, x1);
+        *reinterpret_cast<uint32_t *>(TB + sw128_off(r, c)) = pack_bf16x2(v0 * u0, v1 * u1);
         *reinterpret_cast<uint32_t *>(TG + sw128_off(r, c)) = pack_bf16x2(x0 * g0, x1 * g1);
     }
 };
@@ -233,7 +248,7 @@ __device__ void solve_unit_lower(const float *A, const TOut &out, float *__restr
         const int o = 16 * w;
         if (lane < 16) {
             const int sb = o + 8 * (lane >> 3), c = lane & 7;
-            const float bc = out.bet[sb + c], gc = out.gam[sb + c];
+            const float bc = out.bet[sb + c], gc = out.gam[sb + c], vc = out.vfac(sb + c, bc);
             float a[8][8];  // the block's strictly lower part, read before any lane writes T there
 #pragma unroll
             for (int r = 1; r < 8; ++r)
@@ -251,7 +266,7 @@ __device__ void solve_unit_lower(const float *A, const TOut &out, float *__restr
             __syncwarp(0xffffu);
 #pragma unroll
             for (int r = 0; r < 8; ++r)
-                if (r >= c) out.put(sb + r, sb + c, x[r], bc, gc);
+                if (r >= c) out.put(sb + r, sb + c, x[r], vc, bc, gc);
         }
         __syncwarp();
 #pragma unroll
@@ -264,7 +279,7 @@ __device__ void solve_unit_lower(const float *A, const TOut &out, float *__restr
             xs[i * 8 + j] = acc;
         }
         __syncwarp();
-        const float bj = out.bet[o + (lane & 7)], gj = out.gam[o + (lane & 7)];
+        const float bj = out.bet[o + (lane & 7)], gj = out.gam[o + (lane & 7)], vj = out.vfac(o + (lane & 7), bj);
 #pragma unroll
         for (int q0 = 0; q0 < 64; q0 += 32) {
             const int q = q0 + lane, i = q >> 3, j = q & 7;
@@ -272,7 +287,7 @@ __device__ void solve_unit_lower(const float *A, const TOut &out, float *__restr
 #pragma unroll
             for (int k = 0; k < 8; ++k)
                 if (k < i) acc = fmaf(Tm[(o + 8 + i) * LDF + o + 8 + k], xs[k * 8 + j], acc);
-            out.put(o + 8 + i, o + j, -acc, bj, gj);
+            out.put(o + 8 + i, o + j, -acc, vj, bj, gj);
         }
     }
     named_bar(bar_id, 128);
@@ -306,8 +321,9 @@ __device__ void solve_unit_lower(const float *A, const TOut &out, float *__restr
         }
         const int c0 = oa + 8 * nt + 2 * tq;
         const float b0 = out.bet[c0], b1 = out.bet[c0 + 1], g0 = out.gam[c0], g1 = out.gam[c0 + 1];
-        out.put2(ob + g, c0, -e[0], -e[1], b0, b1, g0, g1, true);
-        out.put2(ob + g + 8, c0, -e[2], -e[3], b0, b1, g0, g1, true);
+        const float u0 = out.vfac(c0, b0), u1 = out.vfac(c0 + 1, b1);
+        out.put2(ob + g, c0, -e[0], -e[1], u0, u1, b0, b1, g0, g1, true);
+        out.put2(ob + g + 8, c0, -e[2], -e[3], u0, u1, b0, b1, g0, g1, true);
     }
     named_bar(bar_id, 128);
     // ---- 32 -> 64: warp w takes output column tile wt = 3 - w ----
@@ -338,6 +354,7 @@ __device__ void solve_unit_lower(const float *A, const TOut &out, float *__restr
         __syncwarp();
         const int c0 = 8 * wt + 2 * tq;
         const float bb0 = out.bet[c0], bb1 = out.bet[c0 + 1], gg0 = out.gam[c0], gg1 = out.gam[c0 + 1];
+        const float uu0 = out.vfac(c0, bb0), uu1 = out.vfac(c0 + 1, bb1);
 #pragma unroll
         for (int mt = 0; mt < 2; ++mt) {
             float e[4] = {0.f, 0.f, 0.f, 0.f};
@@ -352,8 +369,8 @@ __device__ void solve_unit_lower(const float *A, const TOut &out, float *__restr
                          tf(k1 <= rh ? Tm[(32 + rh) * LDF + 32 + k1] : 0.f),
                          tf(xs[k0 * 8 + g]), tf(xs[k1 * 8 + g]));
             }
-            out.put2(32 + rl, c0, -e[0], -e[1], bb0, bb1, gg0, gg1, false);
-            out.put2(32 + rh, c0, -e[2], -e[3], bb0, bb1, gg0, gg1, false);
+            out.put2(32 + rl, c0, -e[0], -e[1], uu0, uu1, bb0, bb1, gg0, gg1, false);
+            out.put2(32 + rh, c0, -e[2], -e[3], uu0, uu1, bb0, bb1, gg0, gg1, false);
         }
     }
 }
@@ -423,10 +440,10 @@ __device__ __forceinline__ void scale_row_bf16(unsigned char *tile, int row, flo
     }
 }
 
-// PRO: fused prologue (kFlagPrologue), a separate instantiation so that the plain path carries
-// none of its code.
-template <int DK, int DV, bool PRO>
-__global__ void __launch_bounds__(TcCfg<DK, DV>::THREADS, 1)
+// PRO: fused prologue (kFlagPrologue), PH: fused complex-phase prologue (kFlagPhase), separate
+// instantiations so that the plain path carries none of their code.
+template <int DK, int DV, bool PRO, bool PH = false>
+__global__ void __launch_bounds__(TcCfg<DK, DV, PH>::THREADS, 1)
     chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const float *__restrict__ log_alpha,
                     const float *__restrict__ beta, const float *__restrict__ S0,
@@ -434,7 +451,7 @@ __global__ void __launch_bounds__(TcCfg<DK, DV>::THREADS, 1)
                     const int32_t *__restrict__ cu_seqlens, int T, int H, int flags, float a_scale,
                     float b_scale, int G)
 {
-    using L = TcCfg<DK, DV>;
+    using L = TcCfg<DK, DV, PH>;
     constexpr int NS = L::NS;
     constexpr int NI = L::NI;
     constexpr int NB = L::NB;
@@ -519,11 +536,19 @@ __global__ void __launch_bounds__(TcCfg<DK, DV>::THREADS, 1)
         }
         cp_async_mbar_arrive(&bars[B::gfull + st]);
         if (lane == 0 && !ctl.aborted()) {
-            mbar_arrive_expect_tx(&bars[B::kq_full + st], (DK / 64) * 16384);
+            mbar_arrive_expect_tx(&bars[B::kq_full + st], L::KQ_STAGE);
             unsigned char *kq = sm + L::KQ + st * L::KQ_STAGE;
-            for (int kb = 0; kb < DK / 64; ++kb) {
-                tma_load_3d(kq + kb * 16384, &tmK, &bars[B::kq_full + st], kb * 64, hq, (int)tk);
-                tma_load_3d(kq + kb * 16384 + 8192, &tmQ, &bars[B::kq_full + st], kb * 64, hq, (int)tk);
+            if constexpr (PH) {
+                // fp32 rows of 64 (32 complex pairs) as two 32-float blocks: K at +0, Q at +16 KB
+                for (int hb = 0; hb < 2; ++hb) {
+                    tma_load_3d(kq + hb * 8192, &tmK, &bars[B::kq_full + st], hb * 32, hq, (int)tk);
+                    tma_load_3d(kq + 16384 + hb * 8192, &tmQ, &bars[B::kq_full + st], hb * 32, hq, (int)tk);
+                }
+            } else {
+                for (int kb = 0; kb < DK / 64; ++kb) {
+                    tma_load_3d(kq + kb * 16384, &tmK, &bars[B::kq_full + st], kb * 64, hq, (int)tk);
+                    tma_load_3d(kq + kb * 16384 + 8192, &tmQ, &bars[B::kq_full + st], kb * 64, hq, (int)tk);
+                }
             }
         }
     };
@@ -574,6 +599,32 @@ __global__ void __launch_bounds__(TcCfg<DK, DV>::THREADS, 1)
             // ---- Gram matrices [K; Q] K^T (issued first: they need no gates, so the scan below
             //      runs while they are in flight) ----
             ctl.wait(B::kq_full + st, (c / NS) & 1);
+            if (PH) {
+                // fp32 (re, im) rows -> bf16 rows of k~ / sqrt(dk) (threads 0-63) and q~ / dk
+                // (threads 64-127), real parts in columns 0-31 and imaginary parts in 32-63,
+                // written over the fp32 rows once all of them have been read
+                const int r = t & 63;
+                const bool isq = t >= 64;
+                const unsigned char *src = Kt + (isq ? 16384 : 0);
+                const float sc = isq ? 1.f / 32.f : 1.f / kPhaseSqrtDk;
+                float x[64];
+#pragma unroll
+                for (int hb = 0; hb < 2; ++hb)
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) {
+                        const float4 f = *reinterpret_cast<const float4 *>(src + hb * 8192 + r * 128 +
+                                                                            (((u ^ r) & 7) << 4));
+                        const int i = 16 * hb + 2 * u;  // complex index of f.x, f.y
+                        x[i] = f.x * sc;
+                        x[32 + i] = f.y * sc;
+                        x[i + 1] = f.z * sc;
+                        x[33 + i] = f.w * sc;
+                    }
+                named_bar(bar_id, 128);
+                st_row_bf16_sw128(Kt + (isq ? 8192 : 0), r, x);
+                fence_proxy_async_smem();
+                named_bar(bar_id, 128);
+            }
             if (PRO) {
                 // fused prologue: unit rows of K (threads 0-63) and Q (threads 64-127)
                 normalize_row_bf16<DK / 64>(Kt + (t >= 64 ? 8192 : 0), t & 63);
@@ -601,6 +652,15 @@ __global__ void __launch_bounds__(TcCfg<DK, DV>::THREADS, 1)
                     g1 = prologue_log_alpha(g1, r1 < n, a_scale);
                     bet[r0] = prologue_beta(bet[r0], r0 < n, b_scale);
                     bet[r1] = prologue_beta(bet[r1], r1 < n, b_scale);
+                }
+                if (PH) {
+                    // U~ factor beta sqrt(dk) (= b v / V), then b = beta / lam (lam > 0; padded rows
+                    // hold beta = 0 and log lam = 0)
+                    float *bv = gv + 7 * CH;
+                    bv[r0] = bet[r0] * kPhaseSqrtDk;
+                    bv[r1] = bet[r1] * kPhaseSqrtDk;
+                    bet[r0] *= expf(-g0);
+                    bet[r1] *= expf(-g1);
                 }
                 const bool f0 = (g0 == -INFINITY), f1 = (g1 == -INFINITY);
                 const float v0 = f0 ? 0.f : g0, v1 = f1 ? 0.f : g1;
@@ -720,7 +780,7 @@ __global__ void __launch_bounds__(TcCfg<DK, DV>::THREADS, 1)
             }
             named_bar(bar_id, 128);
             // ---- T = (I + A)^{-1}, written with the bf16 rows of T diag(b), T diag(b gam) ----
-            solve_unit_lower(AT, TOut{AT, TBs, TGs, bet, gam}, XSm, t, bar_id);
+            solve_unit_lower(AT, TOut{AT, TBs, TGs, bet, gam, PH ? gv + 7 * CH : nullptr}, XSm, t, bar_id);
             fence_proxy_async_smem();
             tc_fence_before();
             named_bar(bar_id, 128);
@@ -1269,6 +1329,22 @@ bool make_map(CUtensorMap *m, const void *base, long tokens, int H, int d)
     return r == CUDA_SUCCESS;
 }
 
+// 3-D view [tokens][H][d] of an fp32 tensor (the phase memory's (re, im) pairs, d = 2 dk); box =
+// 32 floats (128 bytes, the swizzle span) x 1 head x 64 tokens, 128-byte swizzle.
+bool make_map_f32(CUtensorMap *m, const void *base, long tokens, int H, int d)
+{
+    auto enc = get_encode_fn();
+    if (!enc) return false;
+    cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)tokens};
+    cuuint64_t strides[2] = {(cuuint64_t)d * 4, (cuuint64_t)H * d * 4};
+    cuuint32_t box[3] = {32, 1, 64};
+    cuuint32_t es[3] = {1, 1, 1};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void *>(base), dims, strides, box, es,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 // One launch of the chunk kernel over `nseq` sequences given either densely (cu == nullptr:
 // sequence s owns tokens s*T .. s*T+T-1) or by offsets cu[0..nseq].
 struct TcLaunch {
@@ -1297,13 +1373,26 @@ cudaError_t launch_tc(const TcLaunch &a, cudaStream_t st)
     const void *vsrc = (a.flags & kFlagVZero) ? a.k : a.v;
     const int vdim = (a.flags & kFlagVZero) ? DK : DV * a.vblocks;
     const int vheads = (a.flags & kFlagVZero) ? a.H / a.G : a.H;
-    if (!make_map(&mq, a.q, map_tokens, a.H / a.G, DK) || !make_map(&mk, a.k, map_tokens, a.H / a.G, DK) ||
-        !make_map(&mv, vsrc, map_tokens, vheads, vdim)) {
+    const bool ph = (a.flags & kFlagPhase) != 0;
+    const bool qk_ok = ph ? make_map_f32(&mq, a.q, map_tokens, a.H / a.G, DK) &&
+                                make_map_f32(&mk, a.k, map_tokens, a.H / a.G, DK)
+                          : make_map(&mq, a.q, map_tokens, a.H / a.G, DK) &&
+                                make_map(&mk, a.k, map_tokens, a.H / a.G, DK);
+    if (!qk_ok || !make_map(&mv, vsrc, map_tokens, vheads, vdim)) {
         set_error("cuTensorMapEncodeTiled failed");
         return cudaErrorInvalidValue;
     }
-    const int smem = L::TOTAL + 1024;
+    int smem = L::TOTAL + 1024;
     auto kern = (a.flags & kFlagPrologue) ? chunk_tc_kernel<DK, DV, true> : chunk_tc_kernel<DK, DV, false>;
+    if constexpr (DK == 64 && DV == 64) {
+        if (ph) {
+            kern = chunk_tc_kernel<DK, DV, false, true>;
+            smem = TcCfg<DK, DV, true>::TOTAL + 1024;
+        }
+    } else if (ph) {
+        set_error("the fused phase prologue runs at head size 64, value head 64 only");
+        return cudaErrorInvalidValue;
+    }
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     const dim3 grid(a.vblocks, a.H, a.nseq);
@@ -1509,6 +1598,21 @@ size_t chunk_tc_workspace_bytes(int B, int T, int H, int dk, int dv, int varlen,
     const SegPlan p = plan_segments(B, T, H * (dv > 128 ? dv / 128 : 1), varlen, dtype);
     if (p.G <= 1) return 0;
     return seg_layout(nullptr, B, H, dk, dv, p).bytes;
+}
+
+bool phase_fused_ok(int B, int T, int H, int varlen)
+{
+    return plan_segments(B, T, H, varlen, GDN_DTYPE_BF16).G <= 1;
+}
+
+cudaError_t launch_phase_chunk(const float *K, const float *Q, const void *V, const float *log_lam,
+                               const float *beta, const float *S0, void *out, float *S_final, const int32_t *cu,
+                               int B, int T, int H, cudaStream_t stream)
+{
+    const long tokens = cu ? (long)T : (long)B * T;
+    const int lf = (cu && B <= TcCfg<64, 64>::THREADS) ? kFlagLongestFirst : 0;
+    TcLaunch t{Q, K, V, log_lam, beta, S0, out, S_final, cu, B, T, H, tokens, kFlagPhase | lf, 0.f, 0.f, 1};
+    return launch_tc<64, 64>(t, stream);
 }
 
 cudaError_t launch_chunk_tc(const ChunkArgs &a, cudaStream_t stream)

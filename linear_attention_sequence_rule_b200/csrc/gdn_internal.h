@@ -77,6 +77,15 @@ cudaError_t launch_chunk_bwd(const BwdArgs &a, cudaStream_t stream);
 
 // Complex-phase memory with one decay per value channel (gdn_phase_rowdecay.cu): K, Q, M0,
 // M_final as (re, im) fp32 pairs; V and out bf16 (bf16 != 0) or fp32.
+// The complex-phase memory at dk = 32 complex, dv = 64 with its prologue in the chunk kernel: K, Q
+// fp32 (re, im) pairs [tokens, H, 32, 2], V bf16, raw log_lam and beta; S0 / S_final the real
+// state [B, H, 64, 64] ([Re | Im] rows).  phase_fused_ok: the sizes run as one launch (no
+// segment scan), which the fused form requires.
+bool phase_fused_ok(int B, int T, int H, int varlen);
+cudaError_t launch_phase_chunk(const float *K, const float *Q, const void *V, const float *log_lam,
+                               const float *beta, const float *S0, void *out, float *S_final, const int32_t *cu,
+                               int B, int T, int H, cudaStream_t stream);
+
 cudaError_t launch_phase_rowdecay(const float *K, const float *Q, const void *V, const float *log_r,
                                   const float *beta, const float *M0, void *out, float *M_final,
                                   const int32_t *cu_seqlens, int nseq, int T, int H, int dk, int dv, int bf16,

@@ -10,7 +10,9 @@
 // with k~ = (Re K, Im K), q~ = (Re Q, Im Q): the real gated delta rule
 //     S_t = a_t (I - b_t k k^T) S_{t-1} + b_t k v^T,   o_t = S_t^T q
 // at head size 2dk with a = lam, b = beta / lam, k = k~ / sqrt(dk), v = lam sqrt(dk) V, q = q~ / dk
-// (lam > 0).  So one prologue kernel writes those inputs, the chunk kernel runs unchanged, and the
+// (lam > 0).  At dk = 32, dv = 64 with bf16 values the chunk kernel forms those inputs itself
+// (kFlagPhase: K and Q converted in shared memory, b v = beta sqrt(dk) V folded into its U~
+// product); otherwise one prologue kernel writes them and the chunk kernel runs unchanged.  The
 // complex state is converted on the way in and out.
 #include <cuda_bf16.h>
 
@@ -311,6 +313,33 @@ int gdn_phase_fwd(const float *K, const float *Q, const void *v, const float *lo
     const long token_heads = (varlen ? (long)T : (long)B * T) * H;
     const long states = (long)B * H;
     cudaError_t e;
+    // dk = 32, dv = 64, bf16 in one launch: the chunk kernel reads K, Q, V, log_lam and beta as
+    // given and forms the real recurrence's inputs itself (no prologue pass)
+    if (dtype == GDN_DTYPE_BF16 && dk == 32 && dv == 64 && phase_fused_ok(B, T, H, varlen)) {
+        if (M0) {
+            const long n = states * 2 * dk * dv;
+            phase_state_in<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(reinterpret_cast<const float2 *>(M0),
+                                                                         reinterpret_cast<float *>(w + p.s0), dk, dv,
+                                                                         states);
+        }
+        e = cudaGetLastError();
+        if (e == cudaSuccess)
+            e = launch_phase_chunk(K, Q, v, log_lam, beta, M0 ? reinterpret_cast<const float *>(w + p.s0) : nullptr,
+                                   out, M_final ? reinterpret_cast<float *>(w + p.sf) : nullptr, cu_seqlens, B, T, H,
+                                   st);
+        if (e == cudaSuccess && M_final) {
+            const long n = states * dk * dv;
+            phase_state_out<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(reinterpret_cast<const float *>(w + p.sf),
+                                                                          reinterpret_cast<float2 *>(M_final), dk, dv,
+                                                                          states);
+            e = cudaGetLastError();
+        }
+        if (e != cudaSuccess) {
+            set_error("gdn_phase_fwd: launch: %s", cudaGetErrorString(e));
+            return GDN_ERR_CUDA;
+        }
+        return GDN_OK;
+    }
     e = dtype == GDN_DTYPE_BF16
             ? prologue_for<__nv_bfloat16>(dk, dv, K, Q, v, log_lam, beta, token_heads, w, p, st)
             : prologue_for<float>(dk, dv, K, Q, v, log_lam, beta, token_heads, w, p, st);

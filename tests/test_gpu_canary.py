@@ -214,3 +214,21 @@ def test_host_entry():
     torch.cuda.synchronize()
     out.check("host out")
     Sf.check("host S_final")
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("dk,dv", [(32, 6), (64, 130), (32, 64)])
+def test_phase_rowdecay(dtype, dk, dv):
+    # channel blocks with a ragged last block, ragged chunk tails, empty and one-token sequences
+    import linear_attention_sequence_rule_b200 as gdn
+    ph = workloads.make_phase_rowdecay_inputs(H=2, dk=dk, dv=dv, dtype=dtype, seed=91 + dv, m0_std=0.1,
+                                              lengths=[1, 31, 0, 33, 70])
+    d = dev(ph)
+    tv = torch.bfloat16 if dtype == "bf16" else torch.float32
+    out = Guarded(tuple(d["v"].shape), tv)
+    Mf = Guarded((5, 2, dv, dk, 2), torch.float32)
+    gdn.phase_rowdecay_fwd(d["K"], d["Q"], d["v"], d["log_r"], d["beta"], M0=d["M0"], cu_seqlens=d["cu_seqlens"],
+                           out=out.t, M_final=Mf.t)
+    gdn.device_status()
+    out.check("rowdecay out")
+    Mf.check("rowdecay M_final")
