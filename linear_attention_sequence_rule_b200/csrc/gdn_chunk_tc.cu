@@ -794,7 +794,9 @@ __global__ void __launch_bounds__(TcCfg<DK, DV, PH>::THREADS, 1)
                 if (!ctl.aborted()) {
                     tc_fence_after();
                     constexpr uint32_t idU = idesc_bf16(DV, 64, 1, 0);
-                    constexpr uint32_t idW = idesc_bf16(DK, 64, 1, 0);
+                    // TA: -W^T (A operand negated), so that the chain's U MMA (A operand in tensor
+                    // memory) adds S^T (-W^T) onto U~^T without negating its A operand
+                    constexpr uint32_t idW = idesc_bf16(DK, 64, 1, 0, TA ? 1 : 0);
                     if (!v_zero) {
 #pragma unroll
                         for (int kk = 0; kk < 4; ++kk)
@@ -813,30 +815,19 @@ __global__ void __launch_bounds__(TcCfg<DK, DV, PH>::THREADS, 1)
             tc_fence_after();
             if (t == kIssuer && c + NB < nchunks) load_v(c + NB);  // the U~ MMA has read V
             {
-                // W^T rows (one per feature) to shared memory in bf16, then (unless the chain does
-                // it) lam K in place: the W MMA has read K unscaled
-                // TA: -W^T, so that the chain's U MMA (A operand in tensor memory) adds
-                // S^T (-W^T) onto U~^T without negating its A operand
-                constexpr float wsign = TA ? -1.f : 1.f;
+                // W^T rows (one per feature; -W^T with TA) to shared memory in bf16, then (unless the
+                // chain does it) lam K in place: the W MMA has read K unscaled
                 if (DK == 128) {
                     float x[64];
                     tmem_ld32(tl + tG, *reinterpret_cast<float(*)[32]>(&x[0]));
                     tmem_ld32(tl + tG + 32, *reinterpret_cast<float(*)[32]>(&x[32]));
                     tmem_wait_ld();
-                    if (TA) {
-#pragma unroll
-                        for (int i = 0; i < 64; ++i) x[i] *= wsign;
-                    }
                     st_row_bf16_sw128(WTs, t, x);
                 } else {
                     // M = 64 layout: threads lane and lane + 16 take the two halves of a row
                     float x[32];
                     tmem_ld16x2_32<32>(tl + tG, x);
                     tmem_wait_ld();
-                    if (TA) {
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) x[i] *= wsign;
-                    }
                     st_half_row_bf16_sw128(WTs, wi * 16 + (t & 15), (t >> 4) & 1, x);
                 }
                 if (!kChainScales) {
