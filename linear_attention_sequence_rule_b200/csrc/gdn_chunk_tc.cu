@@ -429,7 +429,7 @@ __device__ __forceinline__ void normalize_row_bf16(unsigned char *tile, int row)
 __device__ __forceinline__ void scale_row_bf16(unsigned char *tile, int row, float s, int c0, int c1)
 {
     const __nv_bfloat162 s2 = __float2bfloat162_rn(s);
-#pragma unroll
+#pragma unroll 2
     for (int c = c0; c < c1; ++c) {
         uint4 *p = reinterpret_cast<uint4 *>(tile + row * 128 + (((c + row) & 7) << 4));
         uint4 w = *p;
@@ -711,7 +711,7 @@ __global__ void __launch_bounds__(TcCfg<DK, DV, PH>::THREADS, 1)
                 const float Gr = Gs[r];
                 const int lr = last[r];
                 float *gm = AT + r * LDF + c0;
-#pragma unroll
+#pragma unroll 2
                 for (int j4 = 0; j4 < 32; j4 += 4) {
                     const float4 g4 = *reinterpret_cast<const float4 *>(&Gs[c0 + j4]);
                     const float gi[4] = {g4.x, g4.y, g4.z, g4.w};
@@ -771,6 +771,7 @@ __global__ void __launch_bounds__(TcCfg<DK, DV, PH>::THREADS, 1)
                 // (dk = 128): clear every 16-byte chunk from the diagonal block rightwards (the
                 // solve then writes the lower part)
                 constexpr int kTiles = DK / 64;
+#pragma unroll 1
                 for (int i = t; i < kTiles * 64 * 8; i += 128) {
                     const int r = (i >> 3) & 63, cb = i & 7;
                     unsigned char *tile = (kTiles == 2 && i >= 64 * 8) ? TGs : (kTiles == 2 ? TBs : TGs);
