@@ -462,6 +462,10 @@ __global__ void __launch_bounds__(TcCfg<DK, DV, PH>::THREADS, 1)
     using B = Bars<NS, NI, NB, NBO>;
     // gam Q and lam K are formed in place by the intra side, which runs ahead of the chain
     constexpr bool kChainScales = false;
+    // Unrolling of the intra side's MMA issue loops: rolled at value head 128, where the smaller
+    // code (fewer instruction-cache misses among the three roles) measured faster, unrolled at 64,
+    // where it did not
+    constexpr int kIssueUnroll = TA ? 1 : 8;
     extern __shared__ unsigned char smem_raw[];
     // 1024-aligned base by pointer arithmetic on the shared array, so that the compiler keeps
     // every access below in the shared address space
@@ -634,7 +638,7 @@ __global__ void __launch_bounds__(TcCfg<DK, DV, PH>::THREADS, 1)
             if (t == kIssuer && !ctl.aborted()) {
                 tc_fence_after();
                 constexpr uint32_t id = idesc_bf16(128, 64, 0, 0);
-#pragma unroll
+#pragma unroll(kIssueUnroll)
                 for (int kk = 0; kk < DK / 16; ++kk) {
                     const uint32_t a = smem_u32(Kt + (kk >> 2) * 16384 + (kk & 3) * 32);
                     mma_bf16(tmem + tG, sdesc_sw128(a, 16, 1024), sdesc_sw128(a, 16, 1024), id, kk > 0);
@@ -799,13 +803,13 @@ __global__ void __launch_bounds__(TcCfg<DK, DV, PH>::THREADS, 1)
                     // memory) adds S^T (-W^T) onto U~^T without negating its A operand
                     constexpr uint32_t idW = idesc_bf16(DK, 64, 1, 0, TA ? 1 : 0);
                     if (!v_zero) {
-#pragma unroll
+#pragma unroll(kIssueUnroll)
                         for (int kk = 0; kk < 4; ++kk)
                             mma_bf16(tmem + L::T_U + (TA ? wg : st) * 64,
                                      sdesc_sw128(smem_u32(sm + L::V + (c % NB) * L::V_BUF + kk * 2048), 8192, 1024),
                                      sdesc_sw128(smem_u32(TBs + kk * 32), 16, 1024), idU, kk > 0);
                     }
-#pragma unroll
+#pragma unroll(kIssueUnroll)
                     for (int kk = 0; kk < 4; ++kk)
                         mma_bf16(tmem + tG, sdesc_sw128(smem_u32(Kt + kk * 2048), 16384, 1024),
                                  sdesc_sw128(smem_u32(TGs + kk * 32), 16, 1024), idW, kk > 0);
@@ -1014,7 +1018,7 @@ __global__ void __launch_bounds__(TcCfg<DK, DV, PH>::THREADS, 1)
                     mma_commit(&bars[B::u]);
                     // O^T = S^T (gam Q)^T; its completion is covered by the state MMA's commit
                     if (want_out) {
-#pragma unroll
+#pragma unroll 1
                         for (int kk = 0; kk < DK / 16; ++kk)
                             mma_bf16_ta(tO, tmem + L::T_SB + 8 * kk,
                                         sdesc_sw128(smem_u32(Kt + (kk >> 2) * 16384 + 8192 + (kk & 3) * 32), 16, 1024),
@@ -1053,7 +1057,7 @@ __global__ void __launch_bounds__(TcCfg<DK, DV, PH>::THREADS, 1)
                         mma_bf16_ta(tmem + L::T_S, tU + 8 * kk,
                                     sdesc_sw128(smem_u32(Kt + (kk & 3) * 2048), 16384, 1024), idS, 1);
                     if (want_out) {
-#pragma unroll
+#pragma unroll 1
                         for (int kk = 0; kk < (kUSplit ? 8 : 4); ++kk)  // O^T += (U_hi + U_lo)^T P^T
                             mma_bf16_ta(tO, tU + 8 * kk,
                                         sdesc_sw128(smem_u32(sm + L::PM + st * 8192 + (kk & 3) * 32), 16, 1024), idO, 1);
