@@ -20,13 +20,17 @@
 //       T diag(b) and T diag(b gam) in bf16, then the WY products U~^T = V^T (T diag b)^T and
 //       W^T = K^T (T diag(b gam))^T (tcgen05) and W^T to shared memory.
 //   chain warpgroup (warps 0-3), thread j = value column j, for chunk c:
-//       U^T   = U~^T - S^T W^T           (accumulated onto U~^T, A operand negated)
-//       O     = (gam Q) S + P U          (M = 64 token rows, 16-byte row stores)
+//       U^T   = U~^T - S^T W^T           (accumulated onto U~^T)
+//       O     = (gam Q) S + P U          (value head 64: M = 64 token rows, 16-byte row stores)
 //       S'^T  = gam_C S^T + U^T (lam K)  (accumulated onto the pre-scaled fp32 state in TMEM)
+//   At value head 128 the chain's A operands (the bf16 copy of S^T, U^T as hi + lo parts) stay in
+//   tensor memory, the intra side writes -W^T, and the outputs are formed transposed (O^T) and
+//   leave through shared memory (transposing stmatrix, then 16-byte row stores).
 //   Loads: K/Q through a TMA stage ring (NS stages, reissued as soon as a stage's last MMA
-//   completes), V through NB buffers (two where TMEM holds two output buffers), gates by cp.async
-//   onto an mbarrier.
-// The state chain's critical path per chunk is two MMA round trips plus their epilogues.
+//   completes), V through NB buffers, gates by cp.async onto an mbarrier.
+// The state chain's critical path per chunk is two MMA round trips plus their epilogues.  The
+// three roles run different code on the same SM sub-partitions, so loops whose bodies hold no
+// register arrays are kept rolled where that measured faster (instruction-cache misses).
 //
 // Gates: decays are exp of log_alpha sums taken from the last exact reset (log_alpha = -inf)
 // inside the chunk.  Padded rows of a partial chunk get b = 0 and log_alpha = 0, which makes
@@ -672,7 +676,7 @@ __global__ void __launch_bounds__(TcCfg<DK, DV, PH>::THREADS, 1)
                 float a = f1 ? v1 : v0 + v1;
                 int fa = (f0 || f1) ? 1 : 0;
                 int li = f1 ? r1 : (f0 ? r0 : -1);
-#pragma unroll
+#pragma unroll 1
                 for (int off = 1; off < 32; off <<= 1) {
                     const float ab = __shfl_up_sync(0xffffffffu, a, off);
                     const int fb = __shfl_up_sync(0xffffffffu, fa, off);
@@ -962,7 +966,7 @@ __global__ void __launch_bounds__(TcCfg<DK, DV, PH>::THREADS, 1)
                 named_bar(1, 128);
                 // rows to global memory: eight threads per 256-byte row, each taking 16-byte units
                 // (tid & 7) and (tid & 7) + 8, so a warp stores four rows with full 128-byte runs
-#pragma unroll
+#pragma unroll 1
                 for (int p = 0; p < 4; ++p) {
                     const int r = 16 * p + (tid >> 3);
                     if (r < n) {
