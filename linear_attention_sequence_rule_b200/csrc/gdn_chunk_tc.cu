@@ -170,16 +170,23 @@ template <int NS, int NI, int NB, int NBO> struct Bars {
 __device__ __forceinline__ int scan_warp(int wg) { return wg == 0 ? 1 : 2; }
 constexpr int kIssuer = 96;
 
+// The bounded wait past a first unsuccessful try, out of line: one copy serves every wait site.
+__device__ __noinline__ void wait_slow(uint64_t *b, uint32_t parity, int *abort)
+{
+    if (!mbar_wait_bounded(b, parity, kWaitLimitNs)) {
+        atomicOr(&g_tc_device_error, 1);
+        *(volatile int *)abort = 1;
+    }
+}
+
 struct Ctl {
     uint64_t *bar;
     int *abort;
     __device__ void wait(int i, uint32_t parity) const
     {
         if (*(volatile int *)abort) return;
-        if (!mbar_wait_bounded(&bar[i], parity, kWaitLimitNs)) {
-            atomicOr(&g_tc_device_error, 1);
-            *(volatile int *)abort = 1;
-        }
+        if (mbar_try_wait(&bar[i], parity)) return;
+        wait_slow(&bar[i], parity, abort);
     }
     __device__ bool aborted() const { return *(volatile int *)abort != 0; }
     __device__ void arrive(int i) const
