@@ -378,39 +378,57 @@ def e2e_chunk(gdn, inp, steps, warmup, stream):
     return ms, h2d, d2h
 
 
+def oracle_subproblem(inp, seqs):
+    """fp64 host copies of the given sequences of a workload (all their heads), packed as a varlen
+    batch: (q, k, v, log_alpha, beta, S0, cu_seqlens) and the token-heads they hold.  Built
+    outside the timed regions, so that the CPU legs time the recurrence rather than a conversion
+    of the whole workload to fp64 on every call."""
+    import numpy as np
+    H = inp["H"]
+    seqs = list(seqs)
+    f64 = lambda x: x.detach().to("cpu", torch.float64).numpy()
+    if inp["cu_seqlens"] is None:
+        T = inp["T"]
+        pick = lambda x: f64(x[seqs].reshape(len(seqs) * T, *x.shape[2:]))
+        lengths = [T] * len(seqs)
+    else:
+        cu = inp["cu_seqlens"]
+        spans = [(int(cu[b]), int(cu[b + 1])) for b in seqs]
+        pick = lambda x: f64(torch.cat([x[a:e] for a, e in spans]))
+        lengths = [e - a for a, e in spans]
+    cu_sub = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int32)
+    S0 = None if inp["S0"] is None else f64(inp["S0"][seqs])
+    args = (pick(inp["q"]), pick(inp["k"]), pick(inp["v"]), pick(inp["log_alpha"]), pick(inp["beta"]), S0,
+            cu_sub)
+    return args, H * int(sum(lengths))
+
+
 def cpu_oracle_baseline(inp, budget_s=12.0):
-    """Time the fp64 oracle, as it stands, on the host cores over whole (sequence, head) chains of
-    the workload until about budget_s seconds of work; returns tokens/s and the sample."""
+    """Time the fp64 oracle, as it stands, on the host cores over whole sequences (every head of
+    each: H independent chains per sequence) of the workload until about budget_s seconds of work;
+    returns tokens/s and the sample."""
     import oracle
     H = inp["H"]
-    n_units = inp["B"] * H
     threads = oracle.max_threads()
-    # first a small probe to size the sample
-    probe = list(range(min(n_units, max(threads, 1))))
+    # first a small probe (the first sequence) to size the sample
+    sub, th = oracle_subproblem(inp, [0])
     t0 = time.perf_counter()
-    oracle.forward(inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["beta"], inp["S0"],
-                   cu_seqlens=inp["cu_seqlens"], units=probe)
-    t_probe = time.perf_counter() - t0
-    per_unit = t_probe / len(probe)
-    n = max(len(probe), min(n_units, int(budget_s / max(per_unit, 1e-9))))
-    units = list(range(n))
-    t0 = time.perf_counter()
-    oracle.forward(inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["beta"], inp["S0"],
-                   cu_seqlens=inp["cu_seqlens"], units=units)
-    dt = time.perf_counter() - t0
-    th = chain_token_heads(inp, units)
-    return dict(value=(th / H) / dt, unit="tokens/s", cores=threads, kind="oracle",
-                sample=f"{n} of {n_units} (sequence, head) chains, each in full "
-                       f"({th} token-heads = {th / H:.0f} tokens, {dt:.2f} s, fp64 sequential recurrence)")
-
-
-def chain_token_heads(inp, units):
-    """Token-heads of the given (sequence * H + head) chains: each chain's sequence length."""
-    H = inp["H"]
-    if inp["cu_seqlens"] is None:
-        return len(units) * inp["T"]
+    oracle.forward(*sub[:6], cu_seqlens=sub[6])
+    per_th = (time.perf_counter() - t0) / th
     cu = inp["cu_seqlens"]
-    return sum(int(cu[u // H + 1] - cu[u // H]) for u in units)
+    lengths = [inp["T"]] * inp["B"] if cu is None else [int(cu[b + 1] - cu[b]) for b in range(inp["B"])]
+    m, acc = 0, 0.0
+    while m < inp["B"] and (m == 0 or acc + H * lengths[m] * per_th <= budget_s):
+        acc += H * lengths[m] * per_th
+        m += 1
+    sub, th = oracle_subproblem(inp, range(m))
+    t0 = time.perf_counter()
+    oracle.forward(*sub[:6], cu_seqlens=sub[6])
+    dt = time.perf_counter() - t0
+    return dict(value=(th / H) / dt, unit="tokens/s", cores=threads, kind="oracle",
+                sample=f"{m} of {inp['B']} sequences, every head of each ({m * H} of {inp['B'] * H} "
+                       f"(sequence, head) chains, {th} token-heads = {th / H:.0f} tokens, {dt:.2f} s, "
+                       f"fp64 sequential recurrence; inputs converted to fp64 before the timing)")
 
 
 def cpu_decode_baseline(states=512, steps=200):
@@ -824,27 +842,27 @@ def run_reference(args, world, rank, inp=None):
     if inp is None:
         inp = workloads.config_inputs(HEADLINE)
     H = inp["H"]
-    n_units = inp["B"] * H
     threads = oracle.max_threads()
-    # each step: a bounded sample of whole chains (one per host thread), taken in turn over the
-    # workload's chains, so that the whole run takes a few minutes
-    per_step = max(threads, 8)
+    # each step: enough whole sequences (every head: H independent chains each) to give every host
+    # thread a chain, taken in turn, their inputs converted to fp64 before the step's timing; the
+    # whole run takes a few minutes
+    per_step = min(inp["B"], max(1, -(-threads // H)))
     times, token_heads = [], []
     for i in range(args.warmup + args.steps):
-        units = [(i * per_step + j) % n_units for j in range(per_step)]
+        sub, th = oracle_subproblem(inp, [(i * per_step + j) % inp["B"] for j in range(per_step)])
         t0 = time.perf_counter()
-        oracle.forward(inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["beta"], inp["S0"],
-                       cu_seqlens=inp["cu_seqlens"], units=units)
+        oracle.forward(*sub[:6], cu_seqlens=sub[6])
         dt = time.perf_counter() - t0
         if i >= args.warmup:
             times.append(dt)
-            token_heads.append(chain_token_heads(inp, units))
+            token_heads.append(th)
     s = statistics.mean(times)
     # tokens, not token-heads: a token of the workload is all H of its heads
     value = (sum(token_heads) / H) / sum(times)
-    sample = (f"{per_step} of {n_units} (sequence, head) chains per step, each in full "
-              f"({sum(token_heads) // len(token_heads)} token-heads per step on average, "
-              f"counted as token-heads / {H} tokens), fp64 sequential recurrence")
+    sample = (f"{per_step} of {inp['B']} sequences per step, every head of each ({per_step * H} chains, "
+              f"{sum(token_heads) // len(token_heads)} token-heads per step on average, counted as "
+              f"token-heads / {H} tokens), fp64 sequential recurrence, inputs converted to fp64 "
+              f"before each step's timing")
     line = {
         "impl": "reference",
         "metric": METRIC,

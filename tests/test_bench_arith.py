@@ -63,22 +63,40 @@ def test_backward_product_count():
     assert bench.bwd_products(2, 2) > bench.bwd_products(1, 2) + 26
 
 
-def test_reference_arm_counts_tokens_not_token_heads():
+def test_reference_arm_counts_tokens_not_token_heads(monkeypatch):
     """The reference arm's tokens/s is token-heads / H over the timed seconds, on a varlen pack
-    whose chains differ in length, and agrees with the CPU-baseline leg's count of the same
-    chains."""
+    whose chains differ in length; the per-sequence sub-problems both CPU legs time are the
+    workload's own sequences in full."""
     import argparse
     import workloads
     inp = workloads.make_chunk_inputs(H=3, dk=64, dv=64, dtype="bf16", seed=5, lengths=[70, 5, 130])
     args = argparse.Namespace(steps=2, warmup=3)
+    import oracle
+    # 4 host threads over 3 heads: 2 whole sequences per step, taken in turn
+    monkeypatch.setattr(oracle, "max_threads", lambda: 4)
     line = bench.run_reference(args, 1, 0, inp=inp)
     th, s = line["token_heads_timed"], line["seconds_timed"]
     assert line["unit"] == "tokens/s"
     assert abs(line["value"] - th / 3 / s) <= 1e-9 * line["value"]
-    # every chain of the pack, in full: 3 heads x (70 + 5 + 130) token-heads
-    assert bench.chain_token_heads(inp, range(9)) == 3 * 205
-    assert bench.chain_token_heads(inp, [0, 1, 2]) == 3 * 70
+    # warm-up steps take sequences {0, 1}, {2, 0}, {1, 2}; the timed ones {0, 1} and {2, 0}, all
+    # 3 heads of each
+    assert th == 3 * (70 + 5) + 3 * (130 + 70)
+    # a sub-problem holds its sequences in full, and the oracle on it gives the same numbers as
+    # the oracle on the whole pack
+    import numpy as np
+    sub, th2 = bench.oracle_subproblem(inp, [2, 0])
+    assert th2 == 3 * (130 + 70)
+    o_sub, s_sub = oracle.forward(*sub[:6], cu_seqlens=sub[6])
+    o_all, s_all = oracle.forward(inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["beta"],
+                                  inp["S0"], cu_seqlens=inp["cu_seqlens"])
+    assert np.array_equal(o_sub, np.concatenate([o_all[75:205], o_all[0:70]]))
+    assert np.array_equal(s_sub, s_all[[2, 0]])
     dense = workloads.make_chunk_inputs(B=2, T=40, H=3, dk=64, dv=64, dtype="bf16", seed=5)
-    assert bench.chain_token_heads(dense, range(6)) == 6 * 40
+    sub, th3 = bench.oracle_subproblem(dense, [1])
+    assert th3 == 3 * 40
+    o_sub, _ = oracle.forward(*sub[:6], cu_seqlens=sub[6])
+    o_all, _ = oracle.forward(dense["q"], dense["k"], dense["v"], dense["log_alpha"], dense["beta"],
+                              dense["S0"])
+    assert np.array_equal(o_sub, o_all[1])
     assert bench.run_reference(args, 1, 1, inp=inp) is None
     assert line["config"] == bench.headline_config(1)
