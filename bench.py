@@ -414,17 +414,19 @@ def cpu_oracle_baseline(inp, budget_s=12.0):
     sub, th = oracle_subproblem(inp, [0])
     t0 = time.perf_counter()
     oracle.forward(*sub[:6], cu_seqlens=sub[6])
-    per_th = (time.perf_counter() - t0) / th
+    dt = time.perf_counter() - t0
+    per_th = dt / th
     cu = inp["cu_seqlens"]
     lengths = [inp["T"]] * inp["B"] if cu is None else [int(cu[b + 1] - cu[b]) for b in range(inp["B"])]
     m, acc = 0, 0.0
     while m < inp["B"] and (m == 0 or acc + H * lengths[m] * per_th <= budget_s):
         acc += H * lengths[m] * per_th
         m += 1
-    sub, th = oracle_subproblem(inp, range(m))
-    t0 = time.perf_counter()
-    oracle.forward(*sub[:6], cu_seqlens=sub[6])
-    dt = time.perf_counter() - t0
+    if m > 1:  # else the probe was the sample
+        sub, th = oracle_subproblem(inp, range(m))
+        t0 = time.perf_counter()
+        oracle.forward(*sub[:6], cu_seqlens=sub[6])
+        dt = time.perf_counter() - t0
     return dict(value=(th / H) / dt, unit="tokens/s", cores=threads, kind="oracle",
                 sample=f"{m} of {inp['B']} sequences, every head of each ({m * H} of {inp['B'] * H} "
                        f"(sequence, head) chains, {th} token-heads = {th / H:.0f} tokens, {dt:.2f} s, "
