@@ -161,14 +161,18 @@ GDN_API size_t gdn_chunk_fwd_workspace_bytes(int B, int T, int H, int dk, int dv
  * that has reserved its device memory up front and admits no call-time allocation, or a C host
  * program without a device allocator).  Arguments, layouts and results are those of
  * gdn_chunk_fwd.
- *   - Every call looks up the array's address in the current context.  The first call on a
- *     device also loads the module that holds it; make that first call before any stream
- *     capture on that device.
+ *   - Every argument is checked on the host first, as gdn_chunk_fwd checks it; a rejected call
+ *     touches no device state.  Sizes that need no scratch (enough chains to fill the device:
+ *     gdn_chunk_fwd_workspace_bytes returns 0) run as gdn_chunk_fwd without a workspace and never
+ *     touch the array.
+ *   - Every call that needs scratch looks up the array's address in the current context.  The
+ *     first such call on a device also loads the module that holds it; make that first call
+ *     before any stream capture on that device.
  *   - Footprint: the array takes 32 MiB of device memory on every device where its module is
  *     loaded -- with CUDA's default lazy module loading, from the first gdn_chunk_fwd_noalloc
- *     call on that device; with CUDA_MODULE_LOADING=EAGER, from the CUDA runtime's
- *     initialisation of the device -- until the process exits.  Callers that reserve device
- *     memory up front should budget for it.
+ *     call on that device that needs scratch; with CUDA_MODULE_LOADING=EAGER, from the CUDA
+ *     runtime's initialisation of the device -- until the process exits.  Callers that reserve
+ *     device memory up front should budget for it.
  *   - Calls on the same device must not overlap in time (two streams, two host threads): they
  *     share the one array.  Nothing in it needs to start at zero.
  *   - Sizes whose scratch would exceed 32 MiB return GDN_ERR_WORKSPACE (about 3 * SMs * dk * dv

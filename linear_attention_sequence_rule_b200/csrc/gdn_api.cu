@@ -72,6 +72,28 @@ static int check_chunk_shape(int B, int T, int H, int dk, int dv, int chunk, int
     return GDN_OK;
 }
 
+int chunk_fwd_check(const char *fn, const void *q, const void *k, const void *v, const float *log_alpha,
+                    const float *beta, const float *S0, const void *out, const float *S_final, int B, int T,
+                    int H, int dk, int dv, int chunk, const int32_t *cu_seqlens, int dtype)
+{
+    const int varlen = cu_seqlens != nullptr;
+    int rc = check_chunk_shape(B, T, H, dk, dv, chunk, varlen, dtype);
+    if (rc != GDN_OK) return rc;
+    if (!q || !k || !v || !log_alpha || !beta || !out)
+        return fail(GDN_ERR_INVALID_ARGUMENT, "%s: q, k, v, the two gate arrays and out are required", fn);
+    const void *ptrs[] = {q, k, v, log_alpha, beta, S0, out, S_final, cu_seqlens};
+    for (const void *p : ptrs)
+        if (p && !aligned16(p))
+            return fail(GDN_ERR_INVALID_ARGUMENT, "%s: pointer %p is not 16-byte aligned", fn, p);
+    if (S_final && S_final != S0 && S0) {
+        const size_t bytes = (size_t)B * H * dk * dv * sizeof(float);
+        const char *a0 = (const char *)S0, *b0 = (const char *)S_final;
+        if (a0 < b0 + bytes && b0 < a0 + bytes)
+            return fail(GDN_ERR_INVALID_ARGUMENT, "%s: S0 and S_final overlap partially", fn);
+    }
+    return GDN_OK;
+}
+
 static size_t chunk_workspace(int B, int T, int H, int dk, int dv, int chunk, int varlen, int dtype)
 {
     if (general_path(dk, dv, chunk, dtype)) return chunk_general_workspace_bytes(B, T, H, dk, dv, chunk, varlen);
@@ -120,20 +142,9 @@ static int chunk_fwd_common(const char *fn, const void *q, const void *k, const 
                             int G = 1)
 {
     const int varlen = cu_seqlens != nullptr;
-    int rc = check_chunk_shape(B, T, H, dk, dv, chunk, varlen, dtype);
+    const int rc = chunk_fwd_check(fn, q, k, v, log_alpha, beta, S0, out, S_final, B, T, H, dk, dv, chunk,
+                                   cu_seqlens, dtype);
     if (rc != GDN_OK) return rc;
-    if (!q || !k || !v || !log_alpha || !beta || !out)
-        return fail(GDN_ERR_INVALID_ARGUMENT, "%s: q, k, v, the two gate arrays and out are required", fn);
-    const void *ptrs[] = {q, k, v, log_alpha, beta, S0, out, S_final, cu_seqlens};
-    for (const void *p : ptrs)
-        if (p && !aligned16(p))
-            return fail(GDN_ERR_INVALID_ARGUMENT, "%s: pointer %p is not 16-byte aligned", fn, p);
-    if (S_final && S_final != S0 && S0) {
-        const size_t bytes = (size_t)B * H * dk * dv * sizeof(float);
-        const char *a0 = (const char *)S0, *b0 = (const char *)S_final;
-        if (a0 < b0 + bytes && b0 < a0 + bytes)
-            return fail(GDN_ERR_INVALID_ARGUMENT, "%s: S0 and S_final overlap partially", fn);
-    }
     if (prologue && general_path(dk, dv, chunk, dtype))
         return fail(GDN_ERR_UNSUPPORTED, "%s: the fused prologue takes dk, dv in {64, 128} (dv 256) and chunk 64",
                     fn);

@@ -11,6 +11,13 @@ namespace gdn {
 // Records a one-line reason for the calling host thread (read back by gdn_last_error()).
 void set_error(const char *fmt, ...);
 
+// Every argument check of the plain chunk forward except the workspace's (sizes, dtype, required
+// and aligned pointers, S0 / S_final overlap), on the host only: GDN_OK, or the error code with
+// the reason recorded under the name fn.
+int chunk_fwd_check(const char *fn, const void *q, const void *k, const void *v, const float *log_alpha,
+                    const float *beta, const float *S0, const void *out, const float *S_final, int B, int T,
+                    int H, int dk, int dv, int chunk, const int32_t *cu_seqlens, int dtype);
+
 // Launchers (defined in the kernel .cu files).  They assume the arguments were validated by the
 // C-ABI layer and return the cudaError_t of the launch.
 cudaError_t launch_decode(const void *q, const void *k, const void *v, const float *log_alpha,

@@ -28,8 +28,8 @@ constexpr size_t kScratchBytes = size_t(32) << 20;
 }  // namespace
 
 // The array takes 32 MiB on every device where the module that holds it is loaded: with CUDA's
-// default lazy module loading that happens the first time gdn_chunk_fwd_noalloc runs on the
-// device; with CUDA_MODULE_LOADING=EAGER, when the CUDA runtime initialises the device.  It stays
+// default lazy module loading that happens the first time gdn_chunk_fwd_noalloc needs scratch on
+// the device; with CUDA_MODULE_LOADING=EAGER, when the CUDA runtime initialises the device.  It stays
 // until the process exits (or the context is destroyed).
 static __device__ __align__(256) unsigned char g_scratch[kScratchBytes];
 
@@ -55,19 +55,24 @@ int gdn_chunk_fwd_noalloc(const void *q, const void *k, const void *v, const flo
                           int H, int dk, int dv, int chunk, const int32_t *cu_seqlens, int dtype,
                           void *stream)
 {
+    gdn::set_error("%s", "");
+    // every argument first, on the host, so that a rejected call touches no device state
+    int rc = gdn::chunk_fwd_check("gdn_chunk_fwd_noalloc", q, k, v, log_alpha, beta, S0, out, S_final, B, T,
+                                  H, dk, dv, chunk, cu_seqlens, dtype);
+    if (rc != GDN_OK) return rc;
     const size_t need = gdn_chunk_fwd_workspace_bytes(B, T, H, dk, dv, chunk, cu_seqlens != nullptr, dtype);
-    if (need == (size_t)-1)  // rejected sizes: gdn_chunk_fwd reports why, before touching the device
+    if (need == 0)  // a plan without scratch: the array is not looked up (nor its module loaded)
         return gdn_chunk_fwd(q, k, v, log_alpha, beta, S0, out, S_final, B, T, H, dk, dv, chunk, cu_seqlens,
                              dtype, nullptr, 0, stream);
-    void *scratch = nullptr;
-    const int rc = scratch_on_current_device(&scratch);
-    if (rc != GDN_OK) return rc;
     if (need > kScratchBytes) {
         gdn::set_error("gdn_chunk_fwd_noalloc: these sizes need %zu bytes of scratch; the static scratch "
                        "holds %zu (use gdn_chunk_fwd with a workspace)",
                        need, kScratchBytes);
         return GDN_ERR_WORKSPACE;
     }
+    void *scratch = nullptr;
+    rc = scratch_on_current_device(&scratch);
+    if (rc != GDN_OK) return rc;
     return gdn_chunk_fwd(q, k, v, log_alpha, beta, S0, out, S_final, B, T, H, dk, dv, chunk, cu_seqlens, dtype,
                          scratch, kScratchBytes, stream);
 }

@@ -362,3 +362,40 @@ def test_rowdecay_entry_rejects_before_any_launch():
     # M0 and M_final overlapping partially
     assert rowdecay_call(M0=FAKE, M_final=FAKE + 256) == gdn.GDN_ERR_INVALID_ARGUMENT
     assert "rowdecay" in gdn.gdn_last_error()
+
+
+def noalloc(**kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, log_alpha=FAKE, beta=FAKE, S0=None, out=FAKE, S_final=None,
+             B=1, T=64, H=1, dk=64, dv=64, chunk=64, cu_seqlens=None, dtype=gdn.GDN_DTYPE_BF16,
+             stream=None)
+    a.update(kw)
+    return gdn.gdn_chunk_fwd_noalloc(**a)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(dtype=7), gdn.GDN_ERR_UNSUPPORTED),
+    (dict(dk=96), gdn.GDN_ERR_UNSUPPORTED),
+    (dict(chunk=32), gdn.GDN_ERR_UNSUPPORTED),
+    (dict(B=0), gdn.GDN_ERR_INVALID_ARGUMENT),
+    (dict(q=None), gdn.GDN_ERR_INVALID_ARGUMENT),
+    (dict(out=None), gdn.GDN_ERR_INVALID_ARGUMENT),
+    (dict(k=FAKE + 4), gdn.GDN_ERR_INVALID_ARGUMENT),
+    (dict(S0=FAKE, S_final=FAKE + 16), gdn.GDN_ERR_INVALID_ARGUMENT),
+    # a segmented plan (one long sequence) with a bad pointer: rejected before the scratch lookup
+    (dict(T=65536, q=None), gdn.GDN_ERR_INVALID_ARGUMENT),
+])
+def test_noalloc_entry_rejects_before_touching_the_device(kw, code):
+    """Every argument is checked on the host before the library's scratch array is looked up: on
+    this machine, without a device, a lookup would fail with GDN_ERR_CUDA instead."""
+    assert noalloc(**kw) == code
+    assert "gdn_chunk_fwd" in gdn.gdn_last_error()  # the shape checks are gdn_chunk_fwd's own
+
+
+def test_noalloc_entry_rejects_oversized_scratch_on_the_host():
+    # chunk 128 runs on the general path, whose workspace grows with the token count: far beyond
+    # the 32 MiB array for a long sequence
+    B, T, H, dk, dv = 1, 65536, 16, 128, 128
+    need = gdn.gdn_chunk_fwd_workspace_bytes(B, T, H, dk, dv, 128, 0, gdn.GDN_DTYPE_BF16)
+    assert need > 32 * 2 ** 20
+    assert noalloc(B=B, T=T, H=H, dk=dk, dv=dv, chunk=128) == gdn.GDN_ERR_WORKSPACE
+    assert "32 MiB" in gdn.gdn_last_error() or str(32 * 2 ** 20) in gdn.gdn_last_error()
