@@ -381,7 +381,7 @@ def noalloc(**kw):
     (dict(out=None), gdn.GDN_ERR_INVALID_ARGUMENT),
     (dict(k=FAKE + 4), gdn.GDN_ERR_INVALID_ARGUMENT),
     (dict(S0=FAKE, S_final=FAKE + 16), gdn.GDN_ERR_INVALID_ARGUMENT),
-    # a segmented plan (one long sequence) with a bad pointer: rejected before the scratch lookup
+    # one long sequence (a segmented plan on a device) with a bad pointer
     (dict(T=65536, q=None), gdn.GDN_ERR_INVALID_ARGUMENT),
 ])
 def test_noalloc_entry_rejects_before_touching_the_device(kw, code):
